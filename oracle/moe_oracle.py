@@ -1,0 +1,428 @@
+"""CPU oracle for one MoE layer: route -> balance -> dispatch -> expert FFN -> combine.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path imports, calls or executes this
+module: only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline /
+reference arm may.  It shares no code with the CUDA library (no kernels, headers,
+helpers, tables or constants); both sides get their inputs from the seeded generators in
+``load_balanced_dispatch_warp_b200/inputs.py``.
+
+Every function is the plain definition of its step, written slowly and in fp64 for
+floating point, citing the page passage it follows.  Sources (page title, section):
+
+  [MoonEP]   "Moonshot AI drops MoonEP, claims 2.5x scaling boost for trillion-parameter
+             models" -- news article; para. 2 (maxvio), para. 3 (equal-load invariant,
+             redundant copies planned from router output, prefetch, zero-copy placement,
+             static shapes, one process-global pool), para. 4 (slot policy).
+  [Primer]   "DeepEP-on-EFA Guidance, section 1: What is MoE" -- the four-phase EP
+             pipeline: (a) router/top-k, (b) dispatch, (c) expert FFN as grouped GEMM,
+             (d) combine = transpose of dispatch, gate-weighted sum.
+  [Hotspots] "MoE Load Balancing: Find Expert Hotspots" -- sections "Separate expert
+             demand from rank placement", "Make expert capacity, overflow, and padding
+             explicit", "Count remote routes before celebrating balance", "Work the
+             16-token hotspot fixture", "Reject incomparable MoE load-balancing traces".
+
+Pins (tests/test_oracle_pins.py checks each against something other than this file):
+  topk_route        brute-force rank counting on tiny inputs; k=1 / k=E special cases;
+                    softmax closed forms (k=2 sigmoid, equal logits -> 1/k)
+  expert_histogram  the pages' worked fixture (demand, both rank mappings, 4/9, 8/15, 0.8)
+  capacity_ledger   the pages' worked fixture (cap 5, processed/overflow/padding)
+  remote_routes     the pages' worked fixture (22 vs 25 of 32)
+  plan_balanced     invariants (exact per-rank load, every assignment once, replica
+                    accounting) over exhaustive tiny inputs, plus a plan derived by hand
+                    for the fixture.  WHICH valid plan is chosen is not fixed by the pages
+                    (they give no algorithm): that choice is this oracle's reading.
+  permute/dispatch  bijection and x-row identity checks on random inputs
+  prefetch          bitwise slot = home-expert identity
+  expert_ffn        closed forms: identity / single-entry weights give silu(a)*a with
+                    silu(1) = e/(1+e); transposed operands land in distinct outputs
+  combine           identity experts return x (gates sum to one); per-expert scaling
+                    returns (sum_j gate_j c_e) x
+
+Error bits (OR-ed): 1 non-finite logit, 2 expert id out of range, 4 repeated expert
+within one token, 8 plan needs more than S replicas on some rank.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+ERR_NONFINITE = 1
+ERR_ID_RANGE = 2
+ERR_DUPLICATE = 4
+ERR_SLOTS = 8
+
+
+# --------------------------------------------------------------------------- (a) router
+def topk_route(logits: np.ndarray, k: int):
+    """Top-k expert choice and gate weights per token  ([Primer] phase (a) router).
+
+    For each token the (logit, expert) pairs are ordered by logit descending, ties by
+    the lower expert id first, and the first k are taken.  The gate of the j-th choice
+    is the softmax over the k selected logits:
+        gate_j = exp(l_j - l_max) / sum_{i in top-k} exp(l_i - l_max)
+    computed in fp64 from the fp32 logits, so the weights are finite, non-negative and
+    sum to one ([Hotspots] "starts with one route trace": finite non-negative weights).
+    A non-finite logit anywhere sets error bit 1; that token's outputs are unspecified.
+
+    Returns idx [T,k] int32, gate [T,k] float64, err int.
+    """
+    logits = np.asarray(logits, dtype=np.float32)
+    T, E = logits.shape
+    if not (1 <= k <= E):
+        raise ValueError("need 1 <= k <= E")
+    err = 0
+    if not np.all(np.isfinite(logits)):
+        err |= ERR_NONFINITE
+    idx = np.zeros((T, k), dtype=np.int32)
+    gate = np.zeros((T, k), dtype=np.float64)
+    for t in range(T):
+        row = logits[t].astype(np.float64)
+        if not np.all(np.isfinite(row)):
+            continue
+        # stable sort on -logit keeps equal logits in ascending expert order
+        order = np.argsort(-row, kind="stable")[:k]
+        idx[t] = order
+        sel = row[order]
+        ex = np.exp(sel - sel[0])
+        gate[t] = ex / ex.sum()
+    return idx, gate, err
+
+
+# ------------------------------------------------------------------ demand and imbalance
+def home_rank_map(E: int, R: int) -> np.ndarray:
+    """Contiguous expert->rank ownership e -> floor(e / (E/R)): rank r owns experts
+    [rB, (r+1)B), as in the fixture's initial placement {0,1},{2,3},{4,5},{6,7}
+    ([Hotspots] "Separate expert demand from rank placement")."""
+    B = E // R
+    return (np.arange(E) // B).astype(np.int64)
+
+
+def validate_trace(idx: np.ndarray, E: int) -> int:
+    """Trace validation before anything is sized from it ([Hotspots] "Work the 16-token
+    hotspot fixture": ids must be known experts, no token may repeat an expert).
+    Returns error bits 2 (id outside [0,E)) and 4 (repeat within a token)."""
+    err = 0
+    for row in np.asarray(idx):
+        ids = [int(v) for v in row]
+        if any(v < 0 or v >= E for v in ids):
+            err |= ERR_ID_RANGE
+        if len(set(ids)) != len(ids):
+            err |= ERR_DUPLICATE
+    return err
+
+
+def expert_histogram(idx: np.ndarray, E: int, R: int, expert_to_rank=None):
+    """Expert demand, rank demand and the imbalance scalars.
+
+    [Hotspots] "Separate expert demand from rank placement": first count assignments by
+    expert, then sum those counts over an expert->rank mapping.  Balancedness is
+    average / maximum.  [MoonEP] para. 2: maxvio is 0 when perfectly balanced; adopted as
+    (max rank load - mean) / mean.  With A = T*k assignments and mean = A/R this is the
+    exact rational (R*max - A) / A, rounded once to fp64; balancedness = A / (R*max).
+    Expert-level maxvio uses E buckets instead of R.  Only in-range ids are counted;
+    bad ids set the validation error bits.  A = 0 gives maxvio 0 and balancedness 1.
+
+    Returns dict(counts[E], loads[R], maxvio, balancedness, expert_maxvio,
+    expert_balancedness, err).
+    """
+    idx = np.asarray(idx)
+    T, k = idx.shape
+    A = T * k
+    err = validate_trace(idx, E)
+    counts = np.zeros(E, dtype=np.int64)
+    for t in range(T):
+        for j in range(k):
+            e = int(idx[t, j])
+            if 0 <= e < E:
+                counts[e] += 1
+    if expert_to_rank is None:
+        expert_to_rank = home_rank_map(E, R)
+    loads = np.zeros(R, dtype=np.int64)
+    for e in range(E):
+        loads[int(expert_to_rank[e])] += counts[e]
+    mx = int(loads.max()) if R > 0 else 0
+    emx = int(counts.max()) if E > 0 else 0
+    if A == 0 or mx == 0:
+        maxvio, bal = 0.0, 1.0
+    else:
+        maxvio = float(R * mx - A) / float(A)
+        bal = float(A) / float(R * mx)
+    if A == 0 or emx == 0:
+        emaxvio, ebal = 0.0, 1.0
+    else:
+        emaxvio = float(E * emx - A) / float(A)
+        ebal = float(A) / float(E * emx)
+    return dict(counts=counts, loads=loads, maxvio=maxvio, balancedness=bal,
+                expert_maxvio=emaxvio, expert_balancedness=ebal, err=err)
+
+
+def capacity_ledger(counts, A: int, E: int, cf_num: int = 5, cf_den: int = 4):
+    """Fixed-capacity ledger ([Hotspots] "Make expert capacity, overflow, and padding
+    explicit"): cap = ceil(A / E * cf) per expert, processed = min(count, cap),
+    overflow = max(count - cap, 0), padding = max(cap - count, 0).  The capacity
+    factor is an exact rational cf_num/cf_den so the ceiling is exact."""
+    num = A * cf_num
+    den = E * cf_den
+    cap = -(-num // den)
+    counts = np.asarray(counts, dtype=np.int64)
+    processed = np.minimum(counts, cap)
+    overflow = np.maximum(counts - cap, 0)
+    padding = np.maximum(cap - counts, 0)
+    return dict(cap=int(cap), processed=processed, overflow=overflow, padding=padding)
+
+
+def remote_routes(idx, origin, expert_to_rank) -> int:
+    """Remote-route count ([Hotspots] "Count remote routes before celebrating balance"):
+    an assignment is remote when the token's origin rank differs from the rank that
+    owns its chosen expert."""
+    n = 0
+    for t, row in enumerate(np.asarray(idx)):
+        for e in row:
+            if int(expert_to_rank[int(e)]) != int(origin[t]):
+                n += 1
+    return n
+
+
+# ------------------------------------------------------------------ equal-load plan
+def plan_balanced(counts, T: int, k: int, E: int, R: int, S: int):
+    """Equal-load plan with redundant expert copies ([MoonEP] para. 3-4).
+
+    The article fixes the contract -- every rank receives exactly the same number of
+    rows, C = T*k/R, by placing a few redundant expert copies planned from the router
+    output, each copy occupying one of S prefetch slots per rank -- but gives no
+    algorithm.  The reading used here ("keep small, stream the rest"):
+
+      1. Rank r owns experts [rB, (r+1)B), B = E/R.
+      2. Per rank, order its experts by (count ascending, id ascending).  With room = C,
+         keep each expert whole while its count fits the room (room -= count); the first
+         expert that does not fit and every later one are streamed.  room_r is what is
+         left.
+      3. The stream is the streamed experts in (home rank, id) order, each expert's
+         assignments in token order.  Sum(room_r) equals the stream length.
+      4. The ranks' rooms, concatenated in rank order, cut the stream: position p goes to
+         the rank u with room_prefix[u] <= p < room_prefix[u+1].
+      5. In rank u's piece, each maximal run of one expert whose home is not u is a
+         replica; replicas take slots 0, 1, ... of rank u in order.  More than S sets
+         error bit 8.
+      6. Rank u's rows: [0, kept_u) hold its kept experts in id order (each contiguous),
+         [kept_u, C) hold its stream piece in stream order.
+      7. Groups are those runs in that order, empty ones left out.  weight_ref = e for an
+         expert at its home rank, E + u*S + s for replica slot s of rank u.
+
+    Returns a dict with C, kept_rows[R], room_prefix[R+1], expert_home_off[E] (local
+    row offset of a kept expert, -1 if streamed), stream_off[E+1] (exclusive prefix of
+    streamed counts in id order), replica_expert[R*S] (-1 empty), groups (list per rank
+    of (row_start_global, rows, expert, weight_ref)), err.
+    """
+    counts = [int(c) for c in counts]
+    A = T * k
+    assert A % R == 0 and E % R == 0
+    C = A // R
+    B = E // R
+    kept = [False] * E
+    kept_rows = [0] * R
+    room = [0] * R
+    for r in range(R):
+        home = list(range(r * B, (r + 1) * B))
+        order = sorted(home, key=lambda e: (counts[e], e))
+        left = C
+        for e in order:
+            if counts[e] <= left:
+                kept[e] = True
+                left -= counts[e]
+            else:
+                break
+        room[r] = left
+        kept_rows[r] = C - left
+    room_prefix = [0] * (R + 1)
+    for r in range(R):
+        room_prefix[r + 1] = room_prefix[r] + room[r]
+    stream_off = [0] * (E + 1)
+    for e in range(E):
+        stream_off[e + 1] = stream_off[e] + (0 if kept[e] else counts[e])
+    assert stream_off[E] == room_prefix[R]
+    expert_home_off = [-1] * E
+    for r in range(R):
+        off = 0
+        for e in range(r * B, (r + 1) * B):
+            if kept[e]:
+                expert_home_off[e] = off
+                off += counts[e]
+    replica_expert = [-1] * (R * S)
+    groups = [[] for _ in range(R)]
+    err = 0
+    for u in range(R):
+        for e in range(u * B, (u + 1) * B):
+            if kept[e] and counts[e] > 0:
+                groups[u].append((u * C + expert_home_off[e], counts[e], e, e))
+        lo, hi = room_prefix[u], room_prefix[u + 1]
+        n_rep = 0
+        for e in range(E):
+            if kept[e] or counts[e] == 0:
+                continue
+            a, b = max(lo, stream_off[e]), min(hi, stream_off[e] + counts[e])
+            if a >= b:
+                continue
+            row = u * C + kept_rows[u] + (a - lo)
+            if e // B == u:
+                groups[u].append((row, b - a, e, e))
+            else:
+                if n_rep < S:
+                    replica_expert[u * S + n_rep] = e
+                    groups[u].append((row, b - a, e, E + u * S + n_rep))
+                n_rep += 1
+        if n_rep > S:
+            err |= ERR_SLOTS
+    return dict(C=C, kept=kept, kept_rows=kept_rows, room_prefix=room_prefix,
+                expert_home_off=expert_home_off, stream_off=stream_off,
+                replica_expert=replica_expert, groups=groups, err=err)
+
+
+# ------------------------------------------------------------------ placement of rows
+def permute(idx: np.ndarray, plan, E: int, R: int):
+    """Row of every (token, choice) assignment in the static per-rank buffers.
+
+    Zero-copy placement ([MoonEP] para. 3): each assignment goes straight to its final
+    row.  For assignment (t, j) with expert e, q = number of earlier tokens t' < t that
+    chose e (token order within an expert).  A kept expert's rows start at its home
+    offset: row = home(e)*C + expert_home_off[e] + q.  A streamed expert's assignment
+    sits at stream position p = stream_off[e] + q; the rank u whose room range holds p
+    receives it at row u*C + kept_rows[u] + (p - room_prefix[u]).
+
+    Returns perm [T,k] int32 (row of each assignment) and src [R*C] int32 (token of
+    each row).
+    """
+    idx = np.asarray(idx)
+    T, k = idx.shape
+    C = plan["C"]
+    B = E // R
+    seen = [0] * E
+    perm = np.full((T, k), -1, dtype=np.int32)
+    src = np.full(R * C, -1, dtype=np.int32)
+    rp = plan["room_prefix"]
+    for t in range(T):
+        for j in range(k):
+            e = int(idx[t, j])
+            q = seen[e]
+            seen[e] += 1
+            if plan["kept"][e]:
+                row = (e // B) * C + plan["expert_home_off"][e] + q
+            else:
+                p = plan["stream_off"][e] + q
+                u = 0
+                while not (rp[u] <= p < rp[u + 1]):
+                    u += 1
+                row = u * C + plan["kept_rows"][u] + (p - rp[u])
+            perm[t, j] = row
+            src[row] = t
+    return perm, src
+
+
+def dispatch(x: np.ndarray, src: np.ndarray) -> np.ndarray:
+    """Dispatch ([Primer] phase (b)): row r of the receive buffer is token src[r]'s row.
+    A bitwise copy; each token lands once per chosen expert (O(top-k) volume)."""
+    return np.asarray(x)[np.asarray(src)]
+
+
+def prefetch(plan, W1, W3, W2, R: int, S: int):
+    """Prefetch of redundant copies ([MoonEP] para. 3): pool slot u*S+s receives the
+    home weights of replica_expert[u*S+s], bitwise, for all three projections.
+    Returns dict slot -> (w1, w3, w2) for the filled slots."""
+    out = {}
+    for slot in range(R * S):
+        e = plan["replica_expert"][slot]
+        if e >= 0:
+            out[slot] = (W1[e].copy(), W3[e].copy(), W2[e].copy())
+    return out
+
+
+# ------------------------------------------------------------------ expert FFN
+def silu(z):
+    """silu(z) = z * sigmoid(z) = z / (1 + exp(-z)), fp64."""
+    with np.errstate(over="ignore"):
+        return z / (1.0 + np.exp(-z))
+
+
+def expert_ffn(X, w1, w3, w2):
+    """One SwiGLU expert on a block of rows, fp64 ([Primer] phase (c)):
+    y = (silu(X w1^T) * (X w3^T)) w2^T with w1, w3 [F,d] and w2 [d,F]."""
+    X = np.asarray(X, dtype=np.float64)
+    g = X @ np.asarray(w1, dtype=np.float64).T
+    u = X @ np.asarray(w3, dtype=np.float64).T
+    h = silu(g) * u
+    return h @ np.asarray(w2, dtype=np.float64).T
+
+
+def weights_of(weight_ref: int, E: int, W1, W3, W2, pool):
+    """Weights a group reads: the home tensor for weight_ref < E, else pool slot
+    weight_ref - E."""
+    if weight_ref < E:
+        return W1[weight_ref], W3[weight_ref], W2[weight_ref]
+    return pool[weight_ref - E]
+
+
+def grouped_ffn(recv, plan, E: int, W1, W3, W2, pool, rows=None):
+    """Grouped GEMM over the plan's groups ([Primer] phase (c)): every row of the
+    receive buffer goes through the expert of the group holding it.  ``rows`` limits the
+    evaluation to a subset (sampled parity); returns {row: y_row} then, else y [R*C,d]."""
+    recv = np.asarray(recv)
+    if rows is None:
+        y = np.zeros((recv.shape[0], W2.shape[1]), dtype=np.float64)
+        for u_groups in plan["groups"]:
+            for (r0, n, e, ref) in u_groups:
+                w1, w3, w2 = weights_of(ref, E, W1, W3, W2, pool)
+                y[r0:r0 + n] = expert_ffn(recv[r0:r0 + n], w1, w3, w2)
+        return y
+    want = set(int(r) for r in rows)
+    out = {}
+    for u_groups in plan["groups"]:
+        for (r0, n, e, ref) in u_groups:
+            sel = [r for r in range(r0, r0 + n) if r in want]
+            if not sel:
+                continue
+            w1, w3, w2 = weights_of(ref, E, W1, W3, W2, pool)
+            ys = expert_ffn(recv[sel], w1, w3, w2)
+            for r, yr in zip(sel, ys):
+                out[r] = yr
+    return out
+
+
+# ------------------------------------------------------------------ combine
+def combine(y, perm, gate, tokens=None):
+    """Combine ([Primer] phase (d), the transpose of dispatch): token t's output is
+    sum_j gate[t,j] * y[perm[t,j]], accumulated in j order in fp64.  ``y`` may be an
+    array or a {row: vector} map (sampled parity); ``tokens`` limits the evaluation."""
+    perm = np.asarray(perm)
+    gate = np.asarray(gate, dtype=np.float64)
+    T, k = perm.shape
+    toks = range(T) if tokens is None else tokens
+    out = {}
+    for t in toks:
+        acc = None
+        for j in range(k):
+            v = gate[t, j] * np.asarray(y[int(perm[t, j])], dtype=np.float64)
+            acc = v if acc is None else acc + v
+        out[int(t)] = acc
+    if tokens is None:
+        return np.stack([out[t] for t in range(T)]) if T else np.zeros((0, 0))
+    return out
+
+
+# ------------------------------------------------------------------ whole layer
+def layer(logits, x, W1, W3, W2, k: int, R: int, S: int):
+    """The whole path in the pages' order: route, measure, plan, prefetch, place rows,
+    expert FFN, combine.  Small shapes only (loops are plain Python)."""
+    logits = np.asarray(logits, dtype=np.float32)
+    T, E = logits.shape
+    idx, gate, err = topk_route(logits, k)
+    h = expert_histogram(idx, E, R)
+    err |= h["err"]
+    plan = plan_balanced(h["counts"], T, k, E, R, S)
+    err |= plan["err"]
+    pool = prefetch(plan, W1, W3, W2, R, S)
+    perm, src = permute(idx, plan, E, R)
+    recv = dispatch(x, src)
+    y = grouped_ffn(recv, plan, E, W1, W3, W2, pool)
+    out = combine(y, perm, gate)
+    return dict(idx=idx, gate=gate, hist=h, plan=plan, pool=pool, perm=perm, src=src,
+                recv=recv, y=y, out=out, err=err)
+
