@@ -1,0 +1,404 @@
+"""Throughput of the MoE-layer hot path on B200: one JSON line on stdout (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+A step is one pass of the whole path (top-k, histogram/maxvio, balanced plan, replica
+prefetch, dispatch, grouped SwiGLU FFN, combine) over one batch of seeded synthetic
+inputs already resident in HBM.  The default workload is the near-balanced fine-grained
+layer (4096 tokens, 64 experts, top-6, 8 simulated ranks, 8 slots, d=2048, F=1408).
+Under torchrun (N > 1) every rank runs an independent replica of the same layer on its
+own GPU (no collective on the data path); timing is the max over ranks.
+
+`--impl reference` times the CPU oracle instead (rank 0 only), on a bounded sample of the
+same workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from load_balanced_dispatch_warp_b200 import inputs as I  # noqa: E402
+
+METRIC = "MoE layer tokens/s"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM bytes per launch of the dominant call from an ncu capture, keyed by the workload;
+# valid only while the kernel sources hash to the recorded value.
+TRAFFIC = {}
+
+
+def sources_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("grouped_ffn.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "load_balanced_dispatch_warp_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.gpu = gpu_index
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smmax=float(parts[2]), hw=parts[5], hwt=parts[6],
+                                 swt=parts[7], pcap=parts[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        busy = [r for r in rows if r["sm"] > 0.5 * r["smmax"]] or rows
+        reasons = set()
+        for r in busy:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in busy), "sm_max_mhz": busy[0]["smmax"],
+                "reasons": sorted(reasons), "samples": len(busy)}
+
+
+# ----------------------------------------------------------------------------- work units
+def algorithmic(w: I.Workload, n_rep: int):
+    """Algorithmic bytes (HBM) or flops per call for one step."""
+    T, E, k, d, F, A = w.T, w.E, w.k, w.d, w.F, w.A
+    return {
+        "moe_topk": ("GB/s", T * E * 4 + A * 8),
+        "moe_histogram_maxvio": ("GB/s", A * 4 + E * 4),
+        "moe_plan_balanced": ("us", None),
+        "moe_prefetch_replicas": ("GB/s", 2 * n_rep * 3 * d * F * 2),
+        "moe_dispatch": ("GB/s", T * d * 2 + A * d * 2 + 12 * A),
+        "moe_grouped_ffn": ("TFLOP/s", 6 * A * d * F),
+        "moe_combine": ("GB/s", A * d * 2 + T * d * 2 + 8 * A),
+    }
+
+
+CALLS = ["moe_topk", "moe_histogram_maxvio", "moe_plan_balanced", "moe_prefetch_replicas",
+         "moe_dispatch", "moe_grouped_ffn", "moe_combine"]
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args, w: I.Workload, world, rank, local):
+    import load_balanced_dispatch_warp_b200 as M
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    logits_h = I.make_logits(w).pin_memory()
+    x_h = I.make_x(w).pin_memory()
+    logits = logits_h.to(device)
+    x = x_h.to(device)
+    W1, W3, W2 = I.make_weights(w, device=device)
+    L = M.MoELayer(w.T, w.E, w.k, w.R, w.S, w.d, w.F, device=device)
+    steps = [lambda: L.route(logits), lambda: L.measure(), lambda: L.balance(),
+             lambda: L.prefetch(W1, W3, W2), lambda: L.dispatch(x),
+             lambda: L.expert_ffn(W1, W3, W2), lambda: L.combine()]
+
+    for _ in range(max(args.warmup, 1)):
+        L.forward(logits, x, W1, W3, W2)
+    torch.cuda.synchronize()
+    if int(L.err.item()) != 0:
+        raise RuntimeError(f"device error word {int(L.err.item())} after warm-up")
+    n_rep = int(L.plan_field("replica_list")[0].item())
+
+    # device-timed region: K steps, events between the calls on the launching stream
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(steps) + 1)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.mark_start()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for s in range(args.steps):
+        e = ev[s]
+        e[0].record(stream)
+        for i, f in enumerate(steps):
+            f()
+            e[i + 1].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks.mark_end()
+    clk = clocks.stop()
+    elapsed_ms = start.elapsed_time(end)
+    elapsed_ms = max_over_ranks(elapsed_ms, world, device)
+    if int(L.err.item()) != 0:
+        raise RuntimeError(f"device error word {int(L.err.item())} in the timed region")
+    per_call_ms = {c: sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(args.steps)) / args.steps
+                   for i, c in enumerate(CALLS)}
+
+    # end to end: host buffers in, host result out, every step
+    out_h = torch.empty(w.T, w.d, dtype=torch.bfloat16).pin_memory()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        logits.copy_(logits_h, non_blocking=True)
+        x.copy_(x_h, non_blocking=True)
+        L.forward(logits, x, W1, W3, W2)
+        out_h.copy_(L.out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
+
+    units = algorithmic(w, n_rep)
+    peaks, peak_src = load_peaks()
+    calls = {}
+    for c in CALLS:
+        unit, work = units[c]
+        ms = per_call_ms[c]
+        rec = {"us": round(ms * 1e3, 2)}
+        if work is not None and ms > 0:
+            if unit == "TFLOP/s":
+                ach = work / (ms * 1e-3) / 1e12
+                peak = peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]
+            else:
+                ach = work / (ms * 1e-3) / 1e9
+                peak = peaks["hbm_gbs"]
+            rec.update({unit.replace("/", "_per_"): round(ach, 1), "frac": round(ach / peak, 3)})
+        calls[c] = rec
+    ffn_ms = per_call_ms["moe_grouped_ffn"]
+    ffn_flops = units["moe_grouped_ffn"][1]
+    peak_t = peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]
+    achieved = ffn_flops / (ffn_ms * 1e-3) / 1e12
+    tkey = f"{w.name}:{sources_hash()}"
+    roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak_t, "unit": "TFLOP/s",
+                "frac": round(achieved / peak_t, 3), "traffic": TRAFFIC.get(tkey),
+                "kernel": "moe_grouped_ffn (gate-up and down tcgen05 GEMMs)",
+                "peak_source": f"{peak_src} sustained bf16 GEMM",
+                "work_per_launch": f"6*A*d*F = {ffn_flops:.4g} flop (A=T*k={w.A})"}
+
+    value = w.T * args.steps * world / (elapsed_ms * 1e-3)
+    e2e_value = w.T * args.steps * world / (e2e_ms * 1e-3)
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(elapsed_ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; N(0,1) logits + per-expert bias, N(0,1) tokens, N(0,1/d) weights)",
+        "config": {"workload": w.name, "T": w.T, "E": w.E, "k": w.k, "R": w.R, "S": w.S, "d": w.d,
+                   "F": w.F, "maxvio": round(float(L.maxvio.item()), 4), "replicas": n_rep,
+                   "parallelism": f"replicas x{world} (ranks simulated in one GPU's HBM)",
+                   "l2": "step working set (weights, pool, activations) far above the 126 MB L2",
+                   "launch": "eager, one stream"},
+        "clocks": clk,
+        "e2e": {"value": round(e2e_value, 1), "unit": UNIT,
+                "h2d_bytes_per_step": w.T * w.E * 4 + w.T * w.d * 2,
+                "d2h_bytes_per_step": w.T * w.d * 2},
+        "gpu_launches": L.kernels_per_forward() * args.steps,
+        "roofline": roofline,
+        "calls": calls,
+    }
+    return res
+
+
+# ----------------------------------------------------------------------------- oracle
+def oracle_sample_tokens(w: I.Workload) -> int:
+    """Tokens per CPU-oracle step: a prefix of the batch, a multiple of R/gcd(k,R)."""
+    import math
+    unit = w.R // math.gcd(w.k, w.R)
+    target = max(unit, int(2.0e9 / (6 * w.k * w.d * w.F)))  # about 2 GFLOP of fp64 FFN work
+    target = min(target, w.T)
+    return max(unit, target // unit * unit)
+
+
+def run_oracle_step(w: I.Workload, logits, x, weights64_fn, Ts: int):
+    from oracle import moe_oracle as O
+    lg = logits[:Ts]
+    xs = x[:Ts]
+    idx, gate, err = O.topk_route(lg, w.k)
+    h = O.expert_histogram(idx, w.E, w.R)
+    p = O.plan_balanced(h["counts"], Ts, w.k, w.E, w.R, w.S)
+    perm, src = O.permute(idx, p, w.E, w.R)
+    recv = O.dispatch(xs, src)
+    y = np.zeros((recv.shape[0], w.d))
+    for gl in p["groups"]:
+        for (r0, n, e, ref) in gl:
+            w1, w3, w2 = weights64_fn(e)  # a replica slot holds these weights bitwise
+            y[r0:r0 + n] = O.expert_ffn(recv[r0:r0 + n], w1, w3, w2)
+    return O.combine(y, perm, gate)
+
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_inputs(w: I.Workload):
+    logits = I.make_logits(w).numpy()
+    x = I.make_x(w).double().numpy()
+    cache = {}
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    W = I.make_weights(w, device=dev) if w.E * w.F * w.d * 3 * 2 < 60e9 else None
+
+    def weights64(e):
+        if e not in cache:
+            cache[e] = tuple(t[e].to("cpu", torch.float64).numpy() for t in W)
+        return cache[e]
+    return logits, x, weights64
+
+
+def measure_oracle(w: I.Workload, steps: int, warmup: int, budget_s: float | None = None):
+    logits, x, weights64 = oracle_inputs(w)
+    Ts = oracle_sample_tokens(w)
+    for _ in range(warmup):
+        run_oracle_step(w, logits, x, weights64, Ts)
+    t0 = time.perf_counter()
+    n = 0
+    for _ in range(steps):
+        run_oracle_step(w, logits, x, weights64, Ts)
+        n += 1
+        if budget_s is not None and time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return Ts * n / dt, Ts, n, dt
+
+
+def run_reference(args, w):
+    world, rank, local = dist_env()
+    if rank != 0:
+        return None
+    if torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    value, Ts, n, dt = measure_oracle(w, args.steps, args.warmup)
+    cores = cpu_threads()
+    sample = f"first {Ts} of {w.T} tokens through the whole oracle layer per step, {n} steps"
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": 1,
+        "steps": n, "warmup": args.warmup, "ms_per_step": round(dt / n * 1e3, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": {"workload": w.name, "T": w.T, "E": w.E, "k": w.k, "R": w.R, "S": w.S, "d": w.d,
+                   "F": w.F},
+        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="near_balanced", choices=sorted(I.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = I.WORKLOADS[args.config]
+
+    if args.impl == "reference":
+        res = run_reference(args, w)
+        if res is not None:
+            print(json.dumps(res, sort_keys=True), flush=True)
+        return
+
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    res = run_ours(args, w, world, rank, local)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        value, Ts, n, dt = measure_oracle(w, steps=1000, warmup=0, budget_s=15.0)
+        res["cpu_baseline"] = {"value": round(value, 3), "unit": UNIT, "cores": cpu_threads(),
+                               "kind": "oracle",
+                               "sample": f"first {Ts} of {w.T} tokens through the whole oracle "
+                                         f"layer, {n} passes in {dt:.1f} s"}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res, sort_keys=True), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,225 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) MoE-layer hot path:
+ *          route -> balance -> dispatch -> expert FFN -> combine on one GPU.
+ *
+ * The R expert-parallel ranks are partitions of this GPU's HBM: rank u owns rows
+ * [u*C, (u+1)*C) of every per-rank buffer, C = T*k/R ("a rank may mean one process, one
+ * accelerator, or one partition", "MoE Load Balancing: Find Expert Hotspots", section
+ * "Reject incomparable MoE load-balancing traces").
+ *
+ * Sources cited below (page title, section):
+ *   [MoonEP]   "Moonshot AI drops MoonEP, claims 2.5x scaling boost for trillion-parameter
+ *              models" (news article), paragraphs 2-4.
+ *   [Primer]   "DeepEP-on-EFA Guidance, section 1: What is MoE", the four-phase
+ *              expert-parallel pipeline (a) router, (b) dispatch, (c) expert FFN,
+ *              (d) combine.
+ *   [Hotspots] "MoE Load Balancing: Find Expert Hotspots".
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer argument is a DEVICE pointer unless stated otherwise, allocated and
+ *     owned by the caller; the library never allocates, frees or synchronises.  All work
+ *     is enqueued asynchronously on `stream` (a cudaStream_t; NULL = legacy default).
+ *   - 16-bit tensors are passed as moe_bf16 / moe_f16 (raw bit patterns); layouts are
+ *     row-major and contiguous.  Token rows and the up/gate projections W1, W3 are bf16;
+ *     the down projection W2 and the activations h are fp16 (see moe_grouped_ffn).
+ *   - Return value: a host status (MOE_OK, or an MOE_ERR_* code) decided from the
+ *     scalar arguments and pointer nullness BEFORE anything is enqueued; on a non-zero
+ *     status nothing was enqueued.  MOE_ERR_LAUNCH reports a failed launch.
+ *   - Data-dependent errors are OR-ed into the caller's device word `*err` (int32) with
+ *     the MOE_DERR_* bits.  moe_topk sets *err to 0 first (it begins a layer); a caller
+ *     that skips moe_topk must zero *err itself.  Every other call reads *err on the
+ *     device and does nothing when it is non-zero, so a bad trace stops the layer without
+ *     a host sync; its outputs are then unspecified.  Nothing traps or asserts.
+ *   - Size limits: 1 <= k <= min(E, 32), E <= 1024, E % R == 0, (T*k) % R == 0,
+ *     d % 128 == 0, F % 128 == 0, R*(E/R + S) <= 4096, every element count < 2^31.
+ *     T == 0 is allowed (every call is then a no-op apart from clearing outputs that
+ *     are defined for it).
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t moe_bf16;   /* bfloat16 bit pattern */
+typedef uint16_t moe_f16;    /* IEEE binary16 bit pattern */
+typedef void* moe_stream_t;  /* cudaStream_t */
+
+/* host status codes */
+enum {
+  MOE_OK = 0,
+  MOE_ERR_ARG = 1,     /* null pointer or negative size                              */
+  MOE_ERR_SHAPE = 2,   /* a size limit above is violated                             */
+  MOE_ERR_LAUNCH = 3,  /* a CUDA launch or attribute call failed                     */
+  MOE_ERR_DEVICE = 4   /* no usable sm_100 device / driver entry point               */
+};
+
+/* device error-word bits */
+enum {
+  MOE_DERR_NONFINITE = 1,  /* a router logit is NaN or +-inf                         */
+  MOE_DERR_ID_RANGE = 2,   /* an expert id outside [0, E)                            */
+  MOE_DERR_DUPLICATE = 4,  /* a token names the same expert twice                    */
+  MOE_DERR_SLOTS = 8,      /* the plan needs more than S replicas on some rank       */
+  MOE_DERR_TIMEOUT = 16    /* a bounded wait inside the grouped FFN gave up          */
+};
+
+/* Word offsets of the plan's fields inside the caller's int32 plan buffer. */
+typedef struct moe_plan_layout {
+  int64_t kept_rows;       /* [R]   rows of rank u held by experts kept whole at home      */
+  int64_t room_prefix;     /* [R+1] exclusive prefix of the ranks' rooms (C - kept_rows)   */
+  int64_t expert_home_off; /* [E]   local row offset of a kept expert at home, -1 streamed  */
+  int64_t stream_off;      /* [E+1] exclusive prefix over e of (streamed ? count[e] : 0)    */
+  int64_t replica_expert;  /* [R*S] expert held by pool slot u*S+s, -1 if empty            */
+  int64_t replica_list;    /* [1+R*S] number of filled slots, then their ids ascending     */
+  int64_t n_groups;        /* [R]   groups of rank u                                        */
+  int64_t groups;          /* [R*(B+S)][4] {row_start (global row), rows, expert,
+                                    weight_ref}; weight_ref = e (< E) reads the home
+                                    tensors, E + u*S + s reads pool slot u*S+s; entries
+                                    past n_groups[u] are all -1                             */
+  int64_t words;           /* total int32 words of the plan buffer                          */
+  int32_t max_groups_per_rank; /* B + S                                                     */
+} moe_plan_layout;
+
+/* Fills *out with the plan layout for (E, R, S).  Host only; returns a host status. */
+int moe_plan_get_layout(int E, int R, int S, moe_plan_layout* out);
+
+/* int32 words of the workspace moe_dispatch needs for T tokens and E experts. */
+int64_t moe_dispatch_workspace_words(int T, int E);
+
+/* Static description of a host status code. */
+const char* moe_status_string(int status);
+
+/* ---------------------------------------------------------------------------------
+ * (a) Router: top-k choice and gate weights.   [Primer] phase (a): the router scores
+ * all experts per token, keeps the top-k and produces the routing table (token ->
+ * experts plus combine weights).
+ *   logits [T,E] fp32            router scores.
+ *   idx    [T,k] int32  (out)    the k largest logits per token, descending; equal
+ *                                logits are ordered by the lower expert id (+0 == -0).
+ *   gate   [T,k] fp32   (out)    softmax over the k selected logits,
+ *                                gate_j = exp(l_j - l_0) / sum_i exp(l_i - l_0).
+ *   err    int32        (in/out) set to 0, then bit MOE_DERR_NONFINITE if any logit is
+ *                                not finite (that token's outputs are unspecified).
+ */
+int moe_topk(const float* logits, int T, int E, int k,
+             int32_t* idx, float* gate, int32_t* err, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * Demand histogram and imbalance.   [Hotspots] "Separate expert demand from rank
+ * placement": count assignments per expert, then sum over an expert->rank mapping;
+ * balancedness = mean/max.  [MoonEP] para. 2: maxvio is 0 when perfectly balanced,
+ * here (max rank load - mean)/mean.  [Hotspots] "Work the 16-token hotspot fixture":
+ * ids must be known experts and a token may not repeat one.
+ *   idx            [T,k] int32        expert choices (e.g. from moe_topk).
+ *   expert_to_rank [E] int32 or NULL  owning rank of each expert; NULL = e / (E/R).
+ *   counts         [E] int32  (out)   assignments per expert (in-range ids only).
+ *   loads          [R] int32  (out)   assignments per rank under the mapping.
+ *   maxvio         [1] fp64   (out)   (R*max(loads) - T*k) / (T*k), one rounding;
+ *                                     0 when T == 0.
+ *   balancedness   [1] fp64   (out)   (T*k) / (R*max(loads)); 1 when T == 0.
+ *   err            int32      (in/out) bits MOE_DERR_ID_RANGE, MOE_DERR_DUPLICATE.
+ */
+int moe_histogram_maxvio(const int32_t* idx, int T, int k, int E, int R,
+                         const int32_t* expert_to_rank, int32_t* counts, int32_t* loads,
+                         double* maxvio, double* balancedness, int32_t* err,
+                         moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * Equal-load plan with redundant expert copies.   [MoonEP] para. 3-4: every rank
+ * receives exactly the same number of tokens, by planning a few redundant expert copies
+ * on the fly from the router output; copies live in S prefetch slots per rank drawn
+ * from one process-global pool.  The article gives no algorithm; this one is
+ * "keep small, stream the rest" (deterministic, scan-based):
+ *   1. rank r owns experts [rB, (r+1)B), B = E/R; C = T*k/R;
+ *   2. per rank, experts ordered by (count, id) ascending are kept whole while they fit
+ *      in C; the first that does not fit and all after it are streamed;
+ *   3. the streamed experts in id order form one stream; the ranks' leftover rooms,
+ *      concatenated in rank order, cut it: each rank's piece fills its rows after its
+ *      kept experts;
+ *   4. each run of a foreign expert in a rank's piece is a replica taking the rank's
+ *      next slot; more than S sets MOE_DERR_SLOTS.
+ *   counts [E] int32   expert demand (from moe_histogram_maxvio).
+ *   plan   int32[moe_plan_layout.words] (out)  the fields of moe_plan_layout.
+ *   err    int32       (in/out) bit MOE_DERR_SLOTS; no-op when already non-zero.
+ * One CTA; O(E*B + R*E) work.
+ */
+int moe_plan_balanced(const int32_t* counts, int T, int k, int E, int R, int S,
+                      int32_t* plan, int32_t* err, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * Prefetch of the replicas into the pool.   [MoonEP] para. 3: duplicated experts are
+ * prefetched before computation from one process-global pool, not per layer; the
+ * framework keeps one contiguous weight tensor per projection.
+ *   W1, W3 [E,F,d] bf16, W2 [E,d,F] fp16     home expert weights.
+ *   P1, P3 [R*S,F,d] bf16, P2 [R*S,d,F] fp16 (out) the pool; slot u*S+s receives a
+ *          bitwise copy of expert replica_expert[u*S+s]; empty slots are not written.
+ *          The pool is owned by the caller and may be shared by every layer.
+ *   err    no-op when non-zero.
+ */
+int moe_prefetch_replicas(const int32_t* plan, const moe_bf16* W1, const moe_bf16* W3,
+                          const moe_f16* W2, int E, int R, int S, int d, int F,
+                          moe_bf16* P1, moe_bf16* P3, moe_f16* P2, const int32_t* err,
+                          moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * Zero-copy placement and dispatch.   [Primer] phase (b): every token is sent to its k
+ * chosen experts (O(top-k) volume); [MoonEP] para. 3: tokens go straight to their final
+ * row of a static-shape buffer.  Assignment (t,j) of expert e is the q-th assignment of
+ * e in token order; a kept expert's q-th row is home(e)*C + expert_home_off[e] + q, a
+ * streamed expert's is stream position p = stream_off[e] + q, on the rank u whose room
+ * range holds p, row u*C + kept_rows[u] + p - room_prefix[u].
+ *   x         [T,d] bf16      token rows.
+ *   idx       [T,k] int32     expert choices (validated by moe_histogram_maxvio).
+ *   workspace int32[moe_dispatch_workspace_words(T,E)]  scratch (caller-owned).
+ *   recv      [R*C,d] bf16 (out)  recv[perm[t,j]] = x[t] bitwise.
+ *   perm      [T,k] int32  (out)  row of each assignment.
+ *   src       [R*C] int32  (out)  token of each row.
+ *   err       no-op when non-zero.
+ */
+int moe_dispatch(const moe_bf16* x, const int32_t* idx, const int32_t* plan, int T, int k,
+                 int E, int R, int S, int d, int32_t* workspace, moe_bf16* recv,
+                 int32_t* perm, int32_t* src, int32_t* err, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * Grouped SwiGLU expert FFN.   [Primer] phase (c): each rank runs its local experts
+ * over the rows it received as a batched grouped GEMM.  For every plan group (rows of
+ * one rank holding one expert or replica):
+ *   h = silu(X W1^T) * (X W3^T)   (bf16 x bf16, fp32 accumulate; silu(z) = z/(1+e^-z);
+ *                                  stored as fp16, saturated to +-65504)
+ *   y = h W2^T                    (fp16 x fp16, fp32 accumulate; bf16 out)
+ * with the home tensors (weight_ref < E) or the pool slot (weight_ref >= E).  The down
+ * projection runs in fp16 because a tensor-core MMA takes both operands in one type and
+ * h rounded to bf16 (8 significant bits) leaves y's worst element near the 1e-2 parity
+ * bound when F/d >= 2; fp16 holds 11 bits at the same rate.  bf16 weight values with
+ * 2^-17 <= |w| <= 65504 convert to fp16 exactly.
+ *   recv [R*C,d] bf16           rows from moe_dispatch.
+ *   W1, W3 [E,F,d] bf16; W2 [E,d,F] fp16; P1, P3, P2 the pool (same types).
+ *   h    [R*C,F] fp16 (out)     the SwiGLU activations (caller-owned scratch).
+ *   y    [R*C,d] bf16 (out)     expert outputs.
+ *   err  no-op when non-zero; MOE_DERR_TIMEOUT if a pipeline wait exceeded its bound.
+ * Two persistent tcgen05/TMEM kernels fed by TMA.
+ */
+int moe_grouped_ffn(const moe_bf16* recv, const int32_t* plan, const moe_bf16* W1,
+                    const moe_bf16* W3, const moe_f16* W2, const moe_bf16* P1,
+                    const moe_bf16* P3, const moe_f16* P2, int T, int k, int E, int R,
+                    int S, int d, int F, moe_f16* h, moe_bf16* y, int32_t* err,
+                    moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * Combine.   [Primer] phase (d): expert outputs return to their token and are summed
+ * with the gate weights; the mirror (transpose) of dispatch.
+ *   out[t] = sum_{j=0..k-1} gate[t,j] * y[perm[t,j]]   (fp32, j order; bf16 out)
+ *   y [R*C,d] bf16, perm [T,k] int32, gate [T,k] fp32, out [T,d] bf16 (out).
+ *   err  no-op when non-zero.
+ */
+int moe_combine(const moe_bf16* y, const int32_t* perm, const float* gate, int T, int k,
+                int d, moe_bf16* out, const int32_t* err, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

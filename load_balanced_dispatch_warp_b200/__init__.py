@@ -1,0 +1,264 @@
+"""Python binding of ``libmoe.so``: the MoE-layer hot path on one B200.
+
+Argument marshalling only: each function below checks the tensors' dtype, device and
+contiguity, passes raw device pointers and sizes to the C entry point of the same name
+(declared in ``include/moe.h``) on the current CUDA stream, and raises on a non-zero host
+status.  Every step of the path runs in the library's CUDA kernels; there is no CPU
+fallback, and importing a function raises if the library has not been built.
+
+``MoELayer`` owns the per-layer device buffers (PyTorch allocations) and runs the seven
+calls in order: route, measure, plan, prefetch, dispatch, expert FFN, combine.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+MOE_OK, MOE_ERR_ARG, MOE_ERR_SHAPE, MOE_ERR_LAUNCH, MOE_ERR_DEVICE = range(5)
+DERR_NONFINITE, DERR_ID_RANGE, DERR_DUPLICATE, DERR_SLOTS, DERR_TIMEOUT = 1, 2, 4, 8, 16
+
+ENTRY_POINTS = ("moe_topk", "moe_histogram_maxvio", "moe_plan_balanced", "moe_prefetch_replicas",
+                "moe_dispatch", "moe_grouped_ffn", "moe_combine")
+HELPERS = ("moe_plan_get_layout", "moe_dispatch_workspace_words", "moe_status_string")
+
+
+class MoEError(RuntimeError):
+    pass
+
+
+class PlanLayout(ctypes.Structure):
+    _fields_ = [("kept_rows", ctypes.c_int64), ("room_prefix", ctypes.c_int64),
+                ("expert_home_off", ctypes.c_int64), ("stream_off", ctypes.c_int64),
+                ("replica_expert", ctypes.c_int64), ("replica_list", ctypes.c_int64),
+                ("n_groups", ctypes.c_int64), ("groups", ctypes.c_int64),
+                ("words", ctypes.c_int64), ("max_groups_per_rank", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m load_balanced_dispatch_warp_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, I64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+        sig = {
+            "moe_topk": [P, I, I, I, P, P, P, P],
+            "moe_histogram_maxvio": [P, I, I, I, I, P, P, P, P, P, P, P],
+            "moe_plan_balanced": [P, I, I, I, I, I, P, P, P],
+            "moe_prefetch_replicas": [P, P, P, P, I, I, I, I, I, P, P, P, P, P],
+            "moe_dispatch": [P, P, P, I, I, I, I, I, I, P, P, P, P, P, P],
+            "moe_grouped_ffn": [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, P],
+            "moe_combine": [P, P, P, I, I, I, P, P, P],
+        }
+        for name, args in sig.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = ctypes.c_int
+        L.moe_plan_get_layout.argtypes = [I, I, I, ctypes.POINTER(PlanLayout)]
+        L.moe_plan_get_layout.restype = ctypes.c_int
+        L.moe_dispatch_workspace_words.argtypes = [I, I]
+        L.moe_dispatch_workspace_words.restype = I64
+        L.moe_status_string.argtypes = [I]
+        L.moe_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _check(status: int, what: str):
+    if status != MOE_OK:
+        raise MoEError(f"{what}: {lib().moe_status_string(status).decode()} (status {status})")
+
+
+def _ptr(t, dtype, name):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr() if t.numel() else None
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def plan_layout(E: int, R: int, S: int) -> PlanLayout:
+    L = PlanLayout()
+    _check(lib().moe_plan_get_layout(E, R, S, ctypes.byref(L)), "moe_plan_get_layout")
+    return L
+
+
+def dispatch_workspace_words(T: int, E: int) -> int:
+    return int(lib().moe_dispatch_workspace_words(T, E))
+
+
+# ----------------------------------------------------------------- the seven entry points
+def moe_topk(logits, k, idx, gate, err, stream=None):
+    T, E = logits.shape
+    _check(lib().moe_topk(_ptr(logits, torch.float32, "logits"), T, E, k,
+                          _ptr(idx, torch.int32, "idx"), _ptr(gate, torch.float32, "gate"),
+                          _ptr(err, torch.int32, "err"), _stream(stream)), "moe_topk")
+
+
+def moe_histogram_maxvio(idx, E, R, counts, loads, maxvio, balancedness, err,
+                         expert_to_rank=None, stream=None):
+    T, k = idx.shape
+    _check(lib().moe_histogram_maxvio(
+        _ptr(idx, torch.int32, "idx"), T, k, E, R, _ptr(expert_to_rank, torch.int32, "expert_to_rank"),
+        _ptr(counts, torch.int32, "counts"), _ptr(loads, torch.int32, "loads"),
+        _ptr(maxvio, torch.float64, "maxvio"), _ptr(balancedness, torch.float64, "balancedness"),
+        _ptr(err, torch.int32, "err"), _stream(stream)), "moe_histogram_maxvio")
+
+
+def moe_plan_balanced(counts, T, k, R, S, plan, err, stream=None):
+    E = counts.shape[0]
+    _check(lib().moe_plan_balanced(_ptr(counts, torch.int32, "counts"), T, k, E, R, S,
+                                   _ptr(plan, torch.int32, "plan"), _ptr(err, torch.int32, "err"),
+                                   _stream(stream)), "moe_plan_balanced")
+
+
+def moe_prefetch_replicas(plan, W1, W3, W2, R, S, P1, P3, P2, err, stream=None):
+    E, F, d = W1.shape
+    bf, hf = torch.bfloat16, torch.float16
+    _check(lib().moe_prefetch_replicas(
+        _ptr(plan, torch.int32, "plan"), _ptr(W1, bf, "W1"), _ptr(W3, bf, "W3"), _ptr(W2, hf, "W2"),
+        E, R, S, d, F, _ptr(P1, bf, "P1"), _ptr(P3, bf, "P3"), _ptr(P2, hf, "P2"),
+        _ptr(err, torch.int32, "err"), _stream(stream)), "moe_prefetch_replicas")
+
+
+def moe_dispatch(x, idx, plan, E, R, S, workspace, recv, perm, src, err, stream=None):
+    T, d = x.shape
+    k = idx.shape[1]
+    _check(lib().moe_dispatch(
+        _ptr(x, torch.bfloat16, "x"), _ptr(idx, torch.int32, "idx"), _ptr(plan, torch.int32, "plan"),
+        T, k, E, R, S, d, _ptr(workspace, torch.int32, "workspace"), _ptr(recv, torch.bfloat16, "recv"),
+        _ptr(perm, torch.int32, "perm"), _ptr(src, torch.int32, "src"), _ptr(err, torch.int32, "err"),
+        _stream(stream)), "moe_dispatch")
+
+
+def moe_grouped_ffn(recv, plan, W1, W3, W2, P1, P3, P2, T, k, R, S, h, y, err, stream=None):
+    E, F, d = W1.shape
+    bf, hf = torch.bfloat16, torch.float16
+    _check(lib().moe_grouped_ffn(
+        _ptr(recv, bf, "recv"), _ptr(plan, torch.int32, "plan"), _ptr(W1, bf, "W1"),
+        _ptr(W3, bf, "W3"), _ptr(W2, hf, "W2"), _ptr(P1, bf, "P1"), _ptr(P3, bf, "P3"),
+        _ptr(P2, hf, "P2"), T, k, E, R, S, d, F, _ptr(h, hf, "h"), _ptr(y, bf, "y"),
+        _ptr(err, torch.int32, "err"), _stream(stream)), "moe_grouped_ffn")
+
+
+def moe_combine(y, perm, gate, out, err, stream=None):
+    T, k = perm.shape
+    d = out.shape[1]
+    _check(lib().moe_combine(_ptr(y, torch.bfloat16, "y"), _ptr(perm, torch.int32, "perm"),
+                             _ptr(gate, torch.float32, "gate"), T, k, d,
+                             _ptr(out, torch.bfloat16, "out"), _ptr(err, torch.int32, "err"),
+                             _stream(stream)), "moe_combine")
+
+
+# ----------------------------------------------------------------- one layer
+class MoELayer:
+    """Device buffers of one MoE layer of shape (T, E, k, R, S, d, F) and the seven calls.
+
+    The replica pool (P1, P3, P2: R*S slots) is allocated once here; several layers may
+    share one pool by passing ``pool=`` (it is process-global in the MoonEP design).
+    """
+
+    def __init__(self, T, E, k, R, S, d, F, device="cuda", pool=None):
+        self.T, self.E, self.k, self.R, self.S, self.d, self.F = T, E, k, R, S, d, F
+        self.A = T * k
+        self.C = self.A // R
+        dev = torch.device(device)
+        i32, f32, bf = torch.int32, torch.float32, torch.bfloat16
+        self.layout = plan_layout(E, R, S)
+        self.idx = torch.empty(T, k, dtype=i32, device=dev)
+        self.gate = torch.empty(T, k, dtype=f32, device=dev)
+        self.err = torch.zeros(1, dtype=i32, device=dev)
+        self.counts = torch.empty(E, dtype=i32, device=dev)
+        self.loads = torch.empty(R, dtype=i32, device=dev)
+        self.maxvio = torch.empty(1, dtype=torch.float64, device=dev)
+        self.balancedness = torch.empty(1, dtype=torch.float64, device=dev)
+        self.plan = torch.empty(self.layout.words, dtype=i32, device=dev)
+        self.workspace = torch.empty(max(1, dispatch_workspace_words(T, E)), dtype=i32, device=dev)
+        self.recv = torch.empty(self.A, d, dtype=bf, device=dev)
+        self.perm = torch.empty(T, k, dtype=i32, device=dev)
+        self.src = torch.empty(self.A, dtype=i32, device=dev)
+        self.h = torch.empty(self.A, F, dtype=torch.float16, device=dev)
+        self.y = torch.empty(self.A, d, dtype=bf, device=dev)
+        self.out = torch.empty(T, d, dtype=bf, device=dev)
+        if pool is None and S > 0:
+            pool = (torch.empty(R * S, F, d, dtype=bf, device=dev),
+                    torch.empty(R * S, F, d, dtype=bf, device=dev),
+                    torch.empty(R * S, d, F, dtype=torch.float16, device=dev))
+        self.pool = pool if S > 0 else (None, None, None)
+
+    def plan_field(self, name):
+        L = self.layout
+        sizes = dict(kept_rows=self.R, room_prefix=self.R + 1, expert_home_off=self.E,
+                     stream_off=self.E + 1, replica_expert=self.R * self.S,
+                     replica_list=1 + self.R * self.S, n_groups=self.R,
+                     groups=self.R * L.max_groups_per_rank * 4)
+        off = getattr(L, name)
+        return self.plan[off:off + sizes[name]]
+
+    # each step on its own (the caller orders them)
+    def route(self, logits, stream=None):
+        moe_topk(logits, self.k, self.idx, self.gate, self.err, stream)
+
+    def measure(self, expert_to_rank=None, stream=None):
+        moe_histogram_maxvio(self.idx, self.E, self.R, self.counts, self.loads, self.maxvio,
+                             self.balancedness, self.err, expert_to_rank, stream)
+
+    def balance(self, stream=None):
+        moe_plan_balanced(self.counts, self.T, self.k, self.R, self.S, self.plan, self.err, stream)
+
+    def prefetch(self, W1, W3, W2, stream=None):
+        P1, P3, P2 = self.pool
+        moe_prefetch_replicas(self.plan, W1, W3, W2, self.R, self.S, P1, P3, P2, self.err, stream)
+
+    def dispatch(self, x, stream=None):
+        moe_dispatch(x, self.idx, self.plan, self.E, self.R, self.S, self.workspace, self.recv,
+                     self.perm, self.src, self.err, stream)
+
+    def expert_ffn(self, W1, W3, W2, stream=None):
+        P1, P3, P2 = self.pool
+        moe_grouped_ffn(self.recv, self.plan, W1, W3, W2, P1, P3, P2, self.T, self.k, self.R,
+                        self.S, self.h, self.y, self.err, stream)
+
+    def combine(self, stream=None):
+        moe_combine(self.y, self.perm, self.gate, self.out, self.err, stream)
+
+    def forward(self, logits, x, W1, W3, W2, stream=None):
+        """The whole path on the current stream; returns ``out`` [T,d] bf16 (device)."""
+        self.route(logits, stream)
+        self.measure(None, stream)
+        self.balance(stream)
+        self.prefetch(W1, W3, W2, stream)
+        self.dispatch(x, stream)
+        self.expert_ffn(W1, W3, W2, stream)
+        self.combine(stream)
+        return self.out
+
+    # kernels launched by forward() (for launch accounting)
+    def kernels_per_forward(self) -> int:
+        n = (1 if self.T > 0 else 0) + (2 if self.T > 0 else 1) + 1  # topk, hist, plan
+        n += 1 if self.S > 0 else 0           # prefetch
+        n += 3 if self.T > 0 else 0           # dispatch: tile counts, ranks, row scatter
+        n += 2 if self.T > 0 else 0           # two grouped GEMMs
+        n += 1 if self.T > 0 else 0           # combine
+        return n

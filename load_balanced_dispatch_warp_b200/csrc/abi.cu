@@ -1,0 +1,218 @@
+// The C ABI (include/moe.h): argument checks, then one launcher per step.
+// Every check runs on the host before anything is enqueued.
+#include "common.cuh"
+
+namespace moe {
+
+int num_sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64) {
+    if (!cached[dev]) {
+      int n = 0;
+      if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        n = 148;
+      cached[dev] = n;
+    }
+    return cached[dev];
+  }
+  return 148;
+}
+
+}  // namespace moe
+
+namespace {
+
+constexpr int64_t kMaxElems = (int64_t)1 << 31;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_route(int T, int E, int k) {
+  if (T < 0 || E < 1 || k < 1) return MOE_ERR_ARG;
+  if (E > 1024 || k > E || k > 32) return MOE_ERR_SHAPE;
+  if ((int64_t)T * E >= kMaxElems || (int64_t)T * k >= kMaxElems) return MOE_ERR_SHAPE;
+  return MOE_OK;
+}
+
+int check_ranks(int T, int k, int E, int R, bool need_even_rows) {
+  if (R < 1) return MOE_ERR_ARG;
+  if (R > E || E % R != 0) return MOE_ERR_SHAPE;
+  if (need_even_rows && ((int64_t)T * k) % R != 0) return MOE_ERR_SHAPE;
+  return MOE_OK;
+}
+
+int check_dims(int T, int k, int d, int F) {
+  if (d < 1 || F < 1) return MOE_ERR_ARG;
+  if (d % 128 != 0 || F % 128 != 0) return MOE_ERR_SHAPE;
+  const int64_t rows = (int64_t)T * k;
+  if (rows * d >= kMaxElems || rows * F >= kMaxElems || (int64_t)T * d >= kMaxElems)
+    return MOE_ERR_SHAPE;
+  return MOE_OK;
+}
+
+int check_groups(int E, int R, int S) {
+  if (S < 0) return MOE_ERR_ARG;
+  if ((int64_t)R * (E / R + S) > 4096) return MOE_ERR_SHAPE;
+  return MOE_OK;
+}
+
+cudaStream_t as_stream(moe_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+#define MOE_TRY(expr)          \
+  do {                         \
+    const int st_ = (expr);    \
+    if (st_ != MOE_OK) return st_; \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+int moe_plan_get_layout(int E, int R, int S, moe_plan_layout* out) {
+  if (!out || E < 1 || R < 1 || S < 0) return MOE_ERR_ARG;
+  if (E % R != 0) return MOE_ERR_SHAPE;
+  const int64_t B = E / R;
+  moe_plan_layout L;
+  L.kept_rows = 0;
+  L.room_prefix = L.kept_rows + R;
+  L.expert_home_off = L.room_prefix + R + 1;
+  L.stream_off = L.expert_home_off + E;
+  L.replica_expert = L.stream_off + E + 1;
+  L.replica_list = L.replica_expert + (int64_t)R * S;
+  L.n_groups = L.replica_list + 1 + (int64_t)R * S;
+  L.groups = ((L.n_groups + R) + 3) / 4 * 4;  // 16-byte aligned group records
+  L.words = L.groups + (int64_t)R * (B + S) * 4;
+  L.max_groups_per_rank = (int32_t)(B + S);
+  *out = L;
+  return MOE_OK;
+}
+
+int64_t moe_dispatch_workspace_words(int T, int E) {
+  if (T < 0 || E < 1) return 0;
+  return ((int64_t)T + moe::kPlaceTile - 1) / moe::kPlaceTile * E;
+}
+
+const char* moe_status_string(int status) {
+  switch (status) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_ARG: return "null pointer, misaligned pointer or negative size";
+    case MOE_ERR_SHAPE: return "size limit violated";
+    case MOE_ERR_LAUNCH: return "CUDA launch failed";
+    case MOE_ERR_DEVICE: return "no usable sm_100 device or driver entry point";
+    default: return "unknown status";
+  }
+}
+
+int moe_topk(const float* logits, int T, int E, int k, int32_t* idx, float* gate,
+             int32_t* err, moe_stream_t stream) {
+  if (!err || (T > 0 && (!logits || !idx || !gate))) return MOE_ERR_ARG;
+  MOE_TRY(check_route(T, E, k));
+  return moe::launch_topk(logits, T, E, k, idx, gate, err, as_stream(stream));
+}
+
+int moe_histogram_maxvio(const int32_t* idx, int T, int k, int E, int R,
+                         const int32_t* expert_to_rank, int32_t* counts, int32_t* loads,
+                         double* maxvio, double* balancedness, int32_t* err,
+                         moe_stream_t stream) {
+  if (!counts || !loads || !maxvio || !balancedness || !err || (T > 0 && !idx)) return MOE_ERR_ARG;
+  MOE_TRY(check_route(T, E, k));
+  MOE_TRY(check_ranks(T, k, E, R, false));
+  return moe::launch_histogram(idx, T, k, E, R, expert_to_rank, counts, loads, maxvio,
+                               balancedness, err, as_stream(stream));
+}
+
+int moe_plan_balanced(const int32_t* counts, int T, int k, int E, int R, int S, int32_t* plan,
+                      int32_t* err, moe_stream_t stream) {
+  if (!counts || !plan || !err) return MOE_ERR_ARG;
+  MOE_TRY(check_route(T, E, k));
+  MOE_TRY(check_ranks(T, k, E, R, true));
+  MOE_TRY(check_groups(E, R, S));
+  moe_plan_layout L;
+  MOE_TRY(moe_plan_get_layout(E, R, S, &L));
+  return moe::launch_plan(counts, T, k, E, R, S, plan, L, err, as_stream(stream));
+}
+
+int moe_prefetch_replicas(const int32_t* plan, const moe_bf16* W1, const moe_bf16* W3,
+                          const moe_f16* W2, int E, int R, int S, int d, int F,
+                          moe_bf16* P1, moe_bf16* P3, moe_f16* P2, const int32_t* err,
+                          moe_stream_t stream) {
+  if (!plan || !W1 || !W3 || !W2 || !err) return MOE_ERR_ARG;
+  if (S > 0 && (!P1 || !P3 || !P2)) return MOE_ERR_ARG;
+  if (E < 1 || R < 1) return MOE_ERR_ARG;
+  MOE_TRY(check_ranks(0, 1, E, R, false));
+  MOE_TRY(check_groups(E, R, S));
+  MOE_TRY(check_dims(0, 1, d, F));
+  if ((int64_t)E * d * F >= ((int64_t)1 << 40)) return MOE_ERR_SHAPE;
+  if (!aligned16(W1) || !aligned16(W3) || !aligned16(W2) ||
+      (S > 0 && (!aligned16(P1) || !aligned16(P3) || !aligned16(P2))))
+    return MOE_ERR_ARG;
+  moe_plan_layout L;
+  MOE_TRY(moe_plan_get_layout(E, R, S, &L));
+  return moe::launch_prefetch(plan, L, reinterpret_cast<const __nv_bfloat16*>(W1),
+                              reinterpret_cast<const __nv_bfloat16*>(W3),
+                              reinterpret_cast<const __half*>(W2), E, R, S, d, F,
+                              reinterpret_cast<__nv_bfloat16*>(P1),
+                              reinterpret_cast<__nv_bfloat16*>(P3),
+                              reinterpret_cast<__half*>(P2), err, as_stream(stream));
+}
+
+int moe_dispatch(const moe_bf16* x, const int32_t* idx, const int32_t* plan, int T, int k,
+                 int E, int R, int S, int d, int32_t* workspace, moe_bf16* recv,
+                 int32_t* perm, int32_t* src, int32_t* err, moe_stream_t stream) {
+  if (!plan || !err) return MOE_ERR_ARG;
+  if (T > 0 && (!x || !idx || !workspace || !recv || !perm || !src)) return MOE_ERR_ARG;
+  MOE_TRY(check_route(T, E, k));
+  MOE_TRY(check_ranks(T, k, E, R, true));
+  MOE_TRY(check_groups(E, R, S));
+  MOE_TRY(check_dims(T, k, d, 128));
+  if (!aligned16(x) || !aligned16(recv)) return MOE_ERR_ARG;
+  moe_plan_layout L;
+  MOE_TRY(moe_plan_get_layout(E, R, S, &L));
+  return moe::launch_dispatch(reinterpret_cast<const __nv_bfloat16*>(x), idx, plan, L, T, k, E,
+                              R, d, workspace, reinterpret_cast<__nv_bfloat16*>(recv), perm,
+                              src, err, as_stream(stream));
+}
+
+int moe_grouped_ffn(const moe_bf16* recv, const int32_t* plan, const moe_bf16* W1,
+                    const moe_bf16* W3, const moe_f16* W2, const moe_bf16* P1,
+                    const moe_bf16* P3, const moe_f16* P2, int T, int k, int E, int R,
+                    int S, int d, int F, moe_f16* h, moe_bf16* y, int32_t* err,
+                    moe_stream_t stream) {
+  if (!plan || !W1 || !W3 || !W2 || !err) return MOE_ERR_ARG;
+  if (T > 0 && (!recv || !h || !y)) return MOE_ERR_ARG;
+  if (S > 0 && (!P1 || !P3 || !P2)) return MOE_ERR_ARG;
+  MOE_TRY(check_route(T, E, k));
+  MOE_TRY(check_ranks(T, k, E, R, true));
+  MOE_TRY(check_groups(E, R, S));
+  MOE_TRY(check_dims(T, k, d, F));
+  if ((int64_t)E * F >= kMaxElems || (int64_t)E * d >= kMaxElems ||
+      (int64_t)R * S * F >= kMaxElems || (int64_t)R * S * d >= kMaxElems)
+    return MOE_ERR_SHAPE;
+  if (!aligned16(recv) || !aligned16(h) || !aligned16(y) || !aligned16(W1) || !aligned16(W3) ||
+      !aligned16(W2) || (S > 0 && (!aligned16(P1) || !aligned16(P3) || !aligned16(P2))))
+    return MOE_ERR_ARG;
+  moe_plan_layout L;
+  MOE_TRY(moe_plan_get_layout(E, R, S, &L));
+  return moe::launch_grouped_ffn(
+      reinterpret_cast<const __nv_bfloat16*>(recv), plan, L,
+      reinterpret_cast<const __nv_bfloat16*>(W1), reinterpret_cast<const __nv_bfloat16*>(W3),
+      reinterpret_cast<const __half*>(W2), reinterpret_cast<const __nv_bfloat16*>(P1),
+      reinterpret_cast<const __nv_bfloat16*>(P3), reinterpret_cast<const __half*>(P2), T, k, E,
+      R, S, d, F, reinterpret_cast<__half*>(h), reinterpret_cast<__nv_bfloat16*>(y), err,
+      as_stream(stream));
+}
+
+int moe_combine(const moe_bf16* y, const int32_t* perm, const float* gate, int T, int k, int d,
+                moe_bf16* out, const int32_t* err, moe_stream_t stream) {
+  if (!err) return MOE_ERR_ARG;
+  if (T > 0 && (!y || !perm || !gate || !out)) return MOE_ERR_ARG;
+  if (T < 0 || k < 1) return MOE_ERR_ARG;
+  if (k > 32) return MOE_ERR_SHAPE;
+  MOE_TRY(check_dims(T, k, d, 128));
+  if (!aligned16(y) || !aligned16(out)) return MOE_ERR_ARG;
+  return moe::launch_combine(reinterpret_cast<const __nv_bfloat16*>(y), perm, gate, T, k, d,
+                             reinterpret_cast<__nv_bfloat16*>(out), err, as_stream(stream));
+}
+
+}  // extern "C"

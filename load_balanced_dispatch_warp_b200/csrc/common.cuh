@@ -1,0 +1,119 @@
+// Shared device/host helpers of the MoE-layer library (sm_100a only).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+#define MOE_FULL_MASK 0xffffffffu
+
+namespace moe {
+
+// ----------------------------------------------------------------------------- host side
+// Launch helpers return a host status; every launcher below is called from abi.cu after
+// the argument checks, so it only enqueues.
+inline int launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_LAUNCH;
+}
+
+int num_sms();  // SM count of the current device (cached per device)
+
+// --------------------------------------------------------------- launchers (one per step)
+int launch_topk(const float* logits, int T, int E, int k, int32_t* idx, float* gate,
+                int32_t* err, cudaStream_t s);
+int launch_histogram(const int32_t* idx, int T, int k, int E, int R, const int32_t* map,
+                     int32_t* counts, int32_t* loads, double* maxvio, double* bal,
+                     int32_t* err, cudaStream_t s);
+int launch_plan(const int32_t* counts, int T, int k, int E, int R, int S, int32_t* plan,
+                const moe_plan_layout& L, int32_t* err, cudaStream_t s);
+int launch_prefetch(const int32_t* plan, const moe_plan_layout& L, const __nv_bfloat16* W1,
+                    const __nv_bfloat16* W3, const __half* W2, int E, int R, int S, int d,
+                    int F, __nv_bfloat16* P1, __nv_bfloat16* P3, __half* P2,
+                    const int32_t* err, cudaStream_t s);
+int launch_dispatch(const __nv_bfloat16* x, const int32_t* idx, const int32_t* plan,
+                    const moe_plan_layout& L, int T, int k, int E, int R, int d,
+                    int32_t* ws, __nv_bfloat16* recv, int32_t* perm, int32_t* src,
+                    int32_t* err, cudaStream_t s);
+int launch_grouped_ffn(const __nv_bfloat16* recv, const int32_t* plan,
+                       const moe_plan_layout& L, const __nv_bfloat16* W1,
+                       const __nv_bfloat16* W3, const __half* W2, const __nv_bfloat16* P1,
+                       const __nv_bfloat16* P3, const __half* P2, int T, int k, int E, int R,
+                       int S, int d, int F, __half* h, __nv_bfloat16* y, int32_t* err,
+                       cudaStream_t s);
+int launch_combine(const __nv_bfloat16* y, const int32_t* perm, const float* gate, int T,
+                   int k, int d, __nv_bfloat16* out, const int32_t* err, cudaStream_t s);
+
+// Tokens per tile of the placement kernels (workspace = ceil(T/kPlaceTile) * E words).
+constexpr int kPlaceTile = 256;
+
+// ----------------------------------------------------------------------------- device side
+// Reads the layer's error word once per thread; every kernel after moe_topk returns
+// early when it is non-zero.
+__device__ __forceinline__ int load_err(const int32_t* err) {
+  return *reinterpret_cast<const volatile int32_t*>(err);
+}
+
+// Block-uniform version for kernels with barriers: thread 0 reads the word and the whole
+// block takes the same decision.  Call at most once per kernel, before any other barrier.
+__device__ __forceinline__ bool block_should_stop(const int32_t* err) {
+  __shared__ int s_stop;
+  if (threadIdx.x == 0) s_stop = load_err(err);
+  __syncthreads();
+  return s_stop != 0;
+}
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Warp-wide sum of a float (butterfly).
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(MOE_FULL_MASK, v, o);
+  return v;
+}
+
+// Exclusive prefix sum of n <= 32*blockDim.x ints held in shared memory, in place, by
+// the whole block; returns the total.  Chunked over blockDim.x with a running carry.
+// `scratch` needs 33 ints of shared memory.  Every thread of the block must call it.
+__device__ __forceinline__ int block_exclusive_scan(int* data, int n, int* scratch) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nwarps = (blockDim.x + 31) >> 5;
+  int carry = 0;
+  for (int base = 0; base < n; base += blockDim.x) {
+    const int i = base + tid;
+    const int v = i < n ? data[i] : 0;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int t = __shfl_up_sync(MOE_FULL_MASK, incl, o);
+      if (lane >= o) incl += t;
+    }
+    if (lane == 31) scratch[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      int w = lane < nwarps ? scratch[lane] : 0;
+      int wi = w;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        int t = __shfl_up_sync(MOE_FULL_MASK, wi, o);
+        if (lane >= o) wi += t;
+      }
+      if (lane < nwarps) scratch[lane] = wi - w;  // exclusive warp offsets
+      if (lane == 31) scratch[32] = wi;           // chunk total
+    }
+    __syncthreads();
+    if (i < n) data[i] = carry + scratch[warp] + incl - v;
+    carry += scratch[32];
+    __syncthreads();
+  }
+  return carry;
+}
+
+}  // namespace moe

@@ -1,0 +1,543 @@
+// Grouped SwiGLU expert FFN on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// "DeepEP-on-EFA Guidance, section 1: What is MoE", phase (c): each rank runs its local
+// experts over the rows it received as a batched grouped GEMM.  Here the ranks' rows are
+// one buffer [R*C, d] and the plan's group table names, for each contiguous run of rows,
+// the expert (home tensor) or the pool slot (replica) whose weights it uses.
+//
+//   GEMM 1:  h = silu(X W1^T) * (X W3^T)   per group; one MMA of N = 2*128 covers a
+//            128-column block of W1 and the same block of W3, so the SwiGLU epilogue
+//            reads gate and up values of the same row from one TMEM accumulator.
+//   GEMM 2:  y = h W2^T                    per group; N = 256 (128 when d % 256 != 0).
+//            h and W2 are fp16: rounding h to bf16 (8-bit significand) would put the
+//            worst element of y near the 1e-2 parity bound at F/d >= 2, fp16's 11 bits
+//            keep it below half of it at the same tensor-core rate.
+//
+// Kernel shape (one CTA per SM, persistent, 192 threads):
+//   warp 0      TMA producer: A (128 rows x 64 K) and B (N rows x 64 K) tiles, 128-byte
+//               swizzle, into a 4-stage ring; mbarrier transaction counts signal arrival.
+//   warp 1      TMEM owner (alloc/dealloc of 512 columns) and single-thread MMA issuer:
+//               tcgen05.mma.cta_group::1.kind::f16, bf16 x bf16 -> fp32 in TMEM, two
+//               accumulator buffers of 256 columns so the epilogue of one tile overlaps
+//               the main loop of the next.
+//   warps 2-5   epilogue: tcgen05.ld 32 lanes x 32 columns at a time, SwiGLU or plain
+//               conversion to bf16, masked row stores (a tile's rows past the end of its
+//               group belong to the next group and are not written).
+// Tiles are (group, 128-row block, N block), enumerated m-block-major from a prefix over
+// the group table built in shared memory by every CTA; CTA i takes tiles i, i+grid, ...
+//
+// Every mbarrier wait is bounded (about 2 s of %globaltimer); a wait that runs out sets
+// MOE_DERR_TIMEOUT and a shared abort flag, every role leaves its loop, the producer
+// waits (bounded) for its copies in flight, the MMA thread for its MMAs, and TMEM is
+// freed before the CTA exits.
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128;          // rows per tile (TMEM lanes)
+constexpr int BK = 64;           // K per stage: 64 bf16 = one 128-byte swizzle row
+constexpr int UMMA_K = 16;       // K per tcgen05.mma for 16-bit inputs
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;        // 16 KiB
+constexpr int B_BYTES_MAX = 256 * BK * 2;   // 32 KiB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES_MAX;
+constexpr int ACC_COLS = 256;               // one accumulator buffer
+constexpr int TMEM_COLS = 2 * ACC_COLS;
+constexpr int MAX_GROUPS = 4096;
+constexpr int FFN_THREADS = 192;
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
+
+struct FfnArgs {
+  const int4* groups;   // [G] {row_start, rows, expert, weight_ref}, rows == -1 unused
+  int G;
+  int n_blocks_n;       // output column blocks per row block
+  int k_blocks;         // K / BK
+  int bn_out;           // output columns per tile (128 for SwiGLU, N for plain)
+  int mma_n;            // N of the MMA (256 for SwiGLU, bn_out for plain)
+  int rows_per_expert;  // rows of one expert in the B tensors: F (GEMM 1) or d (GEMM 2)
+  int E;
+  int out_ld;           // columns of the output tensor
+  void* out;            // h (fp16) for GEMM 1, y (bf16) for GEMM 2
+  int32_t* err;
+};
+
+// --------------------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase of `parity` to complete.  Returns false (and raises the
+// abort flag and the error bit) if the bound runs out, or if another role aborted.
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                       int32_t* err) {
+  if (mbar_try(bar, parity)) return true;
+  uint64_t t0 = 0;
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try(bar, parity)) return true;
+    if ((it & 255u) == 0) {
+      if (*abort_flag) return false;
+      const uint64_t now = globaltimer();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > WAIT_LIMIT_NS) {
+        *abort_flag = 1;
+        atomicOr(err, MOE_DERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// 32 TMEM lanes x 32 consecutive 32-bit columns: thread i of the warp gets lane base+i.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major tile written by TMA with the 128-byte
+// swizzle: rows of 128 bytes, 8-row atoms 1024 bytes apart (stride byte offset), leading
+// byte offset unused for swizzled K-major (encoded 1), descriptor version 1 (bits 46-47),
+// layout type 2 = 128-byte swizzle (bits 61-63).  Stepping K by 16 elements inside the
+// 128-byte row adds 32 bytes to the start address.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) |
+         ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Instruction descriptor, kind::f16: fp32 accumulate (bits 4-5 = 1), A and B of one type,
+// bf16 (1) or fp16 (0), at bits 7-9 and 10-12, both K-major (bits 15, 16 = 0), N >> 3 at
+// bits 17-22, M >> 4 at bits 24-28.
+__host__ __device__ constexpr uint32_t make_idesc(int M, int N, bool bf16) {
+  return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+// fp16 pair with saturation to +-65504 (no infinities from large activations)
+__device__ __forceinline__ uint32_t pack_f16_sat(float a, float b) {
+  a = fminf(fmaxf(a, -65504.0f), 65504.0f);
+  b = fminf(fmaxf(b, -65504.0f), 65504.0f);
+  __half2 v = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float silu(float z) { return z / (1.0f + __expf(-z)); }
+
+struct Tile {
+  int a_row;       // first row of the A block
+  int valid_rows;  // rows of the block inside the group (<= BM)
+  int b_row;       // first row of the B block inside its tensor
+  bool pool;       // B from the replica pool instead of the home tensors
+  int n_block;
+};
+
+__device__ __forceinline__ Tile decode_tile(int t, const FfnArgs& a, const int* s_prefix) {
+  const int mt = t / a.n_blocks_n;
+  Tile tl;
+  tl.n_block = t - mt * a.n_blocks_n;
+  // last group whose prefix <= mt (empty groups share their successor's prefix)
+  int lo = 0, hi = a.G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_prefix[mid] <= mt) lo = mid; else hi = mid - 1;
+  }
+  const int4 g = __ldg(a.groups + lo);
+  const int m_local = mt - s_prefix[lo];
+  tl.a_row = g.x + m_local * BM;
+  tl.valid_rows = min(BM, g.y - m_local * BM);
+  const int ref = g.w;
+  tl.pool = ref >= a.E;
+  tl.b_row = (tl.pool ? ref - a.E : ref) * a.rows_per_expert + tl.n_block * a.bn_out;
+  return tl;
+}
+
+template <bool SWIGLU>
+__global__ void __launch_bounds__(FFN_THREADS, 1)
+    ffn_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b0,
+               const __grid_constant__ CUtensorMap tm_b1, const __grid_constant__ CUtensorMap tm_p0,
+               const __grid_constant__ CUtensorMap tm_p1, const FfnArgs args) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte alignment for the swizzle atoms
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* stage_base = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
+  int* s_misc = reinterpret_cast<int*>(bars + 2 * STAGES + 5);  // [0] tmem base, [1] abort, [2] err0
+  int* s_prefix = s_misc + 4;                                     // [G + 1]
+  int* s_scan = s_prefix + MAX_GROUPS + 1;                        // 33 ints
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  volatile int* abort_flag = s_misc + 1;
+
+  if (tid == 0) {
+    s_misc[2] = load_err(args.err);
+    s_misc[1] = 0;
+  }
+  __syncthreads();
+  if (s_misc[2] != 0) return;
+
+  // m-blocks per group, exclusive prefix over the group table
+  for (int g = tid; g < args.G; g += blockDim.x) {
+    const int rows = __ldg(&args.groups[g].y);
+    s_prefix[g] = rows > 0 ? (rows + BM - 1) / BM : 0;
+  }
+  __syncthreads();
+  const int total_m = block_exclusive_scan(s_prefix, args.G, s_scan);
+  if (tid == 0) s_prefix[args.G] = total_m;
+  const int total_tiles = total_m * args.n_blocks_n;
+
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = smem_u32(bars + STAGES);
+  const uint32_t tfull0 = smem_u32(bars + 2 * STAGES);
+  const uint32_t tempty0 = smem_u32(bars + 2 * STAGES + 2);
+  const uint32_t drain = smem_u32(bars + 2 * STAGES + 4);
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull0 + 8 * b, 1);
+      mbar_init(tempty0 + 8 * b, 4);
+    }
+    mbar_init(drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(s_misc)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = static_cast<uint32_t>(s_misc[0]);
+  const uint32_t b_bytes = (uint32_t)args.mma_n * BK * 2;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_phase = 0;  // per stage: issued at least once, parity
+      for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+        const Tile tl = decode_tile(t, args, s_prefix);
+        const CUtensorMap* mb0 = tl.pool ? &tm_p0 : &tm_b0;
+        const CUtensorMap* mb1 = tl.pool ? &tm_p1 : &tm_b1;
+        bool ok = true;
+        for (int kb = 0; kb < args.k_blocks; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, args.err)) { ok = false; break; }
+          const uint32_t fb = full0 + 8 * stage;
+          const uint32_t sa = smem_u32(stage_base + stage * STAGE_BYTES);
+          const uint32_t sb = sa + A_BYTES;
+          mbar_expect_tx(fb, A_BYTES + b_bytes);
+          tma_load_2d(sa, &tm_a, fb, kb * BK, tl.a_row);
+          if (SWIGLU) {
+            tma_load_2d(sb, mb0, fb, kb * BK, tl.b_row);
+            tma_load_2d(sb + (b_bytes >> 1), mb1, fb, kb * BK, tl.b_row);
+          } else {
+            tma_load_2d(sb, mb0, fb, kb * BK, tl.b_row);
+          }
+          issued_mask |= 1u << stage;
+          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+      }
+      // make sure no copy is still landing in shared memory when the CTA leaves
+      for (int s = 0; s < STAGES; ++s)
+        if (issued_mask & (1u << s)) {
+          volatile int no_abort = 0;
+          mbar_wait(full0 + 8 * s, (issued_phase >> s) & 1u, &no_abort, args.err);
+        }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      // GEMM 1: x, W1, W3 in bf16; GEMM 2: h and W2 in fp16
+      const uint32_t idesc = make_idesc(BM, args.mma_n, SWIGLU);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+        if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag, args.err)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+        bool ok = true;
+        for (int kb = 0; kb < args.k_blocks; ++kb) {
+          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, args.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(stage_base + stage * STAGE_BYTES);
+          const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / UMMA_K; ++kk)
+            tc_mma(d_tmem, sw128_desc(sa + kk * UMMA_K * 2), sw128_desc(sb + kk * UMMA_K * 2), idesc,
+                   (kb | kk) != 0);
+          tc_commit(empty0 + 8 * stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(tfull0 + 8 * acc);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      // all MMAs issued by this thread have completed once `drain` flips
+      tc_commit(drain);
+      volatile int no_abort = 0;
+      mbar_wait(drain, 0, &no_abort, args.err);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------- epilogue (warps 2-5)
+    const int quarter = warp & 3;  // TMEM lanes this warp may access
+    const int r_in = quarter * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+      const Tile tl = decode_tile(t, args, s_prefix);
+      const bool ok = mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, args.err);
+      if (!__all_sync(MOE_FULL_MASK, ok)) break;  // warp-uniform exit
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * ACC_COLS;
+      const bool valid = r_in < tl.valid_rows;
+      // both outputs are 16-bit: h (fp16) after GEMM 1, y (bf16) after GEMM 2
+      uint16_t* orow = static_cast<uint16_t*>(args.out) + (int64_t)(tl.a_row + r_in) * args.out_ld +
+                       (int64_t)tl.n_block * args.bn_out;
+      if (SWIGLU) {
+#pragma unroll 1
+        for (int c = 0; c < 128 / 32; ++c) {
+          uint32_t g[32], u[32];
+          tmem_ld32(tbase + c * 32, g);
+          tmem_ld32(tbase + 128 + c * 32, u);
+          tmem_wait_ld();
+          uint32_t p[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+            const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+            p[i] = pack_f16_sat(silu(g0) * u0, silu(g1) * u1);
+          }
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < args.bn_out / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tbase + c * 32, v);
+          tmem_wait_ld();
+          uint32_t p[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) p[i] = pack_bf16(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ----------------------------------------------------------------------------- host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D 16-bit tensor [rows, cols] row-major, box = 64 columns x box_rows rows, 128-byte
+// swizzle.
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows,
+              CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rows <= 0) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, type, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t ffn_smem_bytes() {
+  return 1024 + (size_t)STAGES * STAGE_BYTES + (2 * STAGES + 5) * 8 + 4 * 4 +
+         (MAX_GROUPS + 1) * 4 + 33 * 4;
+}
+
+template <bool SWIGLU>
+int launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+               const CUtensorMap& p0, const CUtensorMap& p1, const FfnArgs& args, cudaStream_t s) {
+  static bool configured[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const size_t smem = ffn_smem_bytes();
+  if (dev < 64 && !configured[dev]) {
+    if (cudaFuncSetAttribute(ffn_kernel<SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return MOE_ERR_LAUNCH;
+    configured[dev] = true;
+  }
+  ffn_kernel<SWIGLU><<<num_sms(), FFN_THREADS, smem, s>>>(a, b0, b1, p0, p1, args);
+  return launch_status();
+}
+
+}  // namespace
+
+int launch_grouped_ffn(const __nv_bfloat16* recv, const int32_t* plan,
+                       const moe_plan_layout& L, const __nv_bfloat16* W1,
+                       const __nv_bfloat16* W3, const __half* W2, const __nv_bfloat16* P1,
+                       const __nv_bfloat16* P3, const __half* P2, int T, int k, int E, int R,
+                       int S, int d, int F, __half* h, __nv_bfloat16* y, int32_t* err,
+                       cudaStream_t s) {
+  if (T == 0) return MOE_OK;
+  const int64_t rows = (int64_t)T * k;  // R * C
+  const int bn2 = (d % 256 == 0) ? 256 : 128;
+  CUtensorMap m_recv, m_w1, m_w3, m_p1, m_p3, m_h, m_w2, m_p2;
+  if (!make_map(&m_recv, recv, rows, d, BM) || !make_map(&m_w1, W1, (int64_t)E * F, d, 128) ||
+      !make_map(&m_w3, W3, (int64_t)E * F, d, 128) ||
+      !make_map(&m_h, h, rows, F, BM, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+      !make_map(&m_w2, W2, (int64_t)E * d, F, bn2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+    return MOE_ERR_DEVICE;
+  if (S > 0) {
+    if (!make_map(&m_p1, P1, (int64_t)R * S * F, d, 128) ||
+        !make_map(&m_p3, P3, (int64_t)R * S * F, d, 128) ||
+        !make_map(&m_p2, P2, (int64_t)R * S * d, F, bn2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+      return MOE_ERR_DEVICE;
+  } else {  // no pool: replica references cannot occur; pass the home maps
+    m_p1 = m_w1;
+    m_p3 = m_w3;
+    m_p2 = m_w2;
+  }
+  FfnArgs a1;
+  a1.groups = reinterpret_cast<const int4*>(plan + L.groups);
+  a1.G = R * L.max_groups_per_rank;
+  a1.n_blocks_n = F / 128;
+  a1.k_blocks = d / BK;
+  a1.bn_out = 128;
+  a1.mma_n = 256;
+  a1.rows_per_expert = F;
+  a1.E = E;
+  a1.out_ld = F;
+  a1.out = h;
+  a1.err = err;
+  int st = launch_one<true>(m_recv, m_w1, m_w3, m_p1, m_p3, a1, s);
+  if (st != MOE_OK) return st;
+  FfnArgs a2 = a1;
+  a2.n_blocks_n = d / bn2;
+  a2.k_blocks = F / BK;
+  a2.bn_out = bn2;
+  a2.mma_n = bn2;
+  a2.rows_per_expert = d;
+  a2.out_ld = d;
+  a2.out = y;
+  return launch_one<false>(m_h, m_w2, m_w2, m_p2, m_p2, a2, s);
+}
+
+}  // namespace moe

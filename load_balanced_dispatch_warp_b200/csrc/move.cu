@@ -1,0 +1,316 @@
+// Row movement of the layer: replica prefetch, zero-copy placement + dispatch, combine.
+//
+// Dispatch and combine are the two all-to-all phases of "DeepEP-on-EFA Guidance, section
+// 1: What is MoE" (dispatch sends each token to its k experts only; combine is its
+// transpose with the gate-weighted sum); with ranks simulated as partitions of one GPU's
+// HBM they are gathers/scatters of whole rows.  Prefetch and zero-copy placement follow
+// the MoonEP news article, paragraph 3.  All of it is HBM-bound: 16-byte vector loads and
+// stores, each token row read once.
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+// ----------------------------------------------------------------------------- prefetch
+constexpr int kCopyThreads = 256;
+constexpr int kCopyVec = 4;  // 16-byte vectors per thread per chunk
+constexpr int kCopyChunk = kCopyThreads * kCopyVec;  // vectors per chunk (16 KiB)
+
+// Grid-stride over (filled slot, projection, chunk).  The plan's compact slot list makes
+// the work proportional to the replicas actually planned.
+__global__ void __launch_bounds__(kCopyThreads) prefetch_kernel(
+    const int32_t* __restrict__ rep, const int32_t* __restrict__ rep_list,
+    const uint4* __restrict__ W1, const uint4* __restrict__ W3, const uint4* __restrict__ W2,
+    uint4* __restrict__ P1, uint4* __restrict__ P3, uint4* __restrict__ P2, int64_t vecs,
+    const int32_t* __restrict__ err) {
+  if (load_err(err)) return;
+  const int n = rep_list[0];
+  const int64_t chunks = (vecs + kCopyChunk - 1) / kCopyChunk;
+  const int64_t total = (int64_t)n * 3 * chunks;
+  for (int64_t w = blockIdx.x; w < total; w += gridDim.x) {
+    const int64_t si = w / (3 * chunks);
+    const int64_t rem = w - si * 3 * chunks;
+    const int proj = (int)(rem / chunks);
+    const int64_t c = rem - (int64_t)proj * chunks;
+    const int slot = rep_list[1 + si];
+    const int e = rep[slot];
+    const uint4* src = (proj == 0 ? W1 : proj == 1 ? W3 : W2) + (int64_t)e * vecs;
+    uint4* dst = (proj == 0 ? P1 : proj == 1 ? P3 : P2) + (int64_t)slot * vecs;
+    const int64_t v0 = c * kCopyChunk + threadIdx.x;
+    uint4 buf[kCopyVec];
+#pragma unroll
+    for (int i = 0; i < kCopyVec; ++i) {
+      const int64_t v = v0 + i * kCopyThreads;
+      if (v < vecs) buf[i] = __ldcs(src + v);
+    }
+#pragma unroll
+    for (int i = 0; i < kCopyVec; ++i) {
+      const int64_t v = v0 + i * kCopyThreads;
+      if (v < vecs) dst[v] = buf[i];
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------- placement
+// Pass 1: per-tile expert counts ws[tile*E + e] (every entry written).
+__global__ void __launch_bounds__(kPlaceTile) tile_count_kernel(const int32_t* __restrict__ idx,
+                                                                int T, int k, int E,
+                                                                int32_t* __restrict__ ws,
+                                                                int32_t* __restrict__ err) {
+  extern __shared__ int s_cnt[];
+  __shared__ int s_bad;
+  if (block_should_stop(err)) return;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_cnt[e] = 0;
+  if (threadIdx.x == 0) s_bad = 0;
+  __syncthreads();
+  const int64_t t = (int64_t)blockIdx.x * kPlaceTile + threadIdx.x;
+  const int lane = threadIdx.x & 31;
+  for (int j = 0; j < k; ++j) {
+    int e = t < T ? __ldg(idx + t * k + j) : -1;
+    if (t < T && (e < 0 || e >= E)) {
+      s_bad = 1;
+      e = -1;
+    }
+    const uint32_t peers = __match_any_sync(MOE_FULL_MASK, e);
+    if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&s_cnt[e], __popc(peers));
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) ws[(int64_t)blockIdx.x * E + e] = s_cnt[e];
+  if (threadIdx.x == 0 && s_bad) atomicOr(err, MOE_DERR_ID_RANGE);
+}
+
+// Pass 2: the token-order rank q of every assignment within its expert, then its row.
+//   q = (assignments of e in earlier tiles) + (in earlier warps of this tile)
+//     + (in earlier lanes of this warp);
+// the last term comes from a per-warp lane mask of each expert (a token names an expert
+// at most once, so one bit per lane suffices).
+__global__ void __launch_bounds__(kPlaceTile) tile_rank_kernel(
+    const int32_t* __restrict__ idx, int T, int k, int E, int R, int C,
+    const int32_t* __restrict__ ws, const int32_t* __restrict__ plan, moe_plan_layout L,
+    int32_t* __restrict__ perm, int32_t* __restrict__ src, int32_t* __restrict__ err) {
+  constexpr int W = kPlaceTile / 32;
+  extern __shared__ int smem[];
+  uint32_t* s_mask = reinterpret_cast<uint32_t*>(smem);  // [W][E]
+  int* s_pre = smem + W * E;                              // [W][E] start of each warp
+  int* s_rp = s_pre + W * E;                              // [R+1] room prefix
+  int* s_kr = s_rp + R + 1;                               // [R] kept rows
+  __shared__ int s_bad;
+  if (block_should_stop(err)) return;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tile = blockIdx.x;
+  for (int i = tid; i < W * E; i += blockDim.x) s_mask[i] = 0;
+  for (int r = tid; r <= R; r += blockDim.x) s_rp[r] = plan[L.room_prefix + r];
+  for (int r = tid; r < R; r += blockDim.x) s_kr[r] = plan[L.kept_rows + r];
+  if (tid == 0) s_bad = 0;
+  __syncthreads();
+  const int64_t t = (int64_t)tile * kPlaceTile + tid;
+  const bool tok = t < T;
+  for (int j = 0; j < k; ++j) {
+    if (!tok) break;
+    const int e = __ldg(idx + t * k + j);
+    if (e >= 0 && e < E) atomicOr(&s_mask[warp * E + e], 1u << lane);
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) {
+    int run = 0;
+    for (int p = 0; p < tile; ++p) run += __ldg(ws + (int64_t)p * E + e);
+    for (int w = 0; w < W; ++w) {
+      s_pre[w * E + e] = run;
+      run += __popc(s_mask[w * E + e]);
+    }
+  }
+  __syncthreads();
+  if (tok) {
+    const uint32_t lt = lanemask_lt();
+    const int64_t rows_total = (int64_t)R * C;
+    const int B = E / R;
+    for (int j = 0; j < k; ++j) {
+      const int e = __ldg(idx + t * k + j);
+      if (e < 0 || e >= E) { s_bad = 1; continue; }
+      const int q = s_pre[warp * E + e] + __popc(s_mask[warp * E + e] & lt);
+      const int off = __ldg(plan + L.expert_home_off + e);
+      int64_t row;
+      if (off >= 0) {
+        row = (int64_t)(e / B) * C + off + q;
+      } else {
+        const int p = __ldg(plan + L.stream_off + e) + q;
+        int a = 0, b = R - 1;  // last rank with room_prefix <= p
+        while (a < b) {
+          const int m = (a + b + 1) >> 1;
+          if (s_rp[m] <= p) a = m; else b = m - 1;
+        }
+        row = (int64_t)a * C + s_kr[a] + (p - s_rp[a]);
+      }
+      if (row < 0 || row >= rows_total) { s_bad = 1; continue; }
+      perm[t * k + j] = (int32_t)row;
+      src[row] = (int32_t)t;
+    }
+  }
+  __syncthreads();
+  if (tid == 0 && s_bad) atomicOr(err, MOE_DERR_ID_RANGE);
+}
+
+// Pass 3: every token row is read once (16-byte vectors) and stored to its k rows.
+constexpr int kRowThreads = 256;
+constexpr int kRowVec = 4;
+
+__global__ void __launch_bounds__(kRowThreads) scatter_rows_kernel(
+    const uint4* __restrict__ x, const int32_t* __restrict__ perm, int T, int k, int dv,
+    int64_t rows_total, uint4* __restrict__ recv, const int32_t* __restrict__ err) {
+  if (load_err(err)) return;
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += nwarps) {
+    int r = lane < k ? __ldg(perm + t * k + lane) : 0;
+    if (r < 0 || r >= rows_total) r = -1;  // never stored
+    const uint4* xs = x + t * dv;
+    for (int v0 = 0; v0 < dv; v0 += 32 * kRowVec) {
+      uint4 buf[kRowVec];
+#pragma unroll
+      for (int u = 0; u < kRowVec; ++u) {
+        const int v = v0 + u * 32 + lane;
+        if (v < dv) buf[u] = __ldcs(xs + v);
+      }
+      for (int j = 0; j < k; ++j) {
+        const int row = __shfl_sync(MOE_FULL_MASK, r, j);
+        if (row < 0) continue;
+        uint4* dst = recv + (int64_t)row * dv;
+#pragma unroll
+        for (int u = 0; u < kRowVec; ++u) {
+          const int v = v0 + u * 32 + lane;
+          if (v < dv) dst[v] = buf[u];
+        }
+      }
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------- combine
+constexpr int kCombVec = 2;
+
+__device__ __forceinline__ void acc_bf16x8(float* acc, const uint4& v, float g) {
+  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(p[i]);
+    acc[2 * i] = fmaf(g, f.x, acc[2 * i]);
+    acc[2 * i + 1] = fmaf(g, f.y, acc[2 * i + 1]);
+  }
+}
+
+// out[t] = sum_j gate[t,j] * y[perm[t,j]], fp32 in j order, one warp per token.
+__global__ void __launch_bounds__(kRowThreads) combine_kernel(
+    const uint4* __restrict__ y, const int32_t* __restrict__ perm,
+    const float* __restrict__ gate, int T, int k, int dv, uint4* __restrict__ out,
+    const int32_t* __restrict__ err) {
+  if (load_err(err)) return;
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += nwarps) {
+    const int r = lane < k ? __ldg(perm + t * k + lane) : 0;
+    const float gl = lane < k ? __ldg(gate + t * k + lane) : 0.f;
+    for (int v0 = 0; v0 < dv; v0 += 32 * kCombVec) {
+      float acc[kCombVec][8];
+#pragma unroll
+      for (int u = 0; u < kCombVec; ++u)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
+      int j = 0;
+      for (; j + 4 <= k; j += 4) {
+        uint4 buf[4][kCombVec];
+        float g[4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int row = __shfl_sync(MOE_FULL_MASK, r, j + jj);
+          g[jj] = __shfl_sync(MOE_FULL_MASK, gl, j + jj);
+#pragma unroll
+          for (int u = 0; u < kCombVec; ++u) {
+            const int v = v0 + u * 32 + lane;
+            if (v < dv) buf[jj][u] = __ldcs(y + (int64_t)row * dv + v);
+          }
+        }
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+          for (int u = 0; u < kCombVec; ++u)
+            if (v0 + u * 32 + lane < dv) acc_bf16x8(acc[u], buf[jj][u], g[jj]);
+      }
+      for (; j < k; ++j) {
+        const int row = __shfl_sync(MOE_FULL_MASK, r, j);
+        const float g = __shfl_sync(MOE_FULL_MASK, gl, j);
+#pragma unroll
+        for (int u = 0; u < kCombVec; ++u) {
+          const int v = v0 + u * 32 + lane;
+          if (v < dv) acc_bf16x8(acc[u], __ldcs(y + (int64_t)row * dv + v), g);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kCombVec; ++u) {
+        const int v = v0 + u * 32 + lane;
+        if (v < dv) {
+          uint4 o;
+          __nv_bfloat162* p = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) p[i] = __floats2bfloat162_rn(acc[u][2 * i], acc[u][2 * i + 1]);
+          out[t * dv + v] = o;
+        }
+      }
+    }
+  }
+}
+
+int row_grid(int T) {
+  const int per_block = kRowThreads / 32;
+  const int64_t want = ((int64_t)T + per_block - 1) / per_block;
+  const int64_t cap = (int64_t)num_sms() * 8;
+  return (int)(want < cap ? want : cap);
+}
+
+}  // namespace
+
+int launch_prefetch(const int32_t* plan, const moe_plan_layout& L, const __nv_bfloat16* W1,
+                    const __nv_bfloat16* W3, const __half* W2, int E, int R, int S, int d,
+                    int F, __nv_bfloat16* P1, __nv_bfloat16* P3, __half* P2,
+                    const int32_t* err, cudaStream_t s) {
+  if (S == 0) return MOE_OK;
+  const int64_t vecs = (int64_t)d * F / 8;
+  prefetch_kernel<<<num_sms() * 4, kCopyThreads, 0, s>>>(
+      plan + L.replica_expert, plan + L.replica_list, reinterpret_cast<const uint4*>(W1),
+      reinterpret_cast<const uint4*>(W3), reinterpret_cast<const uint4*>(W2),
+      reinterpret_cast<uint4*>(P1), reinterpret_cast<uint4*>(P3), reinterpret_cast<uint4*>(P2),
+      vecs, err);
+  return launch_status();
+}
+
+int launch_dispatch(const __nv_bfloat16* x, const int32_t* idx, const int32_t* plan,
+                    const moe_plan_layout& L, int T, int k, int E, int R, int d,
+                    int32_t* ws, __nv_bfloat16* recv, int32_t* perm, int32_t* src,
+                    int32_t* err, cudaStream_t s) {
+  if (T == 0) return MOE_OK;
+  const int C = (int)(((int64_t)T * k) / R);
+  const int tiles = (T + kPlaceTile - 1) / kPlaceTile;
+  tile_count_kernel<<<tiles, kPlaceTile, sizeof(int) * E, s>>>(idx, T, k, E, ws, err);
+  if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
+  const size_t smem = sizeof(int) * (2 * (kPlaceTile / 32) * (size_t)E + 2 * (size_t)R + 1);
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(tile_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return MOE_ERR_LAUNCH;
+  tile_rank_kernel<<<tiles, kPlaceTile, smem, s>>>(idx, T, k, E, R, C, ws, plan, L, perm, src, err);
+  if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
+  scatter_rows_kernel<<<row_grid(T), kRowThreads, 0, s>>>(
+      reinterpret_cast<const uint4*>(x), perm, T, k, d / 8, (int64_t)R * C,
+      reinterpret_cast<uint4*>(recv), err);
+  return launch_status();
+}
+
+int launch_combine(const __nv_bfloat16* y, const int32_t* perm, const float* gate, int T,
+                   int k, int d, __nv_bfloat16* out, const int32_t* err, cudaStream_t s) {
+  if (T == 0) return MOE_OK;
+  combine_kernel<<<row_grid(T), kRowThreads, 0, s>>>(reinterpret_cast<const uint4*>(y), perm,
+                                                      gate, T, k, d / 8,
+                                                      reinterpret_cast<uint4*>(out), err);
+  return launch_status();
+}
+
+}  // namespace moe

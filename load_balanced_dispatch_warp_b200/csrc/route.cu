@@ -1,0 +1,220 @@
+// Router top-k and the demand histogram / maxvio.
+//
+// Top-k follows the router phase of "DeepEP-on-EFA Guidance, section 1: What is MoE":
+// every expert is scored, the top-k are kept, and the gate weights form the routing
+// table.  The histogram follows "MoE Load Balancing: Find Expert Hotspots", section
+// "Separate expert demand from rank placement" (count by expert, then sum over an
+// expert->rank map; balancedness = mean/max), with maxvio = (max - mean)/mean as named in
+// the MoonEP news article.
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+// fp32 -> unsigned key whose unsigned order is the float order (finite values; -0 is
+// folded onto +0 first so that equal logits compare equal).
+__device__ __forceinline__ uint32_t order_key(float v) {
+  v = (v == 0.0f) ? 0.0f : v;
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t key) {
+  const uint32_t u = (key & 0x80000000u) ? (key & 0x7fffffffu) : ~key;
+  return __uint_as_float(u);
+}
+
+// One warp per token.  Lane l holds experts l, l+32, ... (VPL of them); each of the k
+// rounds takes the warp-wide maximum key (redux.sync), then the lowest expert id among
+// the lanes holding it, and retires that entry.  Pad entries have key 0, below every
+// finite float.
+template <int VPL>
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T,
+                                                   int E, int k, int32_t* __restrict__ idx,
+                                                   float* __restrict__ gate,
+                                                   int32_t* __restrict__ err) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const float* row = logits + t * E;
+  uint32_t key[VPL];
+  bool bad = false;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int e = lane + 32 * i;
+    uint32_t kv = 0;
+    if (e < E) {
+      const float v = __ldcs(row + e);
+      bad |= !isfinite(v);
+      kv = order_key(v);
+    }
+    key[i] = kv;
+  }
+  if (__any_sync(MOE_FULL_MASK, bad)) {
+    if (lane == 0) atomicOr(err, MOE_DERR_NONFINITE);
+    return;
+  }
+  uint32_t taken = 0;
+  float my_val = 0.f;
+  int my_id = 0;
+  for (int j = 0; j < k; ++j) {
+    uint32_t best = 0;
+    int best_i = -1;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const bool live = !((taken >> i) & 1u) && (lane + 32 * i < E);
+      if (live && (best_i < 0 || key[i] > best)) {
+        best = key[i];
+        best_i = i;
+      }
+    }
+    const uint32_t wmax = __reduce_max_sync(MOE_FULL_MASK, best);
+    const uint32_t cand = (best_i >= 0 && best == wmax) ? (uint32_t)(lane + 32 * best_i) : 0xffffffffu;
+    const uint32_t wid = __reduce_min_sync(MOE_FULL_MASK, cand);
+    if ((int)(wid & 31u) == lane) taken |= 1u << (wid >> 5);
+    if (lane == j) {
+      my_val = key_value(wmax);
+      my_id = (int)wid;
+    }
+  }
+  const float top = __shfl_sync(MOE_FULL_MASK, my_val, 0);
+  const float ex = lane < k ? expf(my_val - top) : 0.f;
+  const float sum = warp_sum(ex);
+  if (lane < k) {
+    idx[t * k + lane] = my_id;
+    gate[t * k + lane] = ex / sum;
+  }
+}
+
+// Per-block expert histogram over a contiguous token range, with the trace checks of the
+// hotspot fixture (known ids, no expert repeated within a token).  Equal ids in a warp
+// are merged with match.any before one shared-memory add; block totals go to global
+// memory with integer atomics (order-independent, so deterministic).
+__global__ void __launch_bounds__(512) hist_count_kernel(const int32_t* __restrict__ idx, int T,
+                                                         int k, int E, int tokens_per_block,
+                                                         int32_t* __restrict__ counts,
+                                                         int32_t* __restrict__ err) {
+  extern __shared__ int s_hist[];
+  __shared__ int s_err;
+  if (block_should_stop(err)) return;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
+  if (threadIdx.x == 0) s_err = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t t0 = (int64_t)blockIdx.x * tokens_per_block;
+  const int64_t t1 = min((int64_t)T, t0 + tokens_per_block);
+  int my_err = 0;
+  for (int64_t base = t0; base < t1; base += blockDim.x) {
+    const int64_t t = base + threadIdx.x;
+    const bool tok = t < t1;
+    for (int j = 0; j < k; ++j) {
+      int e = tok ? __ldg(idx + t * k + j) : -1;
+      if (tok) {
+        if (e < 0 || e >= E) {
+          my_err |= MOE_DERR_ID_RANGE;
+          e = -1;
+        } else {
+          for (int i = 0; i < j; ++i)
+            if (__ldg(idx + t * k + i) == e) my_err |= MOE_DERR_DUPLICATE;
+        }
+      }
+      const uint32_t peers = __match_any_sync(MOE_FULL_MASK, e);
+      if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&s_hist[e], __popc(peers));
+    }
+  }
+  if (my_err) atomicOr(&s_err, my_err);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    if (s_hist[e]) atomicAdd(counts + e, s_hist[e]);
+  if (threadIdx.x == 0 && s_err) atomicOr(err, s_err);
+}
+
+// Rank loads under the expert->rank map, then maxvio = (R*max - A)/A and balancedness
+// = A/(R*max) from exact integers with one fp64 rounding each.
+__global__ void __launch_bounds__(1024) hist_finalize_kernel(
+    const int32_t* __restrict__ counts, int T, int k, int E, int R,
+    const int32_t* __restrict__ map, int32_t* __restrict__ loads, double* __restrict__ maxvio,
+    double* __restrict__ bal, int32_t* __restrict__ err) {
+  extern __shared__ int s_load[];
+  __shared__ int s_max[32];
+  __shared__ int s_bad;
+  if (block_should_stop(err)) return;
+  const int B = E / R;
+  for (int r = threadIdx.x; r < R; r += blockDim.x) s_load[r] = 0;
+  if (threadIdx.x == 0) s_bad = 0;
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int r = map ? __ldg(map + e) : e / B;
+    if (r < 0 || r >= R) {
+      s_bad = 1;
+    } else {
+      const int c = __ldg(counts + e);
+      if (c) atomicAdd(&s_load[r], c);
+    }
+  }
+  __syncthreads();
+  int mx = 0;
+  for (int r = threadIdx.x; r < R; r += blockDim.x) {
+    loads[r] = s_load[r];
+    mx = max(mx, s_load[r]);
+  }
+  mx = __reduce_max_sync(MOE_FULL_MASK, mx);
+  if ((threadIdx.x & 31) == 0) s_max[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const int nw = (blockDim.x + 31) >> 5;
+    int v = threadIdx.x < nw ? s_max[threadIdx.x] : 0;
+    v = __reduce_max_sync(MOE_FULL_MASK, v);
+    if (threadIdx.x == 0) {
+      const long long A = (long long)T * k;
+      const long long top = (long long)R * v;
+      if (A == 0 || v == 0) {
+        *maxvio = 0.0;
+        *bal = 1.0;
+      } else {
+        *maxvio = (double)(top - A) / (double)A;
+        *bal = (double)A / (double)top;
+      }
+      if (s_bad) atomicOr(err, MOE_DERR_ID_RANGE);
+    }
+  }
+}
+
+}  // namespace
+
+int launch_topk(const float* logits, int T, int E, int k, int32_t* idx, float* gate,
+                int32_t* err, cudaStream_t s) {
+  if (cudaMemsetAsync(err, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_LAUNCH;
+  if (T == 0) return MOE_OK;
+  const int threads = 256, per_block = threads / 32;
+  const unsigned grid = (unsigned)((T + per_block - 1) / per_block);
+#define MOE_TOPK_CASE(V) topk_kernel<V><<<grid, threads, 0, s>>>(logits, T, E, k, idx, gate, err)
+  if (E <= 32) MOE_TOPK_CASE(1);
+  else if (E <= 64) MOE_TOPK_CASE(2);
+  else if (E <= 128) MOE_TOPK_CASE(4);
+  else if (E <= 256) MOE_TOPK_CASE(8);
+  else if (E <= 512) MOE_TOPK_CASE(16);
+  else MOE_TOPK_CASE(32);
+#undef MOE_TOPK_CASE
+  return launch_status();
+}
+
+int launch_histogram(const int32_t* idx, int T, int k, int E, int R, const int32_t* map,
+                     int32_t* counts, int32_t* loads, double* maxvio, double* bal,
+                     int32_t* err, cudaStream_t s) {
+  if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, s) != cudaSuccess) return MOE_ERR_LAUNCH;
+  if (T > 0) {
+    const int threads = 512;
+    // about two blocks per SM, each over a contiguous token range
+    int blocks = 2 * num_sms();
+    int per = (T + blocks - 1) / blocks;
+    per = ((per + 31) / 32) * 32;
+    blocks = (T + per - 1) / per;
+    hist_count_kernel<<<blocks, threads, sizeof(int) * E, s>>>(idx, T, k, E, per, counts, err);
+    if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
+  }
+  hist_finalize_kernel<<<1, 1024, sizeof(int) * R, s>>>(counts, T, k, E, R, map, loads, maxvio,
+                                                       bal, err);
+  return launch_status();
+}
+
+}  // namespace moe

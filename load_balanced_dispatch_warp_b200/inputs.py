@@ -151,18 +151,22 @@ def make_x(w: Workload) -> torch.Tensor:
 
 
 def make_weights(w: Workload, device="cpu"):
-    """Expert weights W1,W3 [E,F,d] and W2 [E,d,F], bf16, N(0, 1/d), drawn on ``device``.
-
-    Each projection is one contiguous tensor (one allocation per projection).
+    """Expert weights W1,W3 [E,F,d] and W2 [E,d,F], N(0, 1/d) rounded to bf16, drawn on
+    ``device``.  W1 and W3 are stored as bf16; W2 holds the same bf16-rounded values in an
+    fp16 tensor (the down projection's storage type), so every input value is identical for
+    the CUDA path and the oracle.  Each projection is one contiguous tensor.
     """
     std = 1.0 / math.sqrt(w.d)
     out = []
-    for stream, shape in ((_S_W1, (w.E, w.F, w.d)), (_S_W3, (w.E, w.F, w.d)), (_S_W2, (w.E, w.d, w.F))):
-        t = torch.empty(shape, dtype=torch.bfloat16, device=device)
+    for stream, shape, dt in ((_S_W1, (w.E, w.F, w.d), torch.bfloat16),
+                              (_S_W3, (w.E, w.F, w.d), torch.bfloat16),
+                              (_S_W2, (w.E, w.d, w.F), torch.float16)):
+        t = torch.empty(shape, dtype=dt, device=device)
         g = _gen(w.seed, stream, device)
         # draw in slabs of one expert to bound the fp32 temporary
         for e in range(w.E):
-            t[e] = (torch.randn(shape[1:], generator=g, dtype=torch.float32, device=device) * std).to(torch.bfloat16)
+            v = torch.randn(shape[1:], generator=g, dtype=torch.float32, device=device) * std
+            t[e] = v.to(torch.bfloat16).to(dt)
         out.append(t)
     return tuple(out)
 

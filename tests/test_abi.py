@@ -1,0 +1,79 @@
+"""The C-ABI library loads, exports every entry point include/moe.h declares, and its
+host-side checks answer without touching a GPU (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import load_balanced_dispatch_warp_b200 as M
+from load_balanced_dispatch_warp_b200 import build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return M.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return set(re.findall(r"^(?:int|int64_t|const char\*)\s+(moe_\w+)\s*\(", text, flags=re.M))
+
+
+def test_header_declares_the_path(lib):
+    names = declared_functions()
+    assert set(M.ENTRY_POINTS) <= names
+    assert set(M.HELPERS) <= names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_plan_layout_is_consistent(lib):
+    E, R, S = 256, 32, 4
+    L = M.plan_layout(E, R, S)
+    B = E // R
+    assert L.max_groups_per_rank == B + S
+    assert L.room_prefix == L.kept_rows + R
+    assert L.expert_home_off == L.room_prefix + R + 1
+    assert L.stream_off == L.expert_home_off + E
+    assert L.replica_expert == L.stream_off + E + 1
+    assert L.replica_list == L.replica_expert + R * S
+    assert L.n_groups == L.replica_list + 1 + R * S
+    assert L.groups % 4 == 0 and L.groups >= L.n_groups + R
+    assert L.words == L.groups + R * (B + S) * 4
+    assert M.dispatch_workspace_words(16384, 256) == 64 * 256
+    assert M.dispatch_workspace_words(257, 8) == 2 * 8
+
+
+def test_host_checks_reject_bad_arguments(lib):
+    P = ctypes.c_void_p
+    fake = P(4096)  # never dereferenced: every call below fails its host checks first
+    # null error word
+    assert lib.moe_topk(fake, 4, 8, 2, fake, fake, None, None) == M.MOE_ERR_ARG
+    # k > E, E > 1024
+    assert lib.moe_topk(fake, 4, 8, 9, fake, fake, fake, None) == M.MOE_ERR_SHAPE
+    assert lib.moe_topk(fake, 4, 2048, 2, fake, fake, fake, None) == M.MOE_ERR_SHAPE
+    # E % R != 0
+    assert lib.moe_histogram_maxvio(fake, 4, 2, 8, 3, None, fake, fake, fake, fake, fake, None) == M.MOE_ERR_SHAPE
+    # T*k % R != 0
+    assert lib.moe_plan_balanced(fake, 3, 1, 8, 2, 2, fake, fake, None) == M.MOE_ERR_SHAPE
+    # too many group slots
+    assert lib.moe_plan_balanced(fake, 4096, 1, 1024, 1024, 4, fake, fake, None) == M.MOE_ERR_SHAPE
+    # d % 128 != 0
+    assert lib.moe_dispatch(fake, fake, fake, 4, 2, 8, 4, 2, 96, fake, fake, fake, fake, fake, None) == M.MOE_ERR_SHAPE
+    # misaligned token rows
+    assert lib.moe_dispatch(P(4098), fake, fake, 4, 2, 8, 4, 2, 128, fake, fake, fake, fake, fake, None) == M.MOE_ERR_ARG
+    # F % 128 != 0, missing pool
+    assert lib.moe_grouped_ffn(fake, fake, fake, fake, fake, fake, fake, fake, 4, 2, 8, 4, 2, 128, 200,
+                               fake, fake, fake, None) == M.MOE_ERR_SHAPE
+    assert lib.moe_grouped_ffn(fake, fake, fake, fake, fake, None, None, None, 4, 2, 8, 4, 2, 128, 256,
+                               fake, fake, fake, None) == M.MOE_ERR_ARG
+    assert lib.moe_combine(fake, fake, fake, 4, 33, 128, fake, fake, None) == M.MOE_ERR_SHAPE
+    assert lib.moe_prefetch_replicas(fake, fake, fake, fake, 8, 4, 2, 128, 256, None, None, None, fake, None) == M.MOE_ERR_ARG
+    assert lib.moe_status_string(M.MOE_ERR_SHAPE) == b"size limit violated"

@@ -1,0 +1,195 @@
+"""CUDA path vs the CPU oracle, call by call, through the C ABI (needs a B200).
+
+Integer outputs (top-k ids, counts, loads, maxvio, the plan, perm/src, recv rows, pool
+slots) must be bit-exact; gates within 1e-6; h, y and out within 1e-2*max(1,|oracle|).
+Small shapes compare every element; the full-size workloads compare every integer output
+and a sample of tokens for the floating-point ones.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import load_balanced_dispatch_warp_b200 as M
+from load_balanced_dispatch_warp_b200 import build
+from load_balanced_dispatch_warp_b200 import inputs as I
+from oracle import moe_oracle as O
+
+from harness import (check_ffn_combine_full, check_ffn_combine_sampled, check_integer_parity,
+                     check_rows_and_pool, make_inputs, oracle_integer_path, run_gpu)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    build.build()
+    M.lib()
+
+
+SMALL = [
+    I.WORKLOADS["tiny"],
+    I.small_workload("ragged", 300, 16, 4, 4, 2, 256, 384, alpha=1.0, seed=1),
+    I.small_workload("mid", 1000, 64, 6, 8, 8, 512, 256, alpha=0.6, seed=2),
+    I.small_workload("k_eq_E", 64, 8, 8, 4, 2, 128, 128, alpha=0.0, seed=3),
+    I.small_workload("k1_d384", 96, 32, 1, 8, 2, 384, 128, alpha=1.5, seed=4),
+    I.small_workload("one_rank", 64, 16, 4, 1, 0, 128, 128, alpha=1.0, seed=5),
+    I.small_workload("rank_per_expert", 256, 8, 2, 8, 3, 256, 256, alpha=0.5, seed=6),
+    I.small_workload("hot", 512, 32, 4, 8, 4, 128, 256, alpha=2.5, seed=7),
+    I.small_workload("wide_E", 200, 512, 8, 16, 12, 128, 128, alpha=0.3, seed=8),
+    I.small_workload("wide_E_few_slots", 200, 512, 8, 16, 4, 128, 128, alpha=0.3, seed=8),
+]
+
+
+@pytest.mark.parametrize("w", SMALL, ids=[w.name for w in SMALL])
+def test_layer_parity_small(w):
+    logits, x, weights = make_inputs(w)
+    ref = oracle_integer_path(w, logits)
+    L = run_gpu(w, logits, x, weights)
+    if ref["err"]:
+        assert int(L.err.item()) == ref["err"]
+        return
+    check_integer_parity(L, w, ref)
+    check_rows_and_pool(L, w, x, weights, ref)
+    check_ffn_combine_full(L, w, x, weights, ref)
+
+
+FULL = ["near_balanced", "qwen_mv0.2", "qwen_mv1", "qwen_mv5", "qwen_mv15", "mixtral", "deepseek"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_layer_parity_full_size(name):
+    w = I.WORKLOADS[name]
+    logits, x, weights = make_inputs(w)
+    ref = oracle_integer_path(w, logits)
+    assert ref["err"] == 0
+    L = run_gpu(w, logits, x, weights)
+    check_integer_parity(L, w, ref)
+    check_rows_and_pool(L, w, x, weights, ref)
+    # every rank holds exactly C rows: the plan's groups tile [u*C, (u+1)*C)
+    rng = np.random.default_rng(11)
+    tokens = sorted(rng.choice(w.T, size=8, replace=False).tolist()) + [w.T - 1]
+    check_ffn_combine_sampled(L, w, x, weights, ref, tokens)
+    del L, weights
+    torch.cuda.empty_cache()
+
+
+def test_histogram_fixture_mappings_on_gpu():
+    """The pages' 16-token trace through moe_histogram_maxvio under both mappings."""
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "hotspot_fixture.json")))
+    idx = torch.tensor([[int(p[0]), int(p[1])] for p in g["pairs"]], dtype=torch.int32, device="cuda")
+    for mapping, loads_exp, bal in ((g["initial_mapping"], g["initial_rank_demand"], 8 / 15),
+                                    (g["proposed_mapping"], g["proposed_rank_demand"], 0.8)):
+        m = torch.zeros(8, dtype=torch.int32)
+        for r, es in enumerate(mapping):
+            m[es] = r
+        counts = torch.empty(8, dtype=torch.int32, device="cuda")
+        loads = torch.empty(4, dtype=torch.int32, device="cuda")
+        mv = torch.empty(1, dtype=torch.float64, device="cuda")
+        b = torch.empty(1, dtype=torch.float64, device="cuda")
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        M.moe_histogram_maxvio(idx, 8, 4, counts, loads, mv, b, err, expert_to_rank=m.cuda())
+        torch.cuda.synchronize()
+        assert err.item() == 0
+        assert counts.tolist() == g["expert_demand"]
+        assert loads.tolist() == loads_exp
+        assert b.item() == bal
+        assert mv.item() == max(loads_exp) / 8 - 1
+
+
+def _hist(idx, E, R):
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    loads = torch.empty(R, dtype=torch.int32, device="cuda")
+    mv = torch.empty(1, dtype=torch.float64, device="cuda")
+    b = torch.empty(1, dtype=torch.float64, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    M.moe_histogram_maxvio(idx, E, R, counts, loads, mv, b, err)
+    torch.cuda.synchronize()
+    return int(err.item())
+
+
+def test_trace_validation_errors():
+    good = torch.tensor([[0, 1], [2, 3], [4, 5]], dtype=torch.int32, device="cuda")
+    assert _hist(good, 8, 4) == 0
+    bad = good.clone()
+    bad[1, 1] = 8
+    assert _hist(bad, 8, 4) == M.DERR_ID_RANGE
+    bad[1, 1] = -3
+    assert _hist(bad, 8, 4) == M.DERR_ID_RANGE
+    dup = good.clone()
+    dup[2, 1] = 4
+    assert _hist(dup, 8, 4) == M.DERR_DUPLICATE
+
+
+def test_nonfinite_logit_stops_the_layer():
+    w = I.small_workload("nan", 64, 8, 2, 4, 2, 128, 128, alpha=1.0, seed=9)
+    logits, x, weights = make_inputs(w)
+    for bad in (float("nan"), float("inf"), float("-inf")):
+        lg = logits.clone()
+        lg[17, 3] = bad
+        L = M.MoELayer(w.T, w.E, w.k, w.R, w.S, w.d, w.F)
+        L.out.fill_(7.0)
+        L.forward(lg.cuda(), x.cuda(), *weights)
+        torch.cuda.synchronize()
+        assert int(L.err.item()) == M.DERR_NONFINITE
+        assert bool((L.out == 7.0).all()), "calls after an error must not run"
+
+
+def test_slot_overflow_sets_error_and_stops():
+    # all tokens on experts 0..3 (rank 0) and no prefetch slots: replicas are needed
+    w = I.small_workload("noslots", 64, 16, 4, 4, 0, 128, 128, alpha=200.0, seed=10)
+    logits, x, weights = make_inputs(w)
+    ref = oracle_integer_path(w, logits)
+    assert ref["err"] == O.ERR_SLOTS
+    L = M.MoELayer(w.T, w.E, w.k, w.R, w.S, w.d, w.F)
+    L.recv.fill_(3.0)
+    L.forward(logits.cuda(), x.cuda(), *weights)
+    torch.cuda.synchronize()
+    assert int(L.err.item()) == M.DERR_SLOTS
+    assert bool((L.recv == 3.0).all())
+
+
+def test_empty_batch():
+    w = I.small_workload("empty", 0, 8, 2, 4, 2, 128, 128)
+    W = I.make_weights(w, device="cuda")
+    L = M.MoELayer(0, 8, 2, 4, 2, 128, 128)
+    L.forward(torch.empty(0, 8, device="cuda"), torch.empty(0, 128, dtype=torch.bfloat16, device="cuda"), *W)
+    torch.cuda.synchronize()
+    assert int(L.err.item()) == 0
+    assert L.maxvio.item() == 0.0 and L.balancedness.item() == 1.0
+    assert L.counts.tolist() == [0] * 8 and L.loads.tolist() == [0] * 4
+
+
+def test_topk_ties_and_signed_zero():
+    T, E, k = 512, 64, 6
+    g = torch.Generator().manual_seed(12)
+    vals = torch.tensor([-1.0, -0.0, 0.0, 0.5, 2.0])
+    logits = vals[torch.randint(0, 5, (T, E), generator=g)].contiguous()
+    idx_ref, gate_ref, err = O.topk_route(logits.numpy(), k)
+    idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    gate = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    e = torch.zeros(1, dtype=torch.int32, device="cuda")
+    M.moe_topk(logits.cuda(), k, idx, gate, e)
+    torch.cuda.synchronize()
+    assert e.item() == 0
+    assert np.array_equal(idx.cpu().numpy(), idx_ref)
+    assert np.abs(gate.cpu().double().numpy() - gate_ref).max() <= 1e-6
+
+
+@pytest.mark.parametrize("E", [1, 3, 33, 100, 257, 700, 1024])
+def test_topk_expert_counts(E):
+    T = 333
+    k = min(E, 8)
+    logits = torch.randn(T, E, generator=torch.Generator().manual_seed(E))
+    idx_ref, gate_ref, _ = O.topk_route(logits.numpy(), k)
+    idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    gate = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    e = torch.zeros(1, dtype=torch.int32, device="cuda")
+    M.moe_topk(logits.cuda(), k, idx, gate, e)
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.cpu().numpy(), idx_ref)
+    assert np.abs(gate.cpu().double().numpy() - gate_ref).max() <= 1e-6
