@@ -209,6 +209,29 @@ int moe_grouped_ffn(const moe_bf16* recv, const int32_t* plan, const moe_bf16* W
                     moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * Dispatch without a workspace argument.  The pages have no counterpart: this is a
+ * convenience of this library for callers that cannot allocate device memory when they
+ * dispatch -- an operator or plugin interface of another runtime that passes only its
+ * input and output buffers, or a host program whose hot path must not call cudaMalloc
+ * (which may synchronise the device).  It computes exactly what moe_dispatch computes,
+ * with the same arguments minus `workspace`, and allocates nothing: the placement
+ * counts live in a static device array of MOE_NOALLOC_SCRATCH_WORDS int32 words (1 MiB)
+ * that every GPU loading the library holds until the process exits.
+ *   - Returns MOE_ERR_SHAPE when moe_dispatch_workspace_words(T, E) exceeds
+ *     MOE_NOALLOC_SCRATCH_WORDS (e.g. T = 65536 with E = 1024 fits, T = 131072 does not).
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call before any
+ *     stream capture.  MOE_ERR_DEVICE if the lookup fails.
+ *   - All calls share the array and it keeps the last call's contents; no word of it has
+ *     to start at zero.  Calls that overlap on the GPU (several streams or host threads
+ *     on one device) race on it: serialise them.
+ */
+#define MOE_NOALLOC_SCRATCH_WORDS 262144
+int moe_dispatch_noalloc(const moe_bf16* x, const int32_t* idx, const int32_t* plan, int T,
+                         int k, int E, int R, int S, int d, moe_bf16* recv, int32_t* perm,
+                         int32_t* src, int32_t* err, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
  * Combine.   [Primer] phase (d): expert outputs return to their token and are summed
  * with the gate weights; the mirror (transpose) of dispatch.
  *   out[t] = sum_{j=0..k-1} gate[t,j] * y[perm[t,j]]   (fp32, j order; bf16 out)

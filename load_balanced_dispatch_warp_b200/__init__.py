@@ -152,6 +152,25 @@ def moe_dispatch(x, idx, plan, E, R, S, workspace, recv, perm, src, err, stream=
         _stream(stream)), "moe_dispatch")
 
 
+NOALLOC_SCRATCH_WORDS = 262144  # MOE_NOALLOC_SCRATCH_WORDS
+
+
+def moe_dispatch_noalloc(x, idx, plan, E, R, S, recv, perm, src, err, stream=None):
+    """moe_dispatch without a workspace: for callers that cannot allocate device memory
+    when they dispatch; the library uses its own static 1 MiB scratch (see moe.h)."""
+    f = lib().moe_dispatch_noalloc
+    if f.restype is not ctypes.c_int or f.argtypes is None:
+        P, I = ctypes.c_void_p, ctypes.c_int
+        f.argtypes = [P, P, P, I, I, I, I, I, I, P, P, P, P, P]
+        f.restype = ctypes.c_int
+    T, d = x.shape
+    k = idx.shape[1]
+    _check(f(_ptr(x, torch.bfloat16, "x"), _ptr(idx, torch.int32, "idx"), _ptr(plan, torch.int32, "plan"),
+             T, k, E, R, S, d, _ptr(recv, torch.bfloat16, "recv"), _ptr(perm, torch.int32, "perm"),
+             _ptr(src, torch.int32, "src"), _ptr(err, torch.int32, "err"), _stream(stream)),
+           "moe_dispatch_noalloc")
+
+
 def moe_grouped_ffn(recv, plan, W1, W3, W2, P1, P3, P2, T, k, R, S, h, y, err, stream=None):
     E, F, d = W1.shape
     bf, hf = torch.bfloat16, torch.float16
