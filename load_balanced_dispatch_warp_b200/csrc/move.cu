@@ -112,8 +112,17 @@ __global__ void __launch_bounds__(kPlaceTile) tile_rank_kernel(
   }
   __syncthreads();
   for (int e = tid; e < E; e += blockDim.x) {
-    int run = 0;
-    for (int p = 0; p < tile; ++p) run += __ldg(ws + (int64_t)p * E + e);
+    // assignments of e in all earlier tiles: independent partial sums keep the loads of
+    // the column in flight together
+    int r0 = 0, r1 = 0, r2 = 0, r3 = 0, p = 0;
+    for (; p + 4 <= tile; p += 4) {
+      r0 += __ldg(ws + (int64_t)p * E + e);
+      r1 += __ldg(ws + (int64_t)(p + 1) * E + e);
+      r2 += __ldg(ws + (int64_t)(p + 2) * E + e);
+      r3 += __ldg(ws + (int64_t)(p + 3) * E + e);
+    }
+    for (; p < tile; ++p) r0 += __ldg(ws + (int64_t)p * E + e);
+    int run = r0 + r1 + r2 + r3;
     for (int w = 0; w < W; ++w) {
       s_pre[w * E + e] = run;
       run += __popc(s_mask[w * E + e]);
@@ -198,7 +207,18 @@ __device__ __forceinline__ void acc_bf16x8(float* acc, const uint4& v, float g) 
   }
 }
 
-// out[t] = sum_j gate[t,j] * y[perm[t,j]], fp32 in j order, one warp per token.
+__device__ __forceinline__ uint4 pack_bf16x8(const float* a) {
+  uint4 o;
+  __nv_bfloat162* p = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) p[i] = __floats2bfloat162_rn(a[2 * i], a[2 * i + 1]);
+  return o;
+}
+
+// out[t] = sum_j gate[t,j] * y[perm[t,j]], fp32 in j order, one warp per token.  With the
+// top-k known at compile time (K > 0) all K x kCombVec gathers of a lane are issued before
+// the first FMA; K == 0 is the generic loop.
+template <int K>
 __global__ void __launch_bounds__(kRowThreads) combine_kernel(
     const uint4* __restrict__ y, const int32_t* __restrict__ perm,
     const float* __restrict__ gate, int T, int k, int dv, uint4* __restrict__ out,
@@ -209,52 +229,40 @@ __global__ void __launch_bounds__(kRowThreads) combine_kernel(
   for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += nwarps) {
     const int r = lane < k ? __ldg(perm + t * k + lane) : 0;
     const float gl = lane < k ? __ldg(gate + t * k + lane) : 0.f;
-    for (int v0 = 0; v0 < dv; v0 += 32 * kCombVec) {
+    for (int v0 = lane; v0 < dv; v0 += 32 * kCombVec) {
       float acc[kCombVec][8];
 #pragma unroll
       for (int u = 0; u < kCombVec; ++u)
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
-      int j = 0;
-      for (; j + 4 <= k; j += 4) {
-        uint4 buf[4][kCombVec];
-        float g[4];
+      if (K > 0) {
+        uint4 buf[K > 0 ? K : 1][kCombVec];
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          const int row = __shfl_sync(MOE_FULL_MASK, r, j + jj);
-          g[jj] = __shfl_sync(MOE_FULL_MASK, gl, j + jj);
-#pragma unroll
-          for (int u = 0; u < kCombVec; ++u) {
-            const int v = v0 + u * 32 + lane;
-            if (v < dv) buf[jj][u] = __ldcs(y + (int64_t)row * dv + v);
-          }
-        }
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj)
+        for (int j = 0; j < K; ++j) {
+          const uint4* yr = y + (int64_t)__shfl_sync(MOE_FULL_MASK, r, j) * dv;
 #pragma unroll
           for (int u = 0; u < kCombVec; ++u)
-            if (v0 + u * 32 + lane < dv) acc_bf16x8(acc[u], buf[jj][u], g[jj]);
-      }
-      for (; j < k; ++j) {
-        const int row = __shfl_sync(MOE_FULL_MASK, r, j);
-        const float g = __shfl_sync(MOE_FULL_MASK, gl, j);
+            if (v0 + u * 32 < dv) buf[j][u] = __ldcs(yr + v0 + u * 32);
+        }
 #pragma unroll
-        for (int u = 0; u < kCombVec; ++u) {
-          const int v = v0 + u * 32 + lane;
-          if (v < dv) acc_bf16x8(acc[u], __ldcs(y + (int64_t)row * dv + v), g);
+        for (int j = 0; j < K; ++j) {
+          const float g = __shfl_sync(MOE_FULL_MASK, gl, j);
+#pragma unroll
+          for (int u = 0; u < kCombVec; ++u)
+            if (v0 + u * 32 < dv) acc_bf16x8(acc[u], buf[j][u], g);
+        }
+      } else {
+        for (int j = 0; j < k; ++j) {
+          const uint4* yr = y + (int64_t)__shfl_sync(MOE_FULL_MASK, r, j) * dv;
+          const float g = __shfl_sync(MOE_FULL_MASK, gl, j);
+#pragma unroll
+          for (int u = 0; u < kCombVec; ++u)
+            if (v0 + u * 32 < dv) acc_bf16x8(acc[u], __ldcs(yr + v0 + u * 32), g);
         }
       }
 #pragma unroll
-      for (int u = 0; u < kCombVec; ++u) {
-        const int v = v0 + u * 32 + lane;
-        if (v < dv) {
-          uint4 o;
-          __nv_bfloat162* p = reinterpret_cast<__nv_bfloat162*>(&o);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) p[i] = __floats2bfloat162_rn(acc[u][2 * i], acc[u][2 * i + 1]);
-          out[t * dv + v] = o;
-        }
-      }
+      for (int u = 0; u < kCombVec; ++u)
+        if (v0 + u * 32 < dv) out[t * dv + v0 + u * 32] = pack_bf16x8(acc[u]);
     }
   }
 }
@@ -307,9 +315,22 @@ int launch_dispatch(const __nv_bfloat16* x, const int32_t* idx, const int32_t* p
 int launch_combine(const __nv_bfloat16* y, const int32_t* perm, const float* gate, int T,
                    int k, int d, __nv_bfloat16* out, const int32_t* err, cudaStream_t s) {
   if (T == 0) return MOE_OK;
-  combine_kernel<<<row_grid(T), kRowThreads, 0, s>>>(reinterpret_cast<const uint4*>(y), perm,
-                                                      gate, T, k, d / 8,
-                                                      reinterpret_cast<uint4*>(out), err);
+  const uint4* yv = reinterpret_cast<const uint4*>(y);
+  uint4* ov = reinterpret_cast<uint4*>(out);
+  const int g = row_grid(T), dv = d / 8;
+#define MOE_COMBINE_CASE(KK) combine_kernel<KK><<<g, kRowThreads, 0, s>>>(yv, perm, gate, T, k, dv, ov, err)
+  switch (k) {
+    case 1: MOE_COMBINE_CASE(1); break;
+    case 2: MOE_COMBINE_CASE(2); break;
+    case 3: MOE_COMBINE_CASE(3); break;
+    case 4: MOE_COMBINE_CASE(4); break;
+    case 5: MOE_COMBINE_CASE(5); break;
+    case 6: MOE_COMBINE_CASE(6); break;
+    case 7: MOE_COMBINE_CASE(7); break;
+    case 8: MOE_COMBINE_CASE(8); break;
+    default: MOE_COMBINE_CASE(0); break;
+  }
+#undef MOE_COMBINE_CASE
   return launch_status();
 }
 
