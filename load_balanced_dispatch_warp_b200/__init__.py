@@ -275,7 +275,7 @@ class MoELayer:
 
     # kernels launched by forward() (for launch accounting)
     def kernels_per_forward(self) -> int:
-        n = (1 if self.T > 0 else 0) + (2 if self.T > 0 else 1) + 1  # topk, hist, plan
+        n = (1 if self.T > 0 else 0) + 1 + 1  # topk, histogram, plan
         n += 1 if self.S > 0 else 0           # prefetch
         n += 3 if self.T > 0 else 0           # dispatch: tile counts, ranks, row scatter
         n += 2 if self.T > 0 else 0           # two grouped GEMMs

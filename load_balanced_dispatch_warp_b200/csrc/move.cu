@@ -94,6 +94,8 @@ __global__ void __launch_bounds__(kPlaceTile) tile_rank_kernel(
   int* s_pre = smem + W * E;                              // [W][E] start of each warp
   int* s_rp = s_pre + W * E;                              // [R+1] room prefix
   int* s_kr = s_rp + R + 1;                               // [R] kept rows
+  int* s_home = s_kr + R;                                 // [E] home offset (-1 streamed)
+  int* s_so = s_home + E;                                 // [E] stream offset
   __shared__ int s_bad;
   if (block_should_stop(err)) return;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -101,6 +103,10 @@ __global__ void __launch_bounds__(kPlaceTile) tile_rank_kernel(
   for (int i = tid; i < W * E; i += blockDim.x) s_mask[i] = 0;
   for (int r = tid; r <= R; r += blockDim.x) s_rp[r] = plan[L.room_prefix + r];
   for (int r = tid; r < R; r += blockDim.x) s_kr[r] = plan[L.kept_rows + r];
+  for (int e = tid; e < E; e += blockDim.x) {
+    s_home[e] = plan[L.expert_home_off + e];
+    s_so[e] = plan[L.stream_off + e];
+  }
   if (tid == 0) s_bad = 0;
   __syncthreads();
   const int64_t t = (int64_t)tile * kPlaceTile + tid;
@@ -137,12 +143,12 @@ __global__ void __launch_bounds__(kPlaceTile) tile_rank_kernel(
       const int e = __ldg(idx + t * k + j);
       if (e < 0 || e >= E) { s_bad = 1; continue; }
       const int q = s_pre[warp * E + e] + __popc(s_mask[warp * E + e] & lt);
-      const int off = __ldg(plan + L.expert_home_off + e);
+      const int off = s_home[e];
       int64_t row;
       if (off >= 0) {
         row = (int64_t)(e / B) * C + off + q;
       } else {
-        const int p = __ldg(plan + L.stream_off + e) + q;
+        const int p = s_so[e] + q;
         int a = 0, b = R - 1;  // last rank with room_prefix <= p
         while (a < b) {
           const int m = (a + b + 1) >> 1;
@@ -299,7 +305,7 @@ int launch_dispatch(const __nv_bfloat16* x, const int32_t* idx, const int32_t* p
   const int tiles = (T + kPlaceTile - 1) / kPlaceTile;
   tile_count_kernel<<<tiles, kPlaceTile, sizeof(int) * E, s>>>(idx, T, k, E, ws, err);
   if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
-  const size_t smem = sizeof(int) * (2 * (kPlaceTile / 32) * (size_t)E + 2 * (size_t)R + 1);
+  const size_t smem = sizeof(int) * (2 * (kPlaceTile / 32) * (size_t)E + 2 * (size_t)R + 1 + 2 * (size_t)E);
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(tile_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)

@@ -8,13 +8,15 @@
 //     are kept whole while their running sum fits in C = T*k/R; the rest are streamed;
 //   - the streamed experts in id order form one stream, cut by the ranks' leftover rooms
 //     in rank order; each foreign run in a rank's piece is a replica taking the next slot.
-// Everything is integer arithmetic, block scans and per-thread walks: deterministic.
+// Everything is integer arithmetic, block scans and ballots (one warp per rank):
+// deterministic.
 #include "common.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int kPlanThreads = 1024;
+constexpr int kPlanThreads = 256;
+constexpr int kPlanWarps = kPlanThreads / 32;
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __restrict__ counts,
                                                             int T, int k, int E, int R, int S,
@@ -27,14 +29,17 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
   __shared__ int s_room[1025];    // rooms, then their exclusive prefix
   __shared__ int s_kr[1024];      // kept rows per rank
   __shared__ int s_off[1024];     // local row offset of a kept expert, -1 otherwise
+  __shared__ int s_sidx[1025];    // streamed experts (non-zero stream length) in id order
   __shared__ int s_nrep[1025];    // replicas per rank, then their exclusive prefix
   __shared__ int s_scan[33];
+  __shared__ int s_ns;
   if (block_should_stop(err)) return;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int B = E / R;
   const int C = (int)(((long long)T * k) / R);
 
   for (int e = tid; e < E; e += blockDim.x) s_c[e] = counts[e];
+  for (int r = tid; r < R; r += blockDim.x) s_kr[r] = 0;
   __syncthreads();
 
   // keep test: inclusive running sum of the rank's experts in (count, id) order <= C
@@ -45,11 +50,13 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
       const int cf = s_c[f];
       if (cf < c || (cf == c && f < e)) cum += cf;
     }
-    s_kept[e] = cum <= C;
+    const int kept = cum <= C;
+    s_kept[e] = kept;
+    if (kept && c) atomicAdd(&s_kr[e / B], c);
   }
   __syncthreads();
 
-  // local offsets of kept experts (id order) and kept rows per rank
+  // local offsets of kept experts (id order); stream lengths; rooms
   for (int e = tid; e < E; e += blockDim.x) {
     int off = -1;
     if (s_kept[e]) {
@@ -59,20 +66,20 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
     }
     s_off[e] = off;
     s_so[e] = s_kept[e] ? 0 : s_c[e];
+    s_nrep[e] = (!s_kept[e] && s_c[e] > 0) ? 1 : 0;  // streamed flag (s_nrep as temp)
   }
-  for (int r = tid; r < R; r += blockDim.x) {
-    int kr = 0;
-    for (int f = r * B; f < (r + 1) * B; ++f)
-      if (s_kept[f]) kr += s_c[f];
-    s_kr[r] = kr;
-    s_room[r] = C - kr;
-  }
+  for (int r = tid; r < R; r += blockDim.x) s_room[r] = C - s_kr[r];
   __syncthreads();
   const int stream_len = block_exclusive_scan(s_so, E, s_scan);
   const int room_total = block_exclusive_scan(s_room, R, s_scan);
+  // compact list of streamed experts in id order (= stream order)
+  const int n_streamed = block_exclusive_scan(s_nrep, E, s_scan);
+  for (int e = tid; e < E; e += blockDim.x)
+    if (!s_kept[e] && s_c[e] > 0) s_sidx[s_nrep[e]] = e;
   if (tid == 0) {
     s_so[E] = stream_len;
     s_room[R] = room_total;
+    s_ns = n_streamed;
   }
   __syncthreads();
 
@@ -89,57 +96,71 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
   for (int e = tid; e < E; e += blockDim.x) home_off[e] = s_off[e];
   for (int e = tid; e <= E; e += blockDim.x) stream_off[e] = s_so[e];
 
-  // one thread per rank: its kept experts, then the runs of its stream piece
+  // one warp per rank: its kept experts (id order), then the runs of its stream piece
   const int G = B + S;
-  int overflow = 0;
-  for (int u = tid; u < R; u += blockDim.x) {
+  for (int u = warp; u < R; u += kPlanWarps) {
     int32_t* gu = groups + (int64_t)u * G * 4;
     int g = 0;
-    for (int e = u * B; e < (u + 1) * B; ++e) {
-      if (s_kept[e] && s_c[e] > 0) {
-        gu[4 * g + 0] = u * C + s_off[e];
-        gu[4 * g + 1] = s_c[e];
-        gu[4 * g + 2] = e;
-        gu[4 * g + 3] = e;
-        ++g;
+    for (int c0 = 0; c0 < B; c0 += 32) {
+      const int e = u * B + c0 + lane;
+      const bool on = c0 + lane < B && s_kept[e] && s_c[e] > 0;
+      const uint32_t m = __ballot_sync(MOE_FULL_MASK, on);
+      if (on) {
+        int4* rec = reinterpret_cast<int4*>(gu) + g + __popc(m & lanemask_lt());
+        *rec = make_int4(u * C + s_off[e], s_c[e], e, e);
       }
+      g += __popc(m);
     }
     const int lo = s_room[u], hi = s_room[u + 1];
     int nrep = 0;
     if (lo < hi) {
-      // first expert whose stream range ends after lo
-      int a = 0, b = E - 1;
+      // first streamed expert whose stream range ends after lo
+      int a = 0, b = s_ns - 1;
       while (a < b) {
-        const int m = (a + b) >> 1;
-        if (s_so[m + 1] > lo) b = m; else a = m + 1;
+        const int mid = (a + b) >> 1;
+        const int em = s_sidx[mid];
+        if (s_so[em] + s_c[em] > lo) b = mid; else a = mid + 1;
       }
-      for (int e = a; e < E && s_so[e] < hi; ++e) {
-        const int s0 = max(lo, s_so[e]), s1 = min(hi, s_so[e + 1]);
-        if (s0 >= s1) continue;  // kept or empty experts have zero stream length
-        const int row = u * C + s_kr[u] + (s0 - lo);
-        int ref;
-        if (e / B == u) {
-          ref = e;
-        } else {
-          if (nrep >= S) { ++nrep; continue; }
-          rep[u * S + nrep] = e;
-          ref = E + u * S + nrep;
-          ++nrep;
+      for (int i0 = a; i0 < s_ns; i0 += 32) {
+        const int i = i0 + lane;
+        int e = -1, s0 = 0, s1 = 0;
+        if (i < s_ns) {
+          e = s_sidx[i];
+          s0 = max(lo, s_so[e]);
+          s1 = min(hi, s_so[e] + s_c[e]);
         }
-        gu[4 * g + 0] = row;
-        gu[4 * g + 1] = s1 - s0;
-        gu[4 * g + 2] = e;
-        gu[4 * g + 3] = ref;
-        ++g;
+        const bool on = e >= 0 && s0 < s1;
+        const bool foreign = on && e / B != u;
+        const uint32_t mfor = __ballot_sync(MOE_FULL_MASK, foreign);
+        const int slot = nrep + __popc(mfor & lanemask_lt());
+        // a run at its home rank is always recorded; a replica only while slots remain
+        // (more than S replicas leaves the plan invalid: MOE_DERR_SLOTS below)
+        const bool write = on && (!foreign || slot < S);
+        const uint32_t mw = __ballot_sync(MOE_FULL_MASK, write);
+        if (write) {
+          int ref = e;
+          if (foreign) {
+            rep[u * S + slot] = e;
+            ref = E + u * S + slot;
+          }
+          int4* rec = reinterpret_cast<int4*>(gu) + g + __popc(mw & lanemask_lt());
+          *rec = make_int4(u * C + s_kr[u] + (s0 - lo), s1 - s0, e, ref);
+        }
+        g += __popc(mw);
+        nrep += __popc(mfor);
+        // stop once this chunk reached past the piece
+        const bool past = e < 0 || s_so[e] >= hi;
+        if (__any_sync(MOE_FULL_MASK, past)) break;
       }
     }
-    for (int i = 4 * g; i < 4 * G; ++i) gu[i] = -1;
-    for (int s = min(nrep, S); s < S; ++s) rep[u * S + s] = -1;
-    n_groups[u] = g;
-    s_nrep[u] = min(nrep, S);
-    if (nrep > S) overflow = 1;
+    for (int i = g * 4 + lane; i < 4 * G; i += 32) gu[i] = -1;
+    for (int s = min(nrep, S) + lane; s < S; s += 32) rep[u * S + s] = -1;
+    if (lane == 0) {
+      n_groups[u] = g;
+      s_nrep[u] = min(nrep, S);
+      if (nrep > S) atomicOr(err, MOE_DERR_SLOTS);
+    }
   }
-  if (overflow) atomicOr(err, MOE_DERR_SLOTS);
   __syncthreads();
   // compact list of filled slots in ascending slot order (for the prefetch copy)
   const int n_filled = block_exclusive_scan(s_nrep, R, s_scan);

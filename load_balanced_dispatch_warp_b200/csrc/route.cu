@@ -23,10 +23,11 @@ __device__ __forceinline__ float key_value(uint32_t key) {
   return __uint_as_float(u);
 }
 
-// One warp per token.  Lane l holds experts l, l+32, ... (VPL of them); each of the k
-// rounds takes the warp-wide maximum key (redux.sync), then the lowest expert id among
-// the lanes holding it, and retires that entry.  Pad entries have key 0, below every
-// finite float.
+// One warp per token.  Lane l holds experts l, l+32, ... (VPL of them) as
+// order-preserving keys; pad entries (e >= E) and taken entries have key 0, below every
+// finite float, so each of the k rounds is a plain max over the lane's keys, a warp-wide
+// max key (redux.sync), the lowest expert id among the lanes holding it (redux.sync), and
+// the winner zeroes that key.  Instruction count, not memory, bounds this kernel.
 template <int VPL>
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T,
                                                    int E, int k, int32_t* __restrict__ idx,
@@ -53,24 +54,25 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
     if (lane == 0) atomicOr(err, MOE_DERR_NONFINITE);
     return;
   }
-  uint32_t taken = 0;
   float my_val = 0.f;
   int my_id = 0;
   for (int j = 0; j < k; ++j) {
-    uint32_t best = 0;
-    int best_i = -1;
+    // lane maximum; equal keys keep the lower slot (= lower expert id)
+    uint32_t best = key[0];
+    int best_i = 0;
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      const bool live = !((taken >> i) & 1u) && (lane + 32 * i < E);
-      if (live && (best_i < 0 || key[i] > best)) {
-        best = key[i];
-        best_i = i;
-      }
+    for (int i = 1; i < VPL; ++i) {
+      const bool gt = key[i] > best;
+      best = gt ? key[i] : best;
+      best_i = gt ? i : best_i;
     }
     const uint32_t wmax = __reduce_max_sync(MOE_FULL_MASK, best);
-    const uint32_t cand = (best_i >= 0 && best == wmax) ? (uint32_t)(lane + 32 * best_i) : 0xffffffffu;
+    const uint32_t cand = best == wmax ? (uint32_t)(lane + 32 * best_i) : 0xffffffffu;
     const uint32_t wid = __reduce_min_sync(MOE_FULL_MASK, cand);
-    if ((int)(wid & 31u) == lane) taken |= 1u << (wid >> 5);
+    const bool mine = (int)(wid & 31u) == lane;
+    const int wi = (int)(wid >> 5);
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) key[i] = (mine && i == wi) ? 0u : key[i];
     if (lane == j) {
       my_val = key_value(wmax);
       my_id = (int)wid;
@@ -88,13 +90,21 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
 // Per-block expert histogram over a contiguous token range, with the trace checks of the
 // hotspot fixture (known ids, no expert repeated within a token).  Equal ids in a warp
 // are merged with match.any before one shared-memory add; block totals go to global
-// memory with integer atomics (order-independent, so deterministic).
-__global__ void __launch_bounds__(512) hist_count_kernel(const int32_t* __restrict__ idx, int T,
-                                                         int k, int E, int tokens_per_block,
-                                                         int32_t* __restrict__ counts,
-                                                         int32_t* __restrict__ err) {
-  extern __shared__ int s_hist[];
-  __shared__ int s_err;
+// memory with integer atomics (order-independent, so deterministic).  The last block to
+// finish (a ticket counter kept in loads[0], zeroed with counts before the launch and
+// overwritten by the result) computes the rank loads under the expert->rank map and
+// maxvio = (R*max - A)/A, balancedness = A/(R*max) from exact integers, one fp64 rounding
+// each.
+__global__ void __launch_bounds__(512) hist_kernel(const int32_t* __restrict__ idx, int T, int k,
+                                                   int E, int R, int tokens_per_block,
+                                                   const int32_t* __restrict__ map,
+                                                   int32_t* __restrict__ counts,
+                                                   int32_t* __restrict__ loads,
+                                                   double* __restrict__ maxvio,
+                                                   double* __restrict__ bal,
+                                                   int32_t* __restrict__ err) {
+  extern __shared__ int s_hist[];  // [max(E, R)]
+  __shared__ int s_err, s_last, s_max[32];
   if (block_should_stop(err)) return;
   for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
   if (threadIdx.x == 0) s_err = 0;
@@ -126,39 +136,35 @@ __global__ void __launch_bounds__(512) hist_count_kernel(const int32_t* __restri
   for (int e = threadIdx.x; e < E; e += blockDim.x)
     if (s_hist[e]) atomicAdd(counts + e, s_hist[e]);
   if (threadIdx.x == 0 && s_err) atomicOr(err, s_err);
-}
-
-// Rank loads under the expert->rank map, then maxvio = (R*max - A)/A and balancedness
-// = A/(R*max) from exact integers with one fp64 rounding each.
-__global__ void __launch_bounds__(1024) hist_finalize_kernel(
-    const int32_t* __restrict__ counts, int T, int k, int E, int R,
-    const int32_t* __restrict__ map, int32_t* __restrict__ loads, double* __restrict__ maxvio,
-    double* __restrict__ bal, int32_t* __restrict__ err) {
-  extern __shared__ int s_load[];
-  __shared__ int s_max[32];
-  __shared__ int s_bad;
-  if (block_should_stop(err)) return;
-  const int B = E / R;
-  for (int r = threadIdx.x; r < R; r += blockDim.x) s_load[r] = 0;
-  if (threadIdx.x == 0) s_bad = 0;
+  // last block: every other block's counts are visible once its ticket is
+  __threadfence();
   __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(loads, 1) == (int)gridDim.x - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const int B = E / R;
+  for (int r = threadIdx.x; r < R; r += blockDim.x) s_hist[r] = 0;
+  __syncthreads();
+  int bad = 0;
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     const int r = map ? __ldg(map + e) : e / B;
     if (r < 0 || r >= R) {
-      s_bad = 1;
+      bad = 1;
     } else {
-      const int c = __ldg(counts + e);
-      if (c) atomicAdd(&s_load[r], c);
+      const int c = __ldcg(counts + e);
+      if (c) atomicAdd(&s_hist[r], c);
     }
   }
+  if (bad) atomicOr(err, MOE_DERR_ID_RANGE);
   __syncthreads();
   int mx = 0;
   for (int r = threadIdx.x; r < R; r += blockDim.x) {
-    loads[r] = s_load[r];
-    mx = max(mx, s_load[r]);
+    loads[r] = s_hist[r];
+    mx = max(mx, s_hist[r]);
   }
   mx = __reduce_max_sync(MOE_FULL_MASK, mx);
-  if ((threadIdx.x & 31) == 0) s_max[threadIdx.x >> 5] = mx;
+  if (lane == 0) s_max[threadIdx.x >> 5] = mx;
   __syncthreads();
   if (threadIdx.x < 32) {
     const int nw = (blockDim.x + 31) >> 5;
@@ -174,7 +180,6 @@ __global__ void __launch_bounds__(1024) hist_finalize_kernel(
         *maxvio = (double)(top - A) / (double)A;
         *bal = (double)A / (double)top;
       }
-      if (s_bad) atomicOr(err, MOE_DERR_ID_RANGE);
     }
   }
 }
@@ -201,19 +206,18 @@ int launch_topk(const float* logits, int T, int E, int k, int32_t* idx, float* g
 int launch_histogram(const int32_t* idx, int T, int k, int E, int R, const int32_t* map,
                      int32_t* counts, int32_t* loads, double* maxvio, double* bal,
                      int32_t* err, cudaStream_t s) {
-  if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, s) != cudaSuccess) return MOE_ERR_LAUNCH;
-  if (T > 0) {
-    const int threads = 512;
-    // about two blocks per SM, each over a contiguous token range
-    int blocks = 2 * num_sms();
-    int per = (T + blocks - 1) / blocks;
-    per = ((per + 31) / 32) * 32;
-    blocks = (T + per - 1) / per;
-    hist_count_kernel<<<blocks, threads, sizeof(int) * E, s>>>(idx, T, k, E, per, counts, err);
-    if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
-  }
-  hist_finalize_kernel<<<1, 1024, sizeof(int) * R, s>>>(counts, T, k, E, R, map, loads, maxvio,
-                                                       bal, err);
+  if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, s) != cudaSuccess ||
+      cudaMemsetAsync(loads, 0, sizeof(int32_t), s) != cudaSuccess)
+    return MOE_ERR_LAUNCH;
+  const int threads = 512;
+  // about two blocks per SM, each over a contiguous token range (one block when T == 0)
+  int blocks = 2 * num_sms();
+  int per = (T + blocks - 1) / blocks;
+  per = ((per + 31) / 32) * 32;
+  if (per == 0) per = 32;
+  blocks = T > 0 ? (T + per - 1) / per : 1;
+  const size_t smem = sizeof(int) * (size_t)(E > R ? E : R);
+  hist_kernel<<<blocks, threads, smem, s>>>(idx, T, k, E, R, per, map, counts, loads, maxvio, bal, err);
   return launch_status();
 }
 
