@@ -201,7 +201,6 @@ __global__ void __launch_bounds__(kRowThreads) scatter_rows_kernel(
 }
 
 // ----------------------------------------------------------------------------- combine
-constexpr int kCombVec = 2;
 
 __device__ __forceinline__ void acc_bf16x8(float* acc, const uint4& v, float g) {
   const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
@@ -222,9 +221,11 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float* a) {
 }
 
 // out[t] = sum_j gate[t,j] * y[perm[t,j]], fp32 in j order, one warp per token.  With the
-// top-k known at compile time (K > 0) all K x kCombVec gathers of a lane are issued before
-// the first FMA; K == 0 is the generic loop.
-template <int K>
+// top-k known at compile time (K > 0) all K x V gathers of a lane are issued before the
+// first FMA; K == 0 is the generic loop.  V (16-byte vectors per lane and gather) is 1
+// for K > 4 so that the kernel stays near 40 registers and enough warps are resident
+// to keep the gathers in flight.
+template <int K, int kCombVec = (K > 4 || K == 0) ? 1 : 2>
 __global__ void __launch_bounds__(kRowThreads) combine_kernel(
     const uint4* __restrict__ y, const int32_t* __restrict__ perm,
     const float* __restrict__ gate, int T, int k, int dv, uint4* __restrict__ out,
