@@ -39,14 +39,19 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) per call of the dominant call (both grouped-FFN kernels) from
 # an ncu capture (profiles/ffn_kernel_near_balanced.md), keyed by workload and kernel
 # sources hash: it reads null as soon as the kernel sources change.
-TRAFFIC = {"near_balanced:a7c69c6f0c5cd3c4": int((946.614784 + 64.048384 + 478.843648 + 85.731584) * 1e6)}
+TRAFFIC = {"near_balanced:cf03cde59b9c0240": int((946.614784 + 64.048384 + 478.843648 + 85.731584) * 1e6)}
 
 
 def sources_hash() -> str:
+    """Hash of the grouped-FFN kernel's device code: grouped_ffn.cu and the device-side
+    helpers of common.cuh (host declarations there do not change the kernel)."""
     h = hashlib.sha256()
-    for f in ("grouped_ffn.cu", "common.cuh"):
-        with open(os.path.join(ROOT, "load_balanced_dispatch_warp_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+    csrc = os.path.join(ROOT, "load_balanced_dispatch_warp_b200", "csrc")
+    with open(os.path.join(csrc, "grouped_ffn.cu"), "rb") as fh:
+        h.update(fh.read())
+    with open(os.path.join(csrc, "common.cuh"), "rb") as fh:
+        text = fh.read()
+    h.update(text[text.index(b"device side"):])
     return h.hexdigest()[:16]
 
 

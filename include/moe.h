@@ -108,6 +108,20 @@ int moe_topk(const float* logits, int T, int E, int k,
              int32_t* idx, float* gate, int32_t* err, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * Router variant: bias-only balancing.   "MoE load balancing: 90/10 routing in
+ * production" (interview page): DeepSeek-V3 balances with a per-expert bias kept outside
+ * the gradient path, which moves the selection without distorting the gate.  The k
+ * experts are chosen by the biased score s_e = logit_e + bias_e (one fp32 addition,
+ * round-to-nearest), descending, equal scores by the lower expert id; the gates are the
+ * softmax over the chosen experts' UNBIASED logits, in the chosen order.
+ *   bias [E] fp32  per-expert selection bias (device).
+ *   other arguments, outputs and err as moe_topk (a non-finite bias also sets
+ *   MOE_DERR_NONFINITE).
+ */
+int moe_topk_biased(const float* logits, const float* bias, int T, int E, int k, int32_t* idx,
+                    float* gate, int32_t* err, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
  * Demand histogram and imbalance.   [Hotspots] "Separate expert demand from rank
  * placement": count assignments per expert, then sum over an expert->rank mapping;
  * balancedness = mean/max.  [MoonEP] para. 2: maxvio is 0 when perfectly balanced,
@@ -126,6 +140,22 @@ int moe_histogram_maxvio(const int32_t* idx, int T, int k, int E, int R,
                          const int32_t* expert_to_rank, int32_t* counts, int32_t* loads,
                          double* maxvio, double* balancedness, int32_t* err,
                          moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * Fixed-capacity ledger.   [Hotspots] "Make expert capacity, overflow, and padding
+ * explicit": per-expert capacity cap = ceil(A / E * cf), A = T*k assignments, with the
+ * capacity factor given as the exact rational cf_num / cf_den (5/4 in the pages' example,
+ * cap 5 for 32 assignments over 8 experts).  Per expert: processed = min(count, cap),
+ * overflow = max(count - cap, 0), padding = max(cap - count, 0).  The ledger reports a
+ * capacity mode; the layer path itself is dropless (no assignment is discarded).
+ *   counts    [E] int32        expert demand (from moe_histogram_maxvio).
+ *   processed, overflow, padding [E] int32 (out).
+ *   totals    [4] int32 (out)  {cap, sum processed, sum overflow, sum padding}.
+ *   err       no-op when non-zero.
+ */
+int moe_capacity_ledger(const int32_t* counts, int T, int k, int E, int cf_num, int cf_den,
+                        int32_t* processed, int32_t* overflow, int32_t* padding,
+                        int32_t* totals, const int32_t* err, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
  * Equal-load plan with redundant expert copies.   [MoonEP] para. 3-4: every rank

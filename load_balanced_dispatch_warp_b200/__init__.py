@@ -24,6 +24,7 @@ DERR_NONFINITE, DERR_ID_RANGE, DERR_DUPLICATE, DERR_SLOTS, DERR_TIMEOUT = 1, 2, 
 
 ENTRY_POINTS = ("moe_topk", "moe_histogram_maxvio", "moe_plan_balanced", "moe_prefetch_replicas",
                 "moe_dispatch", "moe_grouped_ffn", "moe_combine")
+VARIANTS = ("moe_topk_biased", "moe_capacity_ledger")
 HELPERS = ("moe_plan_get_layout", "moe_dispatch_workspace_words", "moe_status_string")
 
 
@@ -59,6 +60,8 @@ def lib() -> ctypes.CDLL:
             "moe_dispatch": [P, P, P, I, I, I, I, I, I, P, P, P, P, P, P],
             "moe_grouped_ffn": [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, P],
             "moe_combine": [P, P, P, I, I, I, P, P, P],
+            "moe_topk_biased": [P, P, I, I, I, P, P, P, P],
+            "moe_capacity_ledger": [P, I, I, I, I, I, P, P, P, P, P, P],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -114,6 +117,23 @@ def moe_topk(logits, k, idx, gate, err, stream=None):
     _check(lib().moe_topk(_ptr(logits, torch.float32, "logits"), T, E, k,
                           _ptr(idx, torch.int32, "idx"), _ptr(gate, torch.float32, "gate"),
                           _ptr(err, torch.int32, "err"), _stream(stream)), "moe_topk")
+
+
+def moe_topk_biased(logits, bias, k, idx, gate, err, stream=None):
+    T, E = logits.shape
+    _check(lib().moe_topk_biased(_ptr(logits, torch.float32, "logits"), _ptr(bias, torch.float32, "bias"),
+                                 T, E, k, _ptr(idx, torch.int32, "idx"), _ptr(gate, torch.float32, "gate"),
+                                 _ptr(err, torch.int32, "err"), _stream(stream)), "moe_topk_biased")
+
+
+def moe_capacity_ledger(counts, T, k, cf_num, cf_den, processed, overflow, padding, totals, err,
+                        stream=None):
+    E = counts.shape[0]
+    i32 = torch.int32
+    _check(lib().moe_capacity_ledger(
+        _ptr(counts, i32, "counts"), T, k, E, cf_num, cf_den, _ptr(processed, i32, "processed"),
+        _ptr(overflow, i32, "overflow"), _ptr(padding, i32, "padding"), _ptr(totals, i32, "totals"),
+        _ptr(err, i32, "err"), _stream(stream)), "moe_capacity_ledger")
 
 
 def moe_histogram_maxvio(idx, E, R, counts, loads, maxvio, balancedness, err,

@@ -111,6 +111,27 @@ int moe_topk(const float* logits, int T, int E, int k, int32_t* idx, float* gate
   return moe::launch_topk(logits, T, E, k, idx, gate, err, as_stream(stream));
 }
 
+int moe_topk_biased(const float* logits, const float* bias, int T, int E, int k, int32_t* idx,
+                    float* gate, int32_t* err, moe_stream_t stream) {
+  if (!err || !bias || (T > 0 && (!logits || !idx || !gate))) return MOE_ERR_ARG;
+  MOE_TRY(check_route(T, E, k));
+  return moe::launch_topk_biased(logits, bias, T, E, k, idx, gate, err, as_stream(stream));
+}
+
+int moe_capacity_ledger(const int32_t* counts, int T, int k, int E, int cf_num, int cf_den,
+                        int32_t* processed, int32_t* overflow, int32_t* padding,
+                        int32_t* totals, const int32_t* err, moe_stream_t stream) {
+  if (!counts || !processed || !overflow || !padding || !totals || !err) return MOE_ERR_ARG;
+  if (cf_num < 1 || cf_den < 1) return MOE_ERR_ARG;
+  MOE_TRY(check_route(T, E, 1));
+  if (k < 1 || k > E) return MOE_ERR_SHAPE;
+  const long long A = (long long)T * k;
+  if ((A * cf_num + (long long)E * cf_den) / ((long long)E * cf_den) >= ((long long)1 << 31))
+    return MOE_ERR_SHAPE;
+  return moe::launch_capacity(counts, E, A, cf_num, cf_den, processed, overflow, padding, totals,
+                              err, as_stream(stream));
+}
+
 int moe_histogram_maxvio(const int32_t* idx, int T, int k, int E, int R,
                          const int32_t* expert_to_rank, int32_t* counts, int32_t* loads,
                          double* maxvio, double* balancedness, int32_t* err,

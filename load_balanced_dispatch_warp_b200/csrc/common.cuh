@@ -25,6 +25,11 @@ int num_sms();  // SM count of the current device (cached per device)
 // --------------------------------------------------------------- launchers (one per step)
 int launch_topk(const float* logits, int T, int E, int k, int32_t* idx, float* gate,
                 int32_t* err, cudaStream_t s);
+int launch_topk_biased(const float* logits, const float* bias, int T, int E, int k,
+                       int32_t* idx, float* gate, int32_t* err, cudaStream_t s);
+int launch_capacity(const int32_t* counts, int E, long long A, int cf_num, int cf_den,
+                    int32_t* processed, int32_t* overflow, int32_t* padding, int32_t* totals,
+                    const int32_t* err, cudaStream_t s);
 int launch_histogram(const int32_t* idx, int T, int k, int E, int R, const int32_t* map,
                      int32_t* counts, int32_t* loads, double* maxvio, double* bal,
                      int32_t* err, cudaStream_t s);

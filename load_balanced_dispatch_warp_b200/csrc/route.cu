@@ -28,8 +28,11 @@ __device__ __forceinline__ float key_value(uint32_t key) {
 // finite float, so each of the k rounds is a plain max over the lane's keys, a warp-wide
 // max key (redux.sync), the lowest expert id among the lanes holding it (redux.sync), and
 // the winner zeroes that key.  Instruction count, not memory, bounds this kernel.
-template <int VPL>
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T,
+// BIASED: keys are built from logit + bias[e] (one fp32 add), the gates from the chosen
+// experts' unbiased logits (bias-only balancing).
+template <int VPL, bool BIASED>
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits,
+                                                   const float* __restrict__ bias, int T,
                                                    int E, int k, int32_t* __restrict__ idx,
                                                    float* __restrict__ gate,
                                                    int32_t* __restrict__ err) {
@@ -38,6 +41,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   if (t >= T) return;
   const float* row = logits + t * E;
   uint32_t key[VPL];
+  float raw[BIASED ? VPL : 1];
   bool bad = false;
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
@@ -46,7 +50,14 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
     if (e < E) {
       const float v = __ldcs(row + e);
       bad |= !isfinite(v);
-      kv = order_key(v);
+      if (BIASED) {
+        const float b = __ldg(bias + e);
+        bad |= !isfinite(b);
+        raw[i] = v;
+        kv = order_key(__fadd_rn(v, b));
+      } else {
+        kv = order_key(v);
+      }
     }
     key[i] = kv;
   }
@@ -71,19 +82,82 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
     const uint32_t wid = __reduce_min_sync(MOE_FULL_MASK, cand);
     const bool mine = (int)(wid & 31u) == lane;
     const int wi = (int)(wid >> 5);
+    float sel = 0.f;
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) key[i] = (mine && i == wi) ? 0u : key[i];
+    for (int i = 0; i < VPL; ++i) {
+      if (BIASED && i == wi) sel = raw[i];
+      key[i] = (mine && i == wi) ? 0u : key[i];
+    }
+    if (BIASED) sel = __shfl_sync(MOE_FULL_MASK, sel, (int)(wid & 31u));
     if (lane == j) {
-      my_val = key_value(wmax);
+      my_val = BIASED ? sel : key_value(wmax);
       my_id = (int)wid;
     }
   }
-  const float top = __shfl_sync(MOE_FULL_MASK, my_val, 0);
+  // softmax over the chosen (unbiased) logits
+  float top = lane < k ? my_val : -INFINITY;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) top = fmaxf(top, __shfl_xor_sync(MOE_FULL_MASK, top, o));
   const float ex = lane < k ? expf(my_val - top) : 0.f;
   const float sum = warp_sum(ex);
   if (lane < k) {
     idx[t * k + lane] = my_id;
     gate[t * k + lane] = ex / sum;
+  }
+}
+
+// Fixed-capacity ledger of "MoE Load Balancing: Find Expert Hotspots" ("Make expert
+// capacity, overflow, and padding explicit"): cap = ceil(A * cf / E) with the capacity
+// factor an exact rational cf_num / cf_den; per expert processed = min(count, cap),
+// overflow = max(count - cap, 0), padding = max(cap - count, 0); totals =
+// {cap, sum processed, sum overflow, sum padding}.  One CTA, integer arithmetic.
+__global__ void __launch_bounds__(256) capacity_kernel(const int32_t* __restrict__ counts, int E,
+                                                       long long A, int cf_num, int cf_den,
+                                                       int32_t* __restrict__ processed,
+                                                       int32_t* __restrict__ overflow,
+                                                       int32_t* __restrict__ padding,
+                                                       int32_t* __restrict__ totals,
+                                                       const int32_t* __restrict__ err) {
+  __shared__ long long s_sum[3][8];
+  if (block_should_stop(err)) return;
+  const long long num = A * cf_num, den = (long long)E * cf_den;
+  const long long cap = (num + den - 1) / den;
+  long long sp = 0, so = 0, sd = 0;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const long long c = counts[e];
+    const long long p = c < cap ? c : cap;
+    const long long o = c > cap ? c - cap : 0;
+    const long long d = cap > c ? cap - c : 0;
+    processed[e] = (int32_t)p;
+    overflow[e] = (int32_t)o;
+    padding[e] = (int32_t)d;
+    sp += p;
+    so += o;
+    sd += d;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sp += __shfl_xor_sync(MOE_FULL_MASK, sp, o);
+    so += __shfl_xor_sync(MOE_FULL_MASK, so, o);
+    sd += __shfl_xor_sync(MOE_FULL_MASK, sd, o);
+  }
+  if ((threadIdx.x & 31) == 0) {
+    s_sum[0][threadIdx.x >> 5] = sp;
+    s_sum[1][threadIdx.x >> 5] = so;
+    s_sum[2][threadIdx.x >> 5] = sd;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    long long a = 0, b = 0, c = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+      a += s_sum[0][w];
+      b += s_sum[1][w];
+      c += s_sum[2][w];
+    }
+    totals[0] = (int32_t)cap;
+    totals[1] = (int32_t)a;
+    totals[2] = (int32_t)b;
+    totals[3] = (int32_t)c;
   }
 }
 
@@ -192,7 +266,7 @@ int launch_topk(const float* logits, int T, int E, int k, int32_t* idx, float* g
   if (T == 0) return MOE_OK;
   const int threads = 256, per_block = threads / 32;
   const unsigned grid = (unsigned)((T + per_block - 1) / per_block);
-#define MOE_TOPK_CASE(V) topk_kernel<V><<<grid, threads, 0, s>>>(logits, T, E, k, idx, gate, err)
+#define MOE_TOPK_CASE(V) topk_kernel<V, false><<<grid, threads, 0, s>>>(logits, nullptr, T, E, k, idx, gate, err)
   if (E <= 32) MOE_TOPK_CASE(1);
   else if (E <= 64) MOE_TOPK_CASE(2);
   else if (E <= 128) MOE_TOPK_CASE(4);
@@ -200,6 +274,31 @@ int launch_topk(const float* logits, int T, int E, int k, int32_t* idx, float* g
   else if (E <= 512) MOE_TOPK_CASE(16);
   else MOE_TOPK_CASE(32);
 #undef MOE_TOPK_CASE
+  return launch_status();
+}
+
+int launch_topk_biased(const float* logits, const float* bias, int T, int E, int k,
+                       int32_t* idx, float* gate, int32_t* err, cudaStream_t s) {
+  if (cudaMemsetAsync(err, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_LAUNCH;
+  if (T == 0) return MOE_OK;
+  const int threads = 256, per_block = threads / 32;
+  const unsigned grid = (unsigned)((T + per_block - 1) / per_block);
+#define MOE_TOPKB_CASE(V) topk_kernel<V, true><<<grid, threads, 0, s>>>(logits, bias, T, E, k, idx, gate, err)
+  if (E <= 32) MOE_TOPKB_CASE(1);
+  else if (E <= 64) MOE_TOPKB_CASE(2);
+  else if (E <= 128) MOE_TOPKB_CASE(4);
+  else if (E <= 256) MOE_TOPKB_CASE(8);
+  else if (E <= 512) MOE_TOPKB_CASE(16);
+  else MOE_TOPKB_CASE(32);
+#undef MOE_TOPKB_CASE
+  return launch_status();
+}
+
+int launch_capacity(const int32_t* counts, int E, long long A, int cf_num, int cf_den,
+                    int32_t* processed, int32_t* overflow, int32_t* padding, int32_t* totals,
+                    const int32_t* err, cudaStream_t s) {
+  capacity_kernel<<<1, 256, 0, s>>>(counts, E, A, cf_num, cf_den, processed, overflow, padding,
+                                    totals, err);
   return launch_status();
 }
 

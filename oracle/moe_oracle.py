@@ -24,6 +24,8 @@ floating point, citing the page passage it follows.  Sources (page title, sectio
 Pins (tests/test_oracle_pins.py checks each against something other than this file):
   topk_route        brute-force rank counting on tiny inputs; k=1 / k=E special cases;
                     softmax closed forms (k=2 sigmoid, equal logits -> 1/k)
+  topk_route_biased zero bias reduces to topk_route; a large bias forces a chosen set;
+                    the gates ignore the bias (closed form for k=2)
   expert_histogram  the pages' worked fixture (demand, both rank mappings, 4/9, 8/15, 0.8)
   capacity_ledger   the pages' worked fixture (cap 5, processed/overflow/padding)
   remote_routes     the pages' worked fixture (22 vs 25 of 32)
@@ -83,6 +85,40 @@ def topk_route(logits: np.ndarray, k: int):
         idx[t] = order
         sel = row[order]
         ex = np.exp(sel - sel[0])
+        gate[t] = ex / ex.sum()
+    return idx, gate, err
+
+
+def topk_route_biased(logits: np.ndarray, bias: np.ndarray, k: int):
+    """Bias-only balancing ("Your MoE router sends 90% of tokens to 10% of the experts":
+    a per-expert bias outside the gradient path, as DeepSeek-V3 used, balances the load
+    without distorting the gate).  The experts are chosen by the top-k of the biased
+    scores s_e = logit_e + bias_e -- the sum taken in fp32, the precision the kernel
+    decides in -- ordered by s descending, ties by the lower expert id; the gate of each
+    chosen expert is the softmax over the chosen experts' UNBIASED logits, in the chosen
+    order, in fp64.  A non-finite logit or bias sets error bit 1.
+
+    Returns idx [T,k] int32, gate [T,k] float64, err int.
+    """
+    logits = np.asarray(logits, dtype=np.float32)
+    bias = np.asarray(bias, dtype=np.float32)
+    T, E = logits.shape
+    if not (1 <= k <= E):
+        raise ValueError("need 1 <= k <= E")
+    err = 0
+    if not (np.all(np.isfinite(logits)) and np.all(np.isfinite(bias))):
+        err |= ERR_NONFINITE
+    idx = np.zeros((T, k), dtype=np.int32)
+    gate = np.zeros((T, k), dtype=np.float64)
+    for t in range(T):
+        if not (np.all(np.isfinite(logits[t])) and np.all(np.isfinite(bias))):
+            continue
+        scores = (logits[t] + bias).astype(np.float32)  # fp32 sum, elementwise
+        order = np.argsort(-scores.astype(np.float64), kind="stable")[:k]
+        idx[t] = order
+        sel = logits[t][order].astype(np.float64)
+        m = sel.max()
+        ex = np.exp(sel - m)
         gate[t] = ex / ex.sum()
     return idx, gate, err
 

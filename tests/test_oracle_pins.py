@@ -373,3 +373,30 @@ def test_layer_identity_experts_returns_x():
     assert res["err"] == 0
     ref = O.silu(x) * x      # every expert computes silu(x)*x, gates sum to one
     assert np.allclose(res["out"], ref, atol=1e-13, rtol=0)
+
+
+# ----------------------------------------------------------- bias-only selection
+def test_biased_topk_pins():
+    rng = np.random.default_rng(20)
+    logits = rng.standard_normal((40, 12)).astype(np.float32)
+    # zero bias is plain top-k
+    i0, g0, _ = O.topk_route(logits, 3)
+    i1, g1, _ = O.topk_route_biased(logits, np.zeros(12, np.float32), 3)
+    assert (i0 == i1).all() and np.array_equal(g0, g1)
+    # a large bias on experts {2, 7} forces them into every token's choice
+    bias = np.zeros(12, np.float32)
+    bias[[2, 7]] = 100.0
+    idx, gate, err = O.topk_route_biased(logits, bias, 2)
+    assert err == 0
+    for t in range(40):
+        assert sorted(idx[t]) == [2, 7]
+        # the gate ignores the bias: softmax of the two unbiased logits, in chosen order
+        a, b = float(logits[t, idx[t, 0]]), float(logits[t, idx[t, 1]])
+        assert abs(gate[t, 0] - 1.0 / (1.0 + math.exp(b - a))) < 1e-15
+    # order follows the biased score: 7 leads where logit7 + 100 > logit2 + 100
+    for t in range(40):
+        first = 7 if np.float32(logits[t, 7] + np.float32(100)) > np.float32(logits[t, 2] + np.float32(100)) else 2
+        assert idx[t, 0] == first or logits[t, 7] + 100 == logits[t, 2] + 100
+    bad = bias.copy()
+    bad[3] = np.nan
+    assert O.topk_route_biased(logits, bad, 2)[2] == O.ERR_NONFINITE
