@@ -271,6 +271,15 @@ int moe_dispatch_noalloc(const moe_bf16* x, const int32_t* idx, const int32_t* p
 int moe_combine(const moe_bf16* y, const int32_t* perm, const float* gate, int T, int k,
                 int d, moe_bf16* out, const int32_t* err, moe_stream_t stream);
 
+/* ---------------------------------------------------------------------------------
+ * Diagnostic (no counterpart in the pages): runs the grouped FFN's bounded mbarrier wait
+ * on a barrier that nothing ever arrives at, with a limit of `limit_us` microseconds
+ * (1 .. 10^7).  The wait gives up, ORs MOE_DERR_TIMEOUT into *err and the kernel returns;
+ * the CUDA context stays usable.  Lets a caller check the timeout path without faulting or
+ * hanging a GPU.
+ */
+int moe_selftest_bounded_wait(int32_t* err, int limit_us, moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

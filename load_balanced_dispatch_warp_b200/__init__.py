@@ -62,6 +62,7 @@ def lib() -> ctypes.CDLL:
             "moe_combine": [P, P, P, I, I, I, P, P, P],
             "moe_topk_biased": [P, P, I, I, I, P, P, P, P],
             "moe_capacity_ledger": [P, I, I, I, I, I, P, P, P, P, P, P],
+            "moe_selftest_bounded_wait": [P, I, P],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -134,6 +135,12 @@ def moe_capacity_ledger(counts, T, k, cf_num, cf_den, processed, overflow, paddi
         _ptr(counts, i32, "counts"), T, k, E, cf_num, cf_den, _ptr(processed, i32, "processed"),
         _ptr(overflow, i32, "overflow"), _ptr(padding, i32, "padding"), _ptr(totals, i32, "totals"),
         _ptr(err, i32, "err"), _stream(stream)), "moe_capacity_ledger")
+
+
+def moe_selftest_bounded_wait(err, limit_us=50000, stream=None):
+    """Run the FFN's bounded wait on a barrier nothing arrives at (sets DERR_TIMEOUT)."""
+    _check(lib().moe_selftest_bounded_wait(_ptr(err, torch.int32, "err"), int(limit_us), _stream(stream)),
+           "moe_selftest_bounded_wait")
 
 
 def moe_histogram_maxvio(idx, E, R, counts, loads, maxvio, balancedness, err,

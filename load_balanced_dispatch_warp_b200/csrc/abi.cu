@@ -236,4 +236,9 @@ int moe_combine(const moe_bf16* y, const int32_t* perm, const float* gate, int T
                              reinterpret_cast<__nv_bfloat16*>(out), err, as_stream(stream));
 }
 
+int moe_selftest_bounded_wait(int32_t* err, int limit_us, moe_stream_t stream) {
+  if (!err || limit_us < 1 || limit_us > 10000000) return MOE_ERR_ARG;
+  return moe::launch_bounded_wait_selftest(err, limit_us, as_stream(stream));
+}
+
 }  // extern "C"

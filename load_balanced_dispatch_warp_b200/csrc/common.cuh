@@ -49,6 +49,7 @@ int launch_grouped_ffn(const __nv_bfloat16* recv, const int32_t* plan,
                        const __nv_bfloat16* P3, const __half* P2, int T, int k, int E, int R,
                        int S, int d, int F, __half* h, __nv_bfloat16* y, int32_t* err,
                        cudaStream_t s);
+int launch_bounded_wait_selftest(int32_t* err, int limit_us, cudaStream_t s);
 int launch_combine(const __nv_bfloat16* y, const int32_t* perm, const float* gate, int T,
                    int k, int d, __nv_bfloat16* out, const int32_t* err, cudaStream_t s);
 

@@ -98,7 +98,7 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
 // Bounded wait for the phase of `parity` to complete.  Returns false (and raises the
 // abort flag and the error bit) if the bound runs out, or if another role aborted.
 __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                       int32_t* err) {
+                                       int32_t* err, uint64_t limit_ns = WAIT_LIMIT_NS) {
   if (mbar_try(bar, parity)) return true;
   uint64_t t0 = 0;
   for (uint32_t it = 1;; ++it) {
@@ -108,7 +108,7 @@ __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile i
       const uint64_t now = globaltimer();
       if (t0 == 0) {
         t0 = now;
-      } else if (now - t0 > WAIT_LIMIT_NS) {
+      } else if (now - t0 > limit_ns) {
         *abort_flag = 1;
         atomicOr(err, MOE_DERR_TIMEOUT);
         return false;
@@ -431,6 +431,19 @@ __global__ void __launch_bounds__(FFN_THREADS, 1)
   }
 }
 
+// Self-test of the bounded wait: one thread waits on an mbarrier that nothing arrives at,
+// with a short limit; the wait gives up, sets MOE_DERR_TIMEOUT and the kernel returns.
+__global__ void bounded_wait_selftest_kernel(int32_t* err, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    mbar_wait(smem_u32(&bar), 0, &abort_flag, err, limit_ns);
+  }
+}
+
 // ----------------------------------------------------------------------------- host side
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -489,6 +502,11 @@ int launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b
 }
 
 }  // namespace
+
+int launch_bounded_wait_selftest(int32_t* err, int limit_us, cudaStream_t s) {
+  bounded_wait_selftest_kernel<<<1, 32, 0, s>>>(err, (uint64_t)limit_us * 1000ull);
+  return launch_status();
+}
 
 int launch_grouped_ffn(const __nv_bfloat16* recv, const int32_t* plan,
                        const moe_plan_layout& L, const __nv_bfloat16* W1,

@@ -236,40 +236,50 @@ __global__ void __launch_bounds__(kRowThreads) combine_kernel(
   for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += nwarps) {
     const int r = lane < k ? __ldg(perm + t * k + lane) : 0;
     const float gl = lane < k ? __ldg(gate + t * k + lane) : 0.f;
-    for (int v0 = lane; v0 < dv; v0 += 32 * kCombVec) {
-      float acc[kCombVec][8];
+    if (K > 0) {
+      // rows and gates of the token broadcast once; the vector loop has no warp collective
+      int rows[K > 0 ? K : 1];
+      float g[K > 0 ? K : 1];
 #pragma unroll
-      for (int u = 0; u < kCombVec; ++u)
+      for (int j = 0; j < K; ++j) {
+        rows[j] = __shfl_sync(MOE_FULL_MASK, r, j);
+        g[j] = __shfl_sync(MOE_FULL_MASK, gl, j);
+      }
+      for (int v0 = lane; v0 < dv; v0 += 32 * kCombVec) {
+        float acc[kCombVec][8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
-      if (K > 0) {
+        for (int u = 0; u < kCombVec; ++u)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
         uint4 buf[K > 0 ? K : 1][kCombVec];
 #pragma unroll
-        for (int j = 0; j < K; ++j) {
-          const uint4* yr = y + (int64_t)__shfl_sync(MOE_FULL_MASK, r, j) * dv;
+        for (int j = 0; j < K; ++j)
 #pragma unroll
           for (int u = 0; u < kCombVec; ++u)
-            if (v0 + u * 32 < dv) buf[j][u] = __ldcs(yr + v0 + u * 32);
-        }
+            if (v0 + u * 32 < dv) buf[j][u] = __ldcs(y + (int64_t)rows[j] * dv + v0 + u * 32);
 #pragma unroll
-        for (int j = 0; j < K; ++j) {
-          const float g = __shfl_sync(MOE_FULL_MASK, gl, j);
+        for (int j = 0; j < K; ++j)
 #pragma unroll
           for (int u = 0; u < kCombVec; ++u)
-            if (v0 + u * 32 < dv) acc_bf16x8(acc[u], buf[j][u], g);
-        }
-      } else {
-        for (int j = 0; j < k; ++j) {
-          const uint4* yr = y + (int64_t)__shfl_sync(MOE_FULL_MASK, r, j) * dv;
-          const float g = __shfl_sync(MOE_FULL_MASK, gl, j);
+            if (v0 + u * 32 < dv) acc_bf16x8(acc[u], buf[j][u], g[j]);
 #pragma unroll
-          for (int u = 0; u < kCombVec; ++u)
-            if (v0 + u * 32 < dv) acc_bf16x8(acc[u], __ldcs(yr + v0 + u * 32), g);
-        }
+        for (int u = 0; u < kCombVec; ++u)
+          if (v0 + u * 32 < dv) out[t * dv + v0 + u * 32] = pack_bf16x8(acc[u]);
       }
+    } else {
+      // generic k: warp-uniform trip count (the shuffles need every lane), lane predicate
+      for (int base = 0; base < dv; base += 32) {
+        const int v = base + lane;
+        float acc[8];
 #pragma unroll
-      for (int u = 0; u < kCombVec; ++u)
-        if (v0 + u * 32 < dv) out[t * dv + v0 + u * 32] = pack_bf16x8(acc[u]);
+        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+        for (int j = 0; j < k; ++j) {
+          const int row = __shfl_sync(MOE_FULL_MASK, r, j);
+          const float gj = __shfl_sync(MOE_FULL_MASK, gl, j);
+          if (v < dv) acc_bf16x8(acc, __ldcs(y + (int64_t)row * dv + v), gj);
+        }
+        if (v < dv) out[t * dv + v] = pack_bf16x8(acc);
+      }
     }
   }
 }

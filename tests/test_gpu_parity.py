@@ -193,3 +193,36 @@ def test_topk_expert_counts(E):
     torch.cuda.synchronize()
     assert np.array_equal(idx.cpu().numpy(), idx_ref)
     assert np.abs(gate.cpu().double().numpy() - gate_ref).max() <= 1e-6
+
+
+def test_bounded_wait_gives_up_and_context_survives():
+    """The FFN's bounded mbarrier wait, on a barrier nothing arrives at, returns with the
+    timeout bit; the next layer on the same context still matches the oracle."""
+    import time
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    t0 = time.time()
+    M.moe_selftest_bounded_wait(err, limit_us=20000)
+    torch.cuda.synchronize()
+    assert err.item() == M.DERR_TIMEOUT
+    assert time.time() - t0 < 5.0
+    w = I.WORKLOADS["tiny"]
+    logits, x, weights = make_inputs(w)
+    ref = oracle_integer_path(w, logits)
+    L = run_gpu(w, logits, x, weights)
+    check_integer_parity(L, w, ref)
+    check_ffn_combine_full(L, w, x, weights, ref)
+
+
+def test_max_shapes():
+    """Limits of the boundary: E = 1024 experts, k = 32, R = 1024 ranks (B = 1), S = 3 slots
+    (R*(B+S) = 4096 group records), through the whole layer."""
+    w = I.small_workload("max", 1024, 1024, 32, 1024, 3, 128, 128, alpha=0.2, seed=13)
+    logits, x, weights = make_inputs(w)
+    ref = oracle_integer_path(w, logits)
+    L = run_gpu(w, logits, x, weights)
+    if ref["err"]:
+        assert int(L.err.item()) == ref["err"]
+        return
+    check_integer_parity(L, w, ref)
+    check_rows_and_pool(L, w, x, weights, ref)
+    check_ffn_combine_full(L, w, x, weights, ref)
