@@ -221,26 +221,39 @@ def run_ours(args, w: I.Workload, world, rank, local):
                 rec(e[i + 1], st)
         rec(end, st)
 
-    graph = None
+    # Two captures of the same K steps: a clean one (the timed headline) and one with an
+    # event-record node between consecutive calls (the per-call table, replayed right
+    # after, also K steps between barriers).
+    graph = graph_ev = None
     if not args.eager:
         rt = cudart()
-        graph = torch.cuda.CUDAGraph()
-        cap = torch.cuda.Stream(device)
-        cap.wait_stream(stream)
-        torch.cuda.synchronize()
 
         def rec_node(event, st):  # an event-record node inside the graph
             rc = rt.cudaEventRecordWithFlags(ctypes.c_void_p(event.cuda_event),
                                              ctypes.c_void_p(st.cuda_stream), 1)
             if rc != 0:
                 raise RuntimeError(f"cudaEventRecordWithFlags failed ({rc})")
-        with torch.cuda.stream(cap):
-            graph.capture_begin()
-            timed_steps(cap, rec_node)
-            graph.capture_end()
-        torch.cuda.synchronize()
-        graph.replay()  # one untimed replay (warm instantiation)
-        torch.cuda.synchronize()
+
+        def capture(with_events):
+            g = torch.cuda.CUDAGraph()
+            cap = torch.cuda.Stream(device)
+            cap.wait_stream(stream)
+            torch.cuda.synchronize()
+            with torch.cuda.stream(cap):
+                g.capture_begin()
+                if with_events:
+                    timed_steps(cap, rec_node)
+                else:
+                    for _ in range(args.steps):
+                        for f in steps:
+                            f()
+                g.capture_end()
+            torch.cuda.synchronize()
+            g.replay()  # one untimed replay (warm instantiation)
+            torch.cuda.synchronize()
+            return g
+        graph = capture(False)
+        graph_ev = capture(True)
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
@@ -248,18 +261,27 @@ def run_ours(args, w: I.Workload, world, rank, local):
     torch.cuda.synchronize()
     clocks.mark_start()
     if graph is not None:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
         graph.replay()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        elapsed_ms = t0.elapsed_time(t1)
+        graph_ev.replay()  # instrumented replay: per-call intervals
     else:
         timed_steps(stream, lambda e, st: e.record(st))
+        torch.cuda.synchronize()
+        elapsed_ms = start.elapsed_time(end)
     torch.cuda.synchronize()
     barrier(world)
     clocks.mark_end()
     clk = clocks.stop()
-    elapsed_ms = start.elapsed_time(end)
     elapsed_ms = max_over_ranks(elapsed_ms, world, device)
     if int(L.err.item()) != 0:
         raise RuntimeError(f"device error word {int(L.err.item())} in the timed region")
-    del graph
+    del graph, graph_ev
     per_call_ms = {c: sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(args.steps)) / args.steps
                    for i, c in enumerate(CALLS)}
 
@@ -325,7 +347,8 @@ def run_ours(args, w: I.Workload, world, rank, local):
                    "parallelism": f"replicas x{world} (ranks simulated in one GPU's HBM)",
                    "l2": "step working set (weights, pool, activations) far above the 126 MB L2",
                    "launch": "eager, one stream" if args.eager else
-                             "K steps captured in one CUDA graph, replayed once"},
+                             "K steps captured in one CUDA graph, replayed once; per-call "
+                             "intervals from a second replay with event nodes between calls"},
         "clocks": clk,
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT,
                 "h2d_bytes_per_step": w.T * w.E * 4 + w.T * w.d * 2,

@@ -24,31 +24,66 @@ __device__ __forceinline__ float key_value(uint32_t key) {
 }
 
 // One warp per token.  Lane l holds experts l, l+32, ... (VPL of them) as
-// order-preserving keys; pad entries (e >= E) and taken entries have key 0, below every
-// finite float, so each of the k rounds is a plain max over the lane's keys, a warp-wide
-// max key (redux.sync), the lowest expert id among the lanes holding it (redux.sync), and
-// the winner zeroes that key.  Instruction count, not memory, bounds this kernel.
-// BIASED: keys are built from logit + bias[e] (one fp32 add), the gates from the chosen
-// experts' unbiased logits (bias-only balancing).
-template <int VPL, bool BIASED>
+// order-preserving keys (pad entries e >= E: key 0, below every finite float).  Exact
+// top-k in three steps:
+//   1. tau = the k-th largest of the 32 lane maxima (k rounds of redux.sync over one
+//      value per lane).  At least k keys are >= tau, so every key of the top-k -- equal
+//      keys at the k-th place included -- is >= tau.
+//   2. The keys >= tau (usually close to k of them) are compacted to one per lane
+//      through shared memory.
+//   3. k rounds over one candidate per lane: warp max key (redux.sync), lowest expert id
+//      among its holders (redux.sync), the winner drops out.
+// More than 32 candidates (many equal keys) falls back to the same rounds over all of
+// the lane's keys.  BIASED: keys from logit + bias[e] (one fp32 add), gates from the
+// chosen experts' unbiased logits (bias-only balancing).
+// Expert held in slot i of a lane: lane + 32 i (scalar loads), or, with 16-byte loads
+// (VEC), 128 (i / 4) + 4 lane + i % 4.
+template <bool VEC>
+__device__ __forceinline__ int slot_id(int i, int lane) {
+  return VEC ? 128 * (i >> 2) + 4 * lane + (i & 3) : lane + 32 * i;
+}
+
+template <int VPL, bool BIASED, bool VEC>
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits,
                                                    const float* __restrict__ bias, int T,
                                                    int E, int k, int32_t* __restrict__ idx,
                                                    float* __restrict__ gate,
                                                    int32_t* __restrict__ err) {
-  const int lane = threadIdx.x & 31;
-  const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t >= T) return;
+  __shared__ uint32_t s_key[8][32];
+  __shared__ int s_id[8][32];
+  __shared__ float s_raw[8][BIASED ? 32 : 1];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + wib; t < T; t += nwarps) {
   const float* row = logits + t * E;
   uint32_t key[VPL];
   float raw[BIASED ? VPL : 1];
+  float val[VPL];
+  if (VEC) {
+#pragma unroll
+    for (int q = 0; q < VPL / 4; ++q) {
+      const int e0 = 128 * q + 4 * lane;
+      float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (e0 < E) v4 = __ldcs(reinterpret_cast<const float4*>(row + e0));
+      val[4 * q] = v4.x;
+      val[4 * q + 1] = v4.y;
+      val[4 * q + 2] = v4.z;
+      val[4 * q + 3] = v4.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int e = lane + 32 * i;
+      val[i] = e < E ? __ldcs(row + e) : 0.f;
+    }
+  }
   bool bad = false;
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
-    const int e = lane + 32 * i;
+    const int e = slot_id<VEC>(i, lane);
     uint32_t kv = 0;
     if (e < E) {
-      const float v = __ldcs(row + e);
+      const float v = val[i];
       bad |= !isfinite(v);
       if (BIASED) {
         const float b = __ldg(bias + e);
@@ -63,35 +98,95 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   }
   if (__any_sync(MOE_FULL_MASK, bad)) {
     if (lane == 0) atomicOr(err, MOE_DERR_NONFINITE);
-    return;
+    continue;
   }
+  // 1. threshold from the lane maxima
+  uint32_t lmax = key[0];
+#pragma unroll
+  for (int i = 1; i < VPL; ++i) lmax = max(lmax, key[i]);
+  uint32_t tau = 0, m = lmax;
+  for (int j = 0; j < k; ++j) {
+    tau = __reduce_max_sync(MOE_FULL_MASK, m);
+    const uint32_t holder = __reduce_min_sync(MOE_FULL_MASK, m == tau ? (uint32_t)lane : 32u);
+    if ((uint32_t)lane == holder) m = 0;
+  }
+  // 2. candidates: keys >= tau (tau > 0: pad keys never qualify)
+  int cnt = 0;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) cnt += key[i] >= tau;
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(MOE_FULL_MASK, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const int total = __shfl_sync(MOE_FULL_MASK, incl, 31);
   float my_val = 0.f;
   int my_id = 0;
-  for (int j = 0; j < k; ++j) {
-    // lane maximum; equal keys keep the lower slot (= lower expert id)
-    uint32_t best = key[0];
-    int best_i = 0;
-#pragma unroll
-    for (int i = 1; i < VPL; ++i) {
-      const bool gt = key[i] > best;
-      best = gt ? key[i] : best;
-      best_i = gt ? i : best_i;
-    }
-    const uint32_t wmax = __reduce_max_sync(MOE_FULL_MASK, best);
-    const uint32_t cand = best == wmax ? (uint32_t)(lane + 32 * best_i) : 0xffffffffu;
-    const uint32_t wid = __reduce_min_sync(MOE_FULL_MASK, cand);
-    const bool mine = (int)(wid & 31u) == lane;
-    const int wi = (int)(wid >> 5);
-    float sel = 0.f;
+  if (total <= 32) {
+    int pos = incl - cnt;
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
-      if (BIASED && i == wi) sel = raw[i];
-      key[i] = (mine && i == wi) ? 0u : key[i];
+      if (key[i] >= tau) {
+        s_key[wib][pos] = key[i];
+        s_id[wib][pos] = slot_id<VEC>(i, lane);
+        if (BIASED) s_raw[wib][pos] = raw[i];
+        ++pos;
+      }
     }
-    if (BIASED) sel = __shfl_sync(MOE_FULL_MASK, sel, (int)(wid & 31u));
-    if (lane == j) {
-      my_val = BIASED ? sel : key_value(wmax);
-      my_id = (int)wid;
+    __syncwarp();
+    uint32_t ck = lane < total ? s_key[wib][lane] : 0u;
+    const int cid = lane < total ? s_id[wib][lane] : 0;
+    const float craw = (BIASED && lane < total) ? s_raw[wib][BIASED ? lane : 0] : 0.f;
+    // 3. k rounds over one candidate per lane
+    for (int j = 0; j < k; ++j) {
+      const uint32_t wmax = __reduce_max_sync(MOE_FULL_MASK, ck);
+      const uint32_t wid =
+          __reduce_min_sync(MOE_FULL_MASK, (ck == wmax && lane < total) ? (uint32_t)cid : 0xffffffffu);
+      const bool mine = lane < total && (uint32_t)cid == wid;
+      if (BIASED) {
+        const uint32_t src = __reduce_min_sync(MOE_FULL_MASK, mine ? (uint32_t)lane : 32u);
+        const float sel = __shfl_sync(MOE_FULL_MASK, craw, (int)src);
+        if (lane == j) my_val = sel;
+      } else if (lane == j) {
+        my_val = key_value(wmax);
+      }
+      if (lane == j) my_id = (int)wid;
+      if (mine) ck = 0;
+    }
+  } else {
+    // many equal keys: rounds over all of the lane's keys
+    for (int j = 0; j < k; ++j) {
+      // lane's best: largest key, equal keys -> lowest expert id
+      uint32_t best = key[0];
+      int best_e = slot_id<VEC>(0, lane);
+#pragma unroll
+      for (int i = 1; i < VPL; ++i) {
+        const int e = slot_id<VEC>(i, lane);
+        const bool gt = key[i] > best || (key[i] == best && e < best_e);
+        best = gt ? key[i] : best;
+        best_e = gt ? e : best_e;
+      }
+      const uint32_t wmax = __reduce_max_sync(MOE_FULL_MASK, best);
+      const uint32_t cand = best == wmax ? (uint32_t)best_e : 0xffffffffu;
+      const uint32_t wid = __reduce_min_sync(MOE_FULL_MASK, cand);
+      float sel = 0.f;
+      bool mine = false;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const bool hit = slot_id<VEC>(i, lane) == (int)wid;
+        mine |= hit;
+        if (BIASED && hit) sel = raw[i];
+        key[i] = hit ? 0u : key[i];
+      }
+      if (BIASED) {
+        const uint32_t src = __reduce_min_sync(MOE_FULL_MASK, mine ? (uint32_t)lane : 32u);
+        sel = __shfl_sync(MOE_FULL_MASK, sel, (int)src);
+      }
+      if (lane == j) {
+        my_val = BIASED ? sel : key_value(wmax);
+        my_id = (int)wid;
+      }
     }
   }
   // softmax over the chosen (unbiased) logits
@@ -103,6 +198,8 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   if (lane < k) {
     idx[t * k + lane] = my_id;
     gate[t * k + lane] = ex / sum;
+  }
+  __syncwarp();  // the warp's candidate buffer is rewritten by its next token
   }
 }
 
@@ -258,40 +355,42 @@ __global__ void __launch_bounds__(512) hist_kernel(const int32_t* __restrict__ i
   }
 }
 
+// One warp per token over a persistent grid (8 warps per block, up to 8 blocks per SM);
+// 16-byte loads when every lane's slots come in aligned groups of four.
+int launch_topk_impl(const float* logits, const float* bias, int T, int E, int k,
+                     int32_t* idx, float* gate, int32_t* err, cudaStream_t s) {
+  const int threads = 256, per_block = threads / 32;
+  const int64_t want = ((int64_t)T + per_block - 1) / per_block;
+  const int64_t cap = (int64_t)num_sms() * 8;
+  const unsigned grid = (unsigned)(want < cap ? want : cap);
+  const bool vec = E % 4 == 0 && (reinterpret_cast<uintptr_t>(logits) & 15u) == 0;
+#define MOE_TOPK_CASE(V, VEC)                                                                  \
+  (bias ? topk_kernel<V, true, VEC><<<grid, threads, 0, s>>>(logits, bias, T, E, k, idx, gate, err) \
+        : topk_kernel<V, false, VEC><<<grid, threads, 0, s>>>(logits, bias, T, E, k, idx, gate, err))
+  if (E <= 32) MOE_TOPK_CASE(1, false);
+  else if (E <= 64) MOE_TOPK_CASE(2, false);
+  else if (E <= 128) { if (vec) MOE_TOPK_CASE(4, true); else MOE_TOPK_CASE(4, false); }
+  else if (E <= 256) { if (vec) MOE_TOPK_CASE(8, true); else MOE_TOPK_CASE(8, false); }
+  else if (E <= 512) { if (vec) MOE_TOPK_CASE(16, true); else MOE_TOPK_CASE(16, false); }
+  else { if (vec) MOE_TOPK_CASE(32, true); else MOE_TOPK_CASE(32, false); }
+#undef MOE_TOPK_CASE
+  return launch_status();
+}
+
 }  // namespace
 
 int launch_topk(const float* logits, int T, int E, int k, int32_t* idx, float* gate,
                 int32_t* err, cudaStream_t s) {
   if (cudaMemsetAsync(err, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_LAUNCH;
   if (T == 0) return MOE_OK;
-  const int threads = 256, per_block = threads / 32;
-  const unsigned grid = (unsigned)((T + per_block - 1) / per_block);
-#define MOE_TOPK_CASE(V) topk_kernel<V, false><<<grid, threads, 0, s>>>(logits, nullptr, T, E, k, idx, gate, err)
-  if (E <= 32) MOE_TOPK_CASE(1);
-  else if (E <= 64) MOE_TOPK_CASE(2);
-  else if (E <= 128) MOE_TOPK_CASE(4);
-  else if (E <= 256) MOE_TOPK_CASE(8);
-  else if (E <= 512) MOE_TOPK_CASE(16);
-  else MOE_TOPK_CASE(32);
-#undef MOE_TOPK_CASE
-  return launch_status();
+  return launch_topk_impl(logits, nullptr, T, E, k, idx, gate, err, s);
 }
 
 int launch_topk_biased(const float* logits, const float* bias, int T, int E, int k,
                        int32_t* idx, float* gate, int32_t* err, cudaStream_t s) {
   if (cudaMemsetAsync(err, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_LAUNCH;
   if (T == 0) return MOE_OK;
-  const int threads = 256, per_block = threads / 32;
-  const unsigned grid = (unsigned)((T + per_block - 1) / per_block);
-#define MOE_TOPKB_CASE(V) topk_kernel<V, true><<<grid, threads, 0, s>>>(logits, bias, T, E, k, idx, gate, err)
-  if (E <= 32) MOE_TOPKB_CASE(1);
-  else if (E <= 64) MOE_TOPKB_CASE(2);
-  else if (E <= 128) MOE_TOPKB_CASE(4);
-  else if (E <= 256) MOE_TOPKB_CASE(8);
-  else if (E <= 512) MOE_TOPKB_CASE(16);
-  else MOE_TOPKB_CASE(32);
-#undef MOE_TOPKB_CASE
-  return launch_status();
+  return launch_topk_impl(logits, bias, T, E, k, idx, gate, err, s);
 }
 
 int launch_capacity(const int32_t* counts, int E, long long A, int cf_num, int cf_den,

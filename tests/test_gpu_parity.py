@@ -164,8 +164,9 @@ def test_empty_batch():
     assert L.counts.tolist() == [0] * 8 and L.loads.tolist() == [0] * 4
 
 
-def test_topk_ties_and_signed_zero():
-    T, E, k = 512, 64, 6
+@pytest.mark.parametrize("E,k", [(64, 6), (256, 8), (100, 5)])
+def test_topk_ties_and_signed_zero(E, k):
+    T = 512
     g = torch.Generator().manual_seed(12)
     vals = torch.tensor([-1.0, -0.0, 0.0, 0.5, 2.0])
     logits = vals[torch.randint(0, 5, (T, E), generator=g)].contiguous()
