@@ -340,10 +340,15 @@ def run_ours(args, w: I.Workload, world, rank, local):
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(elapsed_ms / args.steps, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16+fp16 (gate/up GEMM bf16, down GEMM fp16, fp32 accumulate; routing fp32)",
         "data": "synthetic (seeded; N(0,1) logits + per-expert bias, N(0,1) tokens, N(0,1/d) weights)",
         "config": {"workload": w.name, "T": w.T, "E": w.E, "k": w.k, "R": w.R, "S": w.S, "d": w.d,
                    "F": w.F, "maxvio": round(float(L.maxvio.item()), 4), "replicas": n_rep,
+                   # makespan proxy: rows of the busiest rank / C, with the plan and with
+                   # every expert at its home rank
+                   "max_rank_rows_over_C": 1.0,
+                   "home_only_max_rank_rows_over_C": round(1.0 + float(L.maxvio.item()), 4),
                    "parallelism": f"replicas x{world} (ranks simulated in one GPU's HBM)",
                    "l2": "step working set (weights, pool, activations) far above the 126 MB L2",
                    "launch": "eager, one stream" if args.eager else
