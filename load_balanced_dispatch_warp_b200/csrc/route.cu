@@ -18,89 +18,35 @@ __device__ __forceinline__ uint32_t order_key(float v) {
   const uint32_t u = __float_as_uint(v);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
-__device__ __forceinline__ float key_value(uint32_t key) {
-  const uint32_t u = (key & 0x80000000u) ? (key & 0x7fffffffu) : ~key;
-  return __uint_as_float(u);
+
+// Warp-wide fp32 maximum (one instruction on sm_100a).
+__device__ __forceinline__ float warp_max_f32(float v) {
+  float r;
+  asm("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
 }
 
-// One warp per token.  Lane l holds experts l, l+32, ... (VPL of them) as
-// order-preserving keys (pad entries e >= E: key 0, below every finite float).  Exact
-// top-k in three steps:
-//   1. tau = the k-th largest of the 32 lane maxima (k rounds of redux.sync over one
-//      value per lane).  At least k keys are >= tau, so every key of the top-k -- equal
-//      keys at the k-th place included -- is >= tau.
-//   2. The keys >= tau (usually close to k of them) are compacted to one per lane
-//      through shared memory.
-//   3. k rounds over one candidate per lane: warp max key (redux.sync), lowest expert id
-//      among its holders (redux.sync), the winner drops out.
-// More than 32 candidates (many equal keys) falls back to the same rounds over all of
-// the lane's keys.  BIASED: keys from logit + bias[e] (one fp32 add), gates from the
-// chosen experts' unbiased logits (bias-only balancing).
-// Expert held in slot i of a lane: lane + 32 i (scalar loads), or, with 16-byte loads
-// (VEC), 128 (i / 4) + 4 lane + i % 4.
-template <bool VEC>
-__device__ __forceinline__ int slot_id(int i, int lane) {
-  return VEC ? 128 * (i >> 2) + 4 * lane + (i & 3) : lane + 32 * i;
-}
-
-template <int VPL, bool BIASED, bool VEC>
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits,
-                                                   const float* __restrict__ bias, int T,
-                                                   int E, int k, int32_t* __restrict__ idx,
-                                                   float* __restrict__ gate,
-                                                   int32_t* __restrict__ err) {
-  __shared__ uint32_t s_key[8][32];
-  __shared__ int s_id[8][32];
-  __shared__ float s_raw[8][BIASED ? 32 : 1];
-  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + wib; t < T; t += nwarps) {
-  const float* row = logits + t * E;
+// Exact top-k of one token over order keys, the general procedure (any ties).  Lane l
+// holds experts l, l+32, ... (VPL of them) as raw logits x and, when BIASED, biases b;
+// pad entries (expert >= E) get key 0, below every finite float.  Three steps:
+//   1. tau = the k-th largest of the 32 lane maxima (k rounds over one key per lane).
+//      At least k keys are >= tau, so every key of the top-k -- equal keys at the k-th
+//      place included -- is >= tau.
+//   2. The keys >= tau are compacted to one per lane through shared memory.
+//   3. k rounds over one candidate per lane: warp max key, lowest expert id among its
+//      holders, the winner drops out.
+// More than 32 candidates (many equal keys) runs the rounds over all of the lane's keys.
+// On return lane j < k holds the j-th choice: its expert id and its unbiased logit.
+template <int VPL, bool BIASED>
+__device__ __noinline__ void topk_exact(const float* x, const float* b, int E, int k, int lane,
+                                        uint32_t* s_key, int* s_id, float* s_raw,
+                                        float& my_val, int& my_id) {
   uint32_t key[VPL];
-  float raw[BIASED ? VPL : 1];
-  float val[VPL];
-  if (VEC) {
-#pragma unroll
-    for (int q = 0; q < VPL / 4; ++q) {
-      const int e0 = 128 * q + 4 * lane;
-      float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (e0 < E) v4 = __ldcs(reinterpret_cast<const float4*>(row + e0));
-      val[4 * q] = v4.x;
-      val[4 * q + 1] = v4.y;
-      val[4 * q + 2] = v4.z;
-      val[4 * q + 3] = v4.w;
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      const int e = lane + 32 * i;
-      val[i] = e < E ? __ldcs(row + e) : 0.f;
-    }
-  }
-  bool bad = false;
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
-    const int e = slot_id<VEC>(i, lane);
-    uint32_t kv = 0;
-    if (e < E) {
-      const float v = val[i];
-      bad |= !isfinite(v);
-      if (BIASED) {
-        const float b = __ldg(bias + e);
-        bad |= !isfinite(b);
-        raw[i] = v;
-        kv = order_key(__fadd_rn(v, b));
-      } else {
-        kv = order_key(v);
-      }
-    }
-    key[i] = kv;
+    const int e = lane + 32 * i;
+    key[i] = e < E ? order_key(BIASED ? __fadd_rn(x[i], b[i]) : x[i]) : 0u;
   }
-  if (__any_sync(MOE_FULL_MASK, bad)) {
-    if (lane == 0) atomicOr(err, MOE_DERR_NONFINITE);
-    continue;
-  }
-  // 1. threshold from the lane maxima
   uint32_t lmax = key[0];
 #pragma unroll
   for (int i = 1; i < VPL; ++i) lmax = max(lmax, key[i]);
@@ -110,7 +56,6 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
     const uint32_t holder = __reduce_min_sync(MOE_FULL_MASK, m == tau ? (uint32_t)lane : 32u);
     if ((uint32_t)lane == holder) m = 0;
   }
-  // 2. candidates: keys >= tau (tau > 0: pad keys never qualify)
   int cnt = 0;
 #pragma unroll
   for (int i = 0; i < VPL; ++i) cnt += key[i] >= tau;
@@ -121,75 +66,192 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
     if (lane >= o) incl += v;
   }
   const int total = __shfl_sync(MOE_FULL_MASK, incl, 31);
-  float my_val = 0.f;
-  int my_id = 0;
+  my_val = 0.f;
+  my_id = 0;
   if (total <= 32) {
     int pos = incl - cnt;
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       if (key[i] >= tau) {
-        s_key[wib][pos] = key[i];
-        s_id[wib][pos] = slot_id<VEC>(i, lane);
-        if (BIASED) s_raw[wib][pos] = raw[i];
+        s_key[pos] = key[i];
+        s_id[pos] = lane + 32 * i;
+        s_raw[pos] = x[i];
         ++pos;
       }
     }
     __syncwarp();
-    uint32_t ck = lane < total ? s_key[wib][lane] : 0u;
-    const int cid = lane < total ? s_id[wib][lane] : 0;
-    const float craw = (BIASED && lane < total) ? s_raw[wib][BIASED ? lane : 0] : 0.f;
-    // 3. k rounds over one candidate per lane
+    uint32_t ck = lane < total ? s_key[lane] : 0u;
+    const int cid = lane < total ? s_id[lane] : 0;
+    const float craw = lane < total ? s_raw[lane] : 0.f;
     for (int j = 0; j < k; ++j) {
       const uint32_t wmax = __reduce_max_sync(MOE_FULL_MASK, ck);
-      const uint32_t wid =
-          __reduce_min_sync(MOE_FULL_MASK, (ck == wmax && lane < total) ? (uint32_t)cid : 0xffffffffu);
+      const uint32_t wid = __reduce_min_sync(
+          MOE_FULL_MASK, (ck == wmax && lane < total) ? (uint32_t)cid : 0xffffffffu);
       const bool mine = lane < total && (uint32_t)cid == wid;
-      if (BIASED) {
-        const uint32_t src = __reduce_min_sync(MOE_FULL_MASK, mine ? (uint32_t)lane : 32u);
-        const float sel = __shfl_sync(MOE_FULL_MASK, craw, (int)src);
-        if (lane == j) my_val = sel;
-      } else if (lane == j) {
-        my_val = key_value(wmax);
+      const uint32_t src = __reduce_min_sync(MOE_FULL_MASK, mine ? (uint32_t)lane : 32u);
+      const float sel = __shfl_sync(MOE_FULL_MASK, craw, (int)src);
+      if (lane == j) {
+        my_val = sel;
+        my_id = (int)wid;
       }
-      if (lane == j) my_id = (int)wid;
       if (mine) ck = 0;
     }
+    __syncwarp();  // the candidate buffer is rewritten by the warp's next call
   } else {
-    // many equal keys: rounds over all of the lane's keys
     for (int j = 0; j < k; ++j) {
-      // lane's best: largest key, equal keys -> lowest expert id
+      // lane's best: largest key, equal keys -> lowest expert id (= lowest slot)
       uint32_t best = key[0];
-      int best_e = slot_id<VEC>(0, lane);
+      int best_i = 0;
 #pragma unroll
       for (int i = 1; i < VPL; ++i) {
-        const int e = slot_id<VEC>(i, lane);
-        const bool gt = key[i] > best || (key[i] == best && e < best_e);
+        const bool gt = key[i] > best;
         best = gt ? key[i] : best;
-        best_e = gt ? e : best_e;
+        best_i = gt ? i : best_i;
       }
       const uint32_t wmax = __reduce_max_sync(MOE_FULL_MASK, best);
-      const uint32_t cand = best == wmax ? (uint32_t)best_e : 0xffffffffu;
+      const uint32_t cand = best == wmax ? (uint32_t)(lane + 32 * best_i) : 0xffffffffu;
       const uint32_t wid = __reduce_min_sync(MOE_FULL_MASK, cand);
       float sel = 0.f;
       bool mine = false;
 #pragma unroll
       for (int i = 0; i < VPL; ++i) {
-        const bool hit = slot_id<VEC>(i, lane) == (int)wid;
+        const bool hit = lane + 32 * i == (int)wid;
         mine |= hit;
-        if (BIASED && hit) sel = raw[i];
+        if (hit) sel = x[i];
         key[i] = hit ? 0u : key[i];
       }
-      if (BIASED) {
-        const uint32_t src = __reduce_min_sync(MOE_FULL_MASK, mine ? (uint32_t)lane : 32u);
-        sel = __shfl_sync(MOE_FULL_MASK, sel, (int)src);
-      }
+      const uint32_t src = __reduce_min_sync(MOE_FULL_MASK, mine ? (uint32_t)lane : 32u);
+      sel = __shfl_sync(MOE_FULL_MASK, sel, (int)src);
       if (lane == j) {
-        my_val = BIASED ? sel : key_value(wmax);
+        my_val = sel;
         my_id = (int)wid;
       }
     }
   }
-  // softmax over the chosen (unbiased) logits
+}
+
+// One warp per token; lane l holds experts l, l+32, ... (VPL of them), so neighbouring
+// experts sit in different lanes.  Fast path, exact whenever it is taken:
+//   - each lane keeps its two largest keys h1 >= h2 (a multiset: equal keys count twice);
+//   - k rounds: w = warp max of the lane heads; every lane whose head equals w pops it
+//     (head <- h2, then -inf) and notes the round in a bit mask;
+//   - the rounds are the top-k, in order, iff exactly k pops happened in total and every
+//     lane holds exactly as many keys >= w_last as it popped.  Then the popped keys are
+//     precisely the keys >= w_last, k of them; one pop per round means no two lanes ever
+//     held equal keys at the top, and two equal keys of one lane pop in consecutive
+//     rounds, the lower slot (= lower expert id) first.
+// Otherwise (equal keys across lanes, a lane holding three of the top-k, overflow to
+// -inf) the warp runs topk_exact on the same registers.  Gates: softmax over the chosen
+// experts' unbiased logits in fp32.  K > 0 fixes k at compile time (K == k).
+template <int VPL, int K, bool BIASED>
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits,
+                                                   const float* __restrict__ bias, int T,
+                                                   int E, int k_rt, int32_t* __restrict__ idx,
+                                                   float* __restrict__ gate,
+                                                   int32_t* __restrict__ err) {
+  __shared__ uint32_t s_key[8][32];
+  __shared__ int s_id[8][32];
+  __shared__ float s_raw[8][32];
+  const int k = K > 0 ? K : k_rt;
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int64_t t = (int64_t)blockIdx.x * 8 + wib;
+  if (t >= T) return;
+  float b[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) b[i] = 0.f;
+  if (BIASED) {
+    bool bad = false;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int e = lane + 32 * i;
+      b[i] = e < E ? __ldg(bias + e) : 0.f;
+      bad |= !isfinite(b[i]);
+    }
+    if (__any_sync(MOE_FULL_MASK, bad)) {
+      if (lane == 0) atomicOr(err, MOE_DERR_NONFINITE);
+      return;
+    }
+  }
+  const float* row = logits + t * E;
+  float x[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int e = lane + 32 * i;
+    x[i] = e < E ? __ldcs(row + e) : 0.f;
+  }
+  // non-finite check: x * 0 is +-0 for finite x and NaN otherwise
+  float key[VPL];
+  float z = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    z = __fmaf_rn(x[i], 0.f, z);
+    key[i] = lane + 32 * i < E ? (BIASED ? __fadd_rn(x[i], b[i]) : x[i]) : -INFINITY;
+  }
+  if (__any_sync(MOE_FULL_MASK, !(z == 0.f))) {
+    if (lane == 0) atomicOr(err, MOE_DERR_NONFINITE);
+    return;
+  }
+  float h1 = key[0], h2 = -INFINITY;
+#pragma unroll
+  for (int i = 1; i < VPL; ++i) {
+    h2 = fmaxf(h2, fminf(h1, key[i]));
+    h1 = fmaxf(h1, key[i]);
+  }
+  float head = h1, nxt = h2, w0 = -INFINITY, tau = -INFINITY;
+  uint32_t won = 0;
+#pragma unroll
+  for (int j = 0; j < (K > 0 ? K : 32); ++j) {
+    if (K == 0 && j >= k) break;
+    const float w = warp_max_f32(head);
+    if (j == 0) w0 = w;
+    const bool eq = head == w;
+    won |= eq ? (1u << j) : 0u;
+    head = eq ? nxt : head;
+    nxt = eq ? -INFINITY : nxt;
+    tau = w;
+  }
+  const int npop = __popc(won);
+  uint32_t m_tau = 0, m_h1 = 0;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    m_tau |= key[i] >= tau ? (1u << i) : 0u;
+    m_h1 |= key[i] >= h1 ? (1u << i) : 0u;
+  }
+  const int total = (int)__reduce_add_sync(MOE_FULL_MASK, (unsigned)npop);
+  const bool fast = __all_sync(MOE_FULL_MASK, __popc(m_tau) == npop) && total == k &&
+                    tau > -INFINITY;
+  if (fast) {
+    // slots of the popped keys: s1 holds h1 (lowest slot among equal keys), s2 the other
+    const int s1 = __ffs(m_h1) - 1;
+    const int s2 = __ffs(m_tau & ~(1u << (s1 & 31))) - 1;
+    const int r1 = __ffs(won) - 1;
+    const int r2 = __ffs(won & (won - 1u)) - 1;
+    float v1 = h1, v2 = h2;
+    if (BIASED) {
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        v1 = i == s1 ? x[i] : v1;
+        v2 = i == s2 ? x[i] : v2;
+      }
+    }
+    const float top =
+        BIASED ? warp_max_f32(npop > 0 ? fmaxf(v1, npop > 1 ? v2 : -INFINITY) : -INFINITY) : w0;
+    const float e1 = npop > 0 ? expf(v1 - top) : 0.f;
+    const float e2 = npop > 1 ? expf(v2 - top) : 0.f;
+    const float sum = warp_sum(e1 + e2);
+    if (npop > 0) {
+      idx[t * k + r1] = lane + 32 * s1;
+      gate[t * k + r1] = e1 / sum;
+    }
+    if (npop > 1) {
+      idx[t * k + r2] = lane + 32 * s2;
+      gate[t * k + r2] = e2 / sum;
+    }
+    return;
+  }
+  float my_val;
+  int my_id;
+  topk_exact<VPL, BIASED>(x, b, E, k, lane, s_key[wib], s_id[wib], s_raw[wib], my_val, my_id);
   float top = lane < k ? my_val : -INFINITY;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) top = fmaxf(top, __shfl_xor_sync(MOE_FULL_MASK, top, o));
@@ -198,8 +260,6 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   if (lane < k) {
     idx[t * k + lane] = my_id;
     gate[t * k + lane] = ex / sum;
-  }
-  __syncwarp();  // the warp's candidate buffer is rewritten by its next token
   }
 }
 
@@ -355,25 +415,38 @@ __global__ void __launch_bounds__(512) hist_kernel(const int32_t* __restrict__ i
   }
 }
 
-// One warp per token over a persistent grid (8 warps per block, up to 8 blocks per SM);
-// 16-byte loads when every lane's slots come in aligned groups of four.
+// One warp per token, 8 warps per block.  Unbiased calls with k in {2, 4, 6, 8} and up to
+// 256 experts run a kernel with k fixed at compile time (the rounds unroll).
+template <int VPL>
+void launch_topk_vpl(const float* logits, const float* bias, int T, int E, int k, int32_t* idx,
+                     float* gate, int32_t* err, cudaStream_t s) {
+  const unsigned grid = (unsigned)(((int64_t)T + 7) / 8);
+#define MOE_TOPK(KK, B) topk_kernel<VPL, KK, B><<<grid, 256, 0, s>>>(logits, bias, T, E, k, idx, gate, err)
+  if (bias) {
+    MOE_TOPK(0, true);
+    return;
+  }
+  if constexpr (VPL <= 8) {
+    switch (k) {
+      case 8: MOE_TOPK(8, false); return;
+      case 6: MOE_TOPK(6, false); return;
+      case 4: MOE_TOPK(4, false); return;
+      case 2: MOE_TOPK(2, false); return;
+      default: break;
+    }
+  }
+  MOE_TOPK(0, false);
+#undef MOE_TOPK
+}
+
 int launch_topk_impl(const float* logits, const float* bias, int T, int E, int k,
                      int32_t* idx, float* gate, int32_t* err, cudaStream_t s) {
-  const int threads = 256, per_block = threads / 32;
-  const int64_t want = ((int64_t)T + per_block - 1) / per_block;
-  const int64_t cap = (int64_t)num_sms() * 8;
-  const unsigned grid = (unsigned)(want < cap ? want : cap);
-  const bool vec = E % 4 == 0 && (reinterpret_cast<uintptr_t>(logits) & 15u) == 0;
-#define MOE_TOPK_CASE(V, VEC)                                                                  \
-  (bias ? topk_kernel<V, true, VEC><<<grid, threads, 0, s>>>(logits, bias, T, E, k, idx, gate, err) \
-        : topk_kernel<V, false, VEC><<<grid, threads, 0, s>>>(logits, bias, T, E, k, idx, gate, err))
-  if (E <= 32) MOE_TOPK_CASE(1, false);
-  else if (E <= 64) MOE_TOPK_CASE(2, false);
-  else if (E <= 128) { if (vec) MOE_TOPK_CASE(4, true); else MOE_TOPK_CASE(4, false); }
-  else if (E <= 256) { if (vec) MOE_TOPK_CASE(8, true); else MOE_TOPK_CASE(8, false); }
-  else if (E <= 512) { if (vec) MOE_TOPK_CASE(16, true); else MOE_TOPK_CASE(16, false); }
-  else { if (vec) MOE_TOPK_CASE(32, true); else MOE_TOPK_CASE(32, false); }
-#undef MOE_TOPK_CASE
+  if (E <= 32) launch_topk_vpl<1>(logits, bias, T, E, k, idx, gate, err, s);
+  else if (E <= 64) launch_topk_vpl<2>(logits, bias, T, E, k, idx, gate, err, s);
+  else if (E <= 128) launch_topk_vpl<4>(logits, bias, T, E, k, idx, gate, err, s);
+  else if (E <= 256) launch_topk_vpl<8>(logits, bias, T, E, k, idx, gate, err, s);
+  else if (E <= 512) launch_topk_vpl<16>(logits, bias, T, E, k, idx, gate, err, s);
+  else launch_topk_vpl<32>(logits, bias, T, E, k, idx, gate, err, s);
   return launch_status();
 }
 
