@@ -120,15 +120,16 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- work units
-def algorithmic(w: I.Workload, n_rep: int):
-    """Algorithmic bytes (HBM) or flops per call for one step."""
+def algorithmic(w: I.Workload, n_rep: int, fused: bool = False):
+    """Algorithmic bytes (HBM) or flops per call for one step.  Fused: the dispatch call
+    only reads idx and writes perm and src; the FFN reads the token rows itself."""
     T, E, k, d, F, A = w.T, w.E, w.k, w.d, w.F, w.A
     return {
         "moe_topk": ("GB/s", T * E * 4 + A * 8),
         "moe_histogram_maxvio": ("GB/s", A * 4 + E * 4),
         "moe_plan_balanced": ("us", None),
         "moe_prefetch_replicas": ("GB/s", 2 * n_rep * 3 * d * F * 2),
-        "moe_dispatch": ("GB/s", T * d * 2 + A * d * 2 + 12 * A),
+        "moe_dispatch": ("GB/s", 12 * A if fused else T * d * 2 + A * d * 2 + 12 * A),
         "moe_grouped_ffn": ("TFLOP/s", 6 * A * d * F),
         "moe_combine": ("GB/s", A * d * 2 + T * d * 2 + 8 * A),
     }
@@ -189,7 +190,7 @@ def run_ours(args, w: I.Workload, world, rank, local):
     logits = logits_h.to(device)
     x = x_h.to(device)
     W1, W3, W2 = I.make_weights(w, device=device)
-    L = M.MoELayer(w.T, w.E, w.k, w.R, w.S, w.d, w.F, device=device)
+    L = M.MoELayer(w.T, w.E, w.k, w.R, w.S, w.d, w.F, device=device, fused=args.fused)
     steps = [lambda: L.route(logits), lambda: L.measure(), lambda: L.balance(),
              lambda: L.prefetch(W1, W3, W2), lambda: L.dispatch(x),
              lambda: L.expert_ffn(W1, W3, W2), lambda: L.combine()]
@@ -308,7 +309,7 @@ def run_ours(args, w: I.Workload, world, rank, local):
     if int(L.err.item()) != 0:
         raise RuntimeError(f"device error word {int(L.err.item())} in the end-to-end run")
 
-    units = algorithmic(w, n_rep)
+    units = algorithmic(w, n_rep, args.fused)
     peaks, peak_src = load_peaks()
     calls = {}
     for c in CALLS:
@@ -350,6 +351,8 @@ def run_ours(args, w: I.Workload, world, rank, local):
                    "max_rank_rows_over_C": 1.0,
                    "home_only_max_rank_rows_over_C": round(1.0 + float(L.maxvio.item()), 4),
                    "parallelism": f"replicas x{world} (ranks simulated in one GPU's HBM)",
+                   "dispatch": ("fused: placement only, GEMM 1 gathers x[src[row]]" if args.fused
+                                else "row copy into recv, GEMM 1 reads recv"),
                    "l2": "step working set (weights, pool, activations) far above the 126 MB L2",
                    "launch": "eager, one stream" if args.eager else
                              "K steps captured in one CUDA graph, replayed once; per-call "
@@ -469,6 +472,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="launch the timed steps eagerly")
+    ap.add_argument("--fused", action="store_true",
+                    help="fused dispatch: placement only, GEMM 1 gathers the token rows")
     args = ap.parse_args()
     w = I.WORKLOADS[args.config]
 

@@ -239,6 +239,35 @@ int moe_grouped_ffn(const moe_bf16* recv, const int32_t* plan, const moe_bf16* W
                     moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * Fused dispatch: the row copy folded into GEMM 1's operand load.   [MoonEP] para. 3
+ * (zero-copy dispatch straight into the final static buffers) and [Primer], the second of
+ * the three ideas it credits to DeepEP (routing layout and data movement fused into
+ * dedicated GPU kernels): the rows a rank receives are read where they already are.
+ *
+ * moe_dispatch_index computes what moe_dispatch computes except recv: perm and src only
+ * (same arguments minus x, d and recv; same errors).
+ */
+int moe_dispatch_index(const int32_t* idx, const int32_t* plan, int T, int k, int E, int R,
+                       int S, int32_t* workspace, int32_t* perm, int32_t* src, int32_t* err,
+                       moe_stream_t stream);
+/*
+ * moe_grouped_ffn_gather computes exactly what moe_grouped_ffn computes, bit for bit,
+ * with GEMM 1's row r read as x[src[r]] instead of recv[r] (the same bf16 values), so no
+ * [R*C,d] recv buffer is written or read.  The persistent GEMM-1 kernel's producer warp
+ * gathers the rows with 16-byte copies into the swizzled operand tiles.
+ *   x    [T,d] bf16             token rows (16-byte aligned).
+ *   src  [R*C] int32            token of each row, from moe_dispatch_index (or
+ *                               moe_dispatch).  An entry outside [0, T) sets
+ *                               MOE_DERR_ID_RANGE (that row reads token 0 instead).
+ *   other arguments, outputs and errors as moe_grouped_ffn.
+ */
+int moe_grouped_ffn_gather(const moe_bf16* x, const int32_t* src, const int32_t* plan,
+                           const moe_bf16* W1, const moe_bf16* W3, const moe_f16* W2,
+                           const moe_bf16* P1, const moe_bf16* P3, const moe_f16* P2, int T,
+                           int k, int E, int R, int S, int d, int F, moe_f16* h, moe_bf16* y,
+                           int32_t* err, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
  * Dispatch without a workspace argument.  The pages have no counterpart: this is a
  * convenience of this library for callers that cannot allocate device memory when they
  * dispatch -- an operator or plugin interface of another runtime that passes only its

@@ -7,7 +7,9 @@ status.  Every step of the path runs in the library's CUDA kernels; there is no 
 fallback, and importing a function raises if the library has not been built.
 
 ``MoELayer`` owns the per-layer device buffers (PyTorch allocations) and runs the seven
-calls in order: route, measure, plan, prefetch, dispatch, expert FFN, combine.
+calls in order: route, measure, plan, prefetch, dispatch, expert FFN, combine.  With
+``fused=True`` the dispatch computes the row placement only and the expert FFN gathers its
+rows from ``x`` (``moe_dispatch_index`` + ``moe_grouped_ffn_gather``).
 """
 from __future__ import annotations
 
@@ -25,6 +27,7 @@ DERR_NONFINITE, DERR_ID_RANGE, DERR_DUPLICATE, DERR_SLOTS, DERR_TIMEOUT = 1, 2, 
 ENTRY_POINTS = ("moe_topk", "moe_histogram_maxvio", "moe_plan_balanced", "moe_prefetch_replicas",
                 "moe_dispatch", "moe_grouped_ffn", "moe_combine")
 VARIANTS = ("moe_topk_biased", "moe_capacity_ledger")
+FUSED = ("moe_dispatch_index", "moe_grouped_ffn_gather")
 HELPERS = ("moe_plan_get_layout", "moe_dispatch_workspace_words", "moe_status_string")
 
 
@@ -63,6 +66,8 @@ def lib() -> ctypes.CDLL:
             "moe_topk_biased": [P, P, I, I, I, P, P, P, P],
             "moe_capacity_ledger": [P, I, I, I, I, I, P, P, P, P, P, P],
             "moe_selftest_bounded_wait": [P, I, P],
+            "moe_dispatch_index": [P, P, I, I, I, I, I, P, P, P, P, P],
+            "moe_grouped_ffn_gather": [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, P],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -208,6 +213,29 @@ def moe_grouped_ffn(recv, plan, W1, W3, W2, P1, P3, P2, T, k, R, S, h, y, err, s
         _ptr(err, torch.int32, "err"), _stream(stream)), "moe_grouped_ffn")
 
 
+def moe_dispatch_index(idx, plan, E, R, S, workspace, perm, src, err, stream=None):
+    """moe_dispatch without the row copy: perm and src only (for moe_grouped_ffn_gather)."""
+    T, k = idx.shape
+    _check(lib().moe_dispatch_index(
+        _ptr(idx, torch.int32, "idx"), _ptr(plan, torch.int32, "plan"), T, k, E, R, S,
+        _ptr(workspace, torch.int32, "workspace"), _ptr(perm, torch.int32, "perm"),
+        _ptr(src, torch.int32, "src"), _ptr(err, torch.int32, "err"), _stream(stream)),
+        "moe_dispatch_index")
+
+
+def moe_grouped_ffn_gather(x, src, plan, W1, W3, W2, P1, P3, P2, T, k, R, S, h, y, err,
+                           stream=None):
+    """moe_grouped_ffn with GEMM 1's rows gathered as x[src[row]] (no recv buffer)."""
+    E, F, d = W1.shape
+    bf, hf = torch.bfloat16, torch.float16
+    _check(lib().moe_grouped_ffn_gather(
+        _ptr(x, bf, "x"), _ptr(src, torch.int32, "src"), _ptr(plan, torch.int32, "plan"),
+        _ptr(W1, bf, "W1"), _ptr(W3, bf, "W3"), _ptr(W2, hf, "W2"), _ptr(P1, bf, "P1"),
+        _ptr(P3, bf, "P3"), _ptr(P2, hf, "P2"), T, k, E, R, S, d, F, _ptr(h, hf, "h"),
+        _ptr(y, bf, "y"), _ptr(err, torch.int32, "err"), _stream(stream)),
+        "moe_grouped_ffn_gather")
+
+
 def moe_combine(y, perm, gate, out, err, stream=None):
     T, k = perm.shape
     d = out.shape[1]
@@ -223,10 +251,13 @@ class MoELayer:
 
     The replica pool (P1, P3, P2: R*S slots) is allocated once here; several layers may
     share one pool by passing ``pool=`` (it is process-global in the MoonEP design).
+    ``fused=True``: no recv buffer; the FFN gathers the rows of the ``x`` last dispatched.
     """
 
-    def __init__(self, T, E, k, R, S, d, F, device="cuda", pool=None):
+    def __init__(self, T, E, k, R, S, d, F, device="cuda", pool=None, fused=False):
         self.T, self.E, self.k, self.R, self.S, self.d, self.F = T, E, k, R, S, d, F
+        self.fused = bool(fused)
+        self._x = None
         self.A = T * k
         self.C = self.A // R
         dev = torch.device(device)
@@ -241,7 +272,7 @@ class MoELayer:
         self.balancedness = torch.empty(1, dtype=torch.float64, device=dev)
         self.plan = torch.empty(self.layout.words, dtype=i32, device=dev)
         self.workspace = torch.empty(max(1, dispatch_workspace_words(T, E)), dtype=i32, device=dev)
-        self.recv = torch.empty(self.A, d, dtype=bf, device=dev)
+        self.recv = None if self.fused else torch.empty(self.A, d, dtype=bf, device=dev)
         self.perm = torch.empty(T, k, dtype=i32, device=dev)
         self.src = torch.empty(self.A, dtype=i32, device=dev)
         self.h = torch.empty(self.A, F, dtype=torch.float16, device=dev)
@@ -278,13 +309,26 @@ class MoELayer:
         moe_prefetch_replicas(self.plan, W1, W3, W2, self.R, self.S, P1, P3, P2, self.err, stream)
 
     def dispatch(self, x, stream=None):
-        moe_dispatch(x, self.idx, self.plan, self.E, self.R, self.S, self.workspace, self.recv,
-                     self.perm, self.src, self.err, stream)
+        if self.fused:
+            if x.shape != (self.T, self.d) or x.dtype != torch.bfloat16:
+                raise ValueError("x must be [T,d] bf16")
+            self._x = x
+            moe_dispatch_index(self.idx, self.plan, self.E, self.R, self.S, self.workspace,
+                               self.perm, self.src, self.err, stream)
+        else:
+            moe_dispatch(x, self.idx, self.plan, self.E, self.R, self.S, self.workspace,
+                         self.recv, self.perm, self.src, self.err, stream)
 
     def expert_ffn(self, W1, W3, W2, stream=None):
         P1, P3, P2 = self.pool
-        moe_grouped_ffn(self.recv, self.plan, W1, W3, W2, P1, P3, P2, self.T, self.k, self.R,
-                        self.S, self.h, self.y, self.err, stream)
+        if self.fused:
+            if self._x is None:
+                raise RuntimeError("fused expert_ffn needs a dispatch(x) first")
+            moe_grouped_ffn_gather(self._x, self.src, self.plan, W1, W3, W2, P1, P3, P2, self.T,
+                                   self.k, self.R, self.S, self.h, self.y, self.err, stream)
+        else:
+            moe_grouped_ffn(self.recv, self.plan, W1, W3, W2, P1, P3, P2, self.T, self.k,
+                            self.R, self.S, self.h, self.y, self.err, stream)
 
     def combine(self, stream=None):
         moe_combine(self.y, self.perm, self.gate, self.out, self.err, stream)
@@ -304,7 +348,7 @@ class MoELayer:
     def kernels_per_forward(self) -> int:
         n = (1 if self.T > 0 else 0) + 1 + 1  # topk, histogram, plan
         n += 1 if self.S > 0 else 0           # prefetch
-        n += 3 if self.T > 0 else 0           # dispatch: tile counts, ranks, row scatter
+        n += (2 if self.fused else 3) if self.T > 0 else 0  # tile counts, ranks[, row scatter]
         n += 2 if self.T > 0 else 0           # two grouped GEMMs
         n += 1 if self.T > 0 else 0           # combine
         return n

@@ -195,6 +195,49 @@ int moe_dispatch(const moe_bf16* x, const int32_t* idx, const int32_t* plan, int
                               src, err, as_stream(stream));
 }
 
+int moe_dispatch_index(const int32_t* idx, const int32_t* plan, int T, int k, int E, int R,
+                       int S, int32_t* workspace, int32_t* perm, int32_t* src, int32_t* err,
+                       moe_stream_t stream) {
+  if (!plan || !err) return MOE_ERR_ARG;
+  if (T > 0 && (!idx || !workspace || !perm || !src)) return MOE_ERR_ARG;
+  MOE_TRY(check_route(T, E, k));
+  MOE_TRY(check_ranks(T, k, E, R, true));
+  MOE_TRY(check_groups(E, R, S));
+  moe_plan_layout L;
+  MOE_TRY(moe_plan_get_layout(E, R, S, &L));
+  return moe::launch_dispatch(nullptr, idx, plan, L, T, k, E, R, 0, workspace, nullptr, perm,
+                              src, err, as_stream(stream));
+}
+
+int moe_grouped_ffn_gather(const moe_bf16* x, const int32_t* src, const int32_t* plan,
+                           const moe_bf16* W1, const moe_bf16* W3, const moe_f16* W2,
+                           const moe_bf16* P1, const moe_bf16* P3, const moe_f16* P2, int T,
+                           int k, int E, int R, int S, int d, int F, moe_f16* h, moe_bf16* y,
+                           int32_t* err, moe_stream_t stream) {
+  if (!plan || !W1 || !W3 || !W2 || !err) return MOE_ERR_ARG;
+  if (T > 0 && (!x || !src || !h || !y)) return MOE_ERR_ARG;
+  if (S > 0 && (!P1 || !P3 || !P2)) return MOE_ERR_ARG;
+  MOE_TRY(check_route(T, E, k));
+  MOE_TRY(check_ranks(T, k, E, R, true));
+  MOE_TRY(check_groups(E, R, S));
+  MOE_TRY(check_dims(T, k, d, F));
+  if ((int64_t)E * F >= kMaxElems || (int64_t)E * d >= kMaxElems ||
+      (int64_t)R * S * F >= kMaxElems || (int64_t)R * S * d >= kMaxElems)
+    return MOE_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(h) || !aligned16(y) || !aligned16(W1) || !aligned16(W3) ||
+      !aligned16(W2) || (S > 0 && (!aligned16(P1) || !aligned16(P3) || !aligned16(P2))))
+    return MOE_ERR_ARG;
+  moe_plan_layout L;
+  MOE_TRY(moe_plan_get_layout(E, R, S, &L));
+  return moe::launch_grouped_ffn_gather(
+      reinterpret_cast<const __nv_bfloat16*>(x), src, plan, L,
+      reinterpret_cast<const __nv_bfloat16*>(W1), reinterpret_cast<const __nv_bfloat16*>(W3),
+      reinterpret_cast<const __half*>(W2), reinterpret_cast<const __nv_bfloat16*>(P1),
+      reinterpret_cast<const __nv_bfloat16*>(P3), reinterpret_cast<const __half*>(P2), T, k, E,
+      R, S, d, F, reinterpret_cast<__half*>(h), reinterpret_cast<__nv_bfloat16*>(y), err,
+      as_stream(stream));
+}
+
 int moe_grouped_ffn(const moe_bf16* recv, const int32_t* plan, const moe_bf16* W1,
                     const moe_bf16* W3, const moe_f16* W2, const moe_bf16* P1,
                     const moe_bf16* P3, const moe_f16* P2, int T, int k, int E, int R,

@@ -49,9 +49,17 @@ int launch_grouped_ffn(const __nv_bfloat16* recv, const int32_t* plan,
                        const __nv_bfloat16* P3, const __half* P2, int T, int k, int E, int R,
                        int S, int d, int F, __half* h, __nv_bfloat16* y, int32_t* err,
                        cudaStream_t s);
+int launch_grouped_ffn_gather(const __nv_bfloat16* x, const int32_t* src, const int32_t* plan,
+                              const moe_plan_layout& L, const __nv_bfloat16* W1,
+                              const __nv_bfloat16* W3, const __half* W2,
+                              const __nv_bfloat16* P1, const __nv_bfloat16* P3,
+                              const __half* P2, int T, int k, int E, int R, int S, int d, int F,
+                              __half* h, __nv_bfloat16* y, int32_t* err, cudaStream_t s);
 int launch_bounded_wait_selftest(int32_t* err, int limit_us, cudaStream_t s);
 int launch_combine(const __nv_bfloat16* y, const int32_t* perm, const float* gate, int T,
                    int k, int d, __nv_bfloat16* out, const int32_t* err, cudaStream_t s);
+
+// launch_dispatch with recv == nullptr computes perm and src only (no row copy).
 
 // Tokens per tile of the placement kernels (workspace = ceil(T/kPlaceTile) * E words).
 constexpr int kPlaceTile = 256;

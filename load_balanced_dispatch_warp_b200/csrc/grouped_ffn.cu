@@ -26,6 +26,19 @@
 // Tiles are (group, 128-row block, N block), enumerated m-block-major from a prefix over
 // the group table built in shared memory by every CTA; CTA i takes tiles i, i+grid, ...
 //
+// Gathered GEMM 1 (GATHER): row r of the A operand is the token row x[src[r]] instead of
+// a dispatched copy recv[r] -- the dispatch's row copy folded into the operand load, as
+// the zero-copy dispatch of the MoonEP news article (paragraph 3) and the fused kernels of
+// "DeepEP-on-EFA Guidance, section 1: What is MoE" (routing layout and data movement in
+// dedicated GPU kernels) describe.  The whole producer warp then writes
+// each A tile with 16-byte cp.async copies into the same 128-byte-swizzled layout TMA
+// produces (16-byte chunk c of tile row r at r*128 + ((c ^ (r % 8)) * 16)); one warp
+// instruction reads four whole 128-byte row segments.  Rows past the group's end are
+// zero-filled.  After its copies for a stage each lane posts an arrival that fires when
+// they have landed (cp.async.mbarrier.arrive.noinc), so the producer never blocks on
+// them; the stage's full barrier expects those 32 arrivals plus the B operand's
+// transaction bytes.
+//
 // Every mbarrier wait is bounded (about 2 s of %globaltimer); a wait that runs out sets
 // MOE_DERR_TIMEOUT and a shared abort flag, every role leaves its loop, the producer
 // waits (bounded) for its copies in flight, the MMA thread for its MMAs, and TMEM is
@@ -62,6 +75,10 @@ struct FfnArgs {
   int out_ld;           // columns of the output tensor
   void* out;            // h (fp16) for GEMM 1, y (bf16) for GEMM 2
   int32_t* err;
+  const __nv_bfloat16* gx;  // GATHER: token rows x [T, gd]
+  const int32_t* gsrc;      // GATHER: token of each row, [R*C]
+  int gd;                   // GATHER: row length of x (= d)
+  int gT;                   // GATHER: rows of x (tokens)
 };
 
 // --------------------------------------------------------------------- PTX wrappers
@@ -124,6 +141,25 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
       : "memory");
+}
+
+// 16-byte global -> shared copy, bytes past src_bytes (0 or 16) zero-filled, L2 only
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+// arrival on `bar` once every cp.async this thread issued so far has landed (counts as one
+// of the barrier's expected arrivals)
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+// make this thread's completed shared-memory writes visible to the async proxy (MMA)
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() {
@@ -221,7 +257,7 @@ __device__ __forceinline__ Tile decode_tile(int t, const FfnArgs& a, const int* 
   return tl;
 }
 
-template <bool SWIGLU>
+template <bool SWIGLU, bool GATHER>
 __global__ void __launch_bounds__(FFN_THREADS, 1)
     ffn_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b0,
                const __grid_constant__ CUtensorMap tm_b1, const __grid_constant__ CUtensorMap tm_p0,
@@ -264,7 +300,7 @@ __global__ void __launch_bounds__(FFN_THREADS, 1)
   const uint32_t drain = smem_u32(bars + 2 * STAGES + 4);
   if (tid == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full0 + 8 * s, 1);
+      mbar_init(full0 + 8 * s, GATHER ? 33 : 1);
       mbar_init(empty0 + 8 * s, 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -288,7 +324,81 @@ __global__ void __launch_bounds__(FFN_THREADS, 1)
   const uint32_t tmem_base = static_cast<uint32_t>(s_misc[0]);
   const uint32_t b_bytes = (uint32_t)args.mma_n * BK * 2;
 
-  if (warp == 0) {
+  if (warp == 0 && GATHER) {
+    // ------------------------------------------------ gathering producer (whole warp)
+    const int q = lane >> 3;             // row within each 4-row slice
+    const int c = lane & 7;              // 16-byte chunk of the 128-byte row segment
+    const char* xb = reinterpret_cast<const char*>(args.gx) + c * 16;
+    const int64_t row_bytes = (int64_t)args.gd * 2;
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued_mask = 0, issued_phase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; ok && t < total_tiles; t += gridDim.x) {
+      const Tile tl = decode_tile(t, args, s_prefix);
+      // tokens of rows lane + 32 m; copy i covers row 4 i + q
+      int tokv[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int r = lane + 32 * m;
+        int tv = r < tl.valid_rows ? __ldg(args.gsrc + tl.a_row + r) : 0;
+        if ((unsigned)tv >= (unsigned)args.gT) {  // never read outside x
+          atomicOr(args.err, MOE_DERR_ID_RANGE);
+          tv = 0;
+        }
+        tokv[m] = tv;
+      }
+      int tok[32];
+      uint32_t vmask = 0;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int r = 4 * i + q;
+        tok[i] = __shfl_sync(MOE_FULL_MASK, tokv[i >> 3], r & 31);
+        vmask |= (r < tl.valid_rows ? 1u : 0u) << i;
+      }
+      for (int kb = 0; kb < args.k_blocks; ++kb) {
+        // every lane waits (bounded); the warp goes on only if all of them saw the stage free
+        if (!__all_sync(MOE_FULL_MASK, mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, args.err))) {
+          ok = false;
+          break;
+        }
+        const uint32_t fb = full0 + 8 * stage;
+        const uint32_t sa = smem_u32(stage_base + stage * STAGE_BYTES);
+        const char* kbase = xb + (int64_t)kb * (BK * 2);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int r = 4 * i + q;
+          const int rs = r & 7;
+          const uint32_t dst = sa + ((uint32_t)(r >> 3) << 10) + ((uint32_t)rs << 7) +
+                               ((uint32_t)(c ^ rs) << 4);
+          cp_async16(dst, kbase + (int64_t)tok[i] * row_bytes, ((vmask >> i) & 1u) * 16u);
+        }
+        cp_async_arrive(fb);
+        if (lane == 0) {
+          const CUtensorMap* mb0 = tl.pool ? &tm_p0 : &tm_b0;
+          const CUtensorMap* mb1 = tl.pool ? &tm_p1 : &tm_b1;
+          const uint32_t sb = sa + A_BYTES;
+          mbar_expect_tx(fb, b_bytes);
+          tma_load_2d(sb, mb0, fb, kb * BK, tl.b_row);
+          tma_load_2d(sb + (b_bytes >> 1), mb1, fb, kb * BK, tl.b_row);
+        }
+        issued_mask |= 1u << stage;
+        issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+    // no copy of this warp may still be landing when the CTA leaves
+    cp_async_wait_all();
+    __syncwarp();
+    if (lane == 0) {
+      for (int s = 0; s < STAGES; ++s)
+        if (issued_mask & (1u << s)) {
+          volatile int no_abort = 0;
+          mbar_wait(full0 + 8 * s, (issued_phase >> s) & 1u, &no_abort, args.err);
+        }
+    }
+    __syncwarp();
+  } else if (warp == 0) {
     // ------------------------------------------------------------- TMA producer
     if (lane == 0) {
       int stage = 0;
@@ -342,6 +452,7 @@ __global__ void __launch_bounds__(FFN_THREADS, 1)
         bool ok = true;
         for (int kb = 0; kb < args.k_blocks; ++kb) {
           if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, args.err)) { ok = false; break; }
+          if (GATHER) fence_proxy_async();  // A written by cp.async (generic proxy)
           tc_fence_after();
           const uint32_t sa = smem_u32(stage_base + stage * STAGE_BYTES);
           const uint32_t sb = sa + A_BYTES;
@@ -484,7 +595,7 @@ size_t ffn_smem_bytes() {
          (MAX_GROUPS + 1) * 4 + 33 * 4;
 }
 
-template <bool SWIGLU>
+template <bool SWIGLU, bool GATHER>
 int launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                const CUtensorMap& p0, const CUtensorMap& p1, const FfnArgs& args, cudaStream_t s) {
   static bool configured[64] = {false};
@@ -492,12 +603,12 @@ int launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b
   cudaGetDevice(&dev);
   const size_t smem = ffn_smem_bytes();
   if (dev < 64 && !configured[dev]) {
-    if (cudaFuncSetAttribute(ffn_kernel<SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(ffn_kernel<SWIGLU, GATHER>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return MOE_ERR_LAUNCH;
     configured[dev] = true;
   }
-  ffn_kernel<SWIGLU><<<num_sms(), FFN_THREADS, smem, s>>>(a, b0, b1, p0, p1, args);
+  ffn_kernel<SWIGLU, GATHER><<<num_sms(), FFN_THREADS, smem, s>>>(a, b0, b1, p0, p1, args);
   return launch_status();
 }
 
@@ -508,17 +619,20 @@ int launch_bounded_wait_selftest(int32_t* err, int limit_us, cudaStream_t s) {
   return launch_status();
 }
 
-int launch_grouped_ffn(const __nv_bfloat16* recv, const int32_t* plan,
-                       const moe_plan_layout& L, const __nv_bfloat16* W1,
-                       const __nv_bfloat16* W3, const __half* W2, const __nv_bfloat16* P1,
-                       const __nv_bfloat16* P3, const __half* P2, int T, int k, int E, int R,
-                       int S, int d, int F, __half* h, __nv_bfloat16* y, int32_t* err,
-                       cudaStream_t s) {
+// GEMM 1 reads its rows from recv (x == nullptr) or gathers them as x[src[row]].
+int launch_grouped_ffn_impl(const __nv_bfloat16* recv, const __nv_bfloat16* x,
+                            const int32_t* src, const int32_t* plan, const moe_plan_layout& L,
+                            const __nv_bfloat16* W1, const __nv_bfloat16* W3, const __half* W2,
+                            const __nv_bfloat16* P1, const __nv_bfloat16* P3, const __half* P2,
+                            int T, int k, int E, int R, int S, int d, int F, __half* h,
+                            __nv_bfloat16* y, int32_t* err, cudaStream_t s) {
   if (T == 0) return MOE_OK;
+  const bool gather = x != nullptr;
   const int64_t rows = (int64_t)T * k;  // R * C
   const int bn2 = (d % 256 == 0) ? 256 : 128;
   CUtensorMap m_recv, m_w1, m_w3, m_p1, m_p3, m_h, m_w2, m_p2;
-  if (!make_map(&m_recv, recv, rows, d, BM) || !make_map(&m_w1, W1, (int64_t)E * F, d, 128) ||
+  if (!make_map(&m_w1, W1, (int64_t)E * F, d, 128) ||
+      (!gather && !make_map(&m_recv, recv, rows, d, BM)) ||
       !make_map(&m_w3, W3, (int64_t)E * F, d, 128) ||
       !make_map(&m_h, h, rows, F, BM, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
       !make_map(&m_w2, W2, (int64_t)E * d, F, bn2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
@@ -545,7 +659,12 @@ int launch_grouped_ffn(const __nv_bfloat16* recv, const int32_t* plan,
   a1.out_ld = F;
   a1.out = h;
   a1.err = err;
-  int st = launch_one<true>(m_recv, m_w1, m_w3, m_p1, m_p3, a1, s);
+  a1.gx = x;
+  a1.gsrc = src;
+  a1.gd = d;
+  a1.gT = T;
+  int st = gather ? launch_one<true, true>(m_w1, m_w1, m_w3, m_p1, m_p3, a1, s)
+                  : launch_one<true, false>(m_recv, m_w1, m_w3, m_p1, m_p3, a1, s);
   if (st != MOE_OK) return st;
   FfnArgs a2 = a1;
   a2.n_blocks_n = d / bn2;
@@ -555,7 +674,29 @@ int launch_grouped_ffn(const __nv_bfloat16* recv, const int32_t* plan,
   a2.rows_per_expert = d;
   a2.out_ld = d;
   a2.out = y;
-  return launch_one<false>(m_h, m_w2, m_w2, m_p2, m_p2, a2, s);
+  a2.gx = nullptr;
+  a2.gsrc = nullptr;
+  return launch_one<false, false>(m_h, m_w2, m_w2, m_p2, m_p2, a2, s);
+}
+
+int launch_grouped_ffn(const __nv_bfloat16* recv, const int32_t* plan,
+                       const moe_plan_layout& L, const __nv_bfloat16* W1,
+                       const __nv_bfloat16* W3, const __half* W2, const __nv_bfloat16* P1,
+                       const __nv_bfloat16* P3, const __half* P2, int T, int k, int E, int R,
+                       int S, int d, int F, __half* h, __nv_bfloat16* y, int32_t* err,
+                       cudaStream_t s) {
+  return launch_grouped_ffn_impl(recv, nullptr, nullptr, plan, L, W1, W3, W2, P1, P3, P2, T, k,
+                                 E, R, S, d, F, h, y, err, s);
+}
+
+int launch_grouped_ffn_gather(const __nv_bfloat16* x, const int32_t* src, const int32_t* plan,
+                              const moe_plan_layout& L, const __nv_bfloat16* W1,
+                              const __nv_bfloat16* W3, const __half* W2,
+                              const __nv_bfloat16* P1, const __nv_bfloat16* P3,
+                              const __half* P2, int T, int k, int E, int R, int S, int d, int F,
+                              __half* h, __nv_bfloat16* y, int32_t* err, cudaStream_t s) {
+  return launch_grouped_ffn_impl(nullptr, x, src, plan, L, W1, W3, W2, P1, P3, P2, T, k, E, R,
+                                 S, d, F, h, y, err, s);
 }
 
 }  // namespace moe

@@ -323,6 +323,7 @@ int launch_dispatch(const __nv_bfloat16* x, const int32_t* idx, const int32_t* p
     return MOE_ERR_LAUNCH;
   tile_rank_kernel<<<tiles, kPlaceTile, smem, s>>>(idx, T, k, E, R, C, ws, plan, L, perm, src, err);
   if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
+  if (recv == nullptr) return MOE_OK;  // index-only: the FFN gathers the rows itself
   scatter_rows_kernel<<<row_grid(T), kRowThreads, 0, s>>>(
       reinterpret_cast<const uint4*>(x), perm, T, k, d / 8, (int64_t)R * C,
       reinterpret_cast<uint4*>(recv), err);

@@ -61,8 +61,11 @@ class HostPipeline:
                 L.balance()
                 L.prefetch(W1, W3, W2)
                 L.dispatch(self.x[s])
-                self.inputs_free[s].record(self.s_comp)
+                if not L.fused:
+                    self.inputs_free[s].record(self.s_comp)
                 L.expert_ffn(W1, W3, W2)
+                if L.fused:  # the FFN gathered its rows from x
+                    self.inputs_free[s].record(self.s_comp)
                 if self._used[s]:
                     self.s_comp.wait_event(self.out_free[s])
                 moe_combine(L.y, L.perm, L.gate, self.out[s], L.err)

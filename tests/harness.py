@@ -36,10 +36,10 @@ def make_inputs(w: I.Workload, device="cuda"):
     return logits, x, (W1, W3, W2)
 
 
-def run_gpu(w: I.Workload, logits, x, weights, expert_to_rank=None):
+def run_gpu(w: I.Workload, logits, x, weights, expert_to_rank=None, fused=False):
     """All seven calls in order on the current stream; returns the layer (buffers)."""
     W1, W3, W2 = weights
-    L = M.MoELayer(w.T, w.E, w.k, w.R, w.S, w.d, w.F)
+    L = M.MoELayer(w.T, w.E, w.k, w.R, w.S, w.d, w.F, fused=fused)
     lg = logits.to("cuda")
     xd = x.to("cuda")
     L.forward(lg, xd, W1, W3, W2)
@@ -114,7 +114,8 @@ def expert_weights64(weights, e):
 def check_ffn_combine_full(L, w, x, weights, ref):
     """Every row of h and y, every token of out, against the fp64 oracle."""
     p = ref["plan"]
-    recv = to64(L.recv)
+    # the rows GEMM 1 reads: the dispatched copies, or (fused layer) the oracle's x[src]
+    recv = to64(L.recv) if L.recv is not None else to64(x)[ref["src"]]
     cache = {}
     h_ref = np.zeros((w.A, w.F))
     y_ref = np.zeros((w.A, w.d))
@@ -150,7 +151,10 @@ def check_ffn_combine_sampled(L, w, x, weights, ref, tokens):
                 if r0 <= r < r0 + n:
                     row_group[r] = e
     rows = sorted(want)
-    recv = to64(L.recv[torch.tensor(rows, device="cuda")])
+    if L.recv is not None:
+        recv = to64(L.recv[torch.tensor(rows, device="cuda")])
+    else:
+        recv = to64(x)[ref["src"][rows]]
     ridx = {r: i for i, r in enumerate(rows)}
     y_ref = {}
     by_e = {}

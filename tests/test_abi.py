@@ -27,6 +27,8 @@ def test_header_declares_the_path(lib):
     names = declared_functions()
     assert set(M.ENTRY_POINTS) <= names
     assert set(M.HELPERS) <= names
+    assert set(M.VARIANTS) <= names
+    assert set(M.FUSED) <= names
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -77,3 +79,24 @@ def test_host_checks_reject_bad_arguments(lib):
     assert lib.moe_combine(fake, fake, fake, 4, 33, 128, fake, fake, None) == M.MOE_ERR_SHAPE
     assert lib.moe_prefetch_replicas(fake, fake, fake, fake, 8, 4, 2, 128, 256, None, None, None, fake, None) == M.MOE_ERR_ARG
     assert lib.moe_status_string(M.MOE_ERR_SHAPE) == b"size limit violated"
+
+
+def test_fused_dispatch_host_checks(lib):
+    P = ctypes.c_void_p
+    fake = P(4096)
+    # index-only dispatch: null outputs, T*k % R != 0, E % R != 0
+    assert lib.moe_dispatch_index(fake, fake, 4, 2, 8, 4, 2, fake, fake, None, fake, None) == M.MOE_ERR_ARG
+    assert lib.moe_dispatch_index(fake, fake, 3, 1, 8, 2, 2, fake, fake, fake, fake, None) == M.MOE_ERR_SHAPE
+    assert lib.moe_dispatch_index(fake, fake, 4, 2, 8, 3, 2, fake, fake, fake, fake, None) == M.MOE_ERR_SHAPE
+    # gathered FFN: null x or src, F % 128 != 0, misaligned x, missing pool
+    args = [fake, fake, fake, fake, fake, fake, fake, fake, fake, 4, 2, 8, 4, 2, 128, 256, fake, fake, fake, None]
+    bad = list(args); bad[0] = None
+    assert lib.moe_grouped_ffn_gather(*bad) == M.MOE_ERR_ARG
+    bad = list(args); bad[1] = None
+    assert lib.moe_grouped_ffn_gather(*bad) == M.MOE_ERR_ARG
+    bad = list(args); bad[15] = 200
+    assert lib.moe_grouped_ffn_gather(*bad) == M.MOE_ERR_SHAPE
+    bad = list(args); bad[0] = P(4098)
+    assert lib.moe_grouped_ffn_gather(*bad) == M.MOE_ERR_ARG
+    bad = list(args); bad[6] = None
+    assert lib.moe_grouped_ffn_gather(*bad) == M.MOE_ERR_ARG
