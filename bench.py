@@ -39,7 +39,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) per call of the dominant call (both grouped-FFN kernels) from
 # an ncu capture (profiles/ffn_kernel_near_balanced.md), keyed by workload and kernel
 # sources hash: it reads null as soon as the kernel sources change.
-TRAFFIC = {"near_balanced:cff503e0c0d3a439": int((936.090624 + 65.056768 + 478.813952 + 84.740608) * 1e6)}
+TRAFFIC = {"near_balanced:bd5310e6636697e2": int((921.992960 + 63.940864 + 478.845952 + 84.311296) * 1e6)}
 
 
 def sources_hash() -> str:
