@@ -39,6 +39,10 @@ Pins (tests/test_oracle_pins.py checks each against something other than this fi
                     silu(1) = e/(1+e); transposed operands land in distinct outputs
   combine           identity experts return x (gates sum to one); per-expert scaling
                     returns (sum_j gate_j c_e) x
+  layer_backward    central finite differences of layer() itself (fp64, tiny shapes,
+                    away from top-k ties); torch.autograd (fp64, CPU) through a token-major
+                    formulation with no plan, dispatch or replicas; the weight gradients do
+                    not depend on S (replicas reduced back home)
 
 Error bits (OR-ed): 1 non-finite logit, 2 expert id out of range, 4 repeated expert
 within one token, 8 plan needs more than S replicas on some rank.
@@ -462,3 +466,130 @@ def layer(logits, x, W1, W3, W2, k: int, R: int, S: int):
     return dict(idx=idx, gate=gate, hist=h, plan=plan, pool=pool, perm=perm, src=src,
                 recv=recv, y=y, out=out, err=err)
 
+
+
+# ------------------------------------------------------------------ backward pass
+# [MoonEP] para. 3: the duplicated experts' "gradients get reduced back home during the
+# backward pass".  The pages give no formulas; these are the chain rule through the
+# forward above, with the reading that top-k selection passes no gradient to the
+# experts it did not choose (it is piecewise constant in the logits).
+
+def silu_grad(z):
+    """d silu / dz = sigmoid(z) * (1 + z * (1 - sigmoid(z))), fp64."""
+    z = np.asarray(z, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        s = 1.0 / (1.0 + np.exp(-z))
+    return s * (1.0 + z * (1.0 - s))
+
+
+def combine_backward(dout, y, perm, gate):
+    """Backward of combine: out[t] = sum_j gate[t,j] y[perm[t,j]], so
+    dy[perm[t,j]] = gate[t,j] dout[t] and dgate[t,j] = <dout[t], y[perm[t,j]]>."""
+    dout = np.asarray(dout, dtype=np.float64)
+    y = np.asarray(y, dtype=np.float64)
+    perm = np.asarray(perm)
+    gate = np.asarray(gate, dtype=np.float64)
+    T, k = perm.shape
+    dy = np.zeros_like(y)
+    dgate = np.zeros((T, k))
+    for t in range(T):
+        for j in range(k):
+            r = int(perm[t, j])
+            dy[r] = gate[t, j] * dout[t]
+            dgate[t, j] = float(dout[t] @ y[r])
+    return dy, dgate
+
+
+def expert_ffn_backward(X, w1, w3, w2, dy):
+    """Backward of one SwiGLU expert on a block of rows, fp64.  Forward: g = X w1^T,
+    u = X w3^T, h = silu(g) u, y = h w2^T.  Returns the row gradient dX and the weight
+    gradients of this block, plus the intermediates dh, dg, du."""
+    X = np.asarray(X, dtype=np.float64)
+    w1 = np.asarray(w1, dtype=np.float64)
+    w3 = np.asarray(w3, dtype=np.float64)
+    w2 = np.asarray(w2, dtype=np.float64)
+    dy = np.asarray(dy, dtype=np.float64)
+    g = X @ w1.T
+    u = X @ w3.T
+    sg = silu(g)
+    h = sg * u
+    dh = dy @ w2              # [n,F]
+    dw2 = dy.T @ h            # [d,F]
+    du = dh * sg
+    dg = dh * u * silu_grad(g)
+    dX = dg @ w1 + du @ w3    # [n,d]
+    dw1 = dg.T @ X            # [F,d]
+    dw3 = du.T @ X
+    return dict(dX=dX, dw1=dw1, dw3=dw3, dw2=dw2, dh=dh, dg=dg, du=du, h=h)
+
+
+def grouped_ffn_backward(recv, dy, plan, E: int, W1, W3, W2, pool):
+    """Backward of the grouped FFN: every group's rows through its expert's backward.
+    A replica slot holds its expert's weights bitwise, and the gradient of every group --
+    home or replica -- is added to its expert's home gradient ([MoonEP] para. 3: replica
+    gradients are reduced back home).  Returns dX rows [R*C,d], dW1, dW3 [E,F,d], dW2
+    [E,d,F] and the per-row intermediates dh, dg, du [R*C,F]."""
+    recv = np.asarray(recv, dtype=np.float64)
+    dy = np.asarray(dy, dtype=np.float64)
+    rows, d = recv.shape
+    F = W1.shape[1]
+    dX = np.zeros((rows, d))
+    dh = np.zeros((rows, F))
+    dg = np.zeros((rows, F))
+    du = np.zeros((rows, F))
+    dW1 = np.zeros((E, F, d))
+    dW3 = np.zeros((E, F, d))
+    dW2 = np.zeros((E, d, F))
+    for u_groups in plan["groups"]:
+        for (r0, n, e, ref) in u_groups:
+            w1, w3, w2 = weights_of(ref, E, W1, W3, W2, pool)
+            b = expert_ffn_backward(recv[r0:r0 + n], w1, w3, w2, dy[r0:r0 + n])
+            dX[r0:r0 + n] = b["dX"]
+            dh[r0:r0 + n] = b["dh"]
+            dg[r0:r0 + n] = b["dg"]
+            du[r0:r0 + n] = b["du"]
+            dW1[e] += b["dw1"]
+            dW3[e] += b["dw3"]
+            dW2[e] += b["dw2"]
+    return dict(dX=dX, dW1=dW1, dW3=dW3, dW2=dW2, dh=dh, dg=dg, du=du)
+
+
+def dispatch_backward(dX, perm):
+    """Backward of dispatch (recv[perm[t,j]] = x[t]): dx[t] = sum_j dX[perm[t,j]], in j
+    order."""
+    dX = np.asarray(dX, dtype=np.float64)
+    perm = np.asarray(perm)
+    T, k = perm.shape
+    dx = np.zeros((T, dX.shape[1]))
+    for t in range(T):
+        for j in range(k):
+            dx[t] += dX[int(perm[t, j])]
+    return dx
+
+
+def topk_backward(gate, dgate, idx, E: int):
+    """Backward of the gates: gate = softmax over the chosen logits, so
+    dlogit[t, idx[t,j]] = gate[t,j] (dgate[t,j] - sum_i gate[t,i] dgate[t,i]); experts not
+    chosen get 0 (the selection itself passes no gradient)."""
+    gate = np.asarray(gate, dtype=np.float64)
+    dgate = np.asarray(dgate, dtype=np.float64)
+    idx = np.asarray(idx)
+    T, k = idx.shape
+    dl = np.zeros((T, E))
+    for t in range(T):
+        s = float(gate[t] @ dgate[t])
+        for j in range(k):
+            dl[t, int(idx[t, j])] = gate[t, j] * (dgate[t, j] - s)
+    return dl
+
+
+def layer_backward(fwd, dout, W1, W3, W2, E: int):
+    """The backward of layer() given its outputs ``fwd`` and dout = dLoss/dout [T,d]:
+    combine, expert FFN (replica gradients reduced home), dispatch, gates.  Returns dx
+    [T,d], dlogits [T,E], dW1, dW3, dW2 and the intermediates."""
+    dy, dgate = combine_backward(dout, fwd["y"], fwd["perm"], fwd["gate"])
+    g = grouped_ffn_backward(fwd["recv"], dy, fwd["plan"], E, W1, W3, W2, fwd["pool"])
+    dx = dispatch_backward(g["dX"], fwd["perm"])
+    dlogits = topk_backward(fwd["gate"], dgate, fwd["idx"], E)
+    return dict(dx=dx, dlogits=dlogits, dW1=g["dW1"], dW3=g["dW3"], dW2=g["dW2"], dy=dy,
+                dgate=dgate, dX_rows=g["dX"], dh=g["dh"], dg=g["dg"], du=g["du"])
