@@ -365,7 +365,100 @@ def run_ours(args, w: I.Workload, world, rank, local):
         "roofline": roofline,
         "calls": calls,
     }
+    if args.backward:
+        res["train_step"] = time_training_step(args, w, L, logits, x, W1, W3, W2, world, device, peaks)
     return res
+
+
+BWD_CALLS = ["moe_combine_backward", "moe_grouped_ffn_backward", "moe_dispatch_backward",
+             "moe_topk_backward"]
+
+
+def time_training_step(args, w: I.Workload, L, logits, x, W1, W3, W2, world, device, peaks):
+    """Forward + backward of the layer (dout seeded N(0,1) bf16), K steps in one CUDA graph
+    after warm-up; per-call backward intervals from a replay with event nodes between the
+    calls.  The grouped-FFN backward does 16*A*d*F flops: dH (2AdF), the gate/up GEMM re-run
+    (4AdF), dX rows (4AdF), dW2 (2AdF), dW1 and dW3 (4AdF)."""
+    g = torch.Generator().manual_seed(41)
+    dout = torch.randn(w.T, w.d, generator=g).to(torch.bfloat16).to(device)
+    for _ in range(max(args.warmup, 1)):
+        L.forward(logits, x, W1, W3, W2)
+        L.backward(dout, W1, W3, W2)
+    torch.cuda.synchronize()
+    if int(L.err.item()) != 0:
+        raise RuntimeError(f"device error word {int(L.err.item())} after the backward warm-up")
+    import load_balanced_dispatch_warp_b200 as M
+    b = L._bwd
+    bsteps = [lambda: M.moe_combine_backward(dout, L.y, L.perm, L.gate, b["dy"], b["dgate"], L.err),
+              lambda: M.moe_grouped_ffn_backward(L.recv, b["dy"], L.h, L.plan, W1, W3, W2, L.T, L.k, L.R,
+                                                 L.S, b["dx_rows"], b["dW1"], b["dW3"], b["dW2"],
+                                                 b["workspace"], L.err),
+              lambda: M.moe_dispatch_backward(b["dx_rows"], L.perm, b["dx"], L.err),
+              lambda: M.moe_topk_backward(L.gate, b["dgate"], L.idx, L.E, b["dlogits"], L.err)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(bsteps) + 1)] for _ in range(args.steps)]
+    for row in ev:
+        for e in row:
+            e.record()
+    torch.cuda.synchronize()
+    rt = cudart()
+
+    def rec_node(event, st):
+        rc = rt.cudaEventRecordWithFlags(ctypes.c_void_p(event.cuda_event), ctypes.c_void_p(st.cuda_stream), 1)
+        if rc != 0:
+            raise RuntimeError(f"cudaEventRecordWithFlags failed ({rc})")
+
+    def capture(with_events):
+        gr = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(device)
+        cap.wait_stream(torch.cuda.current_stream(device))
+        torch.cuda.synchronize()
+        with torch.cuda.stream(cap):
+            gr.capture_begin()
+            for st in range(args.steps):
+                L.forward(logits, x, W1, W3, W2)
+                if with_events:
+                    rec_node(ev[st][0], cap)
+                for i, f in enumerate(bsteps):
+                    f()
+                    if with_events:
+                        rec_node(ev[st][i + 1], cap)
+            gr.capture_end()
+        torch.cuda.synchronize()
+        gr.replay()
+        torch.cuda.synchronize()
+        return gr
+
+    clean = capture(False)
+    inst = capture(True)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    stream = torch.cuda.current_stream(device)
+    t0.record(stream)
+    clean.replay()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(t0.elapsed_time(t1), world, device)
+    inst.replay()
+    torch.cuda.synchronize()
+    if int(L.err.item()) != 0:
+        raise RuntimeError(f"device error word {int(L.err.item())} in the timed training steps")
+    del clean, inst
+    per = {c: sum(ev[st][i].elapsed_time(ev[st][i + 1]) for st in range(args.steps)) / args.steps
+           for i, c in enumerate(BWD_CALLS)}
+    A, d, F = w.A, w.d, w.F
+    ffn_flops = 16 * A * d * F
+    peak_t = peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]
+    calls = {c: {"us": round(v * 1e3, 2)} for c, v in per.items()}
+    t_ffn = per["moe_grouped_ffn_backward"] * 1e-3
+    calls["moe_grouped_ffn_backward"].update(
+        {"TFLOP_per_s": round(ffn_flops / t_ffn / 1e12, 1), "frac": round(ffn_flops / t_ffn / 1e12 / peak_t, 3),
+         "work": f"16*A*d*F = {ffn_flops:.4g} flop"})
+    return {"value": round(w.T * args.steps * world / (ms * 1e-3), 1), "unit": "tokens/s",
+            "ms_per_step": round(ms / args.steps, 4),
+            "what": "forward + backward (dx, dlogits, dW1, dW3, dW2) per step, K steps in one CUDA graph",
+            "backward_calls": calls}
 
 
 # ----------------------------------------------------------------------------- oracle
@@ -472,6 +565,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="launch the timed steps eagerly")
+    ap.add_argument("--backward", action="store_true",
+                    help="also time the training step (forward + backward) and the backward calls")
     ap.add_argument("--fused", action="store_true",
                     help="fused dispatch: placement only, GEMM 1 gathers the token rows")
     args = ap.parse_args()

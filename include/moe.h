@@ -268,6 +268,57 @@ int moe_grouped_ffn_gather(const moe_bf16* x, const int32_t* src, const int32_t*
                            int32_t* err, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * Backward pass.   [MoonEP] para. 3: the duplicated experts' gradients are reduced back
+ * home during the backward pass.  The pages give no formulas; these calls apply the
+ * chain rule to the forward above, reading top-k selection as passing no gradient to the
+ * experts it did not choose.  dout = dLoss/dout [T,d] bf16.  Same buffers, layouts and
+ * error word as the forward; each call is a no-op when *err is non-zero.
+ *
+ * moe_combine_backward: dy[perm[t,j]] = gate[t,j] * dout[t] (bf16: its exponent range keeps
+ *   the rows of small gates) and dgate[t,j] = <dout[t], y[perm[t,j]]> (fp32).
+ *   dout [T,d] bf16; y [R*C,d] bf16 (forward output rows); dy [R*C,d] bf16 (out);
+ *   dgate [T,k] fp32 (out).
+ */
+int moe_combine_backward(const moe_bf16* dout, const moe_bf16* y, const int32_t* perm,
+                         const float* gate, int T, int k, int d, moe_bf16* dy, float* dgate,
+                         const int32_t* err, moe_stream_t stream);
+/*
+ * moe_grouped_ffn_backward: for every plan group (rows of one rank, expert e; a replica
+ * slot's rows use their expert's home weights, bitwise the same values):
+ *   dH = dY W2,  dG = dH * u * silu'(g),  dU = dH * silu(g)   (g = X W1^T, u = X W3^T
+ *   recomputed from recv), dX = dG W1 + dU W3;
+ *   dW2[e] = sum over ALL groups of e (home and replica) of dY^T h, dW1[e] = sum dG^T X,
+ *   dW3[e] = sum dU^T X -- replica gradients reduced home; experts without rows get 0.
+ *   recv [R*C,d] bf16 (from moe_dispatch); dy [R*C,d] bf16 (moe_combine_backward);
+ *   h [R*C,F] fp16 (from moe_grouped_ffn); W1, W3 [E,F,d] bf16; W2 [E,d,F] fp16.
+ *   All GEMMs run in bf16 with fp32 accumulation: W2 and h are rounded to bf16 on the way
+ *   into the transposed operands (exact for W2 values that are bf16 numbers).
+ *   dx_rows [R*C,d] bf16 (out); dW1, dW3 [E,F,d] fp32 (out); dW2 [E,d,F] fp32 (out).
+ *   workspace: caller-owned device scratch of moe_ffn_backward_workspace_bytes(...) bytes,
+ *   256-byte aligned (transposed weights and activations, dH fp32, dG|dU bf16).
+ *   Returns MOE_ERR_ARG if workspace_bytes is too small.  Persistent tcgen05 kernels:
+ *   dH, dG|dU (the gate/up GEMM re-run with a SwiGLU-backward epilogue), dX rows, and one
+ *   weight-gradient GEMM per projection whose K loop runs over the zero-padded 64-row
+ *   segments of every group of the expert.
+ */
+int64_t moe_ffn_backward_workspace_bytes(int T, int k, int E, int R, int S, int d, int F);
+int moe_grouped_ffn_backward(const moe_bf16* recv, const moe_bf16* dy, const moe_f16* h,
+                             const int32_t* plan, const moe_bf16* W1, const moe_bf16* W3,
+                             const moe_f16* W2, int T, int k, int E, int R, int S, int d, int F,
+                             moe_bf16* dx_rows, float* dW1, float* dW3, float* dW2,
+                             void* workspace, int64_t workspace_bytes, int32_t* err,
+                             moe_stream_t stream);
+/*
+ * moe_dispatch_backward: dx[t] = sum_j dx_rows[perm[t,j]] (fp32 accumulate, bf16 out).
+ * moe_topk_backward: dlogits[t, idx[t,j]] = gate[t,j] (dgate[t,j] - sum_i gate[t,i]
+ *   dgate[t,i]); every other entry of the row 0.  dlogits [T,E] fp32 (out).
+ */
+int moe_dispatch_backward(const moe_bf16* dx_rows, const int32_t* perm, int T, int k, int d,
+                          moe_bf16* dx, const int32_t* err, moe_stream_t stream);
+int moe_topk_backward(const float* gate, const float* dgate, const int32_t* idx, int T, int E,
+                      int k, float* dlogits, const int32_t* err, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
  * Dispatch without a workspace argument.  The pages have no counterpart: this is a
  * convenience of this library for callers that cannot allocate device memory when they
  * dispatch -- an operator or plugin interface of another runtime that passes only its

@@ -28,6 +28,8 @@ ENTRY_POINTS = ("moe_topk", "moe_histogram_maxvio", "moe_plan_balanced", "moe_pr
                 "moe_dispatch", "moe_grouped_ffn", "moe_combine")
 VARIANTS = ("moe_topk_biased", "moe_capacity_ledger")
 FUSED = ("moe_dispatch_index", "moe_grouped_ffn_gather")
+BACKWARD = ("moe_combine_backward", "moe_grouped_ffn_backward", "moe_dispatch_backward",
+            "moe_topk_backward")
 HELPERS = ("moe_plan_get_layout", "moe_dispatch_workspace_words", "moe_status_string")
 
 
@@ -68,6 +70,11 @@ def lib() -> ctypes.CDLL:
             "moe_selftest_bounded_wait": [P, I, P],
             "moe_dispatch_index": [P, P, I, I, I, I, I, P, P, P, P, P],
             "moe_grouped_ffn_gather": [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, P],
+            "moe_combine_backward": [P, P, P, P, I, I, I, P, P, P, P],
+            "moe_grouped_ffn_backward": [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, P, P,
+                                         I64, P, P],
+            "moe_dispatch_backward": [P, P, I, I, I, P, P, P],
+            "moe_topk_backward": [P, P, P, I, I, I, P, P, P],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -77,6 +84,8 @@ def lib() -> ctypes.CDLL:
         L.moe_plan_get_layout.restype = ctypes.c_int
         L.moe_dispatch_workspace_words.argtypes = [I, I]
         L.moe_dispatch_workspace_words.restype = I64
+        L.moe_ffn_backward_workspace_bytes.argtypes = [I, I, I, I, I, I, I]
+        L.moe_ffn_backward_workspace_bytes.restype = I64
         L.moe_status_string.argtypes = [I]
         L.moe_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -245,6 +254,54 @@ def moe_combine(y, perm, gate, out, err, stream=None):
                              _stream(stream)), "moe_combine")
 
 
+# ----------------------------------------------------------------- backward pass
+def ffn_backward_workspace_bytes(T, k, E, R, S, d, F) -> int:
+    n = int(lib().moe_ffn_backward_workspace_bytes(T, k, E, R, S, d, F))
+    if n < 0:
+        raise MoEError("moe_ffn_backward_workspace_bytes: invalid shape")
+    return n
+
+
+def moe_combine_backward(dout, y, perm, gate, dy, dgate, err, stream=None):
+    T, k = perm.shape
+    d = dout.shape[1]
+    _check(lib().moe_combine_backward(
+        _ptr(dout, torch.bfloat16, "dout"), _ptr(y, torch.bfloat16, "y"), _ptr(perm, torch.int32, "perm"),
+        _ptr(gate, torch.float32, "gate"), T, k, d, _ptr(dy, torch.bfloat16, "dy"),
+        _ptr(dgate, torch.float32, "dgate"), _ptr(err, torch.int32, "err"), _stream(stream)),
+        "moe_combine_backward")
+
+
+def moe_grouped_ffn_backward(recv, dy, h, plan, W1, W3, W2, T, k, R, S, dx_rows, dW1, dW3, dW2,
+                             workspace, err, stream=None):
+    E, F, d = W1.shape
+    bf, hf, f32 = torch.bfloat16, torch.float16, torch.float32
+    _check(lib().moe_grouped_ffn_backward(
+        _ptr(recv, bf, "recv"), _ptr(dy, bf, "dy"), _ptr(h, hf, "h"), _ptr(plan, torch.int32, "plan"),
+        _ptr(W1, bf, "W1"), _ptr(W3, bf, "W3"), _ptr(W2, hf, "W2"), T, k, E, R, S, d, F,
+        _ptr(dx_rows, bf, "dx_rows"), _ptr(dW1, f32, "dW1"), _ptr(dW3, f32, "dW3"),
+        _ptr(dW2, f32, "dW2"), _ptr(workspace, torch.uint8, "workspace"),
+        workspace.numel() if workspace is not None else 0, _ptr(err, torch.int32, "err"),
+        _stream(stream)), "moe_grouped_ffn_backward")
+
+
+def moe_dispatch_backward(dx_rows, perm, dx, err, stream=None):
+    T, k = perm.shape
+    d = dx.shape[1]
+    _check(lib().moe_dispatch_backward(
+        _ptr(dx_rows, torch.bfloat16, "dx_rows"), _ptr(perm, torch.int32, "perm"), T, k, d,
+        _ptr(dx, torch.bfloat16, "dx"), _ptr(err, torch.int32, "err"), _stream(stream)),
+        "moe_dispatch_backward")
+
+
+def moe_topk_backward(gate, dgate, idx, E, dlogits, err, stream=None):
+    T, k = idx.shape
+    _check(lib().moe_topk_backward(
+        _ptr(gate, torch.float32, "gate"), _ptr(dgate, torch.float32, "dgate"),
+        _ptr(idx, torch.int32, "idx"), T, E, k, _ptr(dlogits, torch.float32, "dlogits"),
+        _ptr(err, torch.int32, "err"), _stream(stream)), "moe_topk_backward")
+
+
 # ----------------------------------------------------------------- one layer
 class MoELayer:
     """Device buffers of one MoE layer of shape (T, E, k, R, S, d, F) and the seven calls.
@@ -343,6 +400,36 @@ class MoELayer:
         self.expert_ffn(W1, W3, W2, stream)
         self.combine(stream)
         return self.out
+
+    def backward(self, dout, W1, W3, W2, stream=None):
+        """Backward of the last forward() (unfused layers: it reads recv, y and h):
+        dout [T,d] bf16 -> dict(dx [T,d] bf16, dlogits [T,E] fp32, dW1, dW3 [E,F,d] fp32,
+        dW2 [E,d,F] fp32).  Buffers are allocated on first use and reused."""
+        if self.fused:
+            raise RuntimeError("backward needs the dispatched rows: use an unfused layer")
+        if not hasattr(self, "_bwd"):
+            dev = self.idx.device
+            T, E, k, d, F, A = self.T, self.E, self.k, self.d, self.F, self.A
+            f32 = torch.float32
+            ws = ffn_backward_workspace_bytes(T, k, E, self.R, self.S, d, F)
+            self._bwd = dict(
+                dy=torch.empty(A, d, dtype=torch.bfloat16, device=dev),
+                dgate=torch.empty(T, k, dtype=f32, device=dev),
+                dx_rows=torch.empty(A, d, dtype=torch.bfloat16, device=dev),
+                dx=torch.empty(T, d, dtype=torch.bfloat16, device=dev),
+                dlogits=torch.empty(T, E, dtype=f32, device=dev),
+                dW1=torch.empty(E, F, d, dtype=f32, device=dev),
+                dW3=torch.empty(E, F, d, dtype=f32, device=dev),
+                dW2=torch.empty(E, d, F, dtype=f32, device=dev),
+                workspace=torch.empty(max(ws, 256), dtype=torch.uint8, device=dev))
+        b = self._bwd
+        moe_combine_backward(dout, self.y, self.perm, self.gate, b["dy"], b["dgate"], self.err, stream)
+        moe_grouped_ffn_backward(self.recv, b["dy"], self.h, self.plan, W1, W3, W2, self.T, self.k,
+                                 self.R, self.S, b["dx_rows"], b["dW1"], b["dW3"], b["dW2"],
+                                 b["workspace"], self.err, stream)
+        moe_dispatch_backward(b["dx_rows"], self.perm, b["dx"], self.err, stream)
+        moe_topk_backward(self.gate, b["dgate"], self.idx, self.E, b["dlogits"], self.err, stream)
+        return b
 
     # kernels launched by forward() (for launch accounting)
     def kernels_per_forward(self) -> int:

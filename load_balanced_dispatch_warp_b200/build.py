@@ -17,7 +17,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libmoe.so")
-SOURCES = ["abi.cu", "route.cu", "plan.cu", "move.cu", "grouped_ffn.cu", "dispatch_noalloc.cu"]
+SOURCES = ["abi.cu", "route.cu", "plan.cu", "move.cu", "grouped_ffn.cu", "grouped_ffn_bwd.cu",
+           "dispatch_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

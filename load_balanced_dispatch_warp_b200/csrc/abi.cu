@@ -279,6 +279,79 @@ int moe_combine(const moe_bf16* y, const int32_t* perm, const float* gate, int T
                              reinterpret_cast<__nv_bfloat16*>(out), err, as_stream(stream));
 }
 
+int moe_combine_backward(const moe_bf16* dout, const moe_bf16* y, const int32_t* perm,
+                         const float* gate, int T, int k, int d, moe_bf16* dy, float* dgate,
+                         const int32_t* err, moe_stream_t stream) {
+  if (!err) return MOE_ERR_ARG;
+  if (T > 0 && (!dout || !y || !perm || !gate || !dy || !dgate)) return MOE_ERR_ARG;
+  if (T < 0 || k < 1) return MOE_ERR_ARG;
+  if (k > 32) return MOE_ERR_SHAPE;
+  MOE_TRY(check_dims(T, k, d, 128));
+  if (!aligned16(dout) || !aligned16(y) || !aligned16(dy)) return MOE_ERR_ARG;
+  return moe::launch_combine_backward(reinterpret_cast<const __nv_bfloat16*>(dout),
+                                      reinterpret_cast<const __nv_bfloat16*>(y), perm, gate, T,
+                                      k, d, reinterpret_cast<__nv_bfloat16*>(dy), dgate, err,
+                                      as_stream(stream));
+}
+
+int moe_dispatch_backward(const moe_bf16* dx_rows, const int32_t* perm, int T, int k, int d,
+                          moe_bf16* dx, const int32_t* err, moe_stream_t stream) {
+  if (!err) return MOE_ERR_ARG;
+  if (T > 0 && (!dx_rows || !perm || !dx)) return MOE_ERR_ARG;
+  if (T < 0 || k < 1) return MOE_ERR_ARG;
+  if (k > 32) return MOE_ERR_SHAPE;
+  MOE_TRY(check_dims(T, k, d, 128));
+  if (!aligned16(dx_rows) || !aligned16(dx)) return MOE_ERR_ARG;
+  return moe::launch_combine(reinterpret_cast<const __nv_bfloat16*>(dx_rows), perm, nullptr, T,
+                             k, d, reinterpret_cast<__nv_bfloat16*>(dx), err, as_stream(stream));
+}
+
+int moe_topk_backward(const float* gate, const float* dgate, const int32_t* idx, int T, int E,
+                      int k, float* dlogits, const int32_t* err, moe_stream_t stream) {
+  if (!err) return MOE_ERR_ARG;
+  if (T > 0 && (!gate || !dgate || !idx || !dlogits)) return MOE_ERR_ARG;
+  MOE_TRY(check_route(T, E, k));
+  return moe::launch_topk_backward(gate, dgate, idx, T, E, k, dlogits, err, as_stream(stream));
+}
+
+int64_t moe_ffn_backward_workspace_bytes(int T, int k, int E, int R, int S, int d, int F) {
+  if (T < 0 || k < 1 || E < 1 || R < 1 || S < 0 || d < 1 || F < 1 || E % R != 0) return -1;
+  moe_plan_layout L;
+  if (moe_plan_get_layout(E, R, S, &L) != MOE_OK) return -1;
+  return moe::ffn_backward_workspace_bytes(T, k, E, R, S, d, F, R * L.max_groups_per_rank);
+}
+
+int moe_grouped_ffn_backward(const moe_bf16* recv, const moe_bf16* dy, const moe_f16* h,
+                             const int32_t* plan, const moe_bf16* W1, const moe_bf16* W3,
+                             const moe_f16* W2, int T, int k, int E, int R, int S, int d, int F,
+                             moe_bf16* dx_rows, float* dW1, float* dW3, float* dW2,
+                             void* workspace, int64_t workspace_bytes, int32_t* err,
+                             moe_stream_t stream) {
+  if (!plan || !W1 || !W3 || !W2 || !err || !dW1 || !dW3 || !dW2) return MOE_ERR_ARG;
+  if (T > 0 && (!recv || !dy || !h || !dx_rows || !workspace)) return MOE_ERR_ARG;
+  MOE_TRY(check_route(T, E, k));
+  MOE_TRY(check_ranks(T, k, E, R, true));
+  MOE_TRY(check_groups(E, R, S));
+  MOE_TRY(check_dims(T, k, d, F));
+  if ((int64_t)E * F >= kMaxElems || (int64_t)E * d >= kMaxElems) return MOE_ERR_SHAPE;
+  if ((int64_t)T * k * 2 * F >= kMaxElems) return MOE_ERR_SHAPE;
+  if (!aligned16(recv) || !aligned16(dy) || !aligned16(h) || !aligned16(dx_rows) ||
+      !aligned16(W1) || !aligned16(W3) || !aligned16(W2) || !aligned16(dW1) || !aligned16(dW3) ||
+      !aligned16(dW2) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return MOE_ERR_ARG;
+  moe_plan_layout L;
+  MOE_TRY(moe_plan_get_layout(E, R, S, &L));
+  if (moe::ffn_backward_workspace_bytes(T, k, E, R, S, d, F, R * L.max_groups_per_rank) >
+      workspace_bytes)
+    return MOE_ERR_ARG;
+  return moe::launch_grouped_ffn_backward(
+      reinterpret_cast<const __nv_bfloat16*>(recv), reinterpret_cast<const __nv_bfloat16*>(dy),
+      reinterpret_cast<const __half*>(h), plan, L, reinterpret_cast<const __nv_bfloat16*>(W1),
+      reinterpret_cast<const __nv_bfloat16*>(W3), reinterpret_cast<const __half*>(W2), T, k, E,
+      R, S, d, F, reinterpret_cast<__nv_bfloat16*>(dx_rows), dW1, dW3, dW2, workspace,
+      workspace_bytes, err, as_stream(stream));
+}
+
 int moe_selftest_bounded_wait(int32_t* err, int limit_us, moe_stream_t stream) {
   if (!err || limit_us < 1 || limit_us > 10000000) return MOE_ERR_ARG;
   return moe::launch_bounded_wait_selftest(err, limit_us, as_stream(stream));

@@ -56,6 +56,23 @@ int launch_grouped_ffn_gather(const __nv_bfloat16* x, const int32_t* src, const 
                               const __half* P2, int T, int k, int E, int R, int S, int d, int F,
                               __half* h, __nv_bfloat16* y, int32_t* err, cudaStream_t s);
 int launch_bounded_wait_selftest(int32_t* err, int limit_us, cudaStream_t s);
+// backward pass (grouped_ffn_bwd.cu; the dispatch backward is launch_combine with
+// gate == nullptr)
+int64_t ffn_backward_workspace_bytes(int T, int k, int E, int R, int S, int d, int F, int G);
+int launch_combine_backward(const __nv_bfloat16* dout, const __nv_bfloat16* y,
+                            const int32_t* perm, const float* gate, int T, int k, int d,
+                            __nv_bfloat16* dy, float* dgate, const int32_t* err,
+                            cudaStream_t s);
+int launch_topk_backward(const float* gate, const float* dgate, const int32_t* idx, int T, int E,
+                         int k, float* dlogits, const int32_t* err, cudaStream_t s);
+int launch_grouped_ffn_backward(const __nv_bfloat16* recv, const __nv_bfloat16* dy,
+                                const __half* h,
+                                const int32_t* plan, const moe_plan_layout& L,
+                                const __nv_bfloat16* W1, const __nv_bfloat16* W3,
+                                const __half* W2, int T, int k, int E, int R, int S, int d,
+                                int F, __nv_bfloat16* dx_rows, float* dW1, float* dW3,
+                                float* dW2, void* workspace, int64_t workspace_bytes,
+                                int32_t* err, cudaStream_t s);
 int launch_combine(const __nv_bfloat16* y, const int32_t* perm, const float* gate, int T,
                    int k, int d, __nv_bfloat16* out, const int32_t* err, cudaStream_t s);
 

@@ -1,0 +1,949 @@
+// Backward pass of the MoE layer's expert path (sm_100a).
+//
+// The MoonEP news article (paragraph 3): the duplicated experts' "gradients get reduced
+// back home during the backward pass".  With dy = dLoss/dy for every row of the per-rank
+// buffers (moe_combine_backward), each plan group (rows r0..r0+n of one rank, expert e)
+// runs the chain rule of its SwiGLU expert (forward g = X W1^T, u = X W3^T,
+// h = silu(g) u, y = h W2^T):
+//   dH  = dY W2                    [rows, F]   GEMM, bf16 x bf16 -> fp32
+//   dG  = dH * u * silu'(g),  dU = dH * silu(g)
+//                                  [rows, F]   the gate/up GEMM re-run on the rows, with
+//                                              an epilogue that reads dH (no saved g, u)
+//   dX  = dG W1 + dU W3            [rows, d]   GEMM over K = 2F, bf16
+//   dW2[e] += dY^T h, dW1[e] += dG^T X, dW3[e] += dU^T X
+//                                              GEMMs over the rows of every group of
+//                                              expert e -- home and replica groups in one
+//                                              accumulator: the reduction back home
+// All GEMMs run on one persistent tcgen05 kernel (TMA-fed 4-stage ring, TMEM double
+// buffer, one MMA thread, four epilogue warps) with three epilogues, in bf16: dY is bf16
+// because gate * dout spans the gates' range (fp16 would lose small gates to subnormals),
+// and the fp16 operands it meets (W2, the forward's h) are converted to bf16 by the
+// transposes below.  Every GEMM reads
+// K-major operands, so the operands whose contraction runs along a stored row (W2, W1, W3
+// for the data gradients; dY, h, dG, dU and X for the weight gradients) are first
+// transposed by an HBM-bound kernel; the transposed activations give every group a
+// segment of whole 64-row K steps, zero-padded, so no K step mixes two groups.
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int UMMA_K = 16;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES_MAX = 256 * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES_MAX;
+constexpr int ACC_COLS = 256;
+constexpr int TMEM_COLS = 2 * ACC_COLS;
+constexpr int MAX_GROUPS = 4096;
+constexpr int BWD_THREADS = 192;
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
+
+enum { EPI_BF16 = 0, EPI_F32 = 1, EPI_SWIGLU_BWD = 2 };
+
+struct BwdArgs {
+  const int4* groups;   // plan group records {row_start, rows, expert, weight_ref}
+  int G;
+  int n_blocks_n;       // output column blocks
+  int k_blocks;         // K / BK (row tiles)
+  int bn_out;           // output columns per tile
+  int mma_n;            // N of the MMA (256 with two B halves for the SwiGLU backward)
+  int rows_per_expert;  // rows of one expert in the B tensor (row tiles)
+  int out_ld;           // columns of the output tensor
+  int bf16;             // operand type: 1 bf16, 0 fp16
+  void* out;
+  int32_t* err;
+  // SwiGLU backward epilogue: reads dH [rows, F] fp32, writes dG | dU into dGU [rows, 2F]
+  const float* dh;
+  __nv_bfloat16* dgu;
+  int F;
+  // weight-gradient tiles: (expert, m block, n block), K over the expert's segments
+  const int* seg_off;   // [E+1]
+  const int2* segs;     // {first K step, K steps}
+  int m_blocks;
+  int a_row_base;
+  int64_t out_expert_stride;
+  int E;
+};
+
+// ------------------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait (about 2 s of %globaltimer); false if it ran out or another role aborted.
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                       int32_t* err) {
+  if (mbar_try(bar, parity)) return true;
+  uint64_t t0 = 0;
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try(bar, parity)) return true;
+    if ((it & 255u) == 0) {
+      if (*abort_flag) return false;
+      const uint64_t now = globaltimer();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > WAIT_LIMIT_NS) {
+        *abort_flag = 1;
+        atomicOr(err, MOE_DERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+// K-major tile written by TMA with the 128-byte swizzle (8-row atoms 1024 bytes apart).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) |
+         ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// kind::f16 instruction descriptor: fp32 accumulate, A and B bf16 (1) or fp16 (0),
+// both K-major, N >> 3 at bits 17-22, M >> 4 at bits 24-28.
+__device__ __forceinline__ uint32_t make_idesc(int M, int N, bool bf16) {
+  return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ uint32_t pack_f16_sat(float a, float b) {
+  a = fminf(fmaxf(a, -65504.0f), 65504.0f);
+  b = fminf(fmaxf(b, -65504.0f), 65504.0f);
+  __half2 v = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// ------------------------------------------------------------------- tiles
+struct BTile {
+  int a_row;       // first A row
+  int valid_rows;  // rows of the block to store
+  int b_row;       // first B row
+  int n_block;
+  int seg_lo, seg_hi;  // weight-gradient tiles: the expert's K segments
+  int64_t out_off;     // element offset of the tile's first output row and column
+};
+
+template <bool WGRAD>
+__device__ __forceinline__ BTile decode(int t, const BwdArgs& a, const int* s_prefix) {
+  BTile tl;
+  if (WGRAD) {
+    const int per = a.m_blocks * a.n_blocks_n;
+    const int e = t / per;
+    const int rem = t - e * per;
+    const int mb = rem / a.n_blocks_n;
+    tl.n_block = rem - mb * a.n_blocks_n;
+    tl.a_row = a.a_row_base + mb * BM;
+    tl.valid_rows = BM;
+    tl.b_row = tl.n_block * a.bn_out;
+    tl.seg_lo = __ldg(a.seg_off + e);
+    tl.seg_hi = __ldg(a.seg_off + e + 1);
+    tl.out_off = (int64_t)e * a.out_expert_stride + (int64_t)mb * BM * a.out_ld +
+                 (int64_t)tl.n_block * a.bn_out;
+  } else {
+    const int mt = t / a.n_blocks_n;
+    tl.n_block = t - mt * a.n_blocks_n;
+    int lo = 0, hi = a.G - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_prefix[mid] <= mt) lo = mid; else hi = mid - 1;
+    }
+    const int4 g = __ldg(a.groups + lo);
+    const int m_local = mt - s_prefix[lo];
+    tl.a_row = g.x + m_local * BM;
+    tl.valid_rows = min(BM, g.y - m_local * BM);
+    // a replica slot holds its expert's weights bitwise: read the home tensor
+    tl.b_row = g.z * a.rows_per_expert + tl.n_block * a.bn_out;
+    tl.seg_lo = tl.seg_hi = 0;
+    tl.out_off = (int64_t)tl.a_row * a.out_ld + (int64_t)tl.n_block * a.bn_out;
+  }
+  return tl;
+}
+
+// K steps of a tile, in order: row tiles 0..k_blocks-1; weight-gradient tiles the
+// concatenated segments of the expert.
+template <bool WGRAD, class F>
+__device__ __forceinline__ bool for_k(const BTile& tl, const BwdArgs& a, F&& f) {
+  if (WGRAD) {
+    for (int s = tl.seg_lo; s < tl.seg_hi; ++s) {
+      const int2 sg = __ldg(a.segs + s);
+      for (int kb = sg.x; kb < sg.x + sg.y; ++kb)
+        if (!f(kb)) return false;
+    }
+  } else {
+    for (int kb = 0; kb < a.k_blocks; ++kb)
+      if (!f(kb)) return false;
+  }
+  return true;
+}
+
+template <int EPI, bool WGRAD>
+__global__ void __launch_bounds__(BWD_THREADS, 1)
+    bwd_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
+                    const __grid_constant__ CUtensorMap tm_b0,
+                    const __grid_constant__ CUtensorMap tm_b1, const BwdArgs args) {
+  constexpr bool TWO_B = EPI == EPI_SWIGLU_BWD;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* stage_base = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  int* s_misc = reinterpret_cast<int*>(bars + 2 * STAGES + 5);
+  int* s_prefix = s_misc + 4;
+  int* s_scan = s_prefix + MAX_GROUPS + 1;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  volatile int* abort_flag = s_misc + 1;
+
+  if (tid == 0) {
+    s_misc[2] = load_err(args.err);
+    s_misc[1] = 0;
+  }
+  __syncthreads();
+  if (s_misc[2] != 0) return;
+
+  int total_tiles;
+  if (WGRAD) {
+    total_tiles = args.E * args.m_blocks * args.n_blocks_n;
+  } else {
+    for (int g = tid; g < args.G; g += blockDim.x) {
+      const int rows = __ldg(&args.groups[g].y);
+      s_prefix[g] = rows > 0 ? (rows + BM - 1) / BM : 0;
+    }
+    __syncthreads();
+    const int total_m = block_exclusive_scan(s_prefix, args.G, s_scan);
+    if (tid == 0) s_prefix[args.G] = total_m;
+    total_tiles = total_m * args.n_blocks_n;
+  }
+
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = smem_u32(bars + STAGES);
+  const uint32_t tfull0 = smem_u32(bars + 2 * STAGES);
+  const uint32_t tempty0 = smem_u32(bars + 2 * STAGES + 2);
+  const uint32_t drain = smem_u32(bars + 2 * STAGES + 4);
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull0 + 8 * b, 1);
+      mbar_init(tempty0 + 8 * b, 4);
+    }
+    mbar_init(drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(s_misc)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = static_cast<uint32_t>(s_misc[0]);
+  const uint32_t b_bytes = (uint32_t)args.mma_n * BK * 2;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_phase = 0;
+      for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+        const BTile tl = decode<WGRAD>(t, args, s_prefix);
+        const bool ok = for_k<WGRAD>(tl, args, [&](int kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, args.err)) return false;
+          const uint32_t fb = full0 + 8 * stage;
+          const uint32_t sa = smem_u32(stage_base + stage * STAGE_BYTES);
+          const uint32_t sb = sa + A_BYTES;
+          mbar_expect_tx(fb, A_BYTES + b_bytes);
+          tma_load_2d(sa, &tm_a, fb, kb * BK, tl.a_row);
+          tma_load_2d(sb, &tm_b0, fb, kb * BK, tl.b_row);
+          if (TWO_B) tma_load_2d(sb + (b_bytes >> 1), &tm_b1, fb, kb * BK, tl.b_row);
+          issued_mask |= 1u << stage;
+          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          return true;
+        });
+        if (!ok) break;
+      }
+      for (int s = 0; s < STAGES; ++s)
+        if (issued_mask & (1u << s)) {
+          volatile int no_abort = 0;
+          mbar_wait(full0 + 8 * s, (issued_phase >> s) & 1u, &no_abort, args.err);
+        }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = make_idesc(BM, args.mma_n, args.bf16 != 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+        const BTile tl = decode<WGRAD>(t, args, s_prefix);
+        if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag, args.err)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+        bool first = true;
+        const bool ok = for_k<WGRAD>(tl, args, [&](int) {
+          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, args.err)) return false;
+          tc_fence_after();
+          const uint32_t sa = smem_u32(stage_base + stage * STAGE_BYTES);
+          const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / UMMA_K; ++kk)
+            tc_mma(d_tmem, sw128_desc(sa + kk * UMMA_K * 2), sw128_desc(sb + kk * UMMA_K * 2),
+                   idesc, (first && kk == 0) ? 0u : 1u);
+          first = false;
+          tc_commit(empty0 + 8 * stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          return true;
+        });
+        if (!ok) break;
+        tc_commit(tfull0 + 8 * acc);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      tc_commit(drain);
+      volatile int no_abort = 0;
+      mbar_wait(drain, 0, &no_abort, args.err);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------- epilogue (warps 2-5)
+    const int quarter = warp & 3;
+    const int r_in = quarter * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+      const BTile tl = decode<WGRAD>(t, args, s_prefix);
+      const bool ok = mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, args.err);
+      if (!__all_sync(MOE_FULL_MASK, ok)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * ACC_COLS;
+      const bool valid = r_in < tl.valid_rows;
+      const bool empty_k = WGRAD && tl.seg_lo == tl.seg_hi;  // expert without rows: zeros
+      if (EPI == EPI_SWIGLU_BWD) {
+        const int row = tl.a_row + r_in;
+        const int col0 = tl.n_block * 128;
+        const float* dhrow = args.dh + (int64_t)row * args.F + col0;
+        __nv_bfloat16* grow = args.dgu + (int64_t)row * (2 * args.F) + col0;
+#pragma unroll 1
+        for (int c = 0; c < 128 / 32; ++c) {
+          uint32_t g[32], u[32];
+          tmem_ld32(tbase + c * 32, g);
+          tmem_ld32(tbase + 128 + c * 32, u);
+          tmem_wait_ld();
+          if (valid) {
+            float dh[32];
+            const float4* src = reinterpret_cast<const float4*>(dhrow + c * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float4 v = __ldg(src + i);
+              dh[4 * i] = v.x;
+              dh[4 * i + 1] = v.y;
+              dh[4 * i + 2] = v.z;
+              dh[4 * i + 3] = v.w;
+            }
+            uint32_t pg[16], pu[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float dgv[2], duv[2];
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const float gv = __uint_as_float(g[2 * i + h]);
+                const float uv = __uint_as_float(u[2 * i + h]);
+                const float s = 1.0f / (1.0f + __expf(-gv));
+                const float dhv = dh[2 * i + h];
+                duv[h] = dhv * gv * s;
+                dgv[h] = dhv * uv * s * (1.0f + gv * (1.0f - s));
+              }
+              pg[i] = pack_bf16(dgv[0], dgv[1]);
+              pu[i] = pack_bf16(duv[0], duv[1]);
+            }
+            uint4* dg_dst = reinterpret_cast<uint4*>(grow + c * 32);
+            uint4* du_dst = reinterpret_cast<uint4*>(grow + args.F + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              dg_dst[i] = make_uint4(pg[4 * i], pg[4 * i + 1], pg[4 * i + 2], pg[4 * i + 3]);
+              du_dst[i] = make_uint4(pu[4 * i], pu[4 * i + 1], pu[4 * i + 2], pu[4 * i + 3]);
+            }
+          }
+        }
+      } else if (EPI == EPI_F32) {
+        float* orow = static_cast<float*>(args.out) + tl.out_off + (int64_t)r_in * args.out_ld;
+#pragma unroll 1
+        for (int c = 0; c < args.bn_out / 32; ++c) {
+          uint32_t v[32];
+          if (!empty_k) {
+            tmem_ld32(tbase + c * 32, v);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0u;
+          }
+          if (valid) {
+            float4* dst = reinterpret_cast<float4*>(orow + c * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                   __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+          }
+        }
+      } else {
+        uint16_t* orow = static_cast<uint16_t*>(args.out) + tl.out_off + (int64_t)r_in * args.out_ld;
+#pragma unroll 1
+        for (int c = 0; c < args.bn_out / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tbase + c * 32, v);
+          tmem_wait_ld();
+          uint32_t p[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) p[i] = pack_bf16(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ------------------------------------------------------------------- helpers
+// Padded K layout of the transposed activations: group g's rows occupy columns
+// [padoff[g], padoff[g] + ceil(n_g/64)*64), zero beyond its rows; per expert, the list
+// of its groups' K-step segments in group-table order (home and replica groups alike).
+__global__ void __launch_bounds__(1024) bwd_prepare_kernel(const int4* __restrict__ groups, int G,
+                                                           int E, int* __restrict__ padoff,
+                                                           int* __restrict__ seg_off,
+                                                           int2* __restrict__ segs,
+                                                           const int32_t* __restrict__ err) {
+  __shared__ int s_pad[MAX_GROUPS + 1];
+  __shared__ int s_cnt[1025];
+  __shared__ int s_scan[33];
+  if (block_should_stop(err)) return;
+  for (int g = threadIdx.x; g < G; g += blockDim.x) {
+    const int n = groups[g].y;
+    s_pad[g] = n > 0 ? (n + BK - 1) / BK * BK : 0;
+  }
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_cnt[e] = 0;
+  __syncthreads();
+  for (int g = threadIdx.x; g < G; g += blockDim.x) {
+    const int4 r = groups[g];
+    if (r.y > 0) atomicAdd(&s_cnt[r.z], 1);
+  }
+  __syncthreads();
+  const int total = block_exclusive_scan(s_pad, G, s_scan);
+  const int nseg = block_exclusive_scan(s_cnt, E, s_scan);
+  for (int g = threadIdx.x; g < G; g += blockDim.x) padoff[g] = s_pad[g];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) seg_off[e] = s_cnt[e];
+  __syncthreads();  // thread 0 reuses s_cnt as its fill cursor below
+  if (threadIdx.x == 0) {
+    padoff[G] = total;
+    seg_off[E] = nseg;
+    // stable fill in group-table order (one thread: at most 4096 records)
+    for (int g = 0; g < G; ++g) {
+      const int4 r = groups[g];
+      if (r.y > 0) {
+        const int at = s_cnt[r.z]++;
+        segs[at] = make_int2(s_pad[g] / BK, (r.y + BK - 1) / BK);
+      }
+    }
+  }
+}
+
+// pos[row] = the row's column in the padded K layout
+__global__ void __launch_bounds__(256) row_pos_kernel(const int4* __restrict__ groups,
+                                                      const int* __restrict__ padoff,
+                                                      int* __restrict__ pos,
+                                                      const int32_t* __restrict__ err) {
+  if (load_err(err)) return;
+  const int g = blockIdx.x;
+  const int4 r = groups[g];
+  for (int i = threadIdx.x; i < r.y; i += blockDim.x) pos[r.x + i] = padoff[g] + i;
+}
+
+// out[c][col(r)] = in[r][c] for 16-bit elements, batched over blockIdx.z; col(r) = r, or
+// pos[r] when pos is given.
+// With f16_to_bf16 the fp16 input values are rounded to bf16 on the way.
+__global__ void __launch_bounds__(256) transpose16_kernel(const uint16_t* __restrict__ in,
+                                                          int rows, int cols, int64_t ld_in,
+                                                          int64_t in_bstride,
+                                                          uint16_t* __restrict__ out,
+                                                          int64_t ld_out, int64_t out_bstride,
+                                                          const int* __restrict__ pos,
+                                                          int f16_to_bf16,
+                                                          const int32_t* __restrict__ err) {
+  __shared__ uint16_t tile[32][34];
+  if (load_err(err)) return;
+  const uint16_t* src = in + (int64_t)blockIdx.z * in_bstride;
+  uint16_t* dst = out + (int64_t)blockIdx.z * out_bstride;
+  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    if (r < rows && c < cols) {
+      uint16_t v = src[(int64_t)r * ld_in + c];
+      if (f16_to_bf16) {
+        const __nv_bfloat16 b = __float2bfloat16_rn(__half2float(__ushort_as_half(v)));
+        v = __bfloat16_as_ushort(b);
+      }
+      tile[i][threadIdx.x] = v;
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int c = c0 + i, r = r0 + threadIdx.x;
+    if (r < rows && c < cols) {
+      const int col = pos ? pos[r] : r;
+      dst[(int64_t)c * ld_out + col] = tile[threadIdx.x][i];
+    }
+  }
+}
+
+// Backward of combine: dy[perm[t,j]] = gate[t,j] * dout[t] (bf16), dgate[t,j] =
+// <dout[t], y[perm[t,j]]> (fp32).  One warp per token, 16-byte vectors.
+__global__ void __launch_bounds__(256) combine_backward_kernel(
+    const uint4* __restrict__ dout, const uint4* __restrict__ y, const int32_t* __restrict__ perm,
+    const float* __restrict__ gate, int T, int k, int dv, uint4* __restrict__ dy,
+    float* __restrict__ dgate, const int32_t* __restrict__ err) {
+  if (load_err(err)) return;
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += nwarps) {
+    for (int j = 0; j < k; ++j) {
+      const int r = __ldg(perm + t * k + j);
+      const float gj = __ldg(gate + t * k + j);
+      float dot = 0.f;
+      for (int v = lane; v < dv; v += 32) {
+        const uint4 a = __ldg(dout + t * dv + v);
+        const uint4 b = __ldcs(y + (int64_t)r * dv + v);
+        const __nv_bfloat162* ap = reinterpret_cast<const __nv_bfloat162*>(&a);
+        const __nv_bfloat162* bp = reinterpret_cast<const __nv_bfloat162*>(&b);
+        uint32_t o[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 af = __bfloat1622float2(ap[i]);
+          const float2 bf = __bfloat1622float2(bp[i]);
+          dot = fmaf(af.x, bf.x, dot);
+          dot = fmaf(af.y, bf.y, dot);
+          o[i] = pack_bf16(gj * af.x, gj * af.y);
+        }
+        dy[(int64_t)r * dv + v] = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+      dot = warp_sum(dot);
+      if (lane == 0) dgate[t * k + j] = dot;
+    }
+  }
+}
+
+// Backward of the gates (softmax over the chosen logits): dlogit[t, idx[t,j]] =
+// gate[t,j] (dgate[t,j] - sum_i gate[t,i] dgate[t,i]); every other logit gets 0.
+__global__ void __launch_bounds__(256) topk_backward_kernel(
+    const float* __restrict__ gate, const float* __restrict__ dgate,
+    const int32_t* __restrict__ idx, int T, int E, int k, float* __restrict__ dlogits,
+    const int32_t* __restrict__ err) {
+  if (load_err(err)) return;
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += nwarps) {
+    const float g = lane < k ? __ldg(gate + t * k + lane) : 0.f;
+    const float dg = lane < k ? __ldg(dgate + t * k + lane) : 0.f;
+    const float s = warp_sum(g * dg);
+    float* row = dlogits + t * E;
+    for (int e = lane; e < E; e += 32) row[e] = 0.f;
+    __syncwarp();
+    if (lane < k) row[__ldg(idx + t * k + lane)] = g * (dg - s);
+  }
+}
+
+// ------------------------------------------------------------------- host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn_bwd() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D 16-bit tensor [rows, cols], row pitch `ld` elements, box 64 columns x box_rows rows,
+// 128-byte swizzle.
+bool make_map16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld,
+                int box_rows, bool bf16) {
+  EncodeTiledFn fn = encode_fn_bwd();
+  if (!fn || rows <= 0 || cols <= 0) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+            const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t bwd_smem_bytes() {
+  return 1024 + (size_t)STAGES * STAGE_BYTES + (2 * STAGES + 5) * 8 + 4 * 4 +
+         (MAX_GROUPS + 1) * 4 + 33 * 4;
+}
+
+template <int EPI, bool WGRAD>
+int launch_bwd_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                    const BwdArgs& args, cudaStream_t s) {
+  static bool configured[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const size_t smem = bwd_smem_bytes();
+  if (dev < 64 && !configured[dev]) {
+    if (cudaFuncSetAttribute(bwd_gemm_kernel<EPI, WGRAD>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return MOE_ERR_LAUNCH;
+    configured[dev] = true;
+  }
+  bwd_gemm_kernel<EPI, WGRAD><<<num_sms(), BWD_THREADS, smem, s>>>(a, b0, b1, args);
+  return launch_status();
+}
+
+int transpose16(const void* in, int rows, int cols, int64_t ld_in, int64_t in_bstride, void* out,
+                int64_t ld_out, int64_t out_bstride, int batches, const int* pos,
+                const int32_t* err, cudaStream_t s, bool f16_to_bf16 = false) {
+  if (rows <= 0 || cols <= 0 || batches <= 0) return MOE_OK;
+  dim3 grid((cols + 31) / 32, (rows + 31) / 32, batches), block(32, 8);
+  transpose16_kernel<<<grid, block, 0, s>>>(static_cast<const uint16_t*>(in), rows, cols, ld_in,
+                                            in_bstride, static_cast<uint16_t*>(out), ld_out,
+                                            out_bstride, pos, f16_to_bf16 ? 1 : 0, err);
+  return launch_status();
+}
+
+// Workspace carve-up (every piece 256-byte aligned).
+struct BwdWs {
+  __nv_bfloat16* w2t;   // [E*F, d] (W2 transposed, rounded to bf16)
+  __nv_bfloat16* w13t;  // [E*d, 2F]
+  float* dh;            // [RC, F]
+  __nv_bfloat16* dgu;   // [RC, 2F]
+  int* pos;             // [RC]
+  int* padoff;          // [G+1]
+  int* seg_off;         // [E+1]
+  int2* segs;           // [G]
+  __nv_bfloat16* dyt;   // [d, Kc]
+  __nv_bfloat16* ht;    // [F, Kc] (h rounded to bf16)
+  __nv_bfloat16* dgut;  // [2F, Kc]
+  __nv_bfloat16* xt;    // [d, Kc]
+  int64_t kc;           // padded K capacity
+  int64_t bytes;
+};
+
+BwdWs carve(uint8_t* base, int T, int k, int E, int R, int S, int d, int F, int G) {
+  BwdWs w{};
+  const int64_t RC = (int64_t)T * k;
+  w.kc = ((RC + (int64_t)BK * G + 63) / 64) * 64;
+  int64_t off = 0;
+  auto take = [&](int64_t bytes) {
+    const int64_t at = off;
+    off += (bytes + 255) / 256 * 256;
+    return base ? base + at : nullptr;
+  };
+  w.w2t = reinterpret_cast<__nv_bfloat16*>(take((int64_t)E * F * d * 2));
+  w.w13t = reinterpret_cast<__nv_bfloat16*>(take((int64_t)E * d * 2 * F * 2));
+  w.dh = reinterpret_cast<float*>(take(RC * F * 4));
+  w.dgu = reinterpret_cast<__nv_bfloat16*>(take(RC * 2 * F * 2));
+  w.pos = reinterpret_cast<int*>(take(RC * 4));
+  w.padoff = reinterpret_cast<int*>(take((int64_t)(G + 1) * 4));
+  w.seg_off = reinterpret_cast<int*>(take((int64_t)(E + 1) * 4));
+  w.segs = reinterpret_cast<int2*>(take((int64_t)G * 8));
+  w.dyt = reinterpret_cast<__nv_bfloat16*>(take((int64_t)d * w.kc * 2));
+  w.ht = reinterpret_cast<__nv_bfloat16*>(take((int64_t)F * w.kc * 2));
+  w.dgut = reinterpret_cast<__nv_bfloat16*>(take((int64_t)2 * F * w.kc * 2));
+  w.xt = reinterpret_cast<__nv_bfloat16*>(take((int64_t)d * w.kc * 2));
+  w.bytes = off;
+  (void)R;
+  (void)S;
+  return w;
+}
+
+}  // namespace
+
+int64_t ffn_backward_workspace_bytes(int T, int k, int E, int R, int S, int d, int F, int G) {
+  return carve(nullptr, T, k, E, R, S, d, F, G).bytes;
+}
+
+int launch_combine_backward(const __nv_bfloat16* dout, const __nv_bfloat16* y,
+                            const int32_t* perm, const float* gate, int T, int k, int d,
+                            __nv_bfloat16* dy, float* dgate, const int32_t* err,
+                            cudaStream_t s) {
+  if (T == 0) return MOE_OK;
+  const int64_t want = ((int64_t)T + 7) / 8;
+  const int64_t cap = (int64_t)num_sms() * 8;
+  combine_backward_kernel<<<(unsigned)(want < cap ? want : cap), 256, 0, s>>>(
+      reinterpret_cast<const uint4*>(dout), reinterpret_cast<const uint4*>(y), perm, gate, T, k,
+      d / 8, reinterpret_cast<uint4*>(dy), dgate, err);
+  return launch_status();
+}
+
+int launch_topk_backward(const float* gate, const float* dgate, const int32_t* idx, int T, int E,
+                         int k, float* dlogits, const int32_t* err, cudaStream_t s) {
+  if (T == 0) return MOE_OK;
+  const int64_t want = ((int64_t)T + 7) / 8;
+  const int64_t cap = (int64_t)num_sms() * 8;
+  topk_backward_kernel<<<(unsigned)(want < cap ? want : cap), 256, 0, s>>>(gate, dgate, idx, T, E,
+                                                                           k, dlogits, err);
+  return launch_status();
+}
+
+int launch_grouped_ffn_backward(const __nv_bfloat16* recv, const __nv_bfloat16* dy,
+                                const __half* h,
+                                const int32_t* plan, const moe_plan_layout& L,
+                                const __nv_bfloat16* W1, const __nv_bfloat16* W3,
+                                const __half* W2, int T, int k, int E, int R, int S, int d,
+                                int F, __nv_bfloat16* dx_rows, float* dW1, float* dW3,
+                                float* dW2, void* workspace, int64_t workspace_bytes,
+                                int32_t* err, cudaStream_t s) {
+  const int G = R * L.max_groups_per_rank;
+  BwdWs w = carve(static_cast<uint8_t*>(workspace), T, k, E, R, S, d, F, G);
+  if (w.bytes > workspace_bytes) return MOE_ERR_ARG;
+  const int64_t RC = (int64_t)T * k;
+  const int4* groups = reinterpret_cast<const int4*>(plan + L.groups);
+  int st;
+  // weight gradients of experts without rows are zero; the GEMMs below write every tile
+  // (an expert with no K steps stores zeros), and with T == 0 nothing else runs
+  if (T == 0) {
+    if (cudaMemsetAsync(dW1, 0, (size_t)E * F * d * 4, s) != cudaSuccess ||
+        cudaMemsetAsync(dW3, 0, (size_t)E * F * d * 4, s) != cudaSuccess ||
+        cudaMemsetAsync(dW2, 0, (size_t)E * d * F * 4, s) != cudaSuccess)
+      return MOE_ERR_LAUNCH;
+    return MOE_OK;
+  }
+  // 1. padded K layout and per-expert segments
+  bwd_prepare_kernel<<<1, 1024, 0, s>>>(groups, G, E, w.padoff, w.seg_off, w.segs, err);
+  if ((st = launch_status()) != MOE_OK) return st;
+  row_pos_kernel<<<G, 256, 0, s>>>(groups, w.padoff, w.pos, err);
+  if ((st = launch_status()) != MOE_OK) return st;
+  // 2. transposed weights: W2T[e] = W2[e]^T [F,d]; W13T[e] = [W1[e]^T | W3[e]^T] [d,2F]
+  if ((st = transpose16(W2, d, F, F, (int64_t)d * F, w.w2t, d, (int64_t)F * d, E, nullptr, err, s,
+                        true)))
+    return st;
+  if ((st = transpose16(W1, F, d, d, (int64_t)F * d, w.w13t, 2 * F, (int64_t)d * 2 * F, E, nullptr,
+                        err, s)))
+    return st;
+  if ((st = transpose16(W3, F, d, d, (int64_t)F * d, w.w13t + F, 2 * F, (int64_t)d * 2 * F, E,
+                        nullptr, err, s)))
+    return st;
+  const int bnF = (F % 256 == 0) ? 256 : 128;
+  const int bnD = (d % 256 == 0) ? 256 : 128;
+  BwdArgs base{};
+  base.groups = groups;
+  base.G = G;
+  base.err = err;
+  base.E = E;
+  base.F = F;
+  // 3. dH = dY W2 (per group, fp16 -> fp32)
+  {
+    CUtensorMap ma, mb;
+    if (!make_map16(&ma, dy, RC, d, d, BM, true) ||
+        !make_map16(&mb, w.w2t, (int64_t)E * F, d, d, bnF, true))
+      return MOE_ERR_DEVICE;
+    BwdArgs a = base;
+    a.n_blocks_n = F / bnF;
+    a.k_blocks = d / BK;
+    a.bn_out = bnF;
+    a.mma_n = bnF;
+    a.rows_per_expert = F;
+    a.out_ld = F;
+    a.bf16 = 1;
+    a.out = w.dh;
+    if ((st = launch_bwd_gemm<EPI_F32, false>(ma, mb, mb, a, s))) return st;
+  }
+  // 4. dG, dU: the gate/up GEMM re-run on the rows, SwiGLU backward in the epilogue
+  {
+    CUtensorMap ma, m1, m3;
+    if (!make_map16(&ma, recv, RC, d, d, BM, true) ||
+        !make_map16(&m1, W1, (int64_t)E * F, d, d, 128, true) ||
+        !make_map16(&m3, W3, (int64_t)E * F, d, d, 128, true))
+      return MOE_ERR_DEVICE;
+    BwdArgs a = base;
+    a.n_blocks_n = F / 128;
+    a.k_blocks = d / BK;
+    a.bn_out = 128;
+    a.mma_n = 256;
+    a.rows_per_expert = F;
+    a.out_ld = 2 * F;
+    a.bf16 = 1;
+    a.dh = w.dh;
+    a.dgu = w.dgu;
+    if ((st = launch_bwd_gemm<EPI_SWIGLU_BWD, false>(ma, m1, m3, a, s))) return st;
+  }
+  // 5. dX rows = [dG | dU] [W1; W3] (K = 2F, bf16)
+  {
+    CUtensorMap ma, mb;
+    if (!make_map16(&ma, w.dgu, RC, 2 * F, 2 * F, BM, true) ||
+        !make_map16(&mb, w.w13t, (int64_t)E * d, 2 * F, 2 * F, bnD, true))
+      return MOE_ERR_DEVICE;
+    BwdArgs a = base;
+    a.n_blocks_n = d / bnD;
+    a.k_blocks = 2 * F / BK;
+    a.bn_out = bnD;
+    a.mma_n = bnD;
+    a.rows_per_expert = d;
+    a.out_ld = d;
+    a.bf16 = 1;
+    a.out = dx_rows;
+    if ((st = launch_bwd_gemm<EPI_BF16, false>(ma, mb, mb, a, s))) return st;
+  }
+  // 6. transposed activations in the padded K layout (zero padding)
+  if (cudaMemsetAsync(w.dyt, 0, (size_t)d * w.kc * 2, s) != cudaSuccess ||
+      cudaMemsetAsync(w.ht, 0, (size_t)F * w.kc * 2, s) != cudaSuccess ||
+      cudaMemsetAsync(w.dgut, 0, (size_t)2 * F * w.kc * 2, s) != cudaSuccess ||
+      cudaMemsetAsync(w.xt, 0, (size_t)d * w.kc * 2, s) != cudaSuccess)
+    return MOE_ERR_LAUNCH;
+  if ((st = transpose16(dy, (int)RC, d, d, 0, w.dyt, w.kc, 0, 1, w.pos, err, s))) return st;
+  if ((st = transpose16(h, (int)RC, F, F, 0, w.ht, w.kc, 0, 1, w.pos, err, s, true))) return st;
+  if ((st = transpose16(w.dgu, (int)RC, 2 * F, 2 * F, 0, w.dgut, w.kc, 0, 1, w.pos, err, s)))
+    return st;
+  if ((st = transpose16(recv, (int)RC, d, d, 0, w.xt, w.kc, 0, 1, w.pos, err, s))) return st;
+  // 7. weight gradients, every group of an expert (home and replicas) in one accumulator
+  {
+    CUtensorMap ma, mb;
+    if (!make_map16(&ma, w.dyt, d, w.kc, w.kc, BM, true) ||
+        !make_map16(&mb, w.ht, F, w.kc, w.kc, bnF, true))
+      return MOE_ERR_DEVICE;
+    BwdArgs a = base;
+    a.n_blocks_n = F / bnF;
+    a.bn_out = bnF;
+    a.mma_n = bnF;
+    a.out_ld = F;
+    a.bf16 = 1;
+    a.out = dW2;
+    a.seg_off = w.seg_off;
+    a.segs = w.segs;
+    a.m_blocks = d / BM;
+    a.a_row_base = 0;
+    a.out_expert_stride = (int64_t)d * F;
+    if ((st = launch_bwd_gemm<EPI_F32, true>(ma, mb, mb, a, s))) return st;
+  }
+  {
+    CUtensorMap ma, mb;
+    if (!make_map16(&ma, w.dgut, 2 * F, w.kc, w.kc, BM, true) ||
+        !make_map16(&mb, w.xt, d, w.kc, w.kc, bnD, true))
+      return MOE_ERR_DEVICE;
+    BwdArgs a = base;
+    a.n_blocks_n = d / bnD;
+    a.bn_out = bnD;
+    a.mma_n = bnD;
+    a.out_ld = d;
+    a.bf16 = 1;
+    a.seg_off = w.seg_off;
+    a.segs = w.segs;
+    a.m_blocks = F / BM;
+    a.out_expert_stride = (int64_t)F * d;
+    a.a_row_base = 0;
+    a.out = dW1;
+    if ((st = launch_bwd_gemm<EPI_F32, true>(ma, mb, mb, a, s))) return st;
+    a.a_row_base = F;
+    a.out = dW3;
+    if ((st = launch_bwd_gemm<EPI_F32, true>(ma, mb, mb, a, s))) return st;
+  }
+  return MOE_OK;
+}
+
+}  // namespace moe

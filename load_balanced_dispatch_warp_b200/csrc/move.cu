@@ -235,7 +235,8 @@ __global__ void __launch_bounds__(kRowThreads) combine_kernel(
   const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
   for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += nwarps) {
     const int r = lane < k ? __ldg(perm + t * k + lane) : 0;
-    const float gl = lane < k ? __ldg(gate + t * k + lane) : 0.f;
+    // gate == nullptr: unit weights (the backward of dispatch sums the k rows)
+    const float gl = lane < k ? (gate ? __ldg(gate + t * k + lane) : 1.f) : 0.f;
     if (K > 0) {
       // rows and gates of the token broadcast once; the vector loop has no warp collective
       int rows[K > 0 ? K : 1];

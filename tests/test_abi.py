@@ -29,6 +29,7 @@ def test_header_declares_the_path(lib):
     assert set(M.HELPERS) <= names
     assert set(M.VARIANTS) <= names
     assert set(M.FUSED) <= names
+    assert set(M.BACKWARD) <= names
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -100,3 +101,25 @@ def test_fused_dispatch_host_checks(lib):
     assert lib.moe_grouped_ffn_gather(*bad) == M.MOE_ERR_ARG
     bad = list(args); bad[6] = None
     assert lib.moe_grouped_ffn_gather(*bad) == M.MOE_ERR_ARG
+
+
+def test_backward_host_checks(lib):
+    P = ctypes.c_void_p
+    fake = P(4096)
+    assert lib.moe_combine_backward(fake, fake, fake, fake, 4, 2, 128, fake, fake, None, None) == M.MOE_ERR_ARG
+    assert lib.moe_combine_backward(fake, fake, fake, fake, 4, 33, 128, fake, fake, fake, None) == M.MOE_ERR_SHAPE
+    assert lib.moe_dispatch_backward(fake, fake, 4, 2, 96, fake, fake, None) == M.MOE_ERR_SHAPE
+    assert lib.moe_topk_backward(fake, fake, fake, 4, 8, 9, fake, fake, None) == M.MOE_ERR_SHAPE
+    assert lib.moe_ffn_backward_workspace_bytes(4, 2, 8, 3, 2, 128, 256) == -1  # E % R
+    n = lib.moe_ffn_backward_workspace_bytes(4096, 6, 64, 8, 8, 2048, 1408)
+    assert n > 0 and n % 256 == 0
+    args = [fake, fake, fake, fake, fake, fake, fake, 4, 2, 8, 4, 2, 128, 256, fake, fake, fake, fake,
+            fake, 1 << 30, fake, None]
+    bad = list(args); bad[15] = None  # dW1 missing
+    assert lib.moe_grouped_ffn_backward(*bad) == M.MOE_ERR_ARG
+    bad = list(args); bad[18] = P(4096 + 16)  # workspace not 256-byte aligned
+    assert lib.moe_grouped_ffn_backward(*bad) == M.MOE_ERR_ARG
+    bad = list(args); bad[19] = 1024  # workspace too small
+    assert lib.moe_grouped_ffn_backward(*bad) == M.MOE_ERR_ARG
+    bad = list(args); bad[13] = 200  # F % 128
+    assert lib.moe_grouped_ffn_backward(*bad) == M.MOE_ERR_SHAPE
