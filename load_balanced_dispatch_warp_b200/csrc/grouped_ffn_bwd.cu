@@ -543,51 +543,70 @@ __global__ void __launch_bounds__(1024) bwd_prepare_kernel(const int4* __restric
   }
 }
 
-// pos[row] = the row's column in the padded K layout
-__global__ void __launch_bounds__(256) row_pos_kernel(const int4* __restrict__ groups,
-                                                      const int* __restrict__ padoff,
-                                                      int* __restrict__ pos,
-                                                      const int32_t* __restrict__ err) {
+// src_of[q] = the row whose values sit in column q of the padded K layout, -1 for the
+// zero padding after a group's rows
+__global__ void __launch_bounds__(256) padpos_kernel(const int4* __restrict__ groups,
+                                                     const int* __restrict__ padoff,
+                                                     int* __restrict__ src_of,
+                                                     const int32_t* __restrict__ err) {
   if (load_err(err)) return;
   const int g = blockIdx.x;
   const int4 r = groups[g];
-  for (int i = threadIdx.x; i < r.y; i += blockDim.x) pos[r.x + i] = padoff[g] + i;
+  const int n = max(r.y, 0);
+  const int pad = padoff[g + 1] - padoff[g];
+  for (int i = threadIdx.x; i < pad; i += blockDim.x) src_of[padoff[g] + i] = i < n ? r.x + i : -1;
 }
 
-// out[c][col(r)] = in[r][c] for 16-bit elements, batched over blockIdx.z; col(r) = r, or
-// pos[r] when pos is given.
-// With f16_to_bf16 the fp16 input values are rounded to bf16 on the way.
-__global__ void __launch_bounds__(256) transpose16_kernel(const uint16_t* __restrict__ in,
-                                                          int rows, int cols, int64_t ld_in,
-                                                          int64_t in_bstride,
-                                                          uint16_t* __restrict__ out,
-                                                          int64_t ld_out, int64_t out_bstride,
-                                                          const int* __restrict__ pos,
-                                                          int f16_to_bf16,
-                                                          const int32_t* __restrict__ err) {
-  __shared__ uint16_t tile[32][34];
+// Tiled transpose of 16-bit elements, 64 x 64 per block, 16-byte loads and stores:
+// out[c][q] = in[src(q)][c], src(q) = q (src_of == nullptr) or src_of[q] (0 where it is
+// -1).  q runs over n_out output columns (the padded K layout: blocks past *n_out_dev, when
+// given, return at once).  cols and the row pitches are multiples of 8 elements.  With
+// f16_to_bf16 the fp16 inputs are rounded to bf16 on the way.  Batched over blockIdx.z.
+constexpr int kTp = 64;
+constexpr int kTpPitch = 72;  // smem row pitch (elements): 16-byte rows, conflict-free columns
+__global__ void __launch_bounds__(256) transpose_kernel(
+    const uint16_t* __restrict__ in, int cols, int64_t ld_in, int64_t in_bstride,
+    uint16_t* __restrict__ out, int64_t ld_out, int64_t out_bstride, int n_out,
+    const int* __restrict__ n_out_dev, const int* __restrict__ src_of, int f16_to_bf16,
+    const int32_t* __restrict__ err) {
+  __shared__ __align__(16) uint16_t tile[kTp][kTpPitch];
   if (load_err(err)) return;
+  const int q0 = blockIdx.x * kTp, c0 = blockIdx.y * kTp;
+  const int nq = n_out_dev ? min(n_out, *n_out_dev) : n_out;
+  if (q0 >= nq) return;
   const uint16_t* src = in + (int64_t)blockIdx.z * in_bstride;
   uint16_t* dst = out + (int64_t)blockIdx.z * out_bstride;
-  const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    const int r = r0 + i, c = c0 + threadIdx.x;
-    if (r < rows && c < cols) {
-      uint16_t v = src[(int64_t)r * ld_in + c];
+  for (int i = threadIdx.x; i < kTp * 8; i += blockDim.x) {
+    const int q = i >> 3, ch = i & 7;
+    const int c = c0 + ch * 8;
+    int r = -1;
+    if (q0 + q < nq) r = src_of ? __ldg(src_of + q0 + q) : q0 + q;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (r >= 0 && c < cols) {
+      v = __ldg(reinterpret_cast<const uint4*>(src + (int64_t)r * ld_in + c));
       if (f16_to_bf16) {
-        const __nv_bfloat16 b = __float2bfloat16_rn(__half2float(__ushort_as_half(v)));
-        v = __bfloat16_as_ushort(b);
+        uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[j]));
+          const __nv_bfloat162 bb = __floats2bfloat162_rn(f.x, f.y);
+          w[j] = *reinterpret_cast<const uint32_t*>(&bb);
+        }
       }
-      tile[i][threadIdx.x] = v;
     }
+    *reinterpret_cast<uint4*>(&tile[q][ch * 8]) = v;
   }
   __syncthreads();
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    const int c = c0 + i, r = r0 + threadIdx.x;
-    if (r < rows && c < cols) {
-      const int col = pos ? pos[r] : r;
-      dst[(int64_t)c * ld_out + col] = tile[threadIdx.x][i];
-    }
+  for (int i = threadIdx.x; i < kTp * 8; i += blockDim.x) {
+    const int c = i >> 3, qc = i & 7;
+    if (c0 + c >= cols || q0 + qc * 8 >= nq) continue;
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      w[j] = (uint32_t)tile[qc * 8 + 2 * j][c] | ((uint32_t)tile[qc * 8 + 2 * j + 1][c] << 16);
+    // n_out (and the padded layout) is a multiple of 8: whole 16-byte chunks
+    *reinterpret_cast<uint4*>(dst + (int64_t)(c0 + c) * ld_out + q0 + qc * 8) =
+        make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
@@ -705,14 +724,16 @@ int launch_bwd_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorM
   return launch_status();
 }
 
-int transpose16(const void* in, int rows, int cols, int64_t ld_in, int64_t in_bstride, void* out,
-                int64_t ld_out, int64_t out_bstride, int batches, const int* pos,
-                const int32_t* err, cudaStream_t s, bool f16_to_bf16 = false) {
-  if (rows <= 0 || cols <= 0 || batches <= 0) return MOE_OK;
-  dim3 grid((cols + 31) / 32, (rows + 31) / 32, batches), block(32, 8);
-  transpose16_kernel<<<grid, block, 0, s>>>(static_cast<const uint16_t*>(in), rows, cols, ld_in,
-                                            in_bstride, static_cast<uint16_t*>(out), ld_out,
-                                            out_bstride, pos, f16_to_bf16 ? 1 : 0, err);
+// out[c][q] = in[src(q)][c] for q < n_out (see transpose_kernel), batched.
+int transpose(const void* in, int cols, int64_t ld_in, int64_t in_bstride, void* out,
+              int64_t ld_out, int64_t out_bstride, int n_out, const int* n_out_dev,
+              const int* src_of, int batches, bool f16_to_bf16, const int32_t* err,
+              cudaStream_t s) {
+  if (cols <= 0 || n_out <= 0 || batches <= 0) return MOE_OK;
+  dim3 grid((n_out + kTp - 1) / kTp, (cols + kTp - 1) / kTp, batches);
+  transpose_kernel<<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(in), cols, ld_in, in_bstride,
+                                        static_cast<uint16_t*>(out), ld_out, out_bstride, n_out,
+                                        n_out_dev, src_of, f16_to_bf16 ? 1 : 0, err);
   return launch_status();
 }
 
@@ -722,7 +743,7 @@ struct BwdWs {
   __nv_bfloat16* w13t;  // [E*d, 2F]
   float* dh;            // [RC, F]
   __nv_bfloat16* dgu;   // [RC, 2F]
-  int* pos;             // [RC]
+  int* src_of;          // [Kc] source row of each padded K column, -1 for padding
   int* padoff;          // [G+1]
   int* seg_off;         // [E+1]
   int2* segs;           // [G]
@@ -748,7 +769,7 @@ BwdWs carve(uint8_t* base, int T, int k, int E, int R, int S, int d, int F, int 
   w.w13t = reinterpret_cast<__nv_bfloat16*>(take((int64_t)E * d * 2 * F * 2));
   w.dh = reinterpret_cast<float*>(take(RC * F * 4));
   w.dgu = reinterpret_cast<__nv_bfloat16*>(take(RC * 2 * F * 2));
-  w.pos = reinterpret_cast<int*>(take(RC * 4));
+  w.src_of = reinterpret_cast<int*>(take(w.kc * 4));
   w.padoff = reinterpret_cast<int*>(take((int64_t)(G + 1) * 4));
   w.seg_off = reinterpret_cast<int*>(take((int64_t)(E + 1) * 4));
   w.segs = reinterpret_cast<int2*>(take((int64_t)G * 8));
@@ -817,17 +838,17 @@ int launch_grouped_ffn_backward(const __nv_bfloat16* recv, const __nv_bfloat16* 
   // 1. padded K layout and per-expert segments
   bwd_prepare_kernel<<<1, 1024, 0, s>>>(groups, G, E, w.padoff, w.seg_off, w.segs, err);
   if ((st = launch_status()) != MOE_OK) return st;
-  row_pos_kernel<<<G, 256, 0, s>>>(groups, w.padoff, w.pos, err);
+  padpos_kernel<<<G, 256, 0, s>>>(groups, w.padoff, w.src_of, err);
   if ((st = launch_status()) != MOE_OK) return st;
-  // 2. transposed weights: W2T[e] = W2[e]^T [F,d]; W13T[e] = [W1[e]^T | W3[e]^T] [d,2F]
-  if ((st = transpose16(W2, d, F, F, (int64_t)d * F, w.w2t, d, (int64_t)F * d, E, nullptr, err, s,
-                        true)))
+  // 2. transposed weights: W2T[e] = W2[e]^T [F,d] (rounded to bf16); W13T[e] = [W1[e]^T | W3[e]^T]
+  if ((st = transpose(W2, F, F, (int64_t)d * F, w.w2t, d, (int64_t)F * d, d, nullptr, nullptr, E,
+                      true, err, s)))
     return st;
-  if ((st = transpose16(W1, F, d, d, (int64_t)F * d, w.w13t, 2 * F, (int64_t)d * 2 * F, E, nullptr,
-                        err, s)))
+  if ((st = transpose(W1, d, d, (int64_t)F * d, w.w13t, 2 * F, (int64_t)d * 2 * F, F, nullptr,
+                      nullptr, E, false, err, s)))
     return st;
-  if ((st = transpose16(W3, F, d, d, (int64_t)F * d, w.w13t + F, 2 * F, (int64_t)d * 2 * F, E,
-                        nullptr, err, s)))
+  if ((st = transpose(W3, d, d, (int64_t)F * d, w.w13t + F, 2 * F, (int64_t)d * 2 * F, F, nullptr,
+                      nullptr, E, false, err, s)))
     return st;
   const int bnF = (F % 256 == 0) ? 256 : 128;
   const int bnD = (d % 256 == 0) ? 256 : 128;
@@ -890,17 +911,14 @@ int launch_grouped_ffn_backward(const __nv_bfloat16* recv, const __nv_bfloat16* 
     a.out = dx_rows;
     if ((st = launch_bwd_gemm<EPI_BF16, false>(ma, mb, mb, a, s))) return st;
   }
-  // 6. transposed activations in the padded K layout (zero padding)
-  if (cudaMemsetAsync(w.dyt, 0, (size_t)d * w.kc * 2, s) != cudaSuccess ||
-      cudaMemsetAsync(w.ht, 0, (size_t)F * w.kc * 2, s) != cudaSuccess ||
-      cudaMemsetAsync(w.dgut, 0, (size_t)2 * F * w.kc * 2, s) != cudaSuccess ||
-      cudaMemsetAsync(w.xt, 0, (size_t)d * w.kc * 2, s) != cudaSuccess)
-    return MOE_ERR_LAUNCH;
-  if ((st = transpose16(dy, (int)RC, d, d, 0, w.dyt, w.kc, 0, 1, w.pos, err, s))) return st;
-  if ((st = transpose16(h, (int)RC, F, F, 0, w.ht, w.kc, 0, 1, w.pos, err, s, true))) return st;
-  if ((st = transpose16(w.dgu, (int)RC, 2 * F, 2 * F, 0, w.dgut, w.kc, 0, 1, w.pos, err, s)))
+  // 6. transposed activations in the padded K layout (padding written as zeros)
+  const int kc = (int)w.kc;
+  const int* kp = w.padoff + G;  // used columns of the padded layout
+  if ((st = transpose(dy, d, d, 0, w.dyt, w.kc, 0, kc, kp, w.src_of, 1, false, err, s))) return st;
+  if ((st = transpose(h, F, F, 0, w.ht, w.kc, 0, kc, kp, w.src_of, 1, true, err, s))) return st;
+  if ((st = transpose(w.dgu, 2 * F, 2 * F, 0, w.dgut, w.kc, 0, kc, kp, w.src_of, 1, false, err, s)))
     return st;
-  if ((st = transpose16(recv, (int)RC, d, d, 0, w.xt, w.kc, 0, 1, w.pos, err, s))) return st;
+  if ((st = transpose(recv, d, d, 0, w.xt, w.kc, 0, kc, kp, w.src_of, 1, false, err, s))) return st;
   // 7. weight gradients, every group of an expert (home and replicas) in one accumulator
   {
     CUtensorMap ma, mb;
