@@ -178,12 +178,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);
 }
-__device__ __forceinline__ uint32_t pack_f16_sat(float a, float b) {
-  a = fminf(fmaxf(a, -65504.0f), 65504.0f);
-  b = fminf(fmaxf(b, -65504.0f), 65504.0f);
-  __half2 v = __floats2half2_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
 
 // ------------------------------------------------------------------- tiles
 struct BTile {
