@@ -557,13 +557,14 @@ __global__ void __launch_bounds__(256) padpos_kernel(const int4* __restrict__ gr
 // given, return at once).  cols and the row pitches are multiples of 8 elements.  With
 // f16_to_bf16 the fp16 inputs are rounded to bf16 on the way.  Batched over blockIdx.z.
 constexpr int kTp = 64;
-constexpr int kTpPitch = 72;  // smem row pitch (elements): 16-byte rows, conflict-free columns
+// shared tile [q][c]: the 16-byte chunk j of row q is stored at chunk j ^ ((q / 8) % 8), so
+// that reading one column across rows q = 8i + r (i = 0..7) touches 8 different banks
 __global__ void __launch_bounds__(256) transpose_kernel(
     const uint16_t* __restrict__ in, int cols, int64_t ld_in, int64_t in_bstride,
     uint16_t* __restrict__ out, int64_t ld_out, int64_t out_bstride, int n_out,
     const int* __restrict__ n_out_dev, const int* __restrict__ src_of, int f16_to_bf16,
     const int32_t* __restrict__ err) {
-  __shared__ __align__(16) uint16_t tile[kTp][kTpPitch];
+  __shared__ __align__(16) uint16_t tile[kTp][kTp];
   if (load_err(err)) return;
   const int q0 = blockIdx.x * kTp, c0 = blockIdx.y * kTp;
   const int nq = n_out_dev ? min(n_out, *n_out_dev) : n_out;
@@ -588,16 +589,18 @@ __global__ void __launch_bounds__(256) transpose_kernel(
         }
       }
     }
-    *reinterpret_cast<uint4*>(&tile[q][ch * 8]) = v;
+    *reinterpret_cast<uint4*>(&tile[q][(ch ^ ((q >> 3) & 7)) * 8]) = v;
   }
   __syncthreads();
   for (int i = threadIdx.x; i < kTp * 8; i += blockDim.x) {
     const int c = i >> 3, qc = i & 7;
     if (c0 + c >= cols || q0 + qc * 8 >= nq) continue;
+    // rows qc*8 .. qc*8+7 share (q / 8) = qc: column c sits in chunk (c / 8) ^ qc
+    const int col = (((c >> 3) ^ qc) << 3) | (c & 7);
     uint32_t w[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j)
-      w[j] = (uint32_t)tile[qc * 8 + 2 * j][c] | ((uint32_t)tile[qc * 8 + 2 * j + 1][c] << 16);
+      w[j] = (uint32_t)tile[qc * 8 + 2 * j][col] | ((uint32_t)tile[qc * 8 + 2 * j + 1][col] << 16);
     // n_out (and the padded layout) is a multiple of 8: whole 16-byte chunks
     *reinterpret_cast<uint4*>(dst + (int64_t)(c0 + c) * ld_out + q0 + qc * 8) =
         make_uint4(w[0], w[1], w[2], w[3]);
