@@ -18,11 +18,10 @@
 // buffer, one MMA thread, four epilogue warps) with three epilogues, in bf16: dY is bf16
 // because gate * dout spans the gates' range (fp16 would lose small gates to subnormals),
 // and the fp16 operands it meets (W2, the forward's h) are converted to bf16 by the
-// transposes below.  Every GEMM reads
-// K-major operands, so the operands whose contraction runs along a stored row (W2, W1, W3
-// for the data gradients; dY, h, dG, dU and X for the weight gradients) are first
-// transposed by an HBM-bound kernel; the transposed activations give every group a
-// segment of whole 64-row K steps, zero-padded, so no K step mixes two groups.
+// transposes below.  The dX GEMM reads W1 and W3 as they are stored (MN-major B
+// operand); the dH GEMM reads W2 transposed to bf16, and the weight-gradient GEMMs read
+// dY, h, dG, dU and X transposed by an HBM-bound kernel into a layout that gives every
+// group a segment of whole 64-row K steps, zero-padded, so no K step mixes two groups.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -55,6 +54,7 @@ struct BwdArgs {
   int rows_per_expert;  // rows of one expert in the B tensor (row tiles)
   int out_ld;           // columns of the output tensor
   int bf16;             // operand type: 1 bf16, 0 fp16
+  int kb_split;         // B read MN-major: K steps below it from tm_b0, the rest from tm_b1
   void* out;
   int32_t* err;
   // SwiGLU backward epilogue: reads dH [rows, F] fp32, writes dG | dU into dGU [rows, 2F]
@@ -168,11 +168,20 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
   return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) |
          ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
-// kind::f16 instruction descriptor: fp32 accumulate, A and B bf16 (1) or fp16 (0),
-// both K-major, N >> 3 at bits 17-22, M >> 4 at bits 24-28.
-__device__ __forceinline__ uint32_t make_idesc(int M, int N, bool bf16) {
+// MN-major tile written by TMA with the 128-byte swizzle as boxes of 64 K rows x 64 MN
+// elements (128-byte rows): 8-row K groups 1024 bytes apart (stride byte offset), 64-element
+// MN chunks one box (8 KiB) apart (leading byte offset).  A K step of 16 rows adds 2048
+// bytes to the start address.
+__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(8192 >> 4) << 16) |
+         ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// kind::f16 instruction descriptor: fp32 accumulate, A and B bf16 (1) or fp16 (0), A
+// K-major, B K-major (0) or MN-major (1) at bit 16, N >> 3 at bits 17-22, M >> 4 at bits
+// 24-28.
+__device__ __forceinline__ uint32_t make_idesc(int M, int N, bool bf16, bool b_mn) {
   return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) |
-         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+         ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
@@ -185,6 +194,7 @@ struct BTile {
   int valid_rows;  // rows of the block to store
   int b_row;       // first B row
   int n_block;
+  int e;               // row tiles: the group's expert
   int seg_lo, seg_hi;  // weight-gradient tiles: the expert's K segments
   int64_t out_off;     // element offset of the tile's first output row and column
 };
@@ -201,6 +211,7 @@ __device__ __forceinline__ BTile decode(int t, const BwdArgs& a, const int* s_pr
     tl.a_row = a.a_row_base + mb * BM;
     tl.valid_rows = BM;
     tl.b_row = tl.n_block * a.bn_out;
+    tl.e = e;
     tl.seg_lo = __ldg(a.seg_off + e);
     tl.seg_hi = __ldg(a.seg_off + e + 1);
     tl.out_off = (int64_t)e * a.out_expert_stride + (int64_t)mb * BM * a.out_ld +
@@ -219,6 +230,7 @@ __device__ __forceinline__ BTile decode(int t, const BwdArgs& a, const int* s_pr
     tl.valid_rows = min(BM, g.y - m_local * BM);
     // a replica slot holds its expert's weights bitwise: read the home tensor
     tl.b_row = g.z * a.rows_per_expert + tl.n_block * a.bn_out;
+    tl.e = g.z;
     tl.seg_lo = tl.seg_hi = 0;
     tl.out_off = (int64_t)tl.a_row * a.out_ld + (int64_t)tl.n_block * a.bn_out;
   }
@@ -242,7 +254,7 @@ __device__ __forceinline__ bool for_k(const BTile& tl, const BwdArgs& a, F&& f) 
   return true;
 }
 
-template <int EPI, bool WGRAD>
+template <int EPI, bool WGRAD, bool BMN>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
                     const __grid_constant__ CUtensorMap tm_b0,
@@ -326,8 +338,17 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           const uint32_t sb = sa + A_BYTES;
           mbar_expect_tx(fb, A_BYTES + b_bytes);
           tma_load_2d(sa, &tm_a, fb, kb * BK, tl.a_row);
-          tma_load_2d(sb, &tm_b0, fb, kb * BK, tl.b_row);
-          if (TWO_B) tma_load_2d(sb + (b_bytes >> 1), &tm_b1, fb, kb * BK, tl.b_row);
+          if (BMN) {
+            // B [N][K] read from a tensor stored K-row major: boxes of 64 K rows x 64 N
+            const bool lo = kb < args.kb_split;
+            const int krow = tl.e * args.rows_per_expert + (lo ? kb : kb - args.kb_split) * BK;
+            const int n0 = tl.n_block * args.bn_out;
+            for (int c = 0; c < args.mma_n / 64; ++c)
+              tma_load_2d(sb + c * 8192, lo ? &tm_b0 : &tm_b1, fb, n0 + c * 64, krow);
+          } else {
+            tma_load_2d(sb, &tm_b0, fb, kb * BK, tl.b_row);
+            if (TWO_B) tma_load_2d(sb + (b_bytes >> 1), &tm_b1, fb, kb * BK, tl.b_row);
+          }
           issued_mask |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -345,7 +366,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = make_idesc(BM, args.mma_n, args.bf16 != 0);
+      const uint32_t idesc = make_idesc(BM, args.mma_n, args.bf16 != 0, BMN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -363,7 +384,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           const uint32_t sb = sa + A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / UMMA_K; ++kk)
-            tc_mma(d_tmem, sw128_desc(sa + kk * UMMA_K * 2), sw128_desc(sb + kk * UMMA_K * 2),
+            tc_mma(d_tmem, sw128_desc(sa + kk * UMMA_K * 2),
+                   BMN ? sw128_mn_desc(sb + kk * UMMA_K * 128) : sw128_desc(sb + kk * UMMA_K * 2),
                    idesc, (first && kk == 0) ? 0u : 1u);
           first = false;
           tc_commit(empty0 + 8 * stage);
@@ -704,7 +726,7 @@ size_t bwd_smem_bytes() {
          (MAX_GROUPS + 1) * 4 + 33 * 4;
 }
 
-template <int EPI, bool WGRAD>
+template <int EPI, bool WGRAD, bool BMN = false>
 int launch_bwd_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                     const BwdArgs& args, cudaStream_t s) {
   static bool configured[64] = {false};
@@ -712,12 +734,12 @@ int launch_bwd_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorM
   cudaGetDevice(&dev);
   const size_t smem = bwd_smem_bytes();
   if (dev < 64 && !configured[dev]) {
-    if (cudaFuncSetAttribute(bwd_gemm_kernel<EPI, WGRAD>,
+    if (cudaFuncSetAttribute(bwd_gemm_kernel<EPI, WGRAD, BMN>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return MOE_ERR_LAUNCH;
     configured[dev] = true;
   }
-  bwd_gemm_kernel<EPI, WGRAD><<<num_sms(), BWD_THREADS, smem, s>>>(a, b0, b1, args);
+  bwd_gemm_kernel<EPI, WGRAD, BMN><<<num_sms(), BWD_THREADS, smem, s>>>(a, b0, b1, args);
   return launch_status();
 }
 
@@ -737,7 +759,6 @@ int transpose(const void* in, int cols, int64_t ld_in, int64_t in_bstride, void*
 // Workspace carve-up (every piece 256-byte aligned).
 struct BwdWs {
   __nv_bfloat16* w2t;   // [E*F, d] (W2 transposed, rounded to bf16)
-  __nv_bfloat16* w13t;  // [E*d, 2F]
   float* dh;            // [RC, F]
   __nv_bfloat16* dgu;   // [RC, 2F]
   int* src_of;          // [Kc] source row of each padded K column, -1 for padding
@@ -763,7 +784,6 @@ BwdWs carve(uint8_t* base, int T, int k, int E, int R, int S, int d, int F, int 
     return base ? base + at : nullptr;
   };
   w.w2t = reinterpret_cast<__nv_bfloat16*>(take((int64_t)E * F * d * 2));
-  w.w13t = reinterpret_cast<__nv_bfloat16*>(take((int64_t)E * d * 2 * F * 2));
   w.dh = reinterpret_cast<float*>(take(RC * F * 4));
   w.dgu = reinterpret_cast<__nv_bfloat16*>(take(RC * 2 * F * 2));
   w.src_of = reinterpret_cast<int*>(take(w.kc * 4));
@@ -837,15 +857,10 @@ int launch_grouped_ffn_backward(const __nv_bfloat16* recv, const __nv_bfloat16* 
   if ((st = launch_status()) != MOE_OK) return st;
   padpos_kernel<<<G, 256, 0, s>>>(groups, w.padoff, w.src_of, err);
   if ((st = launch_status()) != MOE_OK) return st;
-  // 2. transposed weights: W2T[e] = W2[e]^T [F,d] (rounded to bf16); W13T[e] = [W1[e]^T | W3[e]^T]
+  // 2. W2T[e] = W2[e]^T [F,d], rounded to bf16 (the dH GEMM reads it K-major; W1 and W3 are
+  //    read MN-major by the dX GEMM, no copy)
   if ((st = transpose(W2, F, F, (int64_t)d * F, w.w2t, d, (int64_t)F * d, d, nullptr, nullptr, E,
                       true, err, s)))
-    return st;
-  if ((st = transpose(W1, d, d, (int64_t)F * d, w.w13t, 2 * F, (int64_t)d * 2 * F, F, nullptr,
-                      nullptr, E, false, err, s)))
-    return st;
-  if ((st = transpose(W3, d, d, (int64_t)F * d, w.w13t + F, 2 * F, (int64_t)d * 2 * F, F, nullptr,
-                      nullptr, E, false, err, s)))
     return st;
   const int bnF = (F % 256 == 0) ? 256 : 128;
   const int bnD = (d % 256 == 0) ? 256 : 128;
@@ -891,22 +906,25 @@ int launch_grouped_ffn_backward(const __nv_bfloat16* recv, const __nv_bfloat16* 
     a.dgu = w.dgu;
     if ((st = launch_bwd_gemm<EPI_SWIGLU_BWD, false>(ma, m1, m3, a, s))) return st;
   }
-  // 5. dX rows = [dG | dU] [W1; W3] (K = 2F, bf16)
+  // 5. dX rows = [dG | dU] [W1; W3] (K = 2F, bf16): B read MN-major from W1 (K steps below
+  //    F/64) and W3 (the rest), each as [E*F rows, d columns] in boxes of 64 x 64
   {
-    CUtensorMap ma, mb;
+    CUtensorMap ma, m1, m3;
     if (!make_map16(&ma, w.dgu, RC, 2 * F, 2 * F, BM, true) ||
-        !make_map16(&mb, w.w13t, (int64_t)E * d, 2 * F, 2 * F, bnD, true))
+        !make_map16(&m1, W1, (int64_t)E * F, d, d, 64, true) ||
+        !make_map16(&m3, W3, (int64_t)E * F, d, d, 64, true))
       return MOE_ERR_DEVICE;
     BwdArgs a = base;
     a.n_blocks_n = d / bnD;
     a.k_blocks = 2 * F / BK;
+    a.kb_split = F / BK;
     a.bn_out = bnD;
     a.mma_n = bnD;
-    a.rows_per_expert = d;
+    a.rows_per_expert = F;
     a.out_ld = d;
     a.bf16 = 1;
     a.out = dx_rows;
-    if ((st = launch_bwd_gemm<EPI_BF16, false>(ma, mb, mb, a, s))) return st;
+    if ((st = launch_bwd_gemm<EPI_BF16, false, true>(ma, m1, m3, a, s))) return st;
   }
   // 6. transposed activations in the padded K layout (padding written as zeros)
   const int kc = (int)w.kc;
