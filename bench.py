@@ -37,9 +37,9 @@ UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes (read + write) per call of the dominant call (both grouped-FFN kernels) from
-# an ncu capture (profiles/ffn_kernel_near_balanced.md), keyed by workload and kernel
-# sources hash: it reads null as soon as the kernel sources change.
-TRAFFIC = {"near_balanced:bd5310e6636697e2": int((921.992960 + 63.940864 + 478.845952 + 84.311296) * 1e6)}
+# an ncu capture (profiles/ffn_kernel_near_balanced.md), keyed by workload, tile mode and
+# kernel sources hash: it reads null as soon as the kernel sources change.
+TRAFFIC = {}
 
 
 def sources_hash() -> str:
@@ -190,6 +190,9 @@ def run_ours(args, w: I.Workload, world, rank, local):
     logits = logits_h.to(device)
     x = x_h.to(device)
     W1, W3, W2 = I.make_weights(w, device=device)
+    if args.ffn_tile is not None:
+        M.set_ffn_tile_mode(args.ffn_tile)
+    ffn_tile = int(M.lib().moe_ffn_tile_mode())
     L = M.MoELayer(w.T, w.E, w.k, w.R, w.S, w.d, w.F, device=device, fused=args.fused)
     steps = [lambda: L.route(logits), lambda: L.measure(), lambda: L.balance(),
              lambda: L.prefetch(W1, W3, W2), lambda: L.dispatch(x),
@@ -329,7 +332,7 @@ def run_ours(args, w: I.Workload, world, rank, local):
     ffn_flops = units["moe_grouped_ffn"][1]
     peak_t = peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]
     achieved = ffn_flops / (ffn_ms * 1e-3) / 1e12
-    tkey = f"{w.name}:{sources_hash()}"
+    tkey = f"{w.name}:{ffn_tile}:{sources_hash()}"
     roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak_t, "unit": "TFLOP/s",
                 "frac": round(achieved / peak_t, 3), "traffic": TRAFFIC.get(tkey),
                 "kernel": "moe_grouped_ffn (gate-up and down tcgen05 GEMMs)",
@@ -353,6 +356,10 @@ def run_ours(args, w: I.Workload, world, rank, local):
                    "parallelism": f"replicas x{world} (ranks simulated in one GPU's HBM)",
                    "dispatch": ("fused: placement only, GEMM 1 gathers x[src[row]]" if args.fused
                                 else "row copy into recv, GEMM 1 reads recv"),
+                   "ffn_tile": ("256-row tiles on 2-CTA clusters (tcgen05 cta_group::2)"
+                                if ffn_tile == 1 and not args.fused
+                                else "128-row tiles, one CTA each (tcgen05 cta_group::1)"),
+                   "ffn_pair_clusters": M.ffn_pair_clusters() if ffn_tile == 1 else None,
                    "l2": "step working set (weights, pool, activations) far above the 126 MB L2",
                    "launch": "eager, one stream" if args.eager else
                              "K steps captured in one CUDA graph, replayed once; per-call "
@@ -569,6 +576,9 @@ def main():
                     help="also time the training step (forward + backward) and the backward calls")
     ap.add_argument("--fused", action="store_true",
                     help="fused dispatch: placement only, GEMM 1 gathers the token rows")
+    ap.add_argument("--ffn-tile", type=int, default=None, choices=[0, 1],
+                    help="grouped-FFN tiling: 0 = 128-row tiles, one CTA each; 1 = 256-row "
+                         "tiles on 2-CTA clusters (default: the library's)")
     args = ap.parse_args()
     w = I.WORKLOADS[args.config]
 

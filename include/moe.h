@@ -352,6 +352,24 @@ int moe_combine(const moe_bf16* y, const int32_t* perm, const float* gate, int T
                 int d, moe_bf16* out, const int32_t* err, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * Grouped-FFN tile mode (a B200 tiling choice; the pages fix no kernel design).
+ *   0  one CTA per 128-row x N tile (tcgen05.mma.cta_group::1), the default.
+ *   1  CTA pairs (2-CTA clusters) on 256-row x N tiles (tcgen05.mma.cta_group::2): each
+ *      SM loads its 128 rows of A and half of B, a third fewer operand bytes per MAC at
+ *      N = 256, at the price of padding each group's last tile to 256 rows.
+ * Process-wide, read when moe_grouped_ffn enqueues its kernels (set it before capturing a
+ * graph); moe_grouped_ffn_gather always uses mode 0.  Both modes compute the same sums in
+ * the same K order; outputs stay within the FFN tolerance of the oracle either way.
+ * moe_set_ffn_tile_mode returns MOE_OK, or MOE_ERR_ARG (mode unchanged) for a mode other
+ * than 0 or 1; moe_ffn_tile_mode returns the current mode.
+ * moe_ffn_pair_clusters: 2-CTA clusters mode 1 launches per GEMM on the current device
+ * (as many as fit at once), 0 before its first launch.
+ */
+int moe_set_ffn_tile_mode(int mode);
+int moe_ffn_tile_mode(void);
+int moe_ffn_pair_clusters(void);
+
+/* ---------------------------------------------------------------------------------
  * Diagnostic (no counterpart in the pages): runs the grouped FFN's bounded mbarrier wait
  * on a barrier that nothing ever arrives at, with a limit of `limit_us` microseconds
  * (1 .. 10^7).  The wait gives up, ORs MOE_DERR_TIMEOUT into *err and the kernel returns;

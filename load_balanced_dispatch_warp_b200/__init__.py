@@ -30,7 +30,8 @@ VARIANTS = ("moe_topk_biased", "moe_capacity_ledger")
 FUSED = ("moe_dispatch_index", "moe_grouped_ffn_gather")
 BACKWARD = ("moe_combine_backward", "moe_grouped_ffn_backward", "moe_dispatch_backward",
             "moe_topk_backward")
-HELPERS = ("moe_plan_get_layout", "moe_dispatch_workspace_words", "moe_status_string")
+HELPERS = ("moe_plan_get_layout", "moe_dispatch_workspace_words", "moe_status_string",
+           "moe_set_ffn_tile_mode", "moe_ffn_tile_mode", "moe_ffn_pair_clusters")
 
 
 class MoEError(RuntimeError):
@@ -86,6 +87,12 @@ def lib() -> ctypes.CDLL:
         L.moe_dispatch_workspace_words.restype = I64
         L.moe_ffn_backward_workspace_bytes.argtypes = [I, I, I, I, I, I, I]
         L.moe_ffn_backward_workspace_bytes.restype = I64
+        L.moe_set_ffn_tile_mode.argtypes = [I]
+        L.moe_set_ffn_tile_mode.restype = I
+        L.moe_ffn_tile_mode.argtypes = []
+        L.moe_ffn_tile_mode.restype = I
+        L.moe_ffn_pair_clusters.argtypes = []
+        L.moe_ffn_pair_clusters.restype = I
         L.moe_status_string.argtypes = [I]
         L.moe_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -149,6 +156,19 @@ def moe_capacity_ledger(counts, T, k, cf_num, cf_den, processed, overflow, paddi
         _ptr(counts, i32, "counts"), T, k, E, cf_num, cf_den, _ptr(processed, i32, "processed"),
         _ptr(overflow, i32, "overflow"), _ptr(padding, i32, "padding"), _ptr(totals, i32, "totals"),
         _ptr(err, i32, "err"), _stream(stream)), "moe_capacity_ledger")
+
+
+def set_ffn_tile_mode(mode: int) -> int:
+    """Grouped-FFN tiling: 0 = one CTA per 128-row tile, 1 = 2-CTA clusters on 256-row tiles
+    (tcgen05 cta_group::2).  Process-wide; returns the previous mode."""
+    prev = int(lib().moe_ffn_tile_mode())
+    _check(lib().moe_set_ffn_tile_mode(int(mode)), "moe_set_ffn_tile_mode")
+    return prev
+
+
+def ffn_pair_clusters() -> int:
+    """2-CTA clusters the pair mode launches per GEMM on the current device (0 before use)."""
+    return int(lib().moe_ffn_pair_clusters())
 
 
 def moe_selftest_bounded_wait(err, limit_us=50000, stream=None):

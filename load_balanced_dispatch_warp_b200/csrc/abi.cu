@@ -352,6 +352,12 @@ int moe_grouped_ffn_backward(const moe_bf16* recv, const moe_bf16* dy, const moe
       workspace_bytes, err, as_stream(stream));
 }
 
+int moe_set_ffn_tile_mode(int mode) { return moe::set_ffn_tile_mode(mode); }
+
+int moe_ffn_tile_mode(void) { return moe::ffn_tile_mode(); }
+
+int moe_ffn_pair_clusters(void) { return moe::ffn_pair_clusters(); }
+
 int moe_selftest_bounded_wait(int32_t* err, int limit_us, moe_stream_t stream) {
   if (!err || limit_us < 1 || limit_us > 10000000) return MOE_ERR_ARG;
   return moe::launch_bounded_wait_selftest(err, limit_us, as_stream(stream));

@@ -56,6 +56,10 @@ int launch_grouped_ffn_gather(const __nv_bfloat16* x, const int32_t* src, const 
                               const __half* P2, int T, int k, int E, int R, int S, int d, int F,
                               __half* h, __nv_bfloat16* y, int32_t* err, cudaStream_t s);
 int launch_bounded_wait_selftest(int32_t* err, int limit_us, cudaStream_t s);
+// grouped FFN tile mode (0: one CTA per 128-row tile, 1: 2-CTA clusters on 256-row tiles)
+int set_ffn_tile_mode(int mode);  // MOE_OK or MOE_ERR_ARG
+int ffn_tile_mode();
+int ffn_pair_clusters();  // clusters the pair mode launches on the current device (0: none yet)
 // backward pass (grouped_ffn_bwd.cu; the dispatch backward is launch_combine with
 // gate == nullptr)
 int64_t ffn_backward_workspace_bytes(int T, int k, int E, int R, int S, int d, int F, int G);

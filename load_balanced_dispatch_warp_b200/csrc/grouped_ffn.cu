@@ -542,6 +542,338 @@ __global__ void __launch_bounds__(FFN_THREADS, 1)
   }
 }
 
+// ----------------------------------------------------------------- CTA-pair variant
+//
+// The same two GEMMs with the 2-SM tensor-core instruction (tcgen05.mma.cta_group::2):
+// two CTAs of a cluster compute one 256-row x N tile.  CTA v of the pair holds rows
+// [128 v, 128 v + 128) of A and columns [v N/2, (v+1) N/2) of B in its own shared memory
+// and receives the accumulator of its 128 rows (all N columns) in its own TMEM; the
+// tensor cores of the two SMs exchange the B halves.  Each SM therefore loads 16 KiB of A
+// and N/2 * 128 bytes of B per K step instead of 16 KiB + N * 128 bytes: a third fewer
+// operand bytes per MAC at N = 256, at the price of 256-row padding of each group's last
+// tile.  For GEMM 1, CTA 0's B half is the W1 block and CTA 1's the W3 block, so the
+// accumulator columns are still gate | up and the SwiGLU epilogue is unchanged.
+//
+// Protocol (leader = CTA rank 0):
+//   full[s]    leader only: the leader's producer posts the transaction bytes of both
+//              CTAs' copies; both CTAs' TMA copies (.cta_group::2) complete on it.
+//   empty[s]   in both CTAs: one commit of the leader's MMA thread arrives on both.
+//   tfull[b]   in both CTAs: the same, after a tile's K loop.
+//   tempty[b]  leader only: 8 arrivals, one per epilogue warp of either CTA.
+//   drain      in both CTAs: committed after the last MMA, before TMEM is freed.
+// TMEM (512 columns, two accumulators of 256) is allocated and freed by warp 1 of both
+// CTAs with cta_group::2.  Barrier initialisation is published to the peer by a cluster
+// barrier before any role starts, and neither CTA leaves before a cluster barrier that
+// follows the last access to the other's shared memory.  A stale error word read by one
+// CTA of a pair and not the other cannot split the pair: the two CTAs OR their reads.
+constexpr int P_STAGES = 6;
+constexpr int P_BM = 2 * BM;                  // rows per pair tile
+constexpr int P_B_BYTES_MAX = 128 * BK * 2;   // this CTA's half of B at N = 256
+constexpr int P_STAGE_BYTES = A_BYTES + P_B_BYTES_MAX;
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_count_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the variable at shared::cta address `saddr` in CTA `rank`
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t caddr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(caddr) : "memory");
+  return v;
+}
+// every thread of both CTAs
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t caddr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr)
+               : "memory");
+}
+// TMA copy into this CTA's shared memory whose completion is counted on `bar_c`, a
+// shared::cluster barrier address that may lie in the peer CTA
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map,
+                                                 uint32_t bar_c, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_c)
+      : "memory");
+}
+// Arrival, once every pair MMA issued so far has completed, on the barrier at shared
+// offset `bar` in both CTAs of the pair (CTA mask 0b11).  A commit, not a copy: nothing is
+// loaded through the cluster.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar),
+      "h"((uint16_t)3)
+      : "memory");
+}
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// This CTA's part of pair tile t: its 128 rows and its half of the B columns.
+__device__ __forceinline__ Tile decode_pair_tile(int t, const FfnArgs& a, const int* s_prefix,
+                                                 int rank, bool swiglu) {
+  const int mt = t / a.n_blocks_n;
+  Tile tl;
+  tl.n_block = t - mt * a.n_blocks_n;
+  int lo = 0, hi = a.G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_prefix[mid] <= mt) lo = mid; else hi = mid - 1;
+  }
+  const int4 g = __ldg(a.groups + lo);
+  const int first = (mt - s_prefix[lo]) * P_BM + rank * BM;  // row offset inside the group
+  tl.a_row = g.x + first;
+  tl.valid_rows = max(0, min(BM, g.y - first));
+  const int ref = g.w;
+  tl.pool = ref >= a.E;
+  tl.b_row = (tl.pool ? ref - a.E : ref) * a.rows_per_expert + tl.n_block * a.bn_out +
+             (swiglu ? 0 : rank * (a.mma_n >> 1));
+  return tl;
+}
+
+template <bool SWIGLU>
+__global__ void __launch_bounds__(FFN_THREADS, 1)
+    ffn_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
+                    const __grid_constant__ CUtensorMap tm_b0,
+                    const __grid_constant__ CUtensorMap tm_b1,
+                    const __grid_constant__ CUtensorMap tm_p0,
+                    const __grid_constant__ CUtensorMap tm_p1, const FfnArgs args) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* stage_base = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P_STAGES * P_STAGE_BYTES);
+  // bars: full[P_STAGES], empty[P_STAGES], tfull[2], tempty[2], drain
+  int* s_misc = reinterpret_cast<int*>(bars + 2 * P_STAGES + 5);
+  // s_misc: [0] tmem base, [1] abort, [2] error word seen by this CTA, [3] by the pair
+  int* s_prefix = s_misc + 4;
+  int* s_scan = s_prefix + MAX_GROUPS + 1;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  volatile int* abort_flag = s_misc + 1;
+
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = smem_u32(bars + P_STAGES);
+  const uint32_t tfull0 = smem_u32(bars + 2 * P_STAGES);
+  const uint32_t tempty0 = smem_u32(bars + 2 * P_STAGES + 2);
+  const uint32_t drain = smem_u32(bars + 2 * P_STAGES + 4);
+  if (tid == 0) {
+    s_misc[1] = 0;
+    s_misc[2] = load_err(args.err);
+    for (int s = 0; s < P_STAGES; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull0 + 8 * b, 1);
+      mbar_init(tempty0 + 8 * b, 8);
+    }
+    mbar_init(drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  for (int g = tid; g < args.G; g += blockDim.x) {
+    const int rows = __ldg(&args.groups[g].y);
+    s_prefix[g] = rows > 0 ? (rows + P_BM - 1) / P_BM : 0;
+  }
+  __syncthreads();
+  const int total_m = block_exclusive_scan(s_prefix, args.G, s_scan);
+  if (tid == 0) s_prefix[args.G] = total_m;
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(s_misc)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  cluster_sync_all();  // barriers initialised and TMEM allocated in both CTAs
+  tc_fence_after();
+  if (tid == 0) s_misc[3] = s_misc[2] | (int)ld_cluster_u32(map_to_rank(smem_u32(s_misc + 2), rank ^ 1u));
+  __syncthreads();
+  const int total_tiles = s_misc[3] != 0 ? 0 : total_m * args.n_blocks_n;
+  const uint32_t tmem_base = static_cast<uint32_t>(s_misc[0]);
+  const int first_tile = (int)cluster_id_x();
+  const int tile_step = (int)cluster_count_x();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      const uint32_t b_half = (uint32_t)(args.mma_n >> 1) * BK * 2;
+      const uint32_t tx = 2u * (A_BYTES + b_half);
+      const uint32_t full_leader0 = map_to_rank(full0, 0);
+      const CUtensorMap* home = (SWIGLU && rank == 1) ? &tm_b1 : &tm_b0;
+      const CUtensorMap* pool = (SWIGLU && rank == 1) ? &tm_p1 : &tm_p0;
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0, issued_phase = 0;
+      bool ok = true;
+      for (int t = first_tile; ok && t < total_tiles; t += tile_step) {
+        const Tile tl = decode_pair_tile(t, args, s_prefix, (int)rank, SWIGLU);
+        const CUtensorMap* mb = tl.pool ? pool : home;
+        for (int kb = 0; kb < args.k_blocks; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, args.err)) { ok = false; break; }
+          const uint32_t sa = smem_u32(stage_base + stage * P_STAGE_BYTES);
+          if (leader) mbar_expect_tx(full0 + 8 * stage, tx);
+          tma_load_2d_pair(sa, &tm_a, full_leader0 + 8 * stage, kb * BK, tl.a_row);
+          tma_load_2d_pair(sa + A_BYTES, mb, full_leader0 + 8 * stage, kb * BK, tl.b_row);
+          issued_mask |= 1u << stage;
+          issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+          if (++stage == P_STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // No copy may still be landing when either CTA leaves.  The leader's full barriers
+      // count both CTAs' bytes; the peer sees its stages consumed on its empty barriers.
+      for (int s = 0; s < P_STAGES; ++s)
+        if (issued_mask & (1u << s)) {
+          volatile int no_abort = 0;
+          const uint32_t par = (issued_phase >> s) & 1u;
+          if (leader) {
+            mbar_wait(full0 + 8 * s, par, &no_abort, args.err);
+          } else if (!mbar_wait(empty0 + 8 * s, par, ok ? &no_abort : abort_flag, args.err)) {
+            const uint64_t t0 = globaltimer();  // error path: let copies in flight land
+            while (globaltimer() - t0 < 100000ull) {
+            }
+          }
+        }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer (leader CTA only)
+    if (lane == 0 && leader) {
+      const uint32_t idesc = make_idesc(P_BM, args.mma_n, SWIGLU);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int t = first_tile; t < total_tiles; t += tile_step) {
+        if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag, args.err)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+        bool ok = true;
+        for (int kb = 0; kb < args.k_blocks; ++kb) {
+          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, args.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(stage_base + stage * P_STAGE_BYTES);
+          const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / UMMA_K; ++kk)
+            tc_mma_pair(d_tmem, sw128_desc(sa + kk * UMMA_K * 2), sw128_desc(sb + kk * UMMA_K * 2),
+                        idesc, (kb | kk) != 0);
+          tc_commit_pair(empty0 + 8 * stage);
+          if (++stage == P_STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit_pair(tfull0 + 8 * acc);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      tc_commit_pair(drain);
+    }
+    if (lane == 0) {
+      // both CTAs: every MMA that reads this CTA's shared memory or writes its TMEM is done
+      volatile int no_abort = 0;
+      mbar_wait(drain, 0, &no_abort, args.err);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------ epilogue (warps 2-5)
+    const int quarter = warp & 3;
+    const int r_in = quarter * 32 + lane;
+    const uint32_t tempty_leader0 = map_to_rank(tempty0, 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = first_tile; t < total_tiles; t += tile_step) {
+      const Tile tl = decode_pair_tile(t, args, s_prefix, (int)rank, SWIGLU);
+      const bool ok = mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, args.err);
+      if (!__all_sync(MOE_FULL_MASK, ok)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * ACC_COLS;
+      const bool valid = r_in < tl.valid_rows;
+      uint16_t* orow = static_cast<uint16_t*>(args.out) + (int64_t)(tl.a_row + r_in) * args.out_ld +
+                       (int64_t)tl.n_block * args.bn_out;
+      if (SWIGLU) {
+#pragma unroll 1
+        for (int c = 0; c < 128 / 32; ++c) {
+          uint32_t g[32], u[32];
+          tmem_ld32(tbase + c * 32, g);
+          tmem_ld32(tbase + 128 + c * 32, u);
+          tmem_wait_ld();
+          uint32_t p[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+            const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+            p[i] = pack_f16_sat(silu(g0) * u0, silu(g1) * u1);
+          }
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < args.bn_out / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tbase + c * 32, v);
+          tmem_wait_ld();
+          uint32_t p[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) p[i] = pack_bf16(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(tempty_leader0 + 8 * acc);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync_all();  // all roles of both CTAs done
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(TMEM_COLS)
+                 : "memory");
+  }
+  cluster_sync_all();
+}
+
 // Self-test of the bounded wait: one thread waits on an mbarrier that nothing arrives at,
 // with a short limit; the wait gives up, sets MOE_DERR_TIMEOUT and the kernel returns.
 __global__ void bounded_wait_selftest_kernel(int32_t* err, uint64_t limit_ns) {
@@ -612,11 +944,77 @@ int launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b
   return launch_status();
 }
 
+
+size_t ffn_pair_smem_bytes() {
+  return 1024 + (size_t)P_STAGES * P_STAGE_BYTES + (2 * P_STAGES + 5) * 8 + 4 * 4 +
+         (MAX_GROUPS + 1) * 4 + 33 * 4;
+}
+
+int g_ffn_tile_mode = 0;        // 0: one CTA per 128-row tile, 1: CTA pairs
+int g_pair_clusters[64] = {0};  // co-resident 2-CTA clusters per device
+
+// Grid of the pair kernels: as many 2-CTA clusters as fit on the device at once (queried
+// once per device; a GPC with an odd number of free SMs leaves one of them idle).
+template <bool SWIGLU>
+int launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                const CUtensorMap& p0, const CUtensorMap& p1, const FfnArgs& args,
+                cudaStream_t s) {
+  static bool configured[64] = {false};
+  static int clusters[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 64) return MOE_ERR_LAUNCH;
+  const size_t smem = ffn_pair_smem_bytes();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(FFN_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (!configured[dev]) {
+    if (cudaFuncSetAttribute(ffn_pair_kernel<SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return MOE_ERR_LAUNCH;
+    cfg.gridDim = dim3(2 * (num_sms() / 2), 1, 1);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, ffn_pair_kernel<SWIGLU>, &cfg) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      return MOE_ERR_LAUNCH;
+    }
+    clusters[dev] = n < num_sms() / 2 ? n : num_sms() / 2;
+    g_pair_clusters[dev] = clusters[dev];
+    configured[dev] = true;
+  }
+  cfg.gridDim = dim3(2 * clusters[dev], 1, 1);
+  if (cudaLaunchKernelEx(&cfg, ffn_pair_kernel<SWIGLU>, a, b0, b1, p0, p1, args) != cudaSuccess)
+    return MOE_ERR_LAUNCH;
+  return launch_status();
+}
+
 }  // namespace
 
 int launch_bounded_wait_selftest(int32_t* err, int limit_us, cudaStream_t s) {
   bounded_wait_selftest_kernel<<<1, 32, 0, s>>>(err, (uint64_t)limit_us * 1000ull);
   return launch_status();
+}
+
+int set_ffn_tile_mode(int mode) {
+  if (mode != 0 && mode != 1) return MOE_ERR_ARG;
+  g_ffn_tile_mode = mode;
+  return MOE_OK;
+}
+
+int ffn_tile_mode() { return g_ffn_tile_mode; }
+
+int ffn_pair_clusters() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return dev < 64 ? g_pair_clusters[dev] : 0;
 }
 
 // GEMM 1 reads its rows from recv (x == nullptr) or gathers them as x[src[row]].
@@ -628,19 +1026,21 @@ int launch_grouped_ffn_impl(const __nv_bfloat16* recv, const __nv_bfloat16* x,
                             __nv_bfloat16* y, int32_t* err, cudaStream_t s) {
   if (T == 0) return MOE_OK;
   const bool gather = x != nullptr;
+  const bool pair = !gather && g_ffn_tile_mode == 1;
   const int64_t rows = (int64_t)T * k;  // R * C
   const int bn2 = (d % 256 == 0) ? 256 : 128;
+  const int w2_box = pair ? bn2 / 2 : bn2;  // a pair CTA loads half of GEMM 2's B rows
   CUtensorMap m_recv, m_w1, m_w3, m_p1, m_p3, m_h, m_w2, m_p2;
   if (!make_map(&m_w1, W1, (int64_t)E * F, d, 128) ||
       (!gather && !make_map(&m_recv, recv, rows, d, BM)) ||
       !make_map(&m_w3, W3, (int64_t)E * F, d, 128) ||
       !make_map(&m_h, h, rows, F, BM, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
-      !make_map(&m_w2, W2, (int64_t)E * d, F, bn2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+      !make_map(&m_w2, W2, (int64_t)E * d, F, w2_box, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
     return MOE_ERR_DEVICE;
   if (S > 0) {
     if (!make_map(&m_p1, P1, (int64_t)R * S * F, d, 128) ||
         !make_map(&m_p3, P3, (int64_t)R * S * F, d, 128) ||
-        !make_map(&m_p2, P2, (int64_t)R * S * d, F, bn2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
+        !make_map(&m_p2, P2, (int64_t)R * S * d, F, w2_box, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
       return MOE_ERR_DEVICE;
   } else {  // no pool: replica references cannot occur; pass the home maps
     m_p1 = m_w1;
@@ -664,6 +1064,7 @@ int launch_grouped_ffn_impl(const __nv_bfloat16* recv, const __nv_bfloat16* x,
   a1.gd = d;
   a1.gT = T;
   int st = gather ? launch_one<true, true>(m_w1, m_w1, m_w3, m_p1, m_p3, a1, s)
+           : pair ? launch_pair<true>(m_recv, m_w1, m_w3, m_p1, m_p3, a1, s)
                   : launch_one<true, false>(m_recv, m_w1, m_w3, m_p1, m_p3, a1, s);
   if (st != MOE_OK) return st;
   FfnArgs a2 = a1;
@@ -676,7 +1077,8 @@ int launch_grouped_ffn_impl(const __nv_bfloat16* recv, const __nv_bfloat16* x,
   a2.out = y;
   a2.gx = nullptr;
   a2.gsrc = nullptr;
-  return launch_one<false, false>(m_h, m_w2, m_w2, m_p2, m_p2, a2, s);
+  return pair ? launch_pair<false>(m_h, m_w2, m_w2, m_p2, m_p2, a2, s)
+              : launch_one<false, false>(m_h, m_w2, m_w2, m_p2, m_p2, a2, s);
 }
 
 int launch_grouped_ffn(const __nv_bfloat16* recv, const int32_t* plan,

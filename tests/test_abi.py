@@ -123,3 +123,19 @@ def test_backward_host_checks(lib):
     assert lib.moe_grouped_ffn_backward(*bad) == M.MOE_ERR_ARG
     bad = list(args); bad[13] = 200  # F % 128
     assert lib.moe_grouped_ffn_backward(*bad) == M.MOE_ERR_SHAPE
+
+
+def test_ffn_tile_mode_switch(lib):
+    """The tile-mode switch is host state only: checked, returns the previous mode."""
+    prev = lib.moe_ffn_tile_mode()
+    assert prev in (0, 1)
+    assert lib.moe_set_ffn_tile_mode(2) == M.MOE_ERR_ARG
+    assert lib.moe_set_ffn_tile_mode(-1) == M.MOE_ERR_ARG
+    assert lib.moe_ffn_tile_mode() == prev
+    assert lib.moe_set_ffn_tile_mode(1 - prev) == M.MOE_OK
+    assert lib.moe_ffn_tile_mode() == 1 - prev
+    assert M.set_ffn_tile_mode(prev) == 1 - prev
+    assert lib.moe_ffn_tile_mode() == prev
+    with pytest.raises(M.MoEError):
+        M.set_ffn_tile_mode(2)
+    assert lib.moe_ffn_tile_mode() == prev
