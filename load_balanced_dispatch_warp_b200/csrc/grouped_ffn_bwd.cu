@@ -268,6 +268,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   int* s_misc = reinterpret_cast<int*>(bars + 2 * STAGES + 5);
   int* s_prefix = s_misc + 4;
   int* s_scan = s_prefix + MAX_GROUPS + 1;
+  // fp32 epilogue: a 32 x 32 staging block per epilogue warp (16-byte aligned)
+  float* s_stage = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(s_scan + 33) + 15) &
+                                            ~static_cast<uintptr_t>(15));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   volatile int* abort_flag = s_misc + 1;
 
@@ -463,7 +466,17 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           }
         }
       } else if (EPI == EPI_F32) {
-        float* orow = static_cast<float*>(args.out) + tl.out_off + (int64_t)r_in * args.out_ld;
+        // Each 32-row x 32-column block goes through shared memory so that one store
+        // instruction writes four whole 128-byte row segments (lanes 8i..8i+7 one row)
+        // instead of 16 bytes in each of 32 rows.  16-byte chunk j of staged row r sits at
+        // chunk j ^ (r % 8): the row-per-lane writes and the segment-per-8-lanes reads are
+        // both free of bank conflicts.
+        float* stg = s_stage + (warp - 2) * 1024;
+        const int sr = lane >> 3;  // row of this lane within each group of four
+        const int sq = lane & 7;   // its 16-byte chunk of the 128-byte segment
+        const int rows_here = tl.valid_rows - quarter * 32;
+        float* obase = static_cast<float*>(args.out) + tl.out_off +
+                       (int64_t)(quarter * 32) * args.out_ld;
 #pragma unroll 1
         for (int c = 0; c < args.bn_out / 32; ++c) {
           uint32_t v[32];
@@ -474,12 +487,19 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = 0u;
           }
-          if (valid) {
-            float4* dst = reinterpret_cast<float4*>(orow + c * 32);
+          __syncwarp();  // the previous block's reads are done
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                   __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<float4*>(stg + lane * 32 + ((j ^ (lane & 7)) << 2)) =
+                make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                            __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int r = 4 * i + sr;
+            const float4 val = *reinterpret_cast<const float4*>(stg + r * 32 + ((sq ^ (r & 7)) << 2));
+            if (r < rows_here)
+              *reinterpret_cast<float4*>(obase + (int64_t)r * args.out_ld + c * 32 + sq * 4) = val;
           }
         }
       } else {
@@ -723,7 +743,7 @@ bool make_map16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, in
 
 size_t bwd_smem_bytes() {
   return 1024 + (size_t)STAGES * STAGE_BYTES + (2 * STAGES + 5) * 8 + 4 * 4 +
-         (MAX_GROUPS + 1) * 4 + 33 * 4;
+         (MAX_GROUPS + 1) * 4 + 33 * 4 + 16 + 4 * 32 * 32 * 4;
 }
 
 template <int EPI, bool WGRAD, bool BMN = false>

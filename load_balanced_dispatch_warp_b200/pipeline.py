@@ -59,8 +59,7 @@ class HostPipeline:
                 L.route(self.logits[s])
                 L.measure()
                 L.balance()
-                L.prefetch(W1, W3, W2)
-                L.dispatch(self.x[s])
+                L.prefetch_dispatch(self.x[s], W1, W3, W2)
                 if not L.fused:
                     self.inputs_free[s].record(self.s_comp)
                 L.expert_ffn(W1, W3, W2)
