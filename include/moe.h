@@ -180,6 +180,31 @@ int moe_plan_balanced(const int32_t* counts, int T, int k, int E, int R, int S,
                       int32_t* plan, int32_t* err, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * Routing, histogram and plan fused: moe_topk (or moe_topk_biased when bias != NULL),
+ * then moe_histogram_maxvio with the default home map (expert_to_rank = NULL), then
+ * moe_plan_balanced, in one kernel launch (plus two memsets: err and the workspace):
+ * every block routes its tokens, counts the chosen ids in shared memory and adds its
+ * counts to one of 16 partial histograms in the workspace (integer atomics); the last
+ * block to finish sums them into counts and computes loads, maxvio, balancedness and the
+ * plan.  Every
+ * output equals the separate calls' bit for bit, including after a non-finite logit
+ * (err = MOE_DERR_NONFINITE, counts and loads[0] zero, loads[1..R), maxvio,
+ * balancedness and plan untouched) and after a slot overflow (MOE_DERR_SLOTS).
+ *   logits [T,E] fp32; bias [E] fp32 or NULL; idx [T,k] int32, gate [T,k] fp32 (out);
+ *   counts [E], loads [R] int32, maxvio, balancedness fp64 (out);
+ *   plan int32[moe_plan_layout.words] (out); err int32 (out, reset to 0 first).
+ *   workspace  int32[moe_route_plan_workspace_words(E)], caller-owned device scratch,
+ *              any contents (zeroed by the call); one call at a time per workspace.
+ * Shape rules and host statuses: those of the three calls.
+ * moe_route_plan_workspace_words: words of that workspace, -1 for E outside [1, 1024].
+ */
+int64_t moe_route_plan_workspace_words(int E);
+int moe_route_plan(const float* logits, const float* bias, int T, int E, int k, int R, int S,
+                   int32_t* idx, float* gate, int32_t* counts, int32_t* loads, double* maxvio,
+                   double* balancedness, int32_t* plan, int32_t* workspace, int32_t* err,
+                   moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
  * Prefetch of the replicas into the pool.   [MoonEP] para. 3: duplicated experts are
  * prefetched before computation from one process-global pool, not per layer; the
  * framework keeps one contiguous weight tensor per projection.

@@ -27,7 +27,7 @@ DERR_NONFINITE, DERR_ID_RANGE, DERR_DUPLICATE, DERR_SLOTS, DERR_TIMEOUT = 1, 2, 
 ENTRY_POINTS = ("moe_topk", "moe_histogram_maxvio", "moe_plan_balanced", "moe_prefetch_replicas",
                 "moe_dispatch", "moe_grouped_ffn", "moe_combine")
 VARIANTS = ("moe_topk_biased", "moe_capacity_ledger")
-FUSED = ("moe_dispatch_index", "moe_grouped_ffn_gather")
+FUSED = ("moe_dispatch_index", "moe_grouped_ffn_gather", "moe_route_plan")
 BACKWARD = ("moe_combine_backward", "moe_grouped_ffn_backward", "moe_dispatch_backward",
             "moe_topk_backward")
 HELPERS = ("moe_plan_get_layout", "moe_dispatch_workspace_words", "moe_status_string",
@@ -76,6 +76,7 @@ def lib() -> ctypes.CDLL:
                                          I64, P, P],
             "moe_dispatch_backward": [P, P, I, I, I, P, P, P],
             "moe_topk_backward": [P, P, P, I, I, I, P, P, P],
+            "moe_route_plan": [P, P, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -85,6 +86,8 @@ def lib() -> ctypes.CDLL:
         L.moe_plan_get_layout.restype = ctypes.c_int
         L.moe_dispatch_workspace_words.argtypes = [I, I]
         L.moe_dispatch_workspace_words.restype = I64
+        L.moe_route_plan_workspace_words.argtypes = [I]
+        L.moe_route_plan_workspace_words.restype = I64
         L.moe_ffn_backward_workspace_bytes.argtypes = [I, I, I, I, I, I, I]
         L.moe_ffn_backward_workspace_bytes.restype = I64
         L.moe_set_ffn_tile_mode.argtypes = [I]
@@ -175,6 +178,29 @@ def moe_selftest_bounded_wait(err, limit_us=50000, stream=None):
     """Run the FFN's bounded wait on a barrier nothing arrives at (sets DERR_TIMEOUT)."""
     _check(lib().moe_selftest_bounded_wait(_ptr(err, torch.int32, "err"), int(limit_us), _stream(stream)),
            "moe_selftest_bounded_wait")
+
+
+def route_plan_workspace_words(E: int) -> int:
+    n = int(lib().moe_route_plan_workspace_words(E))
+    if n < 0:
+        raise MoEError(f"moe_route_plan_workspace_words: bad E={E}")
+    return n
+
+
+def moe_route_plan(logits, k, R, S, idx, gate, counts, loads, maxvio, balancedness, plan,
+                   workspace, err, bias=None, stream=None):
+    """moe_topk[_biased] + moe_histogram_maxvio (home map) + moe_plan_balanced in one launch."""
+    T, E = logits.shape
+    i32 = torch.int32
+    if workspace.numel() < route_plan_workspace_words(E):
+        raise ValueError("workspace smaller than moe_route_plan_workspace_words(E)")
+    _check(lib().moe_route_plan(
+        _ptr(logits, torch.float32, "logits"), _ptr(bias, torch.float32, "bias"), T, E, k, R, S,
+        _ptr(idx, i32, "idx"), _ptr(gate, torch.float32, "gate"), _ptr(counts, i32, "counts"),
+        _ptr(loads, i32, "loads"), _ptr(maxvio, torch.float64, "maxvio"),
+        _ptr(balancedness, torch.float64, "balancedness"), _ptr(plan, i32, "plan"),
+        _ptr(workspace, i32, "workspace"), _ptr(err, i32, "err"), _stream(stream)),
+        "moe_route_plan")
 
 
 def moe_histogram_maxvio(idx, E, R, counts, loads, maxvio, balancedness, err,
@@ -349,6 +375,7 @@ class MoELayer:
         self.balancedness = torch.empty(1, dtype=torch.float64, device=dev)
         self.plan = torch.empty(self.layout.words, dtype=i32, device=dev)
         self.workspace = torch.empty(max(1, dispatch_workspace_words(T, E)), dtype=i32, device=dev)
+        self.rp_workspace = torch.empty(route_plan_workspace_words(E), dtype=i32, device=dev)
         self.recv = None if self.fused else torch.empty(self.A, d, dtype=bf, device=dev)
         self.perm = torch.empty(T, k, dtype=i32, device=dev)
         self.src = torch.empty(self.A, dtype=i32, device=dev)
@@ -412,6 +439,12 @@ class MoELayer:
     def combine(self, stream=None):
         moe_combine(self.y, self.perm, self.gate, self.out, self.err, stream)
 
+    def route_plan(self, logits, stream=None):
+        """route + measure (home map) + balance as one fused launch (same outputs)."""
+        moe_route_plan(logits, self.k, self.R, self.S, self.idx, self.gate, self.counts,
+                       self.loads, self.maxvio, self.balancedness, self.plan, self.rp_workspace,
+                       self.err, stream=stream)
+
     def prefetch_dispatch(self, x, W1, W3, W2, stream=None):
         """Replica prefetch and dispatch, both of which need only the plan.  The prefetch is
         enqueued on a side stream forked from ``stream`` (after everything enqueued there so
@@ -435,11 +468,10 @@ class MoELayer:
         main.wait_event(self._ev_pref)
 
     def forward(self, logits, x, W1, W3, W2, stream=None):
-        """The whole path on the current stream (the prefetch forked off and joined back, see
-        ``prefetch_dispatch``); returns ``out`` [T,d] bf16 (device)."""
-        self.route(logits, stream)
-        self.measure(None, stream)
-        self.balance(stream)
+        """The whole path on the current stream: routing, histogram and plan fused
+        (``route_plan``), the prefetch forked off and joined back (``prefetch_dispatch``),
+        the grouped FFN, the combine; returns ``out`` [T,d] bf16 (device)."""
+        self.route_plan(logits, stream)
         self.prefetch_dispatch(x, W1, W3, W2, stream)
         self.expert_ffn(W1, W3, W2, stream)
         self.combine(stream)
@@ -477,7 +509,7 @@ class MoELayer:
 
     # kernels launched by forward() (for launch accounting)
     def kernels_per_forward(self) -> int:
-        n = (1 if self.T > 0 else 0) + 1 + 1  # topk, histogram, plan
+        n = 1                                 # routing + histogram + plan (fused)
         n += 1 if self.S > 0 else 0           # prefetch
         n += (2 if self.fused else 3) if self.T > 0 else 0  # tile counts, ranks[, row scatter]
         n += 2 if self.T > 0 else 0           # two grouped GEMMs

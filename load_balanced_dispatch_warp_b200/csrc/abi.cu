@@ -154,6 +154,27 @@ int moe_plan_balanced(const int32_t* counts, int T, int k, int E, int R, int S, 
   return moe::launch_plan(counts, T, k, E, R, S, plan, L, err, as_stream(stream));
 }
 
+int64_t moe_route_plan_workspace_words(int E) {
+  if (E < 1 || E > 1024) return -1;
+  return moe::route_plan_workspace_words(E);
+}
+
+int moe_route_plan(const float* logits, const float* bias, int T, int E, int k, int R, int S,
+                   int32_t* idx, float* gate, int32_t* counts, int32_t* loads, double* maxvio,
+                   double* balancedness, int32_t* plan, int32_t* workspace, int32_t* err,
+                   moe_stream_t stream) {
+  if (!err || !counts || !loads || !maxvio || !balancedness || !plan || !workspace)
+    return MOE_ERR_ARG;
+  if (T > 0 && (!logits || !idx || !gate)) return MOE_ERR_ARG;
+  MOE_TRY(check_route(T, E, k));
+  MOE_TRY(check_ranks(T, k, E, R, true));
+  MOE_TRY(check_groups(E, R, S));
+  moe_plan_layout L;
+  MOE_TRY(moe_plan_get_layout(E, R, S, &L));
+  return moe::launch_route_plan(logits, bias, T, E, k, R, S, idx, gate, counts, loads, maxvio,
+                                balancedness, plan, L, workspace, err, as_stream(stream));
+}
+
 int moe_prefetch_replicas(const int32_t* plan, const moe_bf16* W1, const moe_bf16* W3,
                           const moe_f16* W2, int E, int R, int S, int d, int F,
                           moe_bf16* P1, moe_bf16* P3, moe_f16* P2, const int32_t* err,

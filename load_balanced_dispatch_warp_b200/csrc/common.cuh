@@ -35,6 +35,11 @@ int launch_histogram(const int32_t* idx, int T, int k, int E, int R, const int32
                      int32_t* err, cudaStream_t s);
 int launch_plan(const int32_t* counts, int T, int k, int E, int R, int S, int32_t* plan,
                 const moe_plan_layout& L, int32_t* err, cudaStream_t s);
+int64_t route_plan_workspace_words(int E);
+int launch_route_plan(const float* logits, const float* bias, int T, int E, int k, int R,
+                      int S, int32_t* idx, float* gate, int32_t* counts, int32_t* loads,
+                      double* maxvio, double* bal, int32_t* plan, const moe_plan_layout& L,
+                      int32_t* ws, int32_t* err, cudaStream_t s);
 int launch_prefetch(const int32_t* plan, const moe_plan_layout& L, const __nv_bfloat16* W1,
                     const __nv_bfloat16* W3, const __half* W2, int E, int R, int S, int d,
                     int F, __nv_bfloat16* P1, __nv_bfloat16* P3, __half* P2,

@@ -1,183 +1,25 @@
-// Equal-load plan with redundant expert copies, in one CTA.
-//
-// The MoonEP news article (paragraphs 3-4) fixes the contract -- every rank receives
-// exactly T*k/R rows, a few redundant expert copies are planned on the fly from the router
-// output, and each copy takes one of S prefetch slots per rank from one global pool -- but
-// gives no algorithm.  This kernel computes the "keep small, stream the rest" plan:
-//   - rank r owns experts [rB, (r+1)B); ordered by (count, id) ascending, its experts
-//     are kept whole while their running sum fits in C = T*k/R; the rest are streamed;
-//   - the streamed experts in id order form one stream, cut by the ranks' leftover rooms
-//     in rank order; each foreign run in a rank's piece is a replica taking the next slot.
-// Everything is integer arithmetic, block scans and ballots (one warp per rank):
-// deterministic.
-#include "common.cuh"
+// Stand-alone plan call: one CTA runs plan_block (plan_body.cuh) on the histogram's counts.
+#include "plan_body.cuh"
 
 namespace moe {
 namespace {
-
-constexpr int kPlanThreads = 256;
-constexpr int kPlanWarps = kPlanThreads / 32;
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __restrict__ counts,
                                                             int T, int k, int E, int R, int S,
                                                             int32_t* __restrict__ plan,
                                                             moe_plan_layout L,
                                                             int32_t* __restrict__ err) {
-  __shared__ int s_c[1024];       // counts
-  __shared__ int s_kept[1024];    // 1 if kept whole at home
-  __shared__ int s_so[1025];      // stream offsets (exclusive scan of streamed counts)
-  __shared__ int s_room[1025];    // rooms, then their exclusive prefix
-  __shared__ int s_kr[1024];      // kept rows per rank
-  __shared__ int s_off[1024];     // local row offset of a kept expert, -1 otherwise
-  __shared__ int s_sidx[1025];    // streamed experts (non-zero stream length) in id order
-  __shared__ int s_nrep[1025];    // replicas per rank, then their exclusive prefix
-  __shared__ int s_scan[33];
-  __shared__ int s_ns;
+  extern __shared__ int s_plan[];  // plan_smem_words(E, R)
   if (block_should_stop(err)) return;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int B = E / R;
-  const int C = (int)(((long long)T * k) / R);
-
-  for (int e = tid; e < E; e += blockDim.x) s_c[e] = counts[e];
-  for (int r = tid; r < R; r += blockDim.x) s_kr[r] = 0;
-  __syncthreads();
-
-  // keep test: inclusive running sum of the rank's experts in (count, id) order <= C
-  for (int e = tid; e < E; e += blockDim.x) {
-    const int r0 = (e / B) * B, c = s_c[e];
-    long long cum = c;
-    for (int f = r0; f < r0 + B; ++f) {
-      const int cf = s_c[f];
-      if (cf < c || (cf == c && f < e)) cum += cf;
-    }
-    const int kept = cum <= C;
-    s_kept[e] = kept;
-    if (kept && c) atomicAdd(&s_kr[e / B], c);
-  }
-  __syncthreads();
-
-  // local offsets of kept experts (id order); stream lengths; rooms
-  for (int e = tid; e < E; e += blockDim.x) {
-    int off = -1;
-    if (s_kept[e]) {
-      off = 0;
-      for (int f = (e / B) * B; f < e; ++f)
-        if (s_kept[f]) off += s_c[f];
-    }
-    s_off[e] = off;
-    s_so[e] = s_kept[e] ? 0 : s_c[e];
-    s_nrep[e] = (!s_kept[e] && s_c[e] > 0) ? 1 : 0;  // streamed flag (s_nrep as temp)
-  }
-  for (int r = tid; r < R; r += blockDim.x) s_room[r] = C - s_kr[r];
-  __syncthreads();
-  const int stream_len = block_exclusive_scan(s_so, E, s_scan);
-  const int room_total = block_exclusive_scan(s_room, R, s_scan);
-  // compact list of streamed experts in id order (= stream order)
-  const int n_streamed = block_exclusive_scan(s_nrep, E, s_scan);
-  for (int e = tid; e < E; e += blockDim.x)
-    if (!s_kept[e] && s_c[e] > 0) s_sidx[s_nrep[e]] = e;
-  if (tid == 0) {
-    s_so[E] = stream_len;
-    s_room[R] = room_total;
-    s_ns = n_streamed;
-  }
-  __syncthreads();
-
-  int32_t* kept_rows = plan + L.kept_rows;
-  int32_t* room_prefix = plan + L.room_prefix;
-  int32_t* home_off = plan + L.expert_home_off;
-  int32_t* stream_off = plan + L.stream_off;
-  int32_t* rep = plan + L.replica_expert;
-  int32_t* rep_list = plan + L.replica_list;
-  int32_t* n_groups = plan + L.n_groups;
-  int32_t* groups = plan + L.groups;
-  for (int r = tid; r < R; r += blockDim.x) kept_rows[r] = s_kr[r];
-  for (int r = tid; r <= R; r += blockDim.x) room_prefix[r] = s_room[r];
-  for (int e = tid; e < E; e += blockDim.x) home_off[e] = s_off[e];
-  for (int e = tid; e <= E; e += blockDim.x) stream_off[e] = s_so[e];
-
-  // one warp per rank: its kept experts (id order), then the runs of its stream piece
-  const int G = B + S;
-  for (int u = warp; u < R; u += kPlanWarps) {
-    int32_t* gu = groups + (int64_t)u * G * 4;
-    int g = 0;
-    for (int c0 = 0; c0 < B; c0 += 32) {
-      const int e = u * B + c0 + lane;
-      const bool on = c0 + lane < B && s_kept[e] && s_c[e] > 0;
-      const uint32_t m = __ballot_sync(MOE_FULL_MASK, on);
-      if (on) {
-        int4* rec = reinterpret_cast<int4*>(gu) + g + __popc(m & lanemask_lt());
-        *rec = make_int4(u * C + s_off[e], s_c[e], e, e);
-      }
-      g += __popc(m);
-    }
-    const int lo = s_room[u], hi = s_room[u + 1];
-    int nrep = 0;
-    if (lo < hi) {
-      // first streamed expert whose stream range ends after lo
-      int a = 0, b = s_ns - 1;
-      while (a < b) {
-        const int mid = (a + b) >> 1;
-        const int em = s_sidx[mid];
-        if (s_so[em] + s_c[em] > lo) b = mid; else a = mid + 1;
-      }
-      for (int i0 = a; i0 < s_ns; i0 += 32) {
-        const int i = i0 + lane;
-        int e = -1, s0 = 0, s1 = 0;
-        if (i < s_ns) {
-          e = s_sidx[i];
-          s0 = max(lo, s_so[e]);
-          s1 = min(hi, s_so[e] + s_c[e]);
-        }
-        const bool on = e >= 0 && s0 < s1;
-        const bool foreign = on && e / B != u;
-        const uint32_t mfor = __ballot_sync(MOE_FULL_MASK, foreign);
-        const int slot = nrep + __popc(mfor & lanemask_lt());
-        // a run at its home rank is always recorded; a replica only while slots remain
-        // (more than S replicas leaves the plan invalid: MOE_DERR_SLOTS below)
-        const bool write = on && (!foreign || slot < S);
-        const uint32_t mw = __ballot_sync(MOE_FULL_MASK, write);
-        if (write) {
-          int ref = e;
-          if (foreign) {
-            rep[u * S + slot] = e;
-            ref = E + u * S + slot;
-          }
-          int4* rec = reinterpret_cast<int4*>(gu) + g + __popc(mw & lanemask_lt());
-          *rec = make_int4(u * C + s_kr[u] + (s0 - lo), s1 - s0, e, ref);
-        }
-        g += __popc(mw);
-        nrep += __popc(mfor);
-        // stop once this chunk reached past the piece
-        const bool past = e < 0 || s_so[e] >= hi;
-        if (__any_sync(MOE_FULL_MASK, past)) break;
-      }
-    }
-    for (int i = g * 4 + lane; i < 4 * G; i += 32) gu[i] = -1;
-    for (int s = min(nrep, S) + lane; s < S; s += 32) rep[u * S + s] = -1;
-    if (lane == 0) {
-      n_groups[u] = g;
-      s_nrep[u] = min(nrep, S);
-      if (nrep > S) atomicOr(err, MOE_DERR_SLOTS);
-    }
-  }
-  __syncthreads();
-  // compact list of filled slots in ascending slot order (for the prefetch copy)
-  const int n_filled = block_exclusive_scan(s_nrep, R, s_scan);
-  for (int u = tid; u < R; u += blockDim.x) {
-    const int base = s_nrep[u];
-    const int n = (u + 1 < R ? s_nrep[u + 1] : n_filled) - base;
-    for (int s = 0; s < n; ++s) rep_list[1 + base + s] = u * S + s;
-  }
-  for (int i = n_filled + tid; i < R * S; i += blockDim.x) rep_list[1 + i] = -1;
-  if (tid == 0) rep_list[0] = n_filled;
+  plan_block(counts, T, k, E, R, S, plan, L, err, s_plan);
 }
 
 }  // namespace
 
 int launch_plan(const int32_t* counts, int T, int k, int E, int R, int S, int32_t* plan,
                 const moe_plan_layout& L, int32_t* err, cudaStream_t s) {
-  plan_kernel<<<1, kPlanThreads, 0, s>>>(counts, T, k, E, R, S, plan, L, err);
+  plan_kernel<<<1, kPlanThreads, sizeof(int) * plan_smem_words(E, R), s>>>(counts, T, k, E, R,
+                                                                         S, plan, L, err);
   return launch_status();
 }
 

@@ -7,6 +7,7 @@
 // expert->rank map; balancedness = mean/max), with maxvio = (max - mean)/mean as named in
 // the MoonEP news article.
 #include "common.cuh"
+#include "plan_body.cuh"
 
 namespace moe {
 namespace {
@@ -143,19 +144,15 @@ __device__ __noinline__ void topk_exact(const float* x, const float* b, int E, i
 // Otherwise (equal keys across lanes, a lane holding three of the top-k, overflow to
 // -inf) the warp runs topk_exact on the same registers.  Gates: softmax over the chosen
 // experts' unbiased logits in fp32.  K > 0 fixes k at compile time (K == k).
-template <int VPL, int K, bool BIASED>
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits,
-                                                   const float* __restrict__ bias, int T,
-                                                   int E, int k_rt, int32_t* __restrict__ idx,
-                                                   float* __restrict__ gate,
-                                                   int32_t* __restrict__ err) {
-  __shared__ uint32_t s_key[8][32];
-  __shared__ int s_id[8][32];
-  __shared__ float s_raw[8][32];
-  const int k = K > 0 ? K : k_rt;
-  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  const int64_t t = (int64_t)blockIdx.x * 8 + wib;
-  if (t >= T) return;
+// Token t by the calling warp.  Returns false (err flagged, nothing written) on a
+// non-finite logit or bias.  COUNT: each written id is also added to counts[id].
+template <int VPL, int K, bool BIASED, bool COUNT>
+__device__ __forceinline__ bool topk_token(const float* __restrict__ logits,
+                                           const float* __restrict__ bias, int64_t t, int E,
+                                           int k, int lane, uint32_t* s_key, int* s_id,
+                                           float* s_raw, int32_t* __restrict__ idx,
+                                           float* __restrict__ gate, int32_t* __restrict__ counts,
+                                           int32_t* __restrict__ err) {
   float b[VPL];
 #pragma unroll
   for (int i = 0; i < VPL; ++i) b[i] = 0.f;
@@ -169,7 +166,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
     }
     if (__any_sync(MOE_FULL_MASK, bad)) {
       if (lane == 0) atomicOr(err, MOE_DERR_NONFINITE);
-      return;
+      return false;
     }
   }
   const float* row = logits + t * E;
@@ -189,7 +186,7 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   }
   if (__any_sync(MOE_FULL_MASK, !(z == 0.f))) {
     if (lane == 0) atomicOr(err, MOE_DERR_NONFINITE);
-    return;
+    return false;
   }
   float h1 = key[0], h2 = -INFINITY;
 #pragma unroll
@@ -242,16 +239,18 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
     if (npop > 0) {
       idx[t * k + r1] = lane + 32 * s1;
       gate[t * k + r1] = e1 / sum;
+      if (COUNT) atomicAdd(counts + lane + 32 * s1, 1);
     }
     if (npop > 1) {
       idx[t * k + r2] = lane + 32 * s2;
       gate[t * k + r2] = e2 / sum;
+      if (COUNT) atomicAdd(counts + lane + 32 * s2, 1);
     }
-    return;
+    return true;
   }
   float my_val;
   int my_id;
-  topk_exact<VPL, BIASED>(x, b, E, k, lane, s_key[wib], s_id[wib], s_raw[wib], my_val, my_id);
+  topk_exact<VPL, BIASED>(x, b, E, k, lane, s_key, s_id, s_raw, my_val, my_id);
   float top = lane < k ? my_val : -INFINITY;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) top = fmaxf(top, __shfl_xor_sync(MOE_FULL_MASK, top, o));
@@ -260,7 +259,26 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   if (lane < k) {
     idx[t * k + lane] = my_id;
     gate[t * k + lane] = ex / sum;
+    if (COUNT) atomicAdd(counts + my_id, 1);
   }
+  return true;
+}
+
+template <int VPL, int K, bool BIASED>
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits,
+                                                   const float* __restrict__ bias, int T,
+                                                   int E, int k_rt, int32_t* __restrict__ idx,
+                                                   float* __restrict__ gate,
+                                                   int32_t* __restrict__ err) {
+  __shared__ uint32_t s_key[8][32];
+  __shared__ int s_id[8][32];
+  __shared__ float s_raw[8][32];
+  const int k = K > 0 ? K : k_rt;
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int64_t t = (int64_t)blockIdx.x * 8 + wib;
+  if (t >= T) return;
+  topk_token<VPL, K, BIASED, false>(logits, bias, t, E, k, lane, s_key[wib], s_id[wib],
+                                    s_raw[wib], idx, gate, nullptr, err);
 }
 
 // Fixed-capacity ledger of "MoE Load Balancing: Find Expert Hotspots" ("Make expert
@@ -315,6 +333,56 @@ __global__ void __launch_bounds__(256) capacity_kernel(const int32_t* __restrict
     totals[1] = (int32_t)a;
     totals[2] = (int32_t)b;
     totals[3] = (int32_t)c;
+  }
+}
+
+// Last block of a histogram: the rank loads of `counts` under the expert->rank map
+// (nullptr: e / (E/R)), maxvio = (R*max - A)/A and balancedness = A/(R*max) from exact
+// integers, one fp64 rounding each.  s_hist: R ints of shared memory; s_max: 32 ints.
+__device__ __noinline__ void hist_finish(const int32_t* __restrict__ counts, int T, int k, int E,
+                                         int R, const int32_t* __restrict__ map,
+                                         int32_t* __restrict__ loads, double* __restrict__ maxvio,
+                                         double* __restrict__ bal, int32_t* __restrict__ err,
+                                         int* s_hist, int* s_max) {
+  const int lane = threadIdx.x & 31;
+  const int B = E / R;
+  for (int r = threadIdx.x; r < R; r += blockDim.x) s_hist[r] = 0;
+  __syncthreads();
+  int bad = 0;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int r = map ? __ldg(map + e) : e / B;
+    if (r < 0 || r >= R) {
+      bad = 1;
+    } else {
+      const int c = __ldcg(counts + e);
+      if (c) atomicAdd(&s_hist[r], c);
+    }
+  }
+  if (bad) atomicOr(err, MOE_DERR_ID_RANGE);
+  __syncthreads();
+  int mx = 0;
+  for (int r = threadIdx.x; r < R; r += blockDim.x) {
+    loads[r] = s_hist[r];
+    mx = max(mx, s_hist[r]);
+  }
+  mx = __reduce_max_sync(MOE_FULL_MASK, mx);
+  if (lane == 0) s_max[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const int nw = (blockDim.x + 31) >> 5;
+    int v = threadIdx.x < nw ? s_max[threadIdx.x] : 0;
+    v = __reduce_max_sync(MOE_FULL_MASK, v);
+    if (threadIdx.x == 0) {
+      const long long A = (long long)T * k;
+      const long long top = (long long)R * v;
+      if (A == 0 || v == 0) {
+        *maxvio = 0.0;
+        *bal = 1.0;
+      } else {
+        *maxvio = (double)(top - A) / (double)A;
+        *bal = (double)A / (double)top;
+      }
+    }
   }
 }
 
@@ -374,45 +442,7 @@ __global__ void __launch_bounds__(512) hist_kernel(const int32_t* __restrict__ i
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  const int B = E / R;
-  for (int r = threadIdx.x; r < R; r += blockDim.x) s_hist[r] = 0;
-  __syncthreads();
-  int bad = 0;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    const int r = map ? __ldg(map + e) : e / B;
-    if (r < 0 || r >= R) {
-      bad = 1;
-    } else {
-      const int c = __ldcg(counts + e);
-      if (c) atomicAdd(&s_hist[r], c);
-    }
-  }
-  if (bad) atomicOr(err, MOE_DERR_ID_RANGE);
-  __syncthreads();
-  int mx = 0;
-  for (int r = threadIdx.x; r < R; r += blockDim.x) {
-    loads[r] = s_hist[r];
-    mx = max(mx, s_hist[r]);
-  }
-  mx = __reduce_max_sync(MOE_FULL_MASK, mx);
-  if (lane == 0) s_max[threadIdx.x >> 5] = mx;
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    const int nw = (blockDim.x + 31) >> 5;
-    int v = threadIdx.x < nw ? s_max[threadIdx.x] : 0;
-    v = __reduce_max_sync(MOE_FULL_MASK, v);
-    if (threadIdx.x == 0) {
-      const long long A = (long long)T * k;
-      const long long top = (long long)R * v;
-      if (A == 0 || v == 0) {
-        *maxvio = 0.0;
-        *bal = 1.0;
-      } else {
-        *maxvio = (double)(top - A) / (double)A;
-        *bal = (double)A / (double)top;
-      }
-    }
-  }
+  hist_finish(counts, T, k, E, R, map, loads, maxvio, bal, err, s_hist, s_max);
 }
 
 // One warp per token, 8 warps per block.  Unbiased calls with k in {2, 4, 6, 8} and up to
@@ -448,6 +478,98 @@ int launch_topk_impl(const float* logits, const float* bias, int T, int E, int k
   else if (E <= 512) launch_topk_vpl<16>(logits, bias, T, E, k, idx, gate, err, s);
   else launch_topk_vpl<32>(logits, bias, T, E, k, idx, gate, err, s);
   return launch_status();
+}
+
+
+// Routing, histogram and plan in one launch (the three calls' outputs, bit for bit).  Every
+// block runs top-k for its 8 tokens, counting the chosen ids in shared memory, then adds its
+// non-zero counts to one of kCountCopies partial histograms in `ws` (copy = block index
+// mod kCountCopies: integer atomics, order-independent, spread over the copies so that no
+// counter takes more than a 1/kCountCopies share of the blocks).  The last block to finish
+// (ticket in ws[kCountCopies * E]; ws zeroed before the launch) sums the copies into
+// counts, computes the home-map rank loads, maxvio and balancedness, then the plan.  After
+// a non-finite logit it leaves what the separate calls leave: counts and loads[0] zero, the
+// rest untouched.
+constexpr int kCountCopies = 16;
+
+template <int VPL, int K, bool BIASED>
+__global__ void __launch_bounds__(kPlanThreads) route_plan_kernel(
+    const float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int k_rt,
+    int R, int S, int32_t* __restrict__ idx, float* __restrict__ gate,
+    int32_t* __restrict__ counts, int32_t* __restrict__ loads, double* __restrict__ maxvio,
+    double* __restrict__ bal, int32_t* __restrict__ plan, const moe_plan_layout L,
+    int32_t* __restrict__ ws, int32_t* __restrict__ err) {
+  static_assert(kPlanThreads == 256, "8 tokens per block, one warp each");
+  __shared__ uint32_t s_key[8][32];
+  __shared__ int s_id[8][32];
+  __shared__ float s_raw[8][32];
+  // [0, E): this block's counts, later the last block's rank loads; then the plan's words
+  extern __shared__ int s_dyn[];
+  __shared__ int s_max[32];
+  __shared__ int s_last;
+  const int k = K > 0 ? K : k_rt;
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_dyn[e] = 0;
+  __syncthreads();
+  const int64_t t = (int64_t)blockIdx.x * 8 + wib;
+  if (t < T)
+    topk_token<VPL, K, BIASED, true>(logits, bias, t, E, k, lane, s_key[wib], s_id[wib],
+                                     s_raw[wib], idx, gate, s_dyn, err);
+  __syncthreads();
+  int32_t* copy = ws + (int64_t)(blockIdx.x % kCountCopies) * E;
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    if (s_dyn[e]) atomicAdd(copy + e, s_dyn[e]);
+  // last block: every other block's counts are visible once its ticket is
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(ws + kCountCopies * E, 1) == (int)gridDim.x - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  if (load_err(err) != 0) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x) counts[e] = 0;
+    if (threadIdx.x == 0) loads[0] = 0;
+    return;
+  }
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int c = 0;
+#pragma unroll 4
+    for (int p = 0; p < kCountCopies; ++p) c += __ldcg(ws + (int64_t)p * E + e);
+    counts[e] = c;
+  }
+  __threadfence_block();
+  __syncthreads();
+  hist_finish(counts, T, k, E, R, nullptr, loads, maxvio, bal, err, s_dyn, s_max);
+  __syncthreads();
+  plan_block(counts, T, k, E, R, S, plan, L, err, s_dyn + E);
+}
+
+template <int VPL>
+void launch_route_plan_vpl(const float* logits, const float* bias, int T, int E, int k, int R,
+                           int S, int32_t* idx, float* gate, int32_t* counts, int32_t* loads,
+                           double* maxvio, double* bal, int32_t* plan, const moe_plan_layout& L,
+                           int32_t* ws, int32_t* err, cudaStream_t s) {
+  const unsigned grid = T > 0 ? (unsigned)(((int64_t)T + 7) / 8) : 1u;
+  const size_t smem = sizeof(int) * (size_t)(E + plan_smem_words(E, R));
+#define MOE_RP(KK, B)                                                                           \
+  route_plan_kernel<VPL, KK, B><<<grid, kPlanThreads, smem, s>>>(logits, bias, T, E, k, R, S, idx, \
+                                                                 gate, counts, loads, maxvio, bal, \
+                                                                 plan, L, ws, err)
+  if (bias) {
+    MOE_RP(0, true);
+    return;
+  }
+  if constexpr (VPL <= 8) {
+    switch (k) {
+      case 8: MOE_RP(8, false); return;
+      case 6: MOE_RP(6, false); return;
+      case 4: MOE_RP(4, false); return;
+      case 2: MOE_RP(2, false); return;
+      default: break;
+    }
+  }
+  MOE_RP(0, false);
+#undef MOE_RP
 }
 
 }  // namespace
@@ -489,6 +611,28 @@ int launch_histogram(const int32_t* idx, int T, int k, int E, int R, const int32
   blocks = T > 0 ? (T + per - 1) / per : 1;
   const size_t smem = sizeof(int) * (size_t)(E > R ? E : R);
   hist_kernel<<<blocks, threads, smem, s>>>(idx, T, k, E, R, per, map, counts, loads, maxvio, bal, err);
+  return launch_status();
+}
+
+int64_t route_plan_workspace_words(int E) { return (int64_t)kCountCopies * E + 1; }
+
+int launch_route_plan(const float* logits, const float* bias, int T, int E, int k, int R,
+                      int S, int32_t* idx, float* gate, int32_t* counts, int32_t* loads,
+                      double* maxvio, double* bal, int32_t* plan, const moe_plan_layout& L,
+                      int32_t* ws, int32_t* err, cudaStream_t s) {
+  if (cudaMemsetAsync(err, 0, sizeof(int32_t), s) != cudaSuccess ||
+      cudaMemsetAsync(ws, 0, sizeof(int32_t) * (size_t)route_plan_workspace_words(E), s) !=
+          cudaSuccess)
+    return MOE_ERR_LAUNCH;
+#define MOE_RP_VPL(V) \
+  launch_route_plan_vpl<V>(logits, bias, T, E, k, R, S, idx, gate, counts, loads, maxvio, bal, plan, L, ws, err, s)
+  if (E <= 32) MOE_RP_VPL(1);
+  else if (E <= 64) MOE_RP_VPL(2);
+  else if (E <= 128) MOE_RP_VPL(4);
+  else if (E <= 256) MOE_RP_VPL(8);
+  else if (E <= 512) MOE_RP_VPL(16);
+  else MOE_RP_VPL(32);
+#undef MOE_RP_VPL
   return launch_status();
 }
 

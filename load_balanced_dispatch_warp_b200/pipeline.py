@@ -56,9 +56,7 @@ class HostPipeline:
                 self.inputs_ready[s].record(self.s_in)
             with torch.cuda.stream(self.s_comp):
                 self.s_comp.wait_event(self.inputs_ready[s])
-                L.route(self.logits[s])
-                L.measure()
-                L.balance()
+                L.route_plan(self.logits[s])
                 L.prefetch_dispatch(self.x[s], W1, W3, W2)
                 if not L.fused:
                     self.inputs_free[s].record(self.s_comp)

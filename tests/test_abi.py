@@ -139,3 +139,29 @@ def test_ffn_tile_mode_switch(lib):
     with pytest.raises(M.MoEError):
         M.set_ffn_tile_mode(2)
     assert lib.moe_ffn_tile_mode() == prev
+
+
+def test_route_plan_host_checks(lib):
+    """moe_route_plan answers bad arguments on the host, as its three separate calls do."""
+    P = ctypes.c_void_p
+    fake = P(4096)
+    # logits, bias, T, E, k, R, S, idx, gate, counts, loads, maxvio, bal, plan, ws, err, stream
+    args = [fake, None, 16, 8, 2, 4, 2, fake, fake, fake, fake, fake, fake, fake, fake, fake, None]
+    for i in (0, 7, 8, 9, 10, 11, 12, 13, 14, 15):  # null logits / outputs / workspace / err
+        bad = list(args); bad[i] = None
+        assert lib.moe_route_plan(*bad) == M.MOE_ERR_ARG, i
+    bad = list(args); bad[2] = 15  # T*k % R != 0
+    assert lib.moe_route_plan(*bad) == M.MOE_ERR_SHAPE
+    bad = list(args); bad[5] = 3  # E % R != 0
+    assert lib.moe_route_plan(*bad) == M.MOE_ERR_SHAPE
+    bad = list(args); bad[4] = 9  # k > E
+    assert lib.moe_route_plan(*bad) == M.MOE_ERR_SHAPE
+    bad = list(args); bad[3] = 2048; bad[5] = 8  # E > 1024
+    assert lib.moe_route_plan(*bad) == M.MOE_ERR_SHAPE
+    bad = list(args); bad[2] = 0; bad[0] = None; bad[7] = None; bad[8] = None  # T = 0: no rows
+    # (accepted on the host; a launch would follow, so only the null-output case is probed)
+    bad[9] = None
+    assert lib.moe_route_plan(*bad) == M.MOE_ERR_ARG
+    assert lib.moe_route_plan_workspace_words(64) == 16 * 64 + 1
+    assert lib.moe_route_plan_workspace_words(0) == -1
+    assert lib.moe_route_plan_workspace_words(1025) == -1
