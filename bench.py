@@ -362,10 +362,9 @@ def run_ours(args, w: I.Workload, world, rank, local):
                    "l2": "step working set (weights, pool, activations) far above the 126 MB L2",
                    "launch": "eager, one stream, calls in order" if args.eager else
                              "K forward steps (MoELayer.forward: routing/histogram/plan fused in "
-                             "one launch, replica prefetch on a forked stream overlapping the "
-                             "dispatch) captured in one CUDA graph, replayed once; per-call "
-                             "intervals from a second replay of the calls in order with event "
-                             "nodes between them"},
+                             "one launch, then prefetch, dispatch, FFN, combine) captured in one "
+                             "CUDA graph, replayed once; per-call intervals from a second replay "
+                             "with event nodes between the calls"},
         "clocks": clk,
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT,
                 "h2d_bytes_per_step": w.T * w.E * 4 + w.T * w.d * 2,

@@ -387,8 +387,6 @@ class MoELayer:
                     torch.empty(R * S, F, d, dtype=bf, device=dev),
                     torch.empty(R * S, d, F, dtype=torch.float16, device=dev))
         self.pool = pool if S > 0 else (None, None, None)
-        self._side = None  # side stream of prefetch_dispatch, created on first use
-        self._ev_plan = self._ev_pref = None
 
     def plan_field(self, name):
         L = self.layout
@@ -445,34 +443,13 @@ class MoELayer:
                        self.loads, self.maxvio, self.balancedness, self.plan, self.rp_workspace,
                        self.err, stream=stream)
 
-    def prefetch_dispatch(self, x, W1, W3, W2, stream=None):
-        """Replica prefetch and dispatch, both of which need only the plan.  The prefetch is
-        enqueued on a side stream forked from ``stream`` (after everything enqueued there so
-        far) and joined back before this returns, so its weight copies overlap the dispatch;
-        the two write disjoint buffers, so the results are those of prefetch then dispatch.
-        Works under CUDA-graph capture (the fork and join become graph edges)."""
-        main = torch.cuda.current_stream() if stream is None else stream
-        if self.S == 0:
-            self.prefetch(W1, W3, W2, main)
-            self.dispatch(x, main)
-            return
-        if self._side is None or self._side.device != main.device:
-            self._side = torch.cuda.Stream(device=main.device)
-            self._ev_plan = torch.cuda.Event()
-            self._ev_pref = torch.cuda.Event()
-        self._ev_plan.record(main)
-        self._side.wait_event(self._ev_plan)
-        self.prefetch(W1, W3, W2, self._side)
-        self._ev_pref.record(self._side)
-        self.dispatch(x, main)
-        main.wait_event(self._ev_pref)
-
     def forward(self, logits, x, W1, W3, W2, stream=None):
         """The whole path on the current stream: routing, histogram and plan fused
-        (``route_plan``), the prefetch forked off and joined back (``prefetch_dispatch``),
-        the grouped FFN, the combine; returns ``out`` [T,d] bf16 (device)."""
+        (``route_plan``), prefetch, dispatch, the grouped FFN, the combine; returns ``out``
+        [T,d] bf16 (device)."""
         self.route_plan(logits, stream)
-        self.prefetch_dispatch(x, W1, W3, W2, stream)
+        self.prefetch(W1, W3, W2, stream)
+        self.dispatch(x, stream)
         self.expert_ffn(W1, W3, W2, stream)
         self.combine(stream)
         return self.out

@@ -57,7 +57,8 @@ class HostPipeline:
             with torch.cuda.stream(self.s_comp):
                 self.s_comp.wait_event(self.inputs_ready[s])
                 L.route_plan(self.logits[s])
-                L.prefetch_dispatch(self.x[s], W1, W3, W2)
+                L.prefetch(W1, W3, W2)
+                L.dispatch(self.x[s])
                 if not L.fused:
                     self.inputs_free[s].record(self.s_comp)
                 L.expert_ffn(W1, W3, W2)

@@ -32,3 +32,39 @@ def test_pipeline_matches_forward():
     assert int(layer.err.item()) == 0
     for o, r in zip(outs, refs):
         assert torch.equal(o, r.cpu())
+
+
+def test_first_forward_inside_graph_capture():
+    """A layer whose very first forward is captured: replays equal an eager layer's output,
+    and the forward (fused routing call) equals the seven separate calls run in order."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    build.build()
+    w = I.small_workload("cap", 768, 64, 6, 8, 8, 256, 384, alpha=0.8, seed=31)
+    W = I.make_weights(w, device="cuda")
+    lg, x = I.make_logits(w).cuda(), I.make_x(w).cuda()
+    eager = M.MoELayer(w.T, w.E, w.k, w.R, w.S, w.d, w.F)
+    ref = eager.forward(lg, x, *W).clone()
+    seq = M.MoELayer(w.T, w.E, w.k, w.R, w.S, w.d, w.F)
+    seq.route(lg)
+    seq.measure()
+    seq.balance()
+    seq.prefetch(*W)
+    seq.dispatch(x)
+    seq.expert_ffn(*W)
+    seq.combine()
+    torch.cuda.synchronize()
+    assert torch.equal(seq.out, ref)
+    L = M.MoELayer(w.T, w.E, w.k, w.R, w.S, w.d, w.F)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        L.forward(lg, x, *W)
+    for _ in range(2):
+        L.out.zero_()
+        g.replay()
+    torch.cuda.synchronize()
+    assert int(L.err.item()) == 0
+    assert torch.equal(L.out, ref)
+    del g
