@@ -45,6 +45,8 @@
 // freed before the CTA exits.
 #include <cuda.h>
 
+#include <atomic>
+
 #include "common.cuh"
 
 namespace moe {
@@ -950,7 +952,7 @@ size_t ffn_pair_smem_bytes() {
          (MAX_GROUPS + 1) * 4 + 33 * 4;
 }
 
-int g_ffn_tile_mode = 0;        // 0: one CTA per 128-row tile, 1: CTA pairs
+std::atomic<int> g_ffn_tile_mode{0};  // 0: one CTA per 128-row tile, 1: CTA pairs
 int g_pair_clusters[64] = {0};  // co-resident 2-CTA clusters per device
 
 // Grid of the pair kernels: as many 2-CTA clusters as fit on the device at once (queried
@@ -1005,11 +1007,11 @@ int launch_bounded_wait_selftest(int32_t* err, int limit_us, cudaStream_t s) {
 
 int set_ffn_tile_mode(int mode) {
   if (mode != 0 && mode != 1) return MOE_ERR_ARG;
-  g_ffn_tile_mode = mode;
+  g_ffn_tile_mode.store(mode, std::memory_order_relaxed);
   return MOE_OK;
 }
 
-int ffn_tile_mode() { return g_ffn_tile_mode; }
+int ffn_tile_mode() { return g_ffn_tile_mode.load(std::memory_order_relaxed); }
 
 int ffn_pair_clusters() {
   int dev = 0;
@@ -1026,7 +1028,7 @@ int launch_grouped_ffn_impl(const __nv_bfloat16* recv, const __nv_bfloat16* x,
                             __nv_bfloat16* y, int32_t* err, cudaStream_t s) {
   if (T == 0) return MOE_OK;
   const bool gather = x != nullptr;
-  const bool pair = !gather && g_ffn_tile_mode == 1;
+  const bool pair = !gather && g_ffn_tile_mode.load(std::memory_order_relaxed) == 1;
   const int64_t rows = (int64_t)T * k;  // R * C
   const int bn2 = (d % 256 == 0) ? 256 : 128;
   const int w2_box = pair ? bn2 / 2 : bn2;  // a pair CTA loads half of GEMM 2's B rows
