@@ -96,6 +96,14 @@ class ClockSampler:
         time.sleep(0.25)
         self.proc.terminate()
         out, _ = self.proc.communicate(timeout=10)
+        return self.summarize(out)
+
+    @staticmethod
+    def summarize(out: str) -> dict:
+        """Clock record from `nvidia-smi --query-gpu=QUERY --format=csv,noheader,nounits`
+        lines: the median SM clock over the samples under load (above half the max clock;
+        all samples if none is), the max clock, and every throttle reason active in one of
+        those samples.  Malformed lines are skipped."""
         rows = []
         for line in out.strip().splitlines():
             parts = [p.strip() for p in line.split(",")]
