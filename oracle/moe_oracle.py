@@ -43,6 +43,13 @@ Pins (tests/test_oracle_pins.py checks each against something other than this fi
                     away from top-k ties); torch.autograd (fp64, CPU) through a token-major
                     formulation with no plan, dispatch or replicas; the weight gradients do
                     not depend on S (replicas reduced back home)
+  dispatch_backward, combine_backward
+                    the adjoint (dot-product) identity <A v, w> = <v, A^T w> against
+                    dispatch() and combine() on random inputs, for the rows and the gates
+  topk_backward     central differences of topk_route's gates along fp32-exact directions
+  expert_ffn_backward  central differences of expert_ffn() for X, w1, w3, w2
+  (tests/test_oracle_mutants.py plants one plausible mistake in each of the last four and
+  checks that its pin fails)
 
 Error bits (OR-ed): 1 non-finite logit, 2 expert id out of range, 4 repeated expert
 within one token, 8 plan needs more than S replicas on some rank.

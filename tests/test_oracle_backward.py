@@ -127,3 +127,93 @@ def test_gate_backward_closed_form_k2():
     dl = O.topk_backward(gate, dgate, np.array([[2, 0]]), 3)
     v = 0.3 * 0.7 * (1.5 - (-0.5))
     assert np.allclose(dl, [[-v, 0.0, v]])
+
+
+# ----------------------------------------------------------------- per-piece adjoint pins
+# Each linear piece of the layer is pinned by the dot-product (adjoint) identity
+# <A v, w> = <v, A^T w> with random v and w, which holds for the true transpose and fails
+# for a dropped term, a wrong index or a transposed operand in either the forward or the
+# backward; the nonlinear gate softmax is pinned by central differences.
+
+def random_placement(rng, T, k, rows):
+    """A bijection of the T*k assignments onto `rows` rows (perm) and its inverse (src)."""
+    order = rng.permutation(rows)[: T * k]
+    perm = order.reshape(T, k)
+    src = np.full(rows, -1)
+    for t in range(T):
+        for j in range(k):
+            src[perm[t, j]] = t
+    return perm, src
+
+
+def test_dispatch_backward_is_the_adjoint_of_dispatch():
+    rng = np.random.default_rng(11)
+    T, k, d = 9, 3, 5
+    perm, src = random_placement(rng, T, k, T * k)
+    x = rng.standard_normal((T, d))
+    g = rng.standard_normal((T * k, d))
+    lhs = float((O.dispatch(x, src) * g).sum())
+    rhs = float((x * O.dispatch_backward(g, perm)).sum())
+    assert abs(lhs - rhs) <= 1e-12 * max(1.0, abs(lhs))
+
+
+def test_combine_backward_is_the_adjoint_in_rows_and_in_gates():
+    rng = np.random.default_rng(12)
+    T, k, d = 7, 4, 6
+    perm, _ = random_placement(rng, T, k, T * k)
+    y = rng.standard_normal((T * k, d))
+    gate = rng.random((T, k))
+    dout = rng.standard_normal((T, d))
+    dy, dgate = O.combine_backward(dout, y, perm, gate)
+    out = O.combine(y, perm, gate)
+    # combine is linear in y for fixed gates, and linear in the gates for fixed y
+    ip = float((out * dout).sum())
+    assert abs(ip - float((y * dy).sum())) <= 1e-12 * max(1.0, abs(ip))
+    assert abs(ip - float((gate * dgate).sum())) <= 1e-12 * max(1.0, abs(ip))
+
+
+def test_topk_backward_matches_central_differences_of_the_gates():
+    """Gates as a function of the chosen logits (selection held fixed by well-separated
+    logits): <d gate, dgate> / eps against <v, dlogits> for random directions v.  The router
+    computes on fp32 logits, so the logits sit on a 2^-8 grid below 8 in magnitude and move
+    by 2^-16 along directions in {-1, 0, 1}: every perturbed logit is exact in fp32."""
+    rng = np.random.default_rng(13)
+    T, E, k = 5, 10, 3
+    logits = rng.permuted(np.tile(np.arange(E, dtype=np.float64) * 0.7 - 3.0, (T, 1)), axis=1)
+    logits = np.round(logits * 256) / 256
+    idx, gate, err = O.topk_route(logits, k)
+    assert err == 0
+    dgate = rng.standard_normal((T, k))
+    dl = O.topk_backward(gate, dgate, idx, E)
+    eps = 2.0 ** -16
+    for _ in range(4):
+        v = rng.integers(-1, 2, size=(T, E)).astype(np.float64)
+        assert np.array_equal((logits + eps * v).astype(np.float32), logits + eps * v)
+        gp = O.topk_route(logits + eps * v, k)
+        gm = O.topk_route(logits - eps * v, k)
+        assert np.array_equal(gp[0], idx) and np.array_equal(gm[0], idx)
+        num = float(((gp[1] - gm[1]) * dgate).sum()) / (2 * eps)
+        assert abs(num - float((v * dl).sum())) <= 1e-7 * max(1.0, abs(num))
+
+
+def test_expert_ffn_backward_matches_central_differences():
+    rng = np.random.default_rng(14)
+    n, d, F = 6, 5, 4
+    X = rng.standard_normal((n, d))
+    w1 = rng.standard_normal((F, d)) / np.sqrt(d)
+    w3 = rng.standard_normal((F, d)) / np.sqrt(d)
+    w2 = rng.standard_normal((d, F)) / np.sqrt(F)
+    dy = rng.standard_normal((n, d))
+    b = O.expert_ffn_backward(X, w1, w3, w2, dy)
+    args = dict(X=X, w1=w1, w3=w3, w2=w2)
+    grads = dict(X=b["dX"], w1=b["dw1"], w3=b["dw3"], w2=b["dw2"])
+
+    def f(**kw):
+        a = dict(args, **kw)
+        return float((O.expert_ffn(a["X"], a["w1"], a["w3"], a["w2"]) * dy).sum())
+
+    eps = 1e-6
+    for name, grad in grads.items():
+        v = rng.standard_normal(args[name].shape)
+        num = (f(**{name: args[name] + eps * v}) - f(**{name: args[name] - eps * v})) / (2 * eps)
+        assert abs(num - float((v * grad).sum())) <= 1e-7 * max(1.0, abs(num)), name
