@@ -48,8 +48,9 @@ Pins (tests/test_oracle_pins.py checks each against something other than this fi
                     dispatch() and combine() on random inputs, for the rows and the gates
   topk_backward     central differences of topk_route's gates along fp32-exact directions
   expert_ffn_backward  central differences of expert_ffn() for X, w1, w3, w2
-  (tests/test_oracle_mutants.py plants one plausible mistake in each of the last four and
-  checks that its pin fails)
+  (tests/test_oracle_mutants.py plants one plausible mistake at a time in topk_route,
+  expert_histogram, plan_balanced, permute, dispatch, prefetch, expert_ffn, combine and
+  the four backward pieces, and checks that the pin for it fails)
 
 Error bits (OR-ed): 1 non-finite logit, 2 expert id out of range, 4 repeated expert
 within one token, 8 plan needs more than S replicas on some rank.

@@ -1,12 +1,17 @@
-"""The oracle's backward pins fail on plausible mistakes (CPU only).
+"""The oracle's pins fail on plausible mistakes (CPU only).
 
-Each case swaps one oracle function for a copy with one planted mistake (a dropped term, a
-missing factor, a skipped index, a wrong derivative) and checks that the pin written for
-that function fails.  The mistakes live here, in the test, never in the oracle."""
+Each case swaps one oracle function for a copy with one planted mistake (ties broken the
+wrong way, a softmax over the wrong set, a dropped choice, a reordered plan or placement, a
+shifted row, a copied operand, swapped projections, missing gates, a dropped term, a wrong
+derivative) and checks that the pin written for that function fails.  The mistakes live
+here, in the test, never in the oracle."""
+import json
+
 import numpy as np
 import pytest
 
 import test_oracle_backward as P
+import test_oracle_pins as F
 from oracle import moe_oracle as O
 
 ORIG = {n: getattr(O, n) for n in ("topk_backward", "combine_backward", "dispatch_backward",
@@ -67,6 +72,94 @@ CASES = [
 @pytest.mark.parametrize("name,mutant,pin", CASES, ids=[c[0] for c in CASES])
 def test_pin_catches_planted_mistake(monkeypatch, name, mutant, pin):
     pin()  # passes on the oracle as it is
+    monkeypatch.setattr(O, name, mutant)
+    with pytest.raises(AssertionError):
+        pin()
+
+
+# ------------------------------------------------------------------ forward pieces
+FWD = {n: getattr(O, n) for n in ("topk_route", "expert_histogram", "plan_balanced", "permute",
+                                  "dispatch", "prefetch", "expert_ffn", "combine")}
+
+
+def fixture():
+    with open(F.GOLD) as f:
+        g = json.load(f)
+    idx = np.array([[int(p[0]), int(p[1])] for p in g["pairs"]], dtype=np.int32)
+    return g, idx, np.arange(g["tokens"]) % g["ranks"]
+
+
+def topk_ties_to_higher_id(logits, k):
+    logits = np.asarray(logits, dtype=np.float32)
+    idx, gate, err = FWD["topk_route"](logits[:, ::-1], k)
+    return (logits.shape[1] - 1 - idx).astype(np.int32), gate, err
+
+
+def topk_softmax_over_all_experts(logits, k):
+    idx, gate, err = FWD["topk_route"](logits, k)
+    row = np.asarray(logits, dtype=np.float64)
+    ex = np.exp(row - row.max(axis=1, keepdims=True))
+    full = ex / ex.sum(axis=1, keepdims=True)
+    return idx, np.take_along_axis(full, idx.astype(np.int64), axis=1), err
+
+
+def histogram_of_first_choice(idx, E, R, expert_to_rank=None):
+    idx = np.asarray(idx)
+    return FWD["expert_histogram"](idx[:, :1], E, R, expert_to_rank)
+
+
+def plan_groups_reversed(counts, T, k, E, R, S):
+    p = FWD["plan_balanced"](counts, T, k, E, R, S)
+    p["groups"] = [list(reversed(g)) for g in p["groups"]]
+    return p
+
+
+def permute_unstable(idx, plan, E, R):
+    perm, src = FWD["permute"](idx, plan, E, R)
+    perm, src = np.array(perm), np.array(src)
+    e = int(np.asarray(idx)[0, 0])  # the rows of one expert, in reverse token order
+    where = [(t, j) for t in range(len(idx)) for j in range(len(idx[0])) if idx[t][j] == e]
+    rows = [perm[t, j] for t, j in where][::-1]
+    for (t, j), r in zip(where, rows):
+        perm[t, j] = r
+        src[r] = t
+    return perm, src
+
+
+def dispatch_shifted(x, src):
+    return np.asarray(x)[np.roll(np.asarray(src), 1)]
+
+
+def prefetch_w1_twice(plan, W1, W3, W2, R, S):
+    return {s: (a, a, c) for s, (a, b, c) in FWD["prefetch"](plan, W1, W3, W2, R, S).items()}
+
+
+def ffn_gate_and_up_swapped(X, w1, w3, w2):
+    return FWD["expert_ffn"](X, w3, w1, w2)
+
+
+def combine_without_gates(y, perm, gate, tokens=None):
+    return FWD["combine"](y, perm, np.ones_like(np.asarray(gate, dtype=np.float64)), tokens)
+
+
+FWD_CASES = [
+    ("topk_route", topk_ties_to_higher_id, F.test_topk_bruteforce_with_ties),
+    ("topk_route", topk_softmax_over_all_experts, F.test_topk_special_cases),
+    ("expert_histogram", histogram_of_first_choice,
+     lambda: F.test_fixture_demand_and_balancedness(fixture())),
+    ("plan_balanced", plan_groups_reversed, lambda: F.test_fixture_plan_derived_by_hand(fixture())),
+    ("permute", permute_unstable, lambda: F.test_fixture_plan_derived_by_hand(fixture())),
+    ("dispatch", dispatch_shifted, F.test_dispatch_prefetch_identities),
+    ("prefetch", prefetch_w1_twice, F.test_dispatch_prefetch_identities),
+    ("expert_ffn", ffn_gate_and_up_swapped, F.test_ffn_closed_forms),
+    ("combine", combine_without_gates, F.test_combine_identity_and_scaled_experts),
+]
+
+
+@pytest.mark.parametrize("name,mutant,pin", FWD_CASES,
+                         ids=[f"{c[0]}-{c[1].__name__}" for c in FWD_CASES])
+def test_forward_pin_catches_planted_mistake(monkeypatch, name, mutant, pin):
+    pin()
     monkeypatch.setattr(O, name, mutant)
     with pytest.raises(AssertionError):
         pin()
