@@ -25,7 +25,8 @@ Pins (tests/test_oracle_pins.py checks each against something other than this fi
   topk_route        brute-force rank counting on tiny inputs; k=1 / k=E special cases;
                     softmax closed forms (k=2 sigmoid, equal logits -> 1/k)
   topk_route_biased zero bias reduces to topk_route; a large bias forces a chosen set;
-                    the gates ignore the bias (closed form for k=2)
+                    the gates ignore the bias, equal or unequal on the chosen pair
+                    (closed form for k=2)
   expert_histogram  the pages' worked fixture (demand, both rank mappings, 4/9, 8/15, 0.8)
   capacity_ledger   the pages' worked fixture (cap 5, processed/overflow/padding)
   remote_routes     the pages' worked fixture (22 vs 25 of 32)
@@ -49,8 +50,9 @@ Pins (tests/test_oracle_pins.py checks each against something other than this fi
   topk_backward     central differences of topk_route's gates along fp32-exact directions
   expert_ffn_backward  central differences of expert_ffn() for X, w1, w3, w2
   (tests/test_oracle_mutants.py plants one plausible mistake at a time in topk_route,
-  expert_histogram, plan_balanced, permute, dispatch, prefetch, expert_ffn, combine and
-  the four backward pieces, and checks that the pin for it fails)
+  topk_route_biased, validate_trace, expert_histogram, capacity_ledger, remote_routes,
+  plan_balanced, permute, dispatch, prefetch, expert_ffn, combine and the four backward
+  pieces, and checks that the pin for it fails)
 
 Error bits (OR-ed): 1 non-finite logit, 2 expert id out of range, 4 repeated expert
 within one token, 8 plan needs more than S replicas on some rank.

@@ -163,3 +163,47 @@ def test_forward_pin_catches_planted_mistake(monkeypatch, name, mutant, pin):
     monkeypatch.setattr(O, name, mutant)
     with pytest.raises(AssertionError):
         pin()
+
+
+# ------------------------------------------------------------------ ledgers and variants
+VAR = {n: getattr(O, n) for n in ("validate_trace", "capacity_ledger", "remote_routes",
+                                  "topk_route_biased")}
+
+
+def validate_without_repeat_check(idx, E):
+    return VAR["validate_trace"](idx, E) & ~O.ERR_DUPLICATE
+
+
+def ledger_overflow_unclamped(counts, A, E, cf_num=5, cf_den=4):
+    led = VAR["capacity_ledger"](counts, A, E, cf_num, cf_den)
+    led["overflow"] = np.asarray(counts, dtype=np.int64) - led["cap"]
+    return led
+
+
+def remote_counts_local_routes(idx, origin, expert_to_rank):
+    return np.asarray(idx).size - VAR["remote_routes"](idx, origin, expert_to_rank)
+
+
+def biased_gate_from_biased_scores(logits, bias, k):
+    idx, _, err = VAR["topk_route_biased"](logits, bias, k)
+    sc = np.asarray(logits, dtype=np.float64) + np.asarray(bias, dtype=np.float64)
+    sel = np.take_along_axis(sc, idx.astype(np.int64), axis=1)
+    ex = np.exp(sel - sel.max(axis=1, keepdims=True))
+    return idx, ex / ex.sum(axis=1, keepdims=True), err
+
+
+VAR_CASES = [
+    ("validate_trace", validate_without_repeat_check,
+     lambda: F.test_fixture_validation_rules(fixture())),
+    ("capacity_ledger", ledger_overflow_unclamped, lambda: F.test_fixture_capacity_ledger(fixture())),
+    ("remote_routes", remote_counts_local_routes, lambda: F.test_fixture_remote_routes(fixture())),
+    ("topk_route_biased", biased_gate_from_biased_scores, F.test_biased_topk_pins),
+]
+
+
+@pytest.mark.parametrize("name,mutant,pin", VAR_CASES, ids=[c[0] for c in VAR_CASES])
+def test_ledger_and_variant_pins_catch_planted_mistakes(monkeypatch, name, mutant, pin):
+    pin()
+    monkeypatch.setattr(O, name, mutant)
+    with pytest.raises(AssertionError):
+        pin()

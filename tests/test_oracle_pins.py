@@ -397,6 +397,16 @@ def test_biased_topk_pins():
     for t in range(40):
         first = 7 if np.float32(logits[t, 7] + np.float32(100)) > np.float32(logits[t, 2] + np.float32(100)) else 2
         assert idx[t, 0] == first or logits[t, 7] + 100 == logits[t, 2] + 100
+    # unequal biases on the chosen pair: a gate computed from the biased scores would be
+    # shifted by the bias difference; the gate must stay the softmax of the raw logits
+    bias2 = np.zeros(12, np.float32)
+    bias2[2], bias2[7] = 100.0, 101.5
+    idx, gate, err = O.topk_route_biased(logits, bias2, 2)
+    assert err == 0
+    for t in range(40):
+        assert sorted(idx[t]) == [2, 7]
+        a, b = float(logits[t, idx[t, 0]]), float(logits[t, idx[t, 1]])
+        assert abs(gate[t, 0] - 1.0 / (1.0 + math.exp(b - a))) < 1e-15
     bad = bias.copy()
     bad[3] = np.nan
     assert O.topk_route_biased(logits, bad, 2)[2] == O.ERR_NONFINITE
