@@ -69,3 +69,27 @@ def test_work_units_of_the_default_workload():
     assert u["moe_grouped_ffn"] == ("TFLOP/s", 3 * 2 * A * d * F)
     # fused dispatch: no row copy; the FFN reads the token rows itself
     assert bench.algorithmic(w, n_rep, fused=True)["moe_dispatch"] == ("GB/s", 12 * A)
+
+
+def test_reference_arm_line_keeps_the_contract(monkeypatch):
+    """`bench.py --impl reference` on the tiny workload (the oracle on this host's cores):
+    the JSON line carries the keys the contract names, with this arm's metric and unit."""
+    import argparse
+    import json
+    for var in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        monkeypatch.delenv(var, raising=False)
+    args = argparse.Namespace(steps=2, warmup=1)
+    line = bench.run_reference(args, I.WORKLOADS["tiny"])
+    json.dumps(line)  # serialisable as printed
+    assert line["impl"] == "reference"
+    assert line["metric"] == bench.METRIC and line["unit"] == bench.UNIT
+    assert line["value"] > 0 and line["higher_is_better"] is True
+    assert line["n_gpus"] == 1 and line["steps"] >= 1 and line["warmup"] == 1
+    assert line["config"]["workload"] == "tiny"
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"]
+    assert cb["unit"] == bench.UNIT and isinstance(cb["sample"], str)
+    e2e = line["e2e"]
+    assert e2e["value"] == line["value"] and e2e["unit"] == bench.UNIT
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+    assert line["vs_baseline"] is None
