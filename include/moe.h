@@ -129,12 +129,19 @@ int moe_topk_biased(const float* logits, const float* bias, int T, int E, int k,
  * ids must be known experts and a token may not repeat one.
  *   idx            [T,k] int32        expert choices (e.g. from moe_topk).
  *   expert_to_rank [E] int32 or NULL  owning rank of each expert; NULL = e / (E/R).
+ *                                     "If any expert is missing from a mapping, stop": an
+ *                                     entry outside [0, R) sets MOE_DERR_ID_RANGE and that
+ *                                     expert's demand is added to no rank.
  *   counts         [E] int32  (out)   assignments per expert (in-range ids only).
  *   loads          [R] int32  (out)   assignments per rank under the mapping.
  *   maxvio         [1] fp64   (out)   (R*max(loads) - T*k) / (T*k), one rounding;
  *                                     0 when T == 0.
  *   balancedness   [1] fp64   (out)   (T*k) / (R*max(loads)); 1 when T == 0.
- *   err            int32      (in/out) bits MOE_DERR_ID_RANGE, MOE_DERR_DUPLICATE.
+ *   err            int32      (in/out) bits MOE_DERR_ID_RANGE, MOE_DERR_DUPLICATE; a
+ *                                     no-op when already non-zero.  Every bit the trace
+ *                                     deserves is set, counts/loads/maxvio/balancedness
+ *                                     are still written, and none of them depends on the
+ *                                     order in which the GPU runs its blocks.
  */
 int moe_histogram_maxvio(const int32_t* idx, int T, int k, int E, int R,
                          const int32_t* expert_to_rank, int32_t* counts, int32_t* loads,
@@ -354,9 +361,10 @@ int moe_topk_backward(const float* gate, const float* dgate, const int32_t* idx,
  * that every GPU loading the library holds until the process exits.
  *   - Returns MOE_ERR_SHAPE when moe_dispatch_workspace_words(T, E) exceeds
  *     MOE_NOALLOC_SCRATCH_WORDS (e.g. T = 65536 with E = 1024 fits, T = 131072 does not).
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current); make that first call before any
- *     stream capture.  MOE_ERR_DEVICE if the lookup fails.
+ *   - The first call in each CUDA context of a device looks up the array's device
+ *     address (cudaGetSymbolAddress, with that device current) and keeps it for that
+ *     context; after a cudaDeviceReset the next call looks it up again.  Make the first
+ *     call on a device before any stream capture.  MOE_ERR_DEVICE if the lookup fails.
  *   - All calls share the array and it keeps the last call's contents; no word of it has
  *     to start at zero.  Calls that overlap on the GPU (several streams or host threads
  *     on one device) race on it: serialise them.
@@ -372,6 +380,9 @@ int moe_dispatch_noalloc(const moe_bf16* x, const int32_t* idx, const int32_t* p
  *   out[t] = sum_{j=0..k-1} gate[t,j] * y[perm[t,j]]   (fp32, j order; bf16 out)
  *   y [R*C,d] bf16, perm [T,k] int32, gate [T,k] fp32, out [T,d] bf16 (out).
  *   err  no-op when non-zero.
+ *   perm must be the output of a moe_dispatch (or moe_dispatch_index) that left *err at
+ *   0: its rows are not range-checked again here (the call has no R*C argument), and a
+ *   perm from elsewhere must hold rows in [0, rows of y).
  */
 int moe_combine(const moe_bf16* y, const int32_t* perm, const float* gate, int T, int k,
                 int d, moe_bf16* out, const int32_t* err, moe_stream_t stream);

@@ -1,5 +1,6 @@
 // The C ABI (include/moe.h): argument checks, then one launcher per step.
 // Every check runs on the host before anything is enqueued.
+#include "checks.cuh"
 #include "common.cuh"
 
 namespace moe {
@@ -24,38 +25,12 @@ int num_sms() {
 
 namespace {
 
-constexpr int64_t kMaxElems = (int64_t)1 << 31;
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-int check_route(int T, int E, int k) {
-  if (T < 0 || E < 1 || k < 1) return MOE_ERR_ARG;
-  if (E > 1024 || k > E || k > 32) return MOE_ERR_SHAPE;
-  if ((int64_t)T * E >= kMaxElems || (int64_t)T * k >= kMaxElems) return MOE_ERR_SHAPE;
-  return MOE_OK;
-}
-
-int check_ranks(int T, int k, int E, int R, bool need_even_rows) {
-  if (R < 1) return MOE_ERR_ARG;
-  if (R > E || E % R != 0) return MOE_ERR_SHAPE;
-  if (need_even_rows && ((int64_t)T * k) % R != 0) return MOE_ERR_SHAPE;
-  return MOE_OK;
-}
-
-int check_dims(int T, int k, int d, int F) {
-  if (d < 1 || F < 1) return MOE_ERR_ARG;
-  if (d % 128 != 0 || F % 128 != 0) return MOE_ERR_SHAPE;
-  const int64_t rows = (int64_t)T * k;
-  if (rows * d >= kMaxElems || rows * F >= kMaxElems || (int64_t)T * d >= kMaxElems)
-    return MOE_ERR_SHAPE;
-  return MOE_OK;
-}
-
-int check_groups(int E, int R, int S) {
-  if (S < 0) return MOE_ERR_ARG;
-  if ((int64_t)R * (E / R + S) > 4096) return MOE_ERR_SHAPE;
-  return MOE_OK;
-}
+using moe::checks::aligned16;
+using moe::checks::kMaxElems;
+constexpr auto check_route = moe::checks::route;
+constexpr auto check_ranks = moe::checks::ranks;
+constexpr auto check_dims = moe::checks::dims;
+constexpr auto check_groups = moe::checks::groups;
 
 cudaStream_t as_stream(moe_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
@@ -202,13 +177,8 @@ int moe_prefetch_replicas(const int32_t* plan, const moe_bf16* W1, const moe_bf1
 int moe_dispatch(const moe_bf16* x, const int32_t* idx, const int32_t* plan, int T, int k,
                  int E, int R, int S, int d, int32_t* workspace, moe_bf16* recv,
                  int32_t* perm, int32_t* src, int32_t* err, moe_stream_t stream) {
-  if (!plan || !err) return MOE_ERR_ARG;
-  if (T > 0 && (!x || !idx || !workspace || !recv || !perm || !src)) return MOE_ERR_ARG;
-  MOE_TRY(check_route(T, E, k));
-  MOE_TRY(check_ranks(T, k, E, R, true));
-  MOE_TRY(check_groups(E, R, S));
-  MOE_TRY(check_dims(T, k, d, 128));
-  if (!aligned16(x) || !aligned16(recv)) return MOE_ERR_ARG;
+  MOE_TRY(moe::checks::dispatch(x, idx, plan, T, k, E, R, S, d, recv, perm, src, err));
+  if (T > 0 && !workspace) return MOE_ERR_ARG;
   moe_plan_layout L;
   MOE_TRY(moe_plan_get_layout(E, R, S, &L));
   return moe::launch_dispatch(reinterpret_cast<const __nv_bfloat16*>(x), idx, plan, L, T, k, E,

@@ -390,10 +390,19 @@ __device__ __noinline__ void hist_finish(const int32_t* __restrict__ counts, int
 // hotspot fixture (known ids, no expert repeated within a token).  Equal ids in a warp
 // are merged with match.any before one shared-memory add; block totals go to global
 // memory with integer atomics (order-independent, so deterministic).  The last block to
-// finish (a ticket counter kept in loads[0], zeroed with counts before the launch and
-// overwritten by the result) computes the rank loads under the expert->rank map and
-// maxvio = (R*max - A)/A, balancedness = A/(R*max) from exact integers, one fp64 rounding
-// each.
+// finish computes the rank loads under the expert->rank map and maxvio = (R*max - A)/A,
+// balancedness = A/(R*max) from exact integers, one fp64 rounding each.
+//
+// The ticket word is loads[0] (zeroed before the launch, overwritten by the result): its
+// low 24 bits count finished blocks (at most 2 per SM) and bits 24.. carry the trace
+// errors the blocks found (kErrShift).  No block writes *err before the last one
+// publishes those bits, so every block's entry check reads the word as it was before the
+// launch and the whole grid takes the same decision; every block counts all of its
+// in-range ids whatever the others found, so counts and error bits do not depend on
+// block scheduling.
+constexpr int kErrShift = 24;
+constexpr int kTicketMask = (1 << kErrShift) - 1;
+
 __global__ void __launch_bounds__(512) hist_kernel(const int32_t* __restrict__ idx, int T, int k,
                                                    int E, int R, int tokens_per_block,
                                                    const int32_t* __restrict__ map,
@@ -434,14 +443,19 @@ __global__ void __launch_bounds__(512) hist_kernel(const int32_t* __restrict__ i
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x)
     if (s_hist[e]) atomicAdd(counts + e, s_hist[e]);
-  if (threadIdx.x == 0 && s_err) atomicOr(err, s_err);
-  // last block: every other block's counts are visible once its ticket is
+  // last block: every other block's counts and error bits are visible once its ticket is
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) s_last = atomicAdd(loads, 1) == (int)gridDim.x - 1;
+  if (threadIdx.x == 0) {
+    if (s_err) atomicOr(loads, s_err << kErrShift);
+    const int old = atomicAdd(loads, 1);
+    s_last = (old & kTicketMask) == (int)gridDim.x - 1;
+    if (s_last) s_err = (old >> kErrShift) | s_err;
+  }
   __syncthreads();
   if (!s_last) return;
   __threadfence();
+  if (threadIdx.x == 0 && s_err) atomicOr(err, s_err);
   hist_finish(counts, T, k, E, R, map, loads, maxvio, bal, err, s_hist, s_max);
 }
 

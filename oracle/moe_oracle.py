@@ -171,6 +171,11 @@ def expert_histogram(idx: np.ndarray, E: int, R: int, expert_to_rank=None):
     Expert-level maxvio uses E buckets instead of R.  Only in-range ids are counted;
     bad ids set the validation error bits.  A = 0 gives maxvio 0 and balancedness 1.
 
+    The mapping is validated too ("Work the 16-token hotspot fixture": if an expert is
+    missing from a mapping, stop): an entry outside [0, R) -- no owning rank -- sets
+    error bit 2, and that expert's demand is added to no rank (never Python's negative
+    indexing, which would hand -1 to rank R-1).
+
     Returns dict(counts[E], loads[R], maxvio, balancedness, expert_maxvio,
     expert_balancedness, err).
     """
@@ -188,7 +193,11 @@ def expert_histogram(idx: np.ndarray, E: int, R: int, expert_to_rank=None):
         expert_to_rank = home_rank_map(E, R)
     loads = np.zeros(R, dtype=np.int64)
     for e in range(E):
-        loads[int(expert_to_rank[e])] += counts[e]
+        r = int(expert_to_rank[e])
+        if 0 <= r < R:
+            loads[r] += counts[e]
+        else:
+            err |= ERR_ID_RANGE
     mx = int(loads.max()) if R > 0 else 0
     emx = int(counts.max()) if E > 0 else 0
     if A == 0 or mx == 0:

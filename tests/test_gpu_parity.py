@@ -125,6 +125,59 @@ def test_trace_validation_errors():
     assert _hist(dup, 8, 4) == M.DERR_DUPLICATE
 
 
+def _hist_full(idx, E, R, expert_to_rank=None):
+    counts = torch.full((E,), -7, dtype=torch.int32, device="cuda")
+    loads = torch.full((R,), -7, dtype=torch.int32, device="cuda")
+    mv = torch.full((1,), -7.0, dtype=torch.float64, device="cuda")
+    b = torch.full((1,), -7.0, dtype=torch.float64, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    M.moe_histogram_maxvio(idx, E, R, counts, loads, mv, b, err, expert_to_rank=expert_to_rank)
+    torch.cuda.synchronize()
+    return dict(err=int(err.item()), counts=counts.cpu().numpy(), loads=loads.cpu().numpy(),
+                maxvio=float(mv.item()), balancedness=float(b.item()))
+
+
+def _same_as_oracle(got, ref):
+    assert got["err"] == ref["err"]
+    assert np.array_equal(got["counts"], ref["counts"])
+    assert np.array_equal(got["loads"], ref["loads"])
+    assert got["maxvio"] == ref["maxvio"] and got["balancedness"] == ref["balancedness"]
+
+
+def test_histogram_mapping_missing_an_expert():
+    """"If any expert is missing from a mapping, stop": a map entry outside [0, R) sets
+    MOE_DERR_ID_RANGE, and the GPU's counts, loads, maxvio and balancedness equal the
+    oracle's (the unmapped expert's demand goes to no rank)."""
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "hotspot_fixture.json")))
+    idx_h = np.array([[int(p[0]), int(p[1])] for p in g["pairs"]], dtype=np.int32)
+    idx = torch.from_numpy(idx_h).cuda()
+    base = np.zeros(8, dtype=np.int32)
+    for r, es in enumerate(g["initial_mapping"]):
+        base[es] = r
+    for e, r in ((7, -1), (0, 4), (3, -4), (5, 1 << 20)):
+        m = base.copy()
+        m[e] = r
+        ref = O.expert_histogram(idx_h, 8, 4, m)
+        assert ref["err"] == O.ERR_ID_RANGE
+        _same_as_oracle(_hist_full(idx, 8, 4, torch.from_numpy(m).cuda()), ref)
+
+
+def test_histogram_errors_found_in_different_blocks():
+    """A trace spread over every block of the histogram grid, with an unknown id in the
+    first token and a repeated expert in the last: both error bits, and the counts of all
+    in-range ids, whatever order the blocks run in (five calls, identical results)."""
+    T, k, E, R = 65536, 8, 256, 32
+    rng = np.random.default_rng(21)
+    idx_h = np.argsort(rng.random((T, E)), axis=1)[:, :k].astype(np.int32)
+    idx_h[0, 3] = E + 5
+    idx_h[T - 1, 6] = idx_h[T - 1, 2]
+    ref = O.expert_histogram(idx_h, E, R)
+    assert ref["err"] == O.ERR_ID_RANGE | O.ERR_DUPLICATE
+    idx = torch.from_numpy(idx_h).cuda()
+    for _ in range(5):
+        _same_as_oracle(_hist_full(idx, E, R), ref)
+
+
 def test_nonfinite_logit_stops_the_layer():
     w = I.small_workload("nan", 64, 8, 2, 4, 2, 128, 128, alpha=1.0, seed=9)
     logits, x, weights = make_inputs(w)

@@ -108,6 +108,19 @@ def histogram_of_first_choice(idx, E, R, expert_to_rank=None):
     return FWD["expert_histogram"](idx[:, :1], E, R, expert_to_rank)
 
 
+def histogram_without_mapping_check(idx, E, R, expert_to_rank=None):
+    """The rank sum with Python indexing and no range check: -1 wraps to rank R-1, R is
+    clipped to rank R-1, and no error bit is set."""
+    h = FWD["expert_histogram"](idx, E, R)
+    m = O.home_rank_map(E, R) if expert_to_rank is None else np.asarray(expert_to_rank)
+    loads = np.zeros(R, dtype=np.int64)
+    for e in range(E):
+        loads[min(int(m[e]), R - 1)] += h["counts"][e]
+    h["loads"] = loads
+    h["err"] = O.validate_trace(idx, E)
+    return h
+
+
 def plan_groups_reversed(counts, T, k, E, R, S):
     p = FWD["plan_balanced"](counts, T, k, E, R, S)
     p["groups"] = [list(reversed(g)) for g in p["groups"]]
@@ -147,6 +160,8 @@ FWD_CASES = [
     ("topk_route", topk_softmax_over_all_experts, F.test_topk_special_cases),
     ("expert_histogram", histogram_of_first_choice,
      lambda: F.test_fixture_demand_and_balancedness(fixture())),
+    ("expert_histogram", histogram_without_mapping_check,
+     lambda: F.test_fixture_mapping_must_cover_every_expert(fixture())),
     ("plan_balanced", plan_groups_reversed, lambda: F.test_fixture_plan_derived_by_hand(fixture())),
     ("permute", permute_unstable, lambda: F.test_fixture_plan_derived_by_hand(fixture())),
     ("dispatch", dispatch_shifted, F.test_dispatch_prefetch_identities),

@@ -99,6 +99,26 @@ def test_fixture_validation_rules(fx):
     assert O.expert_histogram(bad, 8, 4)["err"] & O.ERR_ID_RANGE
 
 
+def test_fixture_mapping_must_cover_every_expert(fx):
+    """"If any expert is missing from a mapping, stop": a rank outside [0, R) leaves an
+    expert with no owner.  The fixture's initial mapping {0,1},{2,3},{4,5},{6,7} gives
+    rank demand [15,9,5,3]; with expert 7 (demand 1) unmapped (-1) no rank may receive
+    its assignment -- [15,9,5,2], not [15,9,5,3] with rank 3 wrapping round -- and with
+    expert 0 (demand 9) mapped to rank 4 = R the demand is [6,9,5,3].  Both set error
+    bit 2 and nothing else; the expert counts stay [9,6,5,4,3,2,2,1]."""
+    g, idx, _ = fx
+    E, R = g["experts"], g["ranks"]
+    m = _mapping(g["initial_mapping"], E)
+    assert O.expert_histogram(idx, E, R, m)["err"] == 0
+    for e, r, loads in ((7, -1, [15, 9, 5, 2]), (0, R, [6, 9, 5, 3]), (3, -R, [15, 5, 5, 3])):
+        bad = m.copy()
+        bad[e] = r
+        h = O.expert_histogram(idx, E, R, bad)
+        assert h["err"] == O.ERR_ID_RANGE
+        assert list(h["loads"]) == loads
+        assert list(h["counts"]) == g["expert_demand"]
+
+
 def test_fixture_plan_derived_by_hand(fx):
     """The balanced plan of the fixture at R=4, S=2, derived by hand from the plan's
     steps: C = 8; rank 0 keeps e1 (6) and streams e0 (9): room 2; rank 1 keeps e3 (4),
