@@ -4,8 +4,11 @@
 
 A step is one pass of the whole path (top-k, histogram/maxvio, balanced plan, replica
 prefetch, dispatch, grouped SwiGLU FFN, combine) over one batch of seeded synthetic
-inputs already resident in HBM.  The default workload is the near-balanced fine-grained
-layer (4096 tokens, 64 experts, top-6, 8 simulated ranks, 8 slots, d=2048, F=1408).
+inputs already resident in HBM.  The default workload is the largest single-GPU one, the
+DeepSeek-V3-shaped hotspot layer (16384 tokens, 256 experts, top-8, 32 simulated ranks,
+4 slots, d=7168, F=2048, ~90% of assignments on 26 hot experts).  At one GPU the line
+also carries the stand-alone top-k against the copy floor of a launch of its size and the
+Qwen-shaped maxvio sweep (tokens/s vs maxvio), each point with its own clock record.
 Under torchrun (N > 1) every rank runs an independent replica of the same layer on its
 own GPU (no collective on the data path); timing is the max over ranks.
 
@@ -36,10 +39,14 @@ METRIC = "MoE layer tokens/s"
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM bytes (read + write) per call of the dominant call (both grouped-FFN kernels) from
-# an ncu capture (profiles/ffn_kernel_near_balanced.md), keyed by workload, tile mode and
-# kernel sources hash: it reads null as soon as the kernel sources change.
+# DRAM bytes (read + write) per call of the dominant call (both grouped-FFN kernels),
+# dram__bytes_read.sum + dram__bytes_write.sum of one ncu capture of the two FFN kernels
+# (`ncu --set full --clock-control none -k regex:ffn_kernel ...` on the named workload),
+# keyed by workload, tile mode and kernel-sources hash: a kernel edit changes the hash,
+# and the line then reports null (with the reason) until the counters are taken again.
 TRAFFIC = {"near_balanced:0:d4ffa6ea7d84948f": int((926.897408 + 63.862528 + 478.883328 + 81.526272) * 1e6)}
+TRAFFIC_NOTE = {"near_balanced:0:d4ffa6ea7d84948f":
+                "ncu dram__bytes_read.sum + dram__bytes_write.sum, gate-up + down kernels, one call"}
 
 
 def sources_hash() -> str:
@@ -187,64 +194,68 @@ def barrier(world):
 
 
 # ----------------------------------------------------------------------------- our arm
-def run_ours(args, w: I.Workload, world, rank, local):
+def ffn_peak(clk: dict, peaks: dict, peak_src: str):
+    """The bf16 dense peak that matches the clocks the FFN ran at: the burst figure (a
+    GEMM timed alone, SM clock at max) when the median SM clock under load sat within 3%
+    of its max and the power cap never engaged, the sustained figure (seconds-long GEMM
+    under the 1 kW cap) otherwise."""
+    smmax = clk.get("sm_max_mhz") or peaks.get("sm_max_mhz") or 1965.0
+    sm = clk.get("sm_mhz")
+    burst = (sm is not None and sm >= 0.97 * smmax
+             and "sw_power_cap" not in clk.get("reasons", []))
+    if burst or not peaks.get("bf16_tflops_sustained"):
+        return peaks["bf16_tflops"], f"{peak_src} burst bf16 GEMM (SM clock at max, no power cap)"
+    return (peaks["bf16_tflops_sustained"],
+            f"{peak_src} sustained bf16 GEMM (SM clock below max or power cap active)")
+
+
+def rec_node_fn():
+    """An event-record node inside a graph being captured (PyTorch's Event.record does not
+    create one during capture)."""
+    rt = cudart()
+
+    def rec_node(event, st):
+        rc = rt.cudaEventRecordWithFlags(ctypes.c_void_p(event.cuda_event),
+                                         ctypes.c_void_p(st.cuda_stream), 1)
+        if rc != 0:
+            raise RuntimeError(f"cudaEventRecordWithFlags failed ({rc})")
+    return rec_node
+
+
+def measure_layer(args, w: I.Workload, world, device, steps: int, e2e: bool):
+    """K forward steps of one workload: the clean graph (the timed value), the instrumented
+    graph (per-call intervals), the clock record over both, and optionally the end-to-end
+    run through HostPipeline.  Returns a dict of raw measurements and the layer."""
     import load_balanced_dispatch_warp_b200 as M
 
-    device = torch.device("cuda", local)
-    torch.cuda.set_device(device)
     stream = torch.cuda.current_stream(device)
     logits_h = I.make_logits(w).pin_memory()
     x_h = I.make_x(w).pin_memory()
     logits = logits_h.to(device)
     x = x_h.to(device)
     W1, W3, W2 = I.make_weights(w, device=device)
-    if args.ffn_tile is not None:
-        M.set_ffn_tile_mode(args.ffn_tile)
-    ffn_tile = int(M.lib().moe_ffn_tile_mode())
     L = M.MoELayer(w.T, w.E, w.k, w.R, w.S, w.d, w.F, device=device, fused=args.fused)
     # the per-call table: the forward's calls one after the other (event nodes between them)
-    steps = [lambda: L.route_plan(logits), lambda: L.prefetch(W1, W3, W2),
+    calls = [lambda: L.route_plan(logits), lambda: L.prefetch(W1, W3, W2),
              lambda: L.dispatch(x), lambda: L.expert_ffn(W1, W3, W2), lambda: L.combine()]
 
     for _ in range(max(args.warmup, 1)):
         L.forward(logits, x, W1, W3, W2)
     torch.cuda.synchronize()
     if int(L.err.item()) != 0:
-        raise RuntimeError(f"device error word {int(L.err.item())} after warm-up")
+        raise RuntimeError(f"{w.name}: device error word {int(L.err.item())} after warm-up")
     n_rep = int(L.plan_field("replica_list")[0].item())
 
-    # device-timed region: K steps, events between the calls on the launching stream.
-    # The K steps are captured once into a CUDA graph (no host launch gaps) and replayed.
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(steps) + 1)] for _ in range(args.steps)]
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-
-    for e in [start, end] + [x for row in ev for x in row]:
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(steps)]
+    for e in [x for row in ev for x in row]:
         e.record(stream)  # create the CUDA events before any capture
     torch.cuda.synchronize()
 
-    def timed_steps(st, rec):
-        rec(start, st)
-        for s in range(args.steps):
-            e = ev[s]
-            rec(e[0], st)
-            for i, f in enumerate(steps):
-                f()
-                rec(e[i + 1], st)
-        rec(end, st)
-
-    # Two captures of the same K steps: a clean one (the timed headline) and one with an
-    # event-record node between consecutive calls (the per-call table, replayed right
-    # after, also K steps between barriers).
+    # Two captures of the same K steps: a clean one (the timed headline: the layer's forward
+    # as a user calls it) and one with an event-record node between consecutive calls.
     graph = graph_ev = None
     if not args.eager:
-        rt = cudart()
-
-        def rec_node(event, st):  # an event-record node inside the graph
-            rc = rt.cudaEventRecordWithFlags(ctypes.c_void_p(event.cuda_event),
-                                             ctypes.c_void_p(st.cuda_stream), 1)
-            if rc != 0:
-                raise RuntimeError(f"cudaEventRecordWithFlags failed ({rc})")
+        rec_node = rec_node_fn()
 
         def capture(with_events):
             g = torch.cuda.CUDAGraph()
@@ -253,10 +264,13 @@ def run_ours(args, w: I.Workload, world, rank, local):
             torch.cuda.synchronize()
             with torch.cuda.stream(cap):
                 g.capture_begin()
-                if with_events:
-                    timed_steps(cap, rec_node)
-                else:  # the timed headline: the layer's forward as a user calls it
-                    for _ in range(args.steps):
+                for s in range(steps):
+                    if with_events:
+                        rec_node(ev[s][0], cap)
+                        for i, f in enumerate(calls):
+                            f()
+                            rec_node(ev[s][i + 1], cap)
+                    else:
                         L.forward(logits, x, W1, W3, W2)
                 g.capture_end()
             torch.cuda.synchronize()
@@ -265,15 +279,14 @@ def run_ours(args, w: I.Workload, world, rank, local):
             return g
         graph = capture(False)
         graph_ev = capture(True)
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(device.index)
     clocks.start()
     time.sleep(0.3)
     barrier(world)
     torch.cuda.synchronize()
-    clocks.mark_start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
     if graph is not None:
-        t0 = torch.cuda.Event(enable_timing=True)
-        t1 = torch.cuda.Event(enable_timing=True)
         t0.record(stream)
         graph.replay()
         t1.record(stream)
@@ -282,84 +295,181 @@ def run_ours(args, w: I.Workload, world, rank, local):
         elapsed_ms = t0.elapsed_time(t1)
         graph_ev.replay()  # instrumented replay: per-call intervals
     else:
-        timed_steps(stream, lambda e, st: e.record(st))
+        t0.record(stream)
+        for s in range(steps):
+            ev[s][0].record(stream)
+            for i, f in enumerate(calls):
+                f()
+                ev[s][i + 1].record(stream)
+        t1.record(stream)
         torch.cuda.synchronize()
-        elapsed_ms = start.elapsed_time(end)
+        elapsed_ms = t0.elapsed_time(t1)
     torch.cuda.synchronize()
     barrier(world)
-    clocks.mark_end()
     clk = clocks.stop()
     elapsed_ms = max_over_ranks(elapsed_ms, world, device)
     if int(L.err.item()) != 0:
-        raise RuntimeError(f"device error word {int(L.err.item())} in the timed region")
+        raise RuntimeError(f"{w.name}: device error word {int(L.err.item())} in the timed region")
     del graph, graph_ev
-    per_call_ms = {c: sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(args.steps)) / args.steps
+    per_call_ms = {c: sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(steps)) / steps
                    for i, c in enumerate(CALLS)}
+    out = dict(layer=L, n_rep=n_rep, elapsed_ms=elapsed_ms, per_call_ms=per_call_ms, clocks=clk,
+               maxvio=float(L.maxvio.item()))
 
-    # end to end through the public API: every step copies its logits and tokens from
-    # pinned host memory and its output back; HostPipeline overlaps those copies with the
-    # neighbouring steps' compute (two device slots, three streams).
-    from load_balanced_dispatch_warp_b200.pipeline import HostPipeline
-    pipe = HostPipeline(L, W1, W3, W2)
-    outs_h = [torch.empty(w.T, w.d, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    batches = [(logits_h, x_h)] * args.steps
-    pipe.run(batches[:2], outs_h)  # warm the streams and events
-    torch.cuda.synchronize()
-    barrier(world)
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(pipe.s_in)
-    pipe.s_comp.wait_stream(pipe.s_in)
-    pipe.run(batches, [outs_h[i % 2] for i in range(args.steps)])
-    e1.record(pipe.s_out)
-    torch.cuda.synchronize()
-    barrier(world)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
-    if int(L.err.item()) != 0:
-        raise RuntimeError(f"device error word {int(L.err.item())} in the end-to-end run")
+    if e2e:
+        # end to end through the public API: every step copies its logits and tokens from
+        # pinned host memory and its output back; HostPipeline overlaps those copies with
+        # the neighbouring steps' compute (two device slots, three streams).
+        from load_balanced_dispatch_warp_b200.pipeline import HostPipeline
+        pipe = HostPipeline(L, W1, W3, W2)
+        outs_h = [torch.empty(w.T, w.d, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        batches = [(logits_h, x_h)] * steps
+        pipe.run(batches[:2], outs_h)  # warm the streams and events
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(pipe.s_in)
+        pipe.s_comp.wait_stream(pipe.s_in)
+        pipe.run(batches, [outs_h[i % 2] for i in range(steps)])
+        e1.record(pipe.s_out)
+        torch.cuda.synchronize()
+        barrier(world)
+        out["e2e_ms"] = max_over_ranks(e0.elapsed_time(e1), world, device)
+        if int(L.err.item()) != 0:
+            raise RuntimeError(f"{w.name}: device error word {int(L.err.item())} in the e2e run")
+    out["weights"] = (W1, W3, W2)
+    out["inputs"] = (logits, x)
+    return out
 
-    units = algorithmic(w, n_rep, args.fused)
-    peaks, peak_src = load_peaks()
+
+def call_table(w: I.Workload, m: dict, peaks: dict, fused: bool, tflops_peak: float):
+    """Per-call rates: algorithmic work over the in-graph interval, as a fraction of the
+    measured copy peak (HBM-bound calls) or of the clock-matched bf16 peak (the FFN)."""
+    units = algorithmic(w, m["n_rep"], fused)
     calls = {}
     for c in CALLS:
         unit, work = units[c]
-        ms = per_call_ms[c]
+        ms = m["per_call_ms"][c]
         rec = {"us": round(ms * 1e3, 2)}
         if work is not None and ms > 0:
             if unit == "TFLOP/s":
-                ach = work / (ms * 1e-3) / 1e12
-                peak = peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]
+                ach, peak = work / (ms * 1e-3) / 1e12, tflops_peak
             else:
-                ach = work / (ms * 1e-3) / 1e9
-                peak = peaks["hbm_gbs"]
+                ach, peak = work / (ms * 1e-3) / 1e9, peaks["hbm_gbs"]
             rec.update({unit.replace("/", "_per_"): round(ach, 1), "frac": round(ach / peak, 3)})
         calls[c] = rec
-    ffn_ms = per_call_ms["moe_grouped_ffn"]
+    return calls
+
+
+def topk_floor(w: I.Workload, device, reps: int = 200, copies: int = 16):
+    """Stand-alone moe_topk against the copy floor of a launch of its size.  Both run on
+    `copies` rotating input buffers (copies x T*E*4 bytes, far above the 126 MB L2) so that
+    each launch reads HBM, `reps` launches between CUDA events on the current stream.  The
+    floor is a device copy (torch copy_) whose read + write bytes equal the top-k's
+    algorithmic bytes (T*E*4 + A*8), and a copy of exactly T*E*4 bytes for reference."""
+    import load_balanced_dispatch_warp_b200 as M
+    stream = torch.cuda.current_stream(device)
+    g = torch.Generator(device=device).manual_seed(5)
+    srcs = [torch.randn(w.T, w.E, generator=g, device=device) for _ in range(copies)]
+    idx = torch.empty(w.T, w.k, dtype=torch.int32, device=device)
+    gate = torch.empty(w.T, w.k, dtype=torch.float32, device=device)
+    err = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def timed(fn):
+        for i in range(copies):
+            fn(i)
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for r in range(reps):
+            fn(r % copies)
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps * 1e3  # us per launch
+
+    topk_us = timed(lambda i: M.moe_topk(srcs[i], w.k, idx, gate, err))
+    alg = w.T * w.E * 4 + w.A * 8
+    half = [torch.empty(alg // 2 // 4, dtype=torch.float32, device=device) for _ in range(2 * copies)]
+    copy_us = timed(lambda i: half[2 * i].copy_(half[2 * i + 1]))
+    full = [torch.empty(w.T * w.E, dtype=torch.float32, device=device) for _ in range(2 * copies)]
+    copy_full_us = timed(lambda i: full[2 * i].copy_(full[2 * i + 1]))
+    if int(err.item()) != 0:
+        raise RuntimeError("moe_topk set the error word on random logits")
+    del srcs, half, full
+    torch.cuda.empty_cache()
+    topk_gbs = alg / (topk_us * 1e-6) / 1e9
+    floor_gbs = (alg // 2 // 4 * 4 * 2) / (copy_us * 1e-6) / 1e9
+    return {"us": round(topk_us, 2), "GB_per_s": round(topk_gbs, 1),
+            "algorithmic_bytes": alg,
+            "copy_floor_us": round(copy_us, 2), "copy_floor_GB_per_s": round(floor_gbs, 1),
+            "frac_of_copy_floor": round(topk_gbs / floor_gbs, 3),
+            "copy_of_logits_us": round(copy_full_us, 2),
+            "what": f"moe_topk alone, {copies} rotating logits buffers, {reps} launches; floor = "
+                    f"torch copy_ moving the same bytes (read + write), same rotation"}
+
+
+def summarize(w: I.Workload, m: dict, peaks: dict, peak_src: str, fused: bool, steps: int):
+    """Compact record of one workload: tokens/s, the per-call table, the FFN against the
+    clock-matched peak, and the FFN's duration in SM cycles at the median clock."""
+    tpk, tpk_src = ffn_peak(m["clocks"], peaks, peak_src)
+    calls = call_table(w, m, peaks, fused, tpk)
+    ffn_us = m["per_call_ms"]["moe_grouped_ffn"] * 1e3
+    sm = m["clocks"].get("sm_mhz")
+    return {"value": round(w.T * steps / (m["elapsed_ms"] * 1e-3), 1),
+            "ms_per_step": round(m["elapsed_ms"] / steps, 4), "maxvio": round(m["maxvio"], 4),
+            "replicas": m["n_rep"], "calls": calls, "clocks": m["clocks"],
+            "ffn_peak": tpk, "ffn_peak_source": tpk_src,
+            "ffn_mcycles": round(ffn_us * sm / 1e6, 4) if sm else None}
+
+
+def run_ours(args, w: I.Workload, world, rank, local):
+    import load_balanced_dispatch_warp_b200 as M
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if args.ffn_tile is not None:
+        M.set_ffn_tile_mode(args.ffn_tile)
+    ffn_tile = int(M.lib().moe_ffn_tile_mode())
+    peaks, peak_src = load_peaks()
+
+    m = measure_layer(args, w, world, device, args.steps, e2e=True)
+    L = m["layer"]
+    head = summarize(w, m, peaks, peak_src, args.fused, args.steps)
+    units = algorithmic(w, m["n_rep"], args.fused)
+    ffn_ms = m["per_call_ms"]["moe_grouped_ffn"]
     ffn_flops = units["moe_grouped_ffn"][1]
-    peak_t = peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]
     achieved = ffn_flops / (ffn_ms * 1e-3) / 1e12
     tkey = f"{w.name}:{ffn_tile}:{sources_hash()}"
-    roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak_t, "unit": "TFLOP/s",
-                "frac": round(achieved / peak_t, 3), "traffic": TRAFFIC.get(tkey),
+    traffic = TRAFFIC.get(tkey)
+    roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": head["ffn_peak"],
+                "unit": "TFLOP/s", "frac": round(achieved / head["ffn_peak"], 3),
+                "traffic": traffic,
+                "traffic_note": (TRAFFIC_NOTE.get(tkey) if traffic is not None else
+                                 "null: no ncu DRAM capture of this workload at these kernel "
+                                 f"sources (key {tkey})"),
                 "kernel": "moe_grouped_ffn (gate-up and down tcgen05 GEMMs)",
-                "peak_source": f"{peak_src} sustained bf16 GEMM",
+                "peak_source": head["ffn_peak_source"],
+                "ffn_mcycles_at_median_sm_clock": head["ffn_mcycles"],
                 "work_per_launch": f"6*A*d*F = {ffn_flops:.4g} flop (A=T*k={w.A})"}
 
-    value = w.T * args.steps * world / (elapsed_ms * 1e-3)
-    e2e_value = w.T * args.steps * world / (e2e_ms * 1e-3)
+    value = w.T * args.steps * world / (m["elapsed_ms"] * 1e-3)
+    e2e_value = w.T * args.steps * world / (m["e2e_ms"] * 1e-3)
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(elapsed_ms / args.steps, 4),
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(m["elapsed_ms"] / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16+fp16 (gate/up GEMM bf16, down GEMM fp16, fp32 accumulate; routing fp32)",
         "data": "synthetic (seeded; N(0,1) logits + per-expert bias, N(0,1) tokens, N(0,1/d) weights)",
         "config": {"workload": w.name, "T": w.T, "E": w.E, "k": w.k, "R": w.R, "S": w.S, "d": w.d,
-                   "F": w.F, "maxvio": round(float(L.maxvio.item()), 4), "replicas": n_rep,
+                   "F": w.F, "maxvio": round(m["maxvio"], 4), "replicas": m["n_rep"],
                    # makespan proxy: rows of the busiest rank / C, with the plan and with
                    # every expert at its home rank
                    "max_rank_rows_over_C": 1.0,
-                   "home_only_max_rank_rows_over_C": round(1.0 + float(L.maxvio.item()), 4),
+                   "home_only_max_rank_rows_over_C": round(1.0 + m["maxvio"], 4),
                    "parallelism": f"replicas x{world} (ranks simulated in one GPU's HBM)",
                    "dispatch": ("fused: placement only, GEMM 1 gathers x[src[row]]" if args.fused
                                 else "row copy into recv, GEMM 1 reads recv"),
@@ -367,30 +477,54 @@ def run_ours(args, w: I.Workload, world, rank, local):
                                 if ffn_tile == 1 and not args.fused
                                 else "128-row tiles, one CTA each (tcgen05 cta_group::1)"),
                    "ffn_pair_clusters": M.ffn_pair_clusters() if ffn_tile == 1 else None,
-                   "l2": "step working set (weights, pool, activations) far above the 126 MB L2",
+                   "l2": "inputs larger than L2: the step's working set (weights, pool, "
+                         "activations) is far above the 126 MB L2, no flush inserted",
                    "launch": "eager, one stream, calls in order" if args.eager else
                              "K forward steps (MoELayer.forward: routing/histogram/plan fused in "
                              "one launch, then prefetch, dispatch, FFN, combine) captured in one "
                              "CUDA graph, replayed once; per-call intervals from a second replay "
                              "with event nodes between the calls"},
-        "clocks": clk,
+        "clocks": m["clocks"],
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT,
                 "h2d_bytes_per_step": w.T * w.E * 4 + w.T * w.d * 2,
                 "d2h_bytes_per_step": w.T * w.d * 2},
         "gpu_launches": L.kernels_per_forward() * args.steps,
         "roofline": roofline,
-        "calls": calls,
+        "calls": head["calls"],
     }
     if args.backward:
-        res["train_step"] = time_training_step(args, w, L, logits, x, W1, W3, W2, world, device, peaks)
+        W1, W3, W2 = m["weights"]
+        logits, x = m["inputs"]
+        res["train_step"] = time_training_step(args, w, L, logits, x, W1, W3, W2, world, device,
+                                               peaks, head["ffn_peak"])
+    del m, L
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_extras:
+        res["topk_standalone"] = topk_floor(w, device)
+        sweep = {}
+        for name in SWEEP:
+            ws = I.WORKLOADS[name]
+            ms = measure_layer(args, ws, world, device, args.sweep_steps, e2e=False)
+            sweep[name] = summarize(ws, ms, peaks, peak_src, args.fused, args.sweep_steps)
+            del ms
+            torch.cuda.empty_cache()
+        res["maxvio_sweep"] = {"workloads": sweep, "steps": args.sweep_steps,
+                               "what": "Qwen3-30B-A3B-shaped layer (T=8192, E=128, k=8, R=16, "
+                                       "S=8, d=2048, F=768) at maxvio 0.2 / 1 / 5 / 15 "
+                                       "(15 = the largest this R allows, standing in for 20)"}
     return res
+
+
+# Qwen-shaped skew sweep carried beside the headline (tokens/s vs maxvio)
+SWEEP = ["qwen_mv0.2", "qwen_mv1", "qwen_mv5", "qwen_mv15"]
 
 
 BWD_CALLS = ["moe_combine_backward", "moe_grouped_ffn_backward", "moe_dispatch_backward",
              "moe_topk_backward"]
 
 
-def time_training_step(args, w: I.Workload, L, logits, x, W1, W3, W2, world, device, peaks):
+def time_training_step(args, w: I.Workload, L, logits, x, W1, W3, W2, world, device, peaks,
+                       peak_t):
     """Forward + backward of the layer (dout seeded N(0,1) bf16), K steps in one CUDA graph
     after warm-up; per-call backward intervals from a replay with event nodes between the
     calls.  The grouped-FFN backward does 16*A*d*F flops: dH (2AdF), the gate/up GEMM re-run
@@ -416,12 +550,7 @@ def time_training_step(args, w: I.Workload, L, logits, x, W1, W3, W2, world, dev
         for e in row:
             e.record()
     torch.cuda.synchronize()
-    rt = cudart()
-
-    def rec_node(event, st):
-        rc = rt.cudaEventRecordWithFlags(ctypes.c_void_p(event.cuda_event), ctypes.c_void_p(st.cuda_stream), 1)
-        if rc != 0:
-            raise RuntimeError(f"cudaEventRecordWithFlags failed ({rc})")
+    rec_node = rec_node_fn()
 
     def capture(with_events):
         gr = torch.cuda.CUDAGraph()
@@ -465,7 +594,6 @@ def time_training_step(args, w: I.Workload, L, logits, x, W1, W3, W2, world, dev
            for i, c in enumerate(BWD_CALLS)}
     A, d, F = w.A, w.d, w.F
     ffn_flops = 16 * A * d * F
-    peak_t = peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"]
     calls = {c: {"us": round(v * 1e3, 2)} for c, v in per.items()}
     t_ffn = per["moe_grouped_ffn_backward"] * 1e-3
     calls["moe_grouped_ffn_backward"].update(
@@ -575,9 +703,13 @@ def run_reference(args, w):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="near_balanced", choices=sorted(I.WORKLOADS))
+    ap.add_argument("--config", default="deepseek", choices=sorted(I.WORKLOADS))
+    ap.add_argument("--sweep-steps", type=int, default=50,
+                    help="steps per point of the Qwen-shaped maxvio sweep")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the stand-alone top-k floor and the maxvio sweep")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="launch the timed steps eagerly")

@@ -93,3 +93,19 @@ def test_reference_arm_line_keeps_the_contract(monkeypatch):
     assert e2e["value"] == line["value"] and e2e["unit"] == bench.UNIT
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
     assert line["vs_baseline"] is None
+
+
+def test_ffn_peak_follows_the_clock_record():
+    """The FFN's roofline denominator matches the clocks it ran at: the burst GEMM peak
+    when the median SM clock sat at max with no power cap, the sustained one otherwise."""
+    peaks = {"bf16_tflops": 1702.2, "bf16_tflops_sustained": 1430.7, "sm_max_mhz": 1965.0}
+    at_max = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    capped = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    low = {"sm_mhz": 1207.0, "sm_max_mhz": 1965.0, "reasons": []}
+    assert bench.ffn_peak(at_max, peaks, "measured")[0] == 1702.2
+    assert "burst" in bench.ffn_peak(at_max, peaks, "measured")[1]
+    assert bench.ffn_peak(capped, peaks, "measured")[0] == 1430.7
+    assert bench.ffn_peak(low, peaks, "measured")[0] == 1430.7
+    assert "sustained" in bench.ffn_peak(low, peaks, "measured")[1]
+    # a record without samples cannot show the burst conditions
+    assert bench.ffn_peak({"sm_mhz": None, "reasons": ["no samples"]}, peaks, "measured")[0] == 1430.7
