@@ -39,7 +39,12 @@ Pins (tests/test_oracle_pins.py checks each against something other than this fi
   expert_ffn        closed forms: identity / single-entry weights give silu(a)*a with
                     silu(1) = e/(1+e); transposed operands land in distinct outputs
   combine           identity experts return x (gates sum to one); per-expert scaling
-                    returns (sum_j gate_j c_e) x
+                    returns (sum_j gate_j c_e) x; dropped assignments (perm = -1) add
+                    nothing
+  dispatch_capacity the pages' worked fixture at cap 5 (processed [5,5,5,4,3,2,2,1],
+  layer_capacity    overflow [4,1,0,...], padding 13, the dropped assignments derived by
+                    hand); a capacity above every demand reduces to the dropless layer;
+                    identity experts return (sum of kept gates) x
   layer_backward    central finite differences of layer() itself (fp64, tiny shapes,
                     away from top-k ties); torch.autograd (fp64, CPU) through a token-major
                     formulation with no plan, dispatch or replicas; the weight gradients do
@@ -376,6 +381,55 @@ def permute(idx: np.ndarray, plan, E: int, R: int):
     return perm, src
 
 
+def capacity_of(A: int, E: int, cf_num: int = 5, cf_den: int = 4) -> int:
+    """Per-expert capacity of the fixed-capacity mode ([Hotspots] "Make expert capacity,
+    overflow, and padding explicit"): ceil(assignments / experts * capacity factor), the
+    factor an exact rational cf_num / cf_den (1.25 = 5/4 in the page's example)."""
+    return -(-(A * cf_num) // (E * cf_den))
+
+
+def dispatch_capacity(idx: np.ndarray, E: int, cap: int):
+    """Fixed-capacity placement ([Hotspots] "Make expert capacity, overflow, and padding
+    explicit"): every expert owns a static block of cap rows, rows [e*cap, (e+1)*cap), and
+    the limit is applied to each expert independently.  The q-th assignment of expert e
+    in token order (q = 0, 1, ...) is processed when q < cap and lands at row e*cap + q;
+    the ones after it overflow and are dropped (perm = -1).  Rows of a block past the
+    expert's processed count are padding (src = -1).  Which assignments the limit keeps is
+    not on the page; token order is the plainest reading.  Overflow is counted from the
+    raw demand before anything is excluded.
+
+    Returns perm [T,k] int32 (row or -1), src [E*cap] int32 (token or -1), and the
+    per-expert processed / overflow / padding counts as int64 arrays."""
+    idx = np.asarray(idx)
+    T, k = idx.shape
+    seen = [0] * E
+    perm = np.full((T, k), -1, dtype=np.int32)
+    src = np.full(E * cap, -1, dtype=np.int32)
+    for t in range(T):
+        for j in range(k):
+            e = int(idx[t, j])
+            q = seen[e]
+            seen[e] += 1
+            if q < cap:
+                perm[t, j] = e * cap + q
+                src[e * cap + q] = t
+    demand = np.array(seen, dtype=np.int64)
+    processed = np.minimum(demand, cap)
+    return perm, src, dict(processed=processed, overflow=demand - processed,
+                           padding=cap - processed)
+
+
+def dispatch_padded(x: np.ndarray, src: np.ndarray) -> np.ndarray:
+    """Rows of a fixed-capacity buffer: token src[r]'s row, zeros where src[r] = -1
+    (padding)."""
+    x = np.asarray(x)
+    src = np.asarray(src)
+    out = np.zeros((len(src), x.shape[1]), dtype=x.dtype)
+    keep = src >= 0
+    out[keep] = x[src[keep]]
+    return out
+
+
 def dispatch(x: np.ndarray, src: np.ndarray) -> np.ndarray:
     """Dispatch ([Primer] phase (b)): row r of the receive buffer is token src[r]'s row.
     A bitwise copy; each token lands once per chosen expert (O(top-k) volume)."""
@@ -449,18 +503,31 @@ def grouped_ffn(recv, plan, E: int, W1, W3, W2, pool, rows=None):
 def combine(y, perm, gate, tokens=None):
     """Combine ([Primer] phase (d), the transpose of dispatch): token t's output is
     sum_j gate[t,j] * y[perm[t,j]], accumulated in j order in fp64.  ``y`` may be an
-    array or a {row: vector} map (sampled parity); ``tokens`` limits the evaluation."""
+    array or a {row: vector} map (sampled parity); ``tokens`` limits the evaluation.
+    An assignment dropped by the fixed-capacity mode (perm = -1) is left out of the sum;
+    a token whose assignments were all dropped gets zeros."""
     perm = np.asarray(perm)
     gate = np.asarray(gate, dtype=np.float64)
     T, k = perm.shape
     toks = range(T) if tokens is None else tokens
+    width = None
     out = {}
     for t in toks:
         acc = None
         for j in range(k):
-            v = gate[t, j] * np.asarray(y[int(perm[t, j])], dtype=np.float64)
+            r = int(perm[t, j])
+            if r < 0:
+                continue
+            v = gate[t, j] * np.asarray(y[r], dtype=np.float64)
+            width = v.shape[0]
             acc = v if acc is None else acc + v
         out[int(t)] = acc
+    for t in out:
+        if out[t] is None:
+            if width is None:
+                width = (np.asarray(y).shape[1] if not isinstance(y, dict)
+                         else len(next(iter(y.values()))))
+            out[t] = np.zeros(width)
     if tokens is None:
         return np.stack([out[t] for t in range(T)]) if T else np.zeros((0, 0))
     return out
@@ -485,6 +552,31 @@ def layer(logits, x, W1, W3, W2, k: int, R: int, S: int):
     return dict(idx=idx, gate=gate, hist=h, plan=plan, pool=pool, perm=perm, src=src,
                 recv=recv, y=y, out=out, err=err)
 
+
+
+def layer_capacity(logits, x, W1, W3, W2, k: int, cf_num: int = 5, cf_den: int = 4):
+    """The fixed-capacity (dropping) mode of the layer ([Hotspots] "Make expert capacity,
+    overflow, and padding explicit"): route, measure the raw demand (the ledger is taken
+    before any exclusion), place each expert's first cap assignments in its static
+    block, run every expert over its whole block -- padding rows are zeros and cost the
+    same work, the reserved work the page weighs against overflow -- and combine with the
+    dropped assignments left out.  Small shapes only."""
+    logits = np.asarray(logits, dtype=np.float32)
+    T, E = logits.shape
+    A = T * k
+    idx, gate, err = topk_route(logits, k)
+    h = expert_histogram(idx, E, 1)
+    err |= h["err"]
+    cap = capacity_of(A, E, cf_num, cf_den)
+    led = capacity_ledger(h["counts"], A, E, cf_num, cf_den)
+    perm, src, rows = dispatch_capacity(idx, E, cap)
+    recv = dispatch_padded(x, src)
+    y = np.zeros((E * cap, np.asarray(W2).shape[1]))
+    for e in range(E):
+        y[e * cap:(e + 1) * cap] = expert_ffn(recv[e * cap:(e + 1) * cap], W1[e], W3[e], W2[e])
+    out = combine(y, perm, gate)
+    return dict(idx=idx, gate=gate, hist=h, cap=cap, ledger=led, rows=rows, perm=perm, src=src,
+                recv=recv, y=y, out=out, err=err)
 
 
 # ------------------------------------------------------------------ backward pass

@@ -171,3 +171,66 @@ def check_ffn_combine_sampled(L, w, x, weights, ref, tokens):
     out_ref = O.combine(y_ref, ref["perm"], ref["gate"], tokens=tokens)
     out_gpu = to64(L.out[torch.tensor(tokens, device="cuda")])
     assert_close_scaled(out_gpu, np.stack([out_ref[t] for t in tokens]), "out (sampled tokens)")
+
+
+def edge_rows(plan, E: int, tile: int = 128):
+    """Rows of the grouped FFN where a tiling mistake would show, as {name: [rows]}: every
+    row of the last (partial) tile of the largest group; rows 126-129 of a group that spans
+    more than one tile (the first tile boundary); every row of the smallest replica group
+    (weights from a pool slot); every row of the last group of the last rank."""
+    groups = [g for gl in plan["groups"] for g in gl]
+    out = {}
+    r0, n, _, _ = max(groups, key=lambda g: (g[1], -g[0]))
+    last = r0 + tile * ((n - 1) // tile)
+    out["last tile of the largest group"] = list(range(last, r0 + n))
+    multi = [g for g in groups if g[1] > tile + 2]
+    if multi:
+        r0, n, _, _ = multi[0]
+        out["rows 126-129 of a multi-tile group"] = [r0 + i for i in range(tile - 2, tile + 2)]
+    reps = [g for g in groups if g[3] >= E]
+    if reps:
+        r0, n, _, _ = min(reps, key=lambda g: (g[1], g[0]))
+        out["smallest replica group"] = list(range(r0, r0 + n))
+    lastr = [gl for gl in plan["groups"] if gl][-1]
+    r0, n, _, _ = lastr[-1]
+    out["last group of the last rank"] = list(range(r0, r0 + n))
+    return out
+
+
+def check_ffn_edge_rows(L, w, x, weights, ref):
+    """h and y of edge_rows() against the fp64 oracle (each row through its group's expert;
+    a replica slot holds its expert's home weights bitwise)."""
+    p = ref["plan"]
+    row_expert = {}
+    sets = edge_rows(p, w.E)
+    want = sorted({r for rs in sets.values() for r in rs})
+    wanted = set(want)
+    for gl in p["groups"]:
+        for (r0, n, e, _) in gl:
+            for r in range(r0, r0 + n):
+                if r in wanted:
+                    row_expert[r] = e
+    rows_t = torch.tensor(want, device="cuda")
+    if L.recv is not None:
+        recv = to64(L.recv[rows_t])
+    else:
+        recv = to64(x)[ref["src"][want]]
+    ridx = {r: i for i, r in enumerate(want)}
+    h_ref = np.zeros((len(want), w.F))
+    y_ref = np.zeros((len(want), w.d))
+    by_e = {}
+    for r in want:
+        by_e.setdefault(row_expert[r], []).append(r)
+    for e, rs in by_e.items():
+        w1, w3, w2 = expert_weights64(weights, e)
+        X = recv[[ridx[r] for r in rs]]
+        ii = [ridx[r] for r in rs]
+        h_ref[ii] = O.silu(X @ w1.T) * (X @ w3.T)
+        y_ref[ii] = O.expert_ffn(X, w1, w3, w2)
+    h_gpu = to64(L.h[rows_t])
+    y_gpu = to64(L.y[rows_t])
+    for name, rs in sets.items():
+        ii = [ridx[r] for r in rs]
+        assert_close_scaled(h_gpu[ii], h_ref[ii], f"h, {name}")
+        assert_close_scaled(y_gpu[ii], y_ref[ii], f"y, {name}")
+    return sets

@@ -17,8 +17,9 @@ from load_balanced_dispatch_warp_b200 import build
 from load_balanced_dispatch_warp_b200 import inputs as I
 from oracle import moe_oracle as O
 
-from harness import (check_ffn_combine_full, check_ffn_combine_sampled, check_integer_parity,
-                     check_rows_and_pool, make_inputs, oracle_integer_path, run_gpu)
+from harness import (check_ffn_combine_full, check_ffn_combine_sampled, check_ffn_edge_rows,
+                     check_integer_parity, check_rows_and_pool, edge_rows, make_inputs,
+                     oracle_integer_path, run_gpu)
 
 pytestmark = pytest.mark.gpu
 
@@ -74,6 +75,10 @@ def test_layer_parity_full_size(name):
     rng = np.random.default_rng(11)
     tokens = sorted(rng.choice(w.T, size=8, replace=False).tolist()) + [w.T - 1]
     check_ffn_combine_sampled(L, w, x, weights, ref, tokens)
+    # h and y at the rows where tiling breaks: the last partial tile of the largest group,
+    # a 128-row tile boundary, a replica group, the last group of the last rank
+    sets = check_ffn_edge_rows(L, w, x, weights, ref)
+    assert len(sets) == 4, sorted(sets)
     del L, weights
     torch.cuda.empty_cache()
 

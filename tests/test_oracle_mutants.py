@@ -182,7 +182,32 @@ def test_forward_pin_catches_planted_mistake(monkeypatch, name, mutant, pin):
 
 # ------------------------------------------------------------------ ledgers and variants
 VAR = {n: getattr(O, n) for n in ("validate_trace", "capacity_ledger", "remote_routes",
-                                  "topk_route_biased")}
+                                  "topk_route_biased", "dispatch_capacity", "combine")}
+
+
+def capacity_keeps_the_last_assignments(idx, E, cap):
+    """Keeps the LAST cap assignments of each expert (reverse token order)."""
+    idx = np.asarray(idx)
+    T = idx.shape[0]
+    perm, src, rows = VAR["dispatch_capacity"](idx[::-1], E, cap)
+    perm = perm[::-1].copy()
+    src = np.where(src >= 0, T - 1 - src, -1).astype(np.int32)
+    return perm, src, rows
+
+
+def capacity_padding_absorbs_overflow(idx, E, cap):
+    """Padding computed as cap - demand, so overflow cancels padding in the totals."""
+    perm, src, rows = VAR["dispatch_capacity"](idx, E, cap)
+    rows = dict(rows)
+    rows["padding"] = cap - (rows["processed"] + rows["overflow"])
+    return perm, src, rows
+
+
+def combine_reads_dropped_rows(y, perm, gate, tokens=None):
+    """A dropped assignment (perm = -1) read as the last row of y instead of left out."""
+    perm = np.asarray(perm)
+    y = np.asarray(y)
+    return VAR["combine"](y, np.where(perm < 0, len(y) - 1, perm), gate, tokens)
 
 
 def validate_without_repeat_check(idx, E):
@@ -213,10 +238,16 @@ VAR_CASES = [
     ("capacity_ledger", ledger_overflow_unclamped, lambda: F.test_fixture_capacity_ledger(fixture())),
     ("remote_routes", remote_counts_local_routes, lambda: F.test_fixture_remote_routes(fixture())),
     ("topk_route_biased", biased_gate_from_biased_scores, F.test_biased_topk_pins),
+    ("dispatch_capacity", capacity_keeps_the_last_assignments,
+     lambda: F.test_fixture_fixed_capacity_dispatch(fixture())),
+    ("dispatch_capacity", capacity_padding_absorbs_overflow,
+     lambda: F.test_fixture_fixed_capacity_dispatch(fixture())),
+    ("combine", combine_reads_dropped_rows, F.test_combine_leaves_dropped_assignments_out),
 ]
 
 
-@pytest.mark.parametrize("name,mutant,pin", VAR_CASES, ids=[c[0] for c in VAR_CASES])
+@pytest.mark.parametrize("name,mutant,pin", VAR_CASES,
+                         ids=[f"{c[0]}-{c[1].__name__}" for c in VAR_CASES])
 def test_ledger_and_variant_pins_catch_planted_mistakes(monkeypatch, name, mutant, pin):
     pin()
     monkeypatch.setattr(O, name, mutant)

@@ -119,6 +119,108 @@ def test_fixture_mapping_must_cover_every_expert(fx):
         assert list(h["counts"]) == g["expert_demand"]
 
 
+def test_fixture_fixed_capacity_dispatch(fx):
+    """Fixed capacity 5 on the fixture ("Make expert capacity, overflow, and padding
+    explicit"): processed [5,5,5,4,3,2,2,1] (27), overflow [4,1,0,...] (5), padding 13.
+    Derived by hand from the pairs 01,02,03,04,05,06,07,01,02,12,12,12,13,34,34,56 with
+    each expert keeping its first five assignments in token order: expert 0 is chosen by
+    tokens 0..8 and keeps 0..4 (tokens 5,6,7,8 dropped); expert 1 by tokens 0,7,9,10,11,12
+    and drops token 12; expert 2 by 1,8,9,10,11 (all kept); expert 3 by 2,12,13,14 (one
+    padding row)."""
+    g, idx, _ = fx
+    E = g["experts"]
+    cap = O.capacity_of(g["assignments"], E, *g["capacity_factor_num_den"])
+    assert cap == g["capacity"] == 5
+    perm, src, rows = O.dispatch_capacity(idx, E, cap)
+    assert list(rows["processed"]) == g["processed"] and rows["processed"].sum() == 27
+    assert list(rows["overflow"]) == g["overflow"] and rows["overflow"].sum() == 5
+    assert list(rows["padding"]) == g["padding"] and rows["padding"].sum() == 13
+    dropped = sorted((t, j) for t in range(16) for j in range(2) if perm[t, j] < 0)
+    assert dropped == [(5, 0), (6, 0), (7, 0), (8, 0), (12, 0)]
+    assert list(src[0:5]) == [0, 1, 2, 3, 4]
+    assert list(src[5:10]) == [0, 7, 9, 10, 11]
+    assert list(src[10:15]) == [1, 8, 9, 10, 11]
+    assert list(src[15:20]) == [2, 12, 13, 14, -1]
+    assert int((src < 0).sum()) == 13
+    # every kept assignment is the row its block says; rows of one expert hold that expert
+    for t in range(16):
+        for j in range(2):
+            r = int(perm[t, j])
+            if r >= 0:
+                assert src[r] == t and r // cap == idx[t, j]
+
+
+def test_capacity_ledger_invariants_on_random_traces():
+    """On random traces and capacities: processed + overflow = demand, processed +
+    padding = cap, kept assignments fill each block from its first row with no gaps, and
+    the dispatch's counts equal capacity_ledger's (two separate restatements of the page's
+    min / max formulas)."""
+    rng = np.random.default_rng(3)
+    for _ in range(40):
+        E = int(rng.integers(1, 9))
+        k = int(rng.integers(1, E + 1))
+        T = int(rng.integers(0, 30))
+        idx = np.array([rng.permutation(E)[:k] for _ in range(T)], dtype=np.int32).reshape(T, k)
+        num, den = int(rng.integers(1, 9)), int(rng.integers(1, 5))
+        cap = O.capacity_of(T * k, E, num, den)
+        perm, src, rows = O.dispatch_capacity(idx, E, cap)
+        demand = np.bincount(idx.reshape(-1), minlength=E) if T else np.zeros(E, int)
+        assert np.array_equal(rows["processed"] + rows["overflow"], demand)
+        assert np.array_equal(rows["processed"] + rows["padding"], np.full(E, cap))
+        led = O.capacity_ledger(demand, T * k, E, num, den)
+        assert led["cap"] == cap
+        for key in ("processed", "overflow", "padding"):
+            assert np.array_equal(led[key], rows[key])
+        for e in range(E):
+            block = src[e * cap:(e + 1) * cap]
+            n = int(rows["processed"][e])
+            assert (block[:n] >= 0).all() and (block[n:] == -1).all()
+        assert int((perm >= 0).sum()) == int(rows["processed"].sum())
+
+
+def test_capacity_above_every_demand_is_the_dropless_layer():
+    """With a capacity factor large enough that no expert overflows, the fixed-capacity
+    layer computes the dropless layer's output (different row layout, same sums)."""
+    rng = np.random.default_rng(4)
+    T, E, k, d, F = 24, 4, 2, 16, 24
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    x = rng.standard_normal((T, d))
+    W1 = rng.standard_normal((E, F, d)) / 4
+    W3 = rng.standard_normal((E, F, d)) / 4
+    W2 = rng.standard_normal((E, d, F)) / 4
+    ref = O.layer(logits, x, W1, W3, W2, k, 2, 2)
+    cap = O.layer_capacity(logits, x, W1, W3, W2, k, cf_num=E, cf_den=1)
+    assert ref["err"] == 0 and cap["err"] == 0
+    assert (cap["perm"] >= 0).all() and cap["rows"]["overflow"].sum() == 0
+    assert np.allclose(cap["out"], ref["out"], rtol=1e-12, atol=1e-12)
+    # and a small factor drops assignments: those tokens lose the dropped terms
+    tight = O.layer_capacity(logits, x, W1, W3, W2, k, cf_num=1, cf_den=2)
+    assert tight["rows"]["overflow"].sum() > 0
+    assert not np.allclose(tight["out"], ref["out"])
+
+
+def test_combine_leaves_dropped_assignments_out():
+    """Identity experts (y = the dispatched rows) on a fixed-capacity buffer: token t gets
+    (sum of its kept gates) * x_t -- the dropped choices add nothing -- and a token with
+    every choice dropped gets zeros."""
+    rng = np.random.default_rng(5)
+    T, E, k, d = 40, 4, 2, 8
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    logits[:, 0] += 3.0  # expert 0 overflows
+    x = rng.standard_normal((T, d))
+    idx, gate, _ = O.topk_route(logits, k)
+    cap = O.capacity_of(T * k, E, 1, 1)
+    perm, src, rows = O.dispatch_capacity(idx, E, cap)
+    assert rows["overflow"][0] > 0
+    y = O.dispatch_padded(x, src)
+    y[src < 0] = 1e3  # no kept assignment points at a padding row: its contents never show
+    out = O.combine(y, perm, gate)
+    kept = np.where(perm >= 0, gate, 0.0).sum(axis=1)
+    assert np.allclose(out, kept[:, None] * x, rtol=1e-13, atol=1e-13)
+    none = O.combine(np.zeros((4, d)), np.full((3, 2), -1), np.full((3, 2), 0.5))
+    assert none.shape == (3, d) and (none == 0).all()
+
+
 def test_fixture_plan_derived_by_hand(fx):
     """The balanced plan of the fixture at R=4, S=2, derived by hand from the plan's
     steps: C = 8; rank 0 keeps e1 (6) and streams e0 (9): room 2; rank 1 keeps e3 (4),
