@@ -86,7 +86,9 @@ typedef struct moe_plan_layout {
 /* Fills *out with the plan layout for (E, R, S).  Host only; returns a host status. */
 int moe_plan_get_layout(int E, int R, int S, moe_plan_layout* out);
 
-/* int32 words of the workspace moe_dispatch needs for T tokens and E experts. */
+/* int32 words of the workspace moe_dispatch (and moe_dispatch_index,
+ * moe_dispatch_capacity) needs for T tokens and E experts: a few words of status per
+ * 256-token tile and two E-long count vectors per tile. */
 int64_t moe_dispatch_workspace_words(int T, int E);
 
 /* Static description of a host status code. */
@@ -357,22 +359,69 @@ int moe_topk_backward(const float* gate, const float* dgate, const int32_t* idx,
  * input and output buffers, or a host program whose hot path must not call cudaMalloc
  * (which may synchronise the device).  It computes exactly what moe_dispatch computes,
  * with the same arguments minus `workspace`, and allocates nothing: the placement
- * counts live in a static device array of MOE_NOALLOC_SCRATCH_WORDS int32 words (1 MiB)
+ * counts live in a static device array of MOE_NOALLOC_SCRATCH_WORDS int32 words (2 MiB)
  * that every GPU loading the library holds until the process exits.
  *   - Returns MOE_ERR_SHAPE when moe_dispatch_workspace_words(T, E) exceeds
- *     MOE_NOALLOC_SCRATCH_WORDS (e.g. T = 65536 with E = 1024 fits, T = 131072 does not).
+ *     MOE_NOALLOC_SCRATCH_WORDS (e.g. T = 65536 with E = 512 fits, with E = 1024 it does
+ *     not; T = 32768 with E = 1024 fits).
  *   - The first call in each CUDA context of a device looks up the array's device
  *     address (cudaGetSymbolAddress, with that device current) and keeps it for that
  *     context; after a cudaDeviceReset the next call looks it up again.  Make the first
  *     call on a device before any stream capture.  MOE_ERR_DEVICE if the lookup fails.
- *   - All calls share the array and it keeps the last call's contents; no word of it has
- *     to start at zero.  Calls that overlap on the GPU (several streams or host threads
- *     on one device) race on it: serialise them.
+ *   - All calls share the array and it keeps the last call's contents; each call clears
+ *     the words it needs at zero itself.  Calls that overlap on the GPU (several streams or
+ *     host threads on one device) race on it: serialise them.
  */
-#define MOE_NOALLOC_SCRATCH_WORDS 262144
+#define MOE_NOALLOC_SCRATCH_WORDS 524288
 int moe_dispatch_noalloc(const moe_bf16* x, const int32_t* idx, const int32_t* plan, int T,
                          int k, int E, int R, int S, int d, moe_bf16* recv, int32_t* perm,
                          int32_t* src, int32_t* err, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * Fixed-capacity (dropping) mode.   [Hotspots] "Make expert capacity, overflow, and
+ * padding explicit": each expert gets cap = ceil(A / E * cf) rows, the limit applied to
+ * each expert independently; processed = min(demand, cap), overflow = max(demand - cap,
+ * 0) (recorded before anything is excluded: moe_histogram_maxvio's counts and
+ * moe_capacity_ledger), padding = max(cap - demand, 0) unused rows that still cost work.
+ * Which assignments an expert keeps is not on the page: here its first cap assignments in
+ * token order.  The layer path in this mode: moe_topk, moe_histogram_maxvio (raw demand),
+ * moe_capacity_ledger, moe_dispatch_capacity, moe_grouped_ffn_capacity,
+ * moe_combine_capacity.  (The default path above is dropless: zero drops, zero padding.)
+ *
+ * moe_capacity_rows: cap for T*k assignments over E experts at capacity factor
+ *   cf_num / cf_den (an exact rational); -1 for a non-positive argument.  Host only.
+ */
+int64_t moe_capacity_rows(int T, int k, int E, int cf_num, int cf_den);
+/*
+ * moe_dispatch_capacity: expert e owns rows [e*cap, (e+1)*cap) of recv.  Assignment (t,j)
+ * of expert e, the q-th of e in token order, goes to row e*cap + q when q < cap; otherwise
+ * it overflows and is dropped (perm[t,j] = -1).  Rows e*cap + [min(counts[e], cap), cap)
+ * are padding: zero rows in recv, src = -1.
+ *   x [T,d] bf16; idx [T,k] int32; counts [E] int32 (expert demand of idx, from
+ *   moe_histogram_maxvio); workspace int32[moe_dispatch_workspace_words(T, E)];
+ *   recv [E*cap, d] bf16 (out); perm [T,k] int32 (out); src [E*cap] int32 (out).
+ *   err  no-op when non-zero.
+ */
+int moe_dispatch_capacity(const moe_bf16* x, const int32_t* idx, const int32_t* counts, int T,
+                          int k, int E, int cap, int d, int32_t* workspace, moe_bf16* recv,
+                          int32_t* perm, int32_t* src, int32_t* err, moe_stream_t stream);
+/*
+ * moe_grouped_ffn_capacity: moe_grouped_ffn's SwiGLU expert over every row of every
+ * expert's block (padding rows included: zeros in, zeros out), expert e's home weights on
+ * rows [e*cap, (e+1)*cap).  recv [E*cap, d] bf16; W1, W3 [E,F,d] bf16; W2 [E,d,F] fp16;
+ * h [E*cap, F] fp16 (out); y [E*cap, d] bf16 (out); arithmetic and errors as
+ * moe_grouped_ffn.
+ */
+int moe_grouped_ffn_capacity(const moe_bf16* recv, const moe_bf16* W1, const moe_bf16* W3,
+                             const moe_f16* W2, int E, int cap, int d, int F, moe_f16* h,
+                             moe_bf16* y, int32_t* err, moe_stream_t stream);
+/*
+ * moe_combine_capacity: out[t] = sum over j with perm[t,j] >= 0 of gate[t,j] *
+ * y[perm[t,j]] (fp32, j order; bf16 out): a dropped assignment adds nothing, a token with
+ * every assignment dropped gets zeros.  Arguments as moe_combine.
+ */
+int moe_combine_capacity(const moe_bf16* y, const int32_t* perm, const float* gate, int T, int k,
+                         int d, moe_bf16* out, const int32_t* err, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
  * Combine.   [Primer] phase (d): expert outputs return to their token and are summed

@@ -26,7 +26,8 @@ DERR_NONFINITE, DERR_ID_RANGE, DERR_DUPLICATE, DERR_SLOTS, DERR_TIMEOUT = 1, 2, 
 
 ENTRY_POINTS = ("moe_topk", "moe_histogram_maxvio", "moe_plan_balanced", "moe_prefetch_replicas",
                 "moe_dispatch", "moe_grouped_ffn", "moe_combine")
-VARIANTS = ("moe_topk_biased", "moe_capacity_ledger")
+VARIANTS = ("moe_topk_biased", "moe_capacity_ledger", "moe_dispatch_capacity",
+            "moe_grouped_ffn_capacity", "moe_combine_capacity")
 FUSED = ("moe_dispatch_index", "moe_grouped_ffn_gather", "moe_route_plan")
 BACKWARD = ("moe_combine_backward", "moe_grouped_ffn_backward", "moe_dispatch_backward",
             "moe_topk_backward")
@@ -77,6 +78,9 @@ def lib() -> ctypes.CDLL:
             "moe_dispatch_backward": [P, P, I, I, I, P, P, P],
             "moe_topk_backward": [P, P, P, I, I, I, P, P, P],
             "moe_route_plan": [P, P, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P],
+            "moe_dispatch_capacity": [P, P, P, I, I, I, I, I, P, P, P, P, P, P],
+            "moe_grouped_ffn_capacity": [P, P, P, P, I, I, I, I, P, P, P, P],
+            "moe_combine_capacity": [P, P, P, I, I, I, P, P, P],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -86,6 +90,8 @@ def lib() -> ctypes.CDLL:
         L.moe_plan_get_layout.restype = ctypes.c_int
         L.moe_dispatch_workspace_words.argtypes = [I, I]
         L.moe_dispatch_workspace_words.restype = I64
+        L.moe_capacity_rows.argtypes = [I, I, I, I, I]
+        L.moe_capacity_rows.restype = I64
         L.moe_route_plan_workspace_words.argtypes = [I]
         L.moe_route_plan_workspace_words.restype = I64
         L.moe_ffn_backward_workspace_bytes.argtypes = [I, I, I, I, I, I, I]
@@ -239,12 +245,12 @@ def moe_dispatch(x, idx, plan, E, R, S, workspace, recv, perm, src, err, stream=
         _stream(stream)), "moe_dispatch")
 
 
-NOALLOC_SCRATCH_WORDS = 262144  # MOE_NOALLOC_SCRATCH_WORDS
+NOALLOC_SCRATCH_WORDS = 524288  # MOE_NOALLOC_SCRATCH_WORDS
 
 
 def moe_dispatch_noalloc(x, idx, plan, E, R, S, recv, perm, src, err, stream=None):
     """moe_dispatch without a workspace: for callers that cannot allocate device memory
-    when they dispatch; the library uses its own static 1 MiB scratch (see moe.h)."""
+    when they dispatch; the library uses its own static 2 MiB scratch (see moe.h)."""
     f = lib().moe_dispatch_noalloc
     if f.restype is not ctypes.c_int or f.argtypes is None:
         P, I = ctypes.c_void_p, ctypes.c_int
@@ -289,6 +295,91 @@ def moe_grouped_ffn_gather(x, src, plan, W1, W3, W2, P1, P3, P2, T, k, R, S, h, 
         _ptr(P3, bf, "P3"), _ptr(P2, hf, "P2"), T, k, E, R, S, d, F, _ptr(h, hf, "h"),
         _ptr(y, bf, "y"), _ptr(err, torch.int32, "err"), _stream(stream)),
         "moe_grouped_ffn_gather")
+
+
+# ----------------------------------------------------------------- fixed-capacity mode
+def capacity_rows(T: int, k: int, E: int, cf_num: int = 5, cf_den: int = 4) -> int:
+    """cap = ceil(T*k / E * cf_num / cf_den) rows per expert (moe_capacity_rows)."""
+    cap = int(lib().moe_capacity_rows(T, k, E, cf_num, cf_den))
+    if cap < 0:
+        raise MoEError("moe_capacity_rows: non-positive argument")
+    return cap
+
+
+def moe_dispatch_capacity(x, idx, counts, cap, workspace, recv, perm, src, err, stream=None):
+    """Each expert keeps its first cap assignments (token order) in rows [e*cap, (e+1)*cap);
+    the rest are dropped (perm -1); padding rows are zero with src -1."""
+    T, d = x.shape
+    k = idx.shape[1]
+    E = counts.shape[0]
+    _check(lib().moe_dispatch_capacity(
+        _ptr(x, torch.bfloat16, "x"), _ptr(idx, torch.int32, "idx"),
+        _ptr(counts, torch.int32, "counts"), T, k, E, cap, d,
+        _ptr(workspace, torch.int32, "workspace"), _ptr(recv, torch.bfloat16, "recv"),
+        _ptr(perm, torch.int32, "perm"), _ptr(src, torch.int32, "src"),
+        _ptr(err, torch.int32, "err"), _stream(stream)), "moe_dispatch_capacity")
+
+
+def moe_grouped_ffn_capacity(recv, W1, W3, W2, cap, h, y, err, stream=None):
+    E, F, d = W1.shape
+    bf, hf = torch.bfloat16, torch.float16
+    _check(lib().moe_grouped_ffn_capacity(
+        _ptr(recv, bf, "recv"), _ptr(W1, bf, "W1"), _ptr(W3, bf, "W3"), _ptr(W2, hf, "W2"), E, cap,
+        d, F, _ptr(h, hf, "h"), _ptr(y, bf, "y"), _ptr(err, torch.int32, "err"), _stream(stream)),
+        "moe_grouped_ffn_capacity")
+
+
+def moe_combine_capacity(y, perm, gate, out, err, stream=None):
+    T, k = perm.shape
+    d = out.shape[1]
+    _check(lib().moe_combine_capacity(
+        _ptr(y, torch.bfloat16, "y"), _ptr(perm, torch.int32, "perm"),
+        _ptr(gate, torch.float32, "gate"), T, k, d, _ptr(out, torch.bfloat16, "out"),
+        _ptr(err, torch.int32, "err"), _stream(stream)), "moe_combine_capacity")
+
+
+class CapacityLayer:
+    """The fixed-capacity (dropping) mode of one MoE layer: per-layer device buffers and the
+    calls in order -- moe_topk, moe_histogram_maxvio (raw demand, before any exclusion),
+    moe_capacity_ledger, moe_dispatch_capacity, moe_grouped_ffn_capacity,
+    moe_combine_capacity."""
+
+    def __init__(self, T, E, k, d, F, cf_num=5, cf_den=4, device="cuda"):
+        self.T, self.E, self.k, self.d, self.F = T, E, k, d, F
+        self.cf = (cf_num, cf_den)
+        self.cap = capacity_rows(T, k, E, cf_num, cf_den)
+        i32, dev = torch.int32, device
+        rows = E * self.cap
+        self.idx = torch.empty(T, k, dtype=i32, device=dev)
+        self.gate = torch.empty(T, k, dtype=torch.float32, device=dev)
+        self.counts = torch.empty(E, dtype=i32, device=dev)
+        self.loads = torch.empty(1, dtype=i32, device=dev)
+        self.maxvio = torch.empty(1, dtype=torch.float64, device=dev)
+        self.balancedness = torch.empty(1, dtype=torch.float64, device=dev)
+        self.processed = torch.empty(E, dtype=i32, device=dev)
+        self.overflow = torch.empty(E, dtype=i32, device=dev)
+        self.padding = torch.empty(E, dtype=i32, device=dev)
+        self.totals = torch.empty(4, dtype=i32, device=dev)
+        self.workspace = torch.empty(max(1, dispatch_workspace_words(T, E)), dtype=i32, device=dev)
+        self.recv = torch.empty(rows, d, dtype=torch.bfloat16, device=dev)
+        self.perm = torch.empty(T, k, dtype=i32, device=dev)
+        self.src = torch.empty(rows, dtype=i32, device=dev)
+        self.h = torch.empty(rows, F, dtype=torch.float16, device=dev)
+        self.y = torch.empty(rows, d, dtype=torch.bfloat16, device=dev)
+        self.out = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
+        self.err = torch.zeros(1, dtype=i32, device=dev)
+
+    def forward(self, logits, x, W1, W3, W2, stream=None):
+        moe_topk(logits, self.k, self.idx, self.gate, self.err, stream)
+        moe_histogram_maxvio(self.idx, self.E, 1, self.counts, self.loads, self.maxvio,
+                             self.balancedness, self.err, stream=stream)
+        moe_capacity_ledger(self.counts, self.T, self.k, self.cf[0], self.cf[1], self.processed,
+                            self.overflow, self.padding, self.totals, self.err, stream)
+        moe_dispatch_capacity(x, self.idx, self.counts, self.cap, self.workspace, self.recv,
+                              self.perm, self.src, self.err, stream)
+        moe_grouped_ffn_capacity(self.recv, W1, W3, W2, self.cap, self.h, self.y, self.err, stream)
+        moe_combine_capacity(self.y, self.perm, self.gate, self.out, self.err, stream)
+        return self.out
 
 
 def moe_combine(y, perm, gate, out, err, stream=None):
@@ -488,7 +579,7 @@ class MoELayer:
     def kernels_per_forward(self) -> int:
         n = 1                                 # routing + histogram + plan (fused)
         n += 1 if self.S > 0 else 0           # prefetch
-        n += (2 if self.fused else 3) if self.T > 0 else 0  # tile counts, ranks[, row scatter]
+        n += (1 if self.fused else 2) if self.T > 0 else 0  # ranks[, row scatter]
         n += 2 if self.T > 0 else 0           # two grouped GEMMs
         n += 1 if self.T > 0 else 0           # combine
         return n

@@ -65,7 +65,13 @@ int moe_plan_get_layout(int E, int R, int S, moe_plan_layout* out) {
 
 int64_t moe_dispatch_workspace_words(int T, int E) {
   if (T < 0 || E < 1) return 0;
-  return ((int64_t)T + moe::kPlaceTile - 1) / moe::kPlaceTile * E;
+  return moe::dispatch_workspace_words(T, E);
+}
+
+int64_t moe_capacity_rows(int T, int k, int E, int cf_num, int cf_den) {
+  if (T < 0 || k < 1 || E < 1 || cf_num < 1 || cf_den < 1) return -1;
+  const long long num = (long long)T * k * cf_num, den = (long long)E * cf_den;
+  return (num + den - 1) / den;
 }
 
 const char* moe_status_string(int status) {
@@ -256,6 +262,58 @@ int moe_grouped_ffn(const moe_bf16* recv, const int32_t* plan, const moe_bf16* W
       reinterpret_cast<const __nv_bfloat16*>(P3), reinterpret_cast<const __half*>(P2), T, k, E,
       R, S, d, F, reinterpret_cast<__half*>(h), reinterpret_cast<__nv_bfloat16*>(y), err,
       as_stream(stream));
+}
+
+int moe_dispatch_capacity(const moe_bf16* x, const int32_t* idx, const int32_t* counts, int T,
+                          int k, int E, int cap, int d, int32_t* workspace, moe_bf16* recv,
+                          int32_t* perm, int32_t* src, int32_t* err, moe_stream_t stream) {
+  if (!err || !counts || !recv || !src) return MOE_ERR_ARG;
+  if (T > 0 && (!x || !idx || !perm || !workspace)) return MOE_ERR_ARG;
+  if (cap < 0) return MOE_ERR_ARG;
+  MOE_TRY(check_route(T, E, k));
+  MOE_TRY(check_dims(T, k, d, 128));
+  const int64_t rows = (int64_t)E * cap;
+  if (rows * d >= kMaxElems) return MOE_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(recv)) return MOE_ERR_ARG;
+  return moe::launch_dispatch_capacity(reinterpret_cast<const __nv_bfloat16*>(x), idx, counts, T,
+                                       k, E, cap, d, workspace,
+                                       reinterpret_cast<__nv_bfloat16*>(recv), perm, src, err,
+                                       as_stream(stream));
+}
+
+int moe_grouped_ffn_capacity(const moe_bf16* recv, const moe_bf16* W1, const moe_bf16* W3,
+                             const moe_f16* W2, int E, int cap, int d, int F, moe_f16* h,
+                             moe_bf16* y, int32_t* err, moe_stream_t stream) {
+  if (!W1 || !W3 || !W2 || !err) return MOE_ERR_ARG;
+  if (cap > 0 && (!recv || !h || !y)) return MOE_ERR_ARG;
+  if (E < 1 || cap < 0) return MOE_ERR_ARG;
+  if (E > 1024) return MOE_ERR_SHAPE;
+  if (d < 1 || F < 1) return MOE_ERR_ARG;
+  if (d % 128 != 0 || F % 128 != 0) return MOE_ERR_SHAPE;
+  const int64_t rows = (int64_t)E * cap;
+  if (rows * d >= kMaxElems || rows * F >= kMaxElems) return MOE_ERR_SHAPE;
+  if ((int64_t)E * F >= kMaxElems || (int64_t)E * d >= kMaxElems) return MOE_ERR_SHAPE;
+  if (!aligned16(recv) || !aligned16(h) || !aligned16(y) || !aligned16(W1) || !aligned16(W3) ||
+      !aligned16(W2))
+    return MOE_ERR_ARG;
+  return moe::launch_grouped_ffn_capacity(
+      reinterpret_cast<const __nv_bfloat16*>(recv), reinterpret_cast<const __nv_bfloat16*>(W1),
+      reinterpret_cast<const __nv_bfloat16*>(W3), reinterpret_cast<const __half*>(W2), E, cap, d,
+      F, reinterpret_cast<__half*>(h), reinterpret_cast<__nv_bfloat16*>(y), err,
+      as_stream(stream));
+}
+
+int moe_combine_capacity(const moe_bf16* y, const int32_t* perm, const float* gate, int T, int k,
+                         int d, moe_bf16* out, const int32_t* err, moe_stream_t stream) {
+  if (!err) return MOE_ERR_ARG;
+  if (T > 0 && (!y || !perm || !gate || !out)) return MOE_ERR_ARG;
+  if (T < 0 || k < 1) return MOE_ERR_ARG;
+  if (k > 32) return MOE_ERR_SHAPE;
+  MOE_TRY(check_dims(T, k, d, 128));
+  if (!aligned16(y) || !aligned16(out)) return MOE_ERR_ARG;
+  return moe::launch_combine(reinterpret_cast<const __nv_bfloat16*>(y), perm, gate, T, k, d,
+                             reinterpret_cast<__nv_bfloat16*>(out), err, as_stream(stream),
+                             true);
 }
 
 int moe_combine(const moe_bf16* y, const int32_t* perm, const float* gate, int T, int k, int d,

@@ -82,13 +82,26 @@ int launch_grouped_ffn_backward(const __nv_bfloat16* recv, const __nv_bfloat16* 
                                 int F, __nv_bfloat16* dx_rows, float* dW1, float* dW3,
                                 float* dW2, void* workspace, int64_t workspace_bytes,
                                 int32_t* err, cudaStream_t s);
+// drop: assignments with perm < 0 (fixed-capacity overflow) are left out of the sum
 int launch_combine(const __nv_bfloat16* y, const int32_t* perm, const float* gate, int T,
-                   int k, int d, __nv_bfloat16* out, const int32_t* err, cudaStream_t s);
+                   int k, int d, __nv_bfloat16* out, const int32_t* err, cudaStream_t s,
+                   bool drop = false);
 
 // launch_dispatch with recv == nullptr computes perm and src only (no row copy).
-
-// Tokens per tile of the placement kernels (workspace = ceil(T/kPlaceTile) * E words).
-constexpr int kPlaceTile = 256;
+// Workspace words of the dispatch's rank pass (tile statuses and per-tile expert counts).
+int64_t dispatch_workspace_words(int T, int E);
+// Fixed-capacity placement: expert e's q-th assignment (token order) at row e*cap + q when
+// q < cap, else dropped (perm -1); padding rows of each expert zeroed in recv, src -1.
+int launch_dispatch_capacity(const __nv_bfloat16* x, const int32_t* idx, const int32_t* counts,
+                             int T, int k, int E, int cap, int d, int32_t* ws,
+                             __nv_bfloat16* recv, int32_t* perm, int32_t* src, int32_t* err,
+                             cudaStream_t s);
+// The grouped FFN over E uniform groups of cap rows (group e = rows [e*cap, (e+1)*cap),
+// expert e, home weights): the fixed-capacity layout.
+int launch_grouped_ffn_capacity(const __nv_bfloat16* recv, const __nv_bfloat16* W1,
+                                const __nv_bfloat16* W3, const __half* W2, int E, int cap,
+                                int d, int F, __half* h, __nv_bfloat16* y, int32_t* err,
+                                cudaStream_t s);
 
 // ----------------------------------------------------------------------------- device side
 // Reads the layer's error word once per thread; every kernel after moe_topk returns

@@ -68,6 +68,7 @@ constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 struct FfnArgs {
   const int4* groups;   // [G] {row_start, rows, expert, weight_ref}, rows == -1 unused
   int G;
+  int uniform_rows;     // > 0: no table; group g = {g*uniform_rows, uniform_rows, g, g}
   int n_blocks_n;       // output column blocks per row block
   int k_blocks;         // K / BK
   int bn_out;           // output columns per tile (128 for SwiGLU, N for plain)
@@ -231,6 +232,13 @@ __device__ __forceinline__ uint32_t pack_f16_sat(float a, float b) {
 }
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + __expf(-z)); }
 
+// Group g: from the plan's table, or (fixed-capacity layout) expert g's block of
+// uniform_rows rows with its home weights.
+__device__ __forceinline__ int4 group_of(const FfnArgs& a, int g) {
+  if (a.uniform_rows > 0) return make_int4(g * a.uniform_rows, a.uniform_rows, g, g);
+  return __ldg(a.groups + g);
+}
+
 struct Tile {
   int a_row;       // first row of the A block
   int valid_rows;  // rows of the block inside the group (<= BM)
@@ -249,7 +257,7 @@ __device__ __forceinline__ Tile decode_tile(int t, const FfnArgs& a, const int* 
     const int mid = (lo + hi + 1) >> 1;
     if (s_prefix[mid] <= mt) lo = mid; else hi = mid - 1;
   }
-  const int4 g = __ldg(a.groups + lo);
+  const int4 g = group_of(a, lo);
   const int m_local = mt - s_prefix[lo];
   tl.a_row = g.x + m_local * BM;
   tl.valid_rows = min(BM, g.y - m_local * BM);
@@ -287,7 +295,7 @@ __global__ void __launch_bounds__(FFN_THREADS, 1)
 
   // m-blocks per group, exclusive prefix over the group table
   for (int g = tid; g < args.G; g += blockDim.x) {
-    const int rows = __ldg(&args.groups[g].y);
+    const int rows = group_of(args, g).y;
     s_prefix[g] = rows > 0 ? (rows + BM - 1) / BM : 0;
   }
   __syncthreads();
@@ -649,7 +657,7 @@ __device__ __forceinline__ Tile decode_pair_tile(int t, const FfnArgs& a, const 
     const int mid = (lo + hi + 1) >> 1;
     if (s_prefix[mid] <= mt) lo = mid; else hi = mid - 1;
   }
-  const int4 g = __ldg(a.groups + lo);
+  const int4 g = group_of(a, lo);
   const int first = (mt - s_prefix[lo]) * P_BM + rank * BM;  // row offset inside the group
   tl.a_row = g.x + first;
   tl.valid_rows = max(0, min(BM, g.y - first));
@@ -704,7 +712,7 @@ __global__ void __launch_bounds__(FFN_THREADS, 1)
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   for (int g = tid; g < args.G; g += blockDim.x) {
-    const int rows = __ldg(&args.groups[g].y);
+    const int rows = group_of(args, g).y;
     s_prefix[g] = rows > 0 ? (rows + P_BM - 1) / P_BM : 0;
   }
   __syncthreads();
@@ -1019,17 +1027,18 @@ int ffn_pair_clusters() {
   return dev < 64 ? g_pair_clusters[dev] : 0;
 }
 
-// GEMM 1 reads its rows from recv (x == nullptr) or gathers them as x[src[row]].
+// GEMM 1 reads its rows from recv (x == nullptr) or gathers them as x[src[row]].  The
+// groups come from `groups` (G entries) or, with uniform_rows > 0, are E blocks of
+// uniform_rows rows; `rows` is the length of recv, h and y.
 int launch_grouped_ffn_impl(const __nv_bfloat16* recv, const __nv_bfloat16* x,
-                            const int32_t* src, const int32_t* plan, const moe_plan_layout& L,
-                            const __nv_bfloat16* W1, const __nv_bfloat16* W3, const __half* W2,
-                            const __nv_bfloat16* P1, const __nv_bfloat16* P3, const __half* P2,
-                            int T, int k, int E, int R, int S, int d, int F, __half* h,
-                            __nv_bfloat16* y, int32_t* err, cudaStream_t s) {
-  if (T == 0) return MOE_OK;
+                            const int32_t* src, const int4* groups, int G, int uniform_rows,
+                            int64_t rows, const __nv_bfloat16* W1, const __nv_bfloat16* W3,
+                            const __half* W2, const __nv_bfloat16* P1, const __nv_bfloat16* P3,
+                            const __half* P2, int T, int E, int R, int S, int d, int F,
+                            __half* h, __nv_bfloat16* y, int32_t* err, cudaStream_t s) {
+  if (rows == 0) return MOE_OK;
   const bool gather = x != nullptr;
   const bool pair = !gather && g_ffn_tile_mode.load(std::memory_order_relaxed) == 1;
-  const int64_t rows = (int64_t)T * k;  // R * C
   const int bn2 = (d % 256 == 0) ? 256 : 128;
   const int w2_box = pair ? bn2 / 2 : bn2;  // a pair CTA loads half of GEMM 2's B rows
   CUtensorMap m_recv, m_w1, m_w3, m_p1, m_p3, m_h, m_w2, m_p2;
@@ -1050,8 +1059,9 @@ int launch_grouped_ffn_impl(const __nv_bfloat16* recv, const __nv_bfloat16* x,
     m_p2 = m_w2;
   }
   FfnArgs a1;
-  a1.groups = reinterpret_cast<const int4*>(plan + L.groups);
-  a1.G = R * L.max_groups_per_rank;
+  a1.groups = groups;
+  a1.G = G;
+  a1.uniform_rows = uniform_rows;
   a1.n_blocks_n = F / 128;
   a1.k_blocks = d / BK;
   a1.bn_out = 128;
@@ -1089,8 +1099,10 @@ int launch_grouped_ffn(const __nv_bfloat16* recv, const int32_t* plan,
                        const __nv_bfloat16* P3, const __half* P2, int T, int k, int E, int R,
                        int S, int d, int F, __half* h, __nv_bfloat16* y, int32_t* err,
                        cudaStream_t s) {
-  return launch_grouped_ffn_impl(recv, nullptr, nullptr, plan, L, W1, W3, W2, P1, P3, P2, T, k,
-                                 E, R, S, d, F, h, y, err, s);
+  return launch_grouped_ffn_impl(recv, nullptr, nullptr,
+                                 reinterpret_cast<const int4*>(plan + L.groups),
+                                 R * L.max_groups_per_rank, 0, (int64_t)T * k, W1, W3, W2, P1,
+                                 P3, P2, T, E, R, S, d, F, h, y, err, s);
 }
 
 int launch_grouped_ffn_gather(const __nv_bfloat16* x, const int32_t* src, const int32_t* plan,
@@ -1099,8 +1111,19 @@ int launch_grouped_ffn_gather(const __nv_bfloat16* x, const int32_t* src, const 
                               const __nv_bfloat16* P1, const __nv_bfloat16* P3,
                               const __half* P2, int T, int k, int E, int R, int S, int d, int F,
                               __half* h, __nv_bfloat16* y, int32_t* err, cudaStream_t s) {
-  return launch_grouped_ffn_impl(nullptr, x, src, plan, L, W1, W3, W2, P1, P3, P2, T, k, E, R,
-                                 S, d, F, h, y, err, s);
+  return launch_grouped_ffn_impl(nullptr, x, src, reinterpret_cast<const int4*>(plan + L.groups),
+                                 R * L.max_groups_per_rank, 0, (int64_t)T * k, W1, W3, W2, P1,
+                                 P3, P2, T, E, R, S, d, F, h, y, err, s);
+}
+
+int launch_grouped_ffn_capacity(const __nv_bfloat16* recv, const __nv_bfloat16* W1,
+                                const __nv_bfloat16* W3, const __half* W2, int E, int cap,
+                                int d, int F, __half* h, __nv_bfloat16* y, int32_t* err,
+                                cudaStream_t s) {
+  if (cap == 0) return MOE_OK;
+  return launch_grouped_ffn_impl(recv, nullptr, nullptr, nullptr, E, cap, (int64_t)E * cap, W1,
+                                 W3, W2, nullptr, nullptr, nullptr, 0, E, 1, 0, d, F, h, y, err,
+                                 s);
 }
 
 }  // namespace moe

@@ -51,154 +51,7 @@ __global__ void __launch_bounds__(kCopyThreads) prefetch_kernel(
   }
 }
 
-// ----------------------------------------------------------------------------- placement
-// Pass 1: per-tile expert counts ws[tile*E + e] (every entry written).
-__global__ void __launch_bounds__(kPlaceTile) tile_count_kernel(const int32_t* __restrict__ idx,
-                                                                int T, int k, int E,
-                                                                int32_t* __restrict__ ws,
-                                                                int32_t* __restrict__ err) {
-  extern __shared__ int s_cnt[];
-  __shared__ int s_bad;
-  if (block_should_stop(err)) return;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) s_cnt[e] = 0;
-  if (threadIdx.x == 0) s_bad = 0;
-  __syncthreads();
-  const int64_t t = (int64_t)blockIdx.x * kPlaceTile + threadIdx.x;
-  const int lane = threadIdx.x & 31;
-  for (int j = 0; j < k; ++j) {
-    int e = t < T ? __ldg(idx + t * k + j) : -1;
-    if (t < T && (e < 0 || e >= E)) {
-      s_bad = 1;
-      e = -1;
-    }
-    const uint32_t peers = __match_any_sync(MOE_FULL_MASK, e);
-    if (e >= 0 && lane == __ffs(peers) - 1) atomicAdd(&s_cnt[e], __popc(peers));
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) ws[(int64_t)blockIdx.x * E + e] = s_cnt[e];
-  if (threadIdx.x == 0 && s_bad) atomicOr(err, MOE_DERR_ID_RANGE);
-}
-
-// Pass 2: the token-order rank q of every assignment within its expert, then its row.
-//   q = (assignments of e in earlier tiles) + (in earlier warps of this tile)
-//     + (in earlier lanes of this warp);
-// the last term comes from a per-warp lane mask of each expert (a token names an expert
-// at most once, so one bit per lane suffices).
-__global__ void __launch_bounds__(kPlaceTile) tile_rank_kernel(
-    const int32_t* __restrict__ idx, int T, int k, int E, int R, int C,
-    const int32_t* __restrict__ ws, const int32_t* __restrict__ plan, moe_plan_layout L,
-    int32_t* __restrict__ perm, int32_t* __restrict__ src, int32_t* __restrict__ err) {
-  constexpr int W = kPlaceTile / 32;
-  extern __shared__ int smem[];
-  uint32_t* s_mask = reinterpret_cast<uint32_t*>(smem);  // [W][E]
-  int* s_pre = smem + W * E;                              // [W][E] start of each warp
-  int* s_rp = s_pre + W * E;                              // [R+1] room prefix
-  int* s_kr = s_rp + R + 1;                               // [R] kept rows
-  int* s_home = s_kr + R;                                 // [E] home offset (-1 streamed)
-  int* s_so = s_home + E;                                 // [E] stream offset
-  __shared__ int s_bad;
-  if (block_should_stop(err)) return;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int tile = blockIdx.x;
-  for (int i = tid; i < W * E; i += blockDim.x) s_mask[i] = 0;
-  for (int r = tid; r <= R; r += blockDim.x) s_rp[r] = plan[L.room_prefix + r];
-  for (int r = tid; r < R; r += blockDim.x) s_kr[r] = plan[L.kept_rows + r];
-  for (int e = tid; e < E; e += blockDim.x) {
-    s_home[e] = plan[L.expert_home_off + e];
-    s_so[e] = plan[L.stream_off + e];
-  }
-  if (tid == 0) s_bad = 0;
-  __syncthreads();
-  const int64_t t = (int64_t)tile * kPlaceTile + tid;
-  const bool tok = t < T;
-  for (int j = 0; j < k; ++j) {
-    if (!tok) break;
-    const int e = __ldg(idx + t * k + j);
-    if (e >= 0 && e < E) atomicOr(&s_mask[warp * E + e], 1u << lane);
-  }
-  __syncthreads();
-  for (int e = tid; e < E; e += blockDim.x) {
-    // assignments of e in all earlier tiles: independent partial sums keep the loads of
-    // the column in flight together
-    int r0 = 0, r1 = 0, r2 = 0, r3 = 0, p = 0;
-    for (; p + 4 <= tile; p += 4) {
-      r0 += __ldg(ws + (int64_t)p * E + e);
-      r1 += __ldg(ws + (int64_t)(p + 1) * E + e);
-      r2 += __ldg(ws + (int64_t)(p + 2) * E + e);
-      r3 += __ldg(ws + (int64_t)(p + 3) * E + e);
-    }
-    for (; p < tile; ++p) r0 += __ldg(ws + (int64_t)p * E + e);
-    int run = r0 + r1 + r2 + r3;
-    for (int w = 0; w < W; ++w) {
-      s_pre[w * E + e] = run;
-      run += __popc(s_mask[w * E + e]);
-    }
-  }
-  __syncthreads();
-  if (tok) {
-    const uint32_t lt = lanemask_lt();
-    const int64_t rows_total = (int64_t)R * C;
-    const int B = E / R;
-    for (int j = 0; j < k; ++j) {
-      const int e = __ldg(idx + t * k + j);
-      if (e < 0 || e >= E) { s_bad = 1; continue; }
-      const int q = s_pre[warp * E + e] + __popc(s_mask[warp * E + e] & lt);
-      const int off = s_home[e];
-      int64_t row;
-      if (off >= 0) {
-        row = (int64_t)(e / B) * C + off + q;
-      } else {
-        const int p = s_so[e] + q;
-        int a = 0, b = R - 1;  // last rank with room_prefix <= p
-        while (a < b) {
-          const int m = (a + b + 1) >> 1;
-          if (s_rp[m] <= p) a = m; else b = m - 1;
-        }
-        row = (int64_t)a * C + s_kr[a] + (p - s_rp[a]);
-      }
-      if (row < 0 || row >= rows_total) { s_bad = 1; continue; }
-      perm[t * k + j] = (int32_t)row;
-      src[row] = (int32_t)t;
-    }
-  }
-  __syncthreads();
-  if (tid == 0 && s_bad) atomicOr(err, MOE_DERR_ID_RANGE);
-}
-
-// Pass 3: every token row is read once (16-byte vectors) and stored to its k rows.
 constexpr int kRowThreads = 256;
-constexpr int kRowVec = 4;
-
-__global__ void __launch_bounds__(kRowThreads) scatter_rows_kernel(
-    const uint4* __restrict__ x, const int32_t* __restrict__ perm, int T, int k, int dv,
-    int64_t rows_total, uint4* __restrict__ recv, const int32_t* __restrict__ err) {
-  if (load_err(err)) return;
-  const int lane = threadIdx.x & 31;
-  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += nwarps) {
-    int r = lane < k ? __ldg(perm + t * k + lane) : 0;
-    if (r < 0 || r >= rows_total) r = -1;  // never stored
-    const uint4* xs = x + t * dv;
-    for (int v0 = 0; v0 < dv; v0 += 32 * kRowVec) {
-      uint4 buf[kRowVec];
-#pragma unroll
-      for (int u = 0; u < kRowVec; ++u) {
-        const int v = v0 + u * 32 + lane;
-        if (v < dv) buf[u] = __ldcs(xs + v);
-      }
-      for (int j = 0; j < k; ++j) {
-        const int row = __shfl_sync(MOE_FULL_MASK, r, j);
-        if (row < 0) continue;
-        uint4* dst = recv + (int64_t)row * dv;
-#pragma unroll
-        for (int u = 0; u < kRowVec; ++u) {
-          const int v = v0 + u * 32 + lane;
-          if (v < dv) dst[v] = buf[u];
-        }
-      }
-    }
-  }
-}
 
 // ----------------------------------------------------------------------------- combine
 
@@ -225,7 +78,9 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float* a) {
 // first FMA; K == 0 is the generic loop.  V (16-byte vectors per lane and gather) is 1
 // for K > 4 so that the kernel stays near 40 registers and enough warps are resident
 // to keep the gathers in flight.
-template <int K, int kCombVec = (K > 4 || K == 0) ? 1 : 2>
+// DROP: an assignment with perm < 0 (dropped by the fixed-capacity dispatch) is left out
+// of the sum.
+template <int K, bool DROP = false, int kCombVec = (K > 4 || K == 0) ? 1 : 2>
 __global__ void __launch_bounds__(kRowThreads) combine_kernel(
     const uint4* __restrict__ y, const int32_t* __restrict__ perm,
     const float* __restrict__ gate, int T, int k, int dv, uint4* __restrict__ out,
@@ -257,12 +112,13 @@ __global__ void __launch_bounds__(kRowThreads) combine_kernel(
         for (int j = 0; j < K; ++j)
 #pragma unroll
           for (int u = 0; u < kCombVec; ++u)
-            if (v0 + u * 32 < dv) buf[j][u] = __ldcs(y + (int64_t)rows[j] * dv + v0 + u * 32);
+            if (v0 + u * 32 < dv && (!DROP || rows[j] >= 0))
+              buf[j][u] = __ldcs(y + (int64_t)rows[j] * dv + v0 + u * 32);
 #pragma unroll
         for (int j = 0; j < K; ++j)
 #pragma unroll
           for (int u = 0; u < kCombVec; ++u)
-            if (v0 + u * 32 < dv) acc_bf16x8(acc[u], buf[j][u], g[j]);
+            if (v0 + u * 32 < dv && (!DROP || rows[j] >= 0)) acc_bf16x8(acc[u], buf[j][u], g[j]);
 #pragma unroll
         for (int u = 0; u < kCombVec; ++u)
           if (v0 + u * 32 < dv) out[t * dv + v0 + u * 32] = pack_bf16x8(acc[u]);
@@ -277,7 +133,7 @@ __global__ void __launch_bounds__(kRowThreads) combine_kernel(
         for (int j = 0; j < k; ++j) {
           const int row = __shfl_sync(MOE_FULL_MASK, r, j);
           const float gj = __shfl_sync(MOE_FULL_MASK, gl, j);
-          if (v < dv) acc_bf16x8(acc, __ldcs(y + (int64_t)row * dv + v), gj);
+          if (v < dv && (!DROP || row >= 0)) acc_bf16x8(acc, __ldcs(y + (int64_t)row * dv + v), gj);
         }
         if (v < dv) out[t * dv + v] = pack_bf16x8(acc);
       }
@@ -308,35 +164,26 @@ int launch_prefetch(const int32_t* plan, const moe_plan_layout& L, const __nv_bf
   return launch_status();
 }
 
-int launch_dispatch(const __nv_bfloat16* x, const int32_t* idx, const int32_t* plan,
-                    const moe_plan_layout& L, int T, int k, int E, int R, int d,
-                    int32_t* ws, __nv_bfloat16* recv, int32_t* perm, int32_t* src,
-                    int32_t* err, cudaStream_t s) {
-  if (T == 0) return MOE_OK;
-  const int C = (int)(((int64_t)T * k) / R);
-  const int tiles = (T + kPlaceTile - 1) / kPlaceTile;
-  tile_count_kernel<<<tiles, kPlaceTile, sizeof(int) * E, s>>>(idx, T, k, E, ws, err);
-  if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
-  const size_t smem = sizeof(int) * (2 * (kPlaceTile / 32) * (size_t)E + 2 * (size_t)R + 1 + 2 * (size_t)E);
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(tile_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
-    return MOE_ERR_LAUNCH;
-  tile_rank_kernel<<<tiles, kPlaceTile, smem, s>>>(idx, T, k, E, R, C, ws, plan, L, perm, src, err);
-  if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
-  if (recv == nullptr) return MOE_OK;  // index-only: the FFN gathers the rows itself
-  scatter_rows_kernel<<<row_grid(T), kRowThreads, 0, s>>>(
-      reinterpret_cast<const uint4*>(x), perm, T, k, d / 8, (int64_t)R * C,
-      reinterpret_cast<uint4*>(recv), err);
-  return launch_status();
-}
-
 int launch_combine(const __nv_bfloat16* y, const int32_t* perm, const float* gate, int T,
-                   int k, int d, __nv_bfloat16* out, const int32_t* err, cudaStream_t s) {
+                   int k, int d, __nv_bfloat16* out, const int32_t* err, cudaStream_t s,
+                   bool drop) {
   if (T == 0) return MOE_OK;
   const uint4* yv = reinterpret_cast<const uint4*>(y);
   uint4* ov = reinterpret_cast<uint4*>(out);
   const int g = row_grid(T), dv = d / 8;
+  if (drop) {
+#define MOE_COMBINE_DROP(KK) combine_kernel<KK, true><<<g, kRowThreads, 0, s>>>(yv, perm, gate, T, k, dv, ov, err)
+    switch (k) {
+      case 1: MOE_COMBINE_DROP(1); break;
+      case 2: MOE_COMBINE_DROP(2); break;
+      case 4: MOE_COMBINE_DROP(4); break;
+      case 6: MOE_COMBINE_DROP(6); break;
+      case 8: MOE_COMBINE_DROP(8); break;
+      default: MOE_COMBINE_DROP(0); break;
+    }
+#undef MOE_COMBINE_DROP
+    return launch_status();
+  }
 #define MOE_COMBINE_CASE(KK) combine_kernel<KK><<<g, kRowThreads, 0, s>>>(yv, perm, gate, T, k, dv, ov, err)
   switch (k) {
     case 1: MOE_COMBINE_CASE(1); break;

@@ -50,8 +50,16 @@ def test_plan_layout_is_consistent(lib):
     assert L.n_groups == L.replica_list + 1 + R * S
     assert L.groups % 4 == 0 and L.groups >= L.n_groups + R
     assert L.words == L.groups + R * (B + S) * 4
-    assert M.dispatch_workspace_words(16384, 256) == 64 * 256
-    assert M.dispatch_workspace_words(257, 8) == 2 * 8
+    # per 256-token tile: a status word, its expert counts and its inclusive prefix, after
+    # four header words (the status block padded to a multiple of 4 words)
+    assert M.dispatch_workspace_words(16384, 256) == 68 + 2 * 64 * 256
+    assert M.dispatch_workspace_words(257, 8) == 8 + 2 * 2 * 8
+    assert M.dispatch_workspace_words(0, 8) == 4
+    # the fixed-capacity rows: ceil(A / E * cf), the pages' fixture gives 5
+    assert M.capacity_rows(16, 2, 8, 5, 4) == 5
+    assert M.capacity_rows(16384, 8, 256, 1, 1) == 512
+    assert M.capacity_rows(16384, 8, 256, 5, 4) == 640
+    assert M.capacity_rows(0, 8, 256, 5, 4) == 0
 
 
 def test_host_checks_reject_bad_arguments(lib):

@@ -272,6 +272,18 @@ def test_bounded_wait_gives_up_and_context_survives():
     check_ffn_combine_full(L, w, x, weights, ref)
 
 
+def test_many_tile_dispatch():
+    """98304 tokens = 384 placement tiles of 256: the rank pass looks back over a dozen
+    windows of 32 predecessor tiles; perm, src and the received rows stay bit-exact."""
+    w = I.small_workload("tiles", 98304, 64, 4, 8, 8, 128, 128, alpha=0.5, seed=14)
+    logits, x, weights = make_inputs(w)
+    ref = oracle_integer_path(w, logits)
+    assert ref["err"] == 0
+    L = run_gpu(w, logits, x, weights)
+    check_integer_parity(L, w, ref)
+    check_rows_and_pool(L, w, x, weights, ref)
+
+
 def test_max_shapes():
     """Limits of the boundary: E = 1024 experts, k = 32, R = 1024 ranks (B = 1), S = 3 slots
     (R*(B+S) = 4096 group records), through the whole layer."""

@@ -74,8 +74,9 @@ def test_noalloc_matches_dispatch_two_calls(lib):
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(lib):
     fake = ctypes.c_void_p(4096)  # never dereferenced: the size check fails first
-    T, E = 2 * 65536, 1024
+    T, E = 65536, 1024
     assert M.dispatch_workspace_words(T, E) > M.NOALLOC_SCRATCH_WORDS
     st = lib.moe_dispatch_noalloc(fake, fake, fake, T, 8, E, 8, 4, 128, fake, fake, fake, fake, None)
     assert st == M.MOE_ERR_SHAPE
-    assert M.dispatch_workspace_words(65536, 1024) <= M.NOALLOC_SCRATCH_WORDS
+    assert M.dispatch_workspace_words(65536, 512) <= M.NOALLOC_SCRATCH_WORDS
+    assert M.dispatch_workspace_words(32768, 1024) <= M.NOALLOC_SCRATCH_WORDS
