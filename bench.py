@@ -515,6 +515,85 @@ def run_ours(args, w: I.Workload, world, rank, local):
     return res
 
 
+def run_only(args, w: I.Workload):
+    """One call of the path on its own, repeated `--steps` times between CUDA events after
+    `--warmup` calls: the case for kernel-level counter captures (ncu), which must stay a
+    few GB on the device.  Prints one JSON line with the per-call time and rate; it is not
+    the benchmark line."""
+    import load_balanced_dispatch_warp_b200 as M
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    peaks, _ = load_peaks()
+    res = {"only": args.only, "workload": w.name, "steps": args.steps}
+    if args.only == "topk":
+        res.update(topk_floor(w, device, reps=args.steps))
+        print(json.dumps(res, sort_keys=True), flush=True)
+        return
+    stream = torch.cuda.current_stream(device)
+    i32 = torch.int32
+    logits = I.make_logits(w).to(device)
+    x = I.make_x(w).to(device)
+    lay = M.plan_layout(w.E, w.R, w.S)
+    idx = torch.empty(w.T, w.k, dtype=i32, device=device)
+    gate = torch.empty(w.T, w.k, dtype=torch.float32, device=device)
+    counts = torch.empty(w.E, dtype=i32, device=device)
+    loads = torch.empty(w.R, dtype=i32, device=device)
+    mv = torch.empty(1, dtype=torch.float64, device=device)
+    bal = torch.empty(1, dtype=torch.float64, device=device)
+    plan = torch.empty(lay.words, dtype=i32, device=device)
+    rpw = torch.empty(M.route_plan_workspace_words(w.E), dtype=i32, device=device)
+    err = torch.zeros(1, dtype=i32, device=device)
+    ws = torch.empty(max(1, M.dispatch_workspace_words(w.T, w.E)), dtype=i32, device=device)
+    perm = torch.empty(w.T, w.k, dtype=i32, device=device)
+    src = torch.empty(w.A, dtype=i32, device=device)
+    recv = torch.empty(w.A, w.d, dtype=torch.bfloat16, device=device)
+
+    def route():
+        M.moe_route_plan(logits, w.k, w.R, w.S, idx, gate, counts, loads, mv, bal, plan, rpw, err)
+
+    def dispatch():
+        M.moe_dispatch(x, idx, plan, w.E, w.R, w.S, ws, recv, perm, src, err)
+
+    route()
+    dispatch()
+    units = algorithmic(w, 0)
+    if args.only == "route":
+        fn, unit, work = route, *units["moe_route_plan"]
+    elif args.only == "dispatch":
+        fn, unit, work = dispatch, *units["moe_dispatch"]
+    elif args.only == "combine":
+        y = recv.clone()
+        out = torch.empty(w.T, w.d, dtype=torch.bfloat16, device=device)
+        fn, unit, work = (lambda: M.moe_combine(y, perm, gate, out, err)), *units["moe_combine"]
+    else:  # ffn
+        W1, W3, W2 = I.make_weights(w, device=device)
+        P = [torch.empty(w.R * w.S, *t.shape[1:], dtype=t.dtype, device=device) for t in (W1, W3, W2)]
+        M.moe_prefetch_replicas(plan, W1, W3, W2, w.R, w.S, *P, err)
+        h = torch.empty(w.A, w.F, dtype=torch.float16, device=device)
+        y = torch.empty(w.A, w.d, dtype=torch.bfloat16, device=device)
+        fn = lambda: M.moe_grouped_ffn(recv, plan, W1, W3, W2, *P, w.T, w.k, w.R, w.S, h, y, err)
+        unit, work = units["moe_grouped_ffn"]
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error word {int(err.item())}")
+    us = a.elapsed_time(b) / args.steps * 1e3
+    rate = work / (us * 1e-6) / (1e12 if unit == "TFLOP/s" else 1e9)
+    peak = peaks["bf16_tflops"] if unit == "TFLOP/s" else peaks["hbm_gbs"]
+    res.update({"us": round(us, 2), unit.replace("/", "_per_"): round(rate, 1),
+                "frac": round(rate / peak, 3),
+                "peak": "burst bf16 GEMM" if unit == "TFLOP/s" else "copy"})
+    print(json.dumps(res, sort_keys=True), flush=True)
+
+
 # Qwen-shaped skew sweep carried beside the headline (tokens/s vs maxvio)
 SWEEP = ["qwen_mv0.2", "qwen_mv1", "qwen_mv5", "qwen_mv15"]
 
@@ -710,6 +789,9 @@ def main():
                     help="steps per point of the Qwen-shaped maxvio sweep")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the stand-alone top-k floor and the maxvio sweep")
+    ap.add_argument("--only", default=None, choices=["topk", "route", "dispatch", "combine", "ffn"],
+                    help="time one call alone (--steps launches after --warmup) and print its "
+                         "rate instead of the benchmark line: the small case for counter captures")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="launch the timed steps eagerly")
@@ -723,6 +805,9 @@ def main():
     args = ap.parse_args()
     w = I.WORKLOADS[args.config]
 
+    if args.only is not None:
+        run_only(args, w)
+        return
     if args.impl == "reference":
         res = run_reference(args, w)
         if res is not None:

@@ -376,8 +376,9 @@ __global__ void __launch_bounds__(kScatterThreads) scatter_kernel(ScatterArgs a)
       for (int v = u + 1; v < issued; ++v)
         mbar_wait_bounded(smem_addr(&s_bar[v % a.nbuf]), (uint32_t)((v / a.nbuf) & 1));
     }
-  } else if (a.counts != nullptr) {
-    // fixed-capacity padding: experts blockIdx.x, blockIdx.x + gridDim.x, ... ; warps 1..7
+  } else if (tid >= 32 && a.counts != nullptr) {
+    // fixed-capacity padding, by warps 1..7 (wt in [0, blockDim.x - 32)): experts
+    // blockIdx.x, blockIdx.x + gridDim.x, ...; rows e*cap + [min(count, cap), cap)
     const int vec_per_row = a.row_bytes / 16;
     const int wt = tid - 32, nwt = blockDim.x - 32;
     for (int e = blockIdx.x; e < a.E; e += gridDim.x) {

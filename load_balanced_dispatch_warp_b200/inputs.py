@@ -79,6 +79,11 @@ WORKLOADS: dict[str, Workload] = {w.name: w for w in [
              note="coarse experts, 1 expert/rank, S=3 (inference)"),
     Workload("deepseek", 16384, 256, 8, 32, 4, 7168, 2048, "hot", 0.90,
              note="26 hot experts take 90% of assignments, S=4 (inference)"),
+    # the DeepSeek-shaped expert (d = 7168, F = 2048, top-8) with tokens and experts cut so
+    # that the whole layer holds under 3 GB on the device: the case for detailed counter
+    # captures of the grouped FFN, which must stay small
+    Workload("deepseek_small", 2048, 16, 8, 2, 4, 7168, 2048, "zipf", float("nan"),
+             fixed_param=0.5, note="DeepSeek-shaped expert, 2048 tokens, 16 experts"),
 ]}
 
 # Sweep order of the Qwen-shaped skew sweep.
