@@ -524,7 +524,10 @@ def run_only(args, w: I.Workload):
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
     peaks, _ = load_peaks()
-    res = {"only": args.only, "workload": w.name, "steps": args.steps}
+    if args.ffn_tile is not None:
+        M.set_ffn_tile_mode(args.ffn_tile)
+    res = {"only": args.only, "workload": w.name, "steps": args.steps,
+           "ffn_tile": int(M.lib().moe_ffn_tile_mode())}
     if args.only == "topk":
         res.update(topk_floor(w, device, reps=args.steps))
         print(json.dumps(res, sort_keys=True), flush=True)

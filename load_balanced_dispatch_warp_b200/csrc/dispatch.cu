@@ -111,10 +111,18 @@ __global__ void __launch_bounds__(kRankTile) rank_kernel(RankArgs a) {
   const int64_t t = (int64_t)tile * kRankTile + tid;
   const bool tok = t < a.T;
   int my_err = 0;
-  for (int j = 0; tok && j < a.k; ++j) {
-    const int e = __ldg(a.idx + t * a.k + j);
-    if (e < 0 || e >= E) my_err |= MOE_DERR_ID_RANGE;
-    else atomicOr(&s_mask[warp * E + e], 1u << lane);
+  // one lane per distinct expert of the warp ORs in the lanes naming it (a token names an
+  // expert at most once, so one bit per lane per expert); no shared-memory atomics even
+  // when the warp's tokens share hot experts
+  for (int j = 0; j < a.k; ++j) {
+    int e = tok ? __ldg(a.idx + t * a.k + j) : -1;
+    if (tok && (e < 0 || e >= E)) {
+      my_err |= MOE_DERR_ID_RANGE;
+      e = -1;
+    }
+    const uint32_t peers = __match_any_sync(MOE_FULL_MASK, e);
+    if (e >= 0 && lane == __ffs(peers) - 1) s_mask[warp * E + e] |= peers;
+    __syncwarp();
   }
   __syncthreads();
   // counts of this tile; publish them (status 1), or for tile 0 the inclusive prefix

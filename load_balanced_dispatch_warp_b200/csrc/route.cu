@@ -146,13 +146,29 @@ __device__ __noinline__ void topk_exact(const float* x, const float* b, int E, i
 // experts' unbiased logits in fp32.  K > 0 fixes k at compile time (K == k).
 // Token t by the calling warp.  Returns false (err flagged, nothing written) on a
 // non-finite logit or bias.  COUNT: each written id is also added to counts[id].
-template <int VPL, int K, bool BIASED, bool COUNT>
-__device__ __forceinline__ bool topk_token(const float* __restrict__ logits,
-                                           const float* __restrict__ bias, int64_t t, int E,
-                                           int k, int lane, uint32_t* s_key, int* s_id,
-                                           float* s_raw, int32_t* __restrict__ idx,
-                                           float* __restrict__ gate, int32_t* __restrict__ counts,
-                                           int32_t* __restrict__ err) {
+// Lane's share of token t's logits: x[i] = logits[t, lane + 32 i] (0 past E).
+template <int VPL, bool FULL>
+__device__ __forceinline__ void load_row(const float* __restrict__ logits, int64_t t, int E,
+                                         int lane, float (&x)[VPL]) {
+  const float* row = logits + t * E;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int e = lane + 32 * i;
+    x[i] = (FULL || e < E) ? __ldcs(row + e) : 0.f;
+  }
+}
+
+// The selection for token t from the lane's share x of its logits (load_row).  FULL: E is
+// exactly 32 * VPL, so no lane holds a slot past the last expert.
+template <int VPL, int K, bool BIASED, bool COUNT, bool FULL = false>
+__device__ __forceinline__ bool topk_token_loaded(const float (&x)[VPL],
+                                                  const float* __restrict__ bias, int64_t t,
+                                                  int E, int k, int lane, uint32_t* s_key,
+                                                  int* s_id, float* s_raw,
+                                                  int32_t* __restrict__ idx,
+                                                  float* __restrict__ gate,
+                                                  int32_t* __restrict__ counts,
+                                                  int32_t* __restrict__ err) {
   float b[VPL];
 #pragma unroll
   for (int i = 0; i < VPL; ++i) b[i] = 0.f;
@@ -169,20 +185,13 @@ __device__ __forceinline__ bool topk_token(const float* __restrict__ logits,
       return false;
     }
   }
-  const float* row = logits + t * E;
-  float x[VPL];
-#pragma unroll
-  for (int i = 0; i < VPL; ++i) {
-    const int e = lane + 32 * i;
-    x[i] = e < E ? __ldcs(row + e) : 0.f;
-  }
   // non-finite check: x * 0 is +-0 for finite x and NaN otherwise
   float key[VPL];
   float z = 0.f;
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
     z = __fmaf_rn(x[i], 0.f, z);
-    key[i] = lane + 32 * i < E ? (BIASED ? __fadd_rn(x[i], b[i]) : x[i]) : -INFINITY;
+    key[i] = (FULL || lane + 32 * i < E) ? (BIASED ? __fadd_rn(x[i], b[i]) : x[i]) : -INFINITY;
   }
   if (__any_sync(MOE_FULL_MASK, !(z == 0.f))) {
     if (lane == 0) atomicOr(err, MOE_DERR_NONFINITE);
@@ -235,15 +244,15 @@ __device__ __forceinline__ bool topk_token(const float* __restrict__ logits,
         BIASED ? warp_max_f32(npop > 0 ? fmaxf(v1, npop > 1 ? v2 : -INFINITY) : -INFINITY) : w0;
     const float e1 = npop > 0 ? expf(v1 - top) : 0.f;
     const float e2 = npop > 1 ? expf(v2 - top) : 0.f;
-    const float sum = warp_sum(e1 + e2);
+    const float inv = 1.f / warp_sum(e1 + e2);
     if (npop > 0) {
       idx[t * k + r1] = lane + 32 * s1;
-      gate[t * k + r1] = e1 / sum;
+      gate[t * k + r1] = e1 * inv;
       if (COUNT) atomicAdd(counts + lane + 32 * s1, 1);
     }
     if (npop > 1) {
       idx[t * k + r2] = lane + 32 * s2;
-      gate[t * k + r2] = e2 / sum;
+      gate[t * k + r2] = e2 * inv;
       if (COUNT) atomicAdd(counts + lane + 32 * s2, 1);
     }
     return true;
@@ -264,7 +273,20 @@ __device__ __forceinline__ bool topk_token(const float* __restrict__ logits,
   return true;
 }
 
-template <int VPL, int K, bool BIASED>
+template <int VPL, int K, bool BIASED, bool COUNT, bool FULL = false>
+__device__ __forceinline__ bool topk_token(const float* __restrict__ logits,
+                                           const float* __restrict__ bias, int64_t t, int E,
+                                           int k, int lane, uint32_t* s_key, int* s_id,
+                                           float* s_raw, int32_t* __restrict__ idx,
+                                           float* __restrict__ gate, int32_t* __restrict__ counts,
+                                           int32_t* __restrict__ err) {
+  float x[VPL];
+  load_row<VPL, FULL>(logits, t, E, lane, x);
+  return topk_token_loaded<VPL, K, BIASED, COUNT, FULL>(x, bias, t, E, k, lane, s_key, s_id,
+                                                        s_raw, idx, gate, counts, err);
+}
+
+template <int VPL, int K, bool BIASED, bool FULL = false>
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits,
                                                    const float* __restrict__ bias, int T,
                                                    int E, int k_rt, int32_t* __restrict__ idx,
@@ -277,8 +299,8 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int64_t t = (int64_t)blockIdx.x * 8 + wib;
   if (t >= T) return;
-  topk_token<VPL, K, BIASED, false>(logits, bias, t, E, k, lane, s_key[wib], s_id[wib],
-                                    s_raw[wib], idx, gate, nullptr, err);
+  topk_token<VPL, K, BIASED, false, FULL>(logits, bias, t, E, k, lane, s_key[wib], s_id[wib],
+                                          s_raw[wib], idx, gate, nullptr, err);
 }
 
 // Fixed-capacity ledger of "MoE Load Balancing: Find Expert Hotspots" ("Make expert
@@ -461,6 +483,8 @@ __global__ void __launch_bounds__(512) hist_kernel(const int32_t* __restrict__ i
 
 // One warp per token, 8 warps per block.  Unbiased calls with k in {2, 4, 6, 8} and up to
 // 256 experts run a kernel with k fixed at compile time (the rounds unroll).
+// One warp per token, 8 warps per block.  Unbiased calls with k in {2, 4, 6, 8} and up to
+// 256 experts run a kernel with k fixed at compile time (the rounds unroll).
 template <int VPL>
 void launch_topk_vpl(const float* logits, const float* bias, int T, int E, int k, int32_t* idx,
                      float* gate, int32_t* err, cudaStream_t s) {
@@ -471,6 +495,17 @@ void launch_topk_vpl(const float* logits, const float* bias, int T, int E, int k
     return;
   }
   if constexpr (VPL <= 8) {
+    if (E == 32 * VPL) {
+#define MOE_TOPK_FULL(KK) topk_kernel<VPL, KK, false, true><<<grid, 256, 0, s>>>(logits, bias, T, E, k, idx, gate, err)
+      switch (k) {
+        case 8: MOE_TOPK_FULL(8); return;
+        case 6: MOE_TOPK_FULL(6); return;
+        case 4: MOE_TOPK_FULL(4); return;
+        case 2: MOE_TOPK_FULL(2); return;
+        default: break;
+      }
+#undef MOE_TOPK_FULL
+    }
     switch (k) {
       case 8: MOE_TOPK(8, false); return;
       case 6: MOE_TOPK(6, false); return;
@@ -506,7 +541,7 @@ int launch_topk_impl(const float* logits, const float* bias, int T, int E, int k
 // rest untouched.
 constexpr int kCountCopies = 16;
 
-template <int VPL, int K, bool BIASED>
+template <int VPL, int K, bool BIASED, bool FULL = false>
 __global__ void __launch_bounds__(kPlanThreads) route_plan_kernel(
     const float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int k_rt,
     int R, int S, int32_t* __restrict__ idx, float* __restrict__ gate,
@@ -527,8 +562,8 @@ __global__ void __launch_bounds__(kPlanThreads) route_plan_kernel(
   __syncthreads();
   const int64_t t = (int64_t)blockIdx.x * 8 + wib;
   if (t < T)
-    topk_token<VPL, K, BIASED, true>(logits, bias, t, E, k, lane, s_key[wib], s_id[wib],
-                                     s_raw[wib], idx, gate, s_dyn, err);
+    topk_token<VPL, K, BIASED, true, FULL>(logits, bias, t, E, k, lane, s_key[wib], s_id[wib],
+                                           s_raw[wib], idx, gate, s_dyn, err);
   __syncthreads();
   int32_t* copy = ws + (int64_t)(blockIdx.x % kCountCopies) * E;
   for (int e = threadIdx.x; e < E; e += blockDim.x)
@@ -574,6 +609,19 @@ void launch_route_plan_vpl(const float* logits, const float* bias, int T, int E,
     return;
   }
   if constexpr (VPL <= 8) {
+    if (E == 32 * VPL) {
+#define MOE_RP_FULL(KK)                                                                         \
+  route_plan_kernel<VPL, KK, false, true><<<grid, kPlanThreads, smem, s>>>(                        \
+      logits, bias, T, E, k, R, S, idx, gate, counts, loads, maxvio, bal, plan, L, ws, err)
+      switch (k) {
+        case 8: MOE_RP_FULL(8); return;
+        case 6: MOE_RP_FULL(6); return;
+        case 4: MOE_RP_FULL(4); return;
+        case 2: MOE_RP_FULL(2); return;
+        default: break;
+      }
+#undef MOE_RP_FULL
+    }
     switch (k) {
       case 8: MOE_RP(8, false); return;
       case 6: MOE_RP(6, false); return;

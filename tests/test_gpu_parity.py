@@ -254,6 +254,33 @@ def test_topk_expert_counts(E):
     assert np.abs(gate.cpu().double().numpy() - gate_ref).max() <= 1e-6
 
 
+@pytest.mark.parametrize("E,k", [(256, 8), (64, 6), (128, 8), (8, 2)])
+def test_topk_many_tokens_staged_rows(E, k):
+    """From 1024 tokens up (E a multiple of 4) the stand-alone top-k stages its rows through
+    shared memory in blocks of 16 with bulk copies: the DeepSeek workload's logits, then
+    T = 20001 (the last block has one token) of random logits with every fifth row made of
+    ties (the exact path)."""
+    if E == 256:
+        w = I.WORKLOADS["deepseek"]
+        logits = I.make_logits(w)
+    else:
+        g = torch.Generator().manual_seed(E + k)
+        logits = torch.randn(20001, E, generator=g)
+        vals = torch.tensor([-1.0, -0.0, 0.0, 0.5, 2.0])
+        tie = vals[torch.randint(0, 5, (4001, E), generator=g)]
+        logits[::5] = tie
+    T = logits.shape[0]
+    idx_ref, gate_ref, err = O.topk_route(logits.numpy(), k)
+    idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    gate = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    e = torch.zeros(1, dtype=torch.int32, device="cuda")
+    M.moe_topk(logits.cuda(), k, idx, gate, e)
+    torch.cuda.synchronize()
+    assert e.item() == 0
+    assert np.array_equal(idx.cpu().numpy(), idx_ref)
+    assert np.abs(gate.cpu().double().numpy() - gate_ref).max() <= 1e-6
+
+
 def test_bounded_wait_gives_up_and_context_survives():
     """The FFN's bounded mbarrier wait, on a barrier nothing arrives at, returns with the
     timeout bit; the next layer on the same context still matches the oracle."""
