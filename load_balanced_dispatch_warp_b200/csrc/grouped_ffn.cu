@@ -69,6 +69,7 @@ struct FfnArgs {
   const int4* groups;   // [G] {row_start, rows, expert, weight_ref}, rows == -1 unused
   int G;
   int uniform_rows;     // > 0: no table; group g = {g*uniform_rows, uniform_rows, g, g}
+  int half_tiles;       // 1: a tile with at most 64 valid rows runs M = 64 MMAs
   int n_blocks_n;       // output column blocks per row block
   int k_blocks;         // K / BK
   int bn_out;           // output columns per tile (128 for SwiGLU, N for plain)
@@ -242,6 +243,8 @@ __device__ __forceinline__ int4 group_of(const FfnArgs& a, int g) {
 struct Tile {
   int a_row;       // first row of the A block
   int valid_rows;  // rows of the block inside the group (<= BM)
+  bool half;       // M = 64 tile: 64-row A box, M = 64 MMAs, accumulator rows 16 per lane
+                   // quadrant (row r in TMEM lane 32 (r / 16) + r % 16, measured)
   int b_row;       // first row of the B block inside its tensor
   bool pool;       // B from the replica pool instead of the home tensors
   int n_block;
@@ -261,6 +264,7 @@ __device__ __forceinline__ Tile decode_tile(int t, const FfnArgs& a, const int* 
   const int m_local = mt - s_prefix[lo];
   tl.a_row = g.x + m_local * BM;
   tl.valid_rows = min(BM, g.y - m_local * BM);
+  tl.half = a.half_tiles && tl.valid_rows <= BM / 2;
   const int ref = g.w;
   tl.pool = ref >= a.E;
   tl.b_row = (tl.pool ? ref - a.E : ref) * a.rows_per_expert + tl.n_block * a.bn_out;
@@ -269,9 +273,10 @@ __device__ __forceinline__ Tile decode_tile(int t, const FfnArgs& a, const int* 
 
 template <bool SWIGLU, bool GATHER>
 __global__ void __launch_bounds__(FFN_THREADS, 1)
-    ffn_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b0,
-               const __grid_constant__ CUtensorMap tm_b1, const __grid_constant__ CUtensorMap tm_p0,
-               const __grid_constant__ CUtensorMap tm_p1, const FfnArgs args) {
+    ffn_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a64,
+               const __grid_constant__ CUtensorMap tm_b0, const __grid_constant__ CUtensorMap tm_b1,
+               const __grid_constant__ CUtensorMap tm_p0, const __grid_constant__ CUtensorMap tm_p1,
+               const FfnArgs args) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the swizzle atoms
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -424,8 +429,8 @@ __global__ void __launch_bounds__(FFN_THREADS, 1)
           const uint32_t fb = full0 + 8 * stage;
           const uint32_t sa = smem_u32(stage_base + stage * STAGE_BYTES);
           const uint32_t sb = sa + A_BYTES;
-          mbar_expect_tx(fb, A_BYTES + b_bytes);
-          tma_load_2d(sa, &tm_a, fb, kb * BK, tl.a_row);
+          mbar_expect_tx(fb, (tl.half ? A_BYTES / 2 : A_BYTES) + b_bytes);
+          tma_load_2d(sa, tl.half ? &tm_a64 : &tm_a, fb, kb * BK, tl.a_row);
           if (SWIGLU) {
             tma_load_2d(sb, mb0, fb, kb * BK, tl.b_row);
             tma_load_2d(sb + (b_bytes >> 1), mb1, fb, kb * BK, tl.b_row);
@@ -450,12 +455,14 @@ __global__ void __launch_bounds__(FFN_THREADS, 1)
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       // GEMM 1: x, W1, W3 in bf16; GEMM 2: h and W2 in fp16
-      const uint32_t idesc = make_idesc(BM, args.mma_n, SWIGLU);
+      const uint32_t idesc_full = make_idesc(BM, args.mma_n, SWIGLU);
+      const uint32_t idesc_half = make_idesc(BM / 2, args.mma_n, SWIGLU);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+        const uint32_t idesc = decode_tile(t, args, s_prefix).half ? idesc_half : idesc_full;
         if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag, args.err)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
@@ -495,9 +502,11 @@ __global__ void __launch_bounds__(FFN_THREADS, 1)
       if (!__all_sync(MOE_FULL_MASK, ok)) break;  // warp-uniform exit
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * ACC_COLS;
-      const bool valid = r_in < tl.valid_rows;
+      // an M = 64 tile holds its row 16 q + i in lane i < 16 of quadrant q
+      const int row = tl.half ? quarter * 16 + lane : r_in;
+      const bool valid = (!tl.half || lane < 16) && row < tl.valid_rows;
       // both outputs are 16-bit: h (fp16) after GEMM 1, y (bf16) after GEMM 2
-      uint16_t* orow = static_cast<uint16_t*>(args.out) + (int64_t)(tl.a_row + r_in) * args.out_ld +
+      uint16_t* orow = static_cast<uint16_t*>(args.out) + (int64_t)(tl.a_row + row) * args.out_ld +
                        (int64_t)tl.n_block * args.bn_out;
       if (SWIGLU) {
 #pragma unroll 1
@@ -661,6 +670,7 @@ __device__ __forceinline__ Tile decode_pair_tile(int t, const FfnArgs& a, const 
   const int first = (mt - s_prefix[lo]) * P_BM + rank * BM;  // row offset inside the group
   tl.a_row = g.x + first;
   tl.valid_rows = max(0, min(BM, g.y - first));
+  tl.half = false;
   const int ref = g.w;
   tl.pool = ref >= a.E;
   tl.b_row = (tl.pool ? ref - a.E : ref) * a.rows_per_expert + tl.n_block * a.bn_out +
@@ -938,8 +948,9 @@ size_t ffn_smem_bytes() {
 }
 
 template <bool SWIGLU, bool GATHER>
-int launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-               const CUtensorMap& p0, const CUtensorMap& p1, const FfnArgs& args, cudaStream_t s) {
+int launch_one(const CUtensorMap& a, const CUtensorMap& a64, const CUtensorMap& b0,
+               const CUtensorMap& b1, const CUtensorMap& p0, const CUtensorMap& p1,
+               const FfnArgs& args, cudaStream_t s) {
   static bool configured[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -950,7 +961,7 @@ int launch_one(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b
       return MOE_ERR_LAUNCH;
     configured[dev] = true;
   }
-  ffn_kernel<SWIGLU, GATHER><<<num_sms(), FFN_THREADS, smem, s>>>(a, b0, b1, p0, p1, args);
+  ffn_kernel<SWIGLU, GATHER><<<num_sms(), FFN_THREADS, smem, s>>>(a, a64, b0, b1, p0, p1, args);
   return launch_status();
 }
 
@@ -1041,11 +1052,13 @@ int launch_grouped_ffn_impl(const __nv_bfloat16* recv, const __nv_bfloat16* x,
   const bool pair = !gather && g_ffn_tile_mode.load(std::memory_order_relaxed) == 1;
   const int bn2 = (d % 256 == 0) ? 256 : 128;
   const int w2_box = pair ? bn2 / 2 : bn2;  // a pair CTA loads half of GEMM 2's B rows
-  CUtensorMap m_recv, m_w1, m_w3, m_p1, m_p3, m_h, m_w2, m_p2;
+  CUtensorMap m_recv, m_recv64, m_w1, m_w3, m_p1, m_p3, m_h, m_h64, m_w2, m_p2;
   if (!make_map(&m_w1, W1, (int64_t)E * F, d, 128) ||
       (!gather && !make_map(&m_recv, recv, rows, d, BM)) ||
+      (!gather && !make_map(&m_recv64, recv, rows, d, BM / 2)) ||
       !make_map(&m_w3, W3, (int64_t)E * F, d, 128) ||
       !make_map(&m_h, h, rows, F, BM, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+      !make_map(&m_h64, h, rows, F, BM / 2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
       !make_map(&m_w2, W2, (int64_t)E * d, F, w2_box, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
     return MOE_ERR_DEVICE;
   if (S > 0) {
@@ -1062,6 +1075,7 @@ int launch_grouped_ffn_impl(const __nv_bfloat16* recv, const __nv_bfloat16* x,
   a1.groups = groups;
   a1.G = G;
   a1.uniform_rows = uniform_rows;
+  a1.half_tiles = (gather || pair) ? 0 : 1;  // the gathering producer always fills 128 rows
   a1.n_blocks_n = F / 128;
   a1.k_blocks = d / BK;
   a1.bn_out = 128;
@@ -1075,9 +1089,9 @@ int launch_grouped_ffn_impl(const __nv_bfloat16* recv, const __nv_bfloat16* x,
   a1.gsrc = src;
   a1.gd = d;
   a1.gT = T;
-  int st = gather ? launch_one<true, true>(m_w1, m_w1, m_w3, m_p1, m_p3, a1, s)
+  int st = gather ? launch_one<true, true>(m_w1, m_w1, m_w1, m_w3, m_p1, m_p3, a1, s)
            : pair ? launch_pair<true>(m_recv, m_w1, m_w3, m_p1, m_p3, a1, s)
-                  : launch_one<true, false>(m_recv, m_w1, m_w3, m_p1, m_p3, a1, s);
+                  : launch_one<true, false>(m_recv, m_recv64, m_w1, m_w3, m_p1, m_p3, a1, s);
   if (st != MOE_OK) return st;
   FfnArgs a2 = a1;
   a2.n_blocks_n = d / bn2;
@@ -1089,8 +1103,9 @@ int launch_grouped_ffn_impl(const __nv_bfloat16* recv, const __nv_bfloat16* x,
   a2.out = y;
   a2.gx = nullptr;
   a2.gsrc = nullptr;
+  a2.half_tiles = pair ? 0 : 1;
   return pair ? launch_pair<false>(m_h, m_w2, m_w2, m_p2, m_p2, a2, s)
-              : launch_one<false, false>(m_h, m_w2, m_w2, m_p2, m_p2, a2, s);
+              : launch_one<false, false>(m_h, m_h64, m_w2, m_w2, m_p2, m_p2, a2, s);
 }
 
 int launch_grouped_ffn(const __nv_bfloat16* recv, const int32_t* plan,
