@@ -135,10 +135,20 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- work units
-def algorithmic(w: I.Workload, n_rep: int, fused: bool = False):
+def algorithmic(w: I.Workload, n_rep: int, fused: bool = False, fused_combine: bool = False):
     """Algorithmic bytes (HBM) or flops per call for one step.  Fused: the dispatch call
-    only reads idx and writes perm and src; the FFN reads the token rows itself."""
+    only reads idx and writes perm and src; the FFN reads the token rows itself.  Fused
+    combine: the FFN call also does the combine (its rate is still quoted on 6*A*d*F), the
+    combine call does nothing."""
     T, E, k, d, F, A = w.T, w.E, w.k, w.d, w.F, w.A
+    if fused_combine:
+        return {
+            "moe_route_plan": ("GB/s", T * E * 4 + A * 8),
+            "moe_prefetch_replicas": ("GB/s", 2 * n_rep * 3 * d * F * 2),
+            "moe_dispatch": ("GB/s", T * d * 2 + A * d * 2 + 12 * A),
+            "moe_grouped_ffn": ("TFLOP/s", 6 * A * d * F),
+            "moe_combine": ("GB/s", None),
+        }
     return {
         # top-k reads the logits and writes idx and gate; the histogram and the plan
         # (fused into the same launch) add only E-sized traffic
@@ -234,7 +244,8 @@ def measure_layer(args, w: I.Workload, world, device, steps: int, e2e: bool):
     logits = logits_h.to(device)
     x = x_h.to(device)
     W1, W3, W2 = I.make_weights(w, device=device)
-    L = M.MoELayer(w.T, w.E, w.k, w.R, w.S, w.d, w.F, device=device, fused=args.fused)
+    L = M.MoELayer(w.T, w.E, w.k, w.R, w.S, w.d, w.F, device=device, fused=args.fused,
+                   fused_combine=args.fused_combine)
     # the per-call table: the forward's calls one after the other (event nodes between them)
     calls = [lambda: L.route_plan(logits), lambda: L.prefetch(W1, W3, W2),
              lambda: L.dispatch(x), lambda: L.expert_ffn(W1, W3, W2), lambda: L.combine()]
@@ -344,10 +355,11 @@ def measure_layer(args, w: I.Workload, world, device, steps: int, e2e: bool):
     return out
 
 
-def call_table(w: I.Workload, m: dict, peaks: dict, fused: bool, tflops_peak: float):
+def call_table(w: I.Workload, m: dict, peaks: dict, fused: bool, tflops_peak: float,
+               fused_combine: bool = False):
     """Per-call rates: algorithmic work over the in-graph interval, as a fraction of the
     measured copy peak (HBM-bound calls) or of the clock-matched bf16 peak (the FFN)."""
-    units = algorithmic(w, m["n_rep"], fused)
+    units = algorithmic(w, m["n_rep"], fused, fused_combine)
     calls = {}
     for c in CALLS:
         unit, work = units[c]
@@ -411,11 +423,12 @@ def topk_floor(w: I.Workload, device, reps: int = 200, copies: int = 16):
                     f"torch copy_ moving the same bytes (read + write), same rotation"}
 
 
-def summarize(w: I.Workload, m: dict, peaks: dict, peak_src: str, fused: bool, steps: int):
+def summarize(w: I.Workload, m: dict, peaks: dict, peak_src: str, fused: bool, steps: int,
+              fused_combine: bool = False):
     """Compact record of one workload: tokens/s, the per-call table, the FFN against the
     clock-matched peak, and the FFN's duration in SM cycles at the median clock."""
     tpk, tpk_src = ffn_peak(m["clocks"], peaks, peak_src)
-    calls = call_table(w, m, peaks, fused, tpk)
+    calls = call_table(w, m, peaks, fused, tpk, fused_combine)
     ffn_us = m["per_call_ms"]["moe_grouped_ffn"] * 1e3
     sm = m["clocks"].get("sm_mhz")
     return {"value": round(w.T * steps / (m["elapsed_ms"] * 1e-3), 1),
@@ -437,8 +450,8 @@ def run_ours(args, w: I.Workload, world, rank, local):
 
     m = measure_layer(args, w, world, device, args.steps, e2e=True)
     L = m["layer"]
-    head = summarize(w, m, peaks, peak_src, args.fused, args.steps)
-    units = algorithmic(w, m["n_rep"], args.fused)
+    head = summarize(w, m, peaks, peak_src, args.fused, args.steps, args.fused_combine)
+    units = algorithmic(w, m["n_rep"], args.fused, args.fused_combine)
     ffn_ms = m["per_call_ms"]["moe_grouped_ffn"]
     ffn_flops = units["moe_grouped_ffn"][1]
     achieved = ffn_flops / (ffn_ms * 1e-3) / 1e12
@@ -473,6 +486,8 @@ def run_ours(args, w: I.Workload, world, rank, local):
                    "parallelism": f"replicas x{world} (ranks simulated in one GPU's HBM)",
                    "dispatch": ("fused: placement only, GEMM 1 gathers x[src[row]]" if args.fused
                                 else "row copy into recv, GEMM 1 reads recv"),
+                   "combine": ("fused into GEMM 2's epilogue (fp32 atomics, then bf16)"
+                               if args.fused_combine else "separate gather kernel, j-ordered"),
                    "ffn_tile": ("256-row tiles on 2-CTA clusters (tcgen05 cta_group::2)"
                                 if ffn_tile == 1 and not args.fused
                                 else "128-row tiles, one CTA each (tcgen05 cta_group::1)"),
@@ -505,7 +520,8 @@ def run_ours(args, w: I.Workload, world, rank, local):
         for name in SWEEP:
             ws = I.WORKLOADS[name]
             ms = measure_layer(args, ws, world, device, args.sweep_steps, e2e=False)
-            sweep[name] = summarize(ws, ms, peaks, peak_src, args.fused, args.sweep_steps)
+            sweep[name] = summarize(ws, ms, peaks, peak_src, args.fused, args.sweep_steps,
+                                    args.fused_combine)
             del ms
             torch.cuda.empty_cache()
         res["maxvio_sweep"] = {"workloads": sweep, "steps": args.sweep_steps,
@@ -802,6 +818,9 @@ def main():
                     help="also time the training step (forward + backward) and the backward calls")
     ap.add_argument("--fused", action="store_true",
                     help="fused dispatch: placement only, GEMM 1 gathers the token rows")
+    ap.add_argument("--fused-combine", action="store_true",
+                    help="fused combine: GEMM 2's epilogue adds the gate-weighted rows into an "
+                         "fp32 output (atomics), no y buffer and no combine kernel")
     ap.add_argument("--ffn-tile", type=int, default=None, choices=[0, 1],
                     help="grouped-FFN tiling: 0 = 128-row tiles, one CTA each; 1 = 256-row "
                          "tiles on 2-CTA clusters (default: the library's)")

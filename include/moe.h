@@ -302,6 +302,30 @@ int moe_grouped_ffn_gather(const moe_bf16* x, const int32_t* src, const int32_t*
                            int32_t* err, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * Fused combine: the gate-weighted sum folded into GEMM 2's epilogue.   [Primer], the
+ * third of the ideas it credits to DeepEP (the combine reduction fused into dedicated GPU
+ * kernels), and phase (d): the expert outputs return to their token, summed with the gate
+ * weights.  moe_grouped_ffn_combine computes moe_grouped_ffn followed by moe_combine
+ * without writing y: GEMM 2's epilogue adds gate[t,j] * (h W2^T)_row, in fp32 straight from
+ * the tensor-core accumulator, into out32[t] for the token t = src[row] and the choice j
+ * with perm[t,j] == row (16-byte fp32 atomics), then out = bf16(out32).  The k
+ * contributions of a token arrive in no fixed order, so out may differ from moe_combine's
+ * j-ordered sum in the last bits (it also skips y's rounding to bf16); both are within the
+ * combine's tolerance of the fp64 result.
+ *   src [R*C], perm [T,k], gate [T,k] from moe_dispatch and the router; an src entry
+ *   outside [0, T) sets MOE_DERR_ID_RANGE (that row is left out).
+ *   out32 [T,d] fp32: caller-owned scratch, zeroed by the call.  out [T,d] bf16 (out).
+ *   Other arguments, arithmetic and errors as moe_grouped_ffn (128-row tiles; the
+ *   2-CTA tile mode does not apply).
+ */
+int moe_grouped_ffn_combine(const moe_bf16* recv, const int32_t* plan, const moe_bf16* W1,
+                            const moe_bf16* W3, const moe_f16* W2, const moe_bf16* P1,
+                            const moe_bf16* P3, const moe_f16* P2, const int32_t* src,
+                            const int32_t* perm, const float* gate, int T, int k, int E, int R,
+                            int S, int d, int F, moe_f16* h, float* out32, moe_bf16* out,
+                            int32_t* err, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
  * Backward pass.   [MoonEP] para. 3: the duplicated experts' gradients are reduced back
  * home during the backward pass.  The pages give no formulas; these calls apply the
  * chain rule to the forward above, reading top-k selection as passing no gradient to the

@@ -28,7 +28,8 @@ ENTRY_POINTS = ("moe_topk", "moe_histogram_maxvio", "moe_plan_balanced", "moe_pr
                 "moe_dispatch", "moe_grouped_ffn", "moe_combine")
 VARIANTS = ("moe_topk_biased", "moe_capacity_ledger", "moe_dispatch_capacity",
             "moe_grouped_ffn_capacity", "moe_combine_capacity")
-FUSED = ("moe_dispatch_index", "moe_grouped_ffn_gather", "moe_route_plan")
+FUSED = ("moe_dispatch_index", "moe_grouped_ffn_gather", "moe_route_plan",
+         "moe_grouped_ffn_combine")
 BACKWARD = ("moe_combine_backward", "moe_grouped_ffn_backward", "moe_dispatch_backward",
             "moe_topk_backward")
 HELPERS = ("moe_plan_get_layout", "moe_dispatch_workspace_words", "moe_status_string",
@@ -79,6 +80,8 @@ def lib() -> ctypes.CDLL:
             "moe_topk_backward": [P, P, P, I, I, I, P, P, P],
             "moe_route_plan": [P, P, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P],
             "moe_dispatch_capacity": [P, P, P, I, I, I, I, I, P, P, P, P, P, P],
+            "moe_grouped_ffn_combine": [P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P,
+                                        P, P, P, P],
             "moe_grouped_ffn_capacity": [P, P, P, P, I, I, I, I, P, P, P, P],
             "moe_combine_capacity": [P, P, P, I, I, I, P, P, P],
         }
@@ -382,6 +385,22 @@ class CapacityLayer:
         return self.out
 
 
+def moe_grouped_ffn_combine(recv, plan, W1, W3, W2, P1, P3, P2, src, perm, gate, R, S, h, out32,
+                            out, err, stream=None):
+    """moe_grouped_ffn + moe_combine with the gate-weighted sum in GEMM 2's epilogue (fp32
+    atomics into the scratch out32 [T,d], then bf16 into out): no y buffer, no combine
+    kernel."""
+    E, F, d = W1.shape
+    T, k = perm.shape
+    bf, hf, i32 = torch.bfloat16, torch.float16, torch.int32
+    _check(lib().moe_grouped_ffn_combine(
+        _ptr(recv, bf, "recv"), _ptr(plan, i32, "plan"), _ptr(W1, bf, "W1"), _ptr(W3, bf, "W3"),
+        _ptr(W2, hf, "W2"), _ptr(P1, bf, "P1"), _ptr(P3, bf, "P3"), _ptr(P2, hf, "P2"),
+        _ptr(src, i32, "src"), _ptr(perm, i32, "perm"), _ptr(gate, torch.float32, "gate"), T, k,
+        E, R, S, d, F, _ptr(h, hf, "h"), _ptr(out32, torch.float32, "out32"), _ptr(out, bf, "out"),
+        _ptr(err, i32, "err"), _stream(stream)), "moe_grouped_ffn_combine")
+
+
 def moe_combine(y, perm, gate, out, err, stream=None):
     T, k = perm.shape
     d = out.shape[1]
@@ -446,11 +465,18 @@ class MoELayer:
     The replica pool (P1, P3, P2: R*S slots) is allocated once here; several layers may
     share one pool by passing ``pool=`` (it is process-global in the MoonEP design).
     ``fused=True``: no recv buffer; the FFN gathers the rows of the ``x`` last dispatched.
+    ``fused_combine=True``: no y buffer; GEMM 2's epilogue adds the gate-weighted rows into
+    an fp32 [T,d] scratch (``out32``), converted to ``out`` in the same call
+    (``moe_grouped_ffn_combine``); ``combine()`` then has nothing left to do.
     """
 
-    def __init__(self, T, E, k, R, S, d, F, device="cuda", pool=None, fused=False):
+    def __init__(self, T, E, k, R, S, d, F, device="cuda", pool=None, fused=False,
+                 fused_combine=False):
         self.T, self.E, self.k, self.R, self.S, self.d, self.F = T, E, k, R, S, d, F
         self.fused = bool(fused)
+        self.fused_combine = bool(fused_combine)
+        if self.fused and self.fused_combine:
+            raise ValueError("fused (gathering GEMM 1) and fused_combine are separate options")
         self._x = None
         self.A = T * k
         self.C = self.A // R
@@ -471,7 +497,8 @@ class MoELayer:
         self.perm = torch.empty(T, k, dtype=i32, device=dev)
         self.src = torch.empty(self.A, dtype=i32, device=dev)
         self.h = torch.empty(self.A, F, dtype=torch.float16, device=dev)
-        self.y = torch.empty(self.A, d, dtype=bf, device=dev)
+        self.y = None if self.fused_combine else torch.empty(self.A, d, dtype=bf, device=dev)
+        self.out32 = torch.empty(T, d, dtype=f32, device=dev) if self.fused_combine else None
         self.out = torch.empty(T, d, dtype=bf, device=dev)
         if pool is None and S > 0:
             pool = (torch.empty(R * S, F, d, dtype=bf, device=dev),
@@ -516,7 +543,11 @@ class MoELayer:
 
     def expert_ffn(self, W1, W3, W2, stream=None):
         P1, P3, P2 = self.pool
-        if self.fused:
+        if self.fused_combine:
+            moe_grouped_ffn_combine(self.recv, self.plan, W1, W3, W2, P1, P3, P2, self.src,
+                                    self.perm, self.gate, self.R, self.S, self.h, self.out32,
+                                    self.out, self.err, stream)
+        elif self.fused:
             if self._x is None:
                 raise RuntimeError("fused expert_ffn needs a dispatch(x) first")
             moe_grouped_ffn_gather(self._x, self.src, self.plan, W1, W3, W2, P1, P3, P2, self.T,
@@ -526,6 +557,8 @@ class MoELayer:
                             self.R, self.S, self.h, self.y, self.err, stream)
 
     def combine(self, stream=None):
+        if self.fused_combine:
+            return  # done in the expert FFN's epilogue
         moe_combine(self.y, self.perm, self.gate, self.out, self.err, stream)
 
     def route_plan(self, logits, stream=None):
@@ -549,8 +582,8 @@ class MoELayer:
         """Backward of the last forward() (unfused layers: it reads recv, y and h):
         dout [T,d] bf16 -> dict(dx [T,d] bf16, dlogits [T,E] fp32, dW1, dW3 [E,F,d] fp32,
         dW2 [E,d,F] fp32).  Buffers are allocated on first use and reused."""
-        if self.fused:
-            raise RuntimeError("backward needs the dispatched rows: use an unfused layer")
+        if self.fused or self.fused_combine:
+            raise RuntimeError("backward needs the dispatched rows and y: use an unfused layer")
         if not hasattr(self, "_bwd"):
             dev = self.idx.device
             T, E, k, d, F, A = self.T, self.E, self.k, self.d, self.F, self.A
@@ -581,5 +614,5 @@ class MoELayer:
         n += 1 if self.S > 0 else 0           # prefetch
         n += (1 if self.fused else 2) if self.T > 0 else 0  # ranks[, row scatter]
         n += 2 if self.T > 0 else 0           # two grouped GEMMs
-        n += 1 if self.T > 0 else 0           # combine
+        n += 1 if self.T > 0 else 0           # combine (fused: the fp32 -> bf16 pass)
         return n

@@ -264,6 +264,37 @@ int moe_grouped_ffn(const moe_bf16* recv, const int32_t* plan, const moe_bf16* W
       as_stream(stream));
 }
 
+int moe_grouped_ffn_combine(const moe_bf16* recv, const int32_t* plan, const moe_bf16* W1,
+                            const moe_bf16* W3, const moe_f16* W2, const moe_bf16* P1,
+                            const moe_bf16* P3, const moe_f16* P2, const int32_t* src,
+                            const int32_t* perm, const float* gate, int T, int k, int E, int R,
+                            int S, int d, int F, moe_f16* h, float* out32, moe_bf16* out,
+                            int32_t* err, moe_stream_t stream) {
+  if (!plan || !W1 || !W3 || !W2 || !err) return MOE_ERR_ARG;
+  if (T > 0 && (!recv || !src || !perm || !gate || !h || !out32 || !out)) return MOE_ERR_ARG;
+  if (S > 0 && (!P1 || !P3 || !P2)) return MOE_ERR_ARG;
+  MOE_TRY(check_route(T, E, k));
+  MOE_TRY(check_ranks(T, k, E, R, true));
+  MOE_TRY(check_groups(E, R, S));
+  MOE_TRY(check_dims(T, k, d, F));
+  if ((int64_t)E * F >= kMaxElems || (int64_t)E * d >= kMaxElems ||
+      (int64_t)R * S * F >= kMaxElems || (int64_t)R * S * d >= kMaxElems)
+    return MOE_ERR_SHAPE;
+  if (!aligned16(recv) || !aligned16(h) || !aligned16(out32) || !aligned16(out) ||
+      !aligned16(W1) || !aligned16(W3) || !aligned16(W2) ||
+      (S > 0 && (!aligned16(P1) || !aligned16(P3) || !aligned16(P2))))
+    return MOE_ERR_ARG;
+  moe_plan_layout L;
+  MOE_TRY(moe_plan_get_layout(E, R, S, &L));
+  return moe::launch_grouped_ffn_combine(
+      reinterpret_cast<const __nv_bfloat16*>(recv), plan, L,
+      reinterpret_cast<const __nv_bfloat16*>(W1), reinterpret_cast<const __nv_bfloat16*>(W3),
+      reinterpret_cast<const __half*>(W2), reinterpret_cast<const __nv_bfloat16*>(P1),
+      reinterpret_cast<const __nv_bfloat16*>(P3), reinterpret_cast<const __half*>(P2), src, perm,
+      gate, T, k, E, R, S, d, F, reinterpret_cast<__half*>(h), out32,
+      reinterpret_cast<__nv_bfloat16*>(out), err, as_stream(stream));
+}
+
 int moe_dispatch_capacity(const moe_bf16* x, const int32_t* idx, const int32_t* counts, int T,
                           int k, int E, int cap, int d, int32_t* workspace, moe_bf16* recv,
                           int32_t* perm, int32_t* src, int32_t* err, moe_stream_t stream) {

@@ -96,6 +96,16 @@ int launch_dispatch_capacity(const __nv_bfloat16* x, const int32_t* idx, const i
                              int T, int k, int E, int cap, int d, int32_t* ws,
                              __nv_bfloat16* recv, int32_t* perm, int32_t* src, int32_t* err,
                              cudaStream_t s);
+// moe_grouped_ffn with the combine folded into GEMM 2's epilogue: out32 [T,d] fp32
+// (zeroed here) accumulates gate * y of every row; out = bf16(out32).  No y is written.
+int launch_grouped_ffn_combine(const __nv_bfloat16* recv, const int32_t* plan,
+                               const moe_plan_layout& L, const __nv_bfloat16* W1,
+                               const __nv_bfloat16* W3, const __half* W2,
+                               const __nv_bfloat16* P1, const __nv_bfloat16* P3,
+                               const __half* P2, const int32_t* src, const int32_t* perm,
+                               const float* gate, int T, int k, int E, int R, int S, int d,
+                               int F, __half* h, float* out32, __nv_bfloat16* out, int32_t* err,
+                               cudaStream_t s);
 // The grouped FFN over E uniform groups of cap rows (group e = rows [e*cap, (e+1)*cap),
 // expert e, home weights): the fixed-capacity layout.
 int launch_grouped_ffn_capacity(const __nv_bfloat16* recv, const __nv_bfloat16* W1,

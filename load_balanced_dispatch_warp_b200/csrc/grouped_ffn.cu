@@ -83,6 +83,14 @@ struct FfnArgs {
   const int32_t* gsrc;      // GATHER: token of each row, [R*C]
   int gd;                   // GATHER: row length of x (= d)
   int gT;                   // GATHER: rows of x (tokens)
+  // fused combine (GEMM 2 only, when comb_out != nullptr): the epilogue adds
+  // gate[t,j] * y_row into comb_out[t] (fp32 [T, out_ld]) for the token t = comb_src[row]
+  // and the choice j with comb_perm[t,j] == row, instead of storing y
+  float* comb_out;
+  const int32_t* comb_src;
+  const int32_t* comb_perm;
+  const float* comb_gate;
+  int comb_k;
 };
 
 // --------------------------------------------------------------------- PTX wrappers
@@ -526,6 +534,39 @@ __global__ void __launch_bounds__(FFN_THREADS, 1)
             uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
             for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+          }
+        }
+      } else if (args.comb_out != nullptr) {
+        // fused combine: this row's token and gate, then gate * y added into the token's
+        // fp32 output row (16-byte vector atomics, performed at L2)
+        int64_t tok = 0;
+        float gsc = 0.f;
+        bool live = valid;
+        if (live) {
+          const int r = tl.a_row + row;
+          tok = __ldg(args.comb_src + r);
+          if (tok < 0 || tok >= args.gT) {  // never touch a row outside the output
+            atomicOr(args.err, MOE_DERR_ID_RANGE);
+            live = false;
+            tok = 0;
+          } else {
+            for (int j = 0; j < args.comb_k; ++j)
+              if (__ldg(args.comb_perm + tok * args.comb_k + j) == r)
+                gsc = __ldg(args.comb_gate + tok * args.comb_k + j);
+          }
+        }
+        float* crow = args.comb_out + tok * args.out_ld + (int64_t)tl.n_block * args.bn_out;
+#pragma unroll 1
+        for (int c = 0; c < args.bn_out / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tbase + c * 32, v);
+          tmem_wait_ld();
+          if (live) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              atomicAdd(reinterpret_cast<float4*>(crow + c * 32 + 4 * i),
+                        make_float4(gsc * __uint_as_float(v[4 * i]), gsc * __uint_as_float(v[4 * i + 1]),
+                                    gsc * __uint_as_float(v[4 * i + 2]), gsc * __uint_as_float(v[4 * i + 3])));
           }
         }
       } else {
@@ -1038,6 +1079,28 @@ int ffn_pair_clusters() {
   return dev < 64 ? g_pair_clusters[dev] : 0;
 }
 
+// Fused combine operands (moe_grouped_ffn_combine).
+struct CombineArgs {
+  float* out32;  // [T, d] fp32 accumulator, zeroed by the launcher
+  const int32_t* src;
+  const int32_t* perm;
+  const float* gate;
+  int k;
+};
+
+// out[i] = bf16(acc[i]), 8 values per thread and step (16-byte stores)
+__global__ void __launch_bounds__(256) fp32_to_bf16_kernel(const float4* __restrict__ acc,
+                                                           uint4* __restrict__ out, int64_t n8,
+                                                           const int32_t* __restrict__ err) {
+  if (load_err(err)) return;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const float4 a = __ldcs(acc + 2 * i), b = __ldcs(acc + 2 * i + 1);
+    out[i] = make_uint4(pack_bf16(a.x, a.y), pack_bf16(a.z, a.w), pack_bf16(b.x, b.y),
+                        pack_bf16(b.z, b.w));
+  }
+}
+
 // GEMM 1 reads its rows from recv (x == nullptr) or gathers them as x[src[row]].  The
 // groups come from `groups` (G entries) or, with uniform_rows > 0, are E blocks of
 // uniform_rows rows; `rows` is the length of recv, h and y.
@@ -1046,10 +1109,12 @@ int launch_grouped_ffn_impl(const __nv_bfloat16* recv, const __nv_bfloat16* x,
                             int64_t rows, const __nv_bfloat16* W1, const __nv_bfloat16* W3,
                             const __half* W2, const __nv_bfloat16* P1, const __nv_bfloat16* P3,
                             const __half* P2, int T, int E, int R, int S, int d, int F,
-                            __half* h, __nv_bfloat16* y, int32_t* err, cudaStream_t s) {
+                            __half* h, __nv_bfloat16* y, int32_t* err, cudaStream_t s,
+                            const CombineArgs* comb = nullptr) {
   if (rows == 0) return MOE_OK;
   const bool gather = x != nullptr;
-  const bool pair = !gather && g_ffn_tile_mode.load(std::memory_order_relaxed) == 1;
+  const bool pair = !gather && comb == nullptr &&
+                    g_ffn_tile_mode.load(std::memory_order_relaxed) == 1;
   const int bn2 = (d % 256 == 0) ? 256 : 128;
   const int w2_box = pair ? bn2 / 2 : bn2;  // a pair CTA loads half of GEMM 2's B rows
   CUtensorMap m_recv, m_recv64, m_w1, m_w3, m_p1, m_p3, m_h, m_h64, m_w2, m_p2;
@@ -1076,6 +1141,11 @@ int launch_grouped_ffn_impl(const __nv_bfloat16* recv, const __nv_bfloat16* x,
   a1.G = G;
   a1.uniform_rows = uniform_rows;
   a1.half_tiles = (gather || pair) ? 0 : 1;  // the gathering producer always fills 128 rows
+  a1.comb_out = nullptr;
+  a1.comb_src = nullptr;
+  a1.comb_perm = nullptr;
+  a1.comb_gate = nullptr;
+  a1.comb_k = 0;
   a1.n_blocks_n = F / 128;
   a1.k_blocks = d / BK;
   a1.bn_out = 128;
@@ -1104,6 +1174,13 @@ int launch_grouped_ffn_impl(const __nv_bfloat16* recv, const __nv_bfloat16* x,
   a2.gx = nullptr;
   a2.gsrc = nullptr;
   a2.half_tiles = pair ? 0 : 1;
+  if (comb != nullptr) {
+    a2.comb_out = comb->out32;
+    a2.comb_src = comb->src;
+    a2.comb_perm = comb->perm;
+    a2.comb_gate = comb->gate;
+    a2.comb_k = comb->k;
+  }
   return pair ? launch_pair<false>(m_h, m_w2, m_w2, m_p2, m_p2, a2, s)
               : launch_one<false, false>(m_h, m_h64, m_w2, m_w2, m_p2, m_p2, a2, s);
 }
@@ -1129,6 +1206,32 @@ int launch_grouped_ffn_gather(const __nv_bfloat16* x, const int32_t* src, const 
   return launch_grouped_ffn_impl(nullptr, x, src, reinterpret_cast<const int4*>(plan + L.groups),
                                  R * L.max_groups_per_rank, 0, (int64_t)T * k, W1, W3, W2, P1,
                                  P3, P2, T, E, R, S, d, F, h, y, err, s);
+}
+
+int launch_grouped_ffn_combine(const __nv_bfloat16* recv, const int32_t* plan,
+                               const moe_plan_layout& L, const __nv_bfloat16* W1,
+                               const __nv_bfloat16* W3, const __half* W2,
+                               const __nv_bfloat16* P1, const __nv_bfloat16* P3,
+                               const __half* P2, const int32_t* src, const int32_t* perm,
+                               const float* gate, int T, int k, int E, int R, int S, int d,
+                               int F, __half* h, float* out32, __nv_bfloat16* out, int32_t* err,
+                               cudaStream_t s) {
+  if (T == 0) return MOE_OK;
+  if (cudaMemsetAsync(out32, 0, sizeof(float) * (size_t)T * d, s) != cudaSuccess)
+    return MOE_ERR_LAUNCH;
+  CombineArgs comb{out32, src, perm, gate, k};
+  const int st = launch_grouped_ffn_impl(recv, nullptr, nullptr,
+                                         reinterpret_cast<const int4*>(plan + L.groups),
+                                         R * L.max_groups_per_rank, 0, (int64_t)T * k, W1, W3,
+                                         W2, P1, P3, P2, T, E, R, S, d, F, h, nullptr, err, s,
+                                         &comb);
+  if (st != MOE_OK) return st;
+  const int64_t n8 = (int64_t)T * d / 8;
+  const int64_t want = (n8 + 255) / 256;
+  const int grid = (int)(want < (int64_t)num_sms() * 8 ? want : (int64_t)num_sms() * 8);
+  fp32_to_bf16_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const float4*>(out32),
+                                           reinterpret_cast<uint4*>(out), n8, err);
+  return launch_status();
 }
 
 int launch_grouped_ffn_capacity(const __nv_bfloat16* recv, const __nv_bfloat16* W1,

@@ -18,7 +18,7 @@ from __future__ import annotations
 
 import torch
 
-from . import MoELayer, moe_combine
+from . import MoELayer, moe_combine, moe_grouped_ffn_combine
 
 
 class HostPipeline:
@@ -61,12 +61,20 @@ class HostPipeline:
                 L.dispatch(self.x[s])
                 if not L.fused:
                     self.inputs_free[s].record(self.s_comp)
-                L.expert_ffn(W1, W3, W2)
-                if L.fused:  # the FFN gathered its rows from x
-                    self.inputs_free[s].record(self.s_comp)
-                if self._used[s]:
-                    self.s_comp.wait_event(self.out_free[s])
-                moe_combine(L.y, L.perm, L.gate, self.out[s], L.err)
+                if L.fused_combine:
+                    # GEMM 2's epilogue combines straight into this slot's output
+                    if self._used[s]:
+                        self.s_comp.wait_event(self.out_free[s])
+                    P1, P3, P2 = L.pool
+                    moe_grouped_ffn_combine(L.recv, L.plan, W1, W3, W2, P1, P3, P2, L.src, L.perm,
+                                            L.gate, L.R, L.S, L.h, L.out32, self.out[s], L.err)
+                else:
+                    L.expert_ffn(W1, W3, W2)
+                    if L.fused:  # the FFN gathered its rows from x
+                        self.inputs_free[s].record(self.s_comp)
+                    if self._used[s]:
+                        self.s_comp.wait_event(self.out_free[s])
+                    moe_combine(L.y, L.perm, L.gate, self.out[s], L.err)
                 self.out_ready[s].record(self.s_comp)
             with torch.cuda.stream(self.s_out):
                 self.s_out.wait_event(self.out_ready[s])
