@@ -70,8 +70,9 @@ struct FfnArgs {
   int G;
   int uniform_rows;     // > 0: no table; group g = {g*uniform_rows, uniform_rows, g, g}
   int half_tiles;       // 1: a tile with at most 64 valid rows runs M = 64 MMAs
-  int n_major;          // 1: a group's tiles in N-block-major order (consecutive tiles
-                        //    share a weight block), 0: M-block-major
+  int n_chunk;          // > 0: a group's tiles run chunk by chunk of n_chunk weight
+                        //    blocks, every row block of the group within a chunk (1:
+                        //    weight-block-major); 0: row-block-major
   int n_blocks_n;       // output column blocks per row block
   int k_blocks;         // K / BK
   int bn_out;           // output columns per tile (128 for SwiGLU, N for plain)
@@ -272,11 +273,15 @@ __device__ __forceinline__ Tile decode_tile(int t, const FfnArgs& a, const int* 
   }
   const int4 g = group_of(a, lo);
   int m_local = mt - s_prefix[lo];
-  if (a.n_major) {
+  if (a.n_chunk > 0) {
     const int local = t - s_prefix[lo] * a.n_blocks_n;
     const int mc = s_prefix[lo + 1] - s_prefix[lo];
-    tl.n_block = local / mc;
-    m_local = local - tl.n_block * mc;
+    const int per_chunk = mc * a.n_chunk;
+    const int c = local / per_chunk;
+    const int rem = local - c * per_chunk;
+    const int ncw = min(a.n_chunk, a.n_blocks_n - c * a.n_chunk);  // the last chunk may be narrower
+    m_local = rem / ncw;
+    tl.n_block = c * a.n_chunk + (rem - m_local * ncw);
   }
   tl.a_row = g.x + m_local * BM;
   tl.valid_rows = min(BM, g.y - m_local * BM);
@@ -1149,7 +1154,7 @@ int launch_grouped_ffn_impl(const __nv_bfloat16* recv, const __nv_bfloat16* x,
   a1.G = G;
   a1.uniform_rows = uniform_rows;
   a1.half_tiles = (gather || pair) ? 0 : 1;  // the gathering producer always fills 128 rows
-  a1.n_major = 1;  // measured faster at the DeepSeek shape (weight blocks shared by consecutive tiles)
+  a1.n_chunk = 2;  // measured fastest at the DeepSeek shape among 1, 2, 4 and row-block-major
   a1.comb_out = nullptr;
   a1.comb_src = nullptr;
   a1.comb_perm = nullptr;
