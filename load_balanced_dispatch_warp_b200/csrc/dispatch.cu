@@ -21,9 +21,10 @@
 //   scatter_kernel  the row copy on the Tensor Memory Accelerator: one thread per CTA
 //                   drives a ring of shared-memory row buffers, loading token rows with
 //                   cp.async.bulk (completion on an mbarrier) and storing each to its k
-//                   rows with bulk stores, so the copy rate does not depend on the SM
-//                   clock.  In the fixed-capacity layout the other warps zero the padding
-//                   rows meanwhile.
+//                   rows with bulk stores.  In the fixed-capacity layout the other warps
+//                   zero the padding rows meanwhile.  Below 32 tokens per SM the ring
+//                   does not fill, and scatter_warp_kernel (one warp per token, 16-byte
+//                   loads and stores; padding by pad_rows_kernel) runs instead.
 // The error word is read once at each kernel's start.  rank_kernel's blocks never write
 // it during the launch: their error bits collect in the workspace and the block that
 // finishes the last tile publishes them, so every block takes the same entry decision.
@@ -400,6 +401,66 @@ __global__ void __launch_bounds__(kScatterThreads) scatter_kernel(ScatterArgs a)
   }
 }
 
+// The same row copy with generic 16-byte loads and stores: one warp per token reads its
+// row once and stores it to each of its k rows (rows outside [0, rows_total), i.e.
+// dropped assignments, are not stored).
+constexpr int kRowVec = 4;
+
+__global__ void __launch_bounds__(kScatterThreads) scatter_warp_kernel(
+    const uint4* __restrict__ x, const int32_t* __restrict__ perm, int T, int k, int dv,
+    int64_t rows_total, uint4* __restrict__ recv, const int32_t* __restrict__ err) {
+  if (load_err(err)) return;
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T;
+       t += nwarps) {
+    int r = lane < k ? __ldg(perm + t * k + lane) : -1;
+    if (r < 0 || r >= rows_total) r = -1;
+    const uint4* xs = x + t * dv;
+    for (int v0 = 0; v0 < dv; v0 += 32 * kRowVec) {
+      uint4 buf[kRowVec];
+#pragma unroll
+      for (int u = 0; u < kRowVec; ++u) {
+        const int v = v0 + u * 32 + lane;
+        if (v < dv) buf[u] = __ldcs(xs + v);
+      }
+      for (int j = 0; j < k; ++j) {
+        const int row = __shfl_sync(MOE_FULL_MASK, r, j);
+        if (row < 0) continue;
+        uint4* dst = recv + (int64_t)row * dv;
+#pragma unroll
+        for (int u = 0; u < kRowVec; ++u) {
+          const int v = v0 + u * 32 + lane;
+          if (v < dv) dst[v] = buf[u];
+        }
+      }
+    }
+  }
+}
+
+// Fixed-capacity padding rows e*cap + [min(count_e, cap), cap): zero rows, src -1.  One
+// block per expert (grid-stride).
+__global__ void __launch_bounds__(kScatterThreads) pad_rows_kernel(
+    const int32_t* __restrict__ counts, int E, int cap, int row_bytes, uint8_t* __restrict__ recv,
+    int32_t* __restrict__ src, const int32_t* __restrict__ err) {
+  if (load_err(err)) return;
+  const int vec_per_row = row_bytes / 16;
+  for (int e = blockIdx.x; e < E; e += gridDim.x) {
+    const int c = max(0, min(__ldg(counts + e), cap));
+    const int64_t r0 = (int64_t)e * cap + c, r1 = (int64_t)(e + 1) * cap;
+    for (int64_t r = r0 + threadIdx.x; r < r1; r += blockDim.x) src[r] = -1;
+    const int64_t nvec = (r1 - r0) * vec_per_row;
+    uint4* dst = reinterpret_cast<uint4*>(recv + r0 * row_bytes);
+    for (int64_t v = threadIdx.x; v < nvec; v += blockDim.x) dst[v] = make_uint4(0, 0, 0, 0);
+  }
+}
+
+// Which row copy the dispatch runs: the TMA ring from this many tokens per SM up, one warp
+// per token below (measured on one B200, same box: near_balanced, ~28 tokens per SM, 44.1
+// against 46.2 us with the ring; Qwen shape, ~55 per SM, 82.5 against 78.1 us; DeepSeek,
+// ~111 per SM, 414 against 408 us alone and 450 against 441 us in the step).
+constexpr int kTmaScatterMinTokensPerSm = 32;
+
 int num_tiles(int T) { return (T + kRankTile - 1) / kRankTile; }
 
 int launch_rank(const int32_t* idx, int T, int k, int E, int R, int C, int cap,
@@ -436,6 +497,22 @@ int launch_rank(const int32_t* idx, int T, int k, int E, int R, int C, int cap,
 int launch_scatter(const __nv_bfloat16* x, const int32_t* perm, int T, int k, int d,
                    int64_t rows_total, __nv_bfloat16* recv, const int32_t* counts, int E,
                    int cap, int32_t* src, const int32_t* err, cudaStream_t s) {
+  if ((int64_t)T < (int64_t)kTmaScatterMinTokensPerSm * num_sms()) {
+    if (T > 0) {
+      const int64_t want = ((int64_t)T + 7) / 8;
+      const int64_t capb = (int64_t)num_sms() * 8;
+      scatter_warp_kernel<<<(int)(want < capb ? want : capb), kScatterThreads, 0, s>>>(
+          reinterpret_cast<const uint4*>(x), perm, T, k, d / 8, rows_total,
+          reinterpret_cast<uint4*>(recv), err);
+      if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
+    }
+    if (counts != nullptr) {
+      pad_rows_kernel<<<num_sms(), kScatterThreads, 0, s>>>(
+          counts, E, cap, d * 2, reinterpret_cast<uint8_t*>(recv), src, err);
+      return launch_status();
+    }
+    return MOE_OK;
+  }
   ScatterArgs a;
   a.x = reinterpret_cast<const uint8_t*>(x);
   a.perm = perm;

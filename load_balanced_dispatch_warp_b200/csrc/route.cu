@@ -286,18 +286,21 @@ __device__ __forceinline__ bool topk_token(const float* __restrict__ logits,
                                                         s_raw, idx, gate, counts, err);
 }
 
+// Warps (tokens) per block of the stand-alone top-k.
+constexpr int kTopkWarps = 8;
+
 template <int VPL, int K, bool BIASED, bool FULL = false>
-__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits,
+__global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __restrict__ logits,
                                                    const float* __restrict__ bias, int T,
                                                    int E, int k_rt, int32_t* __restrict__ idx,
                                                    float* __restrict__ gate,
                                                    int32_t* __restrict__ err) {
-  __shared__ uint32_t s_key[8][32];
-  __shared__ int s_id[8][32];
-  __shared__ float s_raw[8][32];
+  __shared__ uint32_t s_key[kTopkWarps][32];
+  __shared__ int s_id[kTopkWarps][32];
+  __shared__ float s_raw[kTopkWarps][32];
   const int k = K > 0 ? K : k_rt;
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  const int64_t t = (int64_t)blockIdx.x * 8 + wib;
+  const int64_t t = (int64_t)blockIdx.x * kTopkWarps + wib;
   if (t >= T) return;
   topk_token<VPL, K, BIASED, false, FULL>(logits, bias, t, E, k, lane, s_key[wib], s_id[wib],
                                           s_raw[wib], idx, gate, nullptr, err);
@@ -488,15 +491,15 @@ __global__ void __launch_bounds__(512) hist_kernel(const int32_t* __restrict__ i
 template <int VPL>
 void launch_topk_vpl(const float* logits, const float* bias, int T, int E, int k, int32_t* idx,
                      float* gate, int32_t* err, cudaStream_t s) {
-  const unsigned grid = (unsigned)(((int64_t)T + 7) / 8);
-#define MOE_TOPK(KK, B) topk_kernel<VPL, KK, B><<<grid, 256, 0, s>>>(logits, bias, T, E, k, idx, gate, err)
+  const unsigned grid = (unsigned)(((int64_t)T + kTopkWarps - 1) / kTopkWarps);
+#define MOE_TOPK(KK, B) topk_kernel<VPL, KK, B><<<grid, kTopkWarps * 32, 0, s>>>(logits, bias, T, E, k, idx, gate, err)
   if (bias) {
     MOE_TOPK(0, true);
     return;
   }
   if constexpr (VPL <= 8) {
     if (E == 32 * VPL) {
-#define MOE_TOPK_FULL(KK) topk_kernel<VPL, KK, false, true><<<grid, 256, 0, s>>>(logits, bias, T, E, k, idx, gate, err)
+#define MOE_TOPK_FULL(KK) topk_kernel<VPL, KK, false, true><<<grid, kTopkWarps * 32, 0, s>>>(logits, bias, T, E, k, idx, gate, err)
       switch (k) {
         case 8: MOE_TOPK_FULL(8); return;
         case 6: MOE_TOPK_FULL(6); return;
