@@ -44,9 +44,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (`ncu --set full --clock-control none -k regex:ffn_kernel ...` on the named workload),
 # keyed by workload, tile mode and kernel-sources hash: a kernel edit changes the hash,
 # and the line then reports null (with the reason) until the counters are taken again.
-TRAFFIC = {"near_balanced:0:d4ffa6ea7d84948f": int((926.897408 + 63.862528 + 478.883328 + 81.526272) * 1e6)}
-TRAFFIC_NOTE = {"near_balanced:0:d4ffa6ea7d84948f":
-                "ncu dram__bytes_read.sum + dram__bytes_write.sum, gate-up + down kernels, one call"}
+TRAFFIC = {"deepseek:0:2d07b93bd33b6aa1": 22640495104 + 533791488 + 9036560384 + 1833384192}
+TRAFFIC_NOTE = {"deepseek:0:2d07b93bd33b6aa1":
+                "ncu dram__bytes_read.sum + dram__bytes_write.sum of the gate-up and down "
+                "kernels of one full DeepSeek call (bench.py --only ffn --config deepseek)"}
 
 
 def sources_hash() -> str:
