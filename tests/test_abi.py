@@ -173,3 +173,45 @@ def test_route_plan_host_checks(lib):
     assert lib.moe_route_plan_workspace_words(64) == 16 * 64 + 1
     assert lib.moe_route_plan_workspace_words(0) == -1
     assert lib.moe_route_plan_workspace_words(1025) == -1
+
+
+def test_fixed_capacity_and_fused_combine_host_checks(lib):
+    """Host argument rules of the fixed-capacity calls and the fused combine (nothing is
+    enqueued: every call below fails before any device work)."""
+    P = ctypes.c_void_p
+    fake = P(4096)
+    assert lib.moe_capacity_rows(16, 2, 8, 0, 4) == -1
+    assert lib.moe_capacity_rows(-1, 2, 8, 5, 4) == -1
+    # dispatch_capacity: null counts, negative cap, d % 128, misaligned recv, E*cap*d too big
+    base = [fake, fake, fake, 16, 2, 8, 5, 128, fake, fake, fake, fake, fake, None]
+    bad = list(base); bad[2] = None
+    assert lib.moe_dispatch_capacity(*bad) == M.MOE_ERR_ARG
+    bad = list(base); bad[6] = -1
+    assert lib.moe_dispatch_capacity(*bad) == M.MOE_ERR_ARG
+    bad = list(base); bad[7] = 96
+    assert lib.moe_dispatch_capacity(*bad) == M.MOE_ERR_SHAPE
+    bad = list(base); bad[9] = P(4100)
+    assert lib.moe_dispatch_capacity(*bad) == M.MOE_ERR_ARG
+    bad = list(base); bad[6] = 1 << 20; bad[5] = 1024; bad[7] = 4096
+    assert lib.moe_dispatch_capacity(*bad) == M.MOE_ERR_SHAPE
+    # grouped_ffn_capacity: E > 1024, F % 128, rows * F too big
+    assert lib.moe_grouped_ffn_capacity(fake, fake, fake, fake, 2048, 4, 128, 128, fake, fake, fake, None) == M.MOE_ERR_SHAPE
+    assert lib.moe_grouped_ffn_capacity(fake, fake, fake, fake, 8, 4, 128, 200, fake, fake, fake, None) == M.MOE_ERR_SHAPE
+    assert lib.moe_grouped_ffn_capacity(fake, fake, fake, fake, 1024, 1 << 20, 128, 4096, fake, fake, fake, None) == M.MOE_ERR_SHAPE
+    assert lib.moe_grouped_ffn_capacity(fake, fake, fake, fake, 8, 4, 128, 128, fake, fake, None, None) == M.MOE_ERR_ARG
+    # combine_capacity: k > 32, null gate
+    assert lib.moe_combine_capacity(fake, fake, fake, 4, 33, 128, fake, fake, None) == M.MOE_ERR_SHAPE
+    assert lib.moe_combine_capacity(fake, fake, None, 4, 2, 128, fake, fake, None) == M.MOE_ERR_ARG
+    # fused combine: null out32 or perm, T*k % R != 0, misaligned out32, missing pool
+    args = [fake, fake, fake, fake, fake, fake, fake, fake, fake, fake, fake, 4, 2, 8, 4, 2, 128, 256,
+            fake, fake, fake, fake, None]
+    bad = list(args); bad[19] = None
+    assert lib.moe_grouped_ffn_combine(*bad) == M.MOE_ERR_ARG
+    bad = list(args); bad[9] = None
+    assert lib.moe_grouped_ffn_combine(*bad) == M.MOE_ERR_ARG
+    bad = list(args); bad[11] = 3; bad[12] = 1
+    assert lib.moe_grouped_ffn_combine(*bad) == M.MOE_ERR_SHAPE
+    bad = list(args); bad[19] = P(4100)
+    assert lib.moe_grouped_ffn_combine(*bad) == M.MOE_ERR_ARG
+    bad = list(args); bad[5] = None
+    assert lib.moe_grouped_ffn_combine(*bad) == M.MOE_ERR_ARG
