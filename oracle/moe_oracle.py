@@ -45,6 +45,11 @@ Pins (tests/test_oracle_pins.py checks each against something other than this fi
   layer_capacity    overflow [4,1,0,...], padding 13, the dropped assignments derived by
                     hand); a capacity above every demand reduces to the dropless layer;
                     identity experts return (sum of kept gates) x
+  ep_local_counts, ep_rank_base, ep_permute, ep_layer
+                    W processes computing the undistributed layer() of the rank-major
+                    concatenated batch (same perm, the same rows on every rank, the same
+                    outputs); q_base counted directly on the concatenated trace; one
+                    rank's error reaches the job's error word
   layer_backward    central finite differences of layer() itself (fp64, tiny shapes,
                     away from top-k ties); torch.autograd (fp64, CPU) through a token-major
                     formulation with no plan, dispatch or replicas; the weight gradients do
@@ -56,8 +61,8 @@ Pins (tests/test_oracle_pins.py checks each against something other than this fi
   expert_ffn_backward  central differences of expert_ffn() for X, w1, w3, w2
   (tests/test_oracle_mutants.py plants one plausible mistake at a time in topk_route,
   topk_route_biased, validate_trace, expert_histogram, capacity_ledger, remote_routes,
-  plan_balanced, permute, dispatch, prefetch, expert_ffn, combine and the four backward
-  pieces, and checks that the pin for it fails)
+  plan_balanced, permute, dispatch, prefetch, expert_ffn, combine, ep_rank_base,
+  ep_permute and the four backward pieces, and checks that the pin for it fails)
 
 Error bits (OR-ed): 1 non-finite logit, 2 expert id out of range, 4 repeated expert
 within one token, 8 plan needs more than S replicas on some rank.
@@ -358,27 +363,36 @@ def permute(idx: np.ndarray, plan, E: int, R: int):
     idx = np.asarray(idx)
     T, k = idx.shape
     C = plan["C"]
-    B = E // R
     seen = [0] * E
     perm = np.full((T, k), -1, dtype=np.int32)
     src = np.full(R * C, -1, dtype=np.int32)
-    rp = plan["room_prefix"]
     for t in range(T):
         for j in range(k):
             e = int(idx[t, j])
             q = seen[e]
             seen[e] += 1
-            if plan["kept"][e]:
-                row = (e // B) * C + plan["expert_home_off"][e] + q
-            else:
-                p = plan["stream_off"][e] + q
-                u = 0
-                while not (rp[u] <= p < rp[u + 1]):
-                    u += 1
-                row = u * C + plan["kept_rows"][u] + (p - rp[u])
+            row = placement_row(e, q, plan, E, R)
             perm[t, j] = row
             src[row] = t
     return perm, src
+
+
+def placement_row(e: int, q: int, plan, E: int, R: int) -> int:
+    """Row of the q-th assignment (token order) of expert e under the plan: a kept
+    expert's rows start at its home offset, home(e)*C + expert_home_off[e] + q; a streamed
+    expert's assignment sits at stream position p = stream_off[e] + q and lands on the
+    rank u whose room range [room_prefix[u], room_prefix[u+1]) holds p, at row
+    u*C + kept_rows[u] + (p - room_prefix[u])."""
+    C = plan["C"]
+    B = E // R
+    if plan["kept"][e]:
+        return (e // B) * C + plan["expert_home_off"][e] + q
+    rp = plan["room_prefix"]
+    p = plan["stream_off"][e] + q
+    u = 0
+    while not (rp[u] <= p < rp[u + 1]):
+        u += 1
+    return u * C + plan["kept_rows"][u] + (p - rp[u])
 
 
 def capacity_of(A: int, E: int, cf_num: int = 5, cf_den: int = 4) -> int:
@@ -577,6 +591,106 @@ def layer_capacity(logits, x, W1, W3, W2, k: int, cf_num: int = 5, cf_den: int =
     out = combine(y, perm, gate)
     return dict(idx=idx, gate=gate, hist=h, cap=cap, ledger=led, rows=rows, perm=perm, src=src,
                 recv=recv, y=y, out=out, err=err)
+
+
+# ------------------------------------------------- expert parallelism, one process per GPU
+# [MoonEP] para. 2-3 and [Primer] phases (b), (d): with one rank per GPU, every rank routes
+# its own tokens, all ranks compute the same equal-load plan from the router output of
+# the whole job, dispatch sends each assignment's row to the rank the plan gives it, each
+# rank runs the FFN on the rows it received, and combine brings every processed row back
+# to its token's rank.  Reading: the job's token order is rank-major (rank u's local token
+# t is token u*T + t) and every rank holds the same number T of tokens, so the plan of the
+# job is the plan of the concatenated batch with R = W ranks.
+
+def ep_local_counts(idx_local, E: int):
+    """Demand of one rank's own tokens: counts[e] = number of its assignments naming e
+    (in-range ids only), and its validation bits."""
+    idx_local = np.asarray(idx_local)
+    counts = np.zeros(E, dtype=np.int64)
+    for row in idx_local:
+        for v in row:
+            if 0 <= int(v) < E:
+                counts[int(v)] += 1
+    return counts, validate_trace(idx_local, E)
+
+
+def ep_rank_base(counts_all, me: int):
+    """Assignments of each expert made by lower ranks' tokens: with rank-major token
+    order they come before rank me's in every expert's token order, so rank me's q of an
+    assignment is q_base[e] = sum_{r < me} counts_all[r][e] plus its local rank."""
+    counts_all = np.asarray(counts_all, dtype=np.int64)
+    return counts_all[:me].sum(axis=0) if me > 0 else np.zeros(counts_all.shape[1], np.int64)
+
+
+def ep_permute(idx_local, q_base, plan, E: int, R: int):
+    """Job-wide row of each of one rank's assignments: the placement rule of permute()
+    with q = q_base[e] + number of this rank's earlier tokens that chose e.  Row r lives
+    on rank r // C at local row r % C.  Returns perm [T,k] int32."""
+    idx_local = np.asarray(idx_local)
+    T, k = idx_local.shape
+    seen = [int(v) for v in q_base]
+    perm = np.full((T, k), -1, dtype=np.int32)
+    for t in range(T):
+        for j in range(k):
+            e = int(idx_local[t, j])
+            perm[t, j] = placement_row(e, seen[e], plan, E, R)
+            seen[e] += 1
+    return perm
+
+
+def ep_layer(logits_shards, x_shards, W1, W3, W2, k: int, S: int):
+    """The layer as W processes run it, one per GPU, rank u holding logits_shards[u] and
+    x_shards[u] (T tokens each) and the home experts [u*B, (u+1)*B):
+      1. route locally; count local demand; exchange the counts and error bits;
+      2. every rank: job counts = sum over ranks, the same plan (R = W, T_job = W*T);
+      3. prefetch: rank u's slots copy their experts' weights from the home ranks;
+      4. dispatch: each assignment's row goes to rank perm // C, local row perm % C;
+      5. every rank runs the grouped FFN on its own C rows and groups;
+      6. combine: out[t] = sum_j gate[t,j] * y_{perm // C}[perm % C], in j order.
+    Returns dict(ranks=[per-rank dict(idx, gate, perm, recv, y, out)], plan, counts_all,
+    err)."""
+    W = len(logits_shards)
+    E = np.asarray(logits_shards[0]).shape[1]
+    T = np.asarray(logits_shards[0]).shape[0]
+    ranks = []
+    err = 0
+    for u in range(W):
+        idx, gate, e_route = topk_route(np.asarray(logits_shards[u], dtype=np.float32), k)
+        c, e_val = ep_local_counts(idx, E)
+        ranks.append(dict(idx=idx, gate=gate, counts=c))
+        err |= e_route | e_val
+    counts_all = np.stack([r["counts"] for r in ranks])
+    counts = counts_all.sum(axis=0)
+    plan = plan_balanced(counts, W * T, k, E, W, S)
+    err |= plan["err"]
+    C = plan["C"]
+    pool = prefetch(plan, W1, W3, W2, W, S)
+    d = np.asarray(x_shards[0]).shape[1]
+    recv = [np.zeros((C, d), dtype=np.asarray(x_shards[0]).dtype) for _ in range(W)]
+    for u in range(W):
+        perm = ep_permute(ranks[u]["idx"], ep_rank_base(counts_all, u), plan, E, W)
+        ranks[u]["perm"] = perm
+        xs = np.asarray(x_shards[u])
+        for t in range(T):
+            for j in range(k):
+                r = int(perm[t, j])
+                recv[r // C][r % C] = xs[t]
+    for u in range(W):
+        y = np.zeros((C, np.asarray(W2).shape[1]), dtype=np.float64)
+        for (r0, n, e, ref) in plan["groups"][u]:
+            w1, w3, w2 = weights_of(ref, E, W1, W3, W2, pool)
+            y[r0 - u * C:r0 - u * C + n] = expert_ffn(recv[u][r0 - u * C:r0 - u * C + n], w1, w3, w2)
+        ranks[u]["recv"] = recv[u]
+        ranks[u]["y"] = y
+    for u in range(W):
+        perm, gate = ranks[u]["perm"], ranks[u]["gate"]
+        out = np.zeros((T, np.asarray(W2).shape[1]))
+        for t in range(T):
+            for j in range(k):
+                r = int(perm[t, j])
+                out[t] += float(gate[t, j]) * ranks[r // C]["y"][r % C]
+        ranks[u]["out"] = out
+    return dict(ranks=ranks, plan=plan, counts_all=counts_all, err=err)
 
 
 # ------------------------------------------------------------------ backward pass

@@ -253,3 +253,38 @@ def test_ledger_and_variant_pins_catch_planted_mistakes(monkeypatch, name, mutan
     monkeypatch.setattr(O, name, mutant)
     with pytest.raises(AssertionError):
         pin()
+
+
+# ------------------------------------------------------------------ expert parallelism
+EPF = {n: getattr(O, n) for n in ("ep_rank_base", "ep_permute")}
+
+
+def rank_base_including_own_rank(counts_all, me):
+    """Counts rank me's own assignments into its base as well."""
+    return np.asarray(counts_all, dtype=np.int64)[:me + 1].sum(axis=0)
+
+
+def ep_permute_local_order_only(idx_local, q_base, plan, E, R):
+    """Ranks each assignment within its own rank's tokens only (base dropped)."""
+    return EPF["ep_permute"](idx_local, np.zeros_like(np.asarray(q_base)), plan, E, R)
+
+
+EP_MUTANTS = [
+    ("ep_rank_base", rank_base_including_own_rank,
+     F.test_ep_rank_base_counts_the_lower_ranks_assignments),
+    ("ep_rank_base", rank_base_including_own_rank,
+     F.test_ep_layer_is_the_layer_of_the_rank_major_batch),
+    ("ep_permute", ep_permute_local_order_only,
+     F.test_ep_layer_is_the_layer_of_the_rank_major_batch),
+]
+
+
+@pytest.mark.parametrize("name,mutant,pin", EP_MUTANTS,
+                         ids=[f"{c[0]}-{c[1].__name__}-{c[2].__name__}" for c in EP_MUTANTS])
+def test_ep_pins_catch_planted_mistakes(monkeypatch, name, mutant, pin):
+    pin()
+    monkeypatch.setattr(O, name, mutant)
+    # a base that overshoots can push a stream position past the last rank's room, where
+    # the placement rule finds no rank: that is caught too
+    with pytest.raises((AssertionError, IndexError)):
+        pin()

@@ -532,3 +532,63 @@ def test_biased_topk_pins():
     bad = bias.copy()
     bad[3] = np.nan
     assert O.topk_route_biased(logits, bad, 2)[2] == O.ERR_NONFINITE
+
+
+# ----------------------------------------------------------- expert parallelism
+def _ep_case(seed, W, T, E, k, d=8, F=12, skew=1.0):
+    rng = np.random.default_rng(seed)
+    logits = (rng.standard_normal((W * T, E)) - skew * np.log(np.arange(E) + 1.0)).astype(np.float32)
+    x = rng.standard_normal((W * T, d))
+    W1 = rng.standard_normal((E, F, d)) / 3
+    W3 = rng.standard_normal((E, F, d)) / 3
+    W2 = rng.standard_normal((E, d, F)) / 3
+    return logits, x, W1, W3, W2
+
+
+EP_CASES = [(0, 1, 12, 4, 2, 2), (1, 2, 12, 8, 2, 4), (2, 4, 6, 8, 2, 4), (3, 3, 8, 6, 3, 4),
+            (4, 4, 16, 16, 4, 8)]
+
+
+def test_ep_layer_is_the_layer_of_the_rank_major_batch():
+    """W processes, each routing its own T tokens, compute the undistributed layer of the
+    concatenated batch (rank u's token t = job token u*T + t) with R = W: the same rows in
+    the same places, every rank exactly C rows, the same outputs."""
+    for seed, W, T, E, k, S in EP_CASES:
+        logits, x, W1, W3, W2 = _ep_case(seed, W, T, E, k)
+        ep = O.ep_layer(np.split(logits, W), np.split(x, W), W1, W3, W2, k, S)
+        ref = O.layer(logits, x, W1, W3, W2, k, W, S)
+        assert ep["err"] == 0 and ref["err"] == 0
+        C = ref["plan"]["C"]
+        perm = np.concatenate([r["perm"] for r in ep["ranks"]])
+        assert np.array_equal(perm, ref["perm"])
+        assert sorted(perm.ravel().tolist()) == list(range(W * C))  # every rank: C rows
+        for u, r in enumerate(ep["ranks"]):
+            assert np.array_equal(r["recv"], ref["recv"][u * C:(u + 1) * C])
+            assert np.allclose(r["y"], ref["y"][u * C:(u + 1) * C], rtol=1e-12, atol=1e-12)
+        out = np.concatenate([r["out"] for r in ep["ranks"]])
+        assert np.allclose(out, ref["out"], rtol=1e-12, atol=1e-12)
+
+
+def test_ep_rank_base_counts_the_lower_ranks_assignments():
+    """q_base of rank u and expert e is the number of assignments of e made by the job's
+    tokens before u*T, counted directly on the concatenated batch."""
+    for seed, W, T, E, k, S in EP_CASES:
+        logits, *_ = _ep_case(seed, W, T, E, k)
+        idx = O.topk_route(logits, k)[0]
+        shards = np.split(idx, W)
+        counts_all = np.stack([O.ep_local_counts(s, E)[0] for s in shards])
+        for u in range(W):
+            direct = [int((idx[:u * T] == e).sum()) for e in range(E)]
+            assert O.ep_rank_base(counts_all, u).tolist() == direct
+
+
+def test_ep_error_bits_reach_every_rank():
+    """A non-finite logit on one rank, or a repeated expert in one rank's trace, is an
+    error of the whole job (every rank computes the plan from the exchanged counts)."""
+    logits, x, W1, W3, W2 = _ep_case(5, 2, 8, 8, 2)
+    bad = logits.copy()
+    bad[11, 3] = np.nan  # rank 1's token 3
+    ep = O.ep_layer(np.split(bad, 2), np.split(x, 2), W1, W3, W2, 2, 4)
+    assert ep["err"] & O.ERR_NONFINITE
+    c, e = O.ep_local_counts(np.array([[1, 1], [0, 9]]), 8)
+    assert e == O.ERR_DUPLICATE | O.ERR_ID_RANGE and c.tolist() == [1, 2, 0, 0, 0, 0, 0, 0]
