@@ -461,6 +461,149 @@ int moe_combine(const moe_bf16* y, const int32_t* perm, const float* gate, int T
                 int d, moe_bf16* out, const int32_t* err, moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * Expert parallelism across GPUs: one process per GPU, rank `me` of W.   [MoonEP]
+ * paragraphs 2-3: every rank receives exactly T*k/R rows under a plan computed on the fly
+ * from the router output; [Primer] phases (b) dispatch and (d) combine are the two
+ * all-to-all exchanges between the ranks.  Here the plan's R is W: rank u owns the home
+ * experts [u*B, (u+1)*B), B = E/W, holds S pool slots, and every rank holds the same
+ * number T of tokens.  The job's token order is rank-major (rank u's token t is job token
+ * u*T + t), so the job computes the single-GPU layer of the concatenated batch with
+ * R = W: the same plan, and rank u's receive buffer holds rows [u*C, (u+1)*C) of it,
+ * C = T*k (the job's W*T*k rows over W ranks).
+ *
+ * One step on rank me:
+ *   moe_topk (own logits) -> moe_ep_counts -> [all-gather of the (E+1)-word vectors] ->
+ *   moe_ep_plan -> moe_ep_prefetch -> moe_ep_dispatch -> [barrier] -> moe_ep_grouped_ffn
+ *   -> [barrier] -> moe_ep_combine.
+ * The exchange and the barriers are the caller's (an NCCL all-gather and a one-word
+ * all-reduce on the same stream order the ranks): every rank's dispatch must have
+ * finished before any rank's FFN reads its receive buffer, every FFN before any combine
+ * reads y, and every combine before the next step's FFN overwrites y (the next step's
+ * all-gather orders that, and the dispatch of the next step after every FFN).
+ *
+ * Pointer tables: the arguments named *_ranks are HOST arrays of W device pointers, one
+ * per rank in rank order, each that rank's buffer as addressed from THIS process (this
+ * rank's own buffer at index me, a peer GPU's buffer mapped into this process -- e.g. by
+ * moe_ipc_import -- elsewhere).  The library reads the tables when the call enqueues (they
+ * are passed to the kernels by value; a captured graph keeps them).  Peer buffers are
+ * written with plain 16-byte stores (dispatch) and read with plain 16-byte loads
+ * (prefetch, combine) over NVLink; no call uses TMA multicast.
+ *
+ * Sizes: 1 <= W <= MOE_EP_MAX_RANKS, 0 <= me < W, E % W == 0, W*T*k < 2^31, and the
+ * per-call limits of the single-GPU calls with R = W and T*k local rows.
+ */
+#define MOE_EP_MAX_RANKS 64
+
+/*
+ * moe_ep_counts: this rank's demand and error word, packed for the exchange.
+ *   idx  [T,k] int32   this rank's top-k ids.
+ *   err  int32 (in)    this rank's error word (set by moe_topk).
+ *   send [E+1] int32 (out, device)  send[e] = assignments of this rank's tokens naming e
+ *                      (ids in range only); send[E] = *err | MOE_DERR_ID_RANGE (an id
+ *                      outside [0, E)) | MOE_DERR_DUPLICATE (a token repeating an id).
+ *                      *err itself is not written: the bits reach every rank through
+ *                      the exchanged vectors (moe_ep_plan).  With *err != 0 on entry,
+ *                      send = {0, ..., 0, *err}.
+ */
+int moe_ep_counts(const int32_t* idx, int T, int k, int E, const int32_t* err, int32_t* send,
+                  moe_stream_t stream);
+
+/*
+ * moe_ep_plan: the job's demand, this rank's base offsets and the plan (the same on every
+ * rank, bit for bit, since every rank reads the same vectors).
+ *   gathered [W][E+1] int32   every rank's send vector in rank order (the all-gather).
+ *   T        tokens per rank.
+ *   err      (in/out) |= the OR of every rank's send[E]; when that is non-zero nothing
+ *            else is written (on every rank alike, so the ranks stop together).
+ *   counts   [E] int32 (out)  the job's demand (sum over the ranks).
+ *   q_base   [E] int32 (out)  assignments of expert e made by the ranks below me (the
+ *                             position of this rank's first e-assignment in e's order).
+ *   loads [W] int32, maxvio, balancedness (fp64, device) (out)  as moe_histogram_maxvio
+ *            with R = W, the home map and A = W*T*k.
+ *   plan     int32 buffer of moe_plan_get_layout(E, W, S) (out), as moe_plan_balanced on
+ *            the job's demand with T_job = W*T; MOE_DERR_SLOTS as there.
+ */
+int moe_ep_plan(const int32_t* gathered, int W, int me, int T, int k, int E, int S,
+                int32_t* counts, int32_t* q_base, int32_t* loads, double* maxvio,
+                double* balancedness, int32_t* plan, int32_t* err, moe_stream_t stream);
+
+/*
+ * moe_ep_prefetch: this rank's pool slots receive their experts' weights from the home
+ * ranks (a peer copy into local memory before any FFN reads them).
+ *   W1_ranks, W3_ranks (moe_bf16, each [B,F,d]), W2_ranks (moe_f16, each [B,d,F]): HOST
+ *            tables of every rank's home tensors (see "Pointer tables").
+ *   P1, P3 [S,F,d] bf16, P2 [S,d,F] fp16 (out): this rank's slots; slot s receives
+ *            expert e = replica_expert[me*S + s] (local expert e % B of rank e / B),
+ *            bitwise; empty slots are untouched.
+ *   err  no-op when non-zero.
+ */
+int moe_ep_prefetch(const int32_t* plan, const moe_bf16* const* W1_ranks,
+                    const moe_bf16* const* W3_ranks, const moe_f16* const* W2_ranks, int W,
+                    int me, int E, int S, int d, int F, moe_bf16* P1, moe_bf16* P3, moe_f16* P2,
+                    const int32_t* err, moe_stream_t stream);
+
+/*
+ * moe_ep_dispatch: every assignment of this rank's tokens straight into its final row on
+ * the rank that processes it.
+ *   x [T,d] bf16, idx [T,k]: this rank's tokens and ids; q_base from moe_ep_plan.
+ *   workspace  moe_dispatch_workspace_words(T, E) int32 words.
+ *   recv_ranks HOST table of every rank's receive buffer [C,d] bf16, C = T*k.
+ *   perm [T,k] int32 (out): the job-wide row of each assignment (rank perm / C, local
+ *        row perm % C): the rows moe_dispatch assigns to these tokens in the
+ *        concatenated batch.  Row perm receives x[t] bitwise.
+ *   err  no-op when non-zero; MOE_DERR_ID_RANGE, MOE_DERR_TIMEOUT as moe_dispatch.
+ */
+int moe_ep_dispatch(const moe_bf16* x, const int32_t* idx, const int32_t* q_base,
+                    const int32_t* plan, int W, int T, int k, int E, int S, int d,
+                    int32_t* workspace, moe_bf16* const* recv_ranks, int32_t* perm,
+                    int32_t* err, moe_stream_t stream);
+
+/*
+ * moe_ep_grouped_ffn: the grouped SwiGLU FFN over this rank's C rows and groups.
+ *   recv [C,d] bf16: this rank's receive buffer; W1, W3 [B,F,d] bf16 and W2 [B,d,F] fp16:
+ *   its home experts; P1, P3, P2: its pool (as moe_ep_prefetch).
+ *   groups_ws [4*(B+S)] int32 (device scratch): the rank's group table re-based to local
+ *   rows and local weights (row_start - me*C; expert e -> e - me*B; slot -> B + s).
+ *   h [C,F] fp16, y [C,d] bf16 (out): as moe_grouped_ffn, row for row the rows
+ *   [me*C, (me+1)*C) of the single-GPU layer's h and y.
+ *   err  no-op when non-zero; MOE_DERR_TIMEOUT as moe_grouped_ffn, MOE_DERR_ID_RANGE if a
+ *   group of this rank names weights that are not on it (never, for a plan of moe_ep_plan).
+ */
+int moe_ep_grouped_ffn(const moe_bf16* recv, const int32_t* plan, int W, int me,
+                       const moe_bf16* W1, const moe_bf16* W3, const moe_f16* W2,
+                       const moe_bf16* P1, const moe_bf16* P3, const moe_f16* P2, int T, int k,
+                       int E, int S, int d, int F, int32_t* groups_ws, moe_f16* h, moe_bf16* y,
+                       int32_t* err, moe_stream_t stream);
+
+/*
+ * moe_ep_combine: out[t] = sum_j gate[t,j] * y_{perm[t,j] / C}[perm[t,j] % C] (fp32, j
+ * order; bf16 out), C = T*k: the same sums as moe_combine over the single-GPU layer.
+ *   y_ranks  HOST table of every rank's y [C,d] bf16.
+ *   perm, gate [T,k] of this rank (perm from moe_ep_dispatch with *err left at 0).
+ *   out [T,d] bf16 (out).  err  no-op when non-zero.
+ */
+int moe_ep_combine(const moe_bf16* const* y_ranks, const int32_t* perm, const float* gate,
+                   int W, int T, int k, int d, moe_bf16* out, const int32_t* err,
+                   moe_stream_t stream);
+
+/*
+ * Device-memory sharing between the processes of one node (CUDA IPC), for the pointer
+ * tables above.  Host calls; nothing is enqueued.
+ * moe_ipc_export: handle (host buffer of MOE_IPC_HANDLE_BYTES) names the allocation that
+ *   holds the device pointer ptr; *offset = ptr - the allocation's base.  MOE_ERR_ARG for
+ *   a null argument, MOE_ERR_DEVICE if the runtime refuses (not a device allocation, or
+ *   one that cannot be shared).
+ * moe_ipc_import: maps another process's exported allocation into this one (peer access
+ *   enabled on first use); *ptr = base + offset, *base = the mapping to close later.  A
+ *   process cannot import its own export (MOE_ERR_DEVICE): it uses its own pointer.
+ * moe_ipc_close: unmaps a base returned by moe_ipc_import.
+ */
+#define MOE_IPC_HANDLE_BYTES 64
+int moe_ipc_export(const void* ptr, void* handle, int64_t* offset);
+int moe_ipc_import(const void* handle, int64_t offset, void** ptr, void** base);
+int moe_ipc_close(void* base);
+
+/* ---------------------------------------------------------------------------------
  * Grouped-FFN tile mode (a B200 tiling choice; the pages fix no kernel design).
  *   0  one CTA per 128-row x N tile (tcgen05.mma.cta_group::1), the default.
  *   1  CTA pairs (2-CTA clusters) on 256-row x N tiles (tcgen05.mma.cta_group::2): each

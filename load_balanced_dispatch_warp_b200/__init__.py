@@ -30,6 +30,9 @@ VARIANTS = ("moe_topk_biased", "moe_capacity_ledger", "moe_dispatch_capacity",
             "moe_grouped_ffn_capacity", "moe_combine_capacity")
 FUSED = ("moe_dispatch_index", "moe_grouped_ffn_gather", "moe_route_plan",
          "moe_grouped_ffn_combine")
+EXPERT_PARALLEL = ("moe_ep_counts", "moe_ep_plan", "moe_ep_prefetch", "moe_ep_dispatch",
+                   "moe_ep_grouped_ffn", "moe_ep_combine", "moe_ipc_export", "moe_ipc_import",
+                   "moe_ipc_close")
 BACKWARD = ("moe_combine_backward", "moe_grouped_ffn_backward", "moe_dispatch_backward",
             "moe_topk_backward")
 HELPERS = ("moe_plan_get_layout", "moe_dispatch_workspace_words", "moe_status_string",
@@ -84,6 +87,15 @@ def lib() -> ctypes.CDLL:
                                         P, P, P, P],
             "moe_grouped_ffn_capacity": [P, P, P, P, I, I, I, I, P, P, P, P],
             "moe_combine_capacity": [P, P, P, I, I, I, P, P, P],
+            "moe_ep_counts": [P, I, I, I, P, P, P],
+            "moe_ep_plan": [P, I, I, I, I, I, I, P, P, P, P, P, P, P, P],
+            "moe_ep_prefetch": [P, P, P, P, I, I, I, I, I, I, P, P, P, P, P],
+            "moe_ep_dispatch": [P, P, P, P, I, I, I, I, I, I, P, P, P, P, P],
+            "moe_ep_grouped_ffn": [P, P, I, I, P, P, P, P, P, P, I, I, I, I, I, I, P, P, P, P, P],
+            "moe_ep_combine": [P, P, P, I, I, I, I, P, P, P],
+            "moe_ipc_export": [P, P, ctypes.POINTER(I64)],
+            "moe_ipc_import": [P, I64, ctypes.POINTER(P), ctypes.POINTER(P)],
+            "moe_ipc_close": [P],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -399,6 +411,102 @@ def moe_grouped_ffn_combine(recv, plan, W1, W3, W2, P1, P3, P2, src, perm, gate,
         _ptr(src, i32, "src"), _ptr(perm, i32, "perm"), _ptr(gate, torch.float32, "gate"), T, k,
         E, R, S, d, F, _ptr(h, hf, "h"), _ptr(out32, torch.float32, "out32"), _ptr(out, bf, "out"),
         _ptr(err, i32, "err"), _stream(stream)), "moe_grouped_ffn_combine")
+
+
+# ------------------------------------------------------- expert parallelism across GPUs
+EP_MAX_RANKS = 64           # MOE_EP_MAX_RANKS
+IPC_HANDLE_BYTES = 64       # MOE_IPC_HANDLE_BYTES
+
+
+def _table(ptrs, name):
+    """A host array of device pointers (one per rank) for the *_ranks arguments."""
+    ptrs = [int(p) for p in ptrs]
+    if not ptrs or any(p == 0 for p in ptrs):
+        raise ValueError(f"{name}: one non-null device pointer per rank")
+    return (ctypes.c_void_p * len(ptrs))(*ptrs)
+
+
+def moe_ep_counts(idx, E, err, send, stream=None):
+    T, k = idx.shape
+    _check(lib().moe_ep_counts(_ptr(idx, torch.int32, "idx"), T, k, E, _ptr(err, torch.int32, "err"),
+                               _ptr(send, torch.int32, "send"), _stream(stream)), "moe_ep_counts")
+
+
+def moe_ep_plan(gathered, me, T, k, S, counts, q_base, loads, maxvio, balancedness, plan, err,
+                stream=None):
+    W, E1 = gathered.shape
+    i32 = torch.int32
+    _check(lib().moe_ep_plan(
+        _ptr(gathered, i32, "gathered"), W, me, T, k, E1 - 1, S, _ptr(counts, i32, "counts"),
+        _ptr(q_base, i32, "q_base"), _ptr(loads, i32, "loads"), _ptr(maxvio, torch.float64, "maxvio"),
+        _ptr(balancedness, torch.float64, "balancedness"), _ptr(plan, i32, "plan"),
+        _ptr(err, i32, "err"), _stream(stream)), "moe_ep_plan")
+
+
+def moe_ep_prefetch(plan, W1_ranks, W3_ranks, W2_ranks, me, E, S, d, F, P1, P3, P2, err,
+                    stream=None):
+    W = len(W1_ranks)
+    bf, hf = torch.bfloat16, torch.float16
+    _check(lib().moe_ep_prefetch(
+        _ptr(plan, torch.int32, "plan"), _table(W1_ranks, "W1_ranks"), _table(W3_ranks, "W3_ranks"),
+        _table(W2_ranks, "W2_ranks"), W, me, E, S, d, F, _ptr(P1, bf, "P1"), _ptr(P3, bf, "P3"),
+        _ptr(P2, hf, "P2"), _ptr(err, torch.int32, "err"), _stream(stream)), "moe_ep_prefetch")
+
+
+def moe_ep_dispatch(x, idx, q_base, plan, E, S, workspace, recv_ranks, perm, err, stream=None):
+    T, d = x.shape
+    k = idx.shape[1]
+    i32 = torch.int32
+    _check(lib().moe_ep_dispatch(
+        _ptr(x, torch.bfloat16, "x"), _ptr(idx, i32, "idx"), _ptr(q_base, i32, "q_base"),
+        _ptr(plan, i32, "plan"), len(recv_ranks), T, k, E, S, d,
+        _ptr(workspace, i32, "workspace"), _table(recv_ranks, "recv_ranks"),
+        _ptr(perm, i32, "perm"), _ptr(err, i32, "err"), _stream(stream)), "moe_ep_dispatch")
+
+
+def moe_ep_grouped_ffn(recv, plan, W, me, W1, W3, W2, P1, P3, P2, T, k, E, S, groups_ws, h, y,
+                       err, stream=None):
+    _, F, d = W1.shape
+    bf, hf = torch.bfloat16, torch.float16
+    _check(lib().moe_ep_grouped_ffn(
+        _ptr(recv, bf, "recv"), _ptr(plan, torch.int32, "plan"), W, me, _ptr(W1, bf, "W1"),
+        _ptr(W3, bf, "W3"), _ptr(W2, hf, "W2"), _ptr(P1, bf, "P1"), _ptr(P3, bf, "P3"),
+        _ptr(P2, hf, "P2"), T, k, E, S, d, F, _ptr(groups_ws, torch.int32, "groups_ws"),
+        _ptr(h, hf, "h"), _ptr(y, bf, "y"), _ptr(err, torch.int32, "err"), _stream(stream)),
+        "moe_ep_grouped_ffn")
+
+
+def moe_ep_combine(y_ranks, perm, gate, d, out, err, stream=None):
+    T, k = perm.shape
+    _check(lib().moe_ep_combine(
+        _table(y_ranks, "y_ranks"), _ptr(perm, torch.int32, "perm"), _ptr(gate, torch.float32, "gate"),
+        len(y_ranks), T, k, d, _ptr(out, torch.bfloat16, "out"), _ptr(err, torch.int32, "err"),
+        _stream(stream)), "moe_ep_combine")
+
+
+def ipc_export(t: torch.Tensor):
+    """(handle bytes, offset) naming the allocation that holds tensor t's storage."""
+    if not t.is_cuda:
+        raise TypeError("ipc_export needs a CUDA tensor")
+    h = ctypes.create_string_buffer(IPC_HANDLE_BYTES)
+    off = ctypes.c_int64(0)
+    _check(lib().moe_ipc_export(t.data_ptr(), h, ctypes.byref(off)), "moe_ipc_export")
+    return h.raw, off.value
+
+
+def ipc_import(handle: bytes, offset: int):
+    """(device pointer, mapping base) of another process's exported buffer."""
+    if len(handle) != IPC_HANDLE_BYTES:
+        raise ValueError("IPC handle of the wrong size")
+    ptr, base = ctypes.c_void_p(), ctypes.c_void_p()
+    buf = ctypes.create_string_buffer(handle, IPC_HANDLE_BYTES)
+    _check(lib().moe_ipc_import(buf, offset, ctypes.byref(ptr), ctypes.byref(base)),
+           "moe_ipc_import")
+    return ptr.value, base.value
+
+
+def ipc_close(base: int):
+    _check(lib().moe_ipc_close(base), "moe_ipc_close")
 
 
 def moe_combine(y, perm, gate, out, err, stream=None):

@@ -40,6 +40,27 @@ cudaStream_t as_stream(moe_stream_t s) { return reinterpret_cast<cudaStream_t>(s
     if (st_ != MOE_OK) return st_; \
   } while (0)
 
+// W ranks, rank me, T tokens per rank: the single-GPU rules on the job (W*T tokens,
+// R = W) and on this rank's T*k receive rows.
+int check_ep(int W, int me, int T, int k, int E, int S) {
+  if (W < 1 || me < 0 || me >= W || T < 0) return MOE_ERR_ARG;
+  if (W > MOE_EP_MAX_RANKS) return MOE_ERR_SHAPE;
+  MOE_TRY(check_route(T, E, k));
+  if ((int64_t)W * T * k >= kMaxElems || (int64_t)W * T * E >= kMaxElems) return MOE_ERR_SHAPE;
+  MOE_TRY(check_ranks(W * T, k, E, W, true));
+  return check_groups(E, W, S);
+}
+
+// every entry of a host table of W device pointers non-null and 16-byte aligned
+template <typename P>
+int check_table(P const* table, int W) {
+  if (!table) return MOE_ERR_ARG;
+  for (int u = 0; u < W; ++u)
+    if (!table[u] || !aligned16(table[u])) return MOE_ERR_ARG;
+  return MOE_OK;
+}
+
+
 }  // namespace
 
 extern "C" {
@@ -430,6 +451,121 @@ int moe_grouped_ffn_backward(const moe_bf16* recv, const moe_bf16* dy, const moe
       reinterpret_cast<const __nv_bfloat16*>(W3), reinterpret_cast<const __half*>(W2), T, k, E,
       R, S, d, F, reinterpret_cast<__nv_bfloat16*>(dx_rows), dW1, dW3, dW2, workspace,
       workspace_bytes, err, as_stream(stream));
+}
+
+// ------------------------------------------------------- expert parallelism across GPUs
+
+int moe_ep_counts(const int32_t* idx, int T, int k, int E, const int32_t* err, int32_t* send,
+                  moe_stream_t stream) {
+  if (!err || !send) return MOE_ERR_ARG;
+  if (T > 0 && !idx) return MOE_ERR_ARG;
+  MOE_TRY(check_route(T, E, k));
+  return moe::launch_ep_counts(idx, T, k, E, err, send, as_stream(stream));
+}
+
+int moe_ep_plan(const int32_t* gathered, int W, int me, int T, int k, int E, int S,
+                int32_t* counts, int32_t* q_base, int32_t* loads, double* maxvio,
+                double* balancedness, int32_t* plan, int32_t* err, moe_stream_t stream) {
+  if (!gathered || !counts || !q_base || !loads || !maxvio || !balancedness || !plan || !err)
+    return MOE_ERR_ARG;
+  MOE_TRY(check_ep(W, me, T, k, E, S));
+  moe_plan_layout L;
+  MOE_TRY(moe_plan_get_layout(E, W, S, &L));
+  return moe::launch_ep_plan(gathered, W, me, T, k, E, S, counts, q_base, loads, maxvio,
+                             balancedness, plan, L, err, as_stream(stream));
+}
+
+int moe_ep_prefetch(const int32_t* plan, const moe_bf16* const* W1_ranks,
+                    const moe_bf16* const* W3_ranks, const moe_f16* const* W2_ranks, int W,
+                    int me, int E, int S, int d, int F, moe_bf16* P1, moe_bf16* P3, moe_f16* P2,
+                    const int32_t* err, moe_stream_t stream) {
+  if (!plan || !err) return MOE_ERR_ARG;
+  MOE_TRY(check_ep(W, me, 0, 1, E, S));
+  MOE_TRY(check_dims(0, 1, d, F));
+  if ((int64_t)(E / W) * d * F >= kMaxElems || (int64_t)S * d * F >= kMaxElems)
+    return MOE_ERR_SHAPE;
+  if (S == 0) return MOE_OK;
+  MOE_TRY(check_table(W1_ranks, W));
+  MOE_TRY(check_table(W3_ranks, W));
+  MOE_TRY(check_table(W2_ranks, W));
+  if (!P1 || !P3 || !P2 || !aligned16(P1) || !aligned16(P3) || !aligned16(P2)) return MOE_ERR_ARG;
+  moe_plan_layout L;
+  MOE_TRY(moe_plan_get_layout(E, W, S, &L));
+  return moe::launch_ep_prefetch(
+      plan, L, reinterpret_cast<const __nv_bfloat16* const*>(W1_ranks),
+      reinterpret_cast<const __nv_bfloat16* const*>(W3_ranks),
+      reinterpret_cast<const __half* const*>(W2_ranks), W, me, E, S, d, F,
+      reinterpret_cast<__nv_bfloat16*>(P1), reinterpret_cast<__nv_bfloat16*>(P3),
+      reinterpret_cast<__half*>(P2), err, as_stream(stream));
+}
+
+int moe_ep_dispatch(const moe_bf16* x, const int32_t* idx, const int32_t* q_base,
+                    const int32_t* plan, int W, int T, int k, int E, int S, int d,
+                    int32_t* workspace, moe_bf16* const* recv_ranks, int32_t* perm,
+                    int32_t* err, moe_stream_t stream) {
+  if (!plan || !q_base || !err) return MOE_ERR_ARG;
+  if (T > 0 && (!x || !idx || !workspace || !perm)) return MOE_ERR_ARG;
+  MOE_TRY(check_ep(W, 0, T, k, E, S));
+  MOE_TRY(check_dims(T, k, d, 128));
+  if (T > 0) {
+    MOE_TRY(check_table(recv_ranks, W));
+    if (!aligned16(x)) return MOE_ERR_ARG;
+  }
+  moe_plan_layout L;
+  MOE_TRY(moe_plan_get_layout(E, W, S, &L));
+  return moe::launch_ep_dispatch(reinterpret_cast<const __nv_bfloat16*>(x), idx, q_base, plan, L,
+                                 T, k, E, W, d, workspace,
+                                 reinterpret_cast<__nv_bfloat16* const*>(recv_ranks), perm, err,
+                                 as_stream(stream));
+}
+
+int moe_ep_grouped_ffn(const moe_bf16* recv, const int32_t* plan, int W, int me,
+                       const moe_bf16* W1, const moe_bf16* W3, const moe_f16* W2,
+                       const moe_bf16* P1, const moe_bf16* P3, const moe_f16* P2, int T, int k,
+                       int E, int S, int d, int F, int32_t* groups_ws, moe_f16* h, moe_bf16* y,
+                       int32_t* err, moe_stream_t stream) {
+  if (!plan || !W1 || !W3 || !W2 || !groups_ws || !err) return MOE_ERR_ARG;
+  if (T > 0 && (!recv || !h || !y)) return MOE_ERR_ARG;
+  if (S > 0 && (!P1 || !P3 || !P2)) return MOE_ERR_ARG;
+  MOE_TRY(check_ep(W, me, T, k, E, S));
+  MOE_TRY(check_dims(T, k, d, F));
+  const int B = E / W;
+  if ((int64_t)B * F >= kMaxElems || (int64_t)B * d >= kMaxElems ||
+      (int64_t)S * F >= kMaxElems || (int64_t)S * d >= kMaxElems)
+    return MOE_ERR_SHAPE;
+  if (!aligned16(recv) || !aligned16(h) || !aligned16(y) || !aligned16(W1) || !aligned16(W3) ||
+      !aligned16(W2) || !aligned16(groups_ws) ||
+      (S > 0 && (!aligned16(P1) || !aligned16(P3) || !aligned16(P2))))
+    return MOE_ERR_ARG;
+  if (T == 0) return MOE_OK;
+  moe_plan_layout L;
+  MOE_TRY(moe_plan_get_layout(E, W, S, &L));
+  const int C = T * k;
+  cudaStream_t s = as_stream(stream);
+  MOE_TRY(moe::launch_ep_groups(plan, L, me, E, W, S, C, groups_ws, err, s));
+  return moe::launch_grouped_ffn_groups(
+      reinterpret_cast<const __nv_bfloat16*>(recv), groups_ws, B + S, C,
+      reinterpret_cast<const __nv_bfloat16*>(W1), reinterpret_cast<const __nv_bfloat16*>(W3),
+      reinterpret_cast<const __half*>(W2), reinterpret_cast<const __nv_bfloat16*>(P1),
+      reinterpret_cast<const __nv_bfloat16*>(P3), reinterpret_cast<const __half*>(P2), B, S, d,
+      F, reinterpret_cast<__half*>(h), reinterpret_cast<__nv_bfloat16*>(y), err, s);
+}
+
+int moe_ep_combine(const moe_bf16* const* y_ranks, const int32_t* perm, const float* gate,
+                   int W, int T, int k, int d, moe_bf16* out, const int32_t* err,
+                   moe_stream_t stream) {
+  if (!err) return MOE_ERR_ARG;
+  if (T > 0 && (!perm || !gate || !out)) return MOE_ERR_ARG;
+  if (W < 1 || T < 0 || k < 1) return MOE_ERR_ARG;
+  if (W > MOE_EP_MAX_RANKS || k > 32) return MOE_ERR_SHAPE;
+  if ((int64_t)W * T * k >= kMaxElems) return MOE_ERR_SHAPE;
+  MOE_TRY(check_dims(T, k, d, 128));
+  if (T == 0) return MOE_OK;
+  MOE_TRY(check_table(y_ranks, W));
+  if (!aligned16(out)) return MOE_ERR_ARG;
+  return moe::launch_ep_combine(reinterpret_cast<const __nv_bfloat16* const*>(y_ranks), W, perm,
+                                gate, T, k, d, reinterpret_cast<__nv_bfloat16*>(out), err,
+                                as_stream(stream));
 }
 
 int moe_set_ffn_tile_mode(int mode) { return moe::set_ffn_tile_mode(mode); }

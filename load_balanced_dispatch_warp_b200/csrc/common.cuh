@@ -113,6 +113,38 @@ int launch_grouped_ffn_capacity(const __nv_bfloat16* recv, const __nv_bfloat16* 
                                 int d, int F, __half* h, __nv_bfloat16* y, int32_t* err,
                                 cudaStream_t s);
 
+// The grouped FFN over an explicit group table [G][4] {row_start, rows, expert,
+// weight_ref} (rows == -1: unused) on `rows` receive rows, one rank's worth: weight_ref
+// < E reads the home tensors (E experts), E + s reads pool slot s (S slots).
+int launch_grouped_ffn_groups(const __nv_bfloat16* recv, const int32_t* groups, int G,
+                              int64_t rows, const __nv_bfloat16* W1, const __nv_bfloat16* W3,
+                              const __half* W2, const __nv_bfloat16* P1, const __nv_bfloat16* P3,
+                              const __half* P2, int E, int S, int d, int F, __half* h,
+                              __nv_bfloat16* y, int32_t* err, cudaStream_t s);
+
+// Expert parallelism across GPUs (ep.cu, and the peer forms of dispatch, prefetch and
+// combine).  The *_ranks arrays are HOST arrays of W device pointers, one per rank, as
+// mapped in this process.
+int launch_ep_counts(const int32_t* idx, int T, int k, int E, const int32_t* err,
+                     int32_t* send, cudaStream_t s);
+int launch_ep_plan(const int32_t* gathered, int W, int me, int T, int k, int E, int S,
+                   int32_t* counts, int32_t* q_base, int32_t* loads, double* maxvio, double* bal,
+                   int32_t* plan, const moe_plan_layout& L, int32_t* err, cudaStream_t s);
+int launch_ep_groups(const int32_t* plan, const moe_plan_layout& L, int me, int E, int W, int S,
+                     int C, int32_t* groups, int32_t* err, cudaStream_t s);
+int launch_ep_prefetch(const int32_t* plan, const moe_plan_layout& L,
+                       const __nv_bfloat16* const* W1_ranks, const __nv_bfloat16* const* W3_ranks,
+                       const __half* const* W2_ranks, int W, int me, int E, int S, int d, int F,
+                       __nv_bfloat16* P1, __nv_bfloat16* P3, __half* P2, const int32_t* err,
+                       cudaStream_t s);
+int launch_ep_dispatch(const __nv_bfloat16* x, const int32_t* idx, const int32_t* q_base,
+                       const int32_t* plan, const moe_plan_layout& L, int T, int k, int E,
+                       int W, int d, int32_t* ws, __nv_bfloat16* const* recv_ranks,
+                       int32_t* perm, int32_t* err, cudaStream_t s);
+int launch_ep_combine(const __nv_bfloat16* const* y_ranks, int W, const int32_t* perm,
+                      const float* gate, int T, int k, int d, __nv_bfloat16* out,
+                      const int32_t* err, cudaStream_t s);
+
 // ----------------------------------------------------------------------------- device side
 // Reads the layer's error word once per thread; every kernel after moe_topk returns
 // early when it is non-zero.

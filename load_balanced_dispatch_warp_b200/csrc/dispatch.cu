@@ -63,6 +63,9 @@ struct RankArgs {
   int cap;               // > 0: fixed-capacity layout, row = e * cap + q (q < cap), else -1
   const int32_t* plan;   // dropless layout (cap == 0): the plan's fields
   moe_plan_layout L;
+  const int32_t* q_base; // nullable: [E] assignments of each expert that come before this
+                         // launch's tokens in the job's token order (expert parallelism
+                         // across processes: the lower ranks' tokens)
   int32_t* ws;
   int ntiles;
   int32_t* perm;
@@ -209,7 +212,8 @@ __global__ void __launch_bounds__(kRankTile) rank_kernel(RankArgs a) {
     for (int j = 0; j < a.k; ++j) {
       const int e = __ldg(a.idx + t * a.k + j);
       if (e < 0 || e >= E) continue;
-      const int q = s_pre[warp * E + e] + __popc(s_mask[warp * E + e] & lt);
+      int q = s_pre[warp * E + e] + __popc(s_mask[warp * E + e] & lt);
+      if (a.q_base != nullptr) q += __ldg(a.q_base + e);
       int64_t row;
       if (a.cap > 0) {
         row = q < a.cap ? (int64_t)e * a.cap + q : -1;  // past the capacity: dropped
@@ -232,7 +236,7 @@ __global__ void __launch_bounds__(kRankTile) rank_kernel(RankArgs a) {
         }
       }
       a.perm[t * a.k + j] = (int32_t)row;
-      if (row >= 0) a.src[row] = (int32_t)t;
+      if (row >= 0 && a.src != nullptr) a.src[row] = (int32_t)t;
     }
   }
   if (my_err) atomicOr(&s_err, my_err);
@@ -406,9 +410,26 @@ __global__ void __launch_bounds__(kScatterThreads) scatter_kernel(ScatterArgs a)
 // dropped assignments, are not stored).
 constexpr int kRowVec = 4;
 
+// Where row r of the receive space lives: one buffer on this GPU, or (expert parallelism
+// across GPUs) rank r / C's buffer, local row r % C, through the pointer this process has
+// for it (its own buffer, or a peer GPU's mapped into this process).
+struct LocalRows {
+  uint4* base;
+  __device__ __forceinline__ uint4* row(int64_t r, int dv) const { return base + r * dv; }
+};
+struct RankRows {
+  uint4* base[MOE_EP_MAX_RANKS];
+  int C;
+  __device__ __forceinline__ uint4* row(int64_t r, int dv) const {
+    const int u = (int)(r / C);
+    return base[u] + (r - (int64_t)u * C) * dv;
+  }
+};
+
+template <class Dst>
 __global__ void __launch_bounds__(kScatterThreads) scatter_warp_kernel(
     const uint4* __restrict__ x, const int32_t* __restrict__ perm, int T, int k, int dv,
-    int64_t rows_total, uint4* __restrict__ recv, const int32_t* __restrict__ err) {
+    int64_t rows_total, const __grid_constant__ Dst recv, const int32_t* __restrict__ err) {
   if (load_err(err)) return;
   const int lane = threadIdx.x & 31;
   const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
@@ -427,7 +448,7 @@ __global__ void __launch_bounds__(kScatterThreads) scatter_warp_kernel(
       for (int j = 0; j < k; ++j) {
         const int row = __shfl_sync(MOE_FULL_MASK, r, j);
         if (row < 0) continue;
-        uint4* dst = recv + (int64_t)row * dv;
+        uint4* dst = recv.row(row, dv);
 #pragma unroll
         for (int u = 0; u < kRowVec; ++u) {
           const int v = v0 + u * 32 + lane;
@@ -465,7 +486,7 @@ int num_tiles(int T) { return (T + kRankTile - 1) / kRankTile; }
 
 int launch_rank(const int32_t* idx, int T, int k, int E, int R, int C, int cap,
                 const int32_t* plan, const moe_plan_layout* L, int32_t* ws, int32_t* perm,
-                int32_t* src, int32_t* err, cudaStream_t s) {
+                int32_t* src, int32_t* err, cudaStream_t s, const int32_t* q_base = nullptr) {
   const int ntiles = num_tiles(T);
   if (cudaMemsetAsync(ws, 0, sizeof(int32_t) * (size_t)ws_agg_off(ntiles), s) != cudaSuccess)
     return MOE_ERR_LAUNCH;
@@ -478,6 +499,7 @@ int launch_rank(const int32_t* idx, int T, int k, int E, int R, int C, int cap,
   a.C = C;
   a.cap = cap;
   a.plan = plan;
+  a.q_base = q_base;
   if (L) a.L = *L;
   else memset(&a.L, 0, sizeof(a.L));
   a.ws = ws;
@@ -501,9 +523,9 @@ int launch_scatter(const __nv_bfloat16* x, const int32_t* perm, int T, int k, in
     if (T > 0) {
       const int64_t want = ((int64_t)T + 7) / 8;
       const int64_t capb = (int64_t)num_sms() * 8;
-      scatter_warp_kernel<<<(int)(want < capb ? want : capb), kScatterThreads, 0, s>>>(
+      scatter_warp_kernel<LocalRows><<<(int)(want < capb ? want : capb), kScatterThreads, 0, s>>>(
           reinterpret_cast<const uint4*>(x), perm, T, k, d / 8, rows_total,
-          reinterpret_cast<uint4*>(recv), err);
+          LocalRows{reinterpret_cast<uint4*>(recv)}, err);
       if (launch_status() != MOE_OK) return MOE_ERR_LAUNCH;
     }
     if (counts != nullptr) {
@@ -564,6 +586,25 @@ int launch_dispatch(const __nv_bfloat16* x, const int32_t* idx, const int32_t* p
   const int st = launch_rank(idx, T, k, E, R, C, 0, plan, &L, ws, perm, src, err, s);
   if (st != MOE_OK || recv == nullptr) return st;  // index-only: the FFN gathers the rows
   return launch_scatter(x, perm, T, k, d, (int64_t)R * C, recv, nullptr, E, 0, nullptr, err, s);
+}
+
+int launch_ep_dispatch(const __nv_bfloat16* x, const int32_t* idx, const int32_t* q_base,
+                       const int32_t* plan, const moe_plan_layout& L, int T, int k, int E,
+                       int W, int d, int32_t* ws, __nv_bfloat16* const* recv_ranks,
+                       int32_t* perm, int32_t* err, cudaStream_t s) {
+  if (T == 0) return MOE_OK;
+  const int C = T * k;  // every rank receives (W*T*k)/W rows
+  const int st = launch_rank(idx, T, k, E, W, C, 0, plan, &L, ws, perm, nullptr, err, s, q_base);
+  if (st != MOE_OK) return st;
+  RankRows dst;
+  for (int u = 0; u < MOE_EP_MAX_RANKS; ++u)
+    dst.base[u] = u < W ? reinterpret_cast<uint4*>(recv_ranks[u]) : nullptr;
+  dst.C = C;
+  const int64_t want = ((int64_t)T + 7) / 8;
+  const int64_t capb = (int64_t)num_sms() * 8;
+  scatter_warp_kernel<RankRows><<<(int)(want < capb ? want : capb), kScatterThreads, 0, s>>>(
+      reinterpret_cast<const uint4*>(x), perm, T, k, d / 8, (int64_t)W * C, dst, err);
+  return launch_status();
 }
 
 int launch_dispatch_capacity(const __nv_bfloat16* x, const int32_t* idx, const int32_t* counts,

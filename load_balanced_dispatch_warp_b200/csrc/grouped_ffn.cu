@@ -1258,4 +1258,13 @@ int launch_grouped_ffn_capacity(const __nv_bfloat16* recv, const __nv_bfloat16* 
                                  s);
 }
 
+int launch_grouped_ffn_groups(const __nv_bfloat16* recv, const int32_t* groups, int G,
+                              int64_t rows, const __nv_bfloat16* W1, const __nv_bfloat16* W3,
+                              const __half* W2, const __nv_bfloat16* P1, const __nv_bfloat16* P3,
+                              const __half* P2, int E, int S, int d, int F, __half* h,
+                              __nv_bfloat16* y, int32_t* err, cudaStream_t s) {
+  return launch_grouped_ffn_impl(recv, nullptr, nullptr, reinterpret_cast<const int4*>(groups), G,
+                                 0, rows, W1, W3, W2, P1, P3, P2, 0, E, 1, S, d, F, h, y, err, s);
+}
+
 }  // namespace moe

@@ -51,6 +51,50 @@ __global__ void __launch_bounds__(kCopyThreads) prefetch_kernel(
   }
 }
 
+// Expert parallelism across GPUs: rank `me` fills its own S pool slots.  Slot s holds
+// expert e = replica_expert[me*S + s], whose weights sit on its home rank e / B as local
+// expert e % B; src* are this process's pointers to every rank's home tensors (a peer
+// GPU's memory mapped here, read over NVLink).  Grid-stride over (slot, projection,
+// chunk); empty slots are skipped.
+struct RankTensors {
+  const uint4* w1[MOE_EP_MAX_RANKS];
+  const uint4* w3[MOE_EP_MAX_RANKS];
+  const uint4* w2[MOE_EP_MAX_RANKS];
+};
+
+__global__ void __launch_bounds__(kCopyThreads) ep_prefetch_kernel(
+    const int32_t* __restrict__ rep, int me, int S, int B, const __grid_constant__ RankTensors src,
+    uint4* __restrict__ P1, uint4* __restrict__ P3, uint4* __restrict__ P2, int64_t vecs,
+    const int32_t* __restrict__ err) {
+  if (load_err(err)) return;
+  const int64_t chunks = (vecs + kCopyChunk - 1) / kCopyChunk;
+  const int64_t total = (int64_t)S * 3 * chunks;
+  for (int64_t w = blockIdx.x; w < total; w += gridDim.x) {
+    const int slot = (int)(w / (3 * chunks));
+    const int64_t rem = w - (int64_t)slot * 3 * chunks;
+    const int proj = (int)(rem / chunks);
+    const int64_t c = rem - (int64_t)proj * chunks;
+    const int e = __ldg(rep + (int64_t)me * S + slot);
+    if (e < 0) continue;
+    const int home = e / B;
+    const uint4* from = (proj == 0 ? src.w1[home] : proj == 1 ? src.w3[home] : src.w2[home]) +
+                        (int64_t)(e - home * B) * vecs;
+    uint4* to = (proj == 0 ? P1 : proj == 1 ? P3 : P2) + (int64_t)slot * vecs;
+    const int64_t v0 = c * kCopyChunk + threadIdx.x;
+    uint4 buf[kCopyVec];
+#pragma unroll
+    for (int i = 0; i < kCopyVec; ++i) {
+      const int64_t v = v0 + i * kCopyThreads;
+      if (v < vecs) buf[i] = __ldcs(from + v);
+    }
+#pragma unroll
+    for (int i = 0; i < kCopyVec; ++i) {
+      const int64_t v = v0 + i * kCopyThreads;
+      if (v < vecs) to[v] = buf[i];
+    }
+  }
+}
+
 constexpr int kRowThreads = 256;
 
 // ----------------------------------------------------------------------------- combine
@@ -80,9 +124,28 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float* a) {
 // to keep the gathers in flight.
 // DROP: an assignment with perm < 0 (dropped by the fixed-capacity dispatch) is left out
 // of the sum.
-template <int K, bool DROP = false, int kCombVec = (K > 4 || K == 0) ? 1 : 2>
+// Src says where row r of y lives: one buffer on this GPU (LocalY), or (expert
+// parallelism across GPUs) rank r / C's y, local row r % C, read through this process's
+// pointer to it (RankY; a peer GPU's memory is read over NVLink).  Both sum the same
+// values in the same order.
+struct LocalY {
+  const uint4* base;
+  __device__ __forceinline__ const uint4* row(int r, int dv) const {
+    return base + (int64_t)r * dv;
+  }
+};
+struct RankY {
+  const uint4* base[MOE_EP_MAX_RANKS];
+  int C;
+  __device__ __forceinline__ const uint4* row(int r, int dv) const {
+    const int u = r / C;
+    return base[u] + (int64_t)(r - u * C) * dv;
+  }
+};
+
+template <int K, bool DROP = false, int kCombVec = (K > 4 || K == 0) ? 1 : 2, class Src = LocalY>
 __global__ void __launch_bounds__(kRowThreads) combine_kernel(
-    const uint4* __restrict__ y, const int32_t* __restrict__ perm,
+    const __grid_constant__ Src y, const int32_t* __restrict__ perm,
     const float* __restrict__ gate, int T, int k, int dv, uint4* __restrict__ out,
     const int32_t* __restrict__ err) {
   if (load_err(err)) return;
@@ -113,7 +176,7 @@ __global__ void __launch_bounds__(kRowThreads) combine_kernel(
 #pragma unroll
           for (int u = 0; u < kCombVec; ++u)
             if (v0 + u * 32 < dv && (!DROP || rows[j] >= 0))
-              buf[j][u] = __ldcs(y + (int64_t)rows[j] * dv + v0 + u * 32);
+              buf[j][u] = __ldcs(y.row(rows[j], dv) + v0 + u * 32);
 #pragma unroll
         for (int j = 0; j < K; ++j)
 #pragma unroll
@@ -133,7 +196,7 @@ __global__ void __launch_bounds__(kRowThreads) combine_kernel(
         for (int j = 0; j < k; ++j) {
           const int row = __shfl_sync(MOE_FULL_MASK, r, j);
           const float gj = __shfl_sync(MOE_FULL_MASK, gl, j);
-          if (v < dv && (!DROP || row >= 0)) acc_bf16x8(acc, __ldcs(y + (int64_t)row * dv + v), gj);
+          if (v < dv && (!DROP || row >= 0)) acc_bf16x8(acc, __ldcs(y.row(row, dv) + v), gj);
         }
         if (v < dv) out[t * dv + v] = pack_bf16x8(acc);
       }
@@ -168,7 +231,7 @@ int launch_combine(const __nv_bfloat16* y, const int32_t* perm, const float* gat
                    int k, int d, __nv_bfloat16* out, const int32_t* err, cudaStream_t s,
                    bool drop) {
   if (T == 0) return MOE_OK;
-  const uint4* yv = reinterpret_cast<const uint4*>(y);
+  const LocalY yv{reinterpret_cast<const uint4*>(y)};
   uint4* ov = reinterpret_cast<uint4*>(out);
   const int g = row_grid(T), dv = d / 8;
   if (drop) {
@@ -197,6 +260,49 @@ int launch_combine(const __nv_bfloat16* y, const int32_t* perm, const float* gat
     default: MOE_COMBINE_CASE(0); break;
   }
 #undef MOE_COMBINE_CASE
+  return launch_status();
+}
+
+int launch_ep_prefetch(const int32_t* plan, const moe_plan_layout& L,
+                       const __nv_bfloat16* const* W1_ranks, const __nv_bfloat16* const* W3_ranks,
+                       const __half* const* W2_ranks, int W, int me, int E, int S, int d, int F,
+                       __nv_bfloat16* P1, __nv_bfloat16* P3, __half* P2, const int32_t* err,
+                       cudaStream_t s) {
+  if (S == 0) return MOE_OK;
+  RankTensors src;
+  for (int u = 0; u < MOE_EP_MAX_RANKS; ++u) {
+    src.w1[u] = u < W ? reinterpret_cast<const uint4*>(W1_ranks[u]) : nullptr;
+    src.w3[u] = u < W ? reinterpret_cast<const uint4*>(W3_ranks[u]) : nullptr;
+    src.w2[u] = u < W ? reinterpret_cast<const uint4*>(W2_ranks[u]) : nullptr;
+  }
+  const int64_t vecs = (int64_t)d * F / 8;
+  ep_prefetch_kernel<<<num_sms() * 4, kCopyThreads, 0, s>>>(
+      plan + L.replica_expert, me, S, E / W, src, reinterpret_cast<uint4*>(P1),
+      reinterpret_cast<uint4*>(P3), reinterpret_cast<uint4*>(P2), vecs, err);
+  return launch_status();
+}
+
+int launch_ep_combine(const __nv_bfloat16* const* y_ranks, int W, const int32_t* perm,
+                      const float* gate, int T, int k, int d, __nv_bfloat16* out,
+                      const int32_t* err, cudaStream_t s) {
+  if (T == 0) return MOE_OK;
+  RankY yv;
+  for (int u = 0; u < MOE_EP_MAX_RANKS; ++u)
+    yv.base[u] = u < W ? reinterpret_cast<const uint4*>(y_ranks[u]) : nullptr;
+  yv.C = T * k;
+  uint4* ov = reinterpret_cast<uint4*>(out);
+  const int g = row_grid(T), dv = d / 8;
+#define MOE_EP_COMBINE(KK) \
+  combine_kernel<KK, false, (KK > 4 || KK == 0) ? 1 : 2, RankY><<<g, kRowThreads, 0, s>>>(yv, perm, gate, T, k, dv, ov, err)
+  switch (k) {
+    case 1: MOE_EP_COMBINE(1); break;
+    case 2: MOE_EP_COMBINE(2); break;
+    case 4: MOE_EP_COMBINE(4); break;
+    case 6: MOE_EP_COMBINE(6); break;
+    case 8: MOE_EP_COMBINE(8); break;
+    default: MOE_EP_COMBINE(0); break;
+  }
+#undef MOE_EP_COMBINE
   return launch_status();
 }
 

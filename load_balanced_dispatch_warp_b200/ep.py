@@ -1,0 +1,260 @@
+"""Expert parallelism across GPUs: the MoE layer with one process per GPU.
+
+Rank ``me`` of ``W`` holds its own ``T`` tokens, the home experts [me*B, (me+1)*B) of the
+E experts (B = E/W), ``S`` pool slots for redundant copies and one static receive buffer of
+C = T*k rows.  A step (the MoonEP news article, paragraphs 2-3; "DeepEP-on-EFA Guidance,
+section 1: What is MoE", phases (a)-(d)):
+
+  1. route its tokens (moe_topk) and pack its demand and error word (moe_ep_counts);
+  2. all-gather those vectors, so every rank computes the same plan of the whole job, its
+     base offsets in every expert's token order, and the job's maxvio (moe_ep_plan);
+  3. pull the weights of its planned replicas from their home ranks (moe_ep_prefetch);
+  4. store every assignment's token row straight into its final row on the rank the plan
+     gives it (moe_ep_dispatch, peer stores);  -- barrier --
+  5. run the grouped FFN on its own C rows (moe_ep_grouped_ffn);  -- barrier --
+  6. gather every one of its tokens' k rows back from the ranks that processed them, with
+     the gate-weighted sum (moe_ep_combine, peer loads).
+The job's token order is rank-major, so the job computes exactly the single-GPU layer of
+the concatenated batch with R = W ranks (the same plan, rows and sums).
+
+Every step runs in the library's kernels; this module only owns buffers and orders the
+calls.  The all-gather and the barriers come from a communicator:
+  - ``NcclComm``: torch.distributed with NCCL (one process per GPU), stream-ordered; the
+    pointer tables through CUDA IPC;
+  - ``GlooComm``: any torch.distributed group (e.g. gloo), synchronising the host at every
+    exchange -- for processes that cannot use NCCL, such as several ranks sharing one GPU;
+  - ``LocalRanks``: W ranks inside one process on one GPU (each rank's buffers are
+    separate allocations; the stages run rank by rank, every rank's dispatch before any
+    rank's FFN, which is the order the barriers give across processes).
+"""
+from __future__ import annotations
+
+import torch
+
+from . import (dispatch_workspace_words, ipc_close, ipc_export, ipc_import, moe_ep_combine,
+               moe_ep_counts, moe_ep_dispatch, moe_ep_grouped_ffn, moe_ep_plan,
+               moe_ep_prefetch, moe_topk, plan_layout)
+
+SHARED = ("recv", "y", "W1", "W3", "W2")  # the buffers every rank addresses on its peers
+
+
+class EPRank:
+    """Buffers and per-step calls of rank ``me`` of ``W``.
+
+    W1, W3 [B,F,d] bf16 and W2 [B,d,F] fp16 are this rank's home experts, on its GPU.
+    ``tables`` (set by the communicator) maps each name in SHARED to the W device
+    pointers of that buffer on every rank, as addressed from this process."""
+
+    def __init__(self, me: int, W: int, T: int, E: int, k: int, S: int, W1, W3, W2):
+        B, F, d = W1.shape
+        if B * W != E:
+            raise ValueError(f"rank holds {B} experts, expected E/W = {E}/{W}")
+        self.me, self.W, self.T, self.E, self.k, self.S = me, W, T, E, k, S
+        self.B, self.F, self.d, self.C = B, F, d, T * k
+        dev = W1.device
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.W1, self.W3, self.W2 = W1, W3, W2
+        self.idx = torch.zeros(T, k, **i32)
+        self.gate = torch.zeros(T, k, dtype=torch.float32, device=dev)
+        self.err = torch.zeros(1, **i32)
+        self.send = torch.zeros(E + 1, **i32)
+        self.gathered = torch.zeros(W, E + 1, **i32)
+        self.counts = torch.zeros(E, **i32)
+        self.q_base = torch.zeros(E, **i32)
+        self.loads = torch.zeros(W, **i32)
+        self.maxvio = torch.zeros(1, dtype=torch.float64, device=dev)
+        self.balancedness = torch.zeros(1, dtype=torch.float64, device=dev)
+        self.plan = torch.zeros(plan_layout(E, W, S).words, **i32)
+        self.ws = torch.zeros(max(1, dispatch_workspace_words(T, E)), **i32)
+        self.perm = torch.zeros(T, k, **i32)
+        self.recv = torch.zeros(self.C, d, dtype=torch.bfloat16, device=dev)
+        self.h = torch.zeros(self.C, F, dtype=torch.float16, device=dev)
+        self.y = torch.zeros(self.C, d, dtype=torch.bfloat16, device=dev)
+        self.out = torch.zeros(T, d, dtype=torch.bfloat16, device=dev)
+        ns = max(S, 1)
+        self.P1 = torch.zeros(ns, F, d, dtype=torch.bfloat16, device=dev)
+        self.P3 = torch.zeros(ns, F, d, dtype=torch.bfloat16, device=dev)
+        self.P2 = torch.zeros(ns, d, F, dtype=torch.float16, device=dev)
+        self.groups_ws = torch.zeros(4 * (B + S), **i32)
+        self.tables = None
+
+    def shared(self) -> dict:
+        return {"recv": self.recv, "y": self.y, "W1": self.W1, "W3": self.W3, "W2": self.W2}
+
+    # ---- the steps, in order
+    def route(self, logits):
+        moe_topk(logits, self.k, self.idx, self.gate, self.err)
+        moe_ep_counts(self.idx, self.E, self.err, self.send)
+
+    def plan_step(self):
+        moe_ep_plan(self.gathered, self.me, self.T, self.k, self.S, self.counts, self.q_base,
+                    self.loads, self.maxvio, self.balancedness, self.plan, self.err)
+
+    def prefetch(self):
+        t = self.tables
+        moe_ep_prefetch(self.plan, t["W1"], t["W3"], t["W2"], self.me, self.E, self.S, self.d,
+                        self.F, self.P1, self.P3, self.P2, self.err)
+
+    def dispatch(self, x):
+        moe_ep_dispatch(x, self.idx, self.q_base, self.plan, self.E, self.S, self.ws,
+                        self.tables["recv"], self.perm, self.err)
+
+    def ffn(self):
+        moe_ep_grouped_ffn(self.recv, self.plan, self.W, self.me, self.W1, self.W3, self.W2,
+                           self.P1, self.P3, self.P2, self.T, self.k, self.E, self.S,
+                           self.groups_ws, self.h, self.y, self.err)
+
+    def combine(self):
+        moe_ep_combine(self.tables["y"], self.perm, self.gate, self.d, self.out, self.err)
+
+
+def exchange_pointers(local: dict, me: int, W: int, gather_objects, export, import_base):
+    """Pointer tables of the buffers in ``local`` ({name: tensor}) on every rank.
+
+    Each rank exports (handle, offset) for each of its buffers; ``gather_objects(obj)``
+    returns every rank's object in rank order (all_gather_object); a peer's allocation is
+    mapped once (``import_base(handle)`` -> base address) however many of its buffers it
+    holds.  Returns ({name: [W pointers]}, [mapped bases, to close])."""
+    mine = {name: export(t) for name, t in local.items()}
+    everyone = gather_objects(mine)
+    if len(everyone) != W:
+        raise RuntimeError(f"pointer exchange: {len(everyone)} ranks answered, expected {W}")
+    mapped = {}
+    tables = {}
+    for name, t in local.items():
+        row = []
+        for u in range(W):
+            if u == me:
+                row.append(int(t.data_ptr()))
+                continue
+            handle, offset = everyone[u][name]
+            key = (u, bytes(handle))
+            if key not in mapped:
+                mapped[key] = import_base(handle)
+            row.append(mapped[key] + int(offset))
+        tables[name] = row
+    return tables, list(mapped.values())
+
+
+def _import_base(handle):
+    ptr, base = ipc_import(handle, 0)
+    return base
+
+
+class _DistComm:
+    def __init__(self, group=None):
+        import torch.distributed as dist
+        self.dist = dist
+        self.group = group
+        self.rank = dist.get_rank(group)
+        self.world = dist.get_world_size(group)
+
+    def _gather_objects(self, obj):
+        out = [None] * self.world
+        self.dist.all_gather_object(out, obj, group=self.group)
+        return out
+
+    def pointer_tables(self, local: dict):
+        return exchange_pointers(local, self.rank, self.world, self._gather_objects, ipc_export,
+                                 _import_base)
+
+
+class NcclComm(_DistComm):
+    """All-gather and barriers on the current stream over an NCCL process group (one
+    process per GPU): the ranks never synchronise the host within a step."""
+
+    def __init__(self, group=None):
+        super().__init__(group)
+        self._word = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def all_gather(self, send, out):
+        self.dist.all_gather_into_tensor(out.view(-1), send, group=self.group)
+
+    def barrier(self):
+        # an all-reduce of one word: no rank's later kernels start before every rank has
+        # finished everything it enqueued before it
+        self.dist.all_reduce(self._word, group=self.group)
+
+
+class GlooComm(_DistComm):
+    """All-gather and barriers through host memory over any process group: each
+    exchange synchronises this process's device first."""
+
+    @staticmethod
+    def _sync():
+        if torch.cuda.is_available() and torch.cuda.is_initialized():
+            torch.cuda.synchronize()
+
+    def all_gather(self, send, out):
+        self._sync()
+        parts = [torch.zeros_like(send, device="cpu") for _ in range(self.world)]
+        self.dist.all_gather(parts, send.cpu(), group=self.group)
+        out.copy_(torch.stack(parts))
+
+    def barrier(self):
+        self._sync()
+        self.dist.barrier(group=self.group)
+
+
+class EPLayer:
+    """One rank of the expert-parallel layer (one process per GPU).
+
+    ``forward(logits, x)`` runs one step on this rank's T tokens and returns its [T,d]
+    output.  Weights are shared with the peers through the pointer tables: a caller that
+    updates them in place must make every rank finish its step first."""
+
+    def __init__(self, comm, T: int, E: int, k: int, S: int, W1, W3, W2):
+        self.comm = comm
+        self.rank = EPRank(comm.rank, comm.world, T, E, k, S, W1, W3, W2)
+        self.rank.tables, self._bases = comm.pointer_tables(self.rank.shared())
+
+    def forward(self, logits, x):
+        r = self.rank
+        r.route(logits)
+        self.comm.all_gather(r.send, r.gathered)
+        r.plan_step()
+        r.prefetch()
+        r.dispatch(x)
+        self.comm.barrier()
+        r.ffn()
+        self.comm.barrier()
+        r.combine()
+        return r.out
+
+    def close(self):
+        """Unmaps the peers' buffers (after every rank has finished its last step)."""
+        for b in self._bases:
+            ipc_close(b)
+        self._bases = []
+
+
+class LocalRanks:
+    """W ranks of the expert-parallel layer inside one process on one GPU.
+
+    Each rank's buffers are separate allocations; the pointer tables hold them directly;
+    the all-gather is a copy of the stacked send vectors; the stages run rank by rank, so
+    every rank's dispatch ends before any rank's FFN and every FFN before any combine,
+    as the barriers order them across processes."""
+
+    def __init__(self, ranks):
+        self.ranks = list(ranks)
+        tables = {name: [int(r.shared()[name].data_ptr()) for r in self.ranks] for name in SHARED}
+        for r in self.ranks:
+            r.tables = tables
+
+    def forward(self, logits_shards, x_shards):
+        for r, lg in zip(self.ranks, logits_shards):
+            r.route(lg)
+        gathered = torch.stack([r.send for r in self.ranks])
+        for r in self.ranks:
+            r.gathered.copy_(gathered)
+            r.plan_step()
+        for r in self.ranks:
+            r.prefetch()
+        for r, x in zip(self.ranks, x_shards):
+            r.dispatch(x)
+        for r in self.ranks:
+            r.ffn()
+        for r in self.ranks:
+            r.combine()
+        return [r.out for r in self.ranks]

@@ -30,6 +30,7 @@ def test_header_declares_the_path(lib):
     assert set(M.VARIANTS) <= names
     assert set(M.FUSED) <= names
     assert set(M.BACKWARD) <= names
+    assert set(M.EXPERT_PARALLEL) <= names
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -215,3 +216,60 @@ def test_fixed_capacity_and_fused_combine_host_checks(lib):
     assert lib.moe_grouped_ffn_combine(*bad) == M.MOE_ERR_ARG
     bad = list(args); bad[5] = None
     assert lib.moe_grouped_ffn_combine(*bad) == M.MOE_ERR_ARG
+
+
+def test_expert_parallel_host_checks(lib):
+    """Host argument rules of the expert-parallel calls and the IPC helpers (nothing is
+    enqueued: every call below fails before any device work)."""
+    P = ctypes.c_void_p
+    fake = P(4096)
+
+    def table(n, addr=4096):
+        return (ctypes.c_void_p * n)(*([addr] * n))
+
+    # counts: null send, k > E
+    assert lib.moe_ep_counts(fake, 4, 2, 8, fake, None, None) == M.MOE_ERR_ARG
+    assert lib.moe_ep_counts(fake, 4, 9, 8, fake, fake, None) == M.MOE_ERR_SHAPE
+    # plan: me outside [0, W), W > 64, E % W, too many groups
+    plan_args = [fake, 2, 0, 16, 2, 8, 2, fake, fake, fake, fake, fake, fake, fake, None]
+    bad = list(plan_args); bad[2] = 2
+    assert lib.moe_ep_plan(*bad) == M.MOE_ERR_ARG
+    bad = list(plan_args); bad[1] = 65; bad[5] = 1040
+    assert lib.moe_ep_plan(*bad) == M.MOE_ERR_SHAPE
+    bad = list(plan_args); bad[1] = 3
+    assert lib.moe_ep_plan(*bad) == M.MOE_ERR_SHAPE
+    bad = list(plan_args); bad[6] = 5000
+    assert lib.moe_ep_plan(*bad) == M.MOE_ERR_SHAPE
+    bad = list(plan_args); bad[12] = None
+    assert lib.moe_ep_plan(*bad) == M.MOE_ERR_ARG
+    # dispatch: a null or misaligned entry in the receive table, W*T*k too big
+    disp = [fake, fake, fake, fake, 2, 16, 2, 8, 2, 128, fake, table(2), fake, fake, None]
+    assert lib.moe_ep_dispatch(*disp[:11], table(2, 0), *disp[12:]) == M.MOE_ERR_ARG
+    assert lib.moe_ep_dispatch(*disp[:11], table(2, 4100), *disp[12:]) == M.MOE_ERR_ARG
+    bad = list(disp); bad[4] = 64; bad[5] = 1 << 24; bad[7] = 64
+    assert lib.moe_ep_dispatch(*bad) == M.MOE_ERR_SHAPE
+    bad = list(disp); bad[2] = None
+    assert lib.moe_ep_dispatch(*bad) == M.MOE_ERR_ARG
+    # prefetch: a short weight table is the caller's contract, a null entry is caught
+    pre = [fake, table(2), table(2), table(2), 2, 1, 8, 2, 128, 256, fake, fake, fake, fake, None]
+    bad = list(pre); bad[2] = table(2, 0)
+    assert lib.moe_ep_prefetch(*bad) == M.MOE_ERR_ARG
+    bad = list(pre); bad[9] = 200
+    assert lib.moe_ep_prefetch(*bad) == M.MOE_ERR_SHAPE
+    # grouped FFN: null group scratch, misaligned h
+    ffn = [fake, fake, 2, 1, fake, fake, fake, fake, fake, fake, 16, 2, 8, 2, 128, 256, fake, fake,
+           fake, fake, None]
+    bad = list(ffn); bad[16] = None
+    assert lib.moe_ep_grouped_ffn(*bad) == M.MOE_ERR_ARG
+    bad = list(ffn); bad[17] = P(4098)
+    assert lib.moe_ep_grouped_ffn(*bad) == M.MOE_ERR_ARG
+    # combine: W = 0, k > 32, null table entry
+    assert lib.moe_ep_combine(table(2), fake, fake, 0, 16, 2, 128, fake, fake, None) == M.MOE_ERR_ARG
+    assert lib.moe_ep_combine(table(2), fake, fake, 2, 16, 33, 128, fake, fake, None) == M.MOE_ERR_SHAPE
+    assert lib.moe_ep_combine(table(2, 0), fake, fake, 2, 16, 2, 128, fake, fake, None) == M.MOE_ERR_ARG
+    # IPC helpers: null arguments; a host address is not a device allocation
+    off = ctypes.c_int64(0)
+    h = ctypes.create_string_buffer(M.IPC_HANDLE_BYTES)
+    assert lib.moe_ipc_export(None, h, ctypes.byref(off)) == M.MOE_ERR_ARG
+    assert lib.moe_ipc_import(h, -1, ctypes.byref(P()), ctypes.byref(P())) == M.MOE_ERR_ARG
+    assert lib.moe_ipc_close(None) == M.MOE_ERR_ARG

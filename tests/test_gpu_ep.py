@@ -1,0 +1,233 @@
+"""Expert parallelism across GPUs on one B200.
+
+W ranks run inside one process (``LocalRanks``): each rank's buffers are separate
+allocations, addressed by its peers through the pointer tables, and the stages run rank by
+rank in the order the barriers give across processes.  Checked against the oracle's
+W-process layer (bit-exact integers and rows, the FFN tolerance on y and out) and, bit for
+bit, against the single-GPU layer of the concatenated batch with R = W at full workload
+sizes.  A last case runs two real processes on the one GPU, each rank mapping the other's
+buffers through CUDA IPC, with the exchange over gloo."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+
+import load_balanced_dispatch_warp_b200 as M
+from harness import assert_close_scaled, make_inputs, oracle_plan_fields, to64
+from load_balanced_dispatch_warp_b200 import inputs as I
+from load_balanced_dispatch_warp_b200.ep import EPRank, LocalRanks
+from oracle import moe_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+
+def make_ranks(w, weights):
+    W1, W3, W2 = weights
+    W, B, T = w.R, w.E // w.R, w.T // w.R
+    return LocalRanks([EPRank(u, W, T, w.E, w.k, w.S, W1[u * B:(u + 1) * B],
+                              W3[u * B:(u + 1) * B], W2[u * B:(u + 1) * B]) for u in range(W)])
+
+
+def shards(t, W):
+    T = t.shape[0] // W
+    return [t[u * T:(u + 1) * T].contiguous() for u in range(W)]
+
+
+def plan_fields(r, E, W, S):
+    L = M.plan_layout(E, W, S)
+    sizes = dict(kept_rows=W, room_prefix=W + 1, expert_home_off=E, stream_off=E + 1,
+                 replica_expert=W * S, replica_list=1 + W * S, n_groups=W,
+                 groups=W * L.max_groups_per_rank * 4)
+    return {n: r.plan[getattr(L, n):getattr(L, n) + sz].cpu().numpy() for n, sz in sizes.items()}
+
+
+# (name, T, E, k, W, S, d, F): W = 1 (the single-GPU layer), a ragged last tile, top-3,
+# several tiles per rank, 8 ranks of 8 experts
+SMALL = [("ep_w1", 64, 8, 2, 1, 2, 128, 256), ("ep_w2", 96, 8, 2, 2, 4, 128, 256),
+         ("ep_w4", 256, 16, 4, 4, 4, 256, 128), ("ep_w4_k3", 200, 32, 3, 4, 6, 128, 384),
+         ("ep_w8", 512, 64, 6, 8, 8, 256, 256), ("ep_w2_tiles", 1200, 8, 2, 2, 3, 128, 128)]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+def test_ep_ranks_match_the_oracle(case):
+    w = I.small_workload(*case, alpha=1.2)
+    W = w.R
+    logits, x, weights = make_inputs(w)
+    lr = make_ranks(w, weights)
+    lr.forward([s.cuda() for s in shards(logits, W)], [s.cuda() for s in shards(x, W)])
+    torch.cuda.synchronize()
+    w64 = tuple(to64(t) for t in weights)
+    ref = O.ep_layer(np.split(logits.numpy(), W), np.split(to64(x), W), *w64, w.k, w.S)
+    assert ref["err"] == 0
+    idx_all = np.concatenate([rr["idx"] for rr in ref["ranks"]])
+    hist = O.expert_histogram(idx_all, w.E, W)
+    expect_plan = oracle_plan_fields(ref["plan"], w)
+    for u, r in enumerate(lr.ranks):
+        rr = ref["ranks"][u]
+        assert int(r.err.item()) == 0
+        assert np.array_equal(r.idx.cpu().numpy(), rr["idx"])
+        assert np.abs(r.gate.cpu().double().numpy() - rr["gate"]).max() <= 1e-6
+        assert np.array_equal(r.send.cpu().numpy(), np.append(ref["counts_all"][u], 0))
+        assert np.array_equal(r.counts.cpu().numpy(), ref["counts_all"].sum(axis=0))
+        assert np.array_equal(r.q_base.cpu().numpy(), O.ep_rank_base(ref["counts_all"], u))
+        assert np.array_equal(r.loads.cpu().numpy(), hist["loads"])
+        assert r.maxvio.item() == hist["maxvio"] and r.balancedness.item() == hist["balancedness"]
+        got = plan_fields(r, w.E, W, w.S)
+        for name, v in expect_plan.items():
+            assert np.array_equal(got[name], v), f"rank {u} plan field {name}"
+        assert np.array_equal(r.perm.cpu().numpy(), rr["perm"]), f"rank {u} perm"
+        assert np.array_equal(to64(r.recv), rr["recv"]), f"rank {u} receive rows"
+        for s in range(w.S):
+            e = ref["plan"]["replica_expert"][u * w.S + s]
+            if e >= 0:
+                assert torch.equal(r.P1[s], weights[0][e]) and torch.equal(r.P3[s], weights[1][e])
+                assert torch.equal(r.P2[s], weights[2][e])
+        assert_close_scaled(to64(r.y), rr["y"], f"rank {u} y")
+        assert_close_scaled(to64(r.out), rr["out"], f"rank {u} out")
+
+
+FULL = ["near_balanced", "qwen_mv1", "mixtral", "deepseek"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_ep_is_the_single_gpu_layer_bit_for_bit(name):
+    """W = R ranks on the workload's shards against MoELayer on the whole batch: the same
+    plan, rows, y and out, bit for bit."""
+    w = I.WORKLOADS[name]
+    W = w.R
+    logits, x, weights = make_inputs(w)
+    lg, xd = logits.cuda(), x.cuda()
+    L = M.MoELayer(w.T, w.E, w.k, w.R, w.S, w.d, w.F)
+    L.forward(lg, xd, *weights)
+    lr = make_ranks(w, weights)
+    lr.forward(shards(lg, W), shards(xd, W))
+    torch.cuda.synchronize()
+    assert int(L.err.item()) == 0
+    C = w.C
+    for u, r in enumerate(lr.ranks):
+        assert int(r.err.item()) == 0
+        assert torch.equal(r.plan, L.plan), f"rank {u} plan"
+        assert torch.equal(r.counts, L.counts) and torch.equal(r.loads, L.loads)
+        assert r.maxvio.item() == L.maxvio.item()
+        assert torch.equal(r.perm, L.perm[u * r.T:(u + 1) * r.T]), f"rank {u} perm"
+        assert torch.equal(r.recv, L.recv[u * C:(u + 1) * C]), f"rank {u} receive rows"
+        assert torch.equal(r.y, L.y[u * C:(u + 1) * C]), f"rank {u} y"
+        assert torch.equal(r.out, L.out[u * r.T:(u + 1) * r.T]), f"rank {u} out"
+
+
+def test_ep_error_on_one_rank_stops_every_rank():
+    """A non-finite logit on rank 1 reaches every rank through the exchanged vectors."""
+    w = I.small_workload("ep_err", 64, 8, 2, 2, 2, 128, 128)
+    logits, x, weights = make_inputs(w)
+    logits[40, 3] = float("nan")
+    lr = make_ranks(w, weights)
+    lr.forward([s.cuda() for s in shards(logits, 2)], [s.cuda() for s in shards(x, 2)])
+    torch.cuda.synchronize()
+    for r in lr.ranks:
+        assert int(r.err.item()) & M.DERR_NONFINITE
+    assert int(lr.ranks[1].send[-1].item()) & M.DERR_NONFINITE
+    assert int(lr.ranks[0].send[-1].item()) == 0
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+IPC_CASE = ("ep_ipc", 256, 16, 4, 2, 4, 256, 256)
+
+
+def _ipc_worker(rank, world, port, path):
+    import torch.distributed as dist
+    from load_balanced_dispatch_warp_b200.ep import EPLayer, GlooComm
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        torch.cuda.set_device(0)
+        w = I.small_workload(*IPC_CASE, alpha=1.2)
+        logits, x, weights = make_inputs(w)
+        B, T = w.E // world, w.T // world
+        own = tuple(t[rank * B:(rank + 1) * B].contiguous() for t in weights)
+        layer = EPLayer(GlooComm(), T, w.E, w.k, w.S, *own)
+        out = layer.forward(shards(logits, world)[rank].cuda(), shards(x, world)[rank].cuda())
+        torch.cuda.synchronize()
+        torch.save({"out": out.cpu(), "err": int(layer.rank.err.item()),
+                    "perm": layer.rank.perm.cpu()}, f"{path}.{rank}")
+        dist.barrier()  # no rank unmaps or frees while a peer may still read its buffers
+        layer.close()
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ep_two_processes_through_ipc(tmp_path):
+    """Two processes on the one GPU, each a rank holding its own buffers, its peer's
+    receive buffer, y and weights mapped through CUDA IPC: the result equals the one-process
+    ranks bit for bit."""
+    import torch.multiprocessing as mp
+    if not _gpu_compute_mode_default():
+        pytest.skip("two processes on one GPU need the Default compute mode")
+    world = 2
+    path = str(tmp_path / "ep_out")
+    mp.spawn(_ipc_worker, args=(world, _free_port(), path), nprocs=world, join=True)
+    w = I.small_workload(*IPC_CASE, alpha=1.2)
+    logits, x, weights = make_inputs(w)
+    lr = make_ranks(w, weights)
+    lr.forward([s.cuda() for s in shards(logits, world)], [s.cuda() for s in shards(x, world)])
+    torch.cuda.synchronize()
+    for u in range(world):
+        got = torch.load(f"{path}.{u}")
+        assert got["err"] == 0
+        assert torch.equal(got["perm"], lr.ranks[u].perm.cpu())
+        assert torch.equal(got["out"], lr.ranks[u].out.cpu()), f"rank {u} out"
+
+
+def _gpu_compute_mode_default():
+    import subprocess
+    try:
+        out = subprocess.run(["nvidia-smi", "--query-gpu=compute_mode", "--format=csv,noheader",
+                              "-i", "0"], capture_output=True, text=True, timeout=30).stdout
+    except (OSError, subprocess.SubprocessError):
+        return False
+    return out.strip() == "Default"
+
+
+def _nccl_worker(rank, world, port, path):
+    import torch.distributed as dist
+    from load_balanced_dispatch_warp_b200.ep import EPLayer, NcclComm
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    torch.cuda.set_device(0)
+    dist.init_process_group("nccl", rank=rank, world_size=world,
+                            device_id=torch.device("cuda", 0))
+    try:
+        w = I.small_workload(*IPC_CASE[:4], 1, *IPC_CASE[5:], alpha=1.2)
+        logits, x, weights = make_inputs(w)
+        layer = EPLayer(NcclComm(), w.T, w.E, w.k, w.S, *weights)
+        for _ in range(2):  # a second step reuses every buffer
+            out = layer.forward(logits.cuda(), x.cuda())
+        torch.cuda.synchronize()
+        torch.save({"out": out.cpu(), "err": int(layer.rank.err.item())}, path)
+        layer.close()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ep_nccl_communicator_single_rank(tmp_path):
+    """The NCCL communicator's all-gather and barriers on a one-rank group: the layer's
+    output equals the single-GPU layer's, bit for bit."""
+    import torch.multiprocessing as mp
+    path = str(tmp_path / "ep_nccl")
+    mp.spawn(_nccl_worker, args=(1, _free_port(), path), nprocs=1, join=True)
+    w = I.small_workload(*IPC_CASE[:4], 1, *IPC_CASE[5:], alpha=1.2)
+    logits, x, weights = make_inputs(w)
+    L = M.MoELayer(w.T, w.E, w.k, w.R, w.S, w.d, w.F)
+    L.forward(logits.cuda(), x.cuda(), *weights)
+    torch.cuda.synchronize()
+    got = torch.load(path)
+    assert got["err"] == 0
+    assert torch.equal(got["out"], L.out.cpu())
