@@ -532,6 +532,166 @@ def run_ours(args, w: I.Workload, world, rank, local):
     return res
 
 
+def run_ep(args, w: I.Workload, world, rank, local):
+    """Expert parallelism across GPUs (``--ep``).  N = 1: the workload's R ranks run in one
+    process on this GPU (each rank's buffers separate allocations, the pointer tables
+    standing in for peer mappings, the all-gather a device copy); the timed K steps are
+    captured in one CUDA graph, and a second capture with event nodes between the stages
+    gives each stage's time.  N > 1: one rank per GPU (R = N) over NCCL with the peers'
+    buffers mapped through CUDA IPC, the workload's T tokens split over the ranks
+    (strong scaling), K eager steps between barriers, max over ranks."""
+    import load_balanced_dispatch_warp_b200 as M
+    from load_balanced_dispatch_warp_b200.ep import EPLayer, EPRank, LocalRanks, NcclComm
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    peaks, peak_src = load_peaks()
+    stream = torch.cuda.current_stream(device)
+    W = w.R if world == 1 else world
+    if w.E % W or w.T % W:
+        raise SystemExit(f"--ep: {w.name} cannot be split over {W} ranks (E={w.E}, T={w.T})")
+    B, Tl = w.E // W, w.T // W
+    logits = I.make_logits(w).to(device)
+    x = I.make_x(w).to(device)
+    W1, W3, W2 = I.make_weights(w, device=device)
+
+    def shard(t, u):
+        return t[u * Tl:(u + 1) * Tl].contiguous()
+
+    stages = None
+    if world == 1:
+        lr = LocalRanks([EPRank(u, W, Tl, w.E, w.k, w.S, W1[u * B:(u + 1) * B],
+                                W3[u * B:(u + 1) * B], W2[u * B:(u + 1) * B]) for u in range(W)])
+        stages = lr.stages([shard(logits, u) for u in range(W)], [shard(x, u) for u in range(W)])
+        ranks = lr.ranks
+
+        def step():
+            for _, f in stages:
+                f()
+    else:
+        own = tuple(t[rank * B:(rank + 1) * B].contiguous() for t in (W1, W3, W2))
+        del W1, W3, W2
+        torch.cuda.empty_cache()
+        layer = EPLayer(NcclComm(), Tl, w.E, w.k, w.S, *own)
+        lg, xs = shard(logits, rank), shard(x, rank)
+        ranks = [layer.rank]
+
+        def step():
+            layer.forward(lg, xs)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    errs = [int(r.err.item()) for r in ranks]
+    if any(errs):
+        raise RuntimeError(f"{w.name}: device error words {errs} after warm-up")
+    n_rep = int(ranks[0].plan[M.plan_layout(w.E, W, w.S).replica_list].item())
+    steps = args.steps
+    stage_ms = None
+    if world == 1:
+        rec_node = rec_node_fn()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
+              for _ in range(steps)]
+        for e in [e for row in ev for e in row]:
+            e.record(stream)
+        torch.cuda.synchronize()
+
+        def capture(with_events):
+            g = torch.cuda.CUDAGraph()
+            cap = torch.cuda.Stream(device)
+            cap.wait_stream(stream)
+            torch.cuda.synchronize()
+            with torch.cuda.stream(cap):
+                g.capture_begin()
+                for si in range(steps):
+                    if with_events:
+                        rec_node(ev[si][0], cap)
+                    for i, (_, f) in enumerate(stages):
+                        f()
+                        if with_events:
+                            rec_node(ev[si][i + 1], cap)
+                g.capture_end()
+            torch.cuda.synchronize()
+            g.replay()
+            torch.cuda.synchronize()
+            return g
+        graph, graph_ev = capture(False), capture(True)
+    clocks = ClockSampler(device.index)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    if world == 1:
+        graph.replay()
+    else:
+        for _ in range(steps):
+            step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    elapsed_ms = t0.elapsed_time(t1)
+    if world == 1:
+        graph_ev.replay()
+        torch.cuda.synchronize()
+        stage_ms = {name: sum(ev[si][i].elapsed_time(ev[si][i + 1]) for si in range(steps)) / steps
+                    for i, (name, _) in enumerate(stages)}
+    clk = clocks.stop()
+    elapsed_ms = max_over_ranks(elapsed_ms, world, device)
+    errs = [int(r.err.item()) for r in ranks]
+    if any(errs):
+        raise RuntimeError(f"{w.name}: device error words {errs} in the timed region")
+    row_bytes = w.d * 2
+    work = {"dispatch": (w.T + w.A) * row_bytes, "combine": (w.A + w.T) * row_bytes,
+            "prefetch": 2 * n_rep * 3 * w.d * w.F * 2, "ffn": 6 * w.A * w.d * w.F}
+    ffn_peak_v, ffn_src = ffn_peak(clk, peaks, peak_src)
+    res = {
+        "metric": METRIC, "value": round(w.T * steps / (elapsed_ms * 1e-3), 1), "unit": UNIT,
+        "n_gpus": world, "steps": steps, "warmup": args.warmup,
+        "ms_per_step": round(elapsed_ms / steps, 4), "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None,
+        "dtype": "bf16+fp16 (gate/up GEMM bf16, down GEMM fp16, fp32 accumulate; routing fp32)",
+        "data": "synthetic (seeded; N(0,1) logits + per-expert bias, N(0,1) tokens, N(0,1/d) weights)",
+        "config": {"workload": w.name, "T": w.T, "E": w.E, "k": w.k, "R": W, "S": w.S, "d": w.d,
+                   "F": w.F, "tokens_per_rank": Tl, "replicas": n_rep,
+                   "parallelism": (f"ep{W}: {W} ranks in one process on one GPU (local buffers "
+                                   "through the pointer tables stand in for peer mappings)"
+                                   if world == 1 else
+                                   f"ep{W}: one rank per GPU, NCCL all-gather and barriers, "
+                                   "peer buffers through CUDA IPC"),
+                   "l2": "inputs larger than L2 (weights, pool, activations), no flush",
+                   "launch": ("K steps of every rank's stages captured in one CUDA graph"
+                              if world == 1 else "eager, K steps between barriers")},
+        "clocks": clk,
+        "e2e": None,
+        # per rank and step: top-k, counts, plan, prefetch, dispatch rank pass and row
+        # stores, group table, GEMM 1, GEMM 2, combine
+        "gpu_launches": 10 * len(ranks) * steps,
+    }
+    if stage_ms is not None:
+        st = {}
+        for name, ms in stage_ms.items():
+            row = {"us": round(ms * 1e3, 2)}
+            if name in ("dispatch", "combine", "prefetch") and ms > 0:
+                gbs = work[name] / (ms * 1e-3) / 1e9
+                row.update(GB_per_s=round(gbs, 1), frac=round(gbs / peaks["hbm_gbs"], 3))
+            if name == "ffn" and ms > 0:
+                tf = work["ffn"] / (ms * 1e-3) / 1e12
+                row.update(TFLOP_per_s=round(tf, 1), frac=round(tf / ffn_peak_v, 3),
+                           peak_source=ffn_src)
+            st[name] = row
+        res["ep_stages"] = st
+        res["roofline"] = {"bound": "tensor", "achieved": st["ffn"].get("TFLOP_per_s"),
+                           "peak": ffn_peak_v, "unit": "TFLOP/s", "frac": st["ffn"].get("frac"),
+                           "traffic": None, "kernel": "moe_ep_grouped_ffn, all ranks",
+                           "peak_source": ffn_src}
+    if world > 1:
+        layer.close()
+    return res
+
+
 def run_only(args, w: I.Workload):
     """One call of the path on its own, repeated `--steps` times between CUDA events after
     `--warmup` calls: the case for kernel-level counter captures (ncu), which must stay a
@@ -822,6 +982,9 @@ def main():
     ap.add_argument("--fused-combine", action="store_true",
                     help="fused combine: GEMM 2's epilogue adds the gate-weighted rows into an "
                          "fp32 output (atomics), no y buffer and no combine kernel")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert parallelism across GPUs: one rank per GPU (R = N) for N > 1; "
+                         "at N = 1 the workload's R ranks in one process on this GPU")
     ap.add_argument("--ffn-tile", type=int, default=None, choices=[0, 1],
                     help="grouped-FFN tiling: 0 = 128-row tiles, one CTA each; 1 = 256-row "
                          "tiles on 2-CTA clusters (default: the library's)")
@@ -844,8 +1007,11 @@ def main():
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    res = run_ours(args, w, world, rank, local)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if args.ep:
+        res = run_ep(args, w, world, rank, local)
+    else:
+        res = run_ours(args, w, world, rank, local)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.ep:
         value, Ts, n, dt = measure_oracle(w, steps=1000, warmup=1, budget_s=15.0)
         res["cpu_baseline"] = {"value": round(value, 3), "unit": UNIT, "cores": cpu_threads(),
                                "kind": "oracle",

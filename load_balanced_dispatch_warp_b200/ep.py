@@ -242,19 +242,40 @@ class LocalRanks:
         for r in self.ranks:
             r.tables = tables
 
+    def stages(self, logits_shards, x_shards):
+        """The step as (name, callable) pairs, each running one stage on every rank."""
+        ranks = self.ranks
+
+        def route():
+            for r, lg in zip(ranks, logits_shards):
+                r.route(lg)
+
+        def plan():
+            gathered = torch.stack([r.send for r in ranks])  # the all-gather
+            for r in ranks:
+                r.gathered.copy_(gathered)
+                r.plan_step()
+
+        def prefetch():
+            for r in ranks:
+                r.prefetch()
+
+        def dispatch():
+            for r, x in zip(ranks, x_shards):
+                r.dispatch(x)
+
+        def ffn():
+            for r in ranks:
+                r.ffn()
+
+        def combine():
+            for r in ranks:
+                r.combine()
+
+        return [("route", route), ("plan", plan), ("prefetch", prefetch), ("dispatch", dispatch),
+                ("ffn", ffn), ("combine", combine)]
+
     def forward(self, logits_shards, x_shards):
-        for r, lg in zip(self.ranks, logits_shards):
-            r.route(lg)
-        gathered = torch.stack([r.send for r in self.ranks])
-        for r in self.ranks:
-            r.gathered.copy_(gathered)
-            r.plan_step()
-        for r in self.ranks:
-            r.prefetch()
-        for r, x in zip(self.ranks, x_shards):
-            r.dispatch(x)
-        for r in self.ranks:
-            r.ffn()
-        for r in self.ranks:
-            r.combine()
+        for _, f in self.stages(logits_shards, x_shards):
+            f()
         return [r.out for r in self.ranks]
