@@ -348,16 +348,19 @@ int moe_combine_backward(const moe_bf16* dout, const moe_bf16* y, const int32_t*
  *   dW2[e] = sum over ALL groups of e (home and replica) of dY^T h, dW1[e] = sum dG^T X,
  *   dW3[e] = sum dU^T X -- replica gradients reduced home; experts without rows get 0.
  *   recv [R*C,d] bf16 (from moe_dispatch); dy [R*C,d] bf16 (moe_combine_backward);
- *   h [R*C,F] fp16 (from moe_grouped_ffn); W1, W3 [E,F,d] bf16; W2 [E,d,F] fp16.
- *   All GEMMs run in bf16 with fp32 accumulation: W2 and h are rounded to bf16 on the way
- *   into the transposed operands (exact for W2 values that are bf16 numbers).
+ *   h [R*C,F] fp16: the forward's activations (from moe_grouped_ffn); not read (may be
+ *   NULL): the SwiGLU-backward epilogue recomputes h = silu(g) u from the re-run gate/up
+ *   GEMM and keeps it in bf16 for dW2.  W1, W3 [E,F,d] bf16; W2 [E,d,F] fp16.
+ *   All GEMMs run in bf16 with fp32 accumulation: W2 is rounded to bf16 on the way into its
+ *   transposed copy (exact for W2 values that are bf16 numbers).
  *   dx_rows [R*C,d] bf16 (out); dW1, dW3 [E,F,d] fp32 (out); dW2 [E,d,F] fp32 (out).
  *   workspace: caller-owned device scratch of moe_ffn_backward_workspace_bytes(...) bytes,
- *   256-byte aligned (transposed weights and activations, dH fp32, dG|dU bf16).
+ *   256-byte aligned (W2 transposed in bf16, dH fp32, dG|dU and h bf16, the per-expert
+ *   group lists).
  *   Returns MOE_ERR_ARG if workspace_bytes is too small.  Persistent tcgen05 kernels:
  *   dH, dG|dU (the gate/up GEMM re-run with a SwiGLU-backward epilogue), dX rows, and one
- *   weight-gradient GEMM per projection whose K loop runs over the zero-padded 64-row
- *   segments of every group of the expert.
+ *   weight-gradient GEMM per projection whose K loop runs over the rows of every group of
+ *   the expert, 64 at a time, reading the row-major activations as MN-major operands.
  */
 int64_t moe_ffn_backward_workspace_bytes(int T, int k, int E, int R, int S, int d, int F);
 int moe_grouped_ffn_backward(const moe_bf16* recv, const moe_bf16* dy, const moe_f16* h,

@@ -429,7 +429,7 @@ int moe_grouped_ffn_backward(const moe_bf16* recv, const moe_bf16* dy, const moe
                              void* workspace, int64_t workspace_bytes, int32_t* err,
                              moe_stream_t stream) {
   if (!plan || !W1 || !W3 || !W2 || !err || !dW1 || !dW3 || !dW2) return MOE_ERR_ARG;
-  if (T > 0 && (!recv || !dy || !h || !dx_rows || !workspace)) return MOE_ERR_ARG;
+  if (T > 0 && (!recv || !dy || !dx_rows || !workspace)) return MOE_ERR_ARG;  // h may be NULL
   MOE_TRY(check_route(T, E, k));
   MOE_TRY(check_ranks(T, k, E, R, true));
   MOE_TRY(check_groups(E, R, S));

@@ -17,11 +17,15 @@
 // All GEMMs run on one persistent tcgen05 kernel (TMA-fed 4-stage ring, TMEM double
 // buffer, one MMA thread, four epilogue warps) with three epilogues, in bf16: dY is bf16
 // because gate * dout spans the gates' range (fp16 would lose small gates to subnormals),
-// and the fp16 operands it meets (W2, the forward's h) are converted to bf16 by the
-// transposes below.  The dX GEMM reads W1 and W3 as they are stored (MN-major B
-// operand); the dH GEMM reads W2 transposed to bf16, and the weight-gradient GEMMs read
-// dY, h, dG, dU and X transposed by an HBM-bound kernel into a layout that gives every
-// group a segment of whole 64-row K steps, zero-padded, so no K step mixes two groups.
+// and the fp16 operand it meets in dH (W2) is converted to bf16 by a transpose.  The dX
+// GEMM reads W1 and W3 as they are stored (MN-major B operand).  The weight-gradient
+// GEMMs read dY, h, dG | dU and X as the forward and the other GEMMs left them, row-major
+// [rows, columns] with the K dimension (rows) outermost: both operands MN-major.  Their K
+// steps walk each group of the expert 64 rows at a time; in a group's last, partial step
+// the rows past the group's end belong to the next group, and the MMA warp zeroes them in
+// the A tile (whole 128-byte rows of the swizzled box) before the MMAs read it.  h is
+// recomputed in the SwiGLU-backward epilogue (silu(g) * u from the re-run gate/up GEMM)
+// and stored as bf16, the type dY needs its partner to have.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -58,12 +62,15 @@ struct BwdArgs {
   void* out;
   int32_t* err;
   // SwiGLU backward epilogue: reads dH [rows, F] fp32, writes dG | dU into dGU [rows, 2F]
+  // and h = silu(g) * u into hb [rows, F] (bf16)
   const float* dh;
   __nv_bfloat16* dgu;
+  __nv_bfloat16* hb;
   int F;
-  // weight-gradient tiles: (expert, m block, n block), K over the expert's segments
+  // weight-gradient tiles: (expert, m block, n block), K over the rows of the expert's
+  // groups; A and B are row-major activations read MN-major (column a_row, b_row)
   const int* seg_off;   // [E+1]
-  const int2* segs;     // {first K step, K steps}
+  const int2* segs;     // {row_start, rows} of each group of the expert
   int m_blocks;
   int a_row_base;
   int64_t out_expert_stride;
@@ -177,11 +184,13 @@ __device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr) {
          ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 // kind::f16 instruction descriptor: fp32 accumulate, A and B bf16 (1) or fp16 (0), A
-// K-major, B K-major (0) or MN-major (1) at bit 16, N >> 3 at bits 17-22, M >> 4 at bits
-// 24-28.
-__device__ __forceinline__ uint32_t make_idesc(int M, int N, bool bf16, bool b_mn) {
+// K-major (0) or MN-major (1) at bit 15, B likewise at bit 16, N >> 3 at bits 17-22,
+// M >> 4 at bits 24-28.
+__device__ __forceinline__ uint32_t make_idesc(int M, int N, bool bf16, bool b_mn,
+                                               bool a_mn = false) {
   return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) |
-         ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+         ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
 }
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
@@ -237,19 +246,20 @@ __device__ __forceinline__ BTile decode(int t, const BwdArgs& a, const int* s_pr
   return tl;
 }
 
-// K steps of a tile, in order: row tiles 0..k_blocks-1; weight-gradient tiles the
-// concatenated segments of the expert.
+// K steps of a tile, in order, as f(k, valid): row tiles f(kb, BK) for kb = 0..k_blocks-1;
+// weight-gradient tiles f(first row, rows of the group in the step) for every 64 rows of
+// every group of the expert (valid < BK only in a group's last step).
 template <bool WGRAD, class F>
 __device__ __forceinline__ bool for_k(const BTile& tl, const BwdArgs& a, F&& f) {
   if (WGRAD) {
     for (int s = tl.seg_lo; s < tl.seg_hi; ++s) {
       const int2 sg = __ldg(a.segs + s);
-      for (int kb = sg.x; kb < sg.x + sg.y; ++kb)
-        if (!f(kb)) return false;
+      for (int r = 0; r < sg.y; r += BK)
+        if (!f(sg.x + r, min(BK, sg.y - r))) return false;
     }
   } else {
     for (int kb = 0; kb < a.k_blocks; ++kb)
-      if (!f(kb)) return false;
+      if (!f(kb, BK)) return false;
   }
   return true;
 }
@@ -334,23 +344,32 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       uint32_t issued_mask = 0, issued_phase = 0;
       for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
         const BTile tl = decode<WGRAD>(t, args, s_prefix);
-        const bool ok = for_k<WGRAD>(tl, args, [&](int kb) {
+        const bool ok = for_k<WGRAD>(tl, args, [&](int kb, int) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, args.err)) return false;
           const uint32_t fb = full0 + 8 * stage;
           const uint32_t sa = smem_u32(stage_base + stage * STAGE_BYTES);
           const uint32_t sb = sa + A_BYTES;
           mbar_expect_tx(fb, A_BYTES + b_bytes);
-          tma_load_2d(sa, &tm_a, fb, kb * BK, tl.a_row);
-          if (BMN) {
-            // B [N][K] read from a tensor stored K-row major: boxes of 64 K rows x 64 N
-            const bool lo = kb < args.kb_split;
-            const int krow = tl.e * args.rows_per_expert + (lo ? kb : kb - args.kb_split) * BK;
-            const int n0 = tl.n_block * args.bn_out;
+          if (WGRAD) {
+            // kb is the step's first row: boxes of 64 rows x 64 columns of the row-major
+            // activations, A columns a_row.. (M), B columns b_row.. (N)
+            for (int c = 0; c < BM / 64; ++c)
+              tma_load_2d(sa + c * 8192, &tm_a, fb, tl.a_row + c * 64, kb);
             for (int c = 0; c < args.mma_n / 64; ++c)
-              tma_load_2d(sb + c * 8192, lo ? &tm_b0 : &tm_b1, fb, n0 + c * 64, krow);
+              tma_load_2d(sb + c * 8192, &tm_b0, fb, tl.b_row + c * 64, kb);
           } else {
-            tma_load_2d(sb, &tm_b0, fb, kb * BK, tl.b_row);
-            if (TWO_B) tma_load_2d(sb + (b_bytes >> 1), &tm_b1, fb, kb * BK, tl.b_row);
+            tma_load_2d(sa, &tm_a, fb, kb * BK, tl.a_row);
+            if (BMN) {
+              // B [N][K] read from a tensor stored K-row major: boxes of 64 K rows x 64 N
+              const bool lo = kb < args.kb_split;
+              const int krow = tl.e * args.rows_per_expert + (lo ? kb : kb - args.kb_split) * BK;
+              const int n0 = tl.n_block * args.bn_out;
+              for (int c = 0; c < args.mma_n / 64; ++c)
+                tma_load_2d(sb + c * 8192, lo ? &tm_b0 : &tm_b1, fb, n0 + c * 64, krow);
+            } else {
+              tma_load_2d(sb, &tm_b0, fb, kb * BK, tl.b_row);
+              if (TWO_B) tma_load_2d(sb + (b_bytes >> 1), &tm_b1, fb, kb * BK, tl.b_row);
+            }
           }
           issued_mask |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
@@ -368,40 +387,65 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = make_idesc(BM, args.mma_n, args.bf16 != 0, BMN);
+    // Lane 0 issues.  Weight-gradient tiles run the loop on the whole warp: in a group's
+    // last, partial K step the warp zeroes the A rows past the group's end (they hold the
+    // next group's values) after the TMA has landed and before the MMAs read the stage.
+    if (WGRAD || lane == 0) {
+      const uint32_t idesc = make_idesc(BM, args.mma_n, args.bf16 != 0, BMN || WGRAD, WGRAD);
+      const bool issuer = !WGRAD || lane == 0;
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
         const BTile tl = decode<WGRAD>(t, args, s_prefix);
-        if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag, args.err)) break;
+        bool okt = mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag, args.err);
+        if (WGRAD) okt = __all_sync(MOE_FULL_MASK, okt);
+        if (!okt) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
         bool first = true;
-        const bool ok = for_k<WGRAD>(tl, args, [&](int) {
-          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, args.err)) return false;
+        const bool ok = for_k<WGRAD>(tl, args, [&](int, int valid) {
+          bool okf = mbar_wait(full0 + 8 * stage, phase, abort_flag, args.err);
+          if (WGRAD) okf = __all_sync(MOE_FULL_MASK, okf);
+          if (!okf) return false;
           tc_fence_after();
           const uint32_t sa = smem_u32(stage_base + stage * STAGE_BYTES);
           const uint32_t sb = sa + A_BYTES;
+          if (WGRAD && valid < BK) {
+            // K row r of an MN-major box is the 128-byte line at r * 128 (the swizzle only
+            // permutes 16-byte chunks inside a line): zero lines valid..63 of both boxes
+            uint4* a0 = reinterpret_cast<uint4*>(stage_base + stage * STAGE_BYTES);
+            const int n16 = (BK - valid) * 8;
+            for (int c = 0; c < BM / 64; ++c)
+              for (int i = lane; i < n16; i += 32) a0[c * 512 + valid * 8 + i] = make_uint4(0u, 0u, 0u, 0u);
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+          }
+          if (issuer) {
 #pragma unroll
-          for (int kk = 0; kk < BK / UMMA_K; ++kk)
-            tc_mma(d_tmem, sw128_desc(sa + kk * UMMA_K * 2),
-                   BMN ? sw128_mn_desc(sb + kk * UMMA_K * 128) : sw128_desc(sb + kk * UMMA_K * 2),
-                   idesc, (first && kk == 0) ? 0u : 1u);
+            for (int kk = 0; kk < BK / UMMA_K; ++kk)
+              tc_mma(d_tmem,
+                     WGRAD ? sw128_mn_desc(sa + kk * UMMA_K * 128) : sw128_desc(sa + kk * UMMA_K * 2),
+                     (BMN || WGRAD) ? sw128_mn_desc(sb + kk * UMMA_K * 128)
+                                    : sw128_desc(sb + kk * UMMA_K * 2),
+                     idesc, (first && kk == 0) ? 0u : 1u);
+            tc_commit(empty0 + 8 * stage);
+          }
+          if (WGRAD) __syncwarp();
           first = false;
-          tc_commit(empty0 + 8 * stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
           return true;
         });
         if (!ok) break;
-        tc_commit(tfull0 + 8 * acc);
+        if (issuer) tc_commit(tfull0 + 8 * acc);
         if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
       }
-      tc_commit(drain);
-      volatile int no_abort = 0;
-      mbar_wait(drain, 0, &no_abort, args.err);
+      if (issuer) {
+        tc_commit(drain);
+        volatile int no_abort = 0;
+        mbar_wait(drain, 0, &no_abort, args.err);
+      }
     }
     __syncwarp();
   } else {
@@ -440,10 +484,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
               dh[4 * i + 2] = v.z;
               dh[4 * i + 3] = v.w;
             }
-            uint32_t pg[16], pu[16];
+            uint32_t pg[16], pu[16], ph[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              float dgv[2], duv[2];
+              float dgv[2], duv[2], hv[2];
 #pragma unroll
               for (int h = 0; h < 2; ++h) {
                 const float gv = __uint_as_float(g[2 * i + h]);
@@ -452,16 +496,20 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                 const float dhv = dh[2 * i + h];
                 duv[h] = dhv * gv * s;
                 dgv[h] = dhv * uv * s * (1.0f + gv * (1.0f - s));
+                hv[h] = gv * s * uv;
               }
               pg[i] = pack_bf16(dgv[0], dgv[1]);
               pu[i] = pack_bf16(duv[0], duv[1]);
+              ph[i] = pack_bf16(hv[0], hv[1]);
             }
             uint4* dg_dst = reinterpret_cast<uint4*>(grow + c * 32);
             uint4* du_dst = reinterpret_cast<uint4*>(grow + args.F + c * 32);
+            uint4* h_dst = reinterpret_cast<uint4*>(args.hb + (int64_t)row * args.F + col0 + c * 32);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               dg_dst[i] = make_uint4(pg[4 * i], pg[4 * i + 1], pg[4 * i + 2], pg[4 * i + 3]);
               du_dst[i] = make_uint4(pu[4 * i], pu[4 * i + 1], pu[4 * i + 2], pu[4 * i + 3]);
+              h_dst[i] = make_uint4(ph[4 * i], ph[4 * i + 1], ph[4 * i + 2], ph[4 * i + 3]);
             }
           }
         }
@@ -537,22 +585,15 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 }
 
 // ------------------------------------------------------------------- helpers
-// Padded K layout of the transposed activations: group g's rows occupy columns
-// [padoff[g], padoff[g] + ceil(n_g/64)*64), zero beyond its rows; per expert, the list
-// of its groups' K-step segments in group-table order (home and replica groups alike).
+// Per expert, the list of its groups' row ranges {row_start, rows} in group-table order
+// (home and replica groups alike): the K steps of its weight-gradient tiles.
 __global__ void __launch_bounds__(1024) bwd_prepare_kernel(const int4* __restrict__ groups, int G,
-                                                           int E, int* __restrict__ padoff,
-                                                           int* __restrict__ seg_off,
+                                                           int E, int* __restrict__ seg_off,
                                                            int2* __restrict__ segs,
                                                            const int32_t* __restrict__ err) {
-  __shared__ int s_pad[MAX_GROUPS + 1];
   __shared__ int s_cnt[1025];
   __shared__ int s_scan[33];
   if (block_should_stop(err)) return;
-  for (int g = threadIdx.x; g < G; g += blockDim.x) {
-    const int n = groups[g].y;
-    s_pad[g] = n > 0 ? (n + BK - 1) / BK * BK : 0;
-  }
   for (int e = threadIdx.x; e < E; e += blockDim.x) s_cnt[e] = 0;
   __syncthreads();
   for (int g = threadIdx.x; g < G; g += blockDim.x) {
@@ -560,44 +601,25 @@ __global__ void __launch_bounds__(1024) bwd_prepare_kernel(const int4* __restric
     if (r.y > 0) atomicAdd(&s_cnt[r.z], 1);
   }
   __syncthreads();
-  const int total = block_exclusive_scan(s_pad, G, s_scan);
   const int nseg = block_exclusive_scan(s_cnt, E, s_scan);
-  for (int g = threadIdx.x; g < G; g += blockDim.x) padoff[g] = s_pad[g];
   for (int e = threadIdx.x; e < E; e += blockDim.x) seg_off[e] = s_cnt[e];
   __syncthreads();  // thread 0 reuses s_cnt as its fill cursor below
   if (threadIdx.x == 0) {
-    padoff[G] = total;
     seg_off[E] = nseg;
     // stable fill in group-table order (one thread: at most 4096 records)
     for (int g = 0; g < G; ++g) {
       const int4 r = groups[g];
-      if (r.y > 0) {
-        const int at = s_cnt[r.z]++;
-        segs[at] = make_int2(s_pad[g] / BK, (r.y + BK - 1) / BK);
-      }
+      if (r.y > 0) segs[s_cnt[r.z]++] = make_int2(r.x, r.y);
     }
   }
 }
 
-// src_of[q] = the row whose values sit in column q of the padded K layout, -1 for the
-// zero padding after a group's rows
-__global__ void __launch_bounds__(256) padpos_kernel(const int4* __restrict__ groups,
-                                                     const int* __restrict__ padoff,
-                                                     int* __restrict__ src_of,
-                                                     const int32_t* __restrict__ err) {
-  if (load_err(err)) return;
-  const int g = blockIdx.x;
-  const int4 r = groups[g];
-  const int n = max(r.y, 0);
-  const int pad = padoff[g + 1] - padoff[g];
-  for (int i = threadIdx.x; i < pad; i += blockDim.x) src_of[padoff[g] + i] = i < n ? r.x + i : -1;
-}
-
 // Tiled transpose of 16-bit elements, 64 x 64 per block, 16-byte loads and stores:
 // out[c][q] = in[src(q)][c], src(q) = q (src_of == nullptr) or src_of[q] (0 where it is
-// -1).  q runs over n_out output columns (the padded K layout: blocks past *n_out_dev, when
-// given, return at once).  cols and the row pitches are multiples of 8 elements.  With
-// f16_to_bf16 the fp16 inputs are rounded to bf16 on the way.  Batched over blockIdx.z.
+// -1).  q runs over n_out output columns (blocks past *n_out_dev, when given, return at
+// once).  cols and the row pitches are multiples of 8 elements.  With f16_to_bf16 the fp16
+// inputs are rounded to bf16 on the way.  Batched over blockIdx.z.  (The backward uses it
+// for W2 -> W2^T in bf16.)
 constexpr int kTp = 64;
 // shared tile [q][c]: the 16-byte chunk j of row q is stored at chunk j ^ ((q / 8) % 8), so
 // that reading one column across rows q = 8i + r (i = 0..7) touches 8 different banks
@@ -781,22 +803,15 @@ struct BwdWs {
   __nv_bfloat16* w2t;   // [E*F, d] (W2 transposed, rounded to bf16)
   float* dh;            // [RC, F]
   __nv_bfloat16* dgu;   // [RC, 2F]
-  int* src_of;          // [Kc] source row of each padded K column, -1 for padding
-  int* padoff;          // [G+1]
+  __nv_bfloat16* hb;    // [RC, F] h = silu(g) u recomputed, bf16
   int* seg_off;         // [E+1]
   int2* segs;           // [G]
-  __nv_bfloat16* dyt;   // [d, Kc]
-  __nv_bfloat16* ht;    // [F, Kc] (h rounded to bf16)
-  __nv_bfloat16* dgut;  // [2F, Kc]
-  __nv_bfloat16* xt;    // [d, Kc]
-  int64_t kc;           // padded K capacity
   int64_t bytes;
 };
 
 BwdWs carve(uint8_t* base, int T, int k, int E, int R, int S, int d, int F, int G) {
   BwdWs w{};
   const int64_t RC = (int64_t)T * k;
-  w.kc = ((RC + (int64_t)BK * G + 63) / 64) * 64;
   int64_t off = 0;
   auto take = [&](int64_t bytes) {
     const int64_t at = off;
@@ -806,14 +821,9 @@ BwdWs carve(uint8_t* base, int T, int k, int E, int R, int S, int d, int F, int 
   w.w2t = reinterpret_cast<__nv_bfloat16*>(take((int64_t)E * F * d * 2));
   w.dh = reinterpret_cast<float*>(take(RC * F * 4));
   w.dgu = reinterpret_cast<__nv_bfloat16*>(take(RC * 2 * F * 2));
-  w.src_of = reinterpret_cast<int*>(take(w.kc * 4));
-  w.padoff = reinterpret_cast<int*>(take((int64_t)(G + 1) * 4));
+  w.hb = reinterpret_cast<__nv_bfloat16*>(take(RC * F * 2));
   w.seg_off = reinterpret_cast<int*>(take((int64_t)(E + 1) * 4));
   w.segs = reinterpret_cast<int2*>(take((int64_t)G * 8));
-  w.dyt = reinterpret_cast<__nv_bfloat16*>(take((int64_t)d * w.kc * 2));
-  w.ht = reinterpret_cast<__nv_bfloat16*>(take((int64_t)F * w.kc * 2));
-  w.dgut = reinterpret_cast<__nv_bfloat16*>(take((int64_t)2 * F * w.kc * 2));
-  w.xt = reinterpret_cast<__nv_bfloat16*>(take((int64_t)d * w.kc * 2));
   w.bytes = off;
   (void)R;
   (void)S;
@@ -857,6 +867,7 @@ int launch_grouped_ffn_backward(const __nv_bfloat16* recv, const __nv_bfloat16* 
                                 int F, __nv_bfloat16* dx_rows, float* dW1, float* dW3,
                                 float* dW2, void* workspace, int64_t workspace_bytes,
                                 int32_t* err, cudaStream_t s) {
+  (void)h;  // not read: the SwiGLU-backward epilogue recomputes h (in bf16) for dW2
   const int G = R * L.max_groups_per_rank;
   BwdWs w = carve(static_cast<uint8_t*>(workspace), T, k, E, R, S, d, F, G);
   if (w.bytes > workspace_bytes) return MOE_ERR_ARG;
@@ -872,10 +883,8 @@ int launch_grouped_ffn_backward(const __nv_bfloat16* recv, const __nv_bfloat16* 
       return MOE_ERR_LAUNCH;
     return MOE_OK;
   }
-  // 1. padded K layout and per-expert segments
-  bwd_prepare_kernel<<<1, 1024, 0, s>>>(groups, G, E, w.padoff, w.seg_off, w.segs, err);
-  if ((st = launch_status()) != MOE_OK) return st;
-  padpos_kernel<<<G, 256, 0, s>>>(groups, w.padoff, w.src_of, err);
+  // 1. per-expert lists of group row ranges (the weight gradients' K steps)
+  bwd_prepare_kernel<<<1, 1024, 0, s>>>(groups, G, E, w.seg_off, w.segs, err);
   if ((st = launch_status()) != MOE_OK) return st;
   // 2. W2T[e] = W2[e]^T [F,d], rounded to bf16 (the dH GEMM reads it K-major; W1 and W3 are
   //    read MN-major by the dX GEMM, no copy)
@@ -907,7 +916,8 @@ int launch_grouped_ffn_backward(const __nv_bfloat16* recv, const __nv_bfloat16* 
     a.out = w.dh;
     if ((st = launch_bwd_gemm<EPI_F32, false>(ma, mb, mb, a, s))) return st;
   }
-  // 4. dG, dU: the gate/up GEMM re-run on the rows, SwiGLU backward in the epilogue
+  // 4. dG, dU: the gate/up GEMM re-run on the rows, SwiGLU backward in the epilogue (which
+  //    also stores h = silu(g) u in bf16 for dW2)
   {
     CUtensorMap ma, m1, m3;
     if (!make_map16(&ma, recv, RC, d, d, BM, true) ||
@@ -924,6 +934,7 @@ int launch_grouped_ffn_backward(const __nv_bfloat16* recv, const __nv_bfloat16* 
     a.bf16 = 1;
     a.dh = w.dh;
     a.dgu = w.dgu;
+    a.hb = w.hb;
     if ((st = launch_bwd_gemm<EPI_SWIGLU_BWD, false>(ma, m1, m3, a, s))) return st;
   }
   // 5. dX rows = [dG | dU] [W1; W3] (K = 2F, bf16): B read MN-major from W1 (K steps below
@@ -946,19 +957,11 @@ int launch_grouped_ffn_backward(const __nv_bfloat16* recv, const __nv_bfloat16* 
     a.out = dx_rows;
     if ((st = launch_bwd_gemm<EPI_BF16, false, true>(ma, m1, m3, a, s))) return st;
   }
-  // 6. transposed activations in the padded K layout (padding written as zeros)
-  const int kc = (int)w.kc;
-  const int* kp = w.padoff + G;  // used columns of the padded layout
-  if ((st = transpose(dy, d, d, 0, w.dyt, w.kc, 0, kc, kp, w.src_of, 1, false, err, s))) return st;
-  if ((st = transpose(h, F, F, 0, w.ht, w.kc, 0, kc, kp, w.src_of, 1, true, err, s))) return st;
-  if ((st = transpose(w.dgu, 2 * F, 2 * F, 0, w.dgut, w.kc, 0, kc, kp, w.src_of, 1, false, err, s)))
-    return st;
-  if ((st = transpose(recv, d, d, 0, w.xt, w.kc, 0, kc, kp, w.src_of, 1, false, err, s))) return st;
-  // 7. weight gradients, every group of an expert (home and replicas) in one accumulator
+  // 6. weight gradients, every group of an expert (home and replicas) in one accumulator;
+  //    A and B are the row-major activations read MN-major in boxes of 64 rows x 64 columns
   {
     CUtensorMap ma, mb;
-    if (!make_map16(&ma, w.dyt, d, w.kc, w.kc, BM, true) ||
-        !make_map16(&mb, w.ht, F, w.kc, w.kc, bnF, true))
+    if (!make_map16(&ma, dy, RC, d, d, 64, true) || !make_map16(&mb, w.hb, RC, F, F, 64, true))
       return MOE_ERR_DEVICE;
     BwdArgs a = base;
     a.n_blocks_n = F / bnF;
@@ -976,8 +979,8 @@ int launch_grouped_ffn_backward(const __nv_bfloat16* recv, const __nv_bfloat16* 
   }
   {
     CUtensorMap ma, mb;
-    if (!make_map16(&ma, w.dgut, 2 * F, w.kc, w.kc, BM, true) ||
-        !make_map16(&mb, w.xt, d, w.kc, w.kc, bnD, true))
+    if (!make_map16(&ma, w.dgu, RC, 2 * F, 2 * F, 64, true) ||
+        !make_map16(&mb, recv, RC, d, d, 64, true))
       return MOE_ERR_DEVICE;
     BwdArgs a = base;
     a.n_blocks_n = d / bnD;
