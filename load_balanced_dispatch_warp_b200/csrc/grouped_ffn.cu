@@ -709,7 +709,9 @@ __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t a_desc, ui
       : "memory");
 }
 
-// This CTA's part of pair tile t: its 128 rows and its half of the B columns.
+// This CTA's part of pair tile t: its 128 rows and its half of the B columns.  A group's
+// last block with at most 128 rows left is a half tile (with half_tiles and N = 256): an
+// M = 128 pair MMA, 64 rows in each CTA.
 __device__ __forceinline__ Tile decode_pair_tile(int t, const FfnArgs& a, const int* s_prefix,
                                                  int rank, bool swiglu) {
   const int mt = t / a.n_blocks_n;
@@ -721,10 +723,23 @@ __device__ __forceinline__ Tile decode_pair_tile(int t, const FfnArgs& a, const 
     if (s_prefix[mid] <= mt) lo = mid; else hi = mid - 1;
   }
   const int4 g = group_of(a, lo);
-  const int first = (mt - s_prefix[lo]) * P_BM + rank * BM;  // row offset inside the group
+  int m_local = mt - s_prefix[lo];
+  if (a.n_chunk > 0) {  // the group's weight blocks chunk by chunk, as decode_tile
+    const int local = t - s_prefix[lo] * a.n_blocks_n;
+    const int mc = s_prefix[lo + 1] - s_prefix[lo];
+    const int per_chunk = mc * a.n_chunk;
+    const int c = local / per_chunk;
+    const int rem = local - c * per_chunk;
+    const int ncw = min(a.n_chunk, a.n_blocks_n - c * a.n_chunk);
+    m_local = rem / ncw;
+    tl.n_block = c * a.n_chunk + (rem - m_local * ncw);
+  }
+  const int base = m_local * P_BM;  // first row of the pair tile in the group
+  tl.half = a.half_tiles && a.mma_n == 256 && g.y - base <= BM;
+  const int rows_cta = tl.half ? BM / 2 : BM;
+  const int first = base + rank * rows_cta;  // this CTA's first row inside the group
   tl.a_row = g.x + first;
-  tl.valid_rows = max(0, min(BM, g.y - first));
-  tl.half = false;
+  tl.valid_rows = max(0, min(rows_cta, g.y - first));
   const int ref = g.w;
   tl.pool = ref >= a.E;
   tl.b_row = (tl.pool ? ref - a.E : ref) * a.rows_per_expert + tl.n_block * a.bn_out +
@@ -735,6 +750,7 @@ __device__ __forceinline__ Tile decode_pair_tile(int t, const FfnArgs& a, const 
 template <bool SWIGLU>
 __global__ void __launch_bounds__(FFN_THREADS, 1)
     ffn_pair_kernel(const __grid_constant__ CUtensorMap tm_a,
+                    const __grid_constant__ CUtensorMap tm_a64,
                     const __grid_constant__ CUtensorMap tm_b0,
                     const __grid_constant__ CUtensorMap tm_b1,
                     const __grid_constant__ CUtensorMap tm_p0,
@@ -749,6 +765,13 @@ __global__ void __launch_bounds__(FFN_THREADS, 1)
   // s_misc: [0] tmem base, [1] abort, [2] error word seen by this CTA, [3] by the pair
   int* s_prefix = s_misc + 4;
   int* s_scan = s_prefix + MAX_GROUPS + 1;
+  // half tiles of GEMM 1: the up warps hand their values to the gate warps through
+  // s_xchg ([2][32 rows][32 floats]) under the barriers xfull (up written) and xempty
+  // (read)
+  uint64_t* xbars = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(s_scan + 33) + 7) &
+                                                ~static_cast<uintptr_t>(7));
+  float* s_xchg = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(xbars + 2) + 15) &
+                                           ~static_cast<uintptr_t>(15));
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
@@ -772,6 +795,8 @@ __global__ void __launch_bounds__(FFN_THREADS, 1)
       mbar_init(tempty0 + 8 * b, 8);
     }
     mbar_init(drain, 1);
+    mbar_init(smem_u32(xbars), 2);      // xfull: the two up warps
+    mbar_init(smem_u32(xbars + 1), 2);  // xempty: the two gate warps
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -804,6 +829,7 @@ __global__ void __launch_bounds__(FFN_THREADS, 1)
     if (lane == 0) {
       const uint32_t b_half = (uint32_t)(args.mma_n >> 1) * BK * 2;
       const uint32_t tx = 2u * (A_BYTES + b_half);
+      const uint32_t tx_half = 2u * (A_BYTES / 2 + b_half);  // 64-row A boxes
       const uint32_t full_leader0 = map_to_rank(full0, 0);
       const CUtensorMap* home = (SWIGLU && rank == 1) ? &tm_b1 : &tm_b0;
       const CUtensorMap* pool = (SWIGLU && rank == 1) ? &tm_p1 : &tm_p0;
@@ -817,8 +843,9 @@ __global__ void __launch_bounds__(FFN_THREADS, 1)
         for (int kb = 0; kb < args.k_blocks; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1u, abort_flag, args.err)) { ok = false; break; }
           const uint32_t sa = smem_u32(stage_base + stage * P_STAGE_BYTES);
-          if (leader) mbar_expect_tx(full0 + 8 * stage, tx);
-          tma_load_2d_pair(sa, &tm_a, full_leader0 + 8 * stage, kb * BK, tl.a_row);
+          if (leader) mbar_expect_tx(full0 + 8 * stage, tl.half ? tx_half : tx);
+          tma_load_2d_pair(sa, tl.half ? &tm_a64 : &tm_a, full_leader0 + 8 * stage, kb * BK,
+                           tl.a_row);
           tma_load_2d_pair(sa + A_BYTES, mb, full_leader0 + 8 * stage, kb * BK, tl.b_row);
           issued_mask |= 1u << stage;
           issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
@@ -844,12 +871,15 @@ __global__ void __launch_bounds__(FFN_THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer (leader CTA only)
     if (lane == 0 && leader) {
-      const uint32_t idesc = make_idesc(P_BM, args.mma_n, SWIGLU);
+      const uint32_t idesc_full = make_idesc(P_BM, args.mma_n, SWIGLU);
+      const uint32_t idesc_half = make_idesc(BM, args.mma_n, SWIGLU);  // 64 rows per CTA
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       for (int t = first_tile; t < total_tiles; t += tile_step) {
+        const uint32_t idesc =
+            decode_pair_tile(t, args, s_prefix, 0, SWIGLU).half ? idesc_half : idesc_full;
         if (!mbar_wait(tempty0 + 8 * acc, acc_phase ^ 1u, abort_flag, args.err)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
@@ -880,17 +910,99 @@ __global__ void __launch_bounds__(FFN_THREADS, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------ epilogue (warps 2-5)
+    // Full tiles: lane = row (this CTA's 128), columns as N.  Half tiles (M = 128 pair
+    // MMA, measured layout): this CTA's 64 rows sit in lanes 0-63 with output columns
+    // 0-127 and again in lanes 64-127 with columns 128-255, both in TMEM columns 0-127.
+    // In GEMM 1 the first half is gate and the second up: the up warps (quarters 2, 3)
+    // pass their values to the gate warps (quarters 0, 1) of the same rows through shared
+    // memory.
     const int quarter = warp & 3;
     const int r_in = quarter * 32 + lane;
     const uint32_t tempty_leader0 = map_to_rank(tempty0, 0);
+    const uint32_t xfull = smem_u32(xbars), xempty = smem_u32(xbars + 1);
+    uint32_t xphase = 0;
+    bool xok = true;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = first_tile; t < total_tiles; t += tile_step) {
+    for (int t = first_tile; xok && t < total_tiles; t += tile_step) {
       const Tile tl = decode_pair_tile(t, args, s_prefix, (int)rank, SWIGLU);
       const bool ok = mbar_wait(tfull0 + 8 * acc, acc_phase, abort_flag, args.err);
       if (!__all_sync(MOE_FULL_MASK, ok)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * ACC_COLS;
+      if (tl.half) {
+        const int hrow = (quarter & 1) * 32 + lane;  // row among this CTA's 64
+        const bool hvalid = hrow < tl.valid_rows;
+        float* stg = s_xchg + (quarter & 1) * 1024;  // [32 rows][32 floats]
+        if (SWIGLU) {
+          uint16_t* orow = static_cast<uint16_t*>(args.out) +
+                           (int64_t)(tl.a_row + hrow) * args.out_ld +
+                           (int64_t)tl.n_block * args.bn_out;
+#pragma unroll 1
+          for (int c = 0; c < 128 / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tbase + c * 32, v);
+            tmem_wait_ld();
+            if (quarter >= 2) {
+              // up: wait until the gate warps have read the previous chunk, then stage
+              // row `lane`'s 32 values (16-byte chunk j at j ^ (lane % 8): no conflicts)
+              const bool w = mbar_wait(xempty, xphase ^ 1u, abort_flag, args.err);
+              if (!__all_sync(MOE_FULL_MASK, w)) { xok = false; break; }
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<uint4*>(stg + lane * 32 + ((j ^ (lane & 7)) << 2)) =
+                    make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+              __syncwarp();
+              if (lane == 0) mbar_arrive(xfull);
+            } else {
+              const bool w = mbar_wait(xfull, xphase, abort_flag, args.err);
+              if (!__all_sync(MOE_FULL_MASK, w)) { xok = false; break; }
+              uint32_t u[32];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const uint4 q = *reinterpret_cast<const uint4*>(stg + lane * 32 + ((j ^ (lane & 7)) << 2));
+                u[4 * j] = q.x;
+                u[4 * j + 1] = q.y;
+                u[4 * j + 2] = q.z;
+                u[4 * j + 3] = q.w;
+              }
+              __syncwarp();
+              if (lane == 0) mbar_arrive(xempty);
+              uint32_t p[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float g0 = __uint_as_float(v[2 * i]), g1 = __uint_as_float(v[2 * i + 1]);
+                const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+                p[i] = pack_f16_sat(silu(g0) * u0, silu(g1) * u1);
+              }
+              if (hvalid) {
+                uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+              }
+            }
+            xphase ^= 1u;
+          }
+        } else {
+          uint16_t* orow = static_cast<uint16_t*>(args.out) +
+                           (int64_t)(tl.a_row + hrow) * args.out_ld +
+                           (int64_t)tl.n_block * args.bn_out + (quarter >> 1) * 128;
+#pragma unroll 1
+          for (int c = 0; c < 128 / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tbase + c * 32, v);
+            tmem_wait_ld();
+            uint32_t p[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) p[i] = pack_bf16(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+            if (hvalid) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) dst[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+            }
+          }
+        }
+      } else {
       const bool valid = r_in < tl.valid_rows;
       uint16_t* orow = static_cast<uint16_t*>(args.out) + (int64_t)(tl.a_row + r_in) * args.out_ld +
                        (int64_t)tl.n_block * args.bn_out;
@@ -930,6 +1042,8 @@ __global__ void __launch_bounds__(FFN_THREADS, 1)
           }
         }
       }
+      }
+      if (!xok) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(tempty_leader0 + 8 * acc);
@@ -1022,7 +1136,7 @@ int launch_one(const CUtensorMap& a, const CUtensorMap& a64, const CUtensorMap& 
 
 size_t ffn_pair_smem_bytes() {
   return 1024 + (size_t)P_STAGES * P_STAGE_BYTES + (2 * P_STAGES + 5) * 8 + 4 * 4 +
-         (MAX_GROUPS + 1) * 4 + 33 * 4;
+         (MAX_GROUPS + 1) * 4 + 33 * 4 + 8 + 2 * 8 + 16 + 2 * 32 * 32 * 4;
 }
 
 std::atomic<int> g_ffn_tile_mode{0};  // 0: one CTA per 128-row tile, 1: CTA pairs
@@ -1031,9 +1145,9 @@ int g_pair_clusters[64] = {0};  // co-resident 2-CTA clusters per device
 // Grid of the pair kernels: as many 2-CTA clusters as fit on the device at once (queried
 // once per device; a GPC with an odd number of free SMs leaves one of them idle).
 template <bool SWIGLU>
-int launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                const CUtensorMap& p0, const CUtensorMap& p1, const FfnArgs& args,
-                cudaStream_t s) {
+int launch_pair(const CUtensorMap& a, const CUtensorMap& a64, const CUtensorMap& b0,
+                const CUtensorMap& b1, const CUtensorMap& p0, const CUtensorMap& p1,
+                const FfnArgs& args, cudaStream_t s) {
   static bool configured[64] = {false};
   static int clusters[64] = {0};
   int dev = 0;
@@ -1066,7 +1180,7 @@ int launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& 
     configured[dev] = true;
   }
   cfg.gridDim = dim3(2 * clusters[dev], 1, 1);
-  if (cudaLaunchKernelEx(&cfg, ffn_pair_kernel<SWIGLU>, a, b0, b1, p0, p1, args) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, ffn_pair_kernel<SWIGLU>, a, a64, b0, b1, p0, p1, args) != cudaSuccess)
     return MOE_ERR_LAUNCH;
   return launch_status();
 }
@@ -1153,7 +1267,7 @@ int launch_grouped_ffn_impl(const __nv_bfloat16* recv, const __nv_bfloat16* x,
   a1.groups = groups;
   a1.G = G;
   a1.uniform_rows = uniform_rows;
-  a1.half_tiles = (gather || pair) ? 0 : 1;  // the gathering producer always fills 128 rows
+  a1.half_tiles = gather ? 0 : 1;  // the gathering producer always fills 128 rows
   a1.n_chunk = 2;  // measured fastest at the DeepSeek shape among 1, 2, 4 and row-block-major
   a1.comb_out = nullptr;
   a1.comb_src = nullptr;
@@ -1174,7 +1288,7 @@ int launch_grouped_ffn_impl(const __nv_bfloat16* recv, const __nv_bfloat16* x,
   a1.gd = d;
   a1.gT = T;
   int st = gather ? launch_one<true, true>(m_w1, m_w1, m_w1, m_w3, m_p1, m_p3, a1, s)
-           : pair ? launch_pair<true>(m_recv, m_w1, m_w3, m_p1, m_p3, a1, s)
+           : pair ? launch_pair<true>(m_recv, m_recv64, m_w1, m_w3, m_p1, m_p3, a1, s)
                   : launch_one<true, false>(m_recv, m_recv64, m_w1, m_w3, m_p1, m_p3, a1, s);
   if (st != MOE_OK) return st;
   FfnArgs a2 = a1;
@@ -1187,7 +1301,7 @@ int launch_grouped_ffn_impl(const __nv_bfloat16* recv, const __nv_bfloat16* x,
   a2.out = y;
   a2.gx = nullptr;
   a2.gsrc = nullptr;
-  a2.half_tiles = pair ? 0 : 1;
+  a2.half_tiles = 1;
   if (comb != nullptr) {
     a2.comb_out = comb->out32;
     a2.comb_src = comb->src;
@@ -1195,7 +1309,7 @@ int launch_grouped_ffn_impl(const __nv_bfloat16* recv, const __nv_bfloat16* x,
     a2.comb_gate = comb->gate;
     a2.comb_k = comb->k;
   }
-  return pair ? launch_pair<false>(m_h, m_w2, m_w2, m_p2, m_p2, a2, s)
+  return pair ? launch_pair<false>(m_h, m_h64, m_w2, m_w2, m_p2, m_p2, a2, s)
               : launch_one<false, false>(m_h, m_h64, m_w2, m_w2, m_p2, m_p2, a2, s);
 }
 

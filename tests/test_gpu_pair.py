@@ -2,7 +2,9 @@
 
 moe_set_ffn_tile_mode(1) runs both GEMMs as 2-CTA clusters on 256-row tiles
 (tcgen05.mma.cta_group::2): each CTA holds 128 rows of A and half of B, the pair shares
-one 256 x N accumulator tile.  The bar is the default tiling's: integer outputs bit-exact,
+one 256 x N accumulator tile; a group's last block with at most 128 rows left runs as a
+half tile (an M = 128 pair MMA, 64 rows per CTA; in GEMM 1 the up half of each row reaches
+the gate half through shared memory).  The bar is the default tiling's: integer outputs bit-exact,
 h / y / out within 1e-2 * max(1, |oracle|) (every row for small shapes, sampled tokens at
 full size).  Both tilings add the same products in the same K order, so their outputs are
 also compared with each other element by element.
@@ -48,8 +50,9 @@ def assert_same_ffn(Lp, Lu):
 
 SMALL = [
     I.WORKLOADS["tiny"],
-    # groups of every size class against 256-row tiles: rows % 256 in (0, 128] leave the
-    # second CTA of the last tile without valid rows, (128, 256) splits it
+    # groups of every size class against 256-row tiles: rows % 256 in (0, 128] end in a
+    # half tile (64 rows per CTA, the second CTA possibly without valid rows), (128, 256)
+    # in a full tile split between the CTAs
     I.small_workload("ragged", 300, 16, 4, 4, 2, 256, 384, alpha=1.0, seed=1),
     I.small_workload("mid", 1000, 64, 6, 8, 8, 512, 256, alpha=0.6, seed=2),
     # d % 256 != 0: GEMM 2 runs N = 128, each CTA loads a 64-row half of W2
