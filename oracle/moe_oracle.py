@@ -50,6 +50,8 @@ Pins (tests/test_oracle_pins.py checks each against something other than this fi
                     concatenated batch (same perm, the same rows on every rank, the same
                     outputs); q_base counted directly on the concatenated trace; one
                     rank's error reaches the job's error word
+  ep_layer_backward the W-process backward equals layer_backward() of the concatenated
+                    batch (dx, dlogits, dy and dX rows per rank, every weight gradient)
   layer_backward    central finite differences of layer() itself (fp64, tiny shapes,
                     away from top-k ties); torch.autograd (fp64, CPU) through a token-major
                     formulation with no plan, dispatch or replicas; the weight gradients do
@@ -62,7 +64,8 @@ Pins (tests/test_oracle_pins.py checks each against something other than this fi
   (tests/test_oracle_mutants.py plants one plausible mistake at a time in topk_route,
   topk_route_biased, validate_trace, expert_histogram, capacity_ledger, remote_routes,
   plan_balanced, permute, dispatch, prefetch, expert_ffn, combine, ep_rank_base,
-  ep_permute and the four backward pieces, and checks that the pin for it fails)
+  ep_permute, ep_layer_backward and the four backward pieces, and checks that the pin for
+  it fails)
 
 Error bits (OR-ed): 1 non-finite logit, 2 expert id out of range, 4 repeated expert
 within one token, 8 plan needs more than S replicas on some rank.
@@ -690,7 +693,7 @@ def ep_layer(logits_shards, x_shards, W1, W3, W2, k: int, S: int):
                 r = int(perm[t, j])
                 out[t] += float(gate[t, j]) * ranks[r // C]["y"][r % C]
         ranks[u]["out"] = out
-    return dict(ranks=ranks, plan=plan, counts_all=counts_all, err=err)
+    return dict(ranks=ranks, plan=plan, pool=pool, counts_all=counts_all, err=err)
 
 
 # ------------------------------------------------------------------ backward pass
@@ -818,3 +821,82 @@ def layer_backward(fwd, dout, W1, W3, W2, E: int):
     dlogits = topk_backward(fwd["gate"], dgate, fwd["idx"], E)
     return dict(dx=dx, dlogits=dlogits, dW1=g["dW1"], dW3=g["dW3"], dW2=g["dW2"], dy=dy,
                 dgate=dgate, dX_rows=g["dX"], dh=g["dh"], dg=g["dg"], du=g["du"])
+
+
+def ep_layer_backward(ep, douts, W1, W3, W2, E: int, S: int):
+    """The backward of ep_layer() as the W processes run it, rank u holding douts[u]
+    ([MoonEP] para. 3: the duplicated experts' gradients are reduced back home):
+      1. combine backward across ranks: for each of rank u's assignments (t, j) with row
+         r on rank v = r // C: v's dy[r % C] = gate[t,j] dout[t]; dgate[t,j] =
+         <dout[t], y_v[r % C]>;
+      2. every rank v: each of its groups through its expert's backward on v's own rows
+         (dX rows); a home group's weight gradient goes to v's partial of that home
+         expert, a replica group's to v's partial of that pool slot;
+      3. reduction back home: expert e's gradient, on rank e // B, is its home partial plus
+         the partial of every slot (v, s) that held a copy of e, in (v, s) order;
+      4. dispatch backward across ranks: dx[t] = sum_j dX_v[r % C], in j order;
+      5. the gates' backward, local.
+    Returns dict(ranks=[dict(dy, dgate, dX_rows, dx, dlogits)], dW1, dW3, dW2 [E,...])."""
+    ranks = ep["ranks"]
+    plan = ep["plan"]
+    W = len(ranks)
+    C = plan["C"]
+    B = E // W
+    d = np.asarray(W1).shape[2]
+    F = np.asarray(W1).shape[1]
+    dys = [np.zeros((C, d)) for _ in range(W)]
+    out = [dict() for _ in range(W)]
+    for u, r in enumerate(ranks):
+        dout = np.asarray(douts[u], dtype=np.float64)
+        perm, gate = r["perm"], np.asarray(r["gate"], dtype=np.float64)
+        T, k = perm.shape
+        dgate = np.zeros((T, k))
+        for t in range(T):
+            for j in range(k):
+                row = int(perm[t, j])
+                v = row // C
+                dys[v][row % C] = gate[t, j] * dout[t]
+                dgate[t, j] = float(dout[t] @ np.asarray(ranks[v]["y"], dtype=np.float64)[row % C])
+        out[u]["dgate"] = dgate
+    parts = []
+    for v in range(W):
+        recv = np.asarray(ranks[v]["recv"], dtype=np.float64)
+        dX = np.zeros((C, d))
+        part1 = np.zeros((B + S, F, d))
+        part3 = np.zeros((B + S, F, d))
+        part2 = np.zeros((B + S, d, F))
+        for (r0, n, e, ref) in plan["groups"][v]:
+            lo = r0 - v * C
+            w1, w3, w2 = weights_of(ref, E, W1, W3, W2, ep["pool"])
+            b = expert_ffn_backward(recv[lo:lo + n], w1, w3, w2, dys[v][lo:lo + n])
+            dX[lo:lo + n] = b["dX"]
+            slot = e - v * B if ref < E else B + (ref - E - v * S)
+            part1[slot] += b["dw1"]
+            part3[slot] += b["dw3"]
+            part2[slot] += b["dw2"]
+        out[v]["dy"] = dys[v]
+        out[v]["dX_rows"] = dX
+        parts.append((part1, part3, part2))
+    dW1 = np.zeros((E, F, d))
+    dW3 = np.zeros((E, F, d))
+    dW2 = np.zeros((E, d, F))
+    for e in range(E):
+        home = e // B
+        acc = [parts[home][i][e - home * B].copy() for i in range(3)]
+        for v in range(W):
+            for s in range(S):
+                if plan["replica_expert"][v * S + s] == e:
+                    for i in range(3):
+                        acc[i] += parts[v][i][B + s]
+        dW1[e], dW3[e], dW2[e] = acc
+    for u, r in enumerate(ranks):
+        perm = r["perm"]
+        T, k = perm.shape
+        dx = np.zeros((T, d))
+        for t in range(T):
+            for j in range(k):
+                row = int(perm[t, j])
+                dx[t] += out[row // C]["dX_rows"][row % C]
+        out[u]["dx"] = dx
+        out[u]["dlogits"] = topk_backward(r["gate"], out[u]["dgate"], r["idx"], E)
+    return dict(ranks=out, dW1=dW1, dW3=dW3, dW2=dW2)

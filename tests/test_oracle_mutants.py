@@ -288,3 +288,21 @@ def test_ep_pins_catch_planted_mistakes(monkeypatch, name, mutant, pin):
     # the placement rule finds no rank: that is caught too
     with pytest.raises((AssertionError, IndexError)):
         pin()
+
+
+def ep_backward_keeping_replicas_away(ep, douts, W1, W3, W2, E, S):
+    """Replica gradients left on the ranks that computed them (no reduction back home)."""
+    plan = dict(ep["plan"])
+    plan["replica_expert"] = [-1] * len(plan["replica_expert"])
+    return EPB["ep_layer_backward"](dict(ep, plan=plan), douts, W1, W3, W2, E, S)
+
+
+EPB = {"ep_layer_backward": O.ep_layer_backward}
+
+
+@pytest.mark.parametrize("mutant", [ep_backward_keeping_replicas_away])
+def test_ep_backward_pin_catches_planted_mistake(monkeypatch, mutant):
+    F.test_ep_backward_is_the_backward_of_the_rank_major_batch()
+    monkeypatch.setattr(O, "ep_layer_backward", mutant)
+    with pytest.raises(AssertionError):
+        F.test_ep_backward_is_the_backward_of_the_rank_major_batch()

@@ -592,3 +592,26 @@ def test_ep_error_bits_reach_every_rank():
     assert ep["err"] & O.ERR_NONFINITE
     c, e = O.ep_local_counts(np.array([[1, 1], [0, 9]]), 8)
     assert e == O.ERR_DUPLICATE | O.ERR_ID_RANGE and c.tolist() == [1, 2, 0, 0, 0, 0, 0, 0]
+
+
+def test_ep_backward_is_the_backward_of_the_rank_major_batch():
+    """The W-process backward -- dy written across ranks, each rank's groups on its own rows,
+    replica gradients reduced to the home rank -- equals layer_backward() of the
+    concatenated batch: dx, dlogits and every weight gradient."""
+    for seed, W, T, E, k, S in EP_CASES:
+        logits, x, W1, W3, W2 = _ep_case(seed, W, T, E, k)
+        rng = np.random.default_rng(100 + seed)
+        dout = rng.standard_normal(x.shape)
+        ep = O.ep_layer(np.split(logits, W), np.split(x, W), W1, W3, W2, k, S)
+        ebw = O.ep_layer_backward(ep, np.split(dout, W), W1, W3, W2, E, S)
+        fwd = O.layer(logits, x, W1, W3, W2, k, W, S)
+        ref = O.layer_backward(fwd, dout, W1, W3, W2, E)
+        C = fwd["plan"]["C"]
+        for name in ("dx", "dlogits"):
+            got = np.concatenate([r[name] for r in ebw["ranks"]])
+            assert np.allclose(got, ref[name], rtol=1e-10, atol=1e-12), name
+        for u, r in enumerate(ebw["ranks"]):
+            assert np.allclose(r["dy"], ref["dy"][u * C:(u + 1) * C], rtol=1e-12, atol=1e-12)
+            assert np.allclose(r["dX_rows"], ref["dX_rows"][u * C:(u + 1) * C], rtol=1e-10, atol=1e-12)
+        for name in ("dW1", "dW3", "dW2"):
+            assert np.allclose(ebw[name], ref[name], rtol=1e-10, atol=1e-12), name
