@@ -590,6 +590,70 @@ int moe_ep_combine(const moe_bf16* const* y_ranks, const int32_t* perm, const fl
                    moe_stream_t stream);
 
 /*
+ * Backward of the expert-parallel layer.   [MoonEP] paragraph 3: the duplicated experts'
+ * gradients are reduced back home during the backward pass -- here across GPUs.  One
+ * backward step on rank me, after its forward:
+ *   moe_ep_combine_backward -> [barrier] -> moe_ep_grouped_ffn_backward -> [barrier] ->
+ *   moe_ep_reduce_home, moe_ep_dispatch_backward -> moe_topk_backward (local).
+ * The results equal the single-GPU backward of the concatenated batch (moe_combine_backward,
+ * moe_grouped_ffn_backward, moe_dispatch_backward with R = W): dx, dlogits and the rows bit
+ * for bit; a home expert's weight gradient sums the same products, in a different order
+ * (its own groups in one accumulator, then each copy's partial in fp32).
+ *
+ * moe_ep_combine_backward: for this rank's assignment (t, j) with row r = perm[t,j] on rank
+ *   v = r / C (C = T*k): v's dy[r % C] = gate[t,j] * dout[t] (bf16, a peer store) and
+ *   dgate[t,j] = <dout[t], y_v[r % C]> (fp32, peer loads).
+ *   dout [T,d] bf16; y_ranks, dy_ranks: HOST tables of every rank's y and dy [C,d] bf16;
+ *   perm, gate [T,k] from the forward; dgate [T,k] fp32 (out).  err  no-op when non-zero.
+ */
+int moe_ep_combine_backward(const moe_bf16* dout, const moe_bf16* const* y_ranks,
+                            const int32_t* perm, const float* gate, int W, int T, int k, int d,
+                            moe_bf16* const* dy_ranks, float* dgate, const int32_t* err,
+                            moe_stream_t stream);
+/*
+ * moe_ep_grouped_ffn_backward: the grouped-FFN backward over this rank's C rows and its
+ *   re-based groups (as moe_ep_grouped_ffn: home experts from W1, W3, W2 [B,...], replicas
+ *   from its pool slots P1, P3, P2 [S,...]).
+ *   recv, dy [C,d] bf16: this rank's rows and their gradients.
+ *   dx_rows [C,d] bf16 (out).
+ *   dP1, dP3 [B+S,F,d], dP2 [B+S,d,F] fp32 (out): the weight gradients of this rank's
+ *   groups -- entry b < B its home expert me*B + b, entry B + s its pool slot s (the
+ *   partial that moe_ep_reduce_home adds to the slot's home expert); entries without rows
+ *   are 0.
+ *   groups_ws [4*(B+S)] int32 scratch; workspace of moe_ep_ffn_backward_workspace_bytes
+ *   bytes, 256-byte aligned.  Requires B + S <= 1024.  MOE_ERR_ARG if workspace_bytes is
+ *   too small.  err  no-op when non-zero.
+ * moe_ep_ffn_backward_workspace_bytes: that size, or -1 for an invalid shape.
+ */
+int64_t moe_ep_ffn_backward_workspace_bytes(int T, int k, int E, int W, int S, int d, int F);
+int moe_ep_grouped_ffn_backward(const moe_bf16* recv, const moe_bf16* dy, const int32_t* plan,
+                                int W, int me, const moe_bf16* W1, const moe_bf16* W3,
+                                const moe_f16* W2, const moe_bf16* P1, const moe_bf16* P3,
+                                const moe_f16* P2, int T, int k, int E, int S, int d, int F,
+                                int32_t* groups_ws, moe_bf16* dx_rows, float* dP1, float* dP3,
+                                float* dP2, void* workspace, int64_t workspace_bytes,
+                                int32_t* err, moe_stream_t stream);
+/*
+ * moe_ep_reduce_home: the gradient of this rank's home expert e = me*B + b: its own entry b
+ *   plus, for every pool slot (v, s) of the plan that held a copy of e, in (v, s) order,
+ *   rank v's entry B + s (peer loads).
+ *   dP1_ranks, dP3_ranks, dP2_ranks: HOST tables of every rank's dP1, dP3, dP2.
+ *   dW1, dW3 [B,F,d], dW2 [B,d,F] fp32 (out).  err  no-op when non-zero.
+ */
+int moe_ep_reduce_home(const int32_t* plan, const float* const* dP1_ranks,
+                       const float* const* dP3_ranks, const float* const* dP2_ranks, int W,
+                       int me, int E, int S, int d, int F, float* dW1, float* dW3, float* dW2,
+                       const int32_t* err, moe_stream_t stream);
+/*
+ * moe_ep_dispatch_backward: dx[t] = sum_j dx_rows_v[perm[t,j] % C], v = perm[t,j] / C
+ *   (fp32 in j order, bf16 out; peer loads).  dx_rows_ranks: HOST table of every rank's
+ *   dx_rows [C,d] bf16; dx [T,d] bf16 (out).  err  no-op when non-zero.
+ */
+int moe_ep_dispatch_backward(const moe_bf16* const* dx_rows_ranks, const int32_t* perm, int W,
+                             int T, int k, int d, moe_bf16* dx, const int32_t* err,
+                             moe_stream_t stream);
+
+/*
  * Device-memory sharing between the processes of one node (CUDA IPC), for the pointer
  * tables above.  Host calls; nothing is enqueued.
  * moe_ipc_export: handle (host buffer of MOE_IPC_HANDLE_BYTES) names the allocation that

@@ -32,7 +32,9 @@ FUSED = ("moe_dispatch_index", "moe_grouped_ffn_gather", "moe_route_plan",
          "moe_grouped_ffn_combine")
 EXPERT_PARALLEL = ("moe_ep_counts", "moe_ep_plan", "moe_ep_prefetch", "moe_ep_dispatch",
                    "moe_ep_grouped_ffn", "moe_ep_combine", "moe_ipc_export", "moe_ipc_import",
-                   "moe_ipc_close")
+                   "moe_ipc_close", "moe_ep_combine_backward", "moe_ep_grouped_ffn_backward",
+                   "moe_ep_ffn_backward_workspace_bytes", "moe_ep_reduce_home",
+                   "moe_ep_dispatch_backward")
 BACKWARD = ("moe_combine_backward", "moe_grouped_ffn_backward", "moe_dispatch_backward",
             "moe_topk_backward")
 HELPERS = ("moe_plan_get_layout", "moe_dispatch_workspace_words", "moe_status_string",
@@ -96,6 +98,11 @@ def lib() -> ctypes.CDLL:
             "moe_ipc_export": [P, P, ctypes.POINTER(I64)],
             "moe_ipc_import": [P, I64, ctypes.POINTER(P), ctypes.POINTER(P)],
             "moe_ipc_close": [P],
+            "moe_ep_combine_backward": [P, P, P, P, I, I, I, I, P, P, P, P],
+            "moe_ep_grouped_ffn_backward": [P, P, P, I, I, P, P, P, P, P, P, I, I, I, I, I, I, P,
+                                            P, P, P, P, P, I64, P, P],
+            "moe_ep_reduce_home": [P, P, P, P, I, I, I, I, I, I, P, P, P, P, P],
+            "moe_ep_dispatch_backward": [P, P, I, I, I, I, P, P, P],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -111,6 +118,8 @@ def lib() -> ctypes.CDLL:
         L.moe_route_plan_workspace_words.restype = I64
         L.moe_ffn_backward_workspace_bytes.argtypes = [I, I, I, I, I, I, I]
         L.moe_ffn_backward_workspace_bytes.restype = I64
+        L.moe_ep_ffn_backward_workspace_bytes.argtypes = [I, I, I, I, I, I, I]
+        L.moe_ep_ffn_backward_workspace_bytes.restype = I64
         L.moe_set_ffn_tile_mode.argtypes = [I]
         L.moe_set_ffn_tile_mode.restype = I
         L.moe_ffn_tile_mode.argtypes = []
@@ -482,6 +491,56 @@ def moe_ep_combine(y_ranks, perm, gate, d, out, err, stream=None):
         _table(y_ranks, "y_ranks"), _ptr(perm, torch.int32, "perm"), _ptr(gate, torch.float32, "gate"),
         len(y_ranks), T, k, d, _ptr(out, torch.bfloat16, "out"), _ptr(err, torch.int32, "err"),
         _stream(stream)), "moe_ep_combine")
+
+
+def moe_ep_combine_backward(dout, y_ranks, perm, gate, dy_ranks, dgate, err, stream=None):
+    T, k = perm.shape
+    _check(lib().moe_ep_combine_backward(
+        _ptr(dout, torch.bfloat16, "dout"), _table(y_ranks, "y_ranks"), _ptr(perm, torch.int32, "perm"),
+        _ptr(gate, torch.float32, "gate"), len(y_ranks), T, k, dout.shape[1],
+        _table(dy_ranks, "dy_ranks"), _ptr(dgate, torch.float32, "dgate"),
+        _ptr(err, torch.int32, "err"), _stream(stream)), "moe_ep_combine_backward")
+
+
+def ep_ffn_backward_workspace_bytes(T, k, E, W, S, d, F) -> int:
+    n = int(lib().moe_ep_ffn_backward_workspace_bytes(T, k, E, W, S, d, F))
+    if n < 0:
+        raise MoEError("moe_ep_ffn_backward_workspace_bytes: invalid shape")
+    return n
+
+
+def moe_ep_grouped_ffn_backward(recv, dy, plan, W, me, W1, W3, W2, P1, P3, P2, T, k, E, S,
+                                groups_ws, dx_rows, dP1, dP3, dP2, workspace, err, stream=None):
+    _, F, d = W1.shape
+    bf, hf, f32 = torch.bfloat16, torch.float16, torch.float32
+    if workspace.dtype != torch.uint8 or not workspace.is_cuda:
+        raise TypeError("workspace must be a CUDA uint8 tensor")
+    _check(lib().moe_ep_grouped_ffn_backward(
+        _ptr(recv, bf, "recv"), _ptr(dy, bf, "dy"), _ptr(plan, torch.int32, "plan"), W, me,
+        _ptr(W1, bf, "W1"), _ptr(W3, bf, "W3"), _ptr(W2, hf, "W2"), _ptr(P1, bf, "P1"),
+        _ptr(P3, bf, "P3"), _ptr(P2, hf, "P2"), T, k, E, S, d, F,
+        _ptr(groups_ws, torch.int32, "groups_ws"), _ptr(dx_rows, bf, "dx_rows"),
+        _ptr(dP1, f32, "dP1"), _ptr(dP3, f32, "dP3"), _ptr(dP2, f32, "dP2"),
+        workspace.data_ptr(), workspace.numel(), _ptr(err, torch.int32, "err"), _stream(stream)),
+        "moe_ep_grouped_ffn_backward")
+
+
+def moe_ep_reduce_home(plan, dP1_ranks, dP3_ranks, dP2_ranks, me, E, S, d, F, dW1, dW3, dW2, err,
+                       stream=None):
+    f32 = torch.float32
+    _check(lib().moe_ep_reduce_home(
+        _ptr(plan, torch.int32, "plan"), _table(dP1_ranks, "dP1_ranks"),
+        _table(dP3_ranks, "dP3_ranks"), _table(dP2_ranks, "dP2_ranks"), len(dP1_ranks), me, E,
+        S, d, F, _ptr(dW1, f32, "dW1"), _ptr(dW3, f32, "dW3"), _ptr(dW2, f32, "dW2"),
+        _ptr(err, torch.int32, "err"), _stream(stream)), "moe_ep_reduce_home")
+
+
+def moe_ep_dispatch_backward(dx_rows_ranks, perm, d, dx, err, stream=None):
+    T, k = perm.shape
+    _check(lib().moe_ep_dispatch_backward(
+        _table(dx_rows_ranks, "dx_rows_ranks"), _ptr(perm, torch.int32, "perm"),
+        len(dx_rows_ranks), T, k, d, _ptr(dx, torch.bfloat16, "dx"), _ptr(err, torch.int32, "err"),
+        _stream(stream)), "moe_ep_dispatch_backward")
 
 
 def ipc_export(t: torch.Tensor):

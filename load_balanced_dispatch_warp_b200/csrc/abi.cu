@@ -568,6 +568,106 @@ int moe_ep_combine(const moe_bf16* const* y_ranks, const int32_t* perm, const fl
                                 as_stream(stream));
 }
 
+int moe_ep_combine_backward(const moe_bf16* dout, const moe_bf16* const* y_ranks,
+                            const int32_t* perm, const float* gate, int W, int T, int k, int d,
+                            moe_bf16* const* dy_ranks, float* dgate, const int32_t* err,
+                            moe_stream_t stream) {
+  if (!err) return MOE_ERR_ARG;
+  if (T > 0 && (!dout || !perm || !gate || !dgate)) return MOE_ERR_ARG;
+  if (W < 1 || T < 0 || k < 1) return MOE_ERR_ARG;
+  if (W > MOE_EP_MAX_RANKS || k > 32) return MOE_ERR_SHAPE;
+  if ((int64_t)W * T * k >= kMaxElems) return MOE_ERR_SHAPE;
+  MOE_TRY(check_dims(T, k, d, 128));
+  if (T == 0) return MOE_OK;
+  MOE_TRY(check_table(y_ranks, W));
+  MOE_TRY(check_table(dy_ranks, W));
+  if (!aligned16(dout)) return MOE_ERR_ARG;
+  return moe::launch_ep_combine_backward(
+      reinterpret_cast<const __nv_bfloat16*>(dout),
+      reinterpret_cast<const __nv_bfloat16* const*>(y_ranks), perm, gate, W, T, k, d,
+      reinterpret_cast<__nv_bfloat16* const*>(dy_ranks), dgate, err, as_stream(stream));
+}
+
+int64_t moe_ep_ffn_backward_workspace_bytes(int T, int k, int E, int W, int S, int d, int F) {
+  if (check_ep(W, 0, T, k, E, S) != MOE_OK || check_dims(T, k, d, F) != MOE_OK) return -1;
+  if (E / W + S > 1024) return -1;
+  return moe::ep_ffn_backward_workspace_bytes(T, k, E, W, S, d, F);
+}
+
+int moe_ep_grouped_ffn_backward(const moe_bf16* recv, const moe_bf16* dy, const int32_t* plan,
+                                int W, int me, const moe_bf16* W1, const moe_bf16* W3,
+                                const moe_f16* W2, const moe_bf16* P1, const moe_bf16* P3,
+                                const moe_f16* P2, int T, int k, int E, int S, int d, int F,
+                                int32_t* groups_ws, moe_bf16* dx_rows, float* dP1, float* dP3,
+                                float* dP2, void* workspace, int64_t workspace_bytes,
+                                int32_t* err, moe_stream_t stream) {
+  if (!plan || !W1 || !W3 || !W2 || !groups_ws || !err || !dP1 || !dP3 || !dP2)
+    return MOE_ERR_ARG;
+  if (T > 0 && (!recv || !dy || !dx_rows || !workspace)) return MOE_ERR_ARG;
+  if (S > 0 && (!P1 || !P3 || !P2)) return MOE_ERR_ARG;
+  MOE_TRY(check_ep(W, me, T, k, E, S));
+  MOE_TRY(check_dims(T, k, d, F));
+  const int B = E / W;
+  if (B + S > 1024) return MOE_ERR_SHAPE;
+  if ((int64_t)(B + S) * F * d >= kMaxElems || (int64_t)T * k * 2 * F >= kMaxElems)
+    return MOE_ERR_SHAPE;
+  if (!aligned16(recv) || !aligned16(dy) || !aligned16(dx_rows) || !aligned16(W1) ||
+      !aligned16(W3) || !aligned16(W2) || !aligned16(groups_ws) || !aligned16(dP1) ||
+      !aligned16(dP3) || !aligned16(dP2) ||
+      (S > 0 && (!aligned16(P1) || !aligned16(P3) || !aligned16(P2))) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return MOE_ERR_ARG;
+  if (moe::ep_ffn_backward_workspace_bytes(T, k, E, W, S, d, F) > workspace_bytes)
+    return MOE_ERR_ARG;
+  moe_plan_layout L;
+  MOE_TRY(moe_plan_get_layout(E, W, S, &L));
+  cudaStream_t s = as_stream(stream);
+  const int C = T * k;
+  if (T > 0) MOE_TRY(moe::launch_ep_groups(plan, L, me, E, W, S, C, groups_ws, err, s));
+  return moe::launch_ep_grouped_ffn_backward(
+      reinterpret_cast<const __nv_bfloat16*>(recv), reinterpret_cast<const __nv_bfloat16*>(dy),
+      groups_ws, B, S, C, reinterpret_cast<const __nv_bfloat16*>(W1),
+      reinterpret_cast<const __nv_bfloat16*>(W3), reinterpret_cast<const __half*>(W2),
+      reinterpret_cast<const __nv_bfloat16*>(P1), reinterpret_cast<const __nv_bfloat16*>(P3),
+      reinterpret_cast<const __half*>(P2), d, F, reinterpret_cast<__nv_bfloat16*>(dx_rows), dP1,
+      dP3, dP2, workspace, workspace_bytes, err, s);
+}
+
+int moe_ep_reduce_home(const int32_t* plan, const float* const* dP1_ranks,
+                       const float* const* dP3_ranks, const float* const* dP2_ranks, int W,
+                       int me, int E, int S, int d, int F, float* dW1, float* dW3, float* dW2,
+                       const int32_t* err, moe_stream_t stream) {
+  if (!plan || !err || !dW1 || !dW3 || !dW2) return MOE_ERR_ARG;
+  MOE_TRY(check_ep(W, me, 0, 1, E, S));
+  MOE_TRY(check_dims(0, 1, d, F));
+  if ((int64_t)(E / W + S) * F * d >= kMaxElems) return MOE_ERR_SHAPE;
+  MOE_TRY(check_table(dP1_ranks, W));
+  MOE_TRY(check_table(dP3_ranks, W));
+  MOE_TRY(check_table(dP2_ranks, W));
+  if (!aligned16(dW1) || !aligned16(dW3) || !aligned16(dW2)) return MOE_ERR_ARG;
+  moe_plan_layout L;
+  MOE_TRY(moe_plan_get_layout(E, W, S, &L));
+  return moe::launch_ep_reduce_home(plan, L, dP1_ranks, dP3_ranks, dP2_ranks, W, me, E, S, d, F,
+                                    dW1, dW3, dW2, err, as_stream(stream));
+}
+
+int moe_ep_dispatch_backward(const moe_bf16* const* dx_rows_ranks, const int32_t* perm, int W,
+                             int T, int k, int d, moe_bf16* dx, const int32_t* err,
+                             moe_stream_t stream) {
+  if (!err) return MOE_ERR_ARG;
+  if (T > 0 && (!perm || !dx)) return MOE_ERR_ARG;
+  if (W < 1 || T < 0 || k < 1) return MOE_ERR_ARG;
+  if (W > MOE_EP_MAX_RANKS || k > 32) return MOE_ERR_SHAPE;
+  if ((int64_t)W * T * k >= kMaxElems) return MOE_ERR_SHAPE;
+  MOE_TRY(check_dims(T, k, d, 128));
+  if (T == 0) return MOE_OK;
+  MOE_TRY(check_table(dx_rows_ranks, W));
+  if (!aligned16(dx)) return MOE_ERR_ARG;
+  return moe::launch_ep_combine(reinterpret_cast<const __nv_bfloat16* const*>(dx_rows_ranks), W,
+                                perm, nullptr, T, k, d, reinterpret_cast<__nv_bfloat16*>(dx), err,
+                                as_stream(stream));
+}
+
 int moe_set_ffn_tile_mode(int mode) { return moe::set_ffn_tile_mode(mode); }
 
 int moe_ffn_tile_mode(void) { return moe::ffn_tile_mode(); }

@@ -28,7 +28,7 @@
 // The error word is read once at each kernel's start.  rank_kernel's blocks never write
 // it during the launch: their error bits collect in the workspace and the block that
 // finishes the last tile publishes them, so every block takes the same entry decision.
-#include "common.cuh"
+#include "rows.cuh"
 
 namespace moe {
 namespace {
@@ -410,22 +410,7 @@ __global__ void __launch_bounds__(kScatterThreads) scatter_kernel(ScatterArgs a)
 // dropped assignments, are not stored).
 constexpr int kRowVec = 4;
 
-// Where row r of the receive space lives: one buffer on this GPU, or (expert parallelism
-// across GPUs) rank r / C's buffer, local row r % C, through the pointer this process has
-// for it (its own buffer, or a peer GPU's mapped into this process).
-struct LocalRows {
-  uint4* base;
-  __device__ __forceinline__ uint4* row(int64_t r, int dv) const { return base + r * dv; }
-};
-struct RankRows {
-  uint4* base[MOE_EP_MAX_RANKS];
-  int C;
-  __device__ __forceinline__ uint4* row(int64_t r, int dv) const {
-    const int u = (int)(r / C);
-    return base[u] + (r - (int64_t)u * C) * dv;
-  }
-};
-
+// Dst (rows.cuh): the receive rows on this GPU (LocalRows) or on every rank (RankRows).
 template <class Dst>
 __global__ void __launch_bounds__(kScatterThreads) scatter_warp_kernel(
     const uint4* __restrict__ x, const int32_t* __restrict__ perm, int T, int k, int dv,

@@ -133,9 +133,10 @@ __global__ void __launch_bounds__(kPlanThreads) ep_plan_kernel(
 
 // The group table of rank `me`, re-based for its own buffers: row_start - me*C (local
 // receive rows), weight_ref e -> e - me*B (its home tensors hold experts [me*B, me*B+B)),
-// E + me*S + s -> B + s (its own pool slot s).  Unused entries stay all -1.  A group
-// whose weights are not on this rank (never produced by the plan) raises
-// MOE_DERR_ID_RANGE and is dropped.
+// E + me*S + s -> B + s (its own pool slot s); the expert field gets the same local index
+// (the backward keys its weight gradients on it: home experts, then slots).  Unused
+// entries stay all -1.  A group whose weights are not on this rank (never produced by the
+// plan) raises MOE_DERR_ID_RANGE and is dropped.
 __global__ void __launch_bounds__(128) ep_groups_kernel(const int32_t* __restrict__ plan,
                                                         moe_plan_layout L, int me, int E,
                                                         int W, int S, int C,
@@ -154,6 +155,7 @@ __global__ void __launch_bounds__(128) ep_groups_kernel(const int32_t* __restric
       const bool ok = (ref < E) ? (local >= 0 && local < B) : (local >= B && local < B + S);
       if (ok) {
         v.x -= me * C;
+        v.z = local;
         v.w = local;
       } else {
         atomicOr(err, MOE_DERR_ID_RANGE);

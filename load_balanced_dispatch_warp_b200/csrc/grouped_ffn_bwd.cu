@@ -28,7 +28,7 @@
 // and stored as bf16, the type dY needs its partner to have.
 #include <cuda.h>
 
-#include "common.cuh"
+#include "rows.cuh"
 
 namespace moe {
 namespace {
@@ -59,6 +59,8 @@ struct BwdArgs {
   int out_ld;           // columns of the output tensor
   int bf16;             // operand type: 1 bf16, 0 fp16
   int kb_split;         // B read MN-major: K steps below it from tm_b0, the rest from tm_b1
+  int e_home;           // row tiles: experts of the home maps (tm_b*); a group whose expert
+                        // index is e_home or above reads pool slot index - e_home from tm_p*
   void* out;
   int32_t* err;
   // SwiGLU backward epilogue: reads dH [rows, F] fp32, writes dG | dU into dGU [rows, 2F]
@@ -203,7 +205,9 @@ struct BTile {
   int valid_rows;  // rows of the block to store
   int b_row;       // first B row
   int n_block;
-  int e;               // row tiles: the group's expert
+  int e;               // row tiles: the group's weights inside their tensor; weight-gradient
+                       // tiles: the output expert
+  bool pool;           // row tiles: B from the pool maps
   int seg_lo, seg_hi;  // weight-gradient tiles: the expert's K segments
   int64_t out_off;     // element offset of the tile's first output row and column
 };
@@ -237,9 +241,12 @@ __device__ __forceinline__ BTile decode(int t, const BwdArgs& a, const int* s_pr
     const int m_local = mt - s_prefix[lo];
     tl.a_row = g.x + m_local * BM;
     tl.valid_rows = min(BM, g.y - m_local * BM);
-    // a replica slot holds its expert's weights bitwise: read the home tensor
-    tl.b_row = g.z * a.rows_per_expert + tl.n_block * a.bn_out;
-    tl.e = g.z;
+    // g.z indexes the weights: experts below e_home in the home maps (a replica slot holds
+    // its expert's weights bitwise, so on one GPU every group reads the home tensor), the
+    // rest in the pool maps (a rank of the expert-parallel layer reads its own slots)
+    tl.pool = g.z >= a.e_home;
+    tl.e = tl.pool ? g.z - a.e_home : g.z;  // index inside its tensor (home or pool)
+    tl.b_row = tl.e * a.rows_per_expert + tl.n_block * a.bn_out;
     tl.seg_lo = tl.seg_hi = 0;
     tl.out_off = (int64_t)tl.a_row * a.out_ld + (int64_t)tl.n_block * a.bn_out;
   }
@@ -268,7 +275,9 @@ template <int EPI, bool WGRAD, bool BMN>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
     bwd_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
                     const __grid_constant__ CUtensorMap tm_b0,
-                    const __grid_constant__ CUtensorMap tm_b1, const BwdArgs args) {
+                    const __grid_constant__ CUtensorMap tm_b1,
+                    const __grid_constant__ CUtensorMap tm_p0,
+                    const __grid_constant__ CUtensorMap tm_p1, const BwdArgs args) {
   constexpr bool TWO_B = EPI == EPI_SWIGLU_BWD;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -365,10 +374,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
               const int krow = tl.e * args.rows_per_expert + (lo ? kb : kb - args.kb_split) * BK;
               const int n0 = tl.n_block * args.bn_out;
               for (int c = 0; c < args.mma_n / 64; ++c)
-                tma_load_2d(sb + c * 8192, lo ? &tm_b0 : &tm_b1, fb, n0 + c * 64, krow);
+                tma_load_2d(sb + c * 8192,
+                            lo ? (tl.pool ? &tm_p0 : &tm_b0) : (tl.pool ? &tm_p1 : &tm_b1), fb,
+                            n0 + c * 64, krow);
             } else {
-              tma_load_2d(sb, &tm_b0, fb, kb * BK, tl.b_row);
-              if (TWO_B) tma_load_2d(sb + (b_bytes >> 1), &tm_b1, fb, kb * BK, tl.b_row);
+              tma_load_2d(sb, tl.pool ? &tm_p0 : &tm_b0, fb, kb * BK, tl.b_row);
+              if (TWO_B)
+                tma_load_2d(sb + (b_bytes >> 1), tl.pool ? &tm_p1 : &tm_b1, fb, kb * BK, tl.b_row);
             }
           }
           issued_mask |= 1u << stage;
@@ -673,9 +685,12 @@ __global__ void __launch_bounds__(256) transpose_kernel(
 
 // Backward of combine: dy[perm[t,j]] = gate[t,j] * dout[t] (bf16), dgate[t,j] =
 // <dout[t], y[perm[t,j]]> (fp32).  One warp per token, 16-byte vectors.
+// YSrc / DySink (rows.cuh): y read and dy written on this GPU, or on every rank of the
+// expert-parallel layer through its row tables (peer loads and stores).
+template <class YSrc, class DySink>
 __global__ void __launch_bounds__(256) combine_backward_kernel(
-    const uint4* __restrict__ dout, const uint4* __restrict__ y, const int32_t* __restrict__ perm,
-    const float* __restrict__ gate, int T, int k, int dv, uint4* __restrict__ dy,
+    const uint4* __restrict__ dout, const __grid_constant__ YSrc y, const int32_t* __restrict__ perm,
+    const float* __restrict__ gate, int T, int k, int dv, const __grid_constant__ DySink dy,
     float* __restrict__ dgate, const int32_t* __restrict__ err) {
   if (load_err(err)) return;
   const int lane = threadIdx.x & 31;
@@ -687,7 +702,7 @@ __global__ void __launch_bounds__(256) combine_backward_kernel(
       float dot = 0.f;
       for (int v = lane; v < dv; v += 32) {
         const uint4 a = __ldg(dout + t * dv + v);
-        const uint4 b = __ldcs(y + (int64_t)r * dv + v);
+        const uint4 b = __ldcs(y.row(r, dv) + v);
         const __nv_bfloat162* ap = reinterpret_cast<const __nv_bfloat162*>(&a);
         const __nv_bfloat162* bp = reinterpret_cast<const __nv_bfloat162*>(&b);
         uint32_t o[4];
@@ -699,7 +714,7 @@ __global__ void __launch_bounds__(256) combine_backward_kernel(
           dot = fmaf(af.y, bf.y, dot);
           o[i] = pack_bf16(gj * af.x, gj * af.y);
         }
-        dy[(int64_t)r * dv + v] = make_uint4(o[0], o[1], o[2], o[3]);
+        dy.row(r, dv)[v] = make_uint4(o[0], o[1], o[2], o[3]);
       }
       dot = warp_sum(dot);
       if (lane == 0) dgate[t * k + j] = dot;
@@ -770,7 +785,8 @@ size_t bwd_smem_bytes() {
 
 template <int EPI, bool WGRAD, bool BMN = false>
 int launch_bwd_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                    const BwdArgs& args, cudaStream_t s) {
+                    const CUtensorMap& p0, const CUtensorMap& p1, const BwdArgs& args,
+                    cudaStream_t s) {
   static bool configured[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -781,7 +797,7 @@ int launch_bwd_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorM
       return MOE_ERR_LAUNCH;
     configured[dev] = true;
   }
-  bwd_gemm_kernel<EPI, WGRAD, BMN><<<num_sms(), BWD_THREADS, smem, s>>>(a, b0, b1, args);
+  bwd_gemm_kernel<EPI, WGRAD, BMN><<<num_sms(), BWD_THREADS, smem, s>>>(a, b0, b1, p0, p1, args);
   return launch_status();
 }
 
@@ -798,42 +814,270 @@ int transpose(const void* in, int cols, int64_t ld_in, int64_t in_bstride, void*
   return launch_status();
 }
 
-// Workspace carve-up (every piece 256-byte aligned).
+// Workspace carve-up (every piece 256-byte aligned).  RC rows, Eo experts in the weight
+// gradients (the home experts, then -- for a rank of the expert-parallel layer -- its pool
+// slots), G group records.
 struct BwdWs {
-  __nv_bfloat16* w2t;   // [E*F, d] (W2 transposed, rounded to bf16)
+  __nv_bfloat16* w2t;   // [Eo*F, d] (W2, and the pool's P2, transposed, rounded to bf16)
   float* dh;            // [RC, F]
   __nv_bfloat16* dgu;   // [RC, 2F]
   __nv_bfloat16* hb;    // [RC, F] h = silu(g) u recomputed, bf16
-  int* seg_off;         // [E+1]
+  int* seg_off;         // [Eo+1]
   int2* segs;           // [G]
   int64_t bytes;
 };
 
-BwdWs carve(uint8_t* base, int T, int k, int E, int R, int S, int d, int F, int G) {
+BwdWs carve(uint8_t* base, int64_t RC, int Eo, int d, int F, int G) {
   BwdWs w{};
-  const int64_t RC = (int64_t)T * k;
   int64_t off = 0;
   auto take = [&](int64_t bytes) {
     const int64_t at = off;
     off += (bytes + 255) / 256 * 256;
     return base ? base + at : nullptr;
   };
-  w.w2t = reinterpret_cast<__nv_bfloat16*>(take((int64_t)E * F * d * 2));
+  w.w2t = reinterpret_cast<__nv_bfloat16*>(take((int64_t)Eo * F * d * 2));
   w.dh = reinterpret_cast<float*>(take(RC * F * 4));
   w.dgu = reinterpret_cast<__nv_bfloat16*>(take(RC * 2 * F * 2));
   w.hb = reinterpret_cast<__nv_bfloat16*>(take(RC * F * 2));
-  w.seg_off = reinterpret_cast<int*>(take((int64_t)(E + 1) * 4));
+  w.seg_off = reinterpret_cast<int*>(take((int64_t)(Eo + 1) * 4));
   w.segs = reinterpret_cast<int2*>(take((int64_t)G * 8));
   w.bytes = off;
-  (void)R;
-  (void)S;
   return w;
+}
+
+// The grouped-FFN backward over a group table of G records {row_start, rows, weight index,
+// -} on RC rows: weight index z < e_home reads the home tensors (W1, W3, W2), z >= e_home
+// pool slot z - e_home (P1, P3, P2, n_pool slots); the weight gradients dW* hold Eo =
+// e_home + n_pool entries, each the sum over every group with that index.
+int grouped_ffn_backward_impl(const __nv_bfloat16* recv, const __nv_bfloat16* dy,
+                              const int4* groups, int G, int64_t RC, int e_home, int n_pool,
+                              const __nv_bfloat16* W1, const __nv_bfloat16* W3, const __half* W2,
+                              const __nv_bfloat16* P1, const __nv_bfloat16* P3, const __half* P2,
+                              int d, int F, __nv_bfloat16* dx_rows, float* dW1, float* dW3,
+                              float* dW2, void* workspace, int64_t workspace_bytes, int32_t* err,
+                              cudaStream_t s) {
+  const int Eo = e_home + n_pool;
+  BwdWs w = carve(static_cast<uint8_t*>(workspace), RC, Eo, d, F, G);
+  if (w.bytes > workspace_bytes) return MOE_ERR_ARG;
+  int st;
+  // weight gradients of entries without rows are zero; the GEMMs below write every tile
+  // (an entry with no K steps stores zeros), and with no rows nothing else runs
+  if (RC == 0) {
+    if (cudaMemsetAsync(dW1, 0, (size_t)Eo * F * d * 4, s) != cudaSuccess ||
+        cudaMemsetAsync(dW3, 0, (size_t)Eo * F * d * 4, s) != cudaSuccess ||
+        cudaMemsetAsync(dW2, 0, (size_t)Eo * d * F * 4, s) != cudaSuccess)
+      return MOE_ERR_LAUNCH;
+    return MOE_OK;
+  }
+  // 1. per-entry lists of group row ranges (the weight gradients' K steps)
+  bwd_prepare_kernel<<<1, 1024, 0, s>>>(groups, G, Eo, w.seg_off, w.segs, err);
+  if ((st = launch_status()) != MOE_OK) return st;
+  // 2. W2T[z] = W2[z]^T [F,d], rounded to bf16, the pool's slots after the home experts (the
+  //    dH GEMM reads it K-major; W1 and W3 are read MN-major by the dX GEMM, no copy)
+  if ((st = transpose(W2, F, F, (int64_t)d * F, w.w2t, d, (int64_t)F * d, d, nullptr, nullptr,
+                      e_home, true, err, s)))
+    return st;
+  if (n_pool > 0 &&
+      (st = transpose(P2, F, F, (int64_t)d * F, w.w2t + (int64_t)e_home * F * d, d,
+                      (int64_t)F * d, d, nullptr, nullptr, n_pool, true, err, s)))
+    return st;
+  const int bnF = (F % 256 == 0) ? 256 : 128;
+  const int bnD = (d % 256 == 0) ? 256 : 128;
+  BwdArgs base{};
+  base.groups = groups;
+  base.G = G;
+  base.err = err;
+  base.E = Eo;
+  base.F = F;
+  base.e_home = Eo;  // dH reads W2T, which holds every entry
+  // 3. dH = dY W2 (per group, fp32 out)
+  {
+    CUtensorMap ma, mb;
+    if (!make_map16(&ma, dy, RC, d, d, BM, true) ||
+        !make_map16(&mb, w.w2t, (int64_t)Eo * F, d, d, bnF, true))
+      return MOE_ERR_DEVICE;
+    BwdArgs a = base;
+    a.n_blocks_n = F / bnF;
+    a.k_blocks = d / BK;
+    a.bn_out = bnF;
+    a.mma_n = bnF;
+    a.rows_per_expert = F;
+    a.out_ld = F;
+    a.bf16 = 1;
+    a.out = w.dh;
+    if ((st = launch_bwd_gemm<EPI_F32, false>(ma, mb, mb, mb, mb, a, s))) return st;
+  }
+  // 4. dG, dU: the gate/up GEMM re-run on the rows, SwiGLU backward in the epilogue (which
+  //    also stores h = silu(g) u in bf16 for dW2)
+  {
+    CUtensorMap ma, m1, m3, p1, p3;
+    if (!make_map16(&ma, recv, RC, d, d, BM, true) ||
+        !make_map16(&m1, W1, (int64_t)e_home * F, d, d, 128, true) ||
+        !make_map16(&m3, W3, (int64_t)e_home * F, d, d, 128, true))
+      return MOE_ERR_DEVICE;
+    if (n_pool > 0) {
+      if (!make_map16(&p1, P1, (int64_t)n_pool * F, d, d, 128, true) ||
+          !make_map16(&p3, P3, (int64_t)n_pool * F, d, d, 128, true))
+        return MOE_ERR_DEVICE;
+    } else {
+      p1 = m1;
+      p3 = m3;
+    }
+    BwdArgs a = base;
+    a.e_home = e_home;
+    a.n_blocks_n = F / 128;
+    a.k_blocks = d / BK;
+    a.bn_out = 128;
+    a.mma_n = 256;
+    a.rows_per_expert = F;
+    a.out_ld = 2 * F;
+    a.bf16 = 1;
+    a.dh = w.dh;
+    a.dgu = w.dgu;
+    a.hb = w.hb;
+    if ((st = launch_bwd_gemm<EPI_SWIGLU_BWD, false>(ma, m1, m3, p1, p3, a, s))) return st;
+  }
+  // 5. dX rows = [dG | dU] [W1; W3] (K = 2F, bf16): B read MN-major from W1 (K steps below
+  //    F/64) and W3 (the rest), each as [rows, d columns] in boxes of 64 x 64
+  {
+    CUtensorMap ma, m1, m3, p1, p3;
+    if (!make_map16(&ma, w.dgu, RC, 2 * F, 2 * F, BM, true) ||
+        !make_map16(&m1, W1, (int64_t)e_home * F, d, d, 64, true) ||
+        !make_map16(&m3, W3, (int64_t)e_home * F, d, d, 64, true))
+      return MOE_ERR_DEVICE;
+    if (n_pool > 0) {
+      if (!make_map16(&p1, P1, (int64_t)n_pool * F, d, d, 64, true) ||
+          !make_map16(&p3, P3, (int64_t)n_pool * F, d, d, 64, true))
+        return MOE_ERR_DEVICE;
+    } else {
+      p1 = m1;
+      p3 = m3;
+    }
+    BwdArgs a = base;
+    a.e_home = e_home;
+    a.n_blocks_n = d / bnD;
+    a.k_blocks = 2 * F / BK;
+    a.kb_split = F / BK;
+    a.bn_out = bnD;
+    a.mma_n = bnD;
+    a.rows_per_expert = F;
+    a.out_ld = d;
+    a.bf16 = 1;
+    a.out = dx_rows;
+    if ((st = launch_bwd_gemm<EPI_BF16, false, true>(ma, m1, m3, p1, p3, a, s))) return st;
+  }
+  // 6. weight gradients, every group of an entry in one accumulator (on one GPU: a home
+  //    expert's home and replica groups alike); A and B are the row-major activations
+  //    read MN-major in boxes of 64 rows x 64 columns
+  {
+    CUtensorMap ma, mb;
+    if (!make_map16(&ma, dy, RC, d, d, 64, true) || !make_map16(&mb, w.hb, RC, F, F, 64, true))
+      return MOE_ERR_DEVICE;
+    BwdArgs a = base;
+    a.n_blocks_n = F / bnF;
+    a.bn_out = bnF;
+    a.mma_n = bnF;
+    a.out_ld = F;
+    a.bf16 = 1;
+    a.out = dW2;
+    a.seg_off = w.seg_off;
+    a.segs = w.segs;
+    a.m_blocks = d / BM;
+    a.a_row_base = 0;
+    a.out_expert_stride = (int64_t)d * F;
+    if ((st = launch_bwd_gemm<EPI_F32, true>(ma, mb, mb, mb, mb, a, s))) return st;
+  }
+  {
+    CUtensorMap ma, mb;
+    if (!make_map16(&ma, w.dgu, RC, 2 * F, 2 * F, 64, true) ||
+        !make_map16(&mb, recv, RC, d, d, 64, true))
+      return MOE_ERR_DEVICE;
+    BwdArgs a = base;
+    a.n_blocks_n = d / bnD;
+    a.bn_out = bnD;
+    a.mma_n = bnD;
+    a.out_ld = d;
+    a.bf16 = 1;
+    a.seg_off = w.seg_off;
+    a.segs = w.segs;
+    a.m_blocks = F / BM;
+    a.out_expert_stride = (int64_t)F * d;
+    a.a_row_base = 0;
+    a.out = dW1;
+    if ((st = launch_bwd_gemm<EPI_F32, true>(ma, mb, mb, mb, mb, a, s))) return st;
+    a.a_row_base = F;
+    a.out = dW3;
+    if ((st = launch_bwd_gemm<EPI_F32, true>(ma, mb, mb, mb, mb, a, s))) return st;
+  }
+  return MOE_OK;
+}
+
+// Replica gradients reduced back home across ranks: home expert e_local of rank me gets its
+// own partial plus, in (rank, slot) order, the partial of every pool slot (v, s) of the
+// job's plan that held a copy of it, read from rank v's partials through the rank tables.
+// parts[p][v] -> rank v's [B+S][n4] partials of projection p (fp32, 16-byte vectors).
+struct RankParts {
+  const float4* p[3][MOE_EP_MAX_RANKS];
+};
+
+__global__ void __launch_bounds__(256) ep_reduce_home_kernel(
+    const int32_t* __restrict__ rep, int W, int me, int B, int S, int64_t n4,
+    const __grid_constant__ RankParts parts, float4* __restrict__ dW1, float4* __restrict__ dW3,
+    float4* __restrict__ dW2, const int32_t* __restrict__ err) {
+  __shared__ int s_src[MOE_EP_MAX_RANKS];  // v * S + s of the copies, in order (a rank's
+                                          // slots hold distinct experts: at most W copies)
+  __shared__ int s_n;
+  if (block_should_stop(err)) return;
+  constexpr int kChunk = 256 * 4;  // float4 vectors per block and step
+  const int64_t chunks = (n4 + kChunk - 1) / kChunk;
+  const int64_t total = (int64_t)B * 3 * chunks;
+  int cur = -1;
+  for (int64_t w = blockIdx.x; w < total; w += gridDim.x) {
+    const int el = (int)(w / (3 * chunks));
+    const int64_t rem = w - (int64_t)el * 3 * chunks;
+    const int proj = (int)(rem / chunks);
+    const int64_t c = rem - (int64_t)proj * chunks;
+    if (el != cur) {  // the copies of expert me*B + el, found once per expert
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        int n = 0;
+        const int e = me * B + el;
+        for (int q = 0; q < W * S && n < MOE_EP_MAX_RANKS; ++q)
+          if (__ldg(rep + q) == e) s_src[n++] = q;
+        s_n = n;
+      }
+      __syncthreads();
+      cur = el;
+    }
+    float4* out = (proj == 0 ? dW1 : proj == 1 ? dW3 : dW2) + (int64_t)el * n4;
+    const float4* own = parts.p[proj][me] + (int64_t)el * n4;
+    const int n = s_n;
+    for (int64_t v = c * kChunk + threadIdx.x; v < min(n4, (c + 1) * kChunk); v += blockDim.x) {
+      float4 a = __ldcs(own + v);
+      for (int i = 0; i < n; ++i) {
+        const int q = s_src[i];
+        const float4 b = __ldcs(parts.p[proj][q / S] + (int64_t)(B + q % S) * n4 + v);
+        a.x += b.x;
+        a.y += b.y;
+        a.z += b.z;
+        a.w += b.w;
+      }
+      out[v] = a;
+    }
+  }
 }
 
 }  // namespace
 
 int64_t ffn_backward_workspace_bytes(int T, int k, int E, int R, int S, int d, int F, int G) {
-  return carve(nullptr, T, k, E, R, S, d, F, G).bytes;
+  (void)R;
+  (void)S;
+  return carve(nullptr, (int64_t)T * k, E, d, F, G).bytes;
+}
+
+int64_t ep_ffn_backward_workspace_bytes(int T, int k, int E, int W, int S, int d, int F) {
+  const int B = E / W;
+  return carve(nullptr, (int64_t)T * k, B + S, d, F, B + S).bytes;
 }
 
 int launch_combine_backward(const __nv_bfloat16* dout, const __nv_bfloat16* y,
@@ -843,9 +1087,9 @@ int launch_combine_backward(const __nv_bfloat16* dout, const __nv_bfloat16* y,
   if (T == 0) return MOE_OK;
   const int64_t want = ((int64_t)T + 7) / 8;
   const int64_t cap = (int64_t)num_sms() * 8;
-  combine_backward_kernel<<<(unsigned)(want < cap ? want : cap), 256, 0, s>>>(
-      reinterpret_cast<const uint4*>(dout), reinterpret_cast<const uint4*>(y), perm, gate, T, k,
-      d / 8, reinterpret_cast<uint4*>(dy), dgate, err);
+  combine_backward_kernel<LocalY, LocalRows><<<(unsigned)(want < cap ? want : cap), 256, 0, s>>>(
+      reinterpret_cast<const uint4*>(dout), LocalY{reinterpret_cast<const uint4*>(y)}, perm, gate,
+      T, k, d / 8, LocalRows{reinterpret_cast<uint4*>(dy)}, dgate, err);
   return launch_status();
 }
 
@@ -868,138 +1112,64 @@ int launch_grouped_ffn_backward(const __nv_bfloat16* recv, const __nv_bfloat16* 
                                 float* dW2, void* workspace, int64_t workspace_bytes,
                                 int32_t* err, cudaStream_t s) {
   (void)h;  // not read: the SwiGLU-backward epilogue recomputes h (in bf16) for dW2
-  const int G = R * L.max_groups_per_rank;
-  BwdWs w = carve(static_cast<uint8_t*>(workspace), T, k, E, R, S, d, F, G);
-  if (w.bytes > workspace_bytes) return MOE_ERR_ARG;
-  const int64_t RC = (int64_t)T * k;
-  const int4* groups = reinterpret_cast<const int4*>(plan + L.groups);
-  int st;
-  // weight gradients of experts without rows are zero; the GEMMs below write every tile
-  // (an expert with no K steps stores zeros), and with T == 0 nothing else runs
-  if (T == 0) {
-    if (cudaMemsetAsync(dW1, 0, (size_t)E * F * d * 4, s) != cudaSuccess ||
-        cudaMemsetAsync(dW3, 0, (size_t)E * F * d * 4, s) != cudaSuccess ||
-        cudaMemsetAsync(dW2, 0, (size_t)E * d * F * 4, s) != cudaSuccess)
-      return MOE_ERR_LAUNCH;
-    return MOE_OK;
+  (void)S;
+  // the plan's groups name their expert in z; every group reads the home tensors
+  return grouped_ffn_backward_impl(recv, dy, reinterpret_cast<const int4*>(plan + L.groups),
+                                   R * L.max_groups_per_rank, (int64_t)T * k, E, 0, W1, W3, W2,
+                                   nullptr, nullptr, nullptr, d, F, dx_rows, dW1, dW3, dW2,
+                                   workspace, workspace_bytes, err, s);
+}
+
+int launch_ep_combine_backward(const __nv_bfloat16* dout, const __nv_bfloat16* const* y_ranks,
+                               const int32_t* perm, const float* gate, int W, int T, int k, int d,
+                               __nv_bfloat16* const* dy_ranks, float* dgate, const int32_t* err,
+                               cudaStream_t s) {
+  if (T == 0) return MOE_OK;
+  RankY yv;
+  RankRows dv;
+  for (int u = 0; u < MOE_EP_MAX_RANKS; ++u) {
+    yv.base[u] = u < W ? reinterpret_cast<const uint4*>(y_ranks[u]) : nullptr;
+    dv.base[u] = u < W ? reinterpret_cast<uint4*>(dy_ranks[u]) : nullptr;
   }
-  // 1. per-expert lists of group row ranges (the weight gradients' K steps)
-  bwd_prepare_kernel<<<1, 1024, 0, s>>>(groups, G, E, w.seg_off, w.segs, err);
-  if ((st = launch_status()) != MOE_OK) return st;
-  // 2. W2T[e] = W2[e]^T [F,d], rounded to bf16 (the dH GEMM reads it K-major; W1 and W3 are
-  //    read MN-major by the dX GEMM, no copy)
-  if ((st = transpose(W2, F, F, (int64_t)d * F, w.w2t, d, (int64_t)F * d, d, nullptr, nullptr, E,
-                      true, err, s)))
-    return st;
-  const int bnF = (F % 256 == 0) ? 256 : 128;
-  const int bnD = (d % 256 == 0) ? 256 : 128;
-  BwdArgs base{};
-  base.groups = groups;
-  base.G = G;
-  base.err = err;
-  base.E = E;
-  base.F = F;
-  // 3. dH = dY W2 (per group, fp16 -> fp32)
-  {
-    CUtensorMap ma, mb;
-    if (!make_map16(&ma, dy, RC, d, d, BM, true) ||
-        !make_map16(&mb, w.w2t, (int64_t)E * F, d, d, bnF, true))
-      return MOE_ERR_DEVICE;
-    BwdArgs a = base;
-    a.n_blocks_n = F / bnF;
-    a.k_blocks = d / BK;
-    a.bn_out = bnF;
-    a.mma_n = bnF;
-    a.rows_per_expert = F;
-    a.out_ld = F;
-    a.bf16 = 1;
-    a.out = w.dh;
-    if ((st = launch_bwd_gemm<EPI_F32, false>(ma, mb, mb, a, s))) return st;
+  yv.C = dv.C = T * k;
+  const int64_t want = ((int64_t)T + 7) / 8;
+  const int64_t cap = (int64_t)num_sms() * 8;
+  combine_backward_kernel<RankY, RankRows><<<(unsigned)(want < cap ? want : cap), 256, 0, s>>>(
+      reinterpret_cast<const uint4*>(dout), yv, perm, gate, T, k, d / 8, dv, dgate, err);
+  return launch_status();
+}
+
+int launch_ep_grouped_ffn_backward(const __nv_bfloat16* recv, const __nv_bfloat16* dy,
+                                   const int32_t* groups, int B, int S, int C,
+                                   const __nv_bfloat16* W1, const __nv_bfloat16* W3,
+                                   const __half* W2, const __nv_bfloat16* P1,
+                                   const __nv_bfloat16* P3, const __half* P2, int d, int F,
+                                   __nv_bfloat16* dx_rows, float* dP1, float* dP3, float* dP2,
+                                   void* workspace, int64_t workspace_bytes, int32_t* err,
+                                   cudaStream_t s) {
+  // the re-based group table names each group's weights in z: home expert 0..B-1, pool
+  // slot B + s
+  return grouped_ffn_backward_impl(recv, dy, reinterpret_cast<const int4*>(groups), B + S,
+                                   (int64_t)C, B, S, W1, W3, W2, P1, P3, P2, d, F, dx_rows, dP1,
+                                   dP3, dP2, workspace, workspace_bytes, err, s);
+}
+
+int launch_ep_reduce_home(const int32_t* plan, const moe_plan_layout& L,
+                          const float* const* part1_ranks, const float* const* part3_ranks,
+                          const float* const* part2_ranks, int W, int me, int E, int S, int d,
+                          int F, float* dW1, float* dW3, float* dW2, const int32_t* err,
+                          cudaStream_t s) {
+  RankParts parts;
+  for (int u = 0; u < MOE_EP_MAX_RANKS; ++u) {
+    parts.p[0][u] = u < W ? reinterpret_cast<const float4*>(part1_ranks[u]) : nullptr;
+    parts.p[1][u] = u < W ? reinterpret_cast<const float4*>(part3_ranks[u]) : nullptr;
+    parts.p[2][u] = u < W ? reinterpret_cast<const float4*>(part2_ranks[u]) : nullptr;
   }
-  // 4. dG, dU: the gate/up GEMM re-run on the rows, SwiGLU backward in the epilogue (which
-  //    also stores h = silu(g) u in bf16 for dW2)
-  {
-    CUtensorMap ma, m1, m3;
-    if (!make_map16(&ma, recv, RC, d, d, BM, true) ||
-        !make_map16(&m1, W1, (int64_t)E * F, d, d, 128, true) ||
-        !make_map16(&m3, W3, (int64_t)E * F, d, d, 128, true))
-      return MOE_ERR_DEVICE;
-    BwdArgs a = base;
-    a.n_blocks_n = F / 128;
-    a.k_blocks = d / BK;
-    a.bn_out = 128;
-    a.mma_n = 256;
-    a.rows_per_expert = F;
-    a.out_ld = 2 * F;
-    a.bf16 = 1;
-    a.dh = w.dh;
-    a.dgu = w.dgu;
-    a.hb = w.hb;
-    if ((st = launch_bwd_gemm<EPI_SWIGLU_BWD, false>(ma, m1, m3, a, s))) return st;
-  }
-  // 5. dX rows = [dG | dU] [W1; W3] (K = 2F, bf16): B read MN-major from W1 (K steps below
-  //    F/64) and W3 (the rest), each as [E*F rows, d columns] in boxes of 64 x 64
-  {
-    CUtensorMap ma, m1, m3;
-    if (!make_map16(&ma, w.dgu, RC, 2 * F, 2 * F, BM, true) ||
-        !make_map16(&m1, W1, (int64_t)E * F, d, d, 64, true) ||
-        !make_map16(&m3, W3, (int64_t)E * F, d, d, 64, true))
-      return MOE_ERR_DEVICE;
-    BwdArgs a = base;
-    a.n_blocks_n = d / bnD;
-    a.k_blocks = 2 * F / BK;
-    a.kb_split = F / BK;
-    a.bn_out = bnD;
-    a.mma_n = bnD;
-    a.rows_per_expert = F;
-    a.out_ld = d;
-    a.bf16 = 1;
-    a.out = dx_rows;
-    if ((st = launch_bwd_gemm<EPI_BF16, false, true>(ma, m1, m3, a, s))) return st;
-  }
-  // 6. weight gradients, every group of an expert (home and replicas) in one accumulator;
-  //    A and B are the row-major activations read MN-major in boxes of 64 rows x 64 columns
-  {
-    CUtensorMap ma, mb;
-    if (!make_map16(&ma, dy, RC, d, d, 64, true) || !make_map16(&mb, w.hb, RC, F, F, 64, true))
-      return MOE_ERR_DEVICE;
-    BwdArgs a = base;
-    a.n_blocks_n = F / bnF;
-    a.bn_out = bnF;
-    a.mma_n = bnF;
-    a.out_ld = F;
-    a.bf16 = 1;
-    a.out = dW2;
-    a.seg_off = w.seg_off;
-    a.segs = w.segs;
-    a.m_blocks = d / BM;
-    a.a_row_base = 0;
-    a.out_expert_stride = (int64_t)d * F;
-    if ((st = launch_bwd_gemm<EPI_F32, true>(ma, mb, mb, a, s))) return st;
-  }
-  {
-    CUtensorMap ma, mb;
-    if (!make_map16(&ma, w.dgu, RC, 2 * F, 2 * F, 64, true) ||
-        !make_map16(&mb, recv, RC, d, d, 64, true))
-      return MOE_ERR_DEVICE;
-    BwdArgs a = base;
-    a.n_blocks_n = d / bnD;
-    a.bn_out = bnD;
-    a.mma_n = bnD;
-    a.out_ld = d;
-    a.bf16 = 1;
-    a.seg_off = w.seg_off;
-    a.segs = w.segs;
-    a.m_blocks = F / BM;
-    a.out_expert_stride = (int64_t)F * d;
-    a.a_row_base = 0;
-    a.out = dW1;
-    if ((st = launch_bwd_gemm<EPI_F32, true>(ma, mb, mb, a, s))) return st;
-    a.a_row_base = F;
-    a.out = dW3;
-    if ((st = launch_bwd_gemm<EPI_F32, true>(ma, mb, mb, a, s))) return st;
-  }
-  return MOE_OK;
+  const int64_t n4 = (int64_t)d * F / 4;
+  ep_reduce_home_kernel<<<num_sms() * 4, 256, 0, s>>>(
+      plan + L.replica_expert, W, me, E / W, S, n4, parts, reinterpret_cast<float4*>(dW1),
+      reinterpret_cast<float4*>(dW3), reinterpret_cast<float4*>(dW2), err);
+  return launch_status();
 }
 
 }  // namespace moe

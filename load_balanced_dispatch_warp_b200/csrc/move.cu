@@ -6,7 +6,7 @@
 // HBM they are gathers/scatters of whole rows.  Prefetch and zero-copy placement follow
 // the MoonEP news article, paragraph 3.  All of it is HBM-bound: 16-byte vector loads and
 // stores, each token row read once.
-#include "common.cuh"
+#include "rows.cuh"
 
 namespace moe {
 namespace {
@@ -124,25 +124,8 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float* a) {
 // to keep the gathers in flight.
 // DROP: an assignment with perm < 0 (dropped by the fixed-capacity dispatch) is left out
 // of the sum.
-// Src says where row r of y lives: one buffer on this GPU (LocalY), or (expert
-// parallelism across GPUs) rank r / C's y, local row r % C, read through this process's
-// pointer to it (RankY; a peer GPU's memory is read over NVLink).  Both sum the same
-// values in the same order.
-struct LocalY {
-  const uint4* base;
-  __device__ __forceinline__ const uint4* row(int r, int dv) const {
-    return base + (int64_t)r * dv;
-  }
-};
-struct RankY {
-  const uint4* base[MOE_EP_MAX_RANKS];
-  int C;
-  __device__ __forceinline__ const uint4* row(int r, int dv) const {
-    const int u = r / C;
-    return base[u] + (int64_t)(r - u * C) * dv;
-  }
-};
-
+// Src (rows.cuh) says where row r of y lives: LocalY or RankY; both sum the same values in
+// the same order.
 template <int K, bool DROP = false, int kCombVec = (K > 4 || K == 0) ? 1 : 2, class Src = LocalY>
 __global__ void __launch_bounds__(kRowThreads) combine_kernel(
     const __grid_constant__ Src y, const int32_t* __restrict__ perm,

@@ -31,11 +31,14 @@ from __future__ import annotations
 
 import torch
 
-from . import (dispatch_workspace_words, ipc_close, ipc_export, ipc_import, moe_ep_combine,
-               moe_ep_counts, moe_ep_dispatch, moe_ep_grouped_ffn, moe_ep_plan,
-               moe_ep_prefetch, moe_topk, plan_layout)
+from . import (dispatch_workspace_words, ep_ffn_backward_workspace_bytes, ipc_close, ipc_export,
+               ipc_import, moe_ep_combine, moe_ep_combine_backward, moe_ep_counts,
+               moe_ep_dispatch, moe_ep_dispatch_backward, moe_ep_grouped_ffn,
+               moe_ep_grouped_ffn_backward, moe_ep_plan, moe_ep_prefetch, moe_ep_reduce_home,
+               moe_topk, moe_topk_backward, plan_layout)
 
 SHARED = ("recv", "y", "W1", "W3", "W2")  # the buffers every rank addresses on its peers
+SHARED_BWD = ("dy", "dx_rows", "dP1", "dP3", "dP2")  # and those of the backward
 
 
 class EPRank:
@@ -81,6 +84,34 @@ class EPRank:
     def shared(self) -> dict:
         return {"recv": self.recv, "y": self.y, "W1": self.W1, "W3": self.W3, "W2": self.W2}
 
+    def alloc_backward(self):
+        """Buffers of the backward: dy and dx rows [C,d], the weight-gradient partials of
+        its groups [B+S,...] (home experts, then pool slots), the home experts' gradients
+        [B,...], dx [T,d], dlogits [T,E]."""
+        if hasattr(self, "dy"):
+            return
+        dev = self.W1.device
+        f32, bf = torch.float32, torch.bfloat16
+        B, S, F, d, C, T = self.B, self.S, self.F, self.d, self.C, self.T
+        self.dy = torch.zeros(C, d, dtype=bf, device=dev)
+        self.dgate = torch.zeros(T, self.k, dtype=f32, device=dev)
+        self.dx_rows = torch.zeros(C, d, dtype=bf, device=dev)
+        self.dP1 = torch.zeros(B + S, F, d, dtype=f32, device=dev)
+        self.dP3 = torch.zeros(B + S, F, d, dtype=f32, device=dev)
+        self.dP2 = torch.zeros(B + S, d, F, dtype=f32, device=dev)
+        self.dW1 = torch.zeros(B, F, d, dtype=f32, device=dev)
+        self.dW3 = torch.zeros(B, F, d, dtype=f32, device=dev)
+        self.dW2 = torch.zeros(B, d, F, dtype=f32, device=dev)
+        self.dx = torch.zeros(T, d, dtype=bf, device=dev)
+        self.dlogits = torch.zeros(T, self.E, dtype=f32, device=dev)
+        ws = ep_ffn_backward_workspace_bytes(T, self.k, self.E, self.W, S, d, F)
+        self.bwd_ws = torch.zeros(max(ws, 256), dtype=torch.uint8, device=dev)
+
+    def shared_backward(self) -> dict:
+        self.alloc_backward()
+        return {"dy": self.dy, "dx_rows": self.dx_rows, "dP1": self.dP1, "dP3": self.dP3,
+                "dP2": self.dP2}
+
     # ---- the steps, in order
     def route(self, logits):
         moe_topk(logits, self.k, self.idx, self.gate, self.err)
@@ -106,6 +137,32 @@ class EPRank:
 
     def combine(self):
         moe_ep_combine(self.tables["y"], self.perm, self.gate, self.d, self.out, self.err)
+
+    # ---- the backward steps, in order (the tables must hold SHARED_BWD too)
+    def bwd_combine(self, dout):
+        moe_ep_combine_backward(dout, self.tables["y"], self.perm, self.gate, self.tables["dy"],
+                                self.dgate, self.err)
+
+    def bwd_ffn(self):
+        moe_ep_grouped_ffn_backward(self.recv, self.dy, self.plan, self.W, self.me, self.W1,
+                                    self.W3, self.W2, self.P1, self.P3, self.P2, self.T, self.k,
+                                    self.E, self.S, self.groups_ws, self.dx_rows, self.dP1,
+                                    self.dP3, self.dP2, self.bwd_ws, self.err)
+
+    def bwd_reduce(self):
+        t = self.tables
+        moe_ep_reduce_home(self.plan, t["dP1"], t["dP3"], t["dP2"], self.me, self.E, self.S,
+                           self.d, self.F, self.dW1, self.dW3, self.dW2, self.err)
+
+    def bwd_dispatch(self):
+        moe_ep_dispatch_backward(self.tables["dx_rows"], self.perm, self.d, self.dx, self.err)
+
+    def bwd_gates(self):
+        moe_topk_backward(self.gate, self.dgate, self.idx, self.E, self.dlogits, self.err)
+
+    def grads(self) -> dict:
+        return {"dx": self.dx, "dlogits": self.dlogits, "dW1": self.dW1, "dW3": self.dW3,
+                "dW2": self.dW2}
 
 
 def exchange_pointers(local: dict, me: int, W: int, gather_objects, export, import_base):
@@ -200,13 +257,19 @@ class EPLayer:
     """One rank of the expert-parallel layer (one process per GPU).
 
     ``forward(logits, x)`` runs one step on this rank's T tokens and returns its [T,d]
-    output.  Weights are shared with the peers through the pointer tables: a caller that
-    updates them in place must make every rank finish its step first."""
+    output; with ``backward=True`` the backward buffers are shared too and
+    ``backward(dout)`` returns this rank's dx, dlogits and its home experts' weight
+    gradients (replica gradients reduced back home).  Weights are shared with the peers
+    through the pointer tables: a caller that updates them in place must make every rank
+    finish its step first."""
 
-    def __init__(self, comm, T: int, E: int, k: int, S: int, W1, W3, W2):
+    def __init__(self, comm, T: int, E: int, k: int, S: int, W1, W3, W2, backward=False):
         self.comm = comm
         self.rank = EPRank(comm.rank, comm.world, T, E, k, S, W1, W3, W2)
-        self.rank.tables, self._bases = comm.pointer_tables(self.rank.shared())
+        local = dict(self.rank.shared())
+        if backward:
+            local.update(self.rank.shared_backward())
+        self.rank.tables, self._bases = comm.pointer_tables(local)
 
     def forward(self, logits, x):
         r = self.rank
@@ -220,6 +283,19 @@ class EPLayer:
         self.comm.barrier()
         r.combine()
         return r.out
+
+    def backward(self, dout):
+        r = self.rank
+        if "dy" not in r.tables:
+            raise RuntimeError("EPLayer(..., backward=True) shares the backward buffers")
+        r.bwd_combine(dout)
+        self.comm.barrier()  # every rank's dy rows written
+        r.bwd_ffn()
+        self.comm.barrier()  # every rank's dx rows and partial gradients written
+        r.bwd_reduce()
+        r.bwd_dispatch()
+        r.bwd_gates()
+        return r.grads()
 
     def close(self):
         """Unmaps the peers' buffers (after every rank has finished its last step)."""
@@ -279,3 +355,21 @@ class LocalRanks:
         for _, f in self.stages(logits_shards, x_shards):
             f()
         return [r.out for r in self.ranks]
+
+    def backward(self, dout_shards):
+        """The backward of the last forward, stage by stage over the ranks; returns each
+        rank's gradients (EPRank.grads)."""
+        if "dy" not in self.ranks[0].tables:
+            tables = {name: [int(r.shared_backward()[name].data_ptr()) for r in self.ranks]
+                      for name in SHARED_BWD}
+            for r in self.ranks:
+                r.tables = dict(r.tables, **tables)
+        for r, g in zip(self.ranks, dout_shards):
+            r.bwd_combine(g)
+        for r in self.ranks:
+            r.bwd_ffn()
+        for r in self.ranks:
+            r.bwd_reduce()
+            r.bwd_dispatch()
+            r.bwd_gates()
+        return [r.grads() for r in self.ranks]

@@ -234,3 +234,58 @@ def test_ep_nccl_communicator_single_rank(tmp_path):
     got = torch.load(path)
     assert got["err"] == 0
     assert torch.equal(got["out"], L.out.cpu())
+
+
+# ------------------------------------------------------------------------------ backward
+BWD_SMALL = [("epb_w2", 96, 8, 2, 2, 4, 128, 256), ("epb_w4_k3", 200, 32, 3, 4, 6, 128, 384),
+             ("epb_w8", 512, 64, 6, 8, 8, 256, 256), ("epb_hot", 512, 32, 4, 8, 4, 128, 256)]
+BWD_FULL = ["near_balanced", "qwen_mv1", "mixtral"]
+
+
+def _ep_backward_against_layer(w, alpha=None):
+    W = w.R
+    logits, x, weights = make_inputs(w)
+    g = torch.Generator().manual_seed(41)
+    dout = torch.randn(w.T, w.d, generator=g).to(torch.bfloat16).cuda()
+    lg, xd = logits.cuda(), x.cuda()
+    L = M.MoELayer(w.T, w.E, w.k, w.R, w.S, w.d, w.F)
+    L.forward(lg, xd, *weights)
+    b = L.backward(dout, *weights)
+    lr = make_ranks(w, weights)
+    lr.forward(shards(lg, W), shards(xd, W))
+    lr.backward(shards(dout, W))
+    torch.cuda.synchronize()
+    assert int(L.err.item()) == 0
+    C, Tl = w.C, w.T // W
+    for u, r in enumerate(lr.ranks):
+        assert int(r.err.item()) == 0
+        assert torch.equal(r.dy, b["dy"][u * C:(u + 1) * C]), f"rank {u} dy"
+        assert torch.equal(r.dgate, b["dgate"][u * Tl:(u + 1) * Tl]), f"rank {u} dgate"
+        assert torch.equal(r.dx_rows, b["dx_rows"][u * C:(u + 1) * C]), f"rank {u} dx rows"
+        assert torch.equal(r.dx, b["dx"][u * Tl:(u + 1) * Tl]), f"rank {u} dx"
+        assert torch.equal(r.dlogits, b["dlogits"][u * Tl:(u + 1) * Tl]), f"rank {u} dlogits"
+    # the same fp32 sums of the same products, associated differently (a home expert's own
+    # groups, then each copy's partial): a missing or doubled copy would be off by O(1)
+    for name in ("dW1", "dW3", "dW2"):
+        ep = torch.cat([getattr(r, name) for r in lr.ranks])
+        ref = b[name]
+        tol = 1e-4 * ref.abs().amax(dim=(1, 2), keepdim=True) + 1e-6
+        bad = (ep - ref).abs() > tol
+        assert not bad.any(), f"{name}: {int(bad.sum())} entries off"
+    n_rep = int(lr.ranks[0].plan[M.plan_layout(w.E, W, w.S).replica_list].item())
+    return n_rep
+
+
+@pytest.mark.parametrize("case", BWD_SMALL, ids=[c[0] for c in BWD_SMALL])
+def test_ep_backward_is_the_single_gpu_backward(case):
+    w = I.small_workload(*case, alpha=1.2 if case[0] != "epb_hot" else 2.5)
+    n_rep = _ep_backward_against_layer(w)
+    if case[0] == "epb_hot":
+        assert n_rep >= 1  # replica gradients crossed ranks
+
+
+@pytest.mark.parametrize("name", BWD_FULL)
+def test_ep_backward_full_size(name):
+    n_rep = _ep_backward_against_layer(I.WORKLOADS[name])
+    assert n_rep >= 1
+    torch.cuda.empty_cache()
