@@ -580,6 +580,10 @@ def run_ep(args, w: I.Workload, world, rank, local):
         lr = LocalRanks([EPRank(u, W, Tl, w.E, w.k, w.S, W1[u * B:(u + 1) * B],
                                 W3[u * B:(u + 1) * B], W2[u * B:(u + 1) * B]) for u in range(W)])
         stages = lr.stages([shard(logits, u) for u in range(W)], [shard(x, u) for u in range(W)])
+        if args.backward:
+            g = torch.Generator(device=device).manual_seed(41)
+            dout = torch.randn(w.T, w.d, generator=g, device=device).to(torch.bfloat16)
+            stages = stages + lr.backward_stages([shard(dout, u) for u in range(W)])
         ranks = lr.ranks
 
         def step():
@@ -589,12 +593,17 @@ def run_ep(args, w: I.Workload, world, rank, local):
         own = tuple(t[rank * B:(rank + 1) * B].contiguous() for t in (W1, W3, W2))
         del W1, W3, W2
         torch.cuda.empty_cache()
-        layer = EPLayer(NcclComm(), Tl, w.E, w.k, w.S, *own)
+        layer = EPLayer(NcclComm(), Tl, w.E, w.k, w.S, *own, backward=args.backward)
         lg, xs = shard(logits, rank), shard(x, rank)
         ranks = [layer.rank]
+        if args.backward:
+            g = torch.Generator(device=device).manual_seed(41)
+            dout_own = shard(torch.randn(w.T, w.d, generator=g, device=device).to(torch.bfloat16), rank)
 
         def step():
             layer.forward(lg, xs)
+            if args.backward:
+                layer.backward(dout_own)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -662,7 +671,8 @@ def run_ep(args, w: I.Workload, world, rank, local):
         raise RuntimeError(f"{w.name}: device error words {errs} in the timed region")
     row_bytes = w.d * 2
     work = {"dispatch": (w.T + w.A) * row_bytes, "combine": (w.A + w.T) * row_bytes,
-            "prefetch": 2 * n_rep * 3 * w.d * w.F * 2, "ffn": 6 * w.A * w.d * w.F}
+            "prefetch": 2 * n_rep * 3 * w.d * w.F * 2, "ffn": 6 * w.A * w.d * w.F,
+            "bwd_ffn": 16 * w.A * w.d * w.F}
     ffn_peak_v, ffn_src = ffn_peak(clk, peaks, peak_src)
     res = {
         "metric": METRIC, "value": round(w.T * steps / (elapsed_ms * 1e-3), 1), "unit": UNIT,
@@ -680,7 +690,9 @@ def run_ep(args, w: I.Workload, world, rank, local):
                                    "peer buffers through CUDA IPC"),
                    "l2": "inputs larger than L2 (weights, pool, activations), no flush",
                    "launch": ("K steps of every rank's stages captured in one CUDA graph"
-                              if world == 1 else "eager, K steps between barriers")},
+                              if world == 1 else "eager, K steps between barriers"),
+                   "step": ("forward + backward (dx, dlogits, home experts' weight gradients "
+                            "with the replicas' reduced home)" if args.backward else "forward")},
         "clocks": clk,
         "e2e": None,
         # per rank and step: top-k, counts, plan, prefetch, dispatch rank pass and row
@@ -694,8 +706,8 @@ def run_ep(args, w: I.Workload, world, rank, local):
             if name in ("dispatch", "combine", "prefetch") and ms > 0:
                 gbs = work[name] / (ms * 1e-3) / 1e9
                 row.update(GB_per_s=round(gbs, 1), frac=round(gbs / peaks["hbm_gbs"], 3))
-            if name == "ffn" and ms > 0:
-                tf = work["ffn"] / (ms * 1e-3) / 1e12
+            if name in ("ffn", "bwd_ffn") and ms > 0:
+                tf = work[name] / (ms * 1e-3) / 1e12
                 row.update(TFLOP_per_s=round(tf, 1), frac=round(tf / ffn_peak_v, 3),
                            peak_source=ffn_src)
             st[name] = row

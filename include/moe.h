@@ -634,15 +634,19 @@ int moe_ep_grouped_ffn_backward(const moe_bf16* recv, const moe_bf16* dy, const 
                                 float* dP2, void* workspace, int64_t workspace_bytes,
                                 int32_t* err, moe_stream_t stream);
 /*
- * moe_ep_reduce_home: the gradient of this rank's home expert e = me*B + b: its own entry b
- *   plus, for every pool slot (v, s) of the plan that held a copy of e, in (v, s) order,
- *   rank v's entry B + s (peer loads).
+ * moe_ep_reduce_home: in place on this rank's partials (dP*_ranks[me]): entry b, the
+ *   gradient of home expert e = me*B + b, gets, for every pool slot (v, s) of the plan that
+ *   held a copy of e and in (v, s) order, rank v's entry B + s added (peer loads, fp32);
+ *   experts without copies are left as they are.  Afterwards entries 0..B-1 of this rank's
+ *   dP1, dP3 [B+S,F,d] and dP2 [B+S,d,F] are its home experts' weight gradients.  No rank may
+ *   run this before every rank's moe_ep_grouped_ffn_backward has finished, nor start its next
+ *   backward before every rank's moe_ep_reduce_home has finished (a rank reads its peers'
+ *   slot entries).
  *   dP1_ranks, dP3_ranks, dP2_ranks: HOST tables of every rank's dP1, dP3, dP2.
- *   dW1, dW3 [B,F,d], dW2 [B,d,F] fp32 (out).  err  no-op when non-zero.
+ *   err  no-op when non-zero.
  */
-int moe_ep_reduce_home(const int32_t* plan, const float* const* dP1_ranks,
-                       const float* const* dP3_ranks, const float* const* dP2_ranks, int W,
-                       int me, int E, int S, int d, int F, float* dW1, float* dW3, float* dW2,
+int moe_ep_reduce_home(const int32_t* plan, float* const* dP1_ranks, float* const* dP3_ranks,
+                       float* const* dP2_ranks, int W, int me, int E, int S, int d, int F,
                        const int32_t* err, moe_stream_t stream);
 /*
  * moe_ep_dispatch_backward: dx[t] = sum_j dx_rows_v[perm[t,j] % C], v = perm[t,j] / C

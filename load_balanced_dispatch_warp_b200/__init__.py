@@ -101,7 +101,7 @@ def lib() -> ctypes.CDLL:
             "moe_ep_combine_backward": [P, P, P, P, I, I, I, I, P, P, P, P],
             "moe_ep_grouped_ffn_backward": [P, P, P, I, I, P, P, P, P, P, P, I, I, I, I, I, I, P,
                                             P, P, P, P, P, I64, P, P],
-            "moe_ep_reduce_home": [P, P, P, P, I, I, I, I, I, I, P, P, P, P, P],
+            "moe_ep_reduce_home": [P, P, P, P, I, I, I, I, I, I, P, P],
             "moe_ep_dispatch_backward": [P, P, I, I, I, I, P, P, P],
         }
         for name, args in sig.items():
@@ -525,14 +525,12 @@ def moe_ep_grouped_ffn_backward(recv, dy, plan, W, me, W1, W3, W2, P1, P3, P2, T
         "moe_ep_grouped_ffn_backward")
 
 
-def moe_ep_reduce_home(plan, dP1_ranks, dP3_ranks, dP2_ranks, me, E, S, d, F, dW1, dW3, dW2, err,
+def moe_ep_reduce_home(plan, dP1_ranks, dP3_ranks, dP2_ranks, me, E, S, d, F, err,
                        stream=None):
-    f32 = torch.float32
     _check(lib().moe_ep_reduce_home(
         _ptr(plan, torch.int32, "plan"), _table(dP1_ranks, "dP1_ranks"),
         _table(dP3_ranks, "dP3_ranks"), _table(dP2_ranks, "dP2_ranks"), len(dP1_ranks), me, E,
-        S, d, F, _ptr(dW1, f32, "dW1"), _ptr(dW3, f32, "dW3"), _ptr(dW2, f32, "dW2"),
-        _ptr(err, torch.int32, "err"), _stream(stream)), "moe_ep_reduce_home")
+        S, d, F, _ptr(err, torch.int32, "err"), _stream(stream)), "moe_ep_reduce_home")
 
 
 def moe_ep_dispatch_backward(dx_rows_ranks, perm, d, dx, err, stream=None):

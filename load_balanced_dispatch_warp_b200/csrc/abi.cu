@@ -633,22 +633,20 @@ int moe_ep_grouped_ffn_backward(const moe_bf16* recv, const moe_bf16* dy, const 
       dP3, dP2, workspace, workspace_bytes, err, s);
 }
 
-int moe_ep_reduce_home(const int32_t* plan, const float* const* dP1_ranks,
-                       const float* const* dP3_ranks, const float* const* dP2_ranks, int W,
-                       int me, int E, int S, int d, int F, float* dW1, float* dW3, float* dW2,
+int moe_ep_reduce_home(const int32_t* plan, float* const* dP1_ranks, float* const* dP3_ranks,
+                       float* const* dP2_ranks, int W, int me, int E, int S, int d, int F,
                        const int32_t* err, moe_stream_t stream) {
-  if (!plan || !err || !dW1 || !dW3 || !dW2) return MOE_ERR_ARG;
+  if (!plan || !err) return MOE_ERR_ARG;
   MOE_TRY(check_ep(W, me, 0, 1, E, S));
   MOE_TRY(check_dims(0, 1, d, F));
   if ((int64_t)(E / W + S) * F * d >= kMaxElems) return MOE_ERR_SHAPE;
   MOE_TRY(check_table(dP1_ranks, W));
   MOE_TRY(check_table(dP3_ranks, W));
   MOE_TRY(check_table(dP2_ranks, W));
-  if (!aligned16(dW1) || !aligned16(dW3) || !aligned16(dW2)) return MOE_ERR_ARG;
   moe_plan_layout L;
   MOE_TRY(moe_plan_get_layout(E, W, S, &L));
   return moe::launch_ep_reduce_home(plan, L, dP1_ranks, dP3_ranks, dP2_ranks, W, me, E, S, d, F,
-                                    dW1, dW3, dW2, err, as_stream(stream));
+                                    err, as_stream(stream));
 }
 
 int moe_ep_dispatch_backward(const moe_bf16* const* dx_rows_ranks, const int32_t* perm, int W,

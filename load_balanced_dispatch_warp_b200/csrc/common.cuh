@@ -147,7 +147,7 @@ int launch_ep_combine(const __nv_bfloat16* const* y_ranks, int W, const int32_t*
 // Backward of the expert-parallel layer (grouped_ffn_bwd.cu): dy rows written and y rows
 // read on every rank; one rank's grouped-FFN backward over its re-based group table, the
 // weight gradients of its home experts and of its pool slots ([B+S] entries); the slots'
-// gradients added to their home experts' across ranks.  (The dispatch backward is
+// gradients added, in place, to their home experts' entries across ranks.  (The dispatch backward is
 // launch_ep_combine with gate == nullptr.)
 int64_t ep_ffn_backward_workspace_bytes(int T, int k, int E, int W, int S, int d, int F);
 int launch_ep_combine_backward(const __nv_bfloat16* dout, const __nv_bfloat16* const* y_ranks,
@@ -163,10 +163,9 @@ int launch_ep_grouped_ffn_backward(const __nv_bfloat16* recv, const __nv_bfloat1
                                    void* workspace, int64_t workspace_bytes, int32_t* err,
                                    cudaStream_t s);
 int launch_ep_reduce_home(const int32_t* plan, const moe_plan_layout& L,
-                          const float* const* part1_ranks, const float* const* part3_ranks,
-                          const float* const* part2_ranks, int W, int me, int E, int S, int d,
-                          int F, float* dW1, float* dW3, float* dW2, const int32_t* err,
-                          cudaStream_t s);
+                          float* const* part1_ranks, float* const* part3_ranks,
+                          float* const* part2_ranks, int W, int me, int E, int S, int d, int F,
+                          const int32_t* err, cudaStream_t s);
 
 // ----------------------------------------------------------------------------- device side
 // Reads the layer's error word once per thread; every kernel after moe_topk returns

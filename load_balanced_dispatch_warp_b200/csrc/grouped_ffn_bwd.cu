@@ -1012,18 +1012,18 @@ int grouped_ffn_backward_impl(const __nv_bfloat16* recv, const __nv_bfloat16* dy
   return MOE_OK;
 }
 
-// Replica gradients reduced back home across ranks: home expert e_local of rank me gets its
-// own partial plus, in (rank, slot) order, the partial of every pool slot (v, s) of the
-// job's plan that held a copy of it, read from rank v's partials through the rank tables.
-// parts[p][v] -> rank v's [B+S][n4] partials of projection p (fp32, 16-byte vectors).
+// Replica gradients reduced back home across ranks, in place: home expert e_local of rank me
+// (entry e_local of its own partials) gets, in (rank, slot) order, the partial of every pool
+// slot (v, s) of the job's plan that held a copy of it, read from rank v's partials through
+// the rank tables; an expert without copies is left as it is.  parts[p][v] -> rank v's
+// [B+S][n4] partials of projection p (fp32, 16-byte vectors).
 struct RankParts {
   const float4* p[3][MOE_EP_MAX_RANKS];
 };
 
 __global__ void __launch_bounds__(256) ep_reduce_home_kernel(
     const int32_t* __restrict__ rep, int W, int me, int B, int S, int64_t n4,
-    const __grid_constant__ RankParts parts, float4* __restrict__ dW1, float4* __restrict__ dW3,
-    float4* __restrict__ dW2, const int32_t* __restrict__ err) {
+    const __grid_constant__ RankParts parts, const int32_t* __restrict__ err) {
   __shared__ int s_src[MOE_EP_MAX_RANKS];  // v * S + s of the copies, in order (a rank's
                                           // slots hold distinct experts: at most W copies)
   __shared__ int s_n;
@@ -1049,11 +1049,11 @@ __global__ void __launch_bounds__(256) ep_reduce_home_kernel(
       __syncthreads();
       cur = el;
     }
-    float4* out = (proj == 0 ? dW1 : proj == 1 ? dW3 : dW2) + (int64_t)el * n4;
-    const float4* own = parts.p[proj][me] + (int64_t)el * n4;
     const int n = s_n;
+    if (n == 0) continue;
+    float4* own = const_cast<float4*>(parts.p[proj][me]) + (int64_t)el * n4;
     for (int64_t v = c * kChunk + threadIdx.x; v < min(n4, (c + 1) * kChunk); v += blockDim.x) {
-      float4 a = __ldcs(own + v);
+      float4 a = own[v];
       for (int i = 0; i < n; ++i) {
         const int q = s_src[i];
         const float4 b = __ldcs(parts.p[proj][q / S] + (int64_t)(B + q % S) * n4 + v);
@@ -1062,7 +1062,7 @@ __global__ void __launch_bounds__(256) ep_reduce_home_kernel(
         a.z += b.z;
         a.w += b.w;
       }
-      out[v] = a;
+      own[v] = a;
     }
   }
 }
@@ -1155,10 +1155,9 @@ int launch_ep_grouped_ffn_backward(const __nv_bfloat16* recv, const __nv_bfloat1
 }
 
 int launch_ep_reduce_home(const int32_t* plan, const moe_plan_layout& L,
-                          const float* const* part1_ranks, const float* const* part3_ranks,
-                          const float* const* part2_ranks, int W, int me, int E, int S, int d,
-                          int F, float* dW1, float* dW3, float* dW2, const int32_t* err,
-                          cudaStream_t s) {
+                          float* const* part1_ranks, float* const* part3_ranks,
+                          float* const* part2_ranks, int W, int me, int E, int S, int d, int F,
+                          const int32_t* err, cudaStream_t s) {
   RankParts parts;
   for (int u = 0; u < MOE_EP_MAX_RANKS; ++u) {
     parts.p[0][u] = u < W ? reinterpret_cast<const float4*>(part1_ranks[u]) : nullptr;
@@ -1166,9 +1165,8 @@ int launch_ep_reduce_home(const int32_t* plan, const moe_plan_layout& L,
     parts.p[2][u] = u < W ? reinterpret_cast<const float4*>(part2_ranks[u]) : nullptr;
   }
   const int64_t n4 = (int64_t)d * F / 4;
-  ep_reduce_home_kernel<<<num_sms() * 4, 256, 0, s>>>(
-      plan + L.replica_expert, W, me, E / W, S, n4, parts, reinterpret_cast<float4*>(dW1),
-      reinterpret_cast<float4*>(dW3), reinterpret_cast<float4*>(dW2), err);
+  ep_reduce_home_kernel<<<num_sms() * 4, 256, 0, s>>>(plan + L.replica_expert, W, me, E / W, S,
+                                                     n4, parts, err);
   return launch_status();
 }
 

@@ -86,8 +86,8 @@ class EPRank:
 
     def alloc_backward(self):
         """Buffers of the backward: dy and dx rows [C,d], the weight-gradient partials of
-        its groups [B+S,...] (home experts, then pool slots), the home experts' gradients
-        [B,...], dx [T,d], dlogits [T,E]."""
+        its groups [B+S,...] (home experts, then pool slots; the first B entries become the
+        home experts' gradients), dx [T,d], dlogits [T,E]."""
         if hasattr(self, "dy"):
             return
         dev = self.W1.device
@@ -99,9 +99,8 @@ class EPRank:
         self.dP1 = torch.zeros(B + S, F, d, dtype=f32, device=dev)
         self.dP3 = torch.zeros(B + S, F, d, dtype=f32, device=dev)
         self.dP2 = torch.zeros(B + S, d, F, dtype=f32, device=dev)
-        self.dW1 = torch.zeros(B, F, d, dtype=f32, device=dev)
-        self.dW3 = torch.zeros(B, F, d, dtype=f32, device=dev)
-        self.dW2 = torch.zeros(B, d, F, dtype=f32, device=dev)
+        # the home experts' gradients: entries 0..B-1 of the partials, completed in place
+        self.dW1, self.dW3, self.dW2 = self.dP1[:B], self.dP3[:B], self.dP2[:B]
         self.dx = torch.zeros(T, d, dtype=bf, device=dev)
         self.dlogits = torch.zeros(T, self.E, dtype=f32, device=dev)
         ws = ep_ffn_backward_workspace_bytes(T, self.k, self.E, self.W, S, d, F)
@@ -152,7 +151,7 @@ class EPRank:
     def bwd_reduce(self):
         t = self.tables
         moe_ep_reduce_home(self.plan, t["dP1"], t["dP3"], t["dP2"], self.me, self.E, self.S,
-                           self.d, self.F, self.dW1, self.dW3, self.dW2, self.err)
+                           self.d, self.F, self.err)
 
     def bwd_dispatch(self):
         moe_ep_dispatch_backward(self.tables["dx_rows"], self.perm, self.d, self.dx, self.err)
@@ -356,20 +355,39 @@ class LocalRanks:
             f()
         return [r.out for r in self.ranks]
 
+    def backward_stages(self, dout_shards):
+        """The backward as (name, callable) pairs over every rank (buffers and tables set up
+        here, before any stage runs)."""
+        ranks = self.ranks
+        if "dy" not in ranks[0].tables:
+            tables = {name: [int(r.shared_backward()[name].data_ptr()) for r in ranks]
+                      for name in SHARED_BWD}
+            for r in ranks:
+                r.tables = dict(r.tables, **tables)
+
+        def combine():
+            for r, g in zip(ranks, dout_shards):
+                r.bwd_combine(g)
+
+        def ffn():
+            for r in ranks:
+                r.bwd_ffn()
+
+        def reduce_home():
+            for r in ranks:
+                r.bwd_reduce()
+
+        def dispatch_and_gates():
+            for r in ranks:
+                r.bwd_dispatch()
+                r.bwd_gates()
+
+        return [("bwd_combine", combine), ("bwd_ffn", ffn), ("bwd_reduce_home", reduce_home),
+                ("bwd_dispatch_gates", dispatch_and_gates)]
+
     def backward(self, dout_shards):
         """The backward of the last forward, stage by stage over the ranks; returns each
         rank's gradients (EPRank.grads)."""
-        if "dy" not in self.ranks[0].tables:
-            tables = {name: [int(r.shared_backward()[name].data_ptr()) for r in self.ranks]
-                      for name in SHARED_BWD}
-            for r in self.ranks:
-                r.tables = dict(r.tables, **tables)
-        for r, g in zip(self.ranks, dout_shards):
-            r.bwd_combine(g)
-        for r in self.ranks:
-            r.bwd_ffn()
-        for r in self.ranks:
-            r.bwd_reduce()
-            r.bwd_dispatch()
-            r.bwd_gates()
+        for _, f in self.backward_stages(dout_shards):
+            f()
         return [r.grads() for r in self.ranks]

@@ -273,3 +273,34 @@ def test_expert_parallel_host_checks(lib):
     assert lib.moe_ipc_export(None, h, ctypes.byref(off)) == M.MOE_ERR_ARG
     assert lib.moe_ipc_import(h, -1, ctypes.byref(P()), ctypes.byref(P())) == M.MOE_ERR_ARG
     assert lib.moe_ipc_close(None) == M.MOE_ERR_ARG
+
+
+def test_expert_parallel_backward_host_checks(lib):
+    """Host argument rules of the expert-parallel backward calls (nothing is enqueued)."""
+    P = ctypes.c_void_p
+    fake = P(4096)
+
+    def table(n, addr=4096):
+        return (ctypes.c_void_p * n)(*([addr] * n))
+
+    assert lib.moe_ep_combine_backward(fake, table(2), fake, fake, 2, 16, 2, 128, table(2), None,
+                                       fake, None) == M.MOE_ERR_ARG  # dgate missing
+    assert lib.moe_ep_combine_backward(fake, table(2), fake, fake, 2, 16, 2, 128, table(2, 0), fake,
+                                       fake, None) == M.MOE_ERR_ARG  # null dy entry
+    assert lib.moe_ep_ffn_backward_workspace_bytes(16, 2, 8, 3, 2, 128, 256) == -1  # E % W
+    assert lib.moe_ep_ffn_backward_workspace_bytes(16, 2, 1024, 1, 8, 128, 256) == -1  # B+S > 1024
+    n = lib.moe_ep_ffn_backward_workspace_bytes(512, 6, 64, 8, 8, 2048, 1408)
+    assert n > 0 and n % 256 == 0
+    args = [fake, fake, fake, 2, 1, fake, fake, fake, fake, fake, fake, 16, 2, 8, 2, 128, 256,
+            fake, fake, fake, fake, fake, P(4096 * 64), 1 << 30, fake, None]
+    bad = list(args); bad[19] = None  # dP3 missing
+    assert lib.moe_ep_grouped_ffn_backward(*bad) == M.MOE_ERR_ARG
+    bad = list(args); bad[23] = 1024  # workspace too small
+    assert lib.moe_ep_grouped_ffn_backward(*bad) == M.MOE_ERR_ARG
+    bad = list(args); bad[22] = P(4096 + 16)  # workspace not 256-byte aligned
+    assert lib.moe_ep_grouped_ffn_backward(*bad) == M.MOE_ERR_ARG
+    bad = list(args); bad[4] = 2  # me outside [0, W)
+    assert lib.moe_ep_grouped_ffn_backward(*bad) == M.MOE_ERR_ARG
+    assert lib.moe_ep_reduce_home(fake, table(2), table(2, 0), table(2), 2, 0, 8, 2, 128, 256,
+                                  fake, None) == M.MOE_ERR_ARG
+    assert lib.moe_ep_dispatch_backward(table(2), fake, 2, 16, 2, 96, fake, fake, None) == M.MOE_ERR_SHAPE
