@@ -774,6 +774,12 @@ def run_only(args, w: I.Workload):
         y = recv.clone()
         out = torch.empty(w.T, w.d, dtype=torch.bfloat16, device=device)
         fn, unit, work = (lambda: M.moe_combine(y, perm, gate, out, err)), *units["moe_combine"]
+    elif args.only == "prefetch":
+        W1, W3, W2 = I.make_weights(w, device=device)
+        P = [torch.empty(w.R * w.S, *t.shape[1:], dtype=t.dtype, device=device) for t in (W1, W3, W2)]
+        n_rep = int(plan[lay.replica_list].item())
+        fn = lambda: M.moe_prefetch_replicas(plan, W1, W3, W2, w.R, w.S, *P, err)
+        unit, work = algorithmic(w, n_rep)["moe_prefetch_replicas"]
     else:  # ffn
         W1, W3, W2 = I.make_weights(w, device=device)
         P = [torch.empty(w.R * w.S, *t.shape[1:], dtype=t.dtype, device=device) for t in (W1, W3, W2)]
@@ -1011,7 +1017,8 @@ def main():
                     help="steps per point of the Qwen-shaped maxvio sweep")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the stand-alone top-k floor and the maxvio sweep")
-    ap.add_argument("--only", default=None, choices=["topk", "route", "dispatch", "combine", "ffn"],
+    ap.add_argument("--only", default=None,
+                    choices=["topk", "route", "dispatch", "combine", "prefetch", "ffn"],
                     help="time one call alone (--steps launches after --warmup) and print its "
                          "rate instead of the benchmark line: the small case for counter captures")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
