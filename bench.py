@@ -44,8 +44,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (`ncu --set full --clock-control none -k regex:ffn_kernel ...` on the named workload),
 # keyed by workload, tile mode and kernel-sources hash: a kernel edit changes the hash,
 # and the line then reports null (with the reason) until the counters are taken again.
-TRAFFIC = {"deepseek:0:23c5f631227151ba": 22151061760 + 533245184 + 9019571712 + 1833178624}
-TRAFFIC_NOTE = {"deepseek:0:23c5f631227151ba":
+TRAFFIC = {"deepseek:0:f6968ffe57135168": 22115675136 + 533353216 + 8993779968 + 1833654016}
+TRAFFIC_NOTE = {"deepseek:0:f6968ffe57135168":
                 "ncu dram__bytes_read.sum + dram__bytes_write.sum of the gate-up and down "
                 "kernels of one full DeepSeek call (bench.py --only ffn --config deepseek)"}
 
