@@ -427,10 +427,11 @@ EP_MAX_RANKS = 64           # MOE_EP_MAX_RANKS
 IPC_HANDLE_BYTES = 64       # MOE_IPC_HANDLE_BYTES
 
 
-def _table(ptrs, name):
-    """A host array of device pointers (one per rank) for the *_ranks arguments."""
+def _table(ptrs, name, rows=1):
+    """A host array of device pointers (one per rank) for the *_ranks arguments.  With no
+    rows to move (rows == 0: empty buffers, null pointers) the calls do not read it."""
     ptrs = [int(p) for p in ptrs]
-    if not ptrs or any(p == 0 for p in ptrs):
+    if not ptrs or (rows and any(p == 0 for p in ptrs)):
         raise ValueError(f"{name}: one non-null device pointer per rank")
     return (ctypes.c_void_p * len(ptrs))(*ptrs)
 
@@ -469,7 +470,7 @@ def moe_ep_dispatch(x, idx, q_base, plan, E, S, workspace, recv_ranks, perm, err
     _check(lib().moe_ep_dispatch(
         _ptr(x, torch.bfloat16, "x"), _ptr(idx, i32, "idx"), _ptr(q_base, i32, "q_base"),
         _ptr(plan, i32, "plan"), len(recv_ranks), T, k, E, S, d,
-        _ptr(workspace, i32, "workspace"), _table(recv_ranks, "recv_ranks"),
+        _ptr(workspace, i32, "workspace"), _table(recv_ranks, "recv_ranks", T),
         _ptr(perm, i32, "perm"), _ptr(err, i32, "err"), _stream(stream)), "moe_ep_dispatch")
 
 
@@ -488,7 +489,7 @@ def moe_ep_grouped_ffn(recv, plan, W, me, W1, W3, W2, P1, P3, P2, T, k, E, S, gr
 def moe_ep_combine(y_ranks, perm, gate, d, out, err, stream=None):
     T, k = perm.shape
     _check(lib().moe_ep_combine(
-        _table(y_ranks, "y_ranks"), _ptr(perm, torch.int32, "perm"), _ptr(gate, torch.float32, "gate"),
+        _table(y_ranks, "y_ranks", T), _ptr(perm, torch.int32, "perm"), _ptr(gate, torch.float32, "gate"),
         len(y_ranks), T, k, d, _ptr(out, torch.bfloat16, "out"), _ptr(err, torch.int32, "err"),
         _stream(stream)), "moe_ep_combine")
 
@@ -496,9 +497,9 @@ def moe_ep_combine(y_ranks, perm, gate, d, out, err, stream=None):
 def moe_ep_combine_backward(dout, y_ranks, perm, gate, dy_ranks, dgate, err, stream=None):
     T, k = perm.shape
     _check(lib().moe_ep_combine_backward(
-        _ptr(dout, torch.bfloat16, "dout"), _table(y_ranks, "y_ranks"), _ptr(perm, torch.int32, "perm"),
+        _ptr(dout, torch.bfloat16, "dout"), _table(y_ranks, "y_ranks", T), _ptr(perm, torch.int32, "perm"),
         _ptr(gate, torch.float32, "gate"), len(y_ranks), T, k, dout.shape[1],
-        _table(dy_ranks, "dy_ranks"), _ptr(dgate, torch.float32, "dgate"),
+        _table(dy_ranks, "dy_ranks", T), _ptr(dgate, torch.float32, "dgate"),
         _ptr(err, torch.int32, "err"), _stream(stream)), "moe_ep_combine_backward")
 
 
@@ -536,7 +537,7 @@ def moe_ep_reduce_home(plan, dP1_ranks, dP3_ranks, dP2_ranks, me, E, S, d, F, er
 def moe_ep_dispatch_backward(dx_rows_ranks, perm, d, dx, err, stream=None):
     T, k = perm.shape
     _check(lib().moe_ep_dispatch_backward(
-        _table(dx_rows_ranks, "dx_rows_ranks"), _ptr(perm, torch.int32, "perm"),
+        _table(dx_rows_ranks, "dx_rows_ranks", T), _ptr(perm, torch.int32, "perm"),
         len(dx_rows_ranks), T, k, d, _ptr(dx, torch.bfloat16, "dx"), _ptr(err, torch.int32, "err"),
         _stream(stream)), "moe_ep_dispatch_backward")
 
