@@ -486,8 +486,6 @@ __global__ void __launch_bounds__(512) hist_kernel(const int32_t* __restrict__ i
 
 // One warp per token, 8 warps per block.  Unbiased calls with k in {2, 4, 6, 8} and up to
 // 256 experts run a kernel with k fixed at compile time (the rounds unroll).
-// One warp per token, 8 warps per block.  Unbiased calls with k in {2, 4, 6, 8} and up to
-// 256 experts run a kernel with k fixed at compile time (the rounds unroll).
 template <int VPL>
 void launch_topk_vpl(const float* logits, const float* bias, int T, int E, int k, int32_t* idx,
                      float* gate, int32_t* err, cudaStream_t s) {
