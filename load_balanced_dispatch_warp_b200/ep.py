@@ -258,9 +258,10 @@ class EPLayer:
     ``forward(logits, x)`` runs one step on this rank's T tokens and returns its [T,d]
     output; with ``backward=True`` the backward buffers are shared too and
     ``backward(dout)`` returns this rank's dx, dlogits and its home experts' weight
-    gradients (replica gradients reduced back home).  Weights are shared with the peers
-    through the pointer tables: a caller that updates them in place must make every rank
-    finish its step first."""
+    gradients (replica gradients reduced back home).  Construction, ``forward`` and
+    ``backward`` are collective: every rank calls them in the same order.  Weights are
+    shared with the peers through the pointer tables: a caller that updates them in place
+    must make every rank finish its step first."""
 
     def __init__(self, comm, T: int, E: int, k: int, S: int, W1, W3, W2, backward=False):
         self.comm = comm
