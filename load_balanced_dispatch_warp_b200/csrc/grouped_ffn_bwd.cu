@@ -627,31 +627,27 @@ __global__ void __launch_bounds__(1024) bwd_prepare_kernel(const int4* __restric
 }
 
 // Tiled transpose of 16-bit elements, 64 x 64 per block, 16-byte loads and stores:
-// out[c][q] = in[src(q)][c], src(q) = q (src_of == nullptr) or src_of[q] (0 where it is
-// -1).  q runs over n_out output columns (blocks past *n_out_dev, when given, return at
-// once).  cols and the row pitches are multiples of 8 elements.  With f16_to_bf16 the fp16
-// inputs are rounded to bf16 on the way.  Batched over blockIdx.z.  (The backward uses it
-// for W2 -> W2^T in bf16.)
+// out[c][q] = in[q][c] for q < n_out.  cols, n_out and the row pitches are multiples of 8
+// elements.  With f16_to_bf16 the fp16 inputs are rounded to bf16 on the way.  Batched over
+// blockIdx.z.  (The backward uses it for W2 -> W2^T in bf16.)
 constexpr int kTp = 64;
 // shared tile [q][c]: the 16-byte chunk j of row q is stored at chunk j ^ ((q / 8) % 8), so
 // that reading one column across rows q = 8i + r (i = 0..7) touches 8 different banks
 __global__ void __launch_bounds__(256) transpose_kernel(
     const uint16_t* __restrict__ in, int cols, int64_t ld_in, int64_t in_bstride,
-    uint16_t* __restrict__ out, int64_t ld_out, int64_t out_bstride, int n_out,
-    const int* __restrict__ n_out_dev, const int* __restrict__ src_of, int f16_to_bf16,
+    uint16_t* __restrict__ out, int64_t ld_out, int64_t out_bstride, int n_out, int f16_to_bf16,
     const int32_t* __restrict__ err) {
   __shared__ __align__(16) uint16_t tile[kTp][kTp];
   if (load_err(err)) return;
   const int q0 = blockIdx.x * kTp, c0 = blockIdx.y * kTp;
-  const int nq = n_out_dev ? min(n_out, *n_out_dev) : n_out;
+  const int nq = n_out;
   if (q0 >= nq) return;
   const uint16_t* src = in + (int64_t)blockIdx.z * in_bstride;
   uint16_t* dst = out + (int64_t)blockIdx.z * out_bstride;
   for (int i = threadIdx.x; i < kTp * 8; i += blockDim.x) {
     const int q = i >> 3, ch = i & 7;
     const int c = c0 + ch * 8;
-    int r = -1;
-    if (q0 + q < nq) r = src_of ? __ldg(src_of + q0 + q) : q0 + q;
+    const int r = q0 + q < nq ? q0 + q : -1;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (r >= 0 && c < cols) {
       v = __ldg(reinterpret_cast<const uint4*>(src + (int64_t)r * ld_in + c));
@@ -677,7 +673,7 @@ __global__ void __launch_bounds__(256) transpose_kernel(
 #pragma unroll
     for (int j = 0; j < 4; ++j)
       w[j] = (uint32_t)tile[qc * 8 + 2 * j][col] | ((uint32_t)tile[qc * 8 + 2 * j + 1][col] << 16);
-    // n_out (and the padded layout) is a multiple of 8: whole 16-byte chunks
+    // n_out is a multiple of 8: whole 16-byte chunks
     *reinterpret_cast<uint4*>(dst + (int64_t)(c0 + c) * ld_out + q0 + qc * 8) =
         make_uint4(w[0], w[1], w[2], w[3]);
   }
@@ -801,16 +797,16 @@ int launch_bwd_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorM
   return launch_status();
 }
 
-// out[c][q] = in[src(q)][c] for q < n_out (see transpose_kernel), batched.
+// out[c][q] = in[q][c] for q < n_out (see transpose_kernel), batched.
 int transpose(const void* in, int cols, int64_t ld_in, int64_t in_bstride, void* out,
-              int64_t ld_out, int64_t out_bstride, int n_out, const int* n_out_dev,
-              const int* src_of, int batches, bool f16_to_bf16, const int32_t* err,
+              int64_t ld_out, int64_t out_bstride, int n_out, int batches, bool f16_to_bf16,
+              const int32_t* err,
               cudaStream_t s) {
   if (cols <= 0 || n_out <= 0 || batches <= 0) return MOE_OK;
   dim3 grid((n_out + kTp - 1) / kTp, (cols + kTp - 1) / kTp, batches);
   transpose_kernel<<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(in), cols, ld_in, in_bstride,
                                         static_cast<uint16_t*>(out), ld_out, out_bstride, n_out,
-                                        n_out_dev, src_of, f16_to_bf16 ? 1 : 0, err);
+                                        f16_to_bf16 ? 1 : 0, err);
   return launch_status();
 }
 
@@ -874,12 +870,12 @@ int grouped_ffn_backward_impl(const __nv_bfloat16* recv, const __nv_bfloat16* dy
   if ((st = launch_status()) != MOE_OK) return st;
   // 2. W2T[z] = W2[z]^T [F,d], rounded to bf16, the pool's slots after the home experts (the
   //    dH GEMM reads it K-major; W1 and W3 are read MN-major by the dX GEMM, no copy)
-  if ((st = transpose(W2, F, F, (int64_t)d * F, w.w2t, d, (int64_t)F * d, d, nullptr, nullptr,
-                      e_home, true, err, s)))
+  if ((st = transpose(W2, F, F, (int64_t)d * F, w.w2t, d, (int64_t)F * d, d, e_home, true, err,
+                      s)))
     return st;
   if (n_pool > 0 &&
       (st = transpose(P2, F, F, (int64_t)d * F, w.w2t + (int64_t)e_home * F * d, d,
-                      (int64_t)F * d, d, nullptr, nullptr, n_pool, true, err, s)))
+                      (int64_t)F * d, d, n_pool, true, err, s)))
     return st;
   const int bnF = (F % 256 == 0) ? 256 : 128;
   const int bnD = (d % 256 == 0) ? 256 : 128;
