@@ -675,6 +675,19 @@ int moe_ipc_import(const void* handle, int64_t offset, void** ptr, void** base);
 int moe_ipc_close(void* base);
 
 /* ---------------------------------------------------------------------------------
+ * moe_w2_to_f16: the fp16 copy of a bf16 down projection that moe_prefetch_replicas,
+ * moe_grouped_ffn and the other FFN calls take (GEMM 2 runs with h and W2 both fp16; one
+ * tcgen05 MMA takes one operand type).  A caller holding bf16 weights ([MoonEP] para. 3:
+ * one contiguous tensor per projection) converts W2 once per weight version, not per step.
+ *   w2_bf16 [n] (any shape, e.g. [E,d,F]) bf16 -> w2_f16 [n] fp16 (out), round to nearest
+ *   even: 0 and every bf16 value with 2^-17 <= |w| <= 65504 convert exactly (below 2^-14 as
+ *   fp16 subnormals); smaller values round to the subnormal grid (spacing 2^-24), larger
+ *   ones become +-inf.  n % 8 == 0, both 16-byte aligned.  No error word: a weight
+ *   preparation step, not part of a layer's step.
+ */
+int moe_w2_to_f16(const moe_bf16* w2_bf16, int64_t n, moe_f16* w2_f16, moe_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
  * Grouped-FFN tile mode (a B200 tiling choice; the pages fix no kernel design).
  *   0  one CTA per 128-row x N tile (tcgen05.mma.cta_group::1), the default.
  *   1  CTA pairs (2-CTA clusters) on 256-row x N tiles (tcgen05.mma.cta_group::2): each

@@ -38,7 +38,8 @@ EXPERT_PARALLEL = ("moe_ep_counts", "moe_ep_plan", "moe_ep_prefetch", "moe_ep_di
 BACKWARD = ("moe_combine_backward", "moe_grouped_ffn_backward", "moe_dispatch_backward",
             "moe_topk_backward")
 HELPERS = ("moe_plan_get_layout", "moe_dispatch_workspace_words", "moe_status_string",
-           "moe_set_ffn_tile_mode", "moe_ffn_tile_mode", "moe_ffn_pair_clusters")
+           "moe_set_ffn_tile_mode", "moe_ffn_tile_mode", "moe_ffn_pair_clusters",
+           "moe_w2_to_f16")
 
 
 class MoEError(RuntimeError):
@@ -103,6 +104,7 @@ def lib() -> ctypes.CDLL:
                                             P, P, P, P, P, I64, P, P],
             "moe_ep_reduce_home": [P, P, P, P, I, I, I, I, I, I, P, P],
             "moe_ep_dispatch_backward": [P, P, I, I, I, I, P, P, P],
+            "moe_w2_to_f16": [P, I64, P, P],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -565,6 +567,17 @@ def ipc_import(handle: bytes, offset: int):
 
 def ipc_close(base: int):
     _check(lib().moe_ipc_close(base), "moe_ipc_close")
+
+
+def w2_to_f16(W2_bf16, out=None, stream=None):
+    """The fp16 copy of a bf16 down projection (once per weight version): moe_w2_to_f16."""
+    if out is None:
+        out = torch.empty(W2_bf16.shape, dtype=torch.float16, device=W2_bf16.device)
+    if out.shape != W2_bf16.shape:
+        raise ValueError("out must have W2's shape")
+    _check(lib().moe_w2_to_f16(_ptr(W2_bf16, torch.bfloat16, "W2_bf16"), W2_bf16.numel(),
+                               _ptr(out, torch.float16, "out"), _stream(stream)), "moe_w2_to_f16")
+    return out
 
 
 def moe_combine(y, perm, gate, out, err, stream=None):

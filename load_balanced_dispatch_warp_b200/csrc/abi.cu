@@ -666,6 +666,14 @@ int moe_ep_dispatch_backward(const moe_bf16* const* dx_rows_ranks, const int32_t
                                 as_stream(stream));
 }
 
+int moe_w2_to_f16(const moe_bf16* w2_bf16, int64_t n, moe_f16* w2_f16, moe_stream_t stream) {
+  if (n < 0 || (n > 0 && (!w2_bf16 || !w2_f16))) return MOE_ERR_ARG;
+  if (n % 8 != 0) return MOE_ERR_SHAPE;
+  if (!aligned16(w2_bf16) || !aligned16(w2_f16)) return MOE_ERR_ARG;
+  return moe::launch_bf16_to_f16(reinterpret_cast<const __nv_bfloat16*>(w2_bf16), n,
+                                 reinterpret_cast<__half*>(w2_f16), as_stream(stream));
+}
+
 int moe_set_ffn_tile_mode(int mode) { return moe::set_ffn_tile_mode(mode); }
 
 int moe_ffn_tile_mode(void) { return moe::ffn_tile_mode(); }

@@ -167,6 +167,9 @@ int launch_ep_reduce_home(const int32_t* plan, const moe_plan_layout& L,
                           float* const* part2_ranks, int W, int me, int E, int S, int d, int F,
                           const int32_t* err, cudaStream_t s);
 
+// bf16 -> fp16 copy of n (multiple of 8) values: the down projection's operand type.
+int launch_bf16_to_f16(const __nv_bfloat16* in, int64_t n, __half* out, cudaStream_t s);
+
 // ----------------------------------------------------------------------------- device side
 // Reads the layer's error word once per thread; every kernel after moe_topk returns
 // early when it is non-zero.

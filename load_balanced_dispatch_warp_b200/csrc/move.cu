@@ -194,7 +194,35 @@ int row_grid(int T) {
   return (int)(want < cap ? want : cap);
 }
 
+// bf16 -> fp16, element by element, round to nearest even (exact for 0 and every bf16 value
+// with 2^-17 <= |w| <= 65504; smaller ones round to the fp16 subnormal grid), 8 values per
+// thread and step.
+__global__ void __launch_bounds__(256) bf16_to_f16_kernel(const uint4* __restrict__ in,
+                                                          uint4* __restrict__ out, int64_t n8) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 v = __ldcs(in + i);
+    const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&v);
+    uint4 o;
+    __half2* h = reinterpret_cast<__half2*>(&o);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) h[j] = __float22half2_rn(__bfloat1622float2(b[j]));
+    out[i] = o;
+  }
+}
+
 }  // namespace
+
+int launch_bf16_to_f16(const __nv_bfloat16* in, int64_t n, __half* out, cudaStream_t s) {
+  if (n == 0) return MOE_OK;
+  const int64_t n8 = n / 8;
+  const int64_t want = (n8 + 255) / 256;
+  const int64_t cap = (int64_t)num_sms() * 8;
+  bf16_to_f16_kernel<<<(unsigned)(want < cap ? want : cap), 256, 0, s>>>(
+      reinterpret_cast<const uint4*>(in), reinterpret_cast<uint4*>(out), n8);
+  return launch_status();
+}
+
 
 int launch_prefetch(const int32_t* plan, const moe_plan_layout& L, const __nv_bfloat16* W1,
                     const __nv_bfloat16* W3, const __half* W2, int E, int R, int S, int d,

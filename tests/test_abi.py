@@ -304,3 +304,13 @@ def test_expert_parallel_backward_host_checks(lib):
     assert lib.moe_ep_reduce_home(fake, table(2), table(2, 0), table(2), 2, 0, 8, 2, 128, 256,
                                   fake, None) == M.MOE_ERR_ARG
     assert lib.moe_ep_dispatch_backward(table(2), fake, 2, 16, 2, 96, fake, fake, None) == M.MOE_ERR_SHAPE
+
+
+def test_w2_conversion_host_checks(lib):
+    P = ctypes.c_void_p
+    fake = P(4096)
+    assert lib.moe_w2_to_f16(fake, 12, fake, None) == M.MOE_ERR_SHAPE  # n % 8
+    assert lib.moe_w2_to_f16(fake, -8, fake, None) == M.MOE_ERR_ARG
+    assert lib.moe_w2_to_f16(None, 8, fake, None) == M.MOE_ERR_ARG
+    assert lib.moe_w2_to_f16(P(4098), 8, fake, None) == M.MOE_ERR_ARG  # misaligned
+    assert lib.moe_w2_to_f16(None, 0, None, None) == M.MOE_OK  # nothing to convert

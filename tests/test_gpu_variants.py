@@ -99,3 +99,20 @@ def test_capacity_ledger_parity(name):
         p, o, d, tot = _ledger_gpu(counts.tolist(), w.T, w.k, num, den)
         assert tot == [led["cap"], int(led["processed"].sum()), int(led["overflow"].sum()), int(led["padding"].sum())]
         assert p == led["processed"].tolist() and o == led["overflow"].tolist() and d == led["padding"].tolist()
+
+
+def test_w2_to_f16_matches_the_rounding_of_torch():
+    """bf16 -> fp16 of the down projection: every value equal to torch's conversion (round to
+    nearest even through fp32), including values that become fp16 subnormals or zeros, and
+    the synthetic W2 of the workloads (bf16-rounded N(0, 1/d) values)."""
+    g = torch.Generator().manual_seed(3)
+    v = torch.randn(1 << 16, generator=g) * torch.exp2(torch.randint(-30, 10, (1 << 16,), generator=g).float())
+    w = torch.cat([v, torch.tensor([0.0, -0.0, 65504.0, -65504.0, 2.0 ** -24, 2.0 ** -25, 1e5])])
+    w = torch.cat([w, torch.zeros((-w.numel()) % 8)]).to(torch.bfloat16).cuda()
+    out = M.w2_to_f16(w)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), w.float().to(torch.float16).view(torch.int16))
+    wl = I.small_workload("w2conv", 64, 8, 2, 4, 2, 256, 384)
+    W2 = I.make_weights(wl, device="cuda")[2]  # the fp16 images of bf16 values
+    back = M.w2_to_f16(W2.to(torch.bfloat16))
+    assert torch.equal(back, W2)
