@@ -256,10 +256,9 @@ def test_topk_expert_counts(E):
 
 @pytest.mark.parametrize("E,k", [(256, 8), (64, 6), (128, 8), (8, 2)])
 def test_topk_many_tokens_staged_rows(E, k):
-    """From 1024 tokens up (E a multiple of 4) the stand-alone top-k stages its rows through
-    shared memory in blocks of 16 with bulk copies: the DeepSeek workload's logits, then
-    T = 20001 (the last block has one token) of random logits with every fifth row made of
-    ties (the exact path)."""
+    """Many tokens through the stand-alone top-k: the DeepSeek workload's logits, then
+    T = 20001 random rows (the last block of 8 warps holds one token) with every fifth row
+    made of ties (the exact path)."""
     if E == 256:
         w = I.WORKLOADS["deepseek"]
         logits = I.make_logits(w)
@@ -275,6 +274,27 @@ def test_topk_many_tokens_staged_rows(E, k):
     gate = torch.empty(T, k, dtype=torch.float32, device="cuda")
     e = torch.zeros(1, dtype=torch.int32, device="cuda")
     M.moe_topk(logits.cuda(), k, idx, gate, e)
+    torch.cuda.synchronize()
+    assert e.item() == 0
+    assert np.array_equal(idx.cpu().numpy(), idx_ref)
+    assert np.abs(gate.cpu().double().numpy() - gate_ref).max() <= 1e-6
+
+
+def test_topk_biased_many_tokens():
+    """Bias-only selection over 113741 tokens (14218 blocks, a ragged last block) with
+    ties on every seventh row: ids bit-exact against the oracle, gates within 1e-6."""
+    T, E, k = 113741, 128, 6
+    g = torch.Generator().manual_seed(61)
+    logits = torch.randn(T, E, generator=g)
+    vals = torch.tensor([-1.0, -0.0, 0.0, 0.5, 2.0])
+    logits[::7] = vals[torch.randint(0, 5, logits[::7].shape, generator=g)]
+    bias = torch.randn(E, generator=g) * 0.5
+    idx_ref, gate_ref, err = O.topk_route_biased(logits.numpy(), bias.numpy(), k)
+    assert err == 0
+    idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    gate = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    e = torch.zeros(1, dtype=torch.int32, device="cuda")
+    M.moe_topk_biased(logits.cuda(), bias.cuda(), k, idx, gate, e)
     torch.cuda.synchronize()
     assert e.item() == 0
     assert np.array_equal(idx.cpu().numpy(), idx_ref)
