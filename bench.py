@@ -695,9 +695,10 @@ def run_ep(args, w: I.Workload, world, rank, local):
                             "with the replicas' reduced home)" if args.backward else "forward")},
         "clocks": clk,
         "e2e": None,
-        # per rank and step: top-k, counts, plan, prefetch, dispatch rank pass and row
-        # stores, group table, GEMM 1, GEMM 2, combine
-        "gpu_launches": 10 * len(ranks) * steps,
+        # per rank and step: error-word reset and top-k, send-vector reset and counts,
+        # plan, prefetch, workspace reset, dispatch rank pass and row stores, group table,
+        # GEMM 1, GEMM 2, combine
+        "gpu_launches": 13 * len(ranks) * steps,
     }
     if stage_ms is not None:
         st = {}

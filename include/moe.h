@@ -191,7 +191,8 @@ int moe_plan_balanced(const int32_t* counts, int T, int k, int E, int R, int S,
 /* ---------------------------------------------------------------------------------
  * Routing, histogram and plan fused: moe_topk (or moe_topk_biased when bias != NULL),
  * then moe_histogram_maxvio with the default home map (expert_to_rank = NULL), then
- * moe_plan_balanced, in one kernel launch (plus two memsets: err and the workspace):
+ * moe_plan_balanced, in one kernel launch (after a small one that zeroes err and the
+ * workspace):
  * every block routes its tokens, counts the chosen ids in shared memory and adds its
  * counts to one of 16 partial histograms in the workspace (integer atomics); the last
  * block to finish sums them into counts and computes loads, maxvio, balancedness and the

@@ -789,9 +789,9 @@ class MoELayer:
 
     # kernels launched by forward() (for launch accounting)
     def kernels_per_forward(self) -> int:
-        n = 1                                 # routing + histogram + plan (fused)
+        n = 2                                 # reset (err, workspace); routing + histogram + plan
         n += 1 if self.S > 0 else 0           # prefetch
-        n += (1 if self.fused else 2) if self.T > 0 else 0  # ranks[, row scatter]
+        n += (2 if self.fused else 3) if self.T > 0 else 0  # workspace reset, ranks[, row scatter]
         n += 2 if self.T > 0 else 0           # two grouped GEMMs
         n += 1 if self.T > 0 else 0           # combine (fused: the fp32 -> bf16 pass)
         return n

@@ -23,6 +23,10 @@ inline int launch_status() {
 int num_sms();  // SM count of the current device (cached per device)
 
 // --------------------------------------------------------------- launchers (one per step)
+// a[0, na) = 0 and b[0, nb) = 0 in one kernel launch (b may be null when nb == 0): the
+// small resets of the path (error word, workspaces), cheaper as a kernel node of a CUDA
+// graph than a memset node.
+int launch_zero(int32_t* a, int64_t na, int32_t* b, int64_t nb, cudaStream_t s);
 int launch_topk(const float* logits, int T, int E, int k, int32_t* idx, float* gate,
                 int32_t* err, cudaStream_t s);
 int launch_topk_biased(const float* logits, const float* bias, int T, int E, int k,

@@ -473,8 +473,7 @@ int launch_rank(const int32_t* idx, int T, int k, int E, int R, int C, int cap,
                 const int32_t* plan, const moe_plan_layout* L, int32_t* ws, int32_t* perm,
                 int32_t* src, int32_t* err, cudaStream_t s, const int32_t* q_base = nullptr) {
   const int ntiles = num_tiles(T);
-  if (cudaMemsetAsync(ws, 0, sizeof(int32_t) * (size_t)ws_agg_off(ntiles), s) != cudaSuccess)
-    return MOE_ERR_LAUNCH;
+  if (const int st = launch_zero(ws, ws_agg_off(ntiles), nullptr, 0, s); st != MOE_OK) return st;
   RankArgs a;
   a.idx = idx;
   a.T = T;

@@ -170,8 +170,7 @@ __global__ void __launch_bounds__(128) ep_groups_kernel(const int32_t* __restric
 
 int launch_ep_counts(const int32_t* idx, int T, int k, int E, const int32_t* err,
                      int32_t* send, cudaStream_t s) {
-  if (cudaMemsetAsync(send, 0, sizeof(int32_t) * (size_t)(E + 1), s) != cudaSuccess)
-    return MOE_ERR_LAUNCH;
+  if (const int st = launch_zero(send, E + 1, nullptr, 0, s); st != MOE_OK) return st;
   const int64_t want = ((int64_t)T + kCountThreads - 1) / kCountThreads;
   const int64_t capb = (int64_t)num_sms() * 2;
   const int blocks = (int)(want < 1 ? 1 : (want < capb ? want : capb));

@@ -37,11 +37,22 @@ __device__ __forceinline__ float warp_max_f32(float v) {
 //   3. k rounds over one candidate per lane: warp max key, lowest expert id among its
 //      holders, the winner drops out.
 // More than 32 candidates (many equal keys) runs the rounds over all of the lane's keys.
-// On return lane j < k holds the j-th choice: its expert id and its unbiased logit.
+// On return lane j < k holds the j-th choice: its expert id and its unbiased logit.  The
+// token's logits (row) and the biases are read again here rather than handed over from the
+// caller's registers: an array passed by address would live in local memory, and the
+// caller would store every token's row there although only a few tokens come here.
 template <int VPL, bool BIASED>
-__device__ __noinline__ void topk_exact(const float* x, const float* b, int E, int k, int lane,
+__device__ __noinline__ void topk_exact(const float* __restrict__ row,
+                                        const float* __restrict__ bias, int E, int k, int lane,
                                         uint32_t* s_key, int* s_id, float* s_raw,
                                         float& my_val, int& my_id) {
+  float x[VPL], b[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int e = lane + 32 * i;
+    x[i] = e < E ? row[e] : 0.f;
+    b[i] = (BIASED && e < E) ? __ldg(bias + e) : 0.f;
+  }
   uint32_t key[VPL];
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
@@ -162,6 +173,7 @@ __device__ __forceinline__ void load_row(const float* __restrict__ logits, int64
 // exactly 32 * VPL, so no lane holds a slot past the last expert.
 template <int VPL, int K, bool BIASED, bool COUNT, bool FULL = false>
 __device__ __forceinline__ bool topk_token_loaded(const float (&x)[VPL],
+                                                  const float* __restrict__ row,
                                                   const float* __restrict__ bias, int64_t t,
                                                   int E, int k, int lane, uint32_t* s_key,
                                                   int* s_id, float* s_raw,
@@ -259,7 +271,7 @@ __device__ __forceinline__ bool topk_token_loaded(const float (&x)[VPL],
   }
   float my_val;
   int my_id;
-  topk_exact<VPL, BIASED>(x, b, E, k, lane, s_key, s_id, s_raw, my_val, my_id);
+  topk_exact<VPL, BIASED>(row, bias, E, k, lane, s_key, s_id, s_raw, my_val, my_id);
   float top = lane < k ? my_val : -INFINITY;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) top = fmaxf(top, __shfl_xor_sync(MOE_FULL_MASK, top, o));
@@ -282,8 +294,9 @@ __device__ __forceinline__ bool topk_token(const float* __restrict__ logits,
                                            int32_t* __restrict__ err) {
   float x[VPL];
   load_row<VPL, FULL>(logits, t, E, lane, x);
-  return topk_token_loaded<VPL, K, BIASED, COUNT, FULL>(x, bias, t, E, k, lane, s_key, s_id,
-                                                        s_raw, idx, gate, counts, err);
+  return topk_token_loaded<VPL, K, BIASED, COUNT, FULL>(x, logits + t * E, bias, t, E, k, lane,
+                                                        s_key, s_id, s_raw, idx, gate, counts,
+                                                        err);
 }
 
 // Warps (tokens) per block of the stand-alone top-k.
@@ -635,18 +648,36 @@ void launch_route_plan_vpl(const float* logits, const float* bias, int T, int E,
 #undef MOE_RP
 }
 
+__global__ void __launch_bounds__(256) zero_kernel(int32_t* __restrict__ a, int64_t na,
+                                                   int32_t* __restrict__ b, int64_t nb) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < na + nb; i += stride) {
+    if (i < na) a[i] = 0;
+    else b[i - na] = 0;
+  }
+}
+
 }  // namespace
+
+int launch_zero(int32_t* a, int64_t na, int32_t* b, int64_t nb, cudaStream_t s) {
+  const int64_t n = na + nb;
+  if (n <= 0) return MOE_OK;
+  const int64_t want = (n + 255) / 256;
+  const int grid = (int)(want < (int64_t)num_sms() * 4 ? want : (int64_t)num_sms() * 4);
+  zero_kernel<<<grid, 256, 0, s>>>(a, na, b, nb);
+  return launch_status();
+}
 
 int launch_topk(const float* logits, int T, int E, int k, int32_t* idx, float* gate,
                 int32_t* err, cudaStream_t s) {
-  if (cudaMemsetAsync(err, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_LAUNCH;
+  if (const int st = launch_zero(err, 1, nullptr, 0, s); st != MOE_OK) return st;
   if (T == 0) return MOE_OK;
   return launch_topk_impl(logits, nullptr, T, E, k, idx, gate, err, s);
 }
 
 int launch_topk_biased(const float* logits, const float* bias, int T, int E, int k,
                        int32_t* idx, float* gate, int32_t* err, cudaStream_t s) {
-  if (cudaMemsetAsync(err, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_LAUNCH;
+  if (const int st = launch_zero(err, 1, nullptr, 0, s); st != MOE_OK) return st;
   if (T == 0) return MOE_OK;
   return launch_topk_impl(logits, bias, T, E, k, idx, gate, err, s);
 }
@@ -662,9 +693,7 @@ int launch_capacity(const int32_t* counts, int E, long long A, int cf_num, int c
 int launch_histogram(const int32_t* idx, int T, int k, int E, int R, const int32_t* map,
                      int32_t* counts, int32_t* loads, double* maxvio, double* bal,
                      int32_t* err, cudaStream_t s) {
-  if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, s) != cudaSuccess ||
-      cudaMemsetAsync(loads, 0, sizeof(int32_t), s) != cudaSuccess)
-    return MOE_ERR_LAUNCH;
+  if (const int st = launch_zero(counts, E, loads, 1, s); st != MOE_OK) return st;
   const int threads = 512;
   // about two blocks per SM, each over a contiguous token range (one block when T == 0)
   int blocks = 2 * num_sms();
@@ -683,10 +712,7 @@ int launch_route_plan(const float* logits, const float* bias, int T, int E, int 
                       int S, int32_t* idx, float* gate, int32_t* counts, int32_t* loads,
                       double* maxvio, double* bal, int32_t* plan, const moe_plan_layout& L,
                       int32_t* ws, int32_t* err, cudaStream_t s) {
-  if (cudaMemsetAsync(err, 0, sizeof(int32_t), s) != cudaSuccess ||
-      cudaMemsetAsync(ws, 0, sizeof(int32_t) * (size_t)route_plan_workspace_words(E), s) !=
-          cudaSuccess)
-    return MOE_ERR_LAUNCH;
+  if (const int st = launch_zero(err, 1, ws, route_plan_workspace_words(E), s); st != MOE_OK) return st;
 #define MOE_RP_VPL(V) \
   launch_route_plan_vpl<V>(logits, bias, T, E, k, R, S, idx, gate, counts, loads, maxvio, bal, plan, L, ws, err, s)
   if (E <= 32) MOE_RP_VPL(1);
