@@ -20,6 +20,15 @@ __device__ __forceinline__ uint32_t order_key(float v) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// The routing kernels are launched as programmatic dependents of the small kernel that
+// zeroes the error word (and the routing workspace): they start while it finishes, and
+// wait for it (griddepcontrol.wait: the reset grid complete, its stores visible) only
+// before their first write to a word it zeroes.  Without that launch attribute the wait
+// returns at once.
+__device__ __forceinline__ void wait_for_reset() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // Warp-wide fp32 maximum (one instruction on sm_100a).
 __device__ __forceinline__ float warp_max_f32(float v) {
   float r;
@@ -193,7 +202,10 @@ __device__ __forceinline__ bool topk_token_loaded(const float (&x)[VPL],
       bad |= !isfinite(b[i]);
     }
     if (__any_sync(MOE_FULL_MASK, bad)) {
-      if (lane == 0) atomicOr(err, MOE_DERR_NONFINITE);
+      if (lane == 0) {
+        wait_for_reset();
+        atomicOr(err, MOE_DERR_NONFINITE);
+      }
       return false;
     }
   }
@@ -206,7 +218,10 @@ __device__ __forceinline__ bool topk_token_loaded(const float (&x)[VPL],
     key[i] = (FULL || lane + 32 * i < E) ? (BIASED ? __fadd_rn(x[i], b[i]) : x[i]) : -INFINITY;
   }
   if (__any_sync(MOE_FULL_MASK, !(z == 0.f))) {
-    if (lane == 0) atomicOr(err, MOE_DERR_NONFINITE);
+    if (lane == 0) {
+      wait_for_reset();
+      atomicOr(err, MOE_DERR_NONFINITE);
+    }
     return false;
   }
   float h1 = key[0], h2 = -INFINITY;
@@ -317,6 +332,9 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_kernel(const float* __re
   if (t >= T) return;
   topk_token<VPL, K, BIASED, false, FULL>(logits, bias, t, E, k, lane, s_key[wib], s_id[wib],
                                           s_raw[wib], idx, gate, nullptr, err);
+  // no block ends before the reset grid has (warp 0 of every block has a token), so the
+  // work that follows this grid on the stream also follows the reset
+  wait_for_reset();
 }
 
 // Fixed-capacity ledger of "MoE Load Balancing: Find Expert Hotspots" ("Make expert
@@ -497,20 +515,38 @@ __global__ void __launch_bounds__(512) hist_kernel(const int32_t* __restrict__ i
   hist_finish(counts, T, k, E, R, map, loads, maxvio, bal, err, s_hist, s_max);
 }
 
+// Launch of a routing kernel right after launch_zero on the same stream, as its
+// programmatic dependent (see wait_for_reset).
+template <typename... Params, typename... Args>
+void launch_after_reset(void (*kernel)(Params...), unsigned grid, unsigned block, size_t smem,
+                        cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(block, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kernel, static_cast<Params>(args)...);  // status: launch_status()
+}
+
 // One warp per token, 8 warps per block.  Unbiased calls with k in {2, 4, 6, 8} and up to
 // 256 experts run a kernel with k fixed at compile time (the rounds unroll).
 template <int VPL>
 void launch_topk_vpl(const float* logits, const float* bias, int T, int E, int k, int32_t* idx,
                      float* gate, int32_t* err, cudaStream_t s) {
   const unsigned grid = (unsigned)(((int64_t)T + kTopkWarps - 1) / kTopkWarps);
-#define MOE_TOPK(KK, B) topk_kernel<VPL, KK, B><<<grid, kTopkWarps * 32, 0, s>>>(logits, bias, T, E, k, idx, gate, err)
+#define MOE_TOPK(KK, B) launch_after_reset(topk_kernel<VPL, KK, B>, grid, kTopkWarps * 32, 0, s, logits, bias, T, E, k, idx, gate, err)
   if (bias) {
     MOE_TOPK(0, true);
     return;
   }
   if constexpr (VPL <= 8) {
     if (E == 32 * VPL) {
-#define MOE_TOPK_FULL(KK) topk_kernel<VPL, KK, false, true><<<grid, kTopkWarps * 32, 0, s>>>(logits, bias, T, E, k, idx, gate, err)
+#define MOE_TOPK_FULL(KK) launch_after_reset(topk_kernel<VPL, KK, false, true>, grid, kTopkWarps * 32, 0, s, logits, bias, T, E, k, idx, gate, err)
       switch (k) {
         case 8: MOE_TOPK_FULL(8); return;
         case 6: MOE_TOPK_FULL(6); return;
@@ -579,6 +615,7 @@ __global__ void __launch_bounds__(kPlanThreads) route_plan_kernel(
     topk_token<VPL, K, BIASED, true, FULL>(logits, bias, t, E, k, lane, s_key[wib], s_id[wib],
                                            s_raw[wib], idx, gate, s_dyn, err);
   __syncthreads();
+  wait_for_reset();  // ws and err zeroed
   int32_t* copy = ws + (int64_t)(blockIdx.x % kCountCopies) * E;
   for (int e = threadIdx.x; e < E; e += blockDim.x)
     if (s_dyn[e]) atomicAdd(copy + e, s_dyn[e]);
@@ -615,9 +652,8 @@ void launch_route_plan_vpl(const float* logits, const float* bias, int T, int E,
   const unsigned grid = T > 0 ? (unsigned)(((int64_t)T + 7) / 8) : 1u;
   const size_t smem = sizeof(int) * (size_t)(E + plan_smem_words(E, R));
 #define MOE_RP(KK, B)                                                                           \
-  route_plan_kernel<VPL, KK, B><<<grid, kPlanThreads, smem, s>>>(logits, bias, T, E, k, R, S, idx, \
-                                                                 gate, counts, loads, maxvio, bal, \
-                                                                 plan, L, ws, err)
+  launch_after_reset(route_plan_kernel<VPL, KK, B>, grid, kPlanThreads, smem, s, logits, bias, T, \
+                     E, k, R, S, idx, gate, counts, loads, maxvio, bal, plan, L, ws, err)
   if (bias) {
     MOE_RP(0, true);
     return;
@@ -625,8 +661,8 @@ void launch_route_plan_vpl(const float* logits, const float* bias, int T, int E,
   if constexpr (VPL <= 8) {
     if (E == 32 * VPL) {
 #define MOE_RP_FULL(KK)                                                                         \
-  route_plan_kernel<VPL, KK, false, true><<<grid, kPlanThreads, smem, s>>>(                        \
-      logits, bias, T, E, k, R, S, idx, gate, counts, loads, maxvio, bal, plan, L, ws, err)
+  launch_after_reset(route_plan_kernel<VPL, KK, false, true>, grid, kPlanThreads, smem, s, logits, \
+                     bias, T, E, k, R, S, idx, gate, counts, loads, maxvio, bal, plan, L, ws, err)
       switch (k) {
         case 8: MOE_RP_FULL(8); return;
         case 6: MOE_RP_FULL(6); return;
@@ -650,6 +686,9 @@ void launch_route_plan_vpl(const float* logits, const float* bias, int T, int E,
 
 __global__ void __launch_bounds__(256) zero_kernel(int32_t* __restrict__ a, int64_t na,
                                                    int32_t* __restrict__ b, int64_t nb) {
+  // a dependent launched with programmatic serialisation may start now; it waits for this
+  // grid's completion (griddepcontrol.wait) before touching a or b
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < na + nb; i += stride) {
     if (i < na) a[i] = 0;

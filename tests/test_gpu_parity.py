@@ -301,6 +301,58 @@ def test_topk_biased_many_tokens():
     assert np.abs(gate.cpu().double().numpy() - gate_ref).max() <= 1e-6
 
 
+def test_topk_resets_a_stale_error_word_before_the_next_call():
+    """moe_topk starts while its error-word reset is still finishing (a programmatic
+    dependent launch): a stale non-zero word must read 0 after a clean call, so that the
+    histogram launched next on the stream runs, and exactly NONFINITE after a call with one
+    non-finite logit in the last token; both inside one CUDA graph replayed twice."""
+    T, E, k, R = 4096, 256, 8, 32
+    g = torch.Generator().manual_seed(77)
+    clean = torch.randn(T, E, generator=g).cuda()
+    bad = clean.clone()
+    bad[T - 1, 5] = float("nan")
+    idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    gate = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    err = torch.empty(1, dtype=torch.int32, device="cuda")
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    loads = torch.empty(R, dtype=torch.int32, device="cuda")
+    mv = torch.empty(1, dtype=torch.float64, device="cuda")
+    bal = torch.empty(1, dtype=torch.float64, device="cuda")
+    err_after = torch.empty(2, dtype=torch.int32, device="cuda")
+    counts_after = torch.empty(E, dtype=torch.int32, device="cuda")
+    idx_ref, _, _ = O.topk_route(clean.cpu().numpy(), k)
+    counts_ref = np.bincount(idx_ref.reshape(-1), minlength=E)
+
+    def step():
+        err.fill_(0x7F)  # stale bits from an earlier step
+        M.moe_topk(clean, k, idx, gate, err)
+        M.moe_histogram_maxvio(idx, E, R, counts, loads, mv, bal, err)
+        err_after[0:1].copy_(err)
+        counts_after.copy_(counts)
+        err.fill_(0x7F)
+        M.moe_topk(bad, k, idx, gate, err)
+        err_after[1:2].copy_(err)
+
+    step()
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        graph.capture_begin()
+        step()
+        graph.capture_end()
+    torch.cuda.synchronize()
+    for _ in range(2):
+        err_after.fill_(-1)
+        counts_after.fill_(-1)
+        graph.replay()
+        torch.cuda.synchronize()
+        assert err_after.tolist() == [0, M.DERR_NONFINITE]
+        assert np.array_equal(counts_after.cpu().numpy(), counts_ref)
+    del graph
+
+
 def test_bounded_wait_gives_up_and_context_survives():
     """The FFN's bounded mbarrier wait, on a barrier nothing arrives at, returns with the
     timeout bit; the next layer on the same context still matches the oracle."""
