@@ -43,6 +43,10 @@ SMALL = [
     I.small_workload("hot", 512, 32, 4, 8, 4, 128, 256, alpha=2.5, seed=7),
     I.small_workload("wide_E", 200, 512, 8, 16, 12, 128, 128, alpha=0.3, seed=8),
     I.small_workload("wide_E_few_slots", 200, 512, 8, 16, 4, 128, 128, alpha=0.3, seed=8),
+    # one token: C = 1 row per rank, single-row groups and tiles
+    I.small_workload("single_token", 1, 8, 2, 2, 2, 128, 128, alpha=1.0, seed=15),
+    # one token per expert slot: T*k/R = 1 with every rank's row a replica or a home row
+    I.small_workload("one_row_per_rank", 4, 16, 4, 16, 1, 256, 128, alpha=0.0, seed=16),
 ]
 
 
