@@ -63,7 +63,7 @@ enum {
   MOE_DERR_ID_RANGE = 2,   /* an expert id outside [0, E)                            */
   MOE_DERR_DUPLICATE = 4,  /* a token names the same expert twice                    */
   MOE_DERR_SLOTS = 8,      /* the plan needs more than S replicas on some rank       */
-  MOE_DERR_TIMEOUT = 16    /* a bounded wait inside the grouped FFN gave up          */
+  MOE_DERR_TIMEOUT = 16    /* a bounded wait inside a kernel gave up (FFN, copies)  */
 };
 
 /* Word offsets of the plan's fields inside the caller's int32 plan buffer. */
@@ -222,11 +222,13 @@ int moe_route_plan(const float* logits, const float* bias, int T, int E, int k, 
  *   P1, P3 [R*S,F,d] bf16, P2 [R*S,d,F] fp16 (out) the pool; slot u*S+s receives a
  *          bitwise copy of expert replica_expert[u*S+s]; empty slots are not written.
  *          The pool is owned by the caller and may be shared by every layer.
- *   err    no-op when non-zero.
+ *          The copies run on the bulk-copy engine (32 KiB chunks staged in shared memory).
+ *   err    no-op when non-zero; MOE_DERR_TIMEOUT if a copy's bounded wait runs out (the
+ *          only write to it).
  */
 int moe_prefetch_replicas(const int32_t* plan, const moe_bf16* W1, const moe_bf16* W3,
                           const moe_f16* W2, int E, int R, int S, int d, int F,
-                          moe_bf16* P1, moe_bf16* P3, moe_f16* P2, const int32_t* err,
+                          moe_bf16* P1, moe_bf16* P3, moe_f16* P2, int32_t* err,
                           moe_stream_t stream);
 
 /* ---------------------------------------------------------------------------------

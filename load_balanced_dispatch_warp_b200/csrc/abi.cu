@@ -179,7 +179,7 @@ int moe_route_plan(const float* logits, const float* bias, int T, int E, int k, 
 
 int moe_prefetch_replicas(const int32_t* plan, const moe_bf16* W1, const moe_bf16* W3,
                           const moe_f16* W2, int E, int R, int S, int d, int F,
-                          moe_bf16* P1, moe_bf16* P3, moe_f16* P2, const int32_t* err,
+                          moe_bf16* P1, moe_bf16* P3, moe_f16* P2, int32_t* err,
                           moe_stream_t stream) {
   if (!plan || !W1 || !W3 || !W2 || !err) return MOE_ERR_ARG;
   if (S > 0 && (!P1 || !P3 || !P2)) return MOE_ERR_ARG;

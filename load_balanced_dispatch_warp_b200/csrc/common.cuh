@@ -46,8 +46,8 @@ int launch_route_plan(const float* logits, const float* bias, int T, int E, int 
                       int32_t* ws, int32_t* err, cudaStream_t s);
 int launch_prefetch(const int32_t* plan, const moe_plan_layout& L, const __nv_bfloat16* W1,
                     const __nv_bfloat16* W3, const __half* W2, int E, int R, int S, int d,
-                    int F, __nv_bfloat16* P1, __nv_bfloat16* P3, __half* P2,
-                    const int32_t* err, cudaStream_t s);
+                    int F, __nv_bfloat16* P1, __nv_bfloat16* P3, __half* P2, int32_t* err,
+                    cudaStream_t s);
 int launch_dispatch(const __nv_bfloat16* x, const int32_t* idx, const int32_t* plan,
                     const moe_plan_layout& L, int T, int k, int E, int R, int d,
                     int32_t* ws, __nv_bfloat16* recv, int32_t* perm, int32_t* src,
