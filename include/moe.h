@@ -223,8 +223,9 @@ int moe_route_plan(const float* logits, const float* bias, int T, int E, int k, 
  *          bitwise copy of expert replica_expert[u*S+s]; empty slots are not written.
  *          The pool is owned by the caller and may be shared by every layer.
  *          The copies run on the bulk-copy engine (32 KiB chunks staged in shared memory).
- *   err    no-op when non-zero; MOE_DERR_TIMEOUT if a copy's bounded wait runs out (the
- *          only write to it).
+ *   err    no-op when non-zero; MOE_DERR_ID_RANGE if the plan lists a slot outside
+ *          [0, R*S) or an expert outside [0, E) (that slot is skipped), MOE_DERR_TIMEOUT if
+ *          a copy's bounded wait runs out.
  */
 int moe_prefetch_replicas(const int32_t* plan, const moe_bf16* W1, const moe_bf16* W3,
                           const moe_f16* W2, int E, int R, int S, int d, int F,
@@ -540,13 +541,15 @@ int moe_ep_plan(const int32_t* gathered, int W, int me, int T, int k, int E, int
  *            tables of every rank's home tensors (see "Pointer tables").
  *   P1, P3 [S,F,d] bf16, P2 [S,d,F] fp16 (out): this rank's slots; slot s receives
  *            expert e = replica_expert[me*S + s] (local expert e % B of rank e / B),
- *            bitwise; empty slots are untouched.
- *   err  no-op when non-zero.
+ *            bitwise; empty slots are untouched.  Bulk copies (no multicast) staged in
+ *            this GPU's shared memory, as moe_prefetch_replicas.
+ *   err  no-op when non-zero; MOE_DERR_ID_RANGE if a slot names an expert outside
+ *        [0, W*B) (that slot is skipped), MOE_DERR_TIMEOUT if a copy's bounded wait runs out.
  */
 int moe_ep_prefetch(const int32_t* plan, const moe_bf16* const* W1_ranks,
                     const moe_bf16* const* W3_ranks, const moe_f16* const* W2_ranks, int W,
                     int me, int E, int S, int d, int F, moe_bf16* P1, moe_bf16* P3, moe_f16* P2,
-                    const int32_t* err, moe_stream_t stream);
+                    int32_t* err, moe_stream_t stream);
 
 /*
  * moe_ep_dispatch: every assignment of this rank's tokens straight into its final row on

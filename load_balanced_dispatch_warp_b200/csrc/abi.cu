@@ -478,7 +478,7 @@ int moe_ep_plan(const int32_t* gathered, int W, int me, int T, int k, int E, int
 int moe_ep_prefetch(const int32_t* plan, const moe_bf16* const* W1_ranks,
                     const moe_bf16* const* W3_ranks, const moe_f16* const* W2_ranks, int W,
                     int me, int E, int S, int d, int F, moe_bf16* P1, moe_bf16* P3, moe_f16* P2,
-                    const int32_t* err, moe_stream_t stream) {
+                    int32_t* err, moe_stream_t stream) {
   if (!plan || !err) return MOE_ERR_ARG;
   MOE_TRY(check_ep(W, me, 0, 1, E, S));
   MOE_TRY(check_dims(0, 1, d, F));

@@ -139,7 +139,7 @@ int launch_ep_groups(const int32_t* plan, const moe_plan_layout& L, int me, int 
 int launch_ep_prefetch(const int32_t* plan, const moe_plan_layout& L,
                        const __nv_bfloat16* const* W1_ranks, const __nv_bfloat16* const* W3_ranks,
                        const __half* const* W2_ranks, int W, int me, int E, int S, int d, int F,
-                       __nv_bfloat16* P1, __nv_bfloat16* P3, __half* P2, const int32_t* err,
+                       __nv_bfloat16* P1, __nv_bfloat16* P3, __half* P2, int32_t* err,
                        cudaStream_t s);
 int launch_ep_dispatch(const __nv_bfloat16* x, const int32_t* idx, const int32_t* q_base,
                        const int32_t* plan, const moe_plan_layout& L, int T, int k, int E,

@@ -12,23 +12,28 @@ namespace moe {
 namespace {
 
 // ----------------------------------------------------------------------------- prefetch
-// the expert-parallel prefetch's vector copy (peer memory): threads per block, 16-byte
-// vectors per thread per chunk, vectors per chunk (16 KiB)
-constexpr int kCopyThreads = 256;
-constexpr int kCopyVec = 4;
-constexpr int kCopyChunk = kCopyThreads * kCopyVec;
 
 // Replica prefetch through the bulk-copy engine: one thread per CTA (one CTA per SM)
 // streams 32 KiB chunks global -> shared (completion on the buffer's mbarrier) -> global
 // (bulk group), kBulkBufs buffers in flight, so the copy rate does not depend on how many
 // instructions the SM issues (a 16-byte-vector copy with 1024 threads per SM reached 0.92
 // of the copy peak alone and 0.86 in the power-capped step; this one 0.97 and 0.94).
-// Units are (filled slot from the plan's compact list, projection, chunk); d*F*2 is a
-// multiple of 32 KiB (d and F are multiples of 128).  Every wait is bounded; a wait that
-// runs out ORs MOE_DERR_TIMEOUT into *err and the thread drains its copies before the CTA
-// leaves.
+// Units are (filled slot, projection, chunk); d*F*2 is a multiple of 32 KiB (d and F are
+// multiples of 128).  Every wait is bounded; a wait that runs out ORs MOE_DERR_TIMEOUT into
+// *err and the thread drains its copies before the CTA leaves.
+//
+// Where a slot's expert lives: w[p][u] is rank u's home tensor of projection p (W1, W3,
+// W2) and holds experts [u*B, (u+1)*B).  One GPU: one "rank" with B = E, the slots to fill
+// from the plan's compact list.  Expert parallelism: this process's pointers to every
+// rank's home tensors (a peer GPU's memory mapped here, read over NVLink; bulk loads, no
+// multicast) and rank `me`'s own S slots, the filled ones gathered by the copying thread.
+struct PrefetchSrc {
+  const uint8_t* w[3][MOE_EP_MAX_RANKS];
+  int B;
+};
 constexpr int kBulkChunk = 32768;
 constexpr int kBulkBufs = 6;
+constexpr int kBulkMaxSlots = 4096;  // slots of one rank: the argument rules keep R*(B+S) <= 4096
 constexpr uint64_t kBulkWaitNs = 500000000ull;
 
 __device__ __forceinline__ uint32_t bulk_smem(const void* p) {
@@ -57,38 +62,64 @@ __device__ __forceinline__ bool bulk_wait(uint32_t bar, uint32_t parity) {
   }
 }
 
+// rep[0, nslots): the experts of the slots (-1 empty); list: the plan's compact list of
+// filled slots ({count, slots...}), or null to take the filled ones of rep in slot order.
+// A listed slot outside [0, nslots), or an expert whose home tensor is not in the table,
+// sets MOE_DERR_ID_RANGE and is skipped (never read from or written to).
 __global__ void __launch_bounds__(32) prefetch_bulk_kernel(
-    const int32_t* __restrict__ rep, const int32_t* __restrict__ rep_list,
-    const uint8_t* __restrict__ W1, const uint8_t* __restrict__ W3, const uint8_t* __restrict__ W2,
-    uint8_t* __restrict__ P1, uint8_t* __restrict__ P3, uint8_t* __restrict__ P2,
-    int64_t proj_bytes, int32_t* __restrict__ err) {
+    const int32_t* __restrict__ rep, const int32_t* __restrict__ list, int nslots,
+    const __grid_constant__ PrefetchSrc src, uint8_t* __restrict__ P1, uint8_t* __restrict__ P3,
+    uint8_t* __restrict__ P2, int64_t proj_bytes, int32_t* __restrict__ err) {
   extern __shared__ __align__(128) uint8_t buf[];  // kBulkBufs * kBulkChunk
   __shared__ __align__(8) uint64_t bar[kBulkBufs];
+  __shared__ int s_slots[kBulkMaxSlots];
   if (threadIdx.x != 0) return;
   if (load_err(err)) return;
   for (int b = 0; b < kBulkBufs; ++b)
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bulk_smem(&bar[b])) : "memory");
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  const int n = __ldg(rep_list);
+  const int cand = list != nullptr ? min(__ldg(list), kBulkMaxSlots) : min(nslots, kBulkMaxSlots);
+  int n = 0;
+  bool bad = false;
+  for (int c = 0; c < cand; ++c) {
+    const int q = list != nullptr ? __ldg(list + 1 + c) : c;
+    if (q < 0 || q >= nslots) {
+      bad = true;
+      continue;
+    }
+    const int e = __ldg(rep + q);
+    if (e < 0) {
+      bad |= list != nullptr;  // the plan lists filled slots only
+      continue;
+    }
+    const int home = e / src.B;
+    if (home >= MOE_EP_MAX_RANKS || src.w[0][home] == nullptr) {
+      bad = true;
+      continue;
+    }
+    s_slots[n++] = q;
+  }
+  if (bad) atomicOr(err, MOE_DERR_ID_RANGE);
   const int64_t chunks = proj_bytes / kBulkChunk;
   const int64_t total = (int64_t)n * 3 * chunks;
   // this CTA's units: blockIdx.x + i * gridDim.x, i = 0, 1, ...
   const int64_t mine = total > blockIdx.x ? (total - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
-  auto unit_ptrs = [&](int64_t i, const uint8_t*& src, uint8_t*& dst) {
+  auto unit_ptrs = [&](int64_t i, const uint8_t*& from, uint8_t*& to) {
     const int64_t w = blockIdx.x + i * gridDim.x;
     const int64_t si = w / (3 * chunks);
     const int64_t rem = w - si * 3 * chunks;
     const int proj = (int)(rem / chunks);
     const int64_t off = (rem - (int64_t)proj * chunks) * kBulkChunk;
-    const int slot = __ldg(rep_list + 1 + si);
+    const int slot = s_slots[si];
     const int e = __ldg(rep + slot);
-    src = (proj == 0 ? W1 : proj == 1 ? W3 : W2) + (int64_t)e * proj_bytes + off;
-    dst = (proj == 0 ? P1 : proj == 1 ? P3 : P2) + (int64_t)slot * proj_bytes + off;
+    const int home = e / src.B;
+    from = src.w[proj][home] + (int64_t)(e - home * src.B) * proj_bytes + off;
+    to = (proj == 0 ? P1 : proj == 1 ? P3 : P2) + (int64_t)slot * proj_bytes + off;
   };
   auto issue_load = [&](int64_t i) {
-    const uint8_t* src;
-    uint8_t* dst;
-    unit_ptrs(i, src, dst);
+    const uint8_t* from;
+    uint8_t* to;
+    unit_ptrs(i, from, to);
     const int b = (int)(i % kBulkBufs);
     const uint32_t bb = bulk_smem(&bar[b]);
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bb),
@@ -97,7 +128,7 @@ __global__ void __launch_bounds__(32) prefetch_bulk_kernel(
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
             bulk_smem(buf + (size_t)b * kBulkChunk)),
-        "l"(src), "r"(kBulkChunk), "r"(bb)
+        "l"(from), "r"(kBulkChunk), "r"(bb)
         : "memory");
   };
   int64_t issued = 0, i = 0;
@@ -109,10 +140,10 @@ __global__ void __launch_bounds__(32) prefetch_bulk_kernel(
       ok = false;
       break;
     }
-    const uint8_t* src;
-    uint8_t* dst;
-    unit_ptrs(i, src, dst);
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+    const uint8_t* from;
+    uint8_t* to;
+    unit_ptrs(i, from, to);
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(to),
                  "r"(bulk_smem(buf + (size_t)b * kBulkChunk)), "r"(kBulkChunk)
                  : "memory");
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
@@ -130,48 +161,21 @@ __global__ void __launch_bounds__(32) prefetch_bulk_kernel(
   }
 }
 
-// Expert parallelism across GPUs: rank `me` fills its own S pool slots.  Slot s holds
-// expert e = replica_expert[me*S + s], whose weights sit on its home rank e / B as local
-// expert e % B; src* are this process's pointers to every rank's home tensors (a peer
-// GPU's memory mapped here, read over NVLink).  Grid-stride over (slot, projection,
-// chunk); empty slots are skipped.
-struct RankTensors {
-  const uint4* w1[MOE_EP_MAX_RANKS];
-  const uint4* w3[MOE_EP_MAX_RANKS];
-  const uint4* w2[MOE_EP_MAX_RANKS];
-};
-
-__global__ void __launch_bounds__(kCopyThreads) ep_prefetch_kernel(
-    const int32_t* __restrict__ rep, int me, int S, int B, const __grid_constant__ RankTensors src,
-    uint4* __restrict__ P1, uint4* __restrict__ P3, uint4* __restrict__ P2, int64_t vecs,
-    const int32_t* __restrict__ err) {
-  if (load_err(err)) return;
-  const int64_t chunks = (vecs + kCopyChunk - 1) / kCopyChunk;
-  const int64_t total = (int64_t)S * 3 * chunks;
-  for (int64_t w = blockIdx.x; w < total; w += gridDim.x) {
-    const int slot = (int)(w / (3 * chunks));
-    const int64_t rem = w - (int64_t)slot * 3 * chunks;
-    const int proj = (int)(rem / chunks);
-    const int64_t c = rem - (int64_t)proj * chunks;
-    const int e = __ldg(rep + (int64_t)me * S + slot);
-    if (e < 0) continue;
-    const int home = e / B;
-    const uint4* from = (proj == 0 ? src.w1[home] : proj == 1 ? src.w3[home] : src.w2[home]) +
-                        (int64_t)(e - home * B) * vecs;
-    uint4* to = (proj == 0 ? P1 : proj == 1 ? P3 : P2) + (int64_t)slot * vecs;
-    const int64_t v0 = c * kCopyChunk + threadIdx.x;
-    uint4 buf[kCopyVec];
-#pragma unroll
-    for (int i = 0; i < kCopyVec; ++i) {
-      const int64_t v = v0 + i * kCopyThreads;
-      if (v < vecs) buf[i] = __ldcs(from + v);
-    }
-#pragma unroll
-    for (int i = 0; i < kCopyVec; ++i) {
-      const int64_t v = v0 + i * kCopyThreads;
-      if (v < vecs) to[v] = buf[i];
-    }
+int launch_prefetch_bulk(const int32_t* rep, const int32_t* list, int nslots,
+                         const PrefetchSrc& src, uint8_t* P1, uint8_t* P3, uint8_t* P2,
+                         int64_t proj_bytes, int32_t* err, cudaStream_t s) {
+  const size_t smem = (size_t)kBulkBufs * kBulkChunk;
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !configured[dev]) {
+    cudaFuncSetAttribute(prefetch_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    configured[dev] = true;
   }
+  prefetch_bulk_kernel<<<num_sms(), 32, smem, s>>>(rep, list, nslots, src, P1, P3, P2,
+                                                   proj_bytes, err);
+  return launch_status();
 }
 
 constexpr int kRowThreads = 256;
@@ -308,21 +312,14 @@ int launch_prefetch(const int32_t* plan, const moe_plan_layout& L, const __nv_bf
                     int F, __nv_bfloat16* P1, __nv_bfloat16* P3, __half* P2, int32_t* err,
                     cudaStream_t s) {
   if (S == 0) return MOE_OK;
-  const size_t smem = (size_t)kBulkBufs * kBulkChunk;
-  static bool configured[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !configured[dev]) {
-    cudaFuncSetAttribute(prefetch_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
-    configured[dev] = true;
-  }
-  prefetch_bulk_kernel<<<num_sms(), 32, smem, s>>>(
-      plan + L.replica_expert, plan + L.replica_list, reinterpret_cast<const uint8_t*>(W1),
-      reinterpret_cast<const uint8_t*>(W3), reinterpret_cast<const uint8_t*>(W2),
-      reinterpret_cast<uint8_t*>(P1), reinterpret_cast<uint8_t*>(P3),
-      reinterpret_cast<uint8_t*>(P2), (int64_t)d * F * 2, err);
-  return launch_status();
+  PrefetchSrc src = {};
+  src.w[0][0] = reinterpret_cast<const uint8_t*>(W1);
+  src.w[1][0] = reinterpret_cast<const uint8_t*>(W3);
+  src.w[2][0] = reinterpret_cast<const uint8_t*>(W2);
+  src.B = E;
+  return launch_prefetch_bulk(plan + L.replica_expert, plan + L.replica_list, R * S, src,
+                              reinterpret_cast<uint8_t*>(P1), reinterpret_cast<uint8_t*>(P3),
+                              reinterpret_cast<uint8_t*>(P2), (int64_t)d * F * 2, err, s);
 }
 
 int launch_combine(const __nv_bfloat16* y, const int32_t* perm, const float* gate, int T,
@@ -364,20 +361,20 @@ int launch_combine(const __nv_bfloat16* y, const int32_t* perm, const float* gat
 int launch_ep_prefetch(const int32_t* plan, const moe_plan_layout& L,
                        const __nv_bfloat16* const* W1_ranks, const __nv_bfloat16* const* W3_ranks,
                        const __half* const* W2_ranks, int W, int me, int E, int S, int d, int F,
-                       __nv_bfloat16* P1, __nv_bfloat16* P3, __half* P2, const int32_t* err,
+                       __nv_bfloat16* P1, __nv_bfloat16* P3, __half* P2, int32_t* err,
                        cudaStream_t s) {
   if (S == 0) return MOE_OK;
-  RankTensors src;
-  for (int u = 0; u < MOE_EP_MAX_RANKS; ++u) {
-    src.w1[u] = u < W ? reinterpret_cast<const uint4*>(W1_ranks[u]) : nullptr;
-    src.w3[u] = u < W ? reinterpret_cast<const uint4*>(W3_ranks[u]) : nullptr;
-    src.w2[u] = u < W ? reinterpret_cast<const uint4*>(W2_ranks[u]) : nullptr;
+  if (S > kBulkMaxSlots) return MOE_ERR_SHAPE;
+  PrefetchSrc src = {};
+  for (int u = 0; u < W && u < MOE_EP_MAX_RANKS; ++u) {
+    src.w[0][u] = reinterpret_cast<const uint8_t*>(W1_ranks[u]);
+    src.w[1][u] = reinterpret_cast<const uint8_t*>(W3_ranks[u]);
+    src.w[2][u] = reinterpret_cast<const uint8_t*>(W2_ranks[u]);
   }
-  const int64_t vecs = (int64_t)d * F / 8;
-  ep_prefetch_kernel<<<num_sms() * 4, kCopyThreads, 0, s>>>(
-      plan + L.replica_expert, me, S, E / W, src, reinterpret_cast<uint4*>(P1),
-      reinterpret_cast<uint4*>(P3), reinterpret_cast<uint4*>(P2), vecs, err);
-  return launch_status();
+  src.B = E / W;
+  return launch_prefetch_bulk(plan + L.replica_expert + (int64_t)me * S, nullptr, S, src,
+                              reinterpret_cast<uint8_t*>(P1), reinterpret_cast<uint8_t*>(P3),
+                              reinterpret_cast<uint8_t*>(P2), (int64_t)d * F * 2, err, s);
 }
 
 int launch_ep_combine(const __nv_bfloat16* const* y_ranks, int W, const int32_t* perm,
