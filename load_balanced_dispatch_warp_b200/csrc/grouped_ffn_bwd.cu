@@ -137,6 +137,15 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
       : "memory");
 }
+// shared -> global tile store through the tensor map (bulk group of the issuing thread)
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(x), "r"(y), "r"(src)
+      : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -277,19 +286,20 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                     const __grid_constant__ CUtensorMap tm_b0,
                     const __grid_constant__ CUtensorMap tm_b1,
                     const __grid_constant__ CUtensorMap tm_p0,
-                    const __grid_constant__ CUtensorMap tm_p1, const BwdArgs args) {
+                    const __grid_constant__ CUtensorMap tm_p1,
+                    const __grid_constant__ CUtensorMap tm_o, const BwdArgs args) {
   constexpr bool TWO_B = EPI == EPI_SWIGLU_BWD;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* stage_base = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  // fp32 epilogue: a 32 x 32 staging block per epilogue warp, 1024-byte aligned (the
+  // weight-gradient tiles leave it through a TMA store with the 128-byte swizzle)
+  float* s_stage = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES + 4 * 32 * 32 * 4);
   int* s_misc = reinterpret_cast<int*>(bars + 2 * STAGES + 5);
   int* s_prefix = s_misc + 4;
   int* s_scan = s_prefix + MAX_GROUPS + 1;
-  // fp32 epilogue: a 32 x 32 staging block per epilogue warp (16-byte aligned)
-  float* s_stage = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(s_scan + 33) + 15) &
-                                            ~static_cast<uintptr_t>(15));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   volatile int* abort_flag = s_misc + 1;
 
@@ -531,12 +541,17 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         // instead of 16 bytes in each of 32 rows.  16-byte chunk j of staged row r sits at
         // chunk j ^ (r % 8): the row-per-lane writes and the segment-per-8-lanes reads are
         // both free of bank conflicts.
+        // Weight-gradient tiles are whole 128 x N blocks of the output: each staged block,
+        // laid out as the 128-byte swizzle places it, leaves through one TMA store issued by
+        // lane 0 (the copy engine moves the 4 KiB while the warp stages the next block).
         float* stg = s_stage + (warp - 2) * 1024;
         const int sr = lane >> 3;  // row of this lane within each group of four
         const int sq = lane & 7;   // its 16-byte chunk of the 128-byte segment
         const int rows_here = tl.valid_rows - quarter * 32;
         float* obase = static_cast<float*>(args.out) + tl.out_off +
                        (int64_t)(quarter * 32) * args.out_ld;
+        const int o_row = WGRAD ? (int)(tl.out_off / args.out_ld) + quarter * 32 : 0;
+        const int o_col = WGRAD ? (int)(tl.out_off % args.out_ld) : 0;
 #pragma unroll 1
         for (int c = 0; c < args.bn_out / 32; ++c) {
           uint32_t v[32];
@@ -547,19 +562,30 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] = 0u;
           }
-          __syncwarp();  // the previous block's reads are done
+          // the previous block's reads of the staging block are done (TMA: its store has
+          // read shared memory)
+          if (WGRAD && lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+          __syncwarp();
 #pragma unroll
           for (int j = 0; j < 8; ++j)
             *reinterpret_cast<float4*>(stg + lane * 32 + ((j ^ (lane & 7)) << 2)) =
                 make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
                             __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
-          __syncwarp();
+          if (WGRAD) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) tma_store_2d(&tm_o, smem_u32(stg), o_col + c * 32, o_row);
+          } else {
+            __syncwarp();
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int r = 4 * i + sr;
-            const float4 val = *reinterpret_cast<const float4*>(stg + r * 32 + ((sq ^ (r & 7)) << 2));
-            if (r < rows_here)
-              *reinterpret_cast<float4*>(obase + (int64_t)r * args.out_ld + c * 32 + sq * 4) = val;
+            for (int i = 0; i < 8; ++i) {
+              const int r = 4 * i + sr;
+              const float4 val =
+                  *reinterpret_cast<const float4*>(stg + r * 32 + ((sq ^ (r & 7)) << 2));
+              if (r < rows_here)
+                *reinterpret_cast<float4*>(obase + (int64_t)r * args.out_ld + c * 32 + sq * 4) =
+                    val;
+            }
           }
         }
       } else {
@@ -584,6 +610,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       if (lane == 0) mbar_arrive(tempty0 + 8 * acc);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
+    // every TMA store of this warp has finished before its staging block goes away
+    if (EPI == EPI_F32 && WGRAD && lane == 0)
+      asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -775,14 +805,28 @@ bool make_map16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, in
 }
 
 size_t bwd_smem_bytes() {
-  return 1024 + (size_t)STAGES * STAGE_BYTES + (2 * STAGES + 5) * 8 + 4 * 4 +
-         (MAX_GROUPS + 1) * 4 + 33 * 4 + 16 + 4 * 32 * 32 * 4;
+  return 1024 + (size_t)STAGES * STAGE_BYTES + 4 * 32 * 32 * 4 + (2 * STAGES + 5) * 8 + 4 * 4 +
+         (MAX_GROUPS + 1) * 4 + 33 * 4;
+}
+
+// Output map of the weight-gradient tiles: fp32 [rows, cols] (row stride ld), 32 x 32
+// boxes, the 128-byte swizzle of the staging blocks.
+bool make_map_out32(CUtensorMap* m, void* base, int64_t rows, int64_t cols, int64_t ld) {
+  EncodeTiledFn fn = encode_fn_bwd();
+  if (!fn || rows <= 0 || cols <= 0) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 4};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int EPI, bool WGRAD, bool BMN = false>
 int launch_bwd_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                     const CUtensorMap& p0, const CUtensorMap& p1, const BwdArgs& args,
-                    cudaStream_t s) {
+                    cudaStream_t s, const CUtensorMap* out = nullptr) {
   static bool configured[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -793,7 +837,8 @@ int launch_bwd_gemm(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorM
       return MOE_ERR_LAUNCH;
     configured[dev] = true;
   }
-  bwd_gemm_kernel<EPI, WGRAD, BMN><<<num_sms(), BWD_THREADS, smem, s>>>(a, b0, b1, p0, p1, args);
+  bwd_gemm_kernel<EPI, WGRAD, BMN><<<num_sms(), BWD_THREADS, smem, s>>>(a, b0, b1, p0, p1,
+                                                                     out ? *out : a, args);
   return launch_status();
 }
 
@@ -981,7 +1026,9 @@ int grouped_ffn_backward_impl(const __nv_bfloat16* recv, const __nv_bfloat16* dy
     a.m_blocks = d / BM;
     a.a_row_base = 0;
     a.out_expert_stride = (int64_t)d * F;
-    if ((st = launch_bwd_gemm<EPI_F32, true>(ma, mb, mb, mb, mb, a, s))) return st;
+    CUtensorMap mo;
+    if (!make_map_out32(&mo, dW2, (int64_t)Eo * d, F, F)) return MOE_ERR_DEVICE;
+    if ((st = launch_bwd_gemm<EPI_F32, true>(ma, mb, mb, mb, mb, a, s, &mo))) return st;
   }
   {
     CUtensorMap ma, mb;
@@ -1000,10 +1047,14 @@ int grouped_ffn_backward_impl(const __nv_bfloat16* recv, const __nv_bfloat16* dy
     a.out_expert_stride = (int64_t)F * d;
     a.a_row_base = 0;
     a.out = dW1;
-    if ((st = launch_bwd_gemm<EPI_F32, true>(ma, mb, mb, mb, mb, a, s))) return st;
+    CUtensorMap mo1, mo3;
+    if (!make_map_out32(&mo1, dW1, (int64_t)Eo * F, d, d) ||
+        !make_map_out32(&mo3, dW3, (int64_t)Eo * F, d, d))
+      return MOE_ERR_DEVICE;
+    if ((st = launch_bwd_gemm<EPI_F32, true>(ma, mb, mb, mb, mb, a, s, &mo1))) return st;
     a.a_row_base = F;
     a.out = dW3;
-    if ((st = launch_bwd_gemm<EPI_F32, true>(ma, mb, mb, mb, mb, a, s))) return st;
+    if ((st = launch_bwd_gemm<EPI_F32, true>(ma, mb, mb, mb, mb, a, s, &mo3))) return st;
   }
   return MOE_OK;
 }
