@@ -73,33 +73,42 @@ __global__ void __launch_bounds__(32) prefetch_bulk_kernel(
   extern __shared__ __align__(128) uint8_t buf[];  // kBulkBufs * kBulkChunk
   __shared__ __align__(8) uint64_t bar[kBulkBufs];
   __shared__ int s_slots[kBulkMaxSlots];
-  if (threadIdx.x != 0) return;
+  const int lane = threadIdx.x;
   if (load_err(err)) return;
+  // the slots to fill, in order, gathered by the whole warp (32 candidates per step)
+  const int listed = list != nullptr ? __ldg(list) : nslots;
+  const int cand = min(listed, kBulkMaxSlots);
+  int n = 0;
+  bool bad = listed > kBulkMaxSlots;
+  for (int base = 0; base < cand; base += 32) {
+    const int c = base + lane;
+    bool keep = false;
+    int q = -1;
+    if (c < cand) {
+      q = list != nullptr ? __ldg(list + 1 + c) : c;
+      if (q < 0 || q >= nslots) {
+        bad = true;
+      } else {
+        const int e = __ldg(rep + q);
+        if (e < 0) {
+          bad |= list != nullptr;  // the plan lists filled slots only
+        } else {
+          const int home = e / src.B;
+          if (home >= MOE_EP_MAX_RANKS || src.w[0][home] == nullptr) bad = true;
+          else keep = true;
+        }
+      }
+    }
+    const uint32_t kept = __ballot_sync(MOE_FULL_MASK, keep);
+    if (keep) s_slots[n + __popc(kept & ((1u << lane) - 1u))] = q;
+    n += __popc(kept);
+  }
+  if (__any_sync(MOE_FULL_MASK, bad) && lane == 0) atomicOr(err, MOE_DERR_ID_RANGE);
+  __syncwarp();
+  if (lane != 0) return;
   for (int b = 0; b < kBulkBufs; ++b)
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bulk_smem(&bar[b])) : "memory");
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  const int cand = list != nullptr ? min(__ldg(list), kBulkMaxSlots) : min(nslots, kBulkMaxSlots);
-  int n = 0;
-  bool bad = false;
-  for (int c = 0; c < cand; ++c) {
-    const int q = list != nullptr ? __ldg(list + 1 + c) : c;
-    if (q < 0 || q >= nslots) {
-      bad = true;
-      continue;
-    }
-    const int e = __ldg(rep + q);
-    if (e < 0) {
-      bad |= list != nullptr;  // the plan lists filled slots only
-      continue;
-    }
-    const int home = e / src.B;
-    if (home >= MOE_EP_MAX_RANKS || src.w[0][home] == nullptr) {
-      bad = true;
-      continue;
-    }
-    s_slots[n++] = q;
-  }
-  if (bad) atomicOr(err, MOE_DERR_ID_RANGE);
   const int64_t chunks = proj_bytes / kBulkChunk;
   const int64_t total = (int64_t)n * 3 * chunks;
   // this CTA's units: blockIdx.x + i * gridDim.x, i = 0, 1, ...
