@@ -713,6 +713,8 @@ __global__ void __launch_bounds__(256) transpose_kernel(
 // <dout[t], y[perm[t,j]]> (fp32).  One warp per token, 16-byte vectors.
 // YSrc / DySink (rows.cuh): y read and dy written on this GPU, or on every rank of the
 // expert-parallel layer through its row tables (peer loads and stores).
+constexpr int kCbU = 4;  // 16-byte vectors of each row per lane per step (combine backward)
+
 template <class YSrc, class DySink>
 __global__ void __launch_bounds__(256) combine_backward_kernel(
     const uint4* __restrict__ dout, const __grid_constant__ YSrc y, const int32_t* __restrict__ perm,
@@ -725,25 +727,47 @@ __global__ void __launch_bounds__(256) combine_backward_kernel(
     for (int j = 0; j < k; ++j) {
       const int r = __ldg(perm + t * k + j);
       const float gj = __ldg(gate + t * k + j);
-      float dot = 0.f;
-      for (int v = lane; v < dv; v += 32) {
-        const uint4 a = __ldg(dout + t * dv + v);
-        const uint4 b = __ldcs(y.row(r, dv) + v);
-        const __nv_bfloat162* ap = reinterpret_cast<const __nv_bfloat162*>(&a);
-        const __nv_bfloat162* bp = reinterpret_cast<const __nv_bfloat162*>(&b);
-        uint32_t o[4];
+      const uint4* yr = y.row(r, dv);
+      uint4* dyr = dy.row(r, dv);
+      // kCbU vectors of dout and of y in flight per lane before the first FMA; the partial
+      // dot products are summed in a fixed order, so the result does not depend on timing
+      float dot[kCbU];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 af = __bfloat1622float2(ap[i]);
-          const float2 bf = __bfloat1622float2(bp[i]);
-          dot = fmaf(af.x, bf.x, dot);
-          dot = fmaf(af.y, bf.y, dot);
-          o[i] = pack_bf16(gj * af.x, gj * af.y);
+      for (int u = 0; u < kCbU; ++u) dot[u] = 0.f;
+      for (int v0 = lane; v0 < dv; v0 += 32 * kCbU) {
+        uint4 a[kCbU], b[kCbU];
+#pragma unroll
+        for (int u = 0; u < kCbU; ++u) {
+          const int v = v0 + 32 * u;
+          if (v < dv) {
+            a[u] = __ldg(dout + t * dv + v);
+            b[u] = __ldcs(yr + v);
+          }
         }
-        dy.row(r, dv)[v] = make_uint4(o[0], o[1], o[2], o[3]);
+#pragma unroll
+        for (int u = 0; u < kCbU; ++u) {
+          const int v = v0 + 32 * u;
+          if (v < dv) {
+            const __nv_bfloat162* ap = reinterpret_cast<const __nv_bfloat162*>(&a[u]);
+            const __nv_bfloat162* bp = reinterpret_cast<const __nv_bfloat162*>(&b[u]);
+            uint32_t o[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float2 af = __bfloat1622float2(ap[i]);
+              const float2 bf = __bfloat1622float2(bp[i]);
+              dot[u] = fmaf(af.x, bf.x, dot[u]);
+              dot[u] = fmaf(af.y, bf.y, dot[u]);
+              o[i] = pack_bf16(gj * af.x, gj * af.y);
+            }
+            dyr[v] = make_uint4(o[0], o[1], o[2], o[3]);
+          }
+        }
       }
-      dot = warp_sum(dot);
-      if (lane == 0) dgate[t * k + j] = dot;
+      float total = 0.f;
+#pragma unroll
+      for (int u = 0; u < kCbU; ++u) total += dot[u];
+      total = warp_sum(total);
+      if (lane == 0) dgate[t * k + j] = total;
     }
   }
 }
