@@ -120,3 +120,37 @@ def test_plan_random_demand(E, R, S):
             assert np.array_equal(got, v), (trial, name)
     if S == 0:
         assert n_err > 0  # hot draws cannot be balanced without slots
+
+
+def test_prefetch_rejects_a_corrupted_slot_list():
+    """The bulk-copy prefetch checks every listed slot before copying: a slot outside
+    [0, R*S) or one whose expert is outside [0, E) sets MOE_DERR_ID_RANGE and is skipped
+    (nothing read or written for it); the valid slots are still copied bitwise."""
+    w = I.small_workload("pf", 512, 32, 4, 8, 4, 256, 256, alpha=2.0, seed=23)
+    W1, W3, W2 = I.make_weights(w, device="cuda")
+    L = M.MoELayer(w.T, w.E, w.k, w.R, w.S, w.d, w.F)
+    L.route_plan(I.make_logits(w).cuda())
+    torch.cuda.synchronize()
+    assert int(L.err.item()) == 0
+    lay = M.plan_layout(w.E, w.R, w.S)
+    plan = L.plan.clone()
+    n = int(plan[lay.replica_list].item())
+    assert n >= 2
+    slots = plan[lay.replica_list + 1: lay.replica_list + 1 + n].tolist()
+    good = slots[0]
+    bad_expert_slot = slots[1]
+    plan[lay.replica_expert + bad_expert_slot] = w.E + 3        # an expert outside [0, E)
+    plan[lay.replica_list] = 3
+    plan[lay.replica_list + 1] = good
+    plan[lay.replica_list + 2] = bad_expert_slot
+    plan[lay.replica_list + 3] = w.R * w.S + 1                   # a slot outside the pool
+    P1, P3, P2 = (torch.full_like(p, 7) for p in L.pool)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    M.moe_prefetch_replicas(plan, W1, W3, W2, w.R, w.S, P1, P3, P2, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == M.DERR_ID_RANGE
+    e = int(plan[lay.replica_expert + good].item())
+    assert torch.equal(P1[good], W1[e]) and torch.equal(P3[good], W3[e]) and torch.equal(P2[good], W2[e])
+    for q in range(w.R * w.S):
+        if q != good:
+            assert bool((P1[q] == 7).all()) and bool((P2[q] == 7).all())
