@@ -713,9 +713,9 @@ __global__ void __launch_bounds__(256) transpose_kernel(
 // <dout[t], y[perm[t,j]]> (fp32).  One warp per token, 16-byte vectors.
 // YSrc / DySink (rows.cuh): y read and dy written on this GPU, or on every rank of the
 // expert-parallel layer through its row tables (peer loads and stores).
-constexpr int kCbU = 4;  // 16-byte vectors of each row per lane per step (combine backward)
-
-template <class YSrc, class DySink>
+// U: 16-byte vectors of each row per lane per step (8 for rows of d >= 4096: 847 -> 707 us at
+// d = 7168; 4 below, where 8 gains nothing)
+template <class YSrc, class DySink, int U>
 __global__ void __launch_bounds__(256) combine_backward_kernel(
     const uint4* __restrict__ dout, const __grid_constant__ YSrc y, const int32_t* __restrict__ perm,
     const float* __restrict__ gate, int T, int k, int dv, const __grid_constant__ DySink dy,
@@ -729,15 +729,15 @@ __global__ void __launch_bounds__(256) combine_backward_kernel(
       const float gj = __ldg(gate + t * k + j);
       const uint4* yr = y.row(r, dv);
       uint4* dyr = dy.row(r, dv);
-      // kCbU vectors of dout and of y in flight per lane before the first FMA; the partial
+      // U vectors of dout and of y in flight per lane before the first FMA; the partial
       // dot products are summed in a fixed order, so the result does not depend on timing
-      float dot[kCbU];
+      float dot[U];
 #pragma unroll
-      for (int u = 0; u < kCbU; ++u) dot[u] = 0.f;
-      for (int v0 = lane; v0 < dv; v0 += 32 * kCbU) {
-        uint4 a[kCbU], b[kCbU];
+      for (int u = 0; u < U; ++u) dot[u] = 0.f;
+      for (int v0 = lane; v0 < dv; v0 += 32 * U) {
+        uint4 a[U], b[U];
 #pragma unroll
-        for (int u = 0; u < kCbU; ++u) {
+        for (int u = 0; u < U; ++u) {
           const int v = v0 + 32 * u;
           if (v < dv) {
             a[u] = __ldg(dout + t * dv + v);
@@ -745,7 +745,7 @@ __global__ void __launch_bounds__(256) combine_backward_kernel(
           }
         }
 #pragma unroll
-        for (int u = 0; u < kCbU; ++u) {
+        for (int u = 0; u < U; ++u) {
           const int v = v0 + 32 * u;
           if (v < dv) {
             const __nv_bfloat162* ap = reinterpret_cast<const __nv_bfloat162*>(&a[u]);
@@ -765,7 +765,7 @@ __global__ void __launch_bounds__(256) combine_backward_kernel(
       }
       float total = 0.f;
 #pragma unroll
-      for (int u = 0; u < kCbU; ++u) total += dot[u];
+      for (int u = 0; u < U; ++u) total += dot[u];
       total = warp_sum(total);
       if (lane == 0) dgate[t * k + j] = total;
     }
@@ -1158,9 +1158,15 @@ int launch_combine_backward(const __nv_bfloat16* dout, const __nv_bfloat16* y,
   if (T == 0) return MOE_OK;
   const int64_t want = ((int64_t)T + 7) / 8;
   const int64_t cap = (int64_t)num_sms() * 8;
-  combine_backward_kernel<LocalY, LocalRows><<<(unsigned)(want < cap ? want : cap), 256, 0, s>>>(
-      reinterpret_cast<const uint4*>(dout), LocalY{reinterpret_cast<const uint4*>(y)}, perm, gate,
-      T, k, d / 8, LocalRows{reinterpret_cast<uint4*>(dy)}, dgate, err);
+  const unsigned grid = (unsigned)(want < cap ? want : cap);
+  const LocalY yv{reinterpret_cast<const uint4*>(y)};
+  const LocalRows dv{reinterpret_cast<uint4*>(dy)};
+  if (d / 8 >= 512)
+    combine_backward_kernel<LocalY, LocalRows, 8><<<grid, 256, 0, s>>>(
+        reinterpret_cast<const uint4*>(dout), yv, perm, gate, T, k, d / 8, dv, dgate, err);
+  else
+    combine_backward_kernel<LocalY, LocalRows, 4><<<grid, 256, 0, s>>>(
+        reinterpret_cast<const uint4*>(dout), yv, perm, gate, T, k, d / 8, dv, dgate, err);
   return launch_status();
 }
 
@@ -1205,8 +1211,13 @@ int launch_ep_combine_backward(const __nv_bfloat16* dout, const __nv_bfloat16* c
   yv.C = dv.C = T * k;
   const int64_t want = ((int64_t)T + 7) / 8;
   const int64_t cap = (int64_t)num_sms() * 8;
-  combine_backward_kernel<RankY, RankRows><<<(unsigned)(want < cap ? want : cap), 256, 0, s>>>(
-      reinterpret_cast<const uint4*>(dout), yv, perm, gate, T, k, d / 8, dv, dgate, err);
+  const unsigned grid = (unsigned)(want < cap ? want : cap);
+  if (d / 8 >= 512)  // as the single-GPU launcher, so both sum in the same order
+    combine_backward_kernel<RankY, RankRows, 8><<<grid, 256, 0, s>>>(
+        reinterpret_cast<const uint4*>(dout), yv, perm, gate, T, k, d / 8, dv, dgate, err);
+  else
+    combine_backward_kernel<RankY, RankRows, 4><<<grid, 256, 0, s>>>(
+        reinterpret_cast<const uint4*>(dout), yv, perm, gate, T, k, d / 8, dv, dgate, err);
   return launch_status();
 }
 
